@@ -1,0 +1,187 @@
+/*
+ * tq.h -- C ABI of a B200 (sm_100a) library for TurboQuant KV-cache
+ * compression and decode attention on the compressed cache.
+ *
+ * What the calls compute (citations are the web pages on TurboQuant, by
+ * title and section):
+ *   - TurboQuant_mse: keep ||x|| as is (HN thread on TurboQuant: the radius
+ *     is one number per vector and need not be quantized), rotate x/||x||
+ *     with a seeded random orthogonal map, replace every rotated coordinate by
+ *     the index of its nearest Lloyd-Max centroid, store only the bit-packed
+ *     indices ("TurboQuant của Google: nén KV cache 6 lần", sections "Trick
+ *     đầu tiên: xoay ngẫu nhiên trước khi nén" and "Lloyd-Max quantizer").
+ *   - TurboQuant_prod: (b-1)-bit MSE code of the same kind, then one QJL sign
+ *     bit per coordinate of S r for the residual r, plus ||r||, which makes
+ *     the inner-product estimate unbiased (same page, section "Vấn đề của
+ *     inner product: bias không phải MSE"; "内存厂商的噩梦来了", 4.2-4.3).
+ *   - Decode attention: softmax(q K^T / sqrt(d)) V for one new query per head
+ *     over all cached tokens ("I Spent 31 Hours On The Math Behind
+ *     Turboquant", section "KV Cache: The problem"), with keys scored by the
+ *     asymmetric estimator, a full-precision query against compressed keys
+ *     ("内存厂商的噩梦来了", 4.2 and its asymmetric_attention_score).
+ *
+ * Conventions (all calls):
+ *   - Every call returns tq_status.  Arguments are validated before any
+ *     launch; a failed check returns a non-OK status, launches nothing and
+ *     sets tq_last_error().  A failed launch returns TQ_ECUDA.
+ *   - The library allocates no device memory and keeps no global state.
+ *     The caller owns every buffer and the stream; device calls are
+ *     asynchronous on the given stream (NULL = the legacy default stream).
+ *   - Outputs must not alias inputs.
+ *   - d is 64, 128 or 256.  bits is the total b per coordinate, 1..4.
+ *     The MSE part uses b_m = b bits (mse) or b_m = b - 1 bits (prod).
+ *   - Packed layout per vector ("record"): codes are an LSB-first bitstream,
+ *     index i's bit k at stream bit p = i*b_m + k, byte p >> 3, bit p & 7
+ *     (d*b_m/8 bytes); the QJL sketch puts bit k (1 = (S r)_k >= 0) at byte
+ *     k >> 3, bit k & 7 (d/8 bytes); norms ||x|| and residual norms ||r|| are
+ *     separate fp32 arrays.
+ */
+#ifndef TQ_H
+#define TQ_H
+
+#include <stddef.h>
+#include <stdint.h>
+
+#ifdef __cplusplus
+extern "C" {
+#endif
+
+struct CUstream_st;
+/* A CUDA stream handle (the same object as cudaStream_t). */
+typedef struct CUstream_st *tq_stream_t;
+
+typedef enum {
+  TQ_OK = 0,
+  TQ_EINVAL = 1,        /* bad argument: null pointer, size, alignment, enum */
+  TQ_EUNSUPPORTED = 2,  /* valid request this build does not implement */
+  TQ_ECUDA = 3,         /* a CUDA runtime call or launch failed */
+  TQ_EWORKSPACE = 4,    /* workspace smaller than tq_decode_workspace_bytes */
+  TQ_ETIMEOUT = 5       /* reserved: a bounded device-side wait expired */
+} tq_status;
+
+typedef enum { TQ_MSE = 0, TQ_PROD = 1 } tq_variant;
+
+/* TQ_ROT_HADAMARD: Pi = H diag(sigma) / sqrt(d), H the Sylvester Hadamard
+ * matrix, sigma the seeded signs ("内存厂商的噩梦来了", the note after the
+ * section-4 pseudocode: WHT instead of the dense product).
+ * TQ_ROT_DENSE (a Haar-random d x d matrix) returns TQ_EUNSUPPORTED. */
+typedef enum { TQ_ROT_HADAMARD = 0, TQ_ROT_DENSE = 1 } tq_rotation;
+
+/* Density the codebook is fitted to: N(0, 1/d) (default), or the exact law
+ * C (1 - x^2)^((d-3)/2) of a coordinate of a uniform unit vector
+ * ("TurboQuant của Google", section "Trick đầu tiên"). */
+typedef enum { TQ_CB_GAUSS = 0, TQ_CB_BETA = 1 } tq_codebook_dist;
+
+typedef enum { TQ_F32 = 0, TQ_BF16 = 1, TQ_F16 = 2 } tq_dtype;
+
+/* One quantizer.  A caller-owned value; the pointers are caller-owned DEVICE
+ * memory, filled from tq_make_codebook / tq_make_signs / tq_make_qjl.
+ * centroids/thresholds must be exactly as tq_make_codebook writes them
+ * (ascending, c_i = -c_{K-1-i}, middle threshold 0): the kernels use the
+ * positive half and its mirror image. */
+typedef struct {
+  int32_t d;
+  int32_t bits;            /* total b, 1..4 */
+  int32_t variant;         /* tq_variant */
+  int32_t rotation;        /* tq_rotation */
+  const float *centroids;  /* 2^b_m fp32 (unused when b_m == 0) */
+  const float *thresholds; /* 2^b_m - 1 fp32 */
+  const int8_t *signs;     /* d entries, each +1 or -1 */
+  const float *qjl_S;      /* d*d fp32 row-major, prod only, else NULL */
+} tq_quantizer;
+
+/* A packed cache: records addressed as
+ *   rec(b, h, n) = b*stride_b + h*stride_h + n*stride_n   (in records)
+ * codes + rec*code_bytes, qjl + rec*(d/8), norms + rec, rnorms + rec.
+ * codes is NULL when b_m == 0; qjl and rnorms are NULL for mse.
+ * codes and qjl must be 16-byte aligned; strides may be 0 (a shared cache). */
+typedef struct {
+  uint8_t *codes;
+  uint8_t *qjl;
+  float *norms;
+  float *rnorms;
+  int64_t stride_b, stride_h, stride_n;
+} tq_cache_view;
+
+/* ---- host, synchronous, pure ------------------------------------------ */
+
+/* Lloyd-Max codebook for d and b_m = bits_mse (1..4): 2^b_m centroids and
+ * 2^b_m - 1 thresholds (midpoints), fp32, written to HOST arrays.  Lloyd's
+ * alternation runs in double and is rounded once to fp32 ("TurboQuant của
+ * Google", section "Lloyd-Max quantizer": computed once, shipped, reused). */
+tq_status tq_make_codebook(int32_t d, int32_t bits_mse, tq_codebook_dist dist,
+                           float *centroids, float *thresholds);
+
+/* Seeded Rademacher signs sigma (d int8 values, +1/-1, HOST array): +1 when
+ * bit 63 of SplitMix64 output i is clear. */
+tq_status tq_make_signs(uint64_t seed, int32_t d, int8_t *signs);
+
+/* Seeded QJL matrix S, d x d i.i.d. N(0,1), row-major fp32 HOST array, from
+ * Box-Muller on consecutive SplitMix64 output pairs ("TurboQuant của
+ * Google", section "Vấn đề của inner product": QJL's random projection). */
+tq_status tq_make_qjl(uint64_t seed, int32_t d, float *S);
+
+/* Bytes of one record's codes (d*b_m/8) and QJL sketch (d/8 or 0). */
+size_t tq_code_bytes(int32_t d, int32_t bits, int32_t variant);
+size_t tq_qjl_bytes(int32_t d, int32_t variant);
+
+/* ---- device, asynchronous on `stream` ---------------------------------- */
+
+/* Encode B*H*N vectors.  Vector (b, h, n) starts at element
+ * b*x_stride_b + h*x_stride_h + n*x_stride_n of x (dtype x_dtype, d
+ * contiguous elements); x and every stride times the element size must be
+ * 16-byte aligned.  Writes codes, norms (and qjl, rnorms for prod) of record
+ * (b, h, n) of `out`.  The codes are bit-exact with the canonical fp32
+ * procedure: fold-halves sum of squares, sqrt_rn; FWHT stages h = d/2..1 on
+ * sigma*x; u = y * fl(1/fl(n*fl(sqrt d))) (0 when n == 0);
+ * idx = #{j : u > t_j}.  The QJL projection S r is summed in fp32. */
+tq_status tq_encode(const tq_quantizer *q, const void *x, tq_dtype x_dtype,
+                    int64_t B, int64_t H, int64_t N, int64_t x_stride_b,
+                    int64_t x_stride_h, int64_t x_stride_n,
+                    const tq_cache_view *out, tq_stream_t stream);
+
+/* Reconstruct x_hat = ||x|| Pi^T (c[idx] (+ ||r|| sqrt(pi/2)/d S^T sign))
+ * for the B*H*N records of `in` into out[B][H][N][d] fp32 (DEVICE)
+ * ("内存厂商的噩梦来了", section-4 pseudocode, dequant). */
+tq_status tq_dequant(const tq_quantizer *q, const tq_cache_view *in, int64_t B,
+                     int64_t H, int64_t N, float *out, tq_stream_t stream);
+
+/* Workspace the decode call needs, in bytes (0 means none).  Depends only
+ * on the arguments; the value may change between library versions. */
+size_t tq_decode_workspace_bytes(int32_t B, int32_t Hq, int32_t Hkv,
+                                 int64_t seq_len, int32_t d);
+
+/* Decode attention.  q: [B][Hq][d] (q_dtype, DEVICE).  Query head hq reads
+ * kv head hq / (Hq/Hkv).  Cached tokens 0..L_b-1 of batch b are attended
+ * with L_b = seq_lens[b] (DEVICE int32 [B], each 0..seq_len) or seq_len when
+ * seq_lens is NULL; no causal mask.  The query is rotated once by the key
+ * rotation; scores are
+ *   s_j = n_j (<q', c_K[idx_j]> + [prod] ||r_j|| sqrt(pi/2)/d <S q', sign_j>)
+ * logits s_j * softmax_scale; values are summed in the value-rotated basis
+ * and rotated back once at the end.  out: [B][Hq][d] fp32 (DEVICE); a batch
+ * with L_b == 0 gets zeros.  scores_out: optional [B][Hq][seq_len] fp32 of
+ * the pre-scale estimator s_j (entries j >= L_b untouched), or NULL.
+ * V must be mse (prod values return TQ_EUNSUPPORTED); d must be 128 or 64.
+ * workspace: DEVICE, at least tq_decode_workspace_bytes(...) bytes, 16-byte
+ * aligned, else TQ_EWORKSPACE. */
+tq_status tq_decode_attention(const tq_quantizer *kq, const tq_quantizer *vq,
+                              const void *q, tq_dtype q_dtype, int32_t B,
+                              int32_t Hq, int32_t Hkv, int64_t seq_len,
+                              const int32_t *seq_lens, const tq_cache_view *k,
+                              const tq_cache_view *v, float softmax_scale,
+                              float *out, float *scores_out, void *workspace,
+                              size_t workspace_bytes, tq_stream_t stream);
+
+/* Synchronize `stream` and report any asynchronous CUDA error. */
+tq_status tq_check(tq_stream_t stream);
+
+const char *tq_status_string(tq_status s);
+/* Message of the last failed call on this host thread ("" if none). */
+const char *tq_last_error(void);
+const char *tq_version(void);
+
+#ifdef __cplusplus
+}
+#endif
+
+#endif /* TQ_H */

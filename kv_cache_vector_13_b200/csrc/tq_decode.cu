@@ -1,0 +1,997 @@
+// Decode attention on the packed TurboQuant cache (sm_100a).
+//
+// Attention for one new query per head, softmax(q K^T / sqrt(d)) V over all
+// cached tokens ("I Spent 31 Hours On The Math Behind Turboquant", section
+// "KV Cache: The problem"), with keys scored by the asymmetric estimator: the
+// full-precision query against the compressed keys ("内存厂商的噩梦来了",
+// section 4.2 and its asymmetric_attention_score):
+//   s_j = n_j ( <q', c_K[idx_j]> + [prod] ||r_j|| sqrt(pi/2)/d <S q', sign_j> ),
+// q' = Pi_K q the query rotated once.  Values are summed in the value-rotated
+// basis, o' = sum_j p_j n_j c_V[idx_j], and rotated back once at the end,
+// o = Pi_V^T o'.
+//
+// Kernel 0 (prep), once per call: rotates every query head (sign flips +
+// FWHT, and S q' for prod keys) into the workspace, and for each codebook
+// finds a scale s with fp16(s c_k) close to s c_k for every centroid (a
+// search over 4096 candidates in [1, 2)) and writes the 256-entry pair table
+// entry e -> half2(fp16(s c[e & m]), fp16(s c[(e >> b_m) & m])).
+// Kernel 1 (split), persistent: one CTA of 8 warps per SM; each warp keeps
+// its next chunk's loads in flight while it computes the current one.  The work is the
+// flattened space of (unit = batch x kv head x group of <= 8 query heads,
+// token) pairs, cut into one equal contiguous range per CTA; a range covers
+// one or a few "pieces" (CTA, unit).  Per CTA, once: the two pair tables are
+// copied into shared memory, replicated per lane (entry e, lane l at
+// e*256 + 4l, values at +128) so that table reads never conflict on banks.
+// Per piece: the group's rotated queries are split into hi + lo fp16 halves;
+// then every warp streams its share of 32-token chunks:
+//   * packed K/V words go from HBM straight to registers, one pass;
+//   * two adjacent indices (one byte of the bitstream, or a shifted byte for
+//     b_m < 4) are one table read -> a half2 of centroids;
+//   * scores and PV are mma.m16n8k16 f16 x f16 -> f32: tokens on M for the
+//     scores (K-hat [16 tok x 16 dims] x q' [16 dims x 8]), dims on M for PV
+//     (V-hat^T [16 dims x 16 tok] x W [16 tok x 8]).  A contraction may
+//     permute its summation index as long as both operands agree, so a lane
+//     reads contiguous code bytes and q' is laid out to match.  With <= 4
+//     query heads per kv head the hi and lo halves of q' (and of the PV
+//     weights) share one MMA as columns 0-3 and 4-7; with 5-8 heads they take
+//     two MMAs;
+//   * QJL bits become +-1 halves with one shift and one LOP3 per pair;
+//   * online softmax in base 2 with two running maxima, m over the logits
+//     (for the normaliser l) and M over logit + log2 n_V (for the PV weights
+//     2^(u - M), which keeps p_j n_j in fp16 range).
+// The warps' partials (m, l, M, o') of a piece are merged in shared memory
+// and written to workspace slot (unit + CTA index).
+// Kernel 2 (combine): per (batch, query head), merge the slots of its unit,
+// divide by l, apply Pi_V^T = diag(sigma_V) H / sqrt(d).
+
+#include "../../include/tq.h"
+#include "tq_device.cuh"
+#include "tq_internal.h"
+
+#include <math.h>
+
+namespace tq {
+namespace {
+
+constexpr int kD = 128;
+constexpr int kMaxWarps = 8;
+constexpr int kChunk = 32;               // tokens per warp iteration
+constexpr int kLutBytes = 256 * 256;     // K and V pair tables, per-lane copies
+constexpr int kPW = kD + 4;              // floats per head in a partial: m, l, M, pad, o'[d]
+constexpr int kSlot = 8 * kPW;           // floats per partial slot (8 heads)
+constexpr int kScaleCands = 4096;
+// workspace layout (floats): [0, 2) scales 1/s_K, 1/s_V; [64, 320) K pair
+// table; [320, 576) V pair table; [kHdr, +B*Hq*d) q'; [+B*Hq*d) S q';
+// then (units + CTAs) partial slots of kSlot floats.
+constexpr int kHdr = 1024;
+constexpr float kLog2e = 1.4426950408889634f;
+constexpr float kKappa = 1.2533141373155003f / (float)kD;  // sqrt(pi/2)/d
+
+struct SplitParams {
+  const void *q;
+  int q_dtype;
+  int B, Hq, Hkv, g, groups;
+  int64_t seq_len;
+  const int32_t *seq_lens;
+  int ctas;
+  // keys
+  const uint8_t *kc;
+  const uint8_t *kj;
+  const float *kn;
+  const float *kr;
+  int64_t ksb, ksh, ksn;
+  const float *kcent;
+  const int8_t *ksign;
+  const float *kS;
+  // values
+  const uint8_t *vc;
+  const float *vn;
+  int64_t vsb, vsh, vsn;
+  const float *vcent;
+  float scale_log2;  // softmax_scale * log2(e)
+  float *scores;
+  float *ws;
+  int64_t slot0;  // first float of the partial slots
+};
+
+struct PrepParams {
+  const void *q;
+  int q_dtype;
+  int nheads;  // B * Hq
+  const int8_t *ksign;
+  const float *kS;  // prod keys only
+  const float *kcent;
+  int kbm;
+  const float *vcent;
+  int vbm;
+  float *ws;
+};
+
+struct CombineParams {
+  int B, Hq, Hkv, g, groups;
+  int64_t seq_len;
+  const int32_t *seq_lens;
+  int ctas;
+  int64_t slot0;
+  const float *ws;
+  const int8_t *vsign;
+  float *out;
+};
+
+// ------------------------------------------------------------------ PTX
+
+__device__ __forceinline__ void mma16816(float (&c)[4], const uint32_t (&a)[4], uint32_t b0, uint32_t b1) {
+  asm volatile(
+      "mma.sync.aligned.m16n8k16.row.col.f32.f16.f16.f32 {%0,%1,%2,%3}, {%4,%5,%6,%7}, {%8,%9}, "
+      "{%0,%1,%2,%3};\n"
+      : "+f"(c[0]), "+f"(c[1]), "+f"(c[2]), "+f"(c[3])
+      : "r"(a[0]), "r"(a[1]), "r"(a[2]), "r"(a[3]), "r"(b0), "r"(b1));
+}
+
+__device__ __forceinline__ uint32_t movmatrix_trans(uint32_t x) {
+  uint32_t y;
+  asm volatile("movmatrix.sync.aligned.m8n8.trans.b16 %0, %1;\n" : "=r"(y) : "r"(x));
+  return y;
+}
+
+// table entry at byte offset `off` of a shared table
+__device__ __forceinline__ uint32_t lut(const char *tab, uint32_t off) {
+  return *reinterpret_cast<const uint32_t *>(tab + off);
+}
+
+__device__ __forceinline__ uint32_t pack_half2(float lo, float hi) {
+  const __half2 h = __floats2half2_rn(lo, hi);
+  return *reinterpret_cast<const uint32_t *>(&h);
+}
+
+// hi = fp16(x), lo = fp16(x - hi): x to ~22 significant bits
+__device__ __forceinline__ void split_half(float x, float &hi, float &lo) {
+  hi = __half2float(__float2half_rn(x));
+  lo = x - hi;
+}
+
+__device__ __forceinline__ uint32_t pack_hi(float a, float b) {
+  float ah, al, bh, bl;
+  split_half(a, ah, al);
+  split_half(b, bh, bl);
+  return pack_half2(ah, bh);
+}
+
+__device__ __forceinline__ uint32_t pack_lo(float a, float b) {
+  float ah, al, bh, bl;
+  split_half(a, ah, al);
+  split_half(b, bh, bl);
+  return pack_half2(al, bl);
+}
+
+// The byte starting `SH` bits up the little-endian word pair (w0, w1), moved
+// into byte 1 of the lane's offset (byte 0 = 4*lane, +128 for the value
+// table): the entry's byte offset inside the table.
+template <int SH>
+__device__ __forceinline__ uint32_t lut_addr(uint32_t w0, uint32_t w1, uint32_t laneoff) {
+  constexpr int s = SH & 31;
+  if constexpr (s % 8 == 0) {
+    return __byte_perm(w0, laneoff, 0x7604 | ((s / 8) << 4));
+  } else if constexpr (s + 8 <= 32) {
+    return __byte_perm(w0 >> s, laneoff, 0x7604);
+  } else {
+    return __byte_perm(__funnelshift_r(w0, w1, s), laneoff, 0x7604);
+  }
+}
+
+// pair q (dims 2q, 2q+1) of a BM-bit LSB-first stream held in words W[]
+template <int BM, int Q, int NW>
+__device__ __forceinline__ uint32_t pair_addr(const uint32_t (&W)[NW], uint32_t laneoff) {
+  constexpr int off = 2 * BM * Q;
+  constexpr int w = off >> 5;
+  constexpr int w1 = (w + 1 < NW) ? w + 1 : w;
+  return lut_addr<off>(W[w], W[w1], laneoff);
+}
+
+// +-1 half2 from QJL bits (15 - sh, 31 - sh) of w: bit 1 -> +1, bit 0 -> -1
+template <int SH>
+__device__ __forceinline__ uint32_t qjl_half2(uint32_t w) {
+  return ((w << SH) & 0x80008000u) ^ 0xBC00BC00u;
+}
+
+template <int BM>
+struct VChunk {  // 16 dims of one token: 2*BM bytes
+  static constexpr int NW = (2 * BM + 3) / 4;
+};
+
+template <int BM>
+__device__ __forceinline__ void load_v16(const uint8_t *p, uint32_t (&W)[VChunk<BM>::NW], int g) {
+  // bytes [2*BM*g, 2*BM*g + 2*BM) of the record, naturally aligned pieces only
+  if constexpr (BM == 4) {
+    const uint2 t = __ldg(reinterpret_cast<const uint2 *>(p));
+    W[0] = t.x;
+    W[1] = t.y;
+  } else if constexpr (BM == 2) {
+    W[0] = __ldg(reinterpret_cast<const uint32_t *>(p));
+  } else if constexpr (BM == 1) {
+    W[0] = __ldg(reinterpret_cast<const unsigned short *>(p));
+  } else {  // BM == 3: 6 bytes at 6g, 2-byte aligned
+    if ((g & 1) == 0) {
+      W[0] = __ldg(reinterpret_cast<const uint32_t *>(p));
+      W[1] = __ldg(reinterpret_cast<const unsigned short *>(p + 4));
+    } else {
+      const uint32_t lo = __ldg(reinterpret_cast<const unsigned short *>(p));
+      const uint32_t hi = __ldg(reinterpret_cast<const uint32_t *>(p + 2));
+      W[0] = lo | (hi << 16);
+      W[1] = hi >> 16;
+    }
+  }
+}
+
+template <int BM>
+__device__ __forceinline__ void load_k32(const uint8_t *p, uint32_t (&W)[BM > 0 ? BM : 1]) {
+  // 4*BM bytes (32 dims) at a 4*BM-aligned offset
+  if constexpr (BM == 4) {
+    const uint4 t = __ldg(reinterpret_cast<const uint4 *>(p));
+    W[0] = t.x;
+    W[1] = t.y;
+    W[2] = t.z;
+    W[3] = t.w;
+  } else if constexpr (BM == 2) {
+    const uint2 t = __ldg(reinterpret_cast<const uint2 *>(p));
+    W[0] = t.x;
+    W[1] = t.y;
+  } else {
+#pragma unroll
+    for (int i = 0; i < (BM > 0 ? BM : 1); ++i) W[i] = __ldg(reinterpret_cast<const uint32_t *>(p) + i);
+  }
+}
+
+// ----------------------------------------------------------- work split
+
+// Length of the units of batch b.
+__device__ __forceinline__ int64_t batch_len(const int32_t *seq_lens, int64_t seq_len, int b) {
+  if (!seq_lens) return seq_len;
+  const int64_t L = seq_lens[b];
+  return L < 0 ? 0 : (L > seq_len ? seq_len : L);
+}
+
+// Flattened space: units u = (b, kvh, grp) in that order, unit u of batch b
+// spans batch_len(b) tokens.  Returns the total; *pb gets the start of batch
+// `bq`'s first unit (when bq >= 0).
+__device__ __forceinline__ int64_t flat_total(const int32_t *seq_lens, int64_t seq_len, int B, int UH) {
+  if (!seq_lens) return (int64_t)B * UH * seq_len;
+  int64_t t = 0;
+  for (int b = 0; b < B; ++b) t += batch_len(seq_lens, seq_len, b) * UH;
+  return t;
+}
+
+// CTA c covers [cut(c), cut(c+1)).
+__device__ __forceinline__ int64_t cut(int64_t T, int C, int c) {
+  return (int64_t)(((uint64_t)T * (uint64_t)c) / (uint64_t)C);  // T * C < 2^64 for any real cache
+}
+
+// Unit containing flattened position x (x < T): unit index, its start, length.
+__device__ __forceinline__ void locate(const int32_t *seq_lens, int64_t seq_len, int B, int UH, int64_t x,
+                                       int *u, int64_t *start, int64_t *len) {
+  if (!seq_lens) {
+    const int64_t uu = x / seq_len;
+    *u = (int)uu;
+    *start = uu * seq_len;
+    *len = seq_len;
+    return;
+  }
+  int64_t base = 0;
+  for (int b = 0; b < B; ++b) {
+    const int64_t L = batch_len(seq_lens, seq_len, b);
+    const int64_t span = L * UH;
+    if (x < base + span) {
+      const int64_t r = (x - base) / L;
+      *u = b * UH + (int)r;
+      *start = base + r * L;
+      *len = L;
+      return;
+    }
+    base += span;
+  }
+  *u = B * UH - 1;
+  *start = base;
+  *len = 0;
+}
+
+// ------------------------------------------------------------- prep kernel
+
+// Index i in [0, kScaleCands) minimising the worst relative fp16 rounding
+// error of (1 + i/kScaleCands) * c_k over the K/2 positive centroids (ties ->
+// smallest i); then the pair table for that scale.  One 256-thread block.
+__device__ void scale_and_table(const float *cent, int bm, float *inv_scale, uint32_t *table) {
+  __shared__ uint64_t s_red[8];
+  __shared__ float s_c[16];
+  const int K = 1 << bm;
+  if (threadIdx.x < K) s_c[threadIdx.x] = cent[threadIdx.x];
+  __syncthreads();
+  float c[8], rc[8];
+#pragma unroll
+  for (int k = 0; k < 8; ++k) {
+    c[k] = K / 2 + k < K ? s_c[K / 2 + k] : s_c[K - 1];
+    rc[k] = 1.0f / c[k];
+  }
+  uint64_t best = ~0ull;
+  for (int i = threadIdx.x; i < kScaleCands; i += blockDim.x) {
+    const float s = 1.0f + (float)i * (1.0f / kScaleCands);
+    float worst = 0.f;
+#pragma unroll
+    for (int k = 0; k < 8; ++k) {
+      const float v = s * c[k];
+      worst = fmaxf(worst, fabsf(__half2float(__float2half_rn(v)) - v) * rc[k]);
+    }
+    const uint64_t key = ((uint64_t)__float_as_uint(worst) << 32) | (uint32_t)i;
+    best = key < best ? key : best;
+  }
+#pragma unroll
+  for (int o = 16; o >= 1; o >>= 1) {
+    const uint64_t other = __shfl_xor_sync(dev::kFull, best, o);
+    best = other < best ? other : best;
+  }
+  if ((threadIdx.x & 31) == 0) s_red[threadIdx.x >> 5] = best;
+  __syncthreads();
+  uint64_t b = ~0ull;
+  for (int w = 0; w < (int)(blockDim.x >> 5); ++w) b = s_red[w] < b ? s_red[w] : b;
+  const float sc = 1.0f + (float)(uint32_t)(b & 0xffffffffu) * (1.0f / kScaleCands);
+  const uint32_t m = (uint32_t)K - 1u;
+  for (int e = threadIdx.x; e < 256; e += blockDim.x)
+    table[e] = pack_half2(sc * s_c[e & m], sc * s_c[(e >> bm) & m]);
+  if (threadIdx.x == 0) *inv_scale = 1.0f / sc;
+}
+
+// Blocks [0, nheads/2): two query heads each (128 threads per head):
+// q' = H(sigma q)/sqrt(d) and q_s = S q'.  The last two blocks: the K and
+// V scale and pair table.
+__global__ void __launch_bounds__(256) decode_prep_kernel(PrepParams p) {
+  const int nqb = (p.nheads + 1) / 2;
+  if ((int)blockIdx.x >= nqb) {
+    if (blockIdx.x == (unsigned)nqb) {
+      if (p.kbm > 0) scale_and_table(p.kcent, p.kbm, p.ws + 0, reinterpret_cast<uint32_t *>(p.ws + 64));
+      else if (threadIdx.x == 0) p.ws[0] = 1.0f;
+    } else {
+      scale_and_table(p.vcent, p.vbm, p.ws + 1, reinterpret_cast<uint32_t *>(p.ws + 320));
+    }
+    return;
+  }
+  __shared__ float s_q[2][kD];
+  const int half = threadIdx.x >> 7, t = threadIdx.x & 127;
+  const int head = blockIdx.x * 2 + half;
+  const bool valid = head < p.nheads;
+  const int lane = threadIdx.x & 31;
+  if ((t >> 5) == 0) {  // one warp per head: 4 dims per lane
+    float a[4] = {0.f, 0.f, 0.f, 0.f};
+    if (valid) {
+      const int64_t qoff = (int64_t)head * kD + lane * 4;
+      if (p.q_dtype == TQ_F32) {
+        const float4 v = __ldg(reinterpret_cast<const float4 *>(p.q) + qoff / 4);
+        a[0] = v.x; a[1] = v.y; a[2] = v.z; a[3] = v.w;
+      } else {
+        const uint2 v = __ldg(reinterpret_cast<const uint2 *>(static_cast<const char *>(p.q) + qoff * 2));
+        if (p.q_dtype == TQ_BF16) {
+          a[0] = dev::bf16lo(v.x); a[1] = dev::bf16hi(v.x); a[2] = dev::bf16lo(v.y); a[3] = dev::bf16hi(v.y);
+        } else {
+          a[0] = dev::f16lo(v.x); a[1] = dev::f16hi(v.x); a[2] = dev::f16lo(v.y); a[3] = dev::f16hi(v.y);
+        }
+      }
+#pragma unroll
+      for (int i = 0; i < 4; ++i)
+        if (p.ksign[lane * 4 + i] < 0) a[i] = -a[i];
+    }
+    dev::fwht<32, 4>(a, lane);
+#pragma unroll
+    for (int i = 0; i < 4; ++i) s_q[half][lane * 4 + i] = a[i] * 0.08838834764831845f;
+  }
+  __syncthreads();
+  if (!valid) return;
+  float *qo = p.ws + kHdr + (int64_t)head * kD;
+  qo[t] = s_q[half][t];
+  if (p.kS) {
+    const float4 *Sk = reinterpret_cast<const float4 *>(p.kS + (size_t)t * kD);
+    float acc = 0.f;
+#pragma unroll 8
+    for (int i = 0; i < kD / 4; ++i) {
+      const float4 sv = __ldg(Sk + i);
+      acc = fmaf(sv.x, s_q[half][4 * i], acc);
+      acc = fmaf(sv.y, s_q[half][4 * i + 1], acc);
+      acc = fmaf(sv.z, s_q[half][4 * i + 2], acc);
+      acc = fmaf(sv.w, s_q[half][4 * i + 3], acc);
+    }
+    p.ws[kHdr + (int64_t)p.nheads * kD + (int64_t)head * kD + t] = acc;
+  }
+}
+
+// ------------------------------------------------------------ split kernel
+
+// Everything a lane loads from HBM for one 32-token chunk.  Score rows
+// (ms, r) are tokens j0 + 16 ms + 8 r + g8; PV tokens (ms, q4) are
+// j0 + 16 ms + 2 tig + (q4 & 1) + 8 (q4 >> 1).
+template <int KBM, bool KPROD, int VBM>
+struct ChunkRegs {
+  static constexpr int KW = KBM > 0 ? KBM : 1;
+  static constexpr int VW = VChunk<VBM>::NW;
+  uint32_t kw[2][2][KW];
+  uint32_t qj[2][2];
+  float kn[2][2], kr[2][2], vn[2][2];
+  uint32_t vw[2][4][VW];
+};
+
+template <int KBM, bool KPROD, int VBM>
+__device__ __forceinline__ void load_chunk(ChunkRegs<KBM, KPROD, VBM> &c, const SplitParams &p, int64_t j0,
+                                           int64_t t0, int64_t t1, int64_t kbase, int64_t vbase, int g8,
+                                           int tig) {
+  constexpr int KCB = kD * KBM / 8;
+  constexpr int VCB = kD * VBM / 8;
+#pragma unroll
+  for (int ms = 0; ms < 2; ++ms) {
+#pragma unroll
+    for (int r = 0; r < 2; ++r) {
+      const int64_t j = j0 + 16 * ms + 8 * r + g8;
+      const bool ok = j < t1;
+      const int64_t jj = ok ? j : t0;
+      const int64_t rec = kbase + jj * p.ksn;
+      if constexpr (KBM > 0) load_k32<KBM>(p.kc + rec * KCB + tig * (4 * KBM), c.kw[ms][r]);
+      if constexpr (KPROD) {
+        c.qj[ms][r] = __ldg(reinterpret_cast<const uint32_t *>(p.kj + rec * (kD / 8)) + tig);
+        c.kr[ms][r] = __ldg(p.kr + rec);
+      }
+      c.kn[ms][r] = ok ? __ldg(p.kn + rec) : -1.f;  // -1 marks a masked row
+      c.vn[ms][r] = __ldg(p.vn + vbase + jj * p.vsn);
+    }
+#pragma unroll
+    for (int q4 = 0; q4 < 4; ++q4) {
+      const int64_t j = j0 + 16 * ms + 2 * tig + (q4 & 1) + 8 * (q4 >> 1);
+      const int64_t vrec = vbase + (j < t1 ? j : t0) * p.vsn;
+      load_v16<VBM>(p.vc + vrec * VCB + g8 * (2 * VBM), c.vw[ms][q4], g8);
+    }
+  }
+}
+
+template <int KBM, bool KPROD, int VBM, bool PACK>
+__global__ void __launch_bounds__(8 * 32, 1) decode_split_kernel(SplitParams p) {
+  constexpr int kWarps = 8;
+  constexpr int kThreads = kWarps * 32;
+  constexpr int KW = KBM > 0 ? KBM : 1;
+  constexpr int VW = VChunk<VBM>::NW;
+  using CR = ChunkRegs<KBM, KPROD, VBM>;
+  extern __shared__ float4 smem4[];
+  char *smem = reinterpret_cast<char *>(smem4);
+  float *s_q = reinterpret_cast<float *>(smem + kLutBytes);  // [8][kD] q'
+  float *s_qs = s_q + 8 * kD;                                // [8][kD] S q'
+  float *s_part = s_qs + 8 * kD;                             // [kWarps][8][kPW]
+
+  const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
+  const int g8 = lane >> 2, tig = lane & 3;
+  const int UH = p.Hkv * p.groups;
+  const int64_t T = flat_total(p.seq_lens, p.seq_len, p.B, UH);
+  const int64_t x0 = cut(T, p.ctas, blockIdx.x), x1 = cut(T, p.ctas, blockIdx.x + 1);
+  if (x0 >= x1) return;
+
+  // ---- once per CTA: replicate the two pair tables per lane
+  {
+    const uint32_t *ktab = reinterpret_cast<const uint32_t *>(p.ws + 64);
+    const uint32_t *vtab = reinterpret_cast<const uint32_t *>(p.ws + 320);
+    uint4 *tab = reinterpret_cast<uint4 *>(smem);
+    for (int i = tid; i < 256 * 16; i += kThreads) {  // 16 uint4 per 256-byte row
+      const int e = i >> 4, part = i & 15;
+      const uint32_t v = part < 8 ? (KBM > 0 ? __ldg(ktab + e) : 0u) : __ldg(vtab + e);
+      tab[i] = make_uint4(v, v, v, v);
+    }
+  }
+  const float inv_sK = __ldg(p.ws + 0);
+  const float inv_sV = __ldg(p.ws + 1);
+  const float sK = 1.0f / inv_sK;
+  const uint32_t koff = lane * 4;
+  const uint32_t voff = 128 + lane * 4;
+
+  for (int64_t x = x0; x < x1;) {
+    int u;
+    int64_t ustart, ulen;
+    locate(p.seq_lens, p.seq_len, p.B, UH, x, &u, &ustart, &ulen);
+    const int64_t t0 = x - ustart;
+    const int64_t t1 = min(x1, ustart + ulen) - ustart;
+    x = ustart + t1;
+    const int b = u / UH;
+    const int kvh = (u % UH) / p.groups;
+    const int grp = (u % UH) % p.groups;
+    const int h0 = kvh * p.g + grp * 8;
+    const int gh = min(8, p.g - grp * 8);
+
+    __syncthreads();  // tables ready / previous piece's shared data consumed
+    // ---- this group's rotated queries (zeros for padding heads)
+    for (int o = tid; o < 8 * kD; o += kThreads) {
+      const int hh = o / kD, k = o % kD;
+      const bool ok = hh < gh;
+      const int64_t qi = ((int64_t)b * p.Hq + h0 + hh) * kD + k;
+      s_q[o] = ok ? __ldg(p.ws + kHdr + qi) : 0.f;
+      if constexpr (KPROD) s_qs[o] = ok ? __ldg(p.ws + kHdr + (int64_t)p.B * p.Hq * kD + qi) : 0.f;
+    }
+    __syncthreads();
+
+    // ---- B fragments in this lane's dim order.  PACK: column n < 4 is the
+    // hi half of head n, n >= 4 the lo half of head n - 4.  Else qf = hi and
+    // qf2 = lo of head g8.
+    uint32_t qf[8][2], qf2[PACK ? 1 : 8][2];
+    uint32_t qsf[KPROD ? 8 : 1][2], qsf2[(KPROD && !PACK) ? 8 : 1][2];
+    {
+      const int hsrc = PACK ? (g8 & 3) : g8;
+      const bool lo_col = PACK && g8 >= 4;
+      const float *qv = s_q + hsrc * kD + 32 * tig;
+#pragma unroll
+      for (int s = 0; s < 8; ++s) {
+        if (PACK) {
+          qf[s][0] = lo_col ? pack_lo(qv[4 * s], qv[4 * s + 1]) : pack_hi(qv[4 * s], qv[4 * s + 1]);
+          qf[s][1] = lo_col ? pack_lo(qv[4 * s + 2], qv[4 * s + 3]) : pack_hi(qv[4 * s + 2], qv[4 * s + 3]);
+        } else {
+          qf[s][0] = pack_hi(qv[4 * s], qv[4 * s + 1]);
+          qf[s][1] = pack_hi(qv[4 * s + 2], qv[4 * s + 3]);
+          if constexpr (!PACK) {
+            qf2[s][0] = pack_lo(qv[4 * s], qv[4 * s + 1]);
+            qf2[s][1] = pack_lo(qv[4 * s + 2], qv[4 * s + 3]);
+          }
+        }
+      }
+      if constexpr (KPROD) {
+        const float *sv = s_qs + hsrc * kD + 32 * tig;
+#pragma unroll
+        for (int s = 0; s < 8; ++s) {
+          const float a0 = sv[15 - 2 * s], a1 = sv[31 - 2 * s], a2 = sv[14 - 2 * s], a3 = sv[30 - 2 * s];
+          if (PACK) {
+            qsf[s][0] = lo_col ? pack_lo(a0, a1) : pack_hi(a0, a1);
+            qsf[s][1] = lo_col ? pack_lo(a2, a3) : pack_hi(a2, a3);
+          } else {
+            qsf[s][0] = pack_hi(a0, a1);
+            qsf[s][1] = pack_hi(a2, a3);
+            if constexpr (!PACK) {
+              qsf2[s][0] = pack_lo(a0, a1);
+              qsf2[s][1] = pack_lo(a2, a3);
+            }
+          }
+        }
+      }
+    }
+    float acc[8][4];
+#pragma unroll
+    for (int i = 0; i < 8; ++i) acc[i][0] = acc[i][1] = acc[i][2] = acc[i][3] = 0.f;
+    float m_run[2] = {-INFINITY, -INFINITY}, M_run[2] = {-INFINITY, -INFINITY};
+    float l_run[2] = {0.f, 0.f};
+
+    const int64_t kbase = (int64_t)b * p.ksb + (int64_t)kvh * p.ksh;
+    const int64_t vbase = (int64_t)b * p.vsb + (int64_t)kvh * p.vsh;
+    const int64_t nchunks = (t1 - t0 + kChunk - 1) / kChunk;
+    const int64_t per_warp = (nchunks + kWarps - 1) / kWarps;
+    const int64_t c_begin = min(nchunks, (int64_t)warp * per_warp);
+    const int64_t c_end = min(nchunks, c_begin + per_warp);
+
+    CR nxt;
+    if (c_begin < c_end) load_chunk(nxt, p, t0 + c_begin * kChunk, t0, t1, kbase, vbase, g8, tig);
+    for (int64_t ci = c_begin; ci < c_end; ++ci) {
+      const int64_t j0 = t0 + ci * kChunk;
+      CR cur = nxt;
+      if (ci + 1 < c_end) load_chunk(nxt, p, j0 + kChunk, t0, t1, kbase, vbase, g8, tig);
+      // -------- scores: rows (ms, r) -> token j0 + 16 ms + 8 r + g8
+      float sc[2][4];
+      float nvl[2][2];  // log2 n_V of the lane's rows
+#pragma unroll
+      for (int ms = 0; ms < 2; ++ms) {
+        const auto &kw = cur.kw[ms];
+        const auto &qj = cur.qj[ms];
+        float kn[2], kr[2];
+#pragma unroll
+        for (int r = 0; r < 2; ++r) {
+          const bool ok = cur.kn[ms][r] >= 0.f;
+          kn[r] = ok ? cur.kn[ms][r] * inv_sK : -1.f;
+          kr[r] = KPROD ? cur.kr[ms][r] * (kKappa * sK) : 0.f;  // the table holds s_K c
+          nvl[ms][r] = ok ? __log2f(cur.vn[ms][r]) : -INFINITY;
+        }
+        float cm[4] = {0.f, 0.f, 0.f, 0.f};
+        if constexpr (KBM > 0) {
+#define TQ_KSTEP(S)                                                               \
+  {                                                                               \
+    uint32_t a[4];                                                                \
+    a[0] = lut(smem, pair_addr<KBM, 2 * (S), KW>(kw[0], koff));                   \
+    a[1] = lut(smem, pair_addr<KBM, 2 * (S), KW>(kw[1], koff));                   \
+    a[2] = lut(smem, pair_addr<KBM, 2 * (S) + 1, KW>(kw[0], koff));               \
+    a[3] = lut(smem, pair_addr<KBM, 2 * (S) + 1, KW>(kw[1], koff));               \
+    mma16816(cm, a, qf[S][0], qf[S][1]);                                          \
+    if constexpr (!PACK) mma16816(cm, a, qf2[S][0], qf2[S][1]);                   \
+  }
+          TQ_KSTEP(0) TQ_KSTEP(1) TQ_KSTEP(2) TQ_KSTEP(3)
+          TQ_KSTEP(4) TQ_KSTEP(5) TQ_KSTEP(6) TQ_KSTEP(7)
+#undef TQ_KSTEP
+        }
+        float cq[4] = {0.f, 0.f, 0.f, 0.f};
+        if constexpr (KPROD) {
+#define TQ_QSTEP(S)                                                               \
+  {                                                                               \
+    uint32_t a[4];                                                                \
+    a[0] = qjl_half2<2 * (S)>(qj[0]);                                             \
+    a[1] = qjl_half2<2 * (S)>(qj[1]);                                             \
+    a[2] = qjl_half2<2 * (S) + 1>(qj[0]);                                         \
+    a[3] = qjl_half2<2 * (S) + 1>(qj[1]);                                         \
+    mma16816(cq, a, qsf[S][0], qsf[S][1]);                                        \
+    if constexpr (!PACK) mma16816(cq, a, qsf2[S][0], qsf2[S][1]);                 \
+  }
+          TQ_QSTEP(0) TQ_QSTEP(1) TQ_QSTEP(2) TQ_QSTEP(3)
+          TQ_QSTEP(4) TQ_QSTEP(5) TQ_QSTEP(6) TQ_QSTEP(7)
+#undef TQ_QSTEP
+        }
+        // s = n/s_K * (main + kappa gamma s_K qjl): the LUT holds s_K c
+#pragma unroll
+        for (int i = 0; i < 4; ++i) {
+          float s = cm[i];
+          if constexpr (KPROD) s = fmaf(kr[i >> 1], cq[i], s);
+          if constexpr (PACK) s += __shfl_xor_sync(dev::kFull, s, 2);  // hi + lo columns
+          cm[i] = s;
+        }
+#pragma unroll
+        for (int r = 0; r < 2; ++r) {
+#pragma unroll
+          for (int c = 0; c < 2; ++c) {
+            const float s = cm[2 * r + c] * kn[r];
+            const int head = PACK ? 2 * (tig & 1) + c : 2 * tig + c;
+            if (p.scores && kn[r] >= 0.f && head < gh && (!PACK || tig < 2)) {
+              const int64_t j = j0 + 16 * ms + 8 * r + g8;
+              p.scores[((int64_t)b * p.Hq + h0 + head) * p.seq_len + j] = s;
+            }
+            sc[ms][2 * r + c] = kn[r] >= 0.f ? s * p.scale_log2 : -INFINITY;
+          }
+        }
+      }
+
+      // -------- online softmax, per head column c
+      float wgt[2][4];
+#pragma unroll
+      for (int c = 0; c < 2; ++c) {
+        float mx = fmaxf(fmaxf(sc[0][c], sc[0][2 + c]), fmaxf(sc[1][c], sc[1][2 + c]));
+        float Mx = fmaxf(fmaxf(sc[0][c] + nvl[0][0], sc[0][2 + c] + nvl[0][1]),
+                         fmaxf(sc[1][c] + nvl[1][0], sc[1][2 + c] + nvl[1][1]));
+#pragma unroll
+        for (int o = 4; o <= 16; o <<= 1) {
+          mx = fmaxf(mx, __shfl_xor_sync(dev::kFull, mx, o));
+          Mx = fmaxf(Mx, __shfl_xor_sync(dev::kFull, Mx, o));
+        }
+        const float mn = fmaxf(m_run[c], mx), Mn = fmaxf(M_run[c], Mx);
+        const float ms_ = mn == -INFINITY ? 0.f : mn;
+        const float Ms_ = Mn == -INFINITY ? 0.f : Mn;
+        const float al = exp2f(m_run[c] - ms_), aM = exp2f(M_run[c] - Ms_);
+        m_run[c] = mn;
+        M_run[c] = Mn;
+        float ls = 0.f;
+#pragma unroll
+        for (int ms = 0; ms < 2; ++ms) {
+#pragma unroll
+          for (int r = 0; r < 2; ++r) {
+            const float t = sc[ms][2 * r + c];
+            ls += exp2f(t - ms_);
+            wgt[ms][2 * r + c] = exp2f(t + nvl[ms][r] - Ms_);
+          }
+        }
+        l_run[c] = fmaf(l_run[c], al, ls);
+#pragma unroll
+        for (int mt = 0; mt < 8; ++mt) {
+          acc[mt][c] *= aM;
+          acc[mt][2 + c] *= aM;
+        }
+      }
+
+      // -------- PV: for each 16-token half, B = W^T via movmatrix
+#pragma unroll
+      for (int ms = 0; ms < 2; ++ms) {
+        uint32_t b0, b1, b2 = 0u, b3 = 0u;
+        if constexpr (PACK) {
+          // lanes tig < 2 carry the hi halves (columns 0-3), tig >= 2 the lo
+          const bool lo = tig >= 2;
+          b0 = movmatrix_trans(lo ? pack_lo(wgt[ms][0], wgt[ms][1]) : pack_hi(wgt[ms][0], wgt[ms][1]));
+          b1 = movmatrix_trans(lo ? pack_lo(wgt[ms][2], wgt[ms][3]) : pack_hi(wgt[ms][2], wgt[ms][3]));
+        } else {
+          b0 = movmatrix_trans(pack_hi(wgt[ms][0], wgt[ms][1]));
+          b1 = movmatrix_trans(pack_hi(wgt[ms][2], wgt[ms][3]));
+          b2 = movmatrix_trans(pack_lo(wgt[ms][0], wgt[ms][1]));
+          b3 = movmatrix_trans(pack_lo(wgt[ms][2], wgt[ms][3]));
+        }
+        // this lane's 4 tokens: 2 tig, 2 tig + 1, 2 tig + 8, 2 tig + 9 (of 16)
+        const auto &vw = cur.vw[ms];
+        if constexpr (VBM == 4) {
+          // cross-nibble bytes: (token a, dim) | (token b, dim) << 4
+          uint32_t x0[2][2], x1[2][2];
+#pragma unroll
+          for (int pr = 0; pr < 2; ++pr) {
+#pragma unroll
+            for (int w = 0; w < 2; ++w) {
+              const uint32_t wa = vw[2 * pr][w], wb = vw[2 * pr + 1][w];
+              x0[pr][w] = (wa & 0x0F0F0F0Fu) | ((wb << 4) & 0xF0F0F0F0u);
+              x1[pr][w] = ((wa >> 4) & 0x0F0F0F0Fu) | (wb & 0xF0F0F0F0u);
+            }
+          }
+#define TQ_VSTEP4(MT)                                                             \
+  {                                                                               \
+    uint32_t a[4];                                                                \
+    a[0] = lut(smem, pair_addr<4, MT, 2>(x0[0], voff));                       \
+    a[1] = lut(smem, pair_addr<4, MT, 2>(x1[0], voff));                           \
+    a[2] = lut(smem, pair_addr<4, MT, 2>(x0[1], voff));                           \
+    a[3] = lut(smem, pair_addr<4, MT, 2>(x1[1], voff));                           \
+    mma16816(acc[MT], a, b0, b1);                                                 \
+    if constexpr (!PACK) mma16816(acc[MT], a, b2, b3);                            \
+  }
+          TQ_VSTEP4(0) TQ_VSTEP4(1) TQ_VSTEP4(2) TQ_VSTEP4(3)
+          TQ_VSTEP4(4) TQ_VSTEP4(5) TQ_VSTEP4(6) TQ_VSTEP4(7)
+#undef TQ_VSTEP4
+        } else {
+#define TQ_VSTEP(MT)                                                              \
+  {                                                                               \
+    const uint32_t h0_ = lut(smem, pair_addr<VBM, MT, VW>(vw[0], voff));          \
+    const uint32_t h1_ = lut(smem, pair_addr<VBM, MT, VW>(vw[1], voff));          \
+    const uint32_t h2_ = lut(smem, pair_addr<VBM, MT, VW>(vw[2], voff));          \
+    const uint32_t h3_ = lut(smem, pair_addr<VBM, MT, VW>(vw[3], voff));          \
+    uint32_t a[4];                                                                \
+    a[0] = __byte_perm(h0_, h1_, 0x5410);                                         \
+    a[1] = __byte_perm(h0_, h1_, 0x7632);                                         \
+    a[2] = __byte_perm(h2_, h3_, 0x5410);                                         \
+    a[3] = __byte_perm(h2_, h3_, 0x7632);                                         \
+    mma16816(acc[MT], a, b0, b1);                                                 \
+    if constexpr (!PACK) mma16816(acc[MT], a, b2, b3);                            \
+  }
+          TQ_VSTEP(0) TQ_VSTEP(1) TQ_VSTEP(2) TQ_VSTEP(3)
+          TQ_VSTEP(4) TQ_VSTEP(5) TQ_VSTEP(6) TQ_VSTEP(7)
+#undef TQ_VSTEP
+        }
+      }
+    }
+
+    // ---- warp totals: l over the 8 row groups; PACK: hi + lo columns of acc
+#pragma unroll
+    for (int c = 0; c < 2; ++c) {
+#pragma unroll
+      for (int o = 4; o <= 16; o <<= 1) l_run[c] += __shfl_xor_sync(dev::kFull, l_run[c], o);
+    }
+    if constexpr (PACK) {
+#pragma unroll
+      for (int mt = 0; mt < 8; ++mt) {
+#pragma unroll
+        for (int i = 0; i < 4; ++i) acc[mt][i] += __shfl_xor_sync(dev::kFull, acc[mt][i], 2);
+      }
+    }
+
+    // ---- CTA merge of the warps' partials for this piece
+    {
+      float *wp = s_part + (size_t)warp * 8 * kPW;
+      const bool writer = PACK ? tig < 2 : true;
+      if (writer) {
+#pragma unroll
+        for (int c = 0; c < 2; ++c) {
+          const int hh = PACK ? 2 * tig + c : 2 * tig + c;
+          if (g8 == 0) {
+            wp[hh * kPW + 0] = m_run[c];
+            wp[hh * kPW + 1] = l_run[c];
+            wp[hh * kPW + 2] = M_run[c];
+          }
+#pragma unroll
+          for (int mt = 0; mt < 8; ++mt) {
+            // C row g8 -> dim 16 g8 + 2 mt, row g8 + 8 -> dim 16 g8 + 2 mt + 1
+            wp[hh * kPW + 4 + 16 * g8 + 2 * mt] = acc[mt][c];
+            wp[hh * kPW + 4 + 16 * g8 + 2 * mt + 1] = acc[mt][2 + c];
+          }
+        }
+      }
+    }
+    __syncthreads();
+    {
+      float *dst = p.ws + p.slot0 + ((int64_t)u + blockIdx.x) * kSlot;
+      for (int o = tid; o < gh * (kD + 3); o += kThreads) {
+        const int hh = o / (kD + 3), e = o % (kD + 3);
+        float mstar = -INFINITY, Mstar = -INFINITY;
+#pragma unroll
+        for (int w = 0; w < kWarps; ++w) {
+          mstar = fmaxf(mstar, s_part[(w * 8 + hh) * kPW + 0]);
+          Mstar = fmaxf(Mstar, s_part[(w * 8 + hh) * kPW + 2]);
+        }
+        const float m0 = mstar == -INFINITY ? 0.f : mstar;
+        const float M0 = Mstar == -INFINITY ? 0.f : Mstar;
+        float v = 0.f;
+        if (e == 0) {
+          v = mstar;
+        } else if (e == 2) {
+          v = Mstar;
+        } else if (e == 1) {
+#pragma unroll
+          for (int w = 0; w < kWarps; ++w) {
+            const float *q = s_part + (w * 8 + hh) * kPW;
+            v += q[1] * exp2f(q[0] - m0);
+          }
+        } else {
+          const int dd = e - 3;
+#pragma unroll
+          for (int w = 0; w < kWarps; ++w) {
+            const float *q = s_part + (w * 8 + hh) * kPW;
+            v += q[4 + dd] * exp2f(q[2] - M0);
+          }
+          v *= inv_sV;
+        }
+        dst[hh * kPW + (e < 3 ? e : e + 1)] = v;
+      }
+    }
+  }
+}
+
+// ----------------------------------------------------------- combine
+
+// One warp per (batch, query head): merge the slots of its unit, o' / l,
+// then o = sigma_V * H o' / sqrt(d).
+__global__ void __launch_bounds__(32) decode_combine_kernel(CombineParams p) {
+  const int lane = threadIdx.x;
+  const int bh = blockIdx.x;
+  const int b = bh / p.Hq, hq = bh % p.Hq;
+  const int kvh = hq / p.g, grp = (hq % p.g) / 8, hh = (hq % p.g) % 8;
+  const int UH = p.Hkv * p.groups;
+  const int u = b * UH + kvh * p.groups + grp;
+  float *out = p.out + (int64_t)bh * kD + lane * 4;
+  const int64_t T = flat_total(p.seq_lens, p.seq_len, p.B, UH);
+  int64_t ustart, ulen;
+  if (p.seq_lens) {
+    ustart = 0;
+    for (int bb = 0; bb < b; ++bb) ustart += batch_len(p.seq_lens, p.seq_len, bb) * UH;
+    ulen = batch_len(p.seq_lens, p.seq_len, b);
+    ustart += (int64_t)(kvh * p.groups + grp) * ulen;
+  } else {
+    ustart = (int64_t)u * p.seq_len;
+    ulen = p.seq_len;
+  }
+  float mstar = -INFINITY, Mstar = -INFINITY;
+  int c0 = 0, c1 = -1;
+  if (ulen > 0 && T > 0) {
+    // first CTA whose range [cut(c), cut(c+1)) contains ustart
+    c0 = (int)(((uint64_t)ustart * (uint64_t)p.ctas) / (uint64_t)T);
+    while (c0 > 0 && cut(T, p.ctas, c0) > ustart) --c0;
+    while (c0 + 1 < p.ctas && cut(T, p.ctas, c0 + 1) <= ustart) ++c0;
+    const int64_t uend = ustart + ulen;
+    int64_t lo = cut(T, p.ctas, c0);
+    for (int c = c0; c < p.ctas && lo < uend; ++c) {
+      const int64_t hi = cut(T, p.ctas, c + 1);
+      if (hi > lo) {
+        const float *q = p.ws + p.slot0 + ((int64_t)u + c) * kSlot + hh * kPW;
+        mstar = fmaxf(mstar, q[0]);
+        Mstar = fmaxf(Mstar, q[2]);
+        c1 = c;
+      }
+      lo = hi;
+    }
+  }
+  if (mstar == -INFINITY) {
+    *reinterpret_cast<float4 *>(out) = make_float4(0.f, 0.f, 0.f, 0.f);
+    return;
+  }
+  const float M0 = Mstar == -INFINITY ? 0.f : Mstar;
+  float l = 0.f;
+  float a[4] = {0.f, 0.f, 0.f, 0.f};
+  int64_t lo = cut(T, p.ctas, c0);
+  for (int c = c0; c <= c1; ++c) {
+    const int64_t hi = cut(T, p.ctas, c + 1);
+    if (hi > lo) {
+      const float *q = p.ws + p.slot0 + ((int64_t)u + c) * kSlot + hh * kPW;
+      l += q[1] * exp2f(q[0] - mstar);
+      const float wM = exp2f(q[2] - M0);
+      const float4 v = *reinterpret_cast<const float4 *>(q + 4 + lane * 4);
+      a[0] = fmaf(v.x, wM, a[0]);
+      a[1] = fmaf(v.y, wM, a[1]);
+      a[2] = fmaf(v.z, wM, a[2]);
+      a[3] = fmaf(v.w, wM, a[3]);
+    }
+    lo = hi;
+  }
+  const float f = exp2f(M0 - mstar) / l * 0.08838834764831845f;
+#pragma unroll
+  for (int i = 0; i < 4; ++i) a[i] *= f;
+  dev::fwht<32, 4>(a, lane);
+  float o[4];
+#pragma unroll
+  for (int i = 0; i < 4; ++i) o[i] = p.vsign[lane * 4 + i] < 0 ? -a[i] : a[i];
+  *reinterpret_cast<float4 *>(out) = make_float4(o[0], o[1], o[2], o[3]);
+}
+
+__global__ void zero_out_kernel(float *out, int64_t n) {
+  const int64_t i = (int64_t)blockIdx.x * blockDim.x + threadIdx.x;
+  if (i < n) out[i] = 0.f;
+}
+
+constexpr size_t split_smem_bytes(int warps) {
+  return kLutBytes + 2 * 8 * kD * sizeof(float) + (size_t)warps * 8 * kPW * sizeof(float);
+}
+
+template <int KBM, bool KPROD, int VBM, bool PACK>
+cudaError_t run_split(const SplitParams &sp, cudaStream_t s) {
+  auto kern = decode_split_kernel<KBM, KPROD, VBM, PACK>;
+  const int warps = 8;
+  const size_t smem = split_smem_bytes(warps);
+  cudaError_t e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
+  if (e != cudaSuccess) return e;
+  kern<<<sp.ctas, warps * 32, smem, s>>>(sp);
+  return cudaGetLastError();
+}
+
+template <bool KPROD, int VBM, bool PACK>
+cudaError_t by_kbits(int kbm, const SplitParams &sp, cudaStream_t s) {
+  switch (kbm) {
+    case 0: if constexpr (KPROD) return run_split<0, true, VBM, PACK>(sp, s); else return cudaErrorInvalidValue;
+    case 1: return run_split<1, KPROD, VBM, PACK>(sp, s);
+    case 2: return run_split<2, KPROD, VBM, PACK>(sp, s);
+    case 3: return run_split<3, KPROD, VBM, PACK>(sp, s);
+    case 4: return run_split<4, KPROD, VBM, PACK>(sp, s);
+  }
+  return cudaErrorInvalidValue;
+}
+
+template <int VBM>
+cudaError_t by_kvariant(int kbm, bool kprod, bool pack, const SplitParams &sp, cudaStream_t s) {
+  if (pack) return kprod ? by_kbits<true, VBM, true>(kbm, sp, s) : by_kbits<false, VBM, true>(kbm, sp, s);
+  return kprod ? by_kbits<true, VBM, false>(kbm, sp, s) : by_kbits<false, VBM, false>(kbm, sp, s);
+}
+
+}  // namespace
+
+bool decode_supported(int d, int kbm, bool kprod, int vbm, bool vprod) {
+  return d == kD && !vprod && vbm >= 1 && vbm <= 4 && kbm >= (kprod ? 0 : 1) && kbm <= 4;
+}
+
+size_t decode_workspace_floats(int B, int Hq, int Hkv, bool prod, int ctas) {
+  const int64_t units = (int64_t)B * Hkv * ((Hq / Hkv + 7) / 8);
+  return (size_t)kHdr + (size_t)B * Hq * kD * (prod ? 2 : 1) + (size_t)(units + ctas) * kSlot;
+}
+
+cudaError_t launch_decode(const DecodeArgs &a, cudaStream_t s) {
+  const int64_t outn = (int64_t)a.B * a.Hq * kD;
+  if (a.seq_len == 0) {
+    zero_out_kernel<<<(unsigned)((outn + 255) / 256), 256, 0, s>>>(a.out, outn);
+    return cudaGetLastError();
+  }
+  SplitParams sp{};
+  sp.q = a.q;
+  sp.q_dtype = a.q_dtype;
+  sp.B = a.B;
+  sp.Hq = a.Hq;
+  sp.Hkv = a.Hkv;
+  sp.g = a.Hq / a.Hkv;
+  sp.groups = (sp.g + 7) / 8;
+  sp.seq_len = a.seq_len;
+  sp.seq_lens = a.seq_lens;
+  sp.ctas = a.splits;
+  sp.kc = a.k.codes;
+  sp.kj = a.k.qjl;
+  sp.kn = a.k.norms;
+  sp.kr = a.k.rnorms;
+  sp.ksb = a.k.sb;
+  sp.ksh = a.k.sh;
+  sp.ksn = a.k.sn;
+  sp.kcent = a.kq.centroids;
+  sp.ksign = a.kq.signs;
+  sp.kS = a.kq.S;
+  sp.vc = a.v.codes;
+  sp.vn = a.v.norms;
+  sp.vsb = a.v.sb;
+  sp.vsh = a.v.sh;
+  sp.vsn = a.v.sn;
+  sp.vcent = a.vq.centroids;
+  sp.scale_log2 = a.scale * kLog2e;
+  sp.scores = a.scores;
+  sp.ws = a.ws;
+  sp.slot0 = (int64_t)kHdr + (int64_t)a.B * a.Hq * kD * (a.kq.prod ? 2 : 1);
+  PrepParams pp{a.q, a.q_dtype, a.B * a.Hq, a.kq.signs, a.kq.prod ? a.kq.S : nullptr,
+                a.kq.centroids, a.kq.bm, a.vq.centroids, a.vq.bm, a.ws};
+  decode_prep_kernel<<<(a.B * a.Hq + 1) / 2 + 2, 256, 0, s>>>(pp);
+  cudaError_t pe = cudaGetLastError();
+  if (pe != cudaSuccess) return pe;
+  const bool pack = sp.g <= 4;
+  cudaError_t e = cudaErrorInvalidValue;
+  switch (a.vq.bm) {
+    case 1: e = by_kvariant<1>(a.kq.bm, a.kq.prod, pack, sp, s); break;
+    case 2: e = by_kvariant<2>(a.kq.bm, a.kq.prod, pack, sp, s); break;
+    case 3: e = by_kvariant<3>(a.kq.bm, a.kq.prod, pack, sp, s); break;
+    case 4: e = by_kvariant<4>(a.kq.bm, a.kq.prod, pack, sp, s); break;
+  }
+  if (e != cudaSuccess) return e;
+  CombineParams cp{a.B, a.Hq, a.Hkv, sp.g, sp.groups, a.seq_len, a.seq_lens, sp.ctas, sp.slot0, a.ws,
+                   a.vq.signs, a.out};
+  decode_combine_kernel<<<a.B * a.Hq, 32, 0, s>>>(cp);
+  return cudaGetLastError();
+}
+
+}  // namespace tq

@@ -1,0 +1,223 @@
+// Device helpers shared by the TurboQuant kernels (sm_100a).
+//
+// Vector layout inside a kernel: a d-vector is held by T consecutive lanes,
+// lane t of the group owning the contiguous block of E = d/T elements
+// [t*E, t*E + E) in registers.  Butterfly stages whose stride h is >= E pair
+// lanes t and t ^ (h/E); the rest stay in registers.  Every add, subtract,
+// multiply and square root below is IEEE round-to-nearest with no
+// contraction, so the encode reproduces the canonical fp32 procedure bit for
+// bit whatever T is.
+#pragma once
+
+#include <cuda_bf16.h>
+#include <cuda_fp16.h>
+#include <cuda_runtime.h>
+#include <stdint.h>
+
+namespace tq {
+namespace dev {
+
+constexpr unsigned kFull = 0xffffffffu;
+
+// ---------------------------------------------------------------- loading
+
+__device__ __forceinline__ float bf16lo(uint32_t w) { return __uint_as_float(w << 16); }
+__device__ __forceinline__ float bf16hi(uint32_t w) { return __uint_as_float(w & 0xffff0000u); }
+__device__ __forceinline__ float f16lo(uint32_t w) {
+  return __half2float(__ushort_as_half((unsigned short)(w & 0xffffu)));
+}
+__device__ __forceinline__ float f16hi(uint32_t w) {
+  return __half2float(__ushort_as_half((unsigned short)(w >> 16)));
+}
+
+// E contiguous elements of dtype DT (0 f32, 1 bf16, 2 f16) from a 16-byte
+// aligned address, widened exactly to fp32.
+template <int DT, int E>
+__device__ __forceinline__ void load_block(const void *p, float (&v)[E]) {
+  if constexpr (DT == 0) {
+    const float4 *q = reinterpret_cast<const float4 *>(p);
+#pragma unroll
+    for (int i = 0; i < E / 4; ++i) {
+      const float4 t = __ldg(q + i);
+      v[4 * i + 0] = t.x;
+      v[4 * i + 1] = t.y;
+      v[4 * i + 2] = t.z;
+      v[4 * i + 3] = t.w;
+    }
+  } else {
+    const uint4 *q = reinterpret_cast<const uint4 *>(p);
+#pragma unroll
+    for (int i = 0; i < E / 8; ++i) {
+      const uint4 t = __ldg(q + i);
+      const uint32_t w[4] = {t.x, t.y, t.z, t.w};
+#pragma unroll
+      for (int k = 0; k < 4; ++k) {
+        if constexpr (DT == 1) {
+          v[8 * i + 2 * k] = bf16lo(w[k]);
+          v[8 * i + 2 * k + 1] = bf16hi(w[k]);
+        } else {
+          v[8 * i + 2 * k] = f16lo(w[k]);
+          v[8 * i + 2 * k + 1] = f16hi(w[k]);
+        }
+      }
+    }
+  }
+}
+
+// ------------------------------------------------------------ butterflies
+
+// One cross-lane FWHT stage: the lane whose group index has bit P clear holds
+// a (gets a+b), its partner holds b (gets a-b).
+template <int E>
+__device__ __forceinline__ void fwht_cross(float (&a)[E], int P, bool low) {
+#pragma unroll
+  for (int i = 0; i < E; ++i) {
+    const float o = __shfl_xor_sync(kFull, a[i], P);
+    a[i] = low ? __fadd_rn(a[i], o) : __fsub_rn(o, a[i]);
+  }
+}
+
+// In-register FWHT stages h = E/2, ..., 1.
+template <int E>
+__device__ __forceinline__ void fwht_local(float (&a)[E]) {
+#pragma unroll
+  for (int h = E / 2; h >= 1; h >>= 1) {
+#pragma unroll
+    for (int i = 0; i < E; ++i) {
+      if ((i & h) == 0) {
+        const float x = a[i], y = a[i + h];
+        a[i] = __fadd_rn(x, y);
+        a[i + h] = __fsub_rn(x, y);
+      }
+    }
+  }
+}
+
+// Full unnormalised FWHT of a d = T*E vector, stages h = d/2 .. 1.
+template <int T, int E>
+__device__ __forceinline__ void fwht(float (&a)[E], int t) {
+#pragma unroll
+  for (int P = T / 2; P >= 1; P >>= 1) fwht_cross<E>(a, P, (t & P) == 0);
+  fwht_local<E>(a);
+}
+
+// Fold-halves sum of a[] over the d = T*E vector: for h = d/2, .., 1,
+// a_i <- fl(a_i + a_{i+h}) for i < h.  Destroys a[]; every lane of the group
+// returns the same value (fl(x+y) = fl(y+x)).
+template <int T, int E>
+__device__ __forceinline__ float fold_halves_sum(float (&a)[E]) {
+#pragma unroll
+  for (int P = T / 2; P >= 1; P >>= 1) {
+#pragma unroll
+    for (int i = 0; i < E; ++i) a[i] = __fadd_rn(a[i], __shfl_xor_sync(kFull, a[i], P));
+  }
+#pragma unroll
+  for (int h = E / 2; h >= 1; h >>= 1) {
+#pragma unroll
+    for (int i = 0; i < h; ++i) a[i] = __fadd_rn(a[i], a[i + h]);
+  }
+  return a[0];
+}
+
+// -------------------------------------------------------------- quantize
+
+// idx = #{j : u > t_j} for an antisymmetric codebook with K = 2^BM levels,
+// given the bit patterns P[0..K/2-2] of the positive thresholds
+// t_{K/2}..t_{K-2} (the middle threshold is 0).  For u > 0,
+// idx = K/2 + #{m : P_m < |u|}; for u <= 0 (and NaN), idx = K/2 - 1 -
+// #{m : P_m <= |u|}.  Non-negative floats order like their bit patterns, so
+// both counts are #{m : P_m < A} with A = bits(|u|) + [u <= 0], found by an
+// unrolled binary search over the sorted P.
+template <int BM>
+__device__ __forceinline__ int quantize_sym(float u, const uint32_t (&P)[(1 << BM) / 2]) {
+  constexpr int K = 1 << BM;
+  const bool pos = u > 0.0f;
+  const uint32_t A = (__float_as_uint(u) & 0x7fffffffu) + (pos ? 0u : 1u);
+  int k = 0;
+  if constexpr (BM == 2) {
+    k = A > P[0] ? 1 : 0;
+  } else if constexpr (BM == 3) {
+    k = A > P[1] ? 2 : 0;
+    const uint32_t t = k ? P[2] : P[0];
+    k += A > t ? 1 : 0;
+  } else if constexpr (BM == 4) {
+    k = A > P[3] ? 4 : 0;
+    const uint32_t t1 = k ? P[5] : P[1];
+    k += A > t1 ? 2 : 0;
+    const uint32_t lo = (k & 2) ? P[2] : P[0];
+    const uint32_t hi = (k & 2) ? P[6] : P[4];
+    const uint32_t t2 = (k & 4) ? hi : lo;
+    k += A > t2 ? 1 : 0;
+  }
+  return pos ? (K / 2 + k) : (K / 2 - 1 - k);
+}
+
+// ----------------------------------------------------------- bit packing
+
+// Places the BM-bit field of element j (of E) into the LSB-first bitstream
+// held in W[] (E*BM/32 words).
+template <int BM, int NW>
+__device__ __forceinline__ void put_field(uint32_t (&W)[NW], int j, uint32_t v) {
+  const int p = j * BM;
+  const int w = p >> 5, s = p & 31;
+  W[w] |= v << s;
+  if (s + BM > 32) W[w + 1] |= v >> (32 - s);
+}
+
+template <int BM, int NW>
+__device__ __forceinline__ uint32_t get_field(const uint32_t (&W)[NW], int j) {
+  const int p = j * BM;
+  const int w = p >> 5, s = p & 31;
+  uint32_t v = W[w] >> s;
+  if (s + BM > 32) v |= W[w + 1] << (32 - s);
+  return v & ((1u << BM) - 1u);
+}
+
+// Stores NW words to a 4*NW-byte aligned destination with the widest
+// vector access the size allows.
+template <int NW>
+__device__ __forceinline__ void store_words(void *dst, const uint32_t (&W)[NW]) {
+  if constexpr (NW % 4 == 0) {
+    uint4 *d = reinterpret_cast<uint4 *>(dst);
+#pragma unroll
+    for (int i = 0; i < NW / 4; ++i) d[i] = make_uint4(W[4 * i], W[4 * i + 1], W[4 * i + 2], W[4 * i + 3]);
+  } else if constexpr (NW % 2 == 0) {
+    uint2 *d = reinterpret_cast<uint2 *>(dst);
+#pragma unroll
+    for (int i = 0; i < NW / 2; ++i) d[i] = make_uint2(W[2 * i], W[2 * i + 1]);
+  } else {
+    uint32_t *d = reinterpret_cast<uint32_t *>(dst);
+#pragma unroll
+    for (int i = 0; i < NW; ++i) d[i] = W[i];
+  }
+}
+
+template <int NW>
+__device__ __forceinline__ void load_words(const void *src, uint32_t (&W)[NW]) {
+  if constexpr (NW % 4 == 0) {
+    const uint4 *s = reinterpret_cast<const uint4 *>(src);
+#pragma unroll
+    for (int i = 0; i < NW / 4; ++i) {
+      const uint4 t = __ldg(s + i);
+      W[4 * i] = t.x;
+      W[4 * i + 1] = t.y;
+      W[4 * i + 2] = t.z;
+      W[4 * i + 3] = t.w;
+    }
+  } else if constexpr (NW % 2 == 0) {
+    const uint2 *s = reinterpret_cast<const uint2 *>(src);
+#pragma unroll
+    for (int i = 0; i < NW / 2; ++i) {
+      const uint2 t = __ldg(s + i);
+      W[2 * i] = t.x;
+      W[2 * i + 1] = t.y;
+    }
+  } else {
+    const uint32_t *s = reinterpret_cast<const uint32_t *>(src);
+#pragma unroll
+    for (int i = 0; i < NW; ++i) W[i] = __ldg(s + i);
+  }
+}
+
+}  // namespace dev
+}  // namespace tq

@@ -1,0 +1,442 @@
+// Host half of the TurboQuant C ABI: codebook fitting, seeded parameters,
+// argument validation and dispatch to the CUDA launchers.
+//
+// Codebook: Lloyd-Max scalar quantizer for the coordinate law after a random
+// rotation, N(0, 1/d) by default or the exact C (1-x^2)^((d-3)/2)
+// ("TurboQuant của Google: nén KV cache 6 lần", sections "Trick đầu tiên"
+// and "Lloyd-Max quantizer: chia bucket đúng chỗ"; "The Distortion
+// Guarantee", section "The Gap").  Procedure (the pages give none): Lloyd's
+// alternation in double -- thresholds at midpoints, centroids at conditional
+// means -- from levels equally spaced on [-2, 2] (N(0,1) units) until no
+// centroid moves by 1e-15; the exact law starts from the Gaussian levels
+// / sqrt(d), integrates every cell with 128-node Gauss-Legendre and stops at
+// 1e-16.  The levels are made exactly antisymmetric, the Gaussian ones are
+// divided by sqrt(d), thresholds are double midpoints, and everything is
+// rounded once to fp32.
+//
+// Seeded parameters: SplitMix64 (Steele, Lea, Flood 2014), output k of seed s
+// = mix(s + (k+1) * 0x9E3779B97F4A7C15); sign i is -1 when bit 63 of output i
+// is set; S entry e comes from Box-Muller on outputs 2(e/2), 2(e/2)+1 mapped
+// to (o >> 11) 2^-53, the first replaced by 1-u, cos for even e and sin for
+// odd e, in double, rounded to fp32.
+
+#include "../../include/tq.h"
+#include "tq_internal.h"
+
+#include <cuda_runtime.h>
+
+#include <algorithm>
+#include <cmath>
+#include <cstdarg>
+#include <cstdio>
+#include <cstring>
+#include <string>
+#include <vector>
+
+namespace {
+
+thread_local std::string g_last_error;
+
+tq_status fail(tq_status s, const char *fmt, ...) __attribute__((format(printf, 2, 3)));
+tq_status fail(tq_status s, const char *fmt, ...) {
+  char buf[512];
+  va_list ap;
+  va_start(ap, fmt);
+  vsnprintf(buf, sizeof(buf), fmt, ap);
+  va_end(ap);
+  g_last_error = buf;
+  return s;
+}
+
+tq_status cuda_fail(cudaError_t e, const char *what) {
+  return fail(TQ_ECUDA, "%s: %s", what, cudaGetErrorString(e));
+}
+
+// ---------------------------------------------------------------- codebook
+
+const double kSqrt2 = 1.4142135623730951;
+const double kInvSqrt2Pi = 0.3989422804014327;
+
+double phi(double x) {
+  if (std::isinf(x)) return 0.0;
+  return kInvSqrt2Pi * std::exp(-0.5 * x * x);
+}
+
+double upper_tail(double x) {
+  if (x == INFINITY) return 0.0;
+  if (x == -INFINITY) return 1.0;
+  return 0.5 * std::erfc(x / kSqrt2);
+}
+
+double mass(double a, double b) {
+  if (a >= 0.0) return upper_tail(a) - upper_tail(b);
+  if (b <= 0.0) return upper_tail(-b) - upper_tail(-a);
+  return 1.0 - upper_tail(b) - upper_tail(-a);
+}
+
+void antisymmetrize(std::vector<double> &c) {
+  const int K = (int)c.size();
+  std::vector<double> o(c);
+  for (int i = 0; i < K; ++i) c[i] = 0.5 * (o[i] - o[K - 1 - i]);
+}
+
+std::vector<double> lloyd_max_gauss(int K) {
+  std::vector<double> c(K), t(K + 1), nc(K);
+  for (int i = 0; i < K; ++i) c[i] = -2.0 + 4.0 * i / (K - 1);
+  for (int sweep = 0; sweep < 200000; ++sweep) {
+    t[0] = -INFINITY;
+    t[K] = INFINITY;
+    for (int i = 0; i + 1 < K; ++i) t[i + 1] = 0.5 * (c[i] + c[i + 1]);
+    double delta = 0.0;
+    for (int i = 0; i < K; ++i) {
+      nc[i] = (phi(t[i]) - phi(t[i + 1])) / mass(t[i], t[i + 1]);
+      delta = std::fmax(delta, std::fabs(nc[i] - c[i]));
+    }
+    c = nc;
+    if (delta < 1e-15) break;
+  }
+  antisymmetrize(c);
+  return c;
+}
+
+// Gauss-Legendre nodes/weights on [-1, 1] by Newton on the Legendre
+// recurrence (Golub-Welsch would do as well; any accurate rule works).
+void gauss_legendre(int n, std::vector<double> &x, std::vector<double> &w) {
+  x.assign(n, 0.0);
+  w.assign(n, 0.0);
+  for (int i = 0; i < n; ++i) {
+    double z = std::cos(M_PI * (i + 0.75) / (n + 0.5));
+    double dp = 1.0;
+    for (int it = 0; it < 100; ++it) {
+      double p0 = 1.0, p1 = z;
+      for (int k = 2; k <= n; ++k) {
+        double p2 = ((2.0 * k - 1.0) * z * p1 - (k - 1.0) * p0) / k;
+        p0 = p1;
+        p1 = p2;
+      }
+      dp = n * (z * p1 - p0) / (z * z - 1.0);
+      double dz = p1 / dp;
+      z -= dz;
+      if (std::fabs(dz) < 1e-16) break;
+    }
+    x[n - 1 - i] = z;
+    w[n - 1 - i] = 2.0 / ((1.0 - z * z) * dp * dp);
+  }
+}
+
+std::vector<double> lloyd_max_beta(int K, int d) {
+  std::vector<double> gx, gw;
+  gauss_legendre(128, gx, gw);
+  std::vector<double> c = lloyd_max_gauss(K), t(K + 1), nc(K);
+  const double sd = std::sqrt((double)d);
+  for (int i = 0; i < K; ++i) c[i] /= sd;
+  const double ex = 0.5 * (d - 3);
+  for (int sweep = 0; sweep < 200000; ++sweep) {
+    t[0] = -1.0;
+    t[K] = 1.0;
+    for (int i = 0; i + 1 < K; ++i) t[i + 1] = 0.5 * (c[i] + c[i + 1]);
+    double delta = 0.0;
+    for (int i = 0; i < K; ++i) {
+      const double half = 0.5 * (t[i + 1] - t[i]);
+      const double mid = 0.5 * (t[i + 1] + t[i]);
+      double m0 = 0.0, m1 = 0.0;
+      for (size_t g = 0; g < gx.size(); ++g) {
+        const double xx = mid + half * gx[g];
+        const double f = std::exp(ex * std::log1p(-xx * xx));
+        m0 += gw[g] * f;
+        m1 += gw[g] * xx * f;
+      }
+      nc[i] = (half * m1) / (half * m0);
+      delta = std::fmax(delta, std::fabs(nc[i] - c[i]));
+    }
+    c = nc;
+    if (delta < 1e-16) break;
+  }
+  antisymmetrize(c);
+  return c;
+}
+
+// ------------------------------------------------------------- SplitMix64
+
+uint64_t splitmix64(uint64_t seed, uint64_t k) {
+  uint64_t z = seed + (k + 1) * 0x9E3779B97F4A7C15ull;
+  z = (z ^ (z >> 30)) * 0xBF58476D1CE4E5B9ull;
+  z = (z ^ (z >> 27)) * 0x94D049BB133111EBull;
+  return z ^ (z >> 31);
+}
+
+double unit53(uint64_t v) { return (double)(v >> 11) * (1.0 / 9007199254740992.0); }
+
+// ------------------------------------------------------------- validation
+
+bool valid_d(int d) { return d == 64 || d == 128 || d == 256; }
+
+tq_status check_quantizer(const tq_quantizer *q, const char *name, tq::QuantParams *out) {
+  if (!q) return fail(TQ_EINVAL, "%s: quantizer is NULL", name);
+  if (!valid_d(q->d)) return fail(TQ_EINVAL, "%s: d=%d (expected 64, 128 or 256)", name, q->d);
+  if (q->bits < 1 || q->bits > 4) return fail(TQ_EINVAL, "%s: bits=%d (expected 1..4)", name, q->bits);
+  if (q->variant != TQ_MSE && q->variant != TQ_PROD)
+    return fail(TQ_EINVAL, "%s: variant=%d", name, q->variant);
+  if (q->rotation == TQ_ROT_DENSE)
+    return fail(TQ_EUNSUPPORTED, "%s: dense rotation is not implemented", name);
+  if (q->rotation != TQ_ROT_HADAMARD) return fail(TQ_EINVAL, "%s: rotation=%d", name, q->rotation);
+  const bool prod = q->variant == TQ_PROD;
+  const int bm = prod ? q->bits - 1 : q->bits;
+  if (bm > 0 && (!q->centroids || !q->thresholds))
+    return fail(TQ_EINVAL, "%s: centroids/thresholds are NULL", name);
+  if (!q->signs) return fail(TQ_EINVAL, "%s: signs are NULL", name);
+  if (prod && !q->qjl_S) return fail(TQ_EINVAL, "%s: prod quantizer without qjl_S", name);
+  if (prod && (uintptr_t)q->qjl_S % 16) return fail(TQ_EINVAL, "%s: qjl_S not 16-byte aligned", name);
+  out->d = q->d;
+  out->bm = bm;
+  out->prod = prod;
+  out->centroids = q->centroids;
+  out->thresholds = q->thresholds;
+  out->signs = q->signs;
+  out->S = q->qjl_S;
+  out->sqrt_d = (float)std::sqrt((double)q->d);
+  return TQ_OK;
+}
+
+bool aligned(const void *p, size_t a) { return ((uintptr_t)p % a) == 0; }
+
+size_t dtype_size(int dt) { return dt == TQ_F32 ? 4 : 2; }
+
+tq_status check_view(const tq_cache_view *v, const tq::QuantParams &q, const char *name,
+                     bool need_all, tq::CacheView *out) {
+  if (!v) return fail(TQ_EINVAL, "%s: cache view is NULL", name);
+  if (need_all) {
+    if (q.bm > 0 && !v->codes) return fail(TQ_EINVAL, "%s: codes are NULL", name);
+    if (!v->norms) return fail(TQ_EINVAL, "%s: norms are NULL", name);
+    if (q.prod && (!v->qjl || !v->rnorms)) return fail(TQ_EINVAL, "%s: prod needs qjl and rnorms", name);
+  }
+  if (v->codes && !aligned(v->codes, 16)) return fail(TQ_EINVAL, "%s: codes not 16-byte aligned", name);
+  if (v->qjl && !aligned(v->qjl, 16)) return fail(TQ_EINVAL, "%s: qjl not 16-byte aligned", name);
+  if (v->norms && !aligned(v->norms, 4)) return fail(TQ_EINVAL, "%s: norms not 4-byte aligned", name);
+  if (v->rnorms && !aligned(v->rnorms, 4)) return fail(TQ_EINVAL, "%s: rnorms not 4-byte aligned", name);
+  if (v->stride_b < 0 || v->stride_h < 0 || v->stride_n < 0)
+    return fail(TQ_EINVAL, "%s: negative stride", name);
+  out->codes = v->codes;
+  out->qjl = q.prod ? v->qjl : nullptr;
+  out->norms = v->norms;
+  out->rnorms = q.prod ? v->rnorms : nullptr;
+  out->sb = v->stride_b;
+  out->sh = v->stride_h;
+  out->sn = v->stride_n;
+  return TQ_OK;
+}
+
+int g_num_sms = 0;
+
+int num_sms() {
+  if (g_num_sms > 0) return g_num_sms;
+  int dev = 0, n = 0;
+  if (cudaGetDevice(&dev) == cudaSuccess &&
+      cudaDeviceGetAttribute(&n, cudaDevAttrMultiProcessorCount, dev) == cudaSuccess && n > 0)
+    g_num_sms = n;
+  else
+    g_num_sms = 148;
+  return g_num_sms;
+}
+
+}  // namespace
+
+// ------------------------------------------------------------ split policy
+
+namespace tq {
+
+// One persistent CTA per SM of the current device.
+int decode_ctas() { return num_sms(); }
+
+}  // namespace tq
+
+// -------------------------------------------------------------------- ABI
+
+extern "C" {
+
+tq_status tq_make_codebook(int32_t d, int32_t bits_mse, tq_codebook_dist dist, float *centroids,
+                           float *thresholds) {
+  if (!valid_d(d)) return fail(TQ_EINVAL, "tq_make_codebook: d=%d", d);
+  if (bits_mse < 1 || bits_mse > 4) return fail(TQ_EINVAL, "tq_make_codebook: bits_mse=%d", bits_mse);
+  if (!centroids || !thresholds) return fail(TQ_EINVAL, "tq_make_codebook: NULL output");
+  const int K = 1 << bits_mse;
+  std::vector<double> c;
+  if (dist == TQ_CB_GAUSS) {
+    c = lloyd_max_gauss(K);
+    const double sd = std::sqrt((double)d);
+    for (double &v : c) v /= sd;
+  } else if (dist == TQ_CB_BETA) {
+    c = lloyd_max_beta(K, d);
+  } else {
+    return fail(TQ_EINVAL, "tq_make_codebook: dist=%d", (int)dist);
+  }
+  for (int i = 0; i < K; ++i) centroids[i] = (float)c[i];
+  for (int i = 0; i + 1 < K; ++i) thresholds[i] = (float)(0.5 * (c[i] + c[i + 1]));
+  return TQ_OK;
+}
+
+tq_status tq_make_signs(uint64_t seed, int32_t d, int8_t *signs) {
+  if (!valid_d(d)) return fail(TQ_EINVAL, "tq_make_signs: d=%d", d);
+  if (!signs) return fail(TQ_EINVAL, "tq_make_signs: NULL output");
+  for (int i = 0; i < d; ++i) signs[i] = (splitmix64(seed, (uint64_t)i) >> 63) ? -1 : 1;
+  return TQ_OK;
+}
+
+tq_status tq_make_qjl(uint64_t seed, int32_t d, float *S) {
+  if (!valid_d(d)) return fail(TQ_EINVAL, "tq_make_qjl: d=%d", d);
+  if (!S) return fail(TQ_EINVAL, "tq_make_qjl: NULL output");
+  const int64_t n = (int64_t)d * d;
+  for (int64_t p = 0; p < (n + 1) / 2; ++p) {
+    const double u1 = 1.0 - unit53(splitmix64(seed, 2 * p));
+    const double u2 = unit53(splitmix64(seed, 2 * p + 1));
+    const double r = std::sqrt(-2.0 * std::log(u1));
+    const double ang = 2.0 * M_PI * u2;
+    S[2 * p] = (float)(r * std::cos(ang));
+    if (2 * p + 1 < n) S[2 * p + 1] = (float)(r * std::sin(ang));
+  }
+  return TQ_OK;
+}
+
+size_t tq_code_bytes(int32_t d, int32_t bits, int32_t variant) {
+  const int bm = variant == TQ_PROD ? bits - 1 : bits;
+  return bm > 0 ? (size_t)d * bm / 8 : 0;
+}
+
+size_t tq_qjl_bytes(int32_t d, int32_t variant) { return variant == TQ_PROD ? (size_t)d / 8 : 0; }
+
+tq_status tq_encode(const tq_quantizer *q, const void *x, tq_dtype x_dtype, int64_t B, int64_t H,
+                    int64_t N, int64_t x_stride_b, int64_t x_stride_h, int64_t x_stride_n,
+                    const tq_cache_view *out, tq_stream_t stream) {
+  tq::EncodeArgs a{};
+  tq_status st = check_quantizer(q, "tq_encode", &a.q);
+  if (st != TQ_OK) return st;
+  if (x_dtype != TQ_F32 && x_dtype != TQ_BF16 && x_dtype != TQ_F16)
+    return fail(TQ_EINVAL, "tq_encode: x_dtype=%d", (int)x_dtype);
+  if (B < 0 || H < 0 || N < 0) return fail(TQ_EINVAL, "tq_encode: negative size");
+  if (x_stride_b < 0 || x_stride_h < 0 || x_stride_n < 0)
+    return fail(TQ_EINVAL, "tq_encode: negative stride");
+  if (B == 0 || H == 0 || N == 0) return TQ_OK;
+  st = check_view(out, a.q, "tq_encode(out)", true, &a.out);
+  if (st != TQ_OK) return st;
+  if (!x) return fail(TQ_EINVAL, "tq_encode: x is NULL");
+  const size_t es = dtype_size(x_dtype);
+  if (!aligned(x, 16) || (x_stride_b * es) % 16 || (x_stride_h * es) % 16 || (x_stride_n * es) % 16)
+    return fail(TQ_EINVAL, "tq_encode: x and its strides must be 16-byte aligned");
+  if (!tq::encode_supported(a.q.d, a.q.bm, a.q.prod, x_dtype))
+    return fail(TQ_EUNSUPPORTED, "tq_encode: d=%d b_m=%d prod=%d dtype=%d not built", a.q.d, a.q.bm,
+                (int)a.q.prod, (int)x_dtype);
+  a.x = x;
+  a.dtype = x_dtype;
+  a.B = B;
+  a.H = H;
+  a.N = N;
+  a.xsb = x_stride_b;
+  a.xsh = x_stride_h;
+  a.xsn = x_stride_n;
+  cudaError_t e = tq::launch_encode(a, (cudaStream_t)stream);
+  if (e != cudaSuccess) return cuda_fail(e, "tq_encode launch");
+  return TQ_OK;
+}
+
+tq_status tq_dequant(const tq_quantizer *q, const tq_cache_view *in, int64_t B, int64_t H, int64_t N,
+                     float *out, tq_stream_t stream) {
+  tq::DequantArgs a{};
+  tq_status st = check_quantizer(q, "tq_dequant", &a.q);
+  if (st != TQ_OK) return st;
+  if (B < 0 || H < 0 || N < 0) return fail(TQ_EINVAL, "tq_dequant: negative size");
+  if (B == 0 || H == 0 || N == 0) return TQ_OK;
+  st = check_view(in, a.q, "tq_dequant(in)", true, &a.in);
+  if (st != TQ_OK) return st;
+  if (!out || !aligned(out, 16)) return fail(TQ_EINVAL, "tq_dequant: out NULL or not 16-byte aligned");
+  a.B = B;
+  a.H = H;
+  a.N = N;
+  a.out = out;
+  cudaError_t e = tq::launch_dequant(a, (cudaStream_t)stream);
+  if (e != cudaSuccess) return cuda_fail(e, "tq_dequant launch");
+  return TQ_OK;
+}
+
+size_t tq_decode_workspace_bytes(int32_t B, int32_t Hq, int32_t Hkv, int64_t seq_len, int32_t d) {
+  if (B <= 0 || Hq <= 0 || Hkv <= 0 || seq_len <= 0 || Hq % Hkv || !valid_d(d)) return 0;
+  // sized for TurboQuant_prod keys (the larger case) so the query needs no quantizer
+  return tq::decode_workspace_floats(B, Hq, Hkv, true, tq::decode_ctas()) * sizeof(float);
+}
+
+tq_status tq_decode_attention(const tq_quantizer *kq, const tq_quantizer *vq, const void *q,
+                              tq_dtype q_dtype, int32_t B, int32_t Hq, int32_t Hkv, int64_t seq_len,
+                              const int32_t *seq_lens, const tq_cache_view *k,
+                              const tq_cache_view *v, float softmax_scale, float *out,
+                              float *scores_out, void *workspace, size_t workspace_bytes,
+                              tq_stream_t stream) {
+  tq::DecodeArgs a{};
+  tq_status st = check_quantizer(kq, "tq_decode_attention(kq)", &a.kq);
+  if (st != TQ_OK) return st;
+  st = check_quantizer(vq, "tq_decode_attention(vq)", &a.vq);
+  if (st != TQ_OK) return st;
+  if (a.kq.d != a.vq.d) return fail(TQ_EINVAL, "tq_decode_attention: K d=%d but V d=%d", a.kq.d, a.vq.d);
+  if (a.vq.prod) return fail(TQ_EUNSUPPORTED, "tq_decode_attention: prod values are not implemented");
+  if (q_dtype != TQ_F32 && q_dtype != TQ_BF16 && q_dtype != TQ_F16)
+    return fail(TQ_EINVAL, "tq_decode_attention: q_dtype=%d", (int)q_dtype);
+  if (B < 0 || Hq < 0 || Hkv < 0 || seq_len < 0) return fail(TQ_EINVAL, "tq_decode_attention: negative size");
+  if (Hkv == 0 || Hq % Hkv) return fail(TQ_EINVAL, "tq_decode_attention: Hq=%d not a multiple of Hkv=%d", Hq, Hkv);
+  if (!std::isfinite(softmax_scale)) return fail(TQ_EINVAL, "tq_decode_attention: softmax_scale not finite");
+  if (B == 0 || Hq == 0) return TQ_OK;
+  st = check_view(k, a.kq, "tq_decode_attention(k)", seq_len > 0, &a.k);
+  if (st != TQ_OK) return st;
+  st = check_view(v, a.vq, "tq_decode_attention(v)", seq_len > 0, &a.v);
+  if (st != TQ_OK) return st;
+  if (!q || !aligned(q, 16)) return fail(TQ_EINVAL, "tq_decode_attention: q NULL or not 16-byte aligned");
+  if (!out || !aligned(out, 16)) return fail(TQ_EINVAL, "tq_decode_attention: out NULL or not 16-byte aligned");
+  if (scores_out && !aligned(scores_out, 4)) return fail(TQ_EINVAL, "tq_decode_attention: scores_out misaligned");
+  if (!tq::decode_supported(a.kq.d, a.kq.bm, a.kq.prod, a.vq.bm, a.vq.prod))
+    return fail(TQ_EUNSUPPORTED, "tq_decode_attention: d=%d K b_m=%d prod=%d V b_m=%d not built", a.kq.d,
+                a.kq.bm, (int)a.kq.prod, a.vq.bm);
+  a.q = q;
+  a.q_dtype = q_dtype;
+  a.B = B;
+  a.Hq = Hq;
+  a.Hkv = Hkv;
+  a.seq_len = seq_len;
+  a.seq_lens = seq_lens;
+  a.scale = softmax_scale;
+  a.out = out;
+  a.scores = scores_out;
+  if (seq_len > 0) {
+    const size_t need = tq_decode_workspace_bytes(B, Hq, Hkv, seq_len, a.kq.d);
+    if (workspace_bytes < need || !workspace || !aligned(workspace, 16))
+      return fail(TQ_EWORKSPACE, "tq_decode_attention: workspace %zu bytes, need %zu (16-byte aligned)",
+                  workspace_bytes, need);
+    a.splits = tq::decode_ctas();
+    a.ws = (float *)workspace;
+  }
+  cudaError_t e = tq::launch_decode(a, (cudaStream_t)stream);
+  if (e != cudaSuccess) return cuda_fail(e, "tq_decode_attention launch");
+  return TQ_OK;
+}
+
+tq_status tq_check(tq_stream_t stream) {
+  cudaError_t e = cudaStreamSynchronize((cudaStream_t)stream);
+  if (e != cudaSuccess) return cuda_fail(e, "tq_check");
+  e = cudaGetLastError();
+  if (e != cudaSuccess) return cuda_fail(e, "tq_check");
+  return TQ_OK;
+}
+
+const char *tq_status_string(tq_status s) {
+  switch (s) {
+    case TQ_OK: return "TQ_OK";
+    case TQ_EINVAL: return "TQ_EINVAL";
+    case TQ_EUNSUPPORTED: return "TQ_EUNSUPPORTED";
+    case TQ_ECUDA: return "TQ_ECUDA";
+    case TQ_EWORKSPACE: return "TQ_EWORKSPACE";
+    case TQ_ETIMEOUT: return "TQ_ETIMEOUT";
+  }
+  return "TQ_UNKNOWN";
+}
+
+const char *tq_last_error(void) { return g_last_error.c_str(); }
+
+const char *tq_version(void) { return "tq-b200 0.1.0 (sm_100a)"; }
+
+}  // extern "C"

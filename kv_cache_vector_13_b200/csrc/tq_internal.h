@@ -1,0 +1,76 @@
+// Internal interface between the host library (tq_host.cpp) and the CUDA
+// launchers (tq_encode.cu, tq_dequant.cu, tq_decode.cu).  Not installed.
+#pragma once
+
+#include <cuda_runtime.h>
+#include <stdint.h>
+
+namespace tq {
+
+// Everything a kernel needs about one quantizer, resolved on the host.
+struct QuantParams {
+  int d;
+  int bm;          // MSE bits b_m (0..4)
+  bool prod;
+  const float *centroids;   // 2^bm
+  const float *thresholds;  // 2^bm - 1
+  const int8_t *signs;      // d
+  const float *S;           // d*d (prod)
+  float sqrt_d;             // fl32(sqrt(d)) (double sqrt rounded once)
+};
+
+struct CacheView {
+  uint8_t *codes;
+  uint8_t *qjl;
+  float *norms;
+  float *rnorms;
+  int64_t sb, sh, sn;  // record strides
+};
+
+struct EncodeArgs {
+  QuantParams q;
+  const void *x;
+  int dtype;           // tq_dtype
+  int64_t B, H, N;
+  int64_t xsb, xsh, xsn;  // element strides
+  CacheView out;
+};
+
+struct DequantArgs {
+  QuantParams q;
+  CacheView in;
+  int64_t B, H, N;
+  float *out;
+};
+
+struct DecodeArgs {
+  QuantParams kq, vq;
+  const void *q;
+  int q_dtype;
+  int B, Hq, Hkv;
+  int64_t seq_len;
+  const int32_t *seq_lens;
+  CacheView k, v;
+  float scale;
+  float *out;
+  float *scores;
+  float *ws;           // partial slots
+  int splits;          // persistent CTAs of the split kernel
+};
+
+// Decode work split shared by the workspace query and the launch: the number
+// of persistent CTAs, and the workspace size in floats (a header with the
+// centroid tables, the rotated queries, and (units + CTAs) partial slots,
+// units = B * Hkv * ceil((Hq/Hkv) / 8)).
+int decode_ctas();
+size_t decode_workspace_floats(int B, int Hq, int Hkv, bool prod, int ctas);
+
+cudaError_t launch_encode(const EncodeArgs &a, cudaStream_t s);
+cudaError_t launch_dequant(const DequantArgs &a, cudaStream_t s);
+cudaError_t launch_decode(const DecodeArgs &a, cudaStream_t s);
+
+// Whether a (d, bm, prod, dtype) encode instantiation exists.
+bool encode_supported(int d, int bm, bool prod, int dtype);
+bool decode_supported(int d, int kbm, bool kprod, int vbm, bool vprod);
+
+}  // namespace tq

@@ -31,50 +31,57 @@ from . import rotation as _rot
 LOG2E = 1.4426950408889634
 
 
-def _scores_one(qz, q, cache, lo=0, hi=None, dtype=np.float64):
-    """Estimator <q, k_j> for tokens lo..hi-1 of one (batch, kv head) slice.
+_CHUNK = 1 << 16
+
+
+def _scores_one(qz, q, cache, dtype=np.float64):
+    """Estimator <q, k_j> for every token of one (batch, kv head) slice.
 
     ``cache``: dict(codes [N, nb], norms [N], qjl, rnorms) for that slice.
+    Tokens are unpacked in chunks only to bound memory.
     """
     f = dtype
     d = qz.d
-    if hi is None:
-        hi = cache["norms"].shape[0]
+    N = cache["norms"].shape[0]
     sig = qz.signs.astype(f)
     if f == np.float64:
         qp = _rot.rotate_f64(q, qz.signs)
     else:
         qp = _rot.fwht_f32((np.asarray(q, np.float32) * sig)[None, :])[0] / np.float32(math.sqrt(d))
-    n = cache["norms"][lo:hi].astype(f)
-    if qz.bm > 0:
-        idx = _qz.unpack_bits(cache["codes"][lo:hi], d, qz.bm)
-        main = qz.centroids.astype(f)[idx] @ qp.astype(f)
-    else:
-        main = np.zeros(hi - lo, f)
-    if qz.prod:
-        qs = qz.S.astype(f) @ qp.astype(f)
-        sg = (2 * _qz.unpack_bits(cache["qjl"][lo:hi], d, 1) - 1).astype(f)
-        gam = cache["rnorms"][lo:hi].astype(f)
-        main = main + gam * f(_qz.SQRT_HALF_PI / d) * (sg @ qs)
-    return n * main
+    qs = qz.S.astype(f) @ qp.astype(f) if qz.prod else None
+    out = np.empty(N, f)
+    for lo in range(0, N, _CHUNK):
+        hi = min(N, lo + _CHUNK)
+        n = cache["norms"][lo:hi].astype(f)
+        if qz.bm > 0:
+            idx = _qz.unpack_bits(cache["codes"][lo:hi], d, qz.bm)
+            main = qz.centroids.astype(f)[idx] @ qp.astype(f)
+        else:
+            main = np.zeros(hi - lo, f)
+        if qz.prod:
+            sg = (2 * _qz.unpack_bits(cache["qjl"][lo:hi], d, 1) - 1).astype(f)
+            gam = cache["rnorms"][lo:hi].astype(f)
+            main = main + gam * f(_qz.SQRT_HALF_PI / d) * (sg @ qs)
+        out[lo:hi] = n * main
+    return out
 
 
-def _values_one(vq, p, cache, lo=0, hi=None, dtype=np.float64):
-    """Pi_V^T sum_j p_j n_j v_hat_rot_j for one slice (p already normalised)."""
+def _values_one(vq, p, cache, dtype=np.float64):
+    """Pi_V^T sum_j p_j v_hat_rot_j n_j for one slice (p already normalised)."""
     f = dtype
     d = vq.d
-    if hi is None:
-        hi = cache["norms"].shape[0]
-    w = (p * cache["norms"][lo:hi].astype(f)).astype(f)
-    if vq.bm > 0:
-        idx = _qz.unpack_bits(cache["codes"][lo:hi], d, vq.bm)
-        op = w @ vq.centroids.astype(f)[idx]
-    else:
-        op = np.zeros(d, f)
-    if vq.prod:
-        sg = (2 * _qz.unpack_bits(cache["qjl"][lo:hi], d, 1) - 1).astype(f)
-        gam = cache["rnorms"][lo:hi].astype(f)
-        op = op + ((w * gam) @ sg) @ vq.S.astype(f) * f(_qz.SQRT_HALF_PI / d)
+    N = cache["norms"].shape[0]
+    op = np.zeros(d, f)
+    for lo in range(0, N, _CHUNK):
+        hi = min(N, lo + _CHUNK)
+        w = (p[lo:hi] * cache["norms"][lo:hi].astype(f)).astype(f)
+        if vq.bm > 0:
+            idx = _qz.unpack_bits(cache["codes"][lo:hi], d, vq.bm)
+            op = op + w @ vq.centroids.astype(f)[idx]
+        if vq.prod:
+            sg = (2 * _qz.unpack_bits(cache["qjl"][lo:hi], d, 1) - 1).astype(f)
+            gam = cache["rnorms"][lo:hi].astype(f)
+            op = op + ((w * gam) @ sg) @ vq.S.astype(f) * f(_qz.SQRT_HALF_PI / d)
     if f == np.float64:
         return _rot.unrotate_f64(op, vq.signs)
     sig = vq.signs.astype(np.float32)

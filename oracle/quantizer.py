@@ -109,17 +109,20 @@ def unpack_bits(packed: np.ndarray, d: int, width: int) -> np.ndarray:
     n = packed.shape[0]
     if width == 0:
         return np.zeros((n, d), np.int64)
-    bits = np.unpackbits(packed, axis=1, bitorder="little")[:, : d * width]
-    bits = bits.reshape(n, d, width).astype(np.int64)
-    return (bits << np.arange(width, dtype=np.int64)).sum(axis=2)
+    bits = np.unpackbits(packed, axis=1, bitorder="little")[:, : d * width].reshape(n, d, width)
+    out = np.zeros((n, d), np.int64)
+    for k in range(width):
+        out |= bits[:, :, k].astype(np.int64) << k
+    return out
 
 
-def encode(qz: Quantizer, x: np.ndarray, chunk: int = 8192) -> dict:
+def encode(qz: Quantizer, x: np.ndarray, chunk: int = 8192, aux: bool = True) -> dict:
     """Encode rows of ``x`` ([n, d], any float dtype holding the input values).
 
     Returns dict(codes [n, code_bytes] u8, norms [n] f32, and for prod
-    qjl [n, d/8] u8, rnorms [n] f32, z [n, d] f64 (the projections, kept so
-    tests can measure distance to the sign boundary), u [n, d] f32).
+    qjl [n, d/8] u8, rnorms [n] f32); with ``aux`` also u [n, d] f32 and, for
+    prod, z [n, d] f64 (the projections, kept so tests can measure the
+    distance to the sign boundary).
     """
     x = np.ascontiguousarray(x, dtype=np.float32)
     n, d = x.shape
@@ -143,15 +146,17 @@ def encode(qz: Quantizer, x: np.ndarray, chunk: int = 8192) -> dict:
             idx = np.zeros(u.shape, np.int64)
         out["codes"].append(pack_bits(idx, qz.bm))
         out["norms"].append(nrm)
-        out["u"].append(u)
+        if aux:
+            out["u"].append(u)
         if qz.prod:
             r = u - qz.centroids[idx] if qz.bm > 0 else u.copy()
             gam = np.sqrt(fold_halves_sum_f32(r * r))
             z = r.astype(np.float64) @ qz.S.astype(np.float64).T
             out["qjl"].append(pack_bits((z >= 0).astype(np.int64), 1))
             out["rnorms"].append(gam)
-            out["z"].append(z)
-    return {k: np.concatenate(v, axis=0) for k, v in out.items()}
+            if aux:
+                out["z"].append(z)
+    return {k: np.concatenate(v, axis=0) for k, v in out.items() if v}
 
 
 def rotated_estimate(qz: Quantizer, enc: dict) -> np.ndarray:

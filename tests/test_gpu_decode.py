@@ -1,0 +1,160 @@
+"""GPU parity of tq_decode_attention against the fp32 oracle.
+
+Tolerance: max |o - o_ref| / max |o_ref| <= 2e-3 per (batch, query head),
+against the oracle evaluated in fp32 on the oracle's own encoding of the
+same inputs (codes are bit-exact, so both see the same cache)."""
+
+import math
+
+import numpy as np
+import pytest
+import torch
+
+from kv_cache_vector_13_b200 import api, inputs
+from oracle import attention as OA
+
+from helpers import host, oracle_attention, oracle_cache_slices, oracle_twin, rel_err
+
+pytestmark = pytest.mark.gpu
+DEV = "cuda"
+TOL = 2e-3
+
+
+def run_case(B, Hq, Hkv, N, kspec, vspec, seed=0, seq_lens=None, kv_scale=1.0, heads=None, scores=False):
+    g = torch.Generator(device=DEV).manual_seed(seed)
+    d = 128
+    K = torch.randn((B, Hkv, N, d), generator=g, device=DEV) * kv_scale
+    V = torch.randn((B, Hkv, N, d), generator=g, device=DEV)
+    q = torch.randn((B, Hq, d), generator=g, device=DEV).to(torch.bfloat16)
+    kq = api.Quantizer(d, kspec[0], kspec[1], seed_rot=seed + 1, seed_qjl=seed + 2, device=DEV)
+    vq = api.Quantizer(d, vspec[0], vspec[1], seed_rot=seed + 3, device=DEV)
+    kc, vc = api.encode(kq, K), api.encode(vq, V)
+    sl = None if seq_lens is None else torch.tensor(seq_lens, dtype=torch.int32, device=DEV)
+    sc = torch.full((B, Hq, N), float("nan"), device=DEV) if scores else None
+    out = host(api.decode_attention(kq, vq, q, kc, vc, seq_lens=sl, scores=sc))
+    okq, ovq = oracle_twin(kq), oracle_twin(vq)
+    okc, _ = oracle_cache_slices(okq, host(K))
+    ovc, _ = oracle_cache_slices(ovq, host(V))
+    qh = host(q)
+    todo = heads or [(b, h) for b in range(B) for h in range(Hq)]
+    for (b, h) in todo:
+        L = N if seq_lens is None else seq_lens[b]
+        if L == 0:
+            assert np.all(out[b, h] == 0)
+            continue
+        kcs = {k: v[b:b + 1, :, :L] for k, v in okc.items()}
+        vcs = {k: v[b:b + 1, :, :L] for k, v in ovc.items()}
+        res = OA.decode_attention(okq, ovq, qh[b:b + 1].astype(np.float32), kcs, vcs, dtype=np.float32,
+                                  heads=[(0, h)], return_scores=scores)
+        ref = res[0] if scores else res
+        e = rel_err(out[b, h], ref[0, h])
+        assert e <= TOL, f"(b={b}, h={h}, L={L}) rel err {e:.2e}"
+        if scores:
+            s_gpu = host(sc)[b, h, :L]
+            s_ref = res[1][0, h]
+            np.testing.assert_allclose(s_gpu, s_ref, rtol=2e-3, atol=2e-3 * np.abs(s_ref).max())
+    return out
+
+
+@pytest.mark.parametrize("kspec,vspec", [((4, "mse"), (4, "mse")), ((3, "mse"), (3, "mse")),
+                                         ((3, "prod"), (3, "mse")), ((4, "prod"), (4, "mse")),
+                                         ((2, "mse"), (2, "mse")), ((1, "mse"), (1, "mse")),
+                                         ((2, "prod"), (1, "mse")), ((1, "prod"), (4, "mse"))])
+def test_decode_small_grid(kspec, vspec):
+    run_case(2, 8, 2, 1000 + 29, kspec, vspec, seed=10 * kspec[0] + vspec[0] + (100 if kspec[1] == 'prod' else 0), scores=True)
+
+
+@pytest.mark.parametrize("N", [1, 2, 31, 32, 33, 63, 64, 65, 257, 4097])
+def test_decode_ragged_lengths(N):
+    run_case(1, 4, 1, N, (4, "mse"), (4, "mse"), seed=N)
+
+
+@pytest.mark.parametrize("g", [1, 2, 4, 8, 16])
+def test_decode_gqa_group_sizes(g):
+    run_case(1, 2 * g, 2, 700, (3, "prod"), (3, "mse"), seed=g)
+
+
+def test_decode_per_batch_lengths_including_empty():
+    run_case(4, 4, 2, 900, (4, "mse"), (3, "mse"), seed=7, seq_lens=[900, 0, 1, 333])
+
+
+def test_decode_large_logits():
+    # sharp softmax: keys scaled so that a few tokens dominate
+    run_case(1, 8, 1, 2048, (4, "prod"), (4, "mse"), seed=9, kv_scale=6.0)
+
+
+def test_decode_config1_scores_shared_cache():
+    # one head, d=128, N=4096 keys from seed 0, 16 queries from seed 1, mse b=3:
+    # the 16 queries are a batch of 16 that shares one cache (stride_b = 0)
+    d, N = 128, 4096
+    x = inputs.vectors(N, d, seed=0, device=DEV)
+    qs = inputs.vectors(16, d, seed=1, device=DEV)
+    kq = api.Quantizer(d, 3, "mse", seed_rot=0, device=DEV)
+    vq = api.Quantizer(d, 3, "mse", seed_rot=1, device=DEV)
+    kc = api.encode(kq, x)
+    vc = api.encode(vq, x)
+    shared_k = api.PackedCache(kc.codes.expand(16, 1, N, -1), kc.norms.expand(16, 1, N))
+    shared_v = api.PackedCache(vc.codes.expand(16, 1, N, -1), vc.norms.expand(16, 1, N))
+    sc = torch.empty((16, 1, N), device=DEV)
+    out = host(api.decode_attention(kq, vq, qs[:, None, :].contiguous(), shared_k, shared_v, scores=sc))
+    okq, ovq = oracle_twin(kq), oracle_twin(vq)
+    okc, _ = oracle_cache_slices(okq, host(x)[None, None])
+    ovc, _ = oracle_cache_slices(ovq, host(x)[None, None])
+    qh = host(qs)
+    for i in range(16):
+        o, s = OA.decode_attention(okq, ovq, qh[i][None, None], okc, ovc, dtype=np.float32, return_scores=True)
+        assert rel_err(out[i, 0], o[0, 0]) <= TOL
+        np.testing.assert_allclose(host(sc)[i, 0], s[0, 0], rtol=1e-3, atol=1e-3 * np.abs(s).max())
+
+
+def test_decode_config2_full_size():
+    # Llama-3.1-8B-shaped layer: B=1, 32 q heads, 8 kv heads, N=32768, mse b=4
+    N = 32768
+    K, V = inputs.llama8b_kv(N=N, device=DEV)
+    q = inputs.queries(1, 32, device=DEV)
+    kq = api.Quantizer(128, 4, "mse", seed_rot=10, device=DEV)
+    vq = api.Quantizer(128, 4, "mse", seed_rot=11, device=DEV)
+    kc, vc = api.encode(kq, K), api.encode(vq, V)
+    out = host(api.decode_attention(kq, vq, q, kc, vc))
+    okq, ovq = oracle_twin(kq), oracle_twin(vq)
+    okc, _ = oracle_cache_slices(okq, host(K))
+    ovc, _ = oracle_cache_slices(ovq, host(V))
+    ref = oracle_attention(okq, ovq, host(q), okc, ovc)
+    e = rel_err(out, ref)
+    assert e.max() <= TOL, e.max()
+
+
+def sampled_decode(K, V, q, kq, vq, kv_heads):
+    kc, vc = api.encode(kq, K), api.encode(vq, V)
+    out = host(api.decode_attention(kq, vq, q, kc, vc))
+    okq, ovq = oracle_twin(kq), oracle_twin(vq)
+    Hq, Hkv = q.shape[1], K.shape[1]
+    g = Hq // Hkv
+    worst = 0.0
+    for (b, h) in kv_heads:
+        okc, _ = oracle_cache_slices(okq, host(K[b:b + 1, h:h + 1]))
+        ovc, _ = oracle_cache_slices(ovq, host(V[b:b + 1, h:h + 1]))
+        qb = host(q[b:b + 1, h * g:(h + 1) * g])
+        ref = oracle_attention(okq, ovq, qb, okc, ovc)
+        e = rel_err(out[b, h * g:(h + 1) * g], ref[0]).max()
+        worst = max(worst, e)
+        assert e <= TOL, (b, h, e)
+    return worst
+
+
+def test_decode_config3_sampled():
+    # batch 16, 32/8 heads, N=131072, 2% outlier channels x8; K prod b=3, V mse b=3
+    K, V = inputs.outlier_kv(N=131072, B=16, device=DEV)
+    q = inputs.queries(16, 32, device=DEV)
+    kq = api.Quantizer(128, 3, "prod", seed_rot=20, seed_qjl=21, device=DEV)
+    vq = api.Quantizer(128, 3, "mse", seed_rot=22, device=DEV)
+    sampled_decode(K, V, q, kq, vq, [(0, 0), (15, 7), (9, 3)])
+
+
+def test_decode_config5_sampled():
+    # 70B-shaped long context: B=1, 64/8 heads, N=2^20, Student-t values
+    K, V = inputs.student_kv(N=1 << 20, device=DEV)
+    q = inputs.queries(1, 64, device=DEV)
+    kq = api.Quantizer(128, 4, "prod", seed_rot=30, seed_qjl=31, device=DEV)
+    vq = api.Quantizer(128, 4, "mse", seed_rot=32, device=DEV)
+    sampled_decode(K, V, q, kq, vq, [(0, 0), (0, 5)])
