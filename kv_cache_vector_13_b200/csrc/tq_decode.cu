@@ -15,8 +15,9 @@
 // finds a scale s with fp16(s c_k) close to s c_k for every centroid (a
 // search over 4096 candidates in [1, 2)) and writes the 256-entry pair table
 // entry e -> half2(fp16(s c[e & m]), fp16(s c[(e >> b_m) & m])).
-// Kernel 1 (split), persistent: one CTA of 8 warps per SM; each warp keeps
-// its next chunk's loads in flight while it computes the current one.  The work is the
+// Kernel 1 (split), persistent: one CTA per SM (12 warps when a kv head has
+// <= 4 query heads and the keys are mse, else 8); a warp issues its next chunk's key loads as soon
+// as the current keys are scored and its value loads once PV is done.  The work is the
 // flattened space of (unit = batch x kv head x group of <= 8 query heads,
 // token) pairs, cut into one equal contiguous range per CTA; a range covers
 // one or a few "pieces" (CTA, unit).  Per CTA, once: the two pair tables are
@@ -40,9 +41,10 @@
 //     (for the normaliser l) and M over logit + log2 n_V (for the PV weights
 //     2^(u - M), which keeps p_j n_j in fp16 range).
 // The warps' partials (m, l, M, o') of a piece are merged in shared memory
-// and written to workspace slot (unit + CTA index).
-// Kernel 2 (combine): per (batch, query head), merge the slots of its unit,
-// divide by l, apply Pi_V^T = diag(sigma_V) H / sqrt(d).
+// and written to workspace slot (unit + CTA index).  Each CTA then bumps its
+// unit's counter; the CTA that completes the count merges the unit's slots,
+// divides by l and applies Pi_V^T = diag(sigma_V) H / sqrt(d).  No CTA waits
+// for another.
 
 #include "../../include/tq.h"
 #include "tq_device.cuh"
@@ -54,7 +56,8 @@ namespace tq {
 namespace {
 
 constexpr int kD = 128;
-constexpr int kMaxWarps = 8;
+constexpr int kMaxWarps = 12;
+constexpr int kMaxCtas = 1024;  // persistent CTAs supported (one per SM)
 constexpr int kChunk = 32;               // tokens per warp iteration
 constexpr int kLutBytes = 256 * 256;     // K and V pair tables, per-lane copies
 constexpr int kPW = kD + 4;              // floats per head in a partial: m, l, M, pad, o'[d]
@@ -91,7 +94,10 @@ struct SplitParams {
   float scale_log2;  // softmax_scale * log2(e)
   float *scores;
   float *ws;
-  int64_t slot0;  // first float of the partial slots
+  int64_t slot0;      // first float of the partial slots
+  unsigned *cnt;      // per-unit arrival counters (zeroed by the prep kernel)
+  float *out;
+  const int8_t *vsign;
 };
 
 struct PrepParams {
@@ -105,18 +111,14 @@ struct PrepParams {
   const float *vcent;
   int vbm;
   float *ws;
-};
-
-struct CombineParams {
-  int B, Hq, Hkv, g, groups;
+  unsigned *cnt;
+  int units;
+  int Hq;
   int64_t seq_len;
   const int32_t *seq_lens;
-  int ctas;
-  int64_t slot0;
-  const float *ws;
-  const int8_t *vsign;
   float *out;
 };
+
 
 // ------------------------------------------------------------------ PTX
 
@@ -344,6 +346,7 @@ __device__ void scale_and_table(const float *cent, int bm, float *inv_scale, uin
 // V scale and pair table.
 __global__ void __launch_bounds__(256) decode_prep_kernel(PrepParams p) {
   const int nqb = (p.nheads + 1) / 2;
+  for (int i = blockIdx.x * blockDim.x + threadIdx.x; i < p.units; i += gridDim.x * blockDim.x) p.cnt[i] = 0u;
   if ((int)blockIdx.x >= nqb) {
     if (blockIdx.x == (unsigned)nqb) {
       if (p.kbm > 0) scale_and_table(p.kcent, p.kbm, p.ws + 0, reinterpret_cast<uint32_t *>(p.ws + 64));
@@ -357,6 +360,9 @@ __global__ void __launch_bounds__(256) decode_prep_kernel(PrepParams p) {
   const int half = threadIdx.x >> 7, t = threadIdx.x & 127;
   const int head = blockIdx.x * 2 + half;
   const bool valid = head < p.nheads;
+  // a batch with no cached tokens has no work piece: its output is zero
+  if (valid && p.seq_lens && batch_len(p.seq_lens, p.seq_len, head / p.Hq) == 0)
+    p.out[(int64_t)head * kD + t] = 0.f;
   const int lane = threadIdx.x & 31;
   if ((t >> 5) == 0) {  // one warp per head: 4 dims per lane
     float a[4] = {0.f, 0.f, 0.f, 0.f};
@@ -402,62 +408,232 @@ __global__ void __launch_bounds__(256) decode_prep_kernel(PrepParams p) {
 
 // ------------------------------------------------------------ split kernel
 
-// Everything a lane loads from HBM for one 32-token chunk.  Score rows
-// (ms, r) are tokens j0 + 16 ms + 8 r + g8; PV tokens (ms, q4) are
-// j0 + 16 ms + 2 tig + (q4 & 1) + 8 (q4 >> 1).
-template <int KBM, bool KPROD, int VBM>
-struct ChunkRegs {
-  static constexpr int KW = KBM > 0 ? KBM : 1;
-  static constexpr int VW = VChunk<VBM>::NW;
-  uint32_t kw[2][2][KW];
+// One lane's loads for the key side of a 32-token chunk: score rows (ms, r)
+// are tokens 16 ms + 8 r + g8 of the chunk.  The value norms of the same
+// rows ride along (the softmax needs log2 n_V before PV).
+template <int KBM, bool KPROD>
+struct KBuf {
+  uint32_t w[2][2][KBM > 0 ? KBM : 1];
   uint32_t qj[2][2];
   float kn[2][2], kr[2][2], vn[2][2];
-  uint32_t vw[2][4][VW];
 };
 
-template <int KBM, bool KPROD, int VBM>
-__device__ __forceinline__ void load_chunk(ChunkRegs<KBM, KPROD, VBM> &c, const SplitParams &p, int64_t j0,
-                                           int64_t t0, int64_t t1, int64_t kbase, int64_t vbase, int g8,
-                                           int tig) {
+// The value codes of a chunk: PV tokens (ms, q4) are 16 ms + 2 tig +
+// (q4 & 1) + 8 (q4 >> 1), 16 dims [16 g8, 16 g8 + 16) each.
+template <int VBM>
+struct VBuf {
+  uint32_t w[2][4][VChunk<VBM>::NW];
+};
+
+// Per-piece row offsets (in records) of the lane's tokens inside a chunk.
+struct RowOffs {
+  int32_t k[2][2], kv[2][2], v[2][4];  // K rows, V records of the K rows, V tokens
+  int32_t rk[2][2], rv[2][4];          // token index inside the chunk
+};
+
+// Loads the key side of one chunk.  FAST: unit record strides and a full
+// chunk, so every address is a per-lane base plus a compile-time offset.
+template <bool FAST, int KBM, bool KPROD>
+__device__ __forceinline__ void load_k(KBuf<KBM, KPROD> &c, const SplitParams &p, int64_t krec0, int64_t vrec0,
+                                       int nvalid, const RowOffs &o, int tig, int g8) {
   constexpr int KCB = kD * KBM / 8;
-  constexpr int VCB = kD * VBM / 8;
+  if constexpr (FAST) {
+    const int64_t kr0 = krec0 + g8, vr0 = vrec0 + g8;
+    const uint8_t *kcp = p.kc + kr0 * KCB + tig * (4 * KBM);
+    const uint32_t *kjp = KPROD ? reinterpret_cast<const uint32_t *>(p.kj + kr0 * (kD / 8)) + tig : nullptr;
+    const float *knp = p.kn + kr0, *krp = KPROD ? p.kr + kr0 : nullptr, *vnp = p.vn + vr0;
+#pragma unroll
+    for (int ms = 0; ms < 2; ++ms) {
+#pragma unroll
+      for (int r = 0; r < 2; ++r) {
+        const int t = 16 * ms + 8 * r;  // compile-time after unrolling
+        if constexpr (KBM > 0) load_k32<KBM>(kcp + t * KCB, c.w[ms][r]);
+        if constexpr (KPROD) {
+          c.qj[ms][r] = __ldg(kjp + t * (kD / 32));
+          c.kr[ms][r] = __ldg(krp + t);
+        }
+        c.kn[ms][r] = __ldg(knp + t);
+        c.vn[ms][r] = __ldg(vnp + t);
+      }
+    }
+    return;
+  }
 #pragma unroll
   for (int ms = 0; ms < 2; ++ms) {
 #pragma unroll
     for (int r = 0; r < 2; ++r) {
-      const int64_t j = j0 + 16 * ms + 8 * r + g8;
-      const bool ok = j < t1;
-      const int64_t jj = ok ? j : t0;
-      const int64_t rec = kbase + jj * p.ksn;
-      if constexpr (KBM > 0) load_k32<KBM>(p.kc + rec * KCB + tig * (4 * KBM), c.kw[ms][r]);
+      const bool ok = o.rk[ms][r] < nvalid;
+      const int64_t rec = krec0 + o.k[ms][r];
+      if constexpr (KBM > 0) {
+        if (ok) {
+          load_k32<KBM>(p.kc + rec * KCB + tig * (4 * KBM), c.w[ms][r]);
+        } else {
+#pragma unroll
+          for (int i = 0; i < KBM; ++i) c.w[ms][r][i] = 0u;
+        }
+      }
       if constexpr (KPROD) {
-        c.qj[ms][r] = __ldg(reinterpret_cast<const uint32_t *>(p.kj + rec * (kD / 8)) + tig);
-        c.kr[ms][r] = __ldg(p.kr + rec);
+        c.qj[ms][r] = ok ? __ldg(reinterpret_cast<const uint32_t *>(p.kj + rec * (kD / 8)) + tig) : 0u;
+        c.kr[ms][r] = ok ? __ldg(p.kr + rec) : 0.f;
       }
       c.kn[ms][r] = ok ? __ldg(p.kn + rec) : -1.f;  // -1 marks a masked row
-      c.vn[ms][r] = __ldg(p.vn + vbase + jj * p.vsn);
-    }
-#pragma unroll
-    for (int q4 = 0; q4 < 4; ++q4) {
-      const int64_t j = j0 + 16 * ms + 2 * tig + (q4 & 1) + 8 * (q4 >> 1);
-      const int64_t vrec = vbase + (j < t1 ? j : t0) * p.vsn;
-      load_v16<VBM>(p.vc + vrec * VCB + g8 * (2 * VBM), c.vw[ms][q4], g8);
+      c.vn[ms][r] = ok ? __ldg(p.vn + vrec0 + o.kv[ms][r]) : 1.f;
     }
   }
 }
 
+template <bool FAST, int VBM>
+__device__ __forceinline__ void load_v(VBuf<VBM> &c, const SplitParams &p, int64_t vrec0, int nvalid,
+                                       const RowOffs &o, int g8, int tig) {
+  constexpr int VCB = kD * VBM / 8;
+  constexpr int NW = VChunk<VBM>::NW;
+  if constexpr (FAST) {
+    const uint8_t *vcp = p.vc + (vrec0 + 2 * tig) * VCB + g8 * (2 * VBM);
+#pragma unroll
+    for (int ms = 0; ms < 2; ++ms) {
+#pragma unroll
+      for (int q4 = 0; q4 < 4; ++q4) load_v16<VBM>(vcp + (16 * ms + (q4 & 1) + 8 * (q4 >> 1)) * VCB, c.w[ms][q4], g8);
+    }
+    return;
+  }
+#pragma unroll
+  for (int ms = 0; ms < 2; ++ms) {
+#pragma unroll
+    for (int q4 = 0; q4 < 4; ++q4) {
+      if (o.rv[ms][q4] < nvalid) {
+        load_v16<VBM>(p.vc + (vrec0 + o.v[ms][q4]) * VCB + g8 * (2 * VBM), c.w[ms][q4], g8);
+      } else {
+#pragma unroll
+        for (int i = 0; i < NW; ++i) c.w[ms][q4][i] = 0u;
+      }
+    }
+  }
+}
+
+// L2 prefetch hint for [ptr, ptr + bytes), shrunk inwards to 16-byte
+// boundaries so that every prefetched byte lies inside the range.
+__device__ __forceinline__ void prefetch_l2(const void *ptr, int64_t bytes) {
+  const uint64_t lo = ((uint64_t)ptr + 15u) & ~(uint64_t)15u;
+  const uint64_t hi = ((uint64_t)ptr + (uint64_t)bytes) & ~(uint64_t)15u;
+  if (hi > lo)
+    asm volatile("cp.async.bulk.prefetch.L2.global [%0], %1;\n" ::"l"(lo), "r"((uint32_t)(hi - lo)) : "memory");
+}
+
+// Prefetches the packed records of tokens [j, j + n) of one (batch, kv head)
+// slice into L2 (unit record strides only).
+template <int KBM, bool KPROD, int VBM>
+__device__ __forceinline__ void prefetch_chunk(const SplitParams &p, int64_t kr, int64_t vr, int64_t n) {
+  constexpr int KCB = kD * KBM / 8, VCB = kD * VBM / 8;
+  if constexpr (KBM > 0) prefetch_l2(p.kc + kr * KCB, n * KCB);
+  prefetch_l2(p.vc + vr * VCB, n * VCB);
+  prefetch_l2(p.kn + kr, n * 4);
+  prefetch_l2(p.vn + vr, n * 4);
+  if constexpr (KPROD) {
+    prefetch_l2(p.kj + kr * (kD / 8), n * (kD / 8));
+    prefetch_l2(p.kr + kr, n * 4);
+  }
+}
+
+__device__ __forceinline__ float ex2(float x) {
+  float y;
+  asm("ex2.approx.ftz.f32 %0, %1;\n" : "=f"(y) : "f"(x));
+  return y;
+}
+
+// Merge the slots of unit u (heads < gh) and write out[b, h0 + hh, :] =
+// sigma_V * H (o'/l) / sqrt(d).  One warp per head.  The lanes first read
+// every slot's (m, l, M) in parallel and turn them into weights kept in
+// shared memory (zero for CTAs with empty ranges), so the accumulation loop
+// has no data-dependent branch and its loads can all be in flight at once.
+__device__ void merge_unit(const SplitParams &p, const int64_t *cuts, int u, int c0, int c1, int b, int h0,
+                           int gh, int warp, int nwarps, int lane, float *s_w) {
+  const int n = c1 - c0 + 1;
+  for (int hh = warp; hh < gh; hh += nwarps) {
+    float *w = s_w + warp * (kMaxCtas + 1);
+    float mstar = -INFINITY, Mstar = -INFINITY;
+    for (int i = lane; i < n; i += 32) {
+      const int c = c0 + i;
+      if (cuts[c + 1] > cuts[c]) {
+        const float4 h = __ldcg(reinterpret_cast<const float4 *>(p.ws + p.slot0 + ((int64_t)u + c) * kSlot + hh * kPW));
+        mstar = fmaxf(mstar, h.x);
+        Mstar = fmaxf(Mstar, h.z);
+      }
+    }
+#pragma unroll
+    for (int o = 16; o >= 1; o >>= 1) {
+      mstar = fmaxf(mstar, __shfl_xor_sync(dev::kFull, mstar, o));
+      Mstar = fmaxf(Mstar, __shfl_xor_sync(dev::kFull, Mstar, o));
+    }
+    float *out = p.out + ((int64_t)b * p.Hq + h0 + hh) * kD + lane * 4;
+    if (mstar == -INFINITY) {
+      *reinterpret_cast<float4 *>(out) = make_float4(0.f, 0.f, 0.f, 0.f);
+      continue;
+    }
+    const float M0 = Mstar == -INFINITY ? 0.f : Mstar;
+    float l = 0.f;
+    for (int i = lane; i < n; i += 32) {
+      const int c = c0 + i;
+      float wi = 0.f;
+      if (cuts[c + 1] > cuts[c]) {
+        const float4 h = __ldcg(reinterpret_cast<const float4 *>(p.ws + p.slot0 + ((int64_t)u + c) * kSlot + hh * kPW));
+        l += h.y * ex2(h.x - mstar);
+        wi = ex2(h.z - M0);
+      }
+      w[i] = wi;
+    }
+#pragma unroll
+    for (int o = 16; o >= 1; o >>= 1) l += __shfl_xor_sync(dev::kFull, l, o);
+    __syncwarp();
+    float a[4] = {0.f, 0.f, 0.f, 0.f};
+    const float *base = p.ws + p.slot0 + ((int64_t)u + c0) * kSlot + hh * kPW + 4 + lane * 4;
+#pragma unroll 8
+    for (int i = 0; i < n; ++i) {
+      const float wi = w[i];
+      // an empty CTA never wrote its slot: read nothing there
+      const float4 v = wi != 0.f ? __ldcg(reinterpret_cast<const float4 *>(base + (int64_t)i * kSlot))
+                                 : make_float4(0.f, 0.f, 0.f, 0.f);
+      a[0] = fmaf(v.x, wi, a[0]);
+      a[1] = fmaf(v.y, wi, a[1]);
+      a[2] = fmaf(v.z, wi, a[2]);
+      a[3] = fmaf(v.w, wi, a[3]);
+    }
+    __syncwarp();
+    const float f = ex2(M0 - mstar) / l * 0.08838834764831845f;
+#pragma unroll
+    for (int i = 0; i < 4; ++i) a[i] *= f;
+    dev::fwht<32, 4>(a, lane);
+    float o4[4];
+#pragma unroll
+    for (int i = 0; i < 4; ++i) o4[i] = p.vsign[lane * 4 + i] < 0 ? -a[i] : a[i];
+    *reinterpret_cast<float4 *>(out) = make_float4(o4[0], o4[1], o4[2], o4[3]);
+  }
+}
+
+// Largest CTA index c with cuts[c] <= x: the CTA whose range holds x (CTAs
+// with empty ranges share their start with the next non-empty one, so the
+// largest index is the non-empty one).
+__device__ __forceinline__ int cta_of(const int64_t *cuts, int C, int64_t x) {
+  int lo = 0, hi = C - 1;
+  while (lo < hi) {
+    const int mid = (lo + hi + 1) >> 1;
+    if (cuts[mid] <= x) lo = mid; else hi = mid - 1;
+  }
+  return lo;
+}
+
 template <int KBM, bool KPROD, int VBM, bool PACK>
-__global__ void __launch_bounds__(8 * 32, 1) decode_split_kernel(SplitParams p) {
-  constexpr int kWarps = 8;
+__global__ void __launch_bounds__((PACK && !KPROD ? 12 : 8) * 32, 1) decode_split_kernel(SplitParams p) {
+  constexpr int kWarps = PACK && !KPROD ? 12 : 8;
   constexpr int kThreads = kWarps * 32;
   constexpr int KW = KBM > 0 ? KBM : 1;
   constexpr int VW = VChunk<VBM>::NW;
-  using CR = ChunkRegs<KBM, KPROD, VBM>;
   extern __shared__ float4 smem4[];
   char *smem = reinterpret_cast<char *>(smem4);
   float *s_q = reinterpret_cast<float *>(smem + kLutBytes);  // [8][kD] q'
   float *s_qs = s_q + 8 * kD;                                // [8][kD] S q'
   float *s_part = s_qs + 8 * kD;                             // [kWarps][8][kPW]
+  __shared__ int s_last;
+  __shared__ int64_t s_cut[kMaxCtas + 1];
 
   const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
   const int g8 = lane >> 2, tig = lane & 3;
@@ -465,6 +641,7 @@ __global__ void __launch_bounds__(8 * 32, 1) decode_split_kernel(SplitParams p) 
   const int64_t T = flat_total(p.seq_lens, p.seq_len, p.B, UH);
   const int64_t x0 = cut(T, p.ctas, blockIdx.x), x1 = cut(T, p.ctas, blockIdx.x + 1);
   if (x0 >= x1) return;
+  for (int c = tid; c <= p.ctas; c += kThreads) s_cut[c] = cut(T, p.ctas, c);
 
   // ---- once per CTA: replicate the two pair tables per lane
   {
@@ -478,10 +655,30 @@ __global__ void __launch_bounds__(8 * 32, 1) decode_split_kernel(SplitParams p) 
     }
   }
   const float inv_sK = __ldg(p.ws + 0);
-  const float inv_sV = __ldg(p.ws + 1);
   const float sK = 1.0f / inv_sK;
+  const float inv_sV = __ldg(p.ws + 1);
   const uint32_t koff = lane * 4;
   const uint32_t voff = 128 + lane * 4;
+  const bool want_scores = p.scores != nullptr;
+
+  // this lane's token rows inside a chunk, in records
+  RowOffs ro;
+#pragma unroll
+  for (int ms = 0; ms < 2; ++ms) {
+#pragma unroll
+    for (int r = 0; r < 2; ++r) {
+      const int t = 16 * ms + 8 * r + g8;
+      ro.rk[ms][r] = t;
+      ro.k[ms][r] = (int32_t)(t * p.ksn);
+      ro.kv[ms][r] = (int32_t)(t * p.vsn);
+    }
+#pragma unroll
+    for (int q4 = 0; q4 < 4; ++q4) {
+      const int t = 16 * ms + 2 * tig + (q4 & 1) + 8 * (q4 >> 1);
+      ro.rv[ms][q4] = t;
+      ro.v[ms][q4] = (int32_t)(t * p.vsn);
+    }
+  }
 
   for (int64_t x = x0; x < x1;) {
     int u;
@@ -497,7 +694,6 @@ __global__ void __launch_bounds__(8 * 32, 1) decode_split_kernel(SplitParams p) 
     const int gh = min(8, p.g - grp * 8);
 
     __syncthreads();  // tables ready / previous piece's shared data consumed
-    // ---- this group's rotated queries (zeros for padding heads)
     for (int o = tid; o < 8 * kD; o += kThreads) {
       const int hh = o / kD, k = o % kD;
       const bool ok = hh < gh;
@@ -518,16 +714,14 @@ __global__ void __launch_bounds__(8 * 32, 1) decode_split_kernel(SplitParams p) 
       const float *qv = s_q + hsrc * kD + 32 * tig;
 #pragma unroll
       for (int s = 0; s < 8; ++s) {
-        if (PACK) {
+        if constexpr (PACK) {
           qf[s][0] = lo_col ? pack_lo(qv[4 * s], qv[4 * s + 1]) : pack_hi(qv[4 * s], qv[4 * s + 1]);
           qf[s][1] = lo_col ? pack_lo(qv[4 * s + 2], qv[4 * s + 3]) : pack_hi(qv[4 * s + 2], qv[4 * s + 3]);
         } else {
           qf[s][0] = pack_hi(qv[4 * s], qv[4 * s + 1]);
           qf[s][1] = pack_hi(qv[4 * s + 2], qv[4 * s + 3]);
-          if constexpr (!PACK) {
-            qf2[s][0] = pack_lo(qv[4 * s], qv[4 * s + 1]);
-            qf2[s][1] = pack_lo(qv[4 * s + 2], qv[4 * s + 3]);
-          }
+          qf2[s][0] = pack_lo(qv[4 * s], qv[4 * s + 1]);
+          qf2[s][1] = pack_lo(qv[4 * s + 2], qv[4 * s + 3]);
         }
       }
       if constexpr (KPROD) {
@@ -535,20 +729,19 @@ __global__ void __launch_bounds__(8 * 32, 1) decode_split_kernel(SplitParams p) 
 #pragma unroll
         for (int s = 0; s < 8; ++s) {
           const float a0 = sv[15 - 2 * s], a1 = sv[31 - 2 * s], a2 = sv[14 - 2 * s], a3 = sv[30 - 2 * s];
-          if (PACK) {
+          if constexpr (PACK) {
             qsf[s][0] = lo_col ? pack_lo(a0, a1) : pack_hi(a0, a1);
             qsf[s][1] = lo_col ? pack_lo(a2, a3) : pack_hi(a2, a3);
           } else {
             qsf[s][0] = pack_hi(a0, a1);
             qsf[s][1] = pack_hi(a2, a3);
-            if constexpr (!PACK) {
-              qsf2[s][0] = pack_lo(a0, a1);
-              qsf2[s][1] = pack_lo(a2, a3);
-            }
+            qsf2[s][0] = pack_lo(a0, a1);
+            qsf2[s][1] = pack_lo(a2, a3);
           }
         }
       }
     }
+
     float acc[8][4];
 #pragma unroll
     for (int i = 0; i < 8; ++i) acc[i][0] = acc[i][1] = acc[i][2] = acc[i][3] = 0.f;
@@ -562,26 +755,49 @@ __global__ void __launch_bounds__(8 * 32, 1) decode_split_kernel(SplitParams p) 
     const int64_t c_begin = min(nchunks, (int64_t)warp * per_warp);
     const int64_t c_end = min(nchunks, c_begin + per_warp);
 
-    CR nxt;
-    if (c_begin < c_end) load_chunk(nxt, p, t0 + c_begin * kChunk, t0, t1, kbase, vbase, g8, tig);
+    KBuf<KBM, KPROD> kb;
+    VBuf<VBM> vb;
+    const bool unit = p.ksn == 1 && p.vsn == 1;
+    // warm L2 one chunk beyond the register prefetch
+    if (unit && lane == 0 && c_begin + 1 < c_end) {
+      const int64_t jp = t0 + (c_begin + 1) * kChunk;
+      prefetch_chunk<KBM, KPROD, VBM>(p, kbase + jp, vbase + jp, min((int64_t)kChunk, t1 - jp));
+    }
+    if (c_begin < c_end) {
+      const int64_t j0 = t0 + c_begin * kChunk;
+      const int nv = (int)min((int64_t)kChunk, t1 - j0);
+      if (unit && nv == kChunk) {
+        load_k<true>(kb, p, kbase + j0, vbase + j0, nv, ro, tig, g8);
+        load_v<true>(vb, p, vbase + j0, nv, ro, g8, tig);
+      } else {
+        load_k<false>(kb, p, kbase + j0 * p.ksn, vbase + j0 * p.vsn, nv, ro, tig, g8);
+        load_v<false>(vb, p, vbase + j0 * p.vsn, nv, ro, g8, tig);
+      }
+    }
     for (int64_t ci = c_begin; ci < c_end; ++ci) {
       const int64_t j0 = t0 + ci * kChunk;
-      CR cur = nxt;
-      if (ci + 1 < c_end) load_chunk(nxt, p, j0 + kChunk, t0, t1, kbase, vbase, g8, tig);
+      const int64_t jn = j0 + kChunk;
+      const bool more = ci + 1 < c_end;
+      const int nvn = more ? (int)min((int64_t)kChunk, t1 - jn) : 0;
+      const bool fast_next = unit && nvn == kChunk;
+      if (unit && lane == 0 && ci + 2 < c_end) {
+        const int64_t jp = jn + kChunk;
+        prefetch_chunk<KBM, KPROD, VBM>(p, kbase + jp, vbase + jp, min((int64_t)kChunk, t1 - jp));
+      }
       // -------- scores: rows (ms, r) -> token j0 + 16 ms + 8 r + g8
       float sc[2][4];
       float nvl[2][2];  // log2 n_V of the lane's rows
 #pragma unroll
       for (int ms = 0; ms < 2; ++ms) {
-        const auto &kw = cur.kw[ms];
-        const auto &qj = cur.qj[ms];
+        const auto &kw = kb.w[ms];
+        const auto &qj = kb.qj[ms];
         float kn[2], kr[2];
 #pragma unroll
         for (int r = 0; r < 2; ++r) {
-          const bool ok = cur.kn[ms][r] >= 0.f;
-          kn[r] = ok ? cur.kn[ms][r] * inv_sK : -1.f;
-          kr[r] = KPROD ? cur.kr[ms][r] * (kKappa * sK) : 0.f;  // the table holds s_K c
-          nvl[ms][r] = ok ? __log2f(cur.vn[ms][r]) : -INFINITY;
+          const bool ok = kb.kn[ms][r] >= 0.f;
+          kn[r] = ok ? kb.kn[ms][r] * inv_sK : -1.f;
+          kr[r] = KPROD ? kb.kr[ms][r] * (kKappa * sK) : 0.f;  // the table holds s_K c
+          nvl[ms][r] = ok ? __log2f(kb.vn[ms][r]) : -INFINITY;
         }
         float cm[4] = {0.f, 0.f, 0.f, 0.f};
         if constexpr (KBM > 0) {
@@ -615,7 +831,7 @@ __global__ void __launch_bounds__(8 * 32, 1) decode_split_kernel(SplitParams p) 
           TQ_QSTEP(4) TQ_QSTEP(5) TQ_QSTEP(6) TQ_QSTEP(7)
 #undef TQ_QSTEP
         }
-        // s = n/s_K * (main + kappa gamma s_K qjl): the LUT holds s_K c
+        // s = n/s_K * (main + kappa gamma s_K qjl): the table holds s_K c
 #pragma unroll
         for (int i = 0; i < 4; ++i) {
           float s = cm[i];
@@ -628,18 +844,34 @@ __global__ void __launch_bounds__(8 * 32, 1) decode_split_kernel(SplitParams p) 
 #pragma unroll
           for (int c = 0; c < 2; ++c) {
             const float s = cm[2 * r + c] * kn[r];
-            const int head = PACK ? 2 * (tig & 1) + c : 2 * tig + c;
-            if (p.scores && kn[r] >= 0.f && head < gh && (!PACK || tig < 2)) {
-              const int64_t j = j0 + 16 * ms + 8 * r + g8;
-              p.scores[((int64_t)b * p.Hq + h0 + head) * p.seq_len + j] = s;
-            }
+            cm[2 * r + c] = s;
             sc[ms][2 * r + c] = kn[r] >= 0.f ? s * p.scale_log2 : -INFINITY;
           }
         }
+        if (want_scores) {
+#pragma unroll
+          for (int r = 0; r < 2; ++r) {
+#pragma unroll
+            for (int c = 0; c < 2; ++c) {
+              const int head = PACK ? 2 * (tig & 1) + c : 2 * tig + c;
+              if (kn[r] >= 0.f && head < gh && (!PACK || tig < 2)) {
+                const int64_t j = j0 + 16 * ms + 8 * r + g8;
+                p.scores[((int64_t)b * p.Hq + h0 + head) * p.seq_len + j] = cm[2 * r + c];
+              }
+            }
+          }
+        }
+      }
+      // the key registers are free: start the next chunk's key loads
+      if (more) {
+        if (fast_next) load_k<true>(kb, p, kbase + jn, vbase + jn, nvn, ro, tig, g8);
+        else load_k<false>(kb, p, kbase + jn * p.ksn, vbase + jn * p.vsn, nvn, ro, tig, g8);
       }
 
       // -------- online softmax, per head column c
       float wgt[2][4];
+      float aM[2];
+      bool moved = false;
 #pragma unroll
       for (int c = 0; c < 2; ++c) {
         float mx = fmaxf(fmaxf(sc[0][c], sc[0][2 + c]), fmaxf(sc[1][c], sc[1][2 + c]));
@@ -653,7 +885,9 @@ __global__ void __launch_bounds__(8 * 32, 1) decode_split_kernel(SplitParams p) 
         const float mn = fmaxf(m_run[c], mx), Mn = fmaxf(M_run[c], Mx);
         const float ms_ = mn == -INFINITY ? 0.f : mn;
         const float Ms_ = Mn == -INFINITY ? 0.f : Mn;
-        const float al = exp2f(m_run[c] - ms_), aM = exp2f(M_run[c] - Ms_);
+        const float al = ex2(m_run[c] - ms_);
+        aM[c] = ex2(M_run[c] - Ms_);
+        moved |= Mn != M_run[c];
         m_run[c] = mn;
         M_run[c] = Mn;
         float ls = 0.f;
@@ -662,15 +896,19 @@ __global__ void __launch_bounds__(8 * 32, 1) decode_split_kernel(SplitParams p) 
 #pragma unroll
           for (int r = 0; r < 2; ++r) {
             const float t = sc[ms][2 * r + c];
-            ls += exp2f(t - ms_);
-            wgt[ms][2 * r + c] = exp2f(t + nvl[ms][r] - Ms_);
+            ls += ex2(t - ms_);
+            wgt[ms][2 * r + c] = ex2(t + nvl[ms][r] - Ms_);
           }
         }
         l_run[c] = fmaf(l_run[c], al, ls);
+      }
+      if (__any_sync(dev::kFull, moved)) {
 #pragma unroll
         for (int mt = 0; mt < 8; ++mt) {
-          acc[mt][c] *= aM;
-          acc[mt][2 + c] *= aM;
+          acc[mt][0] *= aM[0];
+          acc[mt][1] *= aM[1];
+          acc[mt][2] *= aM[0];
+          acc[mt][3] *= aM[1];
         }
       }
 
@@ -689,8 +927,7 @@ __global__ void __launch_bounds__(8 * 32, 1) decode_split_kernel(SplitParams p) 
           b2 = movmatrix_trans(pack_lo(wgt[ms][0], wgt[ms][1]));
           b3 = movmatrix_trans(pack_lo(wgt[ms][2], wgt[ms][3]));
         }
-        // this lane's 4 tokens: 2 tig, 2 tig + 1, 2 tig + 8, 2 tig + 9 (of 16)
-        const auto &vw = cur.vw[ms];
+        const auto &vw = vb.w[ms];
         if constexpr (VBM == 4) {
           // cross-nibble bytes: (token a, dim) | (token b, dim) << 4
           uint32_t x0[2][2], x1[2][2];
@@ -706,7 +943,7 @@ __global__ void __launch_bounds__(8 * 32, 1) decode_split_kernel(SplitParams p) 
 #define TQ_VSTEP4(MT)                                                             \
   {                                                                               \
     uint32_t a[4];                                                                \
-    a[0] = lut(smem, pair_addr<4, MT, 2>(x0[0], voff));                       \
+    a[0] = lut(smem, pair_addr<4, MT, 2>(x0[0], voff));                           \
     a[1] = lut(smem, pair_addr<4, MT, 2>(x1[0], voff));                           \
     a[2] = lut(smem, pair_addr<4, MT, 2>(x0[1], voff));                           \
     a[3] = lut(smem, pair_addr<4, MT, 2>(x1[1], voff));                           \
@@ -736,6 +973,11 @@ __global__ void __launch_bounds__(8 * 32, 1) decode_split_kernel(SplitParams p) 
 #undef TQ_VSTEP
         }
       }
+      // the value registers are free: start the next chunk's value loads
+      if (more) {
+        if (fast_next) load_v<true>(vb, p, vbase + jn, nvn, ro, g8, tig);
+        else load_v<false>(vb, p, vbase + jn * p.vsn, nvn, ro, g8, tig);
+      }
     }
 
     // ---- warp totals: l over the 8 row groups; PACK: hi + lo columns of acc
@@ -755,11 +997,10 @@ __global__ void __launch_bounds__(8 * 32, 1) decode_split_kernel(SplitParams p) 
     // ---- CTA merge of the warps' partials for this piece
     {
       float *wp = s_part + (size_t)warp * 8 * kPW;
-      const bool writer = PACK ? tig < 2 : true;
-      if (writer) {
+      if (PACK ? tig < 2 : true) {
 #pragma unroll
         for (int c = 0; c < 2; ++c) {
-          const int hh = PACK ? 2 * tig + c : 2 * tig + c;
+          const int hh = 2 * tig + c;
           if (g8 == 0) {
             wp[hh * kPW + 0] = m_run[c];
             wp[hh * kPW + 1] = l_run[c];
@@ -796,96 +1037,41 @@ __global__ void __launch_bounds__(8 * 32, 1) decode_split_kernel(SplitParams p) 
 #pragma unroll
           for (int w = 0; w < kWarps; ++w) {
             const float *q = s_part + (w * 8 + hh) * kPW;
-            v += q[1] * exp2f(q[0] - m0);
+            v += q[1] * ex2(q[0] - m0);
           }
         } else {
           const int dd = e - 3;
 #pragma unroll
           for (int w = 0; w < kWarps; ++w) {
             const float *q = s_part + (w * 8 + hh) * kPW;
-            v += q[4 + dd] * exp2f(q[2] - M0);
+            v += q[4 + dd] * ex2(q[2] - M0);
           }
           v *= inv_sV;
         }
         dst[hh * kPW + (e < 3 ? e : e + 1)] = v;
       }
     }
-  }
-}
-
-// ----------------------------------------------------------- combine
-
-// One warp per (batch, query head): merge the slots of its unit, o' / l,
-// then o = sigma_V * H o' / sqrt(d).
-__global__ void __launch_bounds__(32) decode_combine_kernel(CombineParams p) {
-  const int lane = threadIdx.x;
-  const int bh = blockIdx.x;
-  const int b = bh / p.Hq, hq = bh % p.Hq;
-  const int kvh = hq / p.g, grp = (hq % p.g) / 8, hh = (hq % p.g) % 8;
-  const int UH = p.Hkv * p.groups;
-  const int u = b * UH + kvh * p.groups + grp;
-  float *out = p.out + (int64_t)bh * kD + lane * 4;
-  const int64_t T = flat_total(p.seq_lens, p.seq_len, p.B, UH);
-  int64_t ustart, ulen;
-  if (p.seq_lens) {
-    ustart = 0;
-    for (int bb = 0; bb < b; ++bb) ustart += batch_len(p.seq_lens, p.seq_len, bb) * UH;
-    ulen = batch_len(p.seq_lens, p.seq_len, b);
-    ustart += (int64_t)(kvh * p.groups + grp) * ulen;
-  } else {
-    ustart = (int64_t)u * p.seq_len;
-    ulen = p.seq_len;
-  }
-  float mstar = -INFINITY, Mstar = -INFINITY;
-  int c0 = 0, c1 = -1;
-  if (ulen > 0 && T > 0) {
-    // first CTA whose range [cut(c), cut(c+1)) contains ustart
-    c0 = (int)(((uint64_t)ustart * (uint64_t)p.ctas) / (uint64_t)T);
-    while (c0 > 0 && cut(T, p.ctas, c0) > ustart) --c0;
-    while (c0 + 1 < p.ctas && cut(T, p.ctas, c0 + 1) <= ustart) ++c0;
-    const int64_t uend = ustart + ulen;
-    int64_t lo = cut(T, p.ctas, c0);
-    for (int c = c0; c < p.ctas && lo < uend; ++c) {
-      const int64_t hi = cut(T, p.ctas, c + 1);
-      if (hi > lo) {
-        const float *q = p.ws + p.slot0 + ((int64_t)u + c) * kSlot + hh * kPW;
-        mstar = fmaxf(mstar, q[0]);
-        Mstar = fmaxf(Mstar, q[2]);
-        c1 = c;
-      }
-      lo = hi;
+    // ---- the last CTA to finish a unit merges its slots into the output.
+    // Classic fence-then-count: every CTA publishes its slot, fences, and
+    // bumps the unit's counter once; no CTA ever waits on another.
+    __threadfence();
+    __syncthreads();
+    if (tid == 0) {
+      const int c0 = cta_of(s_cut, p.ctas, ustart), c1 = cta_of(s_cut, p.ctas, ustart + ulen - 1);
+      // CTAs with an empty range (only when the space is shorter than the
+      // grid) never arrive, so count the non-empty ones of the span
+      unsigned n = 0;
+      for (int c = c0; c <= c1; ++c) n += s_cut[c + 1] > s_cut[c] ? 1u : 0u;
+      const unsigned prev = atomicAdd(p.cnt + u, 1u);
+      s_last = (prev + 1 == n) ? 1 : 0;
+    }
+    __syncthreads();
+    if (s_last) {
+      __threadfence();
+      const int c0 = cta_of(s_cut, p.ctas, ustart), c1 = cta_of(s_cut, p.ctas, ustart + ulen - 1);
+      merge_unit(p, s_cut, u, c0, c1, b, h0, gh, warp, kWarps, lane, s_part);
     }
   }
-  if (mstar == -INFINITY) {
-    *reinterpret_cast<float4 *>(out) = make_float4(0.f, 0.f, 0.f, 0.f);
-    return;
-  }
-  const float M0 = Mstar == -INFINITY ? 0.f : Mstar;
-  float l = 0.f;
-  float a[4] = {0.f, 0.f, 0.f, 0.f};
-  int64_t lo = cut(T, p.ctas, c0);
-  for (int c = c0; c <= c1; ++c) {
-    const int64_t hi = cut(T, p.ctas, c + 1);
-    if (hi > lo) {
-      const float *q = p.ws + p.slot0 + ((int64_t)u + c) * kSlot + hh * kPW;
-      l += q[1] * exp2f(q[0] - mstar);
-      const float wM = exp2f(q[2] - M0);
-      const float4 v = *reinterpret_cast<const float4 *>(q + 4 + lane * 4);
-      a[0] = fmaf(v.x, wM, a[0]);
-      a[1] = fmaf(v.y, wM, a[1]);
-      a[2] = fmaf(v.z, wM, a[2]);
-      a[3] = fmaf(v.w, wM, a[3]);
-    }
-    lo = hi;
-  }
-  const float f = exp2f(M0 - mstar) / l * 0.08838834764831845f;
-#pragma unroll
-  for (int i = 0; i < 4; ++i) a[i] *= f;
-  dev::fwht<32, 4>(a, lane);
-  float o[4];
-#pragma unroll
-  for (int i = 0; i < 4; ++i) o[i] = p.vsign[lane * 4 + i] < 0 ? -a[i] : a[i];
-  *reinterpret_cast<float4 *>(out) = make_float4(o[0], o[1], o[2], o[3]);
 }
 
 __global__ void zero_out_kernel(float *out, int64_t n) {
@@ -900,7 +1086,7 @@ constexpr size_t split_smem_bytes(int warps) {
 template <int KBM, bool KPROD, int VBM, bool PACK>
 cudaError_t run_split(const SplitParams &sp, cudaStream_t s) {
   auto kern = decode_split_kernel<KBM, KPROD, VBM, PACK>;
-  const int warps = 8;
+  const int warps = PACK && !KPROD ? 12 : 8;
   const size_t smem = split_smem_bytes(warps);
   cudaError_t e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
   if (e != cudaSuccess) return e;
@@ -934,7 +1120,7 @@ bool decode_supported(int d, int kbm, bool kprod, int vbm, bool vprod) {
 
 size_t decode_workspace_floats(int B, int Hq, int Hkv, bool prod, int ctas) {
   const int64_t units = (int64_t)B * Hkv * ((Hq / Hkv + 7) / 8);
-  return (size_t)kHdr + (size_t)B * Hq * kD * (prod ? 2 : 1) + (size_t)(units + ctas) * kSlot;
+  return (size_t)kHdr + (size_t)B * Hq * kD * (prod ? 2 : 1) + (size_t)(units + ctas) * kSlot + (size_t)units;
 }
 
 cudaError_t launch_decode(const DecodeArgs &a, cudaStream_t s) {
@@ -974,8 +1160,13 @@ cudaError_t launch_decode(const DecodeArgs &a, cudaStream_t s) {
   sp.scores = a.scores;
   sp.ws = a.ws;
   sp.slot0 = (int64_t)kHdr + (int64_t)a.B * a.Hq * kD * (a.kq.prod ? 2 : 1);
+  const int units = a.B * a.Hkv * sp.groups;
+  sp.cnt = reinterpret_cast<unsigned *>(a.ws + sp.slot0 + (int64_t)(units + sp.ctas) * kSlot);
+  sp.out = a.out;
+  sp.vsign = a.vq.signs;
   PrepParams pp{a.q, a.q_dtype, a.B * a.Hq, a.kq.signs, a.kq.prod ? a.kq.S : nullptr,
-                a.kq.centroids, a.kq.bm, a.vq.centroids, a.vq.bm, a.ws};
+                a.kq.centroids, a.kq.bm, a.vq.centroids, a.vq.bm, a.ws, sp.cnt, units,
+                a.Hq, a.seq_len, a.seq_lens, a.out};
   decode_prep_kernel<<<(a.B * a.Hq + 1) / 2 + 2, 256, 0, s>>>(pp);
   cudaError_t pe = cudaGetLastError();
   if (pe != cudaSuccess) return pe;
@@ -988,9 +1179,6 @@ cudaError_t launch_decode(const DecodeArgs &a, cudaStream_t s) {
     case 4: e = by_kvariant<4>(a.kq.bm, a.kq.prod, pack, sp, s); break;
   }
   if (e != cudaSuccess) return e;
-  CombineParams cp{a.B, a.Hq, a.Hkv, sp.g, sp.groups, a.seq_len, a.seq_lens, sp.ctas, sp.slot0, a.ws,
-                   a.vq.signs, a.out};
-  decode_combine_kernel<<<a.B * a.Hq, 32, 0, s>>>(cp);
   return cudaGetLastError();
 }
 

@@ -7,9 +7,11 @@
 // coordinate to its Lloyd-Max index, bit-pack; for prod, take the residual,
 // its norm, and the signs of S r.
 //
-// Work layout: T = d/64 lanes per vector (one lane for d = 64), each lane
-// owning 64 contiguous coordinates in registers; the butterfly stages with
-// stride >= 64 and the first folds of the norm go through warp shuffles.
+// Work layout: T = d/E lanes per vector, each lane owning E contiguous
+// coordinates in registers (E = 64 for large batches; E = 16 for small ones,
+// such as appending one token, where short per-lane chains matter more than
+// shuffle count); the butterfly stages with stride >= E and the first folds
+// of the norm go through warp shuffles.
 // Memory traffic per vector is the input read once and the packed record
 // written once; nothing else touches HBM.
 
@@ -38,9 +40,9 @@ struct EncParams {
   float sqrt_d;
 };
 
-template <int D>
+template <int D, int EE = 64>
 struct Shape {
-  static constexpr int T = D <= 64 ? 1 : D / 64;  // lanes per vector
+  static constexpr int T = D <= EE ? 1 : D / EE;  // lanes per vector
   static constexpr int E = D / T;                 // coordinates per lane
   static constexpr int VPB = kEncThreads / T;     // vectors per block
   static constexpr int RS = D + 4;                // padded smem row (floats)
@@ -48,20 +50,42 @@ struct Shape {
   static constexpr bool kSmemS = (size_t)D * RS * 4 + (size_t)VPB * RS * 4 <= 200 * 1024;
 };
 
-template <int D, bool PROD>
+template <int D, bool PROD, int EE>
 constexpr size_t enc_smem_bytes() {
-  using Sh = Shape<D>;
+  using Sh = Shape<D, EE>;
   if constexpr (!PROD) return 0;
   return (size_t)Sh::VPB * Sh::RS * 4 + (Sh::kSmemS ? (size_t)D * Sh::RS * 4 : 0);
 }
 
-template <int D, int BM, bool PROD, int DT>
+// Stores the low NB bytes of W (little-endian) to dst, which is aligned to
+// the largest power of two dividing NB (at most 16).
+template <int NB, int NW>
+__device__ __forceinline__ void store_bytes(uint8_t *dst, const uint32_t (&W)[NW]) {
+  if constexpr (NB % 16 == 0) {
+#pragma unroll
+    for (int i = 0; i < NB / 16; ++i)
+      reinterpret_cast<uint4 *>(dst)[i] = make_uint4(W[4 * i], W[4 * i + 1], W[4 * i + 2], W[4 * i + 3]);
+  } else if constexpr (NB % 8 == 0) {
+#pragma unroll
+    for (int i = 0; i < NB / 8; ++i) reinterpret_cast<uint2 *>(dst)[i] = make_uint2(W[2 * i], W[2 * i + 1]);
+  } else if constexpr (NB % 4 == 0) {
+#pragma unroll
+    for (int i = 0; i < NB / 4; ++i) reinterpret_cast<uint32_t *>(dst)[i] = W[i];
+  } else {
+    static_assert(NB % 2 == 0, "odd byte count");
+#pragma unroll
+    for (int i = 0; i < NB / 2; ++i)
+      reinterpret_cast<unsigned short *>(dst)[i] = (unsigned short)(W[i >> 1] >> (16 * (i & 1)));
+  }
+}
+
+template <int D, int BM, bool PROD, int DT, int EE>
 __global__ void __launch_bounds__(kEncThreads) encode_kernel(EncParams p) {
-  using Sh = Shape<D>;
+  using Sh = Shape<D, EE>;
   constexpr int T = Sh::T, E = Sh::E, VPB = Sh::VPB, RS = Sh::RS;
   constexpr int K = 1 << BM;
-  constexpr int NWC = BM > 0 ? E * BM / 32 : 1;  // code words per lane
-  constexpr int NWQ = E / 32;                    // qjl words per lane
+  constexpr int NWC = BM > 0 ? (E * BM + 31) / 32 : 1;  // code words per lane
+  constexpr int NWQ = (E + 31) / 32;                    // qjl words per lane
 
   __shared__ uint32_t s_sign[D / 32];
   __shared__ float s_cent[16];
@@ -71,10 +95,12 @@ __global__ void __launch_bounds__(kEncThreads) encode_kernel(EncParams p) {
   float *s_S = s_dyn + (size_t)VPB * RS;  // [D][RS] projection (prod, if it fits)
 
   const int tid = threadIdx.x;
-  for (int w = tid; w < D / 32; w += blockDim.x) {
-    uint32_t m = 0;
-    for (int j = 0; j < 32; ++j) m |= (p.signs[32 * w + j] < 0 ? 1u : 0u) << j;
-    s_sign[w] = m;
+  if (tid < 32) {  // sign bit masks, one ballot per 32 coordinates
+#pragma unroll
+    for (int w = 0; w < D / 32; ++w) {
+      const unsigned m = __ballot_sync(dev::kFull, p.signs[32 * w + tid] < 0);
+      if (tid == 0) s_sign[w] = m;
+    }
   }
   if constexpr (PROD && BM > 0) {
     if (tid < K) s_cent[tid] = p.cent[tid];
@@ -110,9 +136,9 @@ __global__ void __launch_bounds__(kEncThreads) encode_kernel(EncParams p) {
   const float nrm = __fsqrt_rn(dev::fold_halves_sum<T, E>(sq));
 
   // rotate: sign flips, then the unnormalised FWHT
-  uint32_t sw[E / 32];
+  uint32_t sw[(E + 31) / 32];
 #pragma unroll
-  for (int w = 0; w < E / 32; ++w) sw[w] = s_sign[t * (E / 32) + w];
+  for (int w = 0; w < (E + 31) / 32; ++w) sw[w] = s_sign[(t * E) / 32 + w] >> ((t * E) & 31);
 #pragma unroll
   for (int i = 0; i < E; ++i)
     a[i] = __uint_as_float(__float_as_uint(a[i]) ^ (((sw[i >> 5] >> (i & 31)) & 1u) << 31));
@@ -140,7 +166,7 @@ __global__ void __launch_bounds__(kEncThreads) encode_kernel(EncParams p) {
       dev::put_field<BM>(W, i, (uint32_t)idx);
       if constexpr (PROD) a[i] = __fsub_rn(a[i], s_cent[idx]);
     }
-    if (active) dev::store_words<NWC>(p.codes + rec * (D * BM / 8) + t * (E * BM / 8), W);
+    if (active) store_bytes<E * BM / 8>(p.codes + rec * (D * BM / 8) + t * (E * BM / 8), W);
   }
   if (active && t == 0) p.norms[rec] = nrm;
 
@@ -155,11 +181,11 @@ __global__ void __launch_bounds__(kEncThreads) encode_kernel(EncParams p) {
     for (int i = 0; i < E; ++i) rv[t * E + i] = a[i];
     __syncwarp();
     uint32_t Q[NWQ];
-    const int rot = t * (32 / T);  // rotates the column order per lane: no bank clash
+    const int rot = (t * 32 / T) & 31;  // rotates the column order per lane: no bank clash
 #pragma unroll
     for (int w = 0; w < NWQ; ++w) {
       uint32_t qw = 0u;
-      for (int kb = 0; kb < 32; ++kb) {
+      for (int kb = 0; kb < (E < 32 ? E : 32); ++kb) {
         const int k = t * E + w * 32 + kb;
         float acc = 0.0f;
         if constexpr (Sh::kSmemS) {
@@ -182,15 +208,15 @@ __global__ void __launch_bounds__(kEncThreads) encode_kernel(EncParams p) {
       Q[w] = qw;
     }
     if (active) {
-      dev::store_words<NWQ>(p.qjl + rec * (D / 8) + t * (E / 8), Q);
+      store_bytes<E / 8>(p.qjl + rec * (D / 8) + t * (E / 8), Q);
       if (t == 0) p.rnorms[rec] = gam;
     }
   }
 }
 
-template <int D, int BM, bool PROD, int DT>
-cudaError_t run(const EncodeArgs &a, cudaStream_t s) {
-  using Sh = Shape<D>;
+template <int D, int BM, bool PROD, int DT, int EE>
+cudaError_t run_e(const EncodeArgs &a, cudaStream_t s) {
+  using Sh = Shape<D, EE>;
   EncParams p;
   p.x = a.x;
   p.xsb = a.xsb;
@@ -211,8 +237,8 @@ cudaError_t run(const EncodeArgs &a, cudaStream_t s) {
   p.signs = a.q.signs;
   p.S = a.q.S;
   p.sqrt_d = a.q.sqrt_d;
-  const size_t smem = enc_smem_bytes<D, PROD>();
-  auto kern = encode_kernel<D, BM, PROD, DT>;
+  const size_t smem = enc_smem_bytes<D, PROD, EE>();
+  auto kern = encode_kernel<D, BM, PROD, DT, EE>;
   if (smem > 48 * 1024) {
     cudaError_t e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
     if (e != cudaSuccess) return e;
@@ -220,6 +246,15 @@ cudaError_t run(const EncodeArgs &a, cudaStream_t s) {
   const int64_t blocks = (p.nvec + Sh::VPB - 1) / Sh::VPB;
   kern<<<(unsigned)blocks, kEncThreads, smem, s>>>(p);
   return cudaGetLastError();
+}
+
+// Small batches (up to one vector per lane of a full wave at E = 64) take
+// the E = 16 layout: four times more lanes per vector, shorter chains.
+template <int D, int BM, bool PROD, int DT>
+cudaError_t run(const EncodeArgs &a, cudaStream_t s) {
+  const int64_t nvec = a.B * a.H * a.N;
+  if (nvec <= 148 * (kEncThreads / Shape<D, 64>::T)) return run_e<D, BM, PROD, DT, 16>(a, s);
+  return run_e<D, BM, PROD, DT, 64>(a, s);
 }
 
 template <int D, int BM, bool PROD>

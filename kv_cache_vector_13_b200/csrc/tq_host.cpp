@@ -246,7 +246,7 @@ int num_sms() {
 namespace tq {
 
 // One persistent CTA per SM of the current device.
-int decode_ctas() { return num_sms(); }
+int decode_ctas() { return std::min(num_sms(), 1024); }
 
 }  // namespace tq
 
