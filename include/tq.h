@@ -24,9 +24,11 @@
  *   - Every call returns tq_status.  Arguments are validated before any
  *     launch; a failed check returns a non-OK status, launches nothing and
  *     sets tq_last_error().  A failed launch returns TQ_ECUDA.
- *   - The library allocates no device memory and keeps no global state.
- *     The caller owns every buffer and the stream; device calls are
- *     asynchronous on the given stream (NULL = the legacy default stream).
+ *   - The library allocates no device memory and keeps no global state
+ *     (tq_decode_attention_noalloc alone uses a fixed scratch array compiled
+ *     into the library).  The caller owns every buffer and the stream;
+ *     device calls are asynchronous on the given stream (NULL = the legacy
+ *     default stream).
  *   - Outputs must not alias inputs.
  *   - d is 64, 128 or 256.  bits is the total b per coordinate, 1..4.
  *     The MSE part uses b_m = b bits (mse) or b_m = b - 1 bits (prod).
@@ -171,6 +173,35 @@ tq_status tq_decode_attention(const tq_quantizer *kq, const tq_quantizer *vq,
                               const tq_cache_view *v, float softmax_scale,
                               float *out, float *scores_out, void *workspace,
                               size_t workspace_bytes, tq_stream_t stream);
+
+/* Decode attention without a caller workspace.  The pages have no
+ * counterpart to this call: it exists for callers that cannot allocate
+ * device memory at run time, such as a plugin whose enqueue runs inside
+ * another engine that owns every device allocation, or a service that
+ * forbids cudaMalloc after start-up.  Same arguments, meaning and results
+ * as tq_decode_attention, minus the workspace: the scratch it needs lives in
+ * a fixed array of TQ_NOALLOC_SCRATCH_BYTES compiled into the library, one
+ * copy per GPU that loads the library, kept until the process exits.
+ *   - The first call on a device looks up that device's copy of the array
+ *     (cudaGetSymbolAddress, with the device current); make that first call
+ *     before any stream capture.
+ *   - It allocates nothing: no cudaMalloc, no cudaFree, no allocating
+ *     library call.
+ *   - A problem whose tq_decode_workspace_bytes exceeds
+ *     TQ_NOALLOC_SCRATCH_BYTES returns TQ_EWORKSPACE, with the sizes in
+ *     tq_last_error().
+ *   - All calls share the one array, and it keeps the previous call's
+ *     contents.  Every call clears the counters it needs at its start.
+ *     Calls whose work overlaps on the GPU (different streams without
+ *     ordering between them) race on the array; keep them ordered. */
+#define TQ_NOALLOC_SCRATCH_BYTES ((size_t)16 << 20)
+tq_status tq_decode_attention_noalloc(const tq_quantizer *kq, const tq_quantizer *vq,
+                                      const void *q, tq_dtype q_dtype, int32_t B,
+                                      int32_t Hq, int32_t Hkv, int64_t seq_len,
+                                      const int32_t *seq_lens,
+                                      const tq_cache_view *k, const tq_cache_view *v,
+                                      float softmax_scale, float *out,
+                                      float *scores_out, tq_stream_t stream);
 
 /* Synchronize `stream` and report any asynchronous CUDA error. */
 tq_status tq_check(tq_stream_t stream);

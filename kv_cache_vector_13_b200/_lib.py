@@ -15,11 +15,13 @@ TQ_MSE, TQ_PROD = 0, 1
 TQ_ROT_HADAMARD, TQ_ROT_DENSE = 0, 1
 TQ_CB_GAUSS, TQ_CB_BETA = 0, 1
 TQ_F32, TQ_BF16, TQ_F16 = 0, 1, 2
+TQ_NOALLOC_SCRATCH_BYTES = 16 << 20  # include/tq.h
 
 # every symbol include/tq.h declares
 EXPORTS = (
     "tq_make_codebook", "tq_make_signs", "tq_make_qjl", "tq_code_bytes", "tq_qjl_bytes",
     "tq_encode", "tq_dequant", "tq_decode_workspace_bytes", "tq_decode_attention",
+    "tq_decode_attention_noalloc",
     "tq_check", "tq_status_string", "tq_last_error", "tq_version",
 )
 
@@ -79,6 +81,11 @@ def lib() -> ctypes.CDLL:
         c_int64, c_void_p, POINTER(TqCacheView), POINTER(TqCacheView), c_float, c_void_p, c_void_p,
         c_void_p, c_size_t, c_void_p]
     L.tq_decode_attention.restype = c_int32
+    L.tq_decode_attention_noalloc.argtypes = [
+        POINTER(TqQuantizer), POINTER(TqQuantizer), c_void_p, c_int32, c_int32, c_int32, c_int32,
+        c_int64, c_void_p, POINTER(TqCacheView), POINTER(TqCacheView), c_float, c_void_p, c_void_p,
+        c_void_p]
+    L.tq_decode_attention_noalloc.restype = c_int32
     L.tq_check.argtypes = [c_void_p]
     L.tq_check.restype = c_int32
     L.tq_status_string.argtypes = [c_int32]

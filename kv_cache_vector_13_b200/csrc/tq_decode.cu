@@ -52,6 +52,14 @@
 
 #include <math.h>
 
+#include <mutex>
+
+// Scratch for tq_decode_attention_noalloc: a fixed array in device memory,
+// one copy per GPU that loads the library, held until the process exits.
+// Host code must not use its name as a device address; the address comes
+// from cudaGetSymbolAddress (static_scratch below).
+static __device__ __align__(256) unsigned char g_tq_noalloc_scratch[TQ_NOALLOC_SCRATCH_BYTES];
+
 namespace tq {
 namespace {
 
@@ -1121,6 +1129,26 @@ bool decode_supported(int d, int kbm, bool kprod, int vbm, bool vprod) {
 size_t decode_workspace_floats(int B, int Hq, int Hkv, bool prod, int ctas) {
   const int64_t units = (int64_t)B * Hkv * ((Hq / Hkv + 7) / 8);
   return (size_t)kHdr + (size_t)B * Hq * kD * (prod ? 2 : 1) + (size_t)(units + ctas) * kSlot + (size_t)units;
+}
+
+cudaError_t static_scratch(void **ptr) {
+  // Looked up once per device, with that device current, and cached.
+  constexpr int kMaxDevices = 64;
+  static std::mutex mu;
+  static void *addr[kMaxDevices] = {};
+  int dev = 0;
+  cudaError_t e = cudaGetDevice(&dev);
+  if (e != cudaSuccess) return e;
+  if (dev < 0 || dev >= kMaxDevices) return cudaErrorInvalidDevice;
+  std::lock_guard<std::mutex> lock(mu);
+  if (!addr[dev]) {
+    void *a = nullptr;
+    e = cudaGetSymbolAddress(&a, g_tq_noalloc_scratch);
+    if (e != cudaSuccess) return e;
+    addr[dev] = a;
+  }
+  *ptr = addr[dev];
+  return cudaSuccess;
 }
 
 cudaError_t launch_decode(const DecodeArgs &a, cudaStream_t s) {

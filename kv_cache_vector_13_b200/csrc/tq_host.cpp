@@ -415,6 +415,25 @@ tq_status tq_decode_attention(const tq_quantizer *kq, const tq_quantizer *vq, co
   return TQ_OK;
 }
 
+tq_status tq_decode_attention_noalloc(const tq_quantizer *kq, const tq_quantizer *vq, const void *q,
+                                      tq_dtype q_dtype, int32_t B, int32_t Hq, int32_t Hkv, int64_t seq_len,
+                                      const int32_t *seq_lens, const tq_cache_view *k, const tq_cache_view *v,
+                                      float softmax_scale, float *out, float *scores_out, tq_stream_t stream) {
+  const size_t need = tq_decode_workspace_bytes(B, Hq, Hkv, seq_len, kq ? kq->d : 0);
+  if (need > (size_t)TQ_NOALLOC_SCRATCH_BYTES)
+    return fail(TQ_EWORKSPACE,
+                "tq_decode_attention_noalloc: B=%d Hq=%d Hkv=%d seq_len=%lld needs %zu bytes of scratch, "
+                "more than the %zu-byte static scratch; use tq_decode_attention with a caller workspace",
+                B, Hq, Hkv, (long long)seq_len, need, (size_t)TQ_NOALLOC_SCRATCH_BYTES);
+  void *ws = nullptr;
+  if (need > 0) {
+    const cudaError_t e = tq::static_scratch(&ws);
+    if (e != cudaSuccess) return cuda_fail(e, "tq_decode_attention_noalloc: scratch lookup");
+  }
+  return tq_decode_attention(kq, vq, q, q_dtype, B, Hq, Hkv, seq_len, seq_lens, k, v, softmax_scale, out,
+                             scores_out, ws, need, stream);
+}
+
 tq_status tq_check(tq_stream_t stream) {
   cudaError_t e = cudaStreamSynchronize((cudaStream_t)stream);
   if (e != cudaSuccess) return cuda_fail(e, "tq_check");

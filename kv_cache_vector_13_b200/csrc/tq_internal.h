@@ -65,6 +65,10 @@ struct DecodeArgs {
 int decode_ctas();
 size_t decode_workspace_floats(int B, int Hq, int Hkv, bool prod, int ctas);
 
+// Device address of the allocation-free decode's fixed scratch array on
+// the current device (looked up once per device with cudaGetSymbolAddress).
+cudaError_t static_scratch(void **ptr);
+
 cudaError_t launch_encode(const EncodeArgs &a, cudaStream_t s);
 cudaError_t launch_dequant(const DequantArgs &a, cudaStream_t s);
 cudaError_t launch_decode(const DecodeArgs &a, cudaStream_t s);
