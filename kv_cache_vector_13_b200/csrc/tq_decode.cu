@@ -549,71 +549,100 @@ __device__ __forceinline__ float ex2(float x) {
 }
 
 // Merge the slots of unit u (heads < gh) and write out[b, h0 + hh, :] =
-// sigma_V * H (o'/l) / sqrt(d).  One warp per head.  The lanes first read
-// every slot's (m, l, M) in parallel and turn them into weights kept in
-// shared memory (zero for CTAs with empty ranges), so the accumulation loop
-// has no data-dependent branch and its loads can all be in flight at once.
+// sigma_V * H (o'/l) / sqrt(d).  The CTA's warps split the work as (head,
+// part): warp (hh, part) merges a contiguous share of the slots, 4 dims per
+// lane, kMergeBatch slots at a time with an online rescale.  Every load of a
+// batch (the slot headers, broadcast to all lanes, and the lane's 4 dims) is
+// issued before any is used, so a batch costs one round trip to L2.  The
+// parts of a head are then combined through shared memory by one warp,
+// which applies the inverse rotation.  CTAs with an empty range never wrote
+// their slot and are skipped.  Called by every thread of the CTA.
+constexpr int kMergeBatch = 8;
+
 __device__ void merge_unit(const SplitParams &p, const int64_t *cuts, int u, int c0, int c1, int b, int h0,
-                           int gh, int warp, int nwarps, int lane, float *s_w) {
+                           int gh, int warp, int nwarps, int lane, float *s_m) {
   const int n = c1 - c0 + 1;
-  for (int hh = warp; hh < gh; hh += nwarps) {
-    float *w = s_w + warp * (kMaxCtas + 1);
-    float mstar = -INFINITY, Mstar = -INFINITY;
-    for (int i = lane; i < n; i += 32) {
-      const int c = c0 + i;
-      if (cuts[c + 1] > cuts[c]) {
-        const float4 h = __ldcg(reinterpret_cast<const float4 *>(p.ws + p.slot0 + ((int64_t)u + c) * kSlot + hh * kPW));
-        mstar = fmaxf(mstar, h.x);
-        Mstar = fmaxf(Mstar, h.z);
+  const int parts = nwarps / gh;  // gh <= 8 <= nwarps
+  if (warp < gh * parts) {
+    const int hh = warp % gh, part = warp / gh;
+    const int i_lo = part * n / parts, i_hi = (part + 1) * n / parts;
+    const float *slots = p.ws + p.slot0 + ((int64_t)u + c0) * kSlot + hh * kPW;
+    float m_run = -INFINITY, M_run = -INFINITY, l = 0.f;
+    float a[4] = {0.f, 0.f, 0.f, 0.f};
+    for (int i0 = i_lo; i0 < i_hi; i0 += kMergeBatch) {
+      float4 hd[kMergeBatch], v[kMergeBatch];
+#pragma unroll
+      for (int j = 0; j < kMergeBatch; ++j) {
+        const int i = i0 + j;
+        const bool live = i < i_hi && cuts[c0 + i + 1] > cuts[c0 + i];
+        const float *sl = slots + (int64_t)(live ? i : 0) * kSlot;
+        hd[j] = live ? __ldcg(reinterpret_cast<const float4 *>(sl)) : make_float4(-INFINITY, 0.f, -INFINITY, 0.f);
+        v[j] = live ? __ldcg(reinterpret_cast<const float4 *>(sl + 4 + lane * 4)) : make_float4(0.f, 0.f, 0.f, 0.f);
+      }
+      float mb = m_run, Mb = M_run;
+#pragma unroll
+      for (int j = 0; j < kMergeBatch; ++j) {
+        mb = fmaxf(mb, hd[j].x);
+        Mb = fmaxf(Mb, hd[j].z);
+      }
+      const float ms = mb == -INFINITY ? 0.f : mb, Ms = Mb == -INFINITY ? 0.f : Mb;
+      l *= ex2(m_run - ms);
+      const float r = ex2(M_run - Ms);
+#pragma unroll
+      for (int i = 0; i < 4; ++i) a[i] *= r;
+      m_run = mb;
+      M_run = Mb;
+#pragma unroll
+      for (int j = 0; j < kMergeBatch; ++j) {
+        l = fmaf(hd[j].y, ex2(hd[j].x - ms), l);
+        const float w = ex2(hd[j].z - Ms);
+        a[0] = fmaf(v[j].x, w, a[0]);
+        a[1] = fmaf(v[j].y, w, a[1]);
+        a[2] = fmaf(v[j].z, w, a[2]);
+        a[3] = fmaf(v[j].w, w, a[3]);
       }
     }
-#pragma unroll
-    for (int o = 16; o >= 1; o >>= 1) {
-      mstar = fmaxf(mstar, __shfl_xor_sync(dev::kFull, mstar, o));
-      Mstar = fmaxf(Mstar, __shfl_xor_sync(dev::kFull, Mstar, o));
+    float *mine = s_m + warp * kPW;
+    if (lane == 0) {
+      mine[0] = m_run;
+      mine[1] = l;
+      mine[2] = M_run;
+    }
+    *reinterpret_cast<float4 *>(mine + 4 + lane * 4) = make_float4(a[0], a[1], a[2], a[3]);
+  }
+  __syncthreads();
+  if (warp < gh) {
+    const int hh = warp;
+    float m_all = -INFINITY, M_all = -INFINITY;
+    for (int part = 0; part < parts; ++part) {
+      m_all = fmaxf(m_all, s_m[(part * gh + hh) * kPW + 0]);
+      M_all = fmaxf(M_all, s_m[(part * gh + hh) * kPW + 2]);
     }
     float *out = p.out + ((int64_t)b * p.Hq + h0 + hh) * kD + lane * 4;
-    if (mstar == -INFINITY) {
+    if (m_all == -INFINITY) {
       *reinterpret_cast<float4 *>(out) = make_float4(0.f, 0.f, 0.f, 0.f);
-      continue;
-    }
-    const float M0 = Mstar == -INFINITY ? 0.f : Mstar;
-    float l = 0.f;
-    for (int i = lane; i < n; i += 32) {
-      const int c = c0 + i;
-      float wi = 0.f;
-      if (cuts[c + 1] > cuts[c]) {
-        const float4 h = __ldcg(reinterpret_cast<const float4 *>(p.ws + p.slot0 + ((int64_t)u + c) * kSlot + hh * kPW));
-        l += h.y * ex2(h.x - mstar);
-        wi = ex2(h.z - M0);
+    } else {
+      const float Ms = M_all == -INFINITY ? 0.f : M_all;
+      float l = 0.f, a[4] = {0.f, 0.f, 0.f, 0.f};
+      for (int part = 0; part < parts; ++part) {
+        const float *q = s_m + (part * gh + hh) * kPW;
+        l = fmaf(q[1], ex2(q[0] - m_all), l);
+        const float w = ex2(q[2] - Ms);
+        const float4 v = *reinterpret_cast<const float4 *>(q + 4 + lane * 4);
+        a[0] = fmaf(v.x, w, a[0]);
+        a[1] = fmaf(v.y, w, a[1]);
+        a[2] = fmaf(v.z, w, a[2]);
+        a[3] = fmaf(v.w, w, a[3]);
       }
-      w[i] = wi;
+      const float f = ex2(Ms - m_all) / l * 0.08838834764831845f;
+#pragma unroll
+      for (int i = 0; i < 4; ++i) a[i] *= f;
+      dev::fwht<32, 4>(a, lane);
+      float o4[4];
+#pragma unroll
+      for (int i = 0; i < 4; ++i) o4[i] = p.vsign[lane * 4 + i] < 0 ? -a[i] : a[i];
+      *reinterpret_cast<float4 *>(out) = make_float4(o4[0], o4[1], o4[2], o4[3]);
     }
-#pragma unroll
-    for (int o = 16; o >= 1; o >>= 1) l += __shfl_xor_sync(dev::kFull, l, o);
-    __syncwarp();
-    float a[4] = {0.f, 0.f, 0.f, 0.f};
-    const float *base = p.ws + p.slot0 + ((int64_t)u + c0) * kSlot + hh * kPW + 4 + lane * 4;
-#pragma unroll 8
-    for (int i = 0; i < n; ++i) {
-      const float wi = w[i];
-      // an empty CTA never wrote its slot: read nothing there
-      const float4 v = wi != 0.f ? __ldcg(reinterpret_cast<const float4 *>(base + (int64_t)i * kSlot))
-                                 : make_float4(0.f, 0.f, 0.f, 0.f);
-      a[0] = fmaf(v.x, wi, a[0]);
-      a[1] = fmaf(v.y, wi, a[1]);
-      a[2] = fmaf(v.z, wi, a[2]);
-      a[3] = fmaf(v.w, wi, a[3]);
-    }
-    __syncwarp();
-    const float f = ex2(M0 - mstar) / l * 0.08838834764831845f;
-#pragma unroll
-    for (int i = 0; i < 4; ++i) a[i] *= f;
-    dev::fwht<32, 4>(a, lane);
-    float o4[4];
-#pragma unroll
-    for (int i = 0; i < 4; ++i) o4[i] = p.vsign[lane * 4 + i] < 0 ? -a[i] : a[i];
-    *reinterpret_cast<float4 *>(out) = make_float4(o4[0], o4[1], o4[2], o4[3]);
   }
 }
 
@@ -649,22 +678,50 @@ __global__ void __launch_bounds__((PACK && !KPROD ? 12 : 8) * 32, 1) decode_spli
   const int64_t T = flat_total(p.seq_lens, p.seq_len, p.B, UH);
   const int64_t x0 = cut(T, p.ctas, blockIdx.x), x1 = cut(T, p.ctas, blockIdx.x + 1);
   if (x0 >= x1) return;
-  for (int c = tid; c <= p.ctas; c += kThreads) s_cut[c] = cut(T, p.ctas, c);
+  const bool unit = p.ksn == 1 && p.vsn == 1;
+  // warm L2 with this warp's first two chunks while the tables are set up
+  if (unit && lane == 0) {
+    int u;
+    int64_t ustart, ulen;
+    locate(p.seq_lens, p.seq_len, p.B, UH, x0, &u, &ustart, &ulen);
+    const int64_t t0 = x0 - ustart, t1 = min(x1, ustart + ulen) - ustart;
+    const int64_t nch = (t1 - t0 + kChunk - 1) / kChunk, pw = (nch + kWarps - 1) / kWarps;
+    const int64_t cb = min(nch, (int64_t)warp * pw), ce = min(nch, cb + pw);
+    const int b = u / UH, kvh = (u % UH) / p.groups;
+    if (cb < ce) {
+      const int64_t j = t0 + cb * kChunk;
+      prefetch_chunk<KBM, KPROD, VBM>(p, (int64_t)b * p.ksb + (int64_t)kvh * p.ksh + j,
+                                      (int64_t)b * p.vsb + (int64_t)kvh * p.vsh + j, min(2 * (int64_t)kChunk, t1 - j));
+    }
+  }
 
-  // ---- once per CTA: replicate the two pair tables per lane
+  // ---- once per CTA: the two pair tables (512 words), every load in
+  // flight before any store, staged in shared memory, then one copy per lane
+  float inv_sK, inv_sV;
   {
     const uint32_t *ktab = reinterpret_cast<const uint32_t *>(p.ws + 64);
     const uint32_t *vtab = reinterpret_cast<const uint32_t *>(p.ws + 320);
+    uint32_t *stage = reinterpret_cast<uint32_t *>(s_part);
+    static_assert(kThreads >= 256, "two staging loads per thread cover the 512 words");
+    const int i0 = tid, i1 = tid + kThreads;
+    uint32_t v0 = 0u, v1 = 0u;
+    if (i0 < 256) v0 = KBM > 0 ? __ldg(ktab + i0) : 0u;
+    else if (i0 < 512) v0 = __ldg(vtab + (i0 - 256));
+    if (i1 < 512) v1 = __ldg(vtab + (i1 - 256));
+    inv_sK = __ldg(p.ws + 0);
+    inv_sV = __ldg(p.ws + 1);
+    for (int c = tid; c <= p.ctas; c += kThreads) s_cut[c] = cut(T, p.ctas, c);
+    if (i0 < 512) stage[i0] = v0;
+    if (i1 < 512) stage[i1] = v1;
+    __syncthreads();
     uint4 *tab = reinterpret_cast<uint4 *>(smem);
     for (int i = tid; i < 256 * 16; i += kThreads) {  // 16 uint4 per 256-byte row
       const int e = i >> 4, part = i & 15;
-      const uint32_t v = part < 8 ? (KBM > 0 ? __ldg(ktab + e) : 0u) : __ldg(vtab + e);
+      const uint32_t v = stage[part < 8 ? e : 256 + e];
       tab[i] = make_uint4(v, v, v, v);
     }
   }
-  const float inv_sK = __ldg(p.ws + 0);
   const float sK = 1.0f / inv_sK;
-  const float inv_sV = __ldg(p.ws + 1);
   const uint32_t koff = lane * 4;
   const uint32_t voff = 128 + lane * 4;
   const bool want_scores = p.scores != nullptr;
@@ -701,15 +758,29 @@ __global__ void __launch_bounds__((PACK && !KPROD ? 12 : 8) * 32, 1) decode_spli
     const int h0 = kvh * p.g + grp * 8;
     const int gh = min(8, p.g - grp * 8);
 
-    __syncthreads();  // tables ready / previous piece's shared data consumed
-    for (int o = tid; o < 8 * kD; o += kThreads) {
-      const int hh = o / kD, k = o % kD;
-      const bool ok = hh < gh;
-      const int64_t qi = ((int64_t)b * p.Hq + h0 + hh) * kD + k;
-      s_q[o] = ok ? __ldg(p.ws + kHdr + qi) : 0.f;
-      if constexpr (KPROD) s_qs[o] = ok ? __ldg(p.ws + kHdr + (int64_t)p.B * p.Hq * kD + qi) : 0.f;
+    {
+      // q' (and S q') of the piece's heads: all loads in flight, then stored
+      constexpr int kQPer = (8 * kD + kThreads - 1) / kThreads;
+      float qv[kQPer], qsv[KPROD ? kQPer : 1];
+#pragma unroll
+      for (int j = 0; j < kQPer; ++j) {
+        const int o = tid + j * kThreads;
+        const bool ok = o < 8 * kD && (o / kD) < gh;
+        const int64_t qi = ((int64_t)b * p.Hq + h0) * kD + o;
+        qv[j] = ok ? __ldg(p.ws + kHdr + qi) : 0.f;
+        if constexpr (KPROD) qsv[j] = ok ? __ldg(p.ws + kHdr + (int64_t)p.B * p.Hq * kD + qi) : 0.f;
+      }
+      __syncthreads();  // tables ready / previous piece's shared data consumed
+#pragma unroll
+      for (int j = 0; j < kQPer; ++j) {
+        const int o = tid + j * kThreads;
+        if (o < 8 * kD) {
+          s_q[o] = qv[j];
+          if constexpr (KPROD) s_qs[o] = qsv[j];
+        }
+      }
+      __syncthreads();
     }
-    __syncthreads();
 
     // ---- B fragments in this lane's dim order.  PACK: column n < 4 is the
     // hi half of head n, n >= 4 the lo half of head n - 4.  Else qf = hi and
@@ -765,7 +836,6 @@ __global__ void __launch_bounds__((PACK && !KPROD ? 12 : 8) * 32, 1) decode_spli
 
     KBuf<KBM, KPROD> kb;
     VBuf<VBM> vb;
-    const bool unit = p.ksn == 1 && p.vsn == 1;
     // warm L2 one chunk beyond the register prefetch
     if (unit && lane == 0 && c_begin + 1 < c_end) {
       const int64_t jp = t0 + (c_begin + 1) * kChunk;
@@ -1060,11 +1130,13 @@ __global__ void __launch_bounds__((PACK && !KPROD ? 12 : 8) * 32, 1) decode_spli
       }
     }
     // ---- the last CTA to finish a unit merges its slots into the output.
-    // Classic fence-then-count: every CTA publishes its slot, fences, and
-    // bumps the unit's counter once; no CTA ever waits on another.
-    __threadfence();
+    // Every CTA publishes its slot, then thread 0 fences (after the barrier,
+    // so the fence covers the whole CTA's stores) and bumps the unit's
+    // counter once; the last arrival fences again before the merge reads.
+    // No CTA ever waits on another.
     __syncthreads();
     if (tid == 0) {
+      __threadfence();
       const int c0 = cta_of(s_cut, p.ctas, ustart), c1 = cta_of(s_cut, p.ctas, ustart + ulen - 1);
       // CTAs with an empty range (only when the space is shorter than the
       // grid) never arrive, so count the non-empty ones of the span
@@ -1072,10 +1144,10 @@ __global__ void __launch_bounds__((PACK && !KPROD ? 12 : 8) * 32, 1) decode_spli
       for (int c = c0; c <= c1; ++c) n += s_cut[c + 1] > s_cut[c] ? 1u : 0u;
       const unsigned prev = atomicAdd(p.cnt + u, 1u);
       s_last = (prev + 1 == n) ? 1 : 0;
+      if (prev + 1 == n) __threadfence();
     }
     __syncthreads();
     if (s_last) {
-      __threadfence();
       const int c0 = cta_of(s_cut, p.ctas, ustart), c1 = cta_of(s_cut, p.ctas, ustart + ulen - 1);
       merge_unit(p, s_cut, u, c0, c1, b, h0, gh, warp, kWarps, lane, s_part);
     }
@@ -1167,7 +1239,18 @@ cudaError_t launch_decode(const DecodeArgs &a, cudaStream_t s) {
   sp.groups = (sp.g + 7) / 8;
   sp.seq_len = a.seq_len;
   sp.seq_lens = a.seq_lens;
-  sp.ctas = a.splits;
+  // When the units fit the grid, a CTA count that is a multiple of the unit
+  // count (if it idles at most 5% of the CTAs) keeps every CTA inside one
+  // unit: no CTA then works on two pieces in sequence.
+  {
+    const int64_t units = (int64_t)a.B * a.Hkv * sp.groups;
+    int ctas = a.splits;
+    if (units <= ctas) {
+      const int64_t aligned = (ctas / units) * units;
+      if (aligned * 20 >= (int64_t)ctas * 19) ctas = (int)aligned;
+    }
+    sp.ctas = ctas;
+  }
   sp.kc = a.k.codes;
   sp.kj = a.k.qjl;
   sp.kn = a.k.norms;
