@@ -189,7 +189,7 @@ def run_ours(args):
         barrier()
     t_ms = ev0.elapsed_time(ev1)
 
-    # the dominant kernel pair (split + combine of tq_decode_attention), live
+    # the dominant kernels (prep + split of tq_decode_attention), live
     d_reps = max(1, reps)
     e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
     with torch.cuda.stream(stream):
@@ -250,7 +250,7 @@ def run_ours(args):
                                    "d=128 N=32768, K/V TurboQuant_mse b=4, randomized Hadamard",
                        "global_batch": B * ws, "seq_len": N, "parallelism": f"replicas x{ws}",
                        "l2": f"{COPIES} rotating cache copies ({COPIES * dec_bytes / 1e6:.0f} MB > 126 MB L2)"},
-            "roofline": {"kernel": "tq_decode_attention (split + combine)", "bound": "hbm",
+            "roofline": {"kernel": "tq_decode_attention (prep + split)", "bound": "hbm",
                          "achieved": achieved, "peak": pk["hbm_gbs"], "unit": "GB/s",
                          "frac": achieved / pk["hbm_gbs"], "peak_kind": pk_kind,
                          "bytes_per_launch": dec_bytes, "ms_per_launch": dec_ms,

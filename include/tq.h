@@ -155,7 +155,7 @@ size_t tq_decode_workspace_bytes(int32_t B, int32_t Hq, int32_t Hkv,
 
 /* Decode attention.  q: [B][Hq][d] (q_dtype, DEVICE).  Query head hq reads
  * kv head hq / (Hq/Hkv).  Cached tokens 0..L_b-1 of batch b are attended
- * with L_b = seq_lens[b] (DEVICE int32 [B], each 0..seq_len) or seq_len when
+ * with L_b = seq_lens[b] (DEVICE int32 [B], each 0..seq_len; seq_len < 2^31) or seq_len when
  * seq_lens is NULL; no causal mask.  The query is rotated once by the key
  * rotation; scores are
  *   s_j = n_j (<q', c_K[idx_j]> + [prod] ||r_j|| sqrt(pi/2)/d <S q', sign_j>)
@@ -163,7 +163,8 @@ size_t tq_decode_workspace_bytes(int32_t B, int32_t Hq, int32_t Hkv,
  * and rotated back once at the end.  out: [B][Hq][d] fp32 (DEVICE); a batch
  * with L_b == 0 gets zeros.  scores_out: optional [B][Hq][seq_len] fp32 of
  * the pre-scale estimator s_j (entries j >= L_b untouched), or NULL.
- * V must be mse (prod values return TQ_EUNSUPPORTED); d must be 128 or 64.
+ * V must be mse (prod values return TQ_EUNSUPPORTED); d must be 128 (other d
+ * return TQ_EUNSUPPORTED).
  * workspace: DEVICE, at least tq_decode_workspace_bytes(...) bytes, 16-byte
  * aligned, else TQ_EWORKSPACE. */
 tq_status tq_decode_attention(const tq_quantizer *kq, const tq_quantizer *vq,

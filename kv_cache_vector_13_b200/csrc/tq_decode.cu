@@ -16,13 +16,18 @@
 // search over 4096 candidates in [1, 2)) and writes the 256-entry pair table
 // entry e -> half2(fp16(s c[e & m]), fp16(s c[(e >> b_m) & m])).
 // Kernel 1 (split), persistent: one CTA per SM (12 warps when a kv head has
-// <= 4 query heads and the keys are mse, else 8); a warp issues its next chunk's key loads as soon
-// as the current keys are scored and its value loads once PV is done.  The work is the
-// flattened space of (unit = batch x kv head x group of <= 8 query heads,
-// token) pairs, cut into one equal contiguous range per CTA; a range covers
-// one or a few "pieces" (CTA, unit).  Per CTA, once: the two pair tables are
-// copied into shared memory, replicated per lane (entry e, lane l at
-// e*256 + 4l, values at +128) so that table reads never conflict on banks.
+// <= 4 query heads and the keys are mse, else 8); a warp issues its next
+// chunk's key loads as soon as the current keys are scored and its value
+// loads once PV is done, and warms L2 with bulk prefetches a window of 4
+// chunks ahead.  The work is the flattened space of (unit = batch x kv head
+// x group of <= 8 query heads, token) pairs, cut into one equal contiguous
+// range per CTA; a range covers one or a few "pieces" (CTA, unit).  When the
+// units fit the grid, the host rounds the CTA count down to a multiple of
+// the unit count if that idles at most 5% of the SMs, so each CTA stays
+// inside one unit.  Per CTA, once: the two pair tables are copied into
+// shared memory at address 64 KiB, replicated per lane (entry e, lane l at
+// 64 KiB + e*256 + 4l, values at +128) so that table reads never conflict
+// on banks and one byte permute forms a lookup's whole address.
 // Per piece: the group's rotated queries are split into hi + lo fp16 halves;
 // then every warp streams its share of 32-token chunks:
 //   * packed K/V words go from HBM straight to registers, one pass;
@@ -64,17 +69,32 @@ namespace tq {
 namespace {
 
 constexpr int kD = 128;
-constexpr int kMaxWarps = 12;
 constexpr int kMaxCtas = 1024;  // persistent CTAs supported (one per SM)
 constexpr int kChunk = 32;               // tokens per warp iteration
 constexpr int kLutBytes = 256 * 256;     // K and V pair tables, per-lane copies
+// Shared-window address of the pair tables.  Entry e, lane l sits at
+// kLutAddr + 256 e + 4 l (+128 for the value table): with the tables on a
+// 64 KiB boundary, one byte permute of (code byte, lane offset) yields the
+// complete shared address of a lookup.
+constexpr uint32_t kLutAddr = 0x10000;
+constexpr int kPfWin = 4;                // chunks per L2 prefetch window
 constexpr int kPW = kD + 4;              // floats per head in a partial: m, l, M, pad, o'[d]
 constexpr int kSlot = 8 * kPW;           // floats per partial slot (8 heads)
 constexpr int kScaleCands = 4096;
 // workspace layout (floats): [0, 2) scales 1/s_K, 1/s_V; [64, 320) K pair
-// table; [320, 576) V pair table; [kHdr, +B*Hq*d) q'; [+B*Hq*d) S q';
-// then (units + CTAs) partial slots of kSlot floats.
+// table; [320, 576) V pair table; [kHdr, +units * kFragWords) the query
+// fragments of every unit; then (units + CTAs) partial slots of kSlot
+// floats; then one arrival counter per unit.
 constexpr int kHdr = 1024;
+// Query fragments of a unit: 64 words per lane, stored as [16][32 lanes][4]
+// so that a warp loads 4 words per lane with one coalesced 16-byte load.
+// Word w of lane (g8, tig), with q' the unit's rotated queries and
+// sel = lo half for PACK lanes g8 >= 4:
+//   PACK (<= 4 heads): w = 2s + j      : sel(q'[g8 & 3][32 tig + 4s + 2j, +1])
+//                      w = 16 + 2s + j : sel(Sq'[g8 & 3][32 tig + 15 - 2s - j, +16])
+//   8 heads          : w = 2s + j / 16 + 2s + j  : hi / lo of q'[g8][32 tig + 4s + 2j, +1]
+//                      w = 32 + ... / 48 + ...   : hi / lo of Sq'[g8][32 tig + 15 - 2s - j, +16]
+constexpr int kFragWords = 32 * 64;
 constexpr float kLog2e = 1.4426950408889634f;
 constexpr float kKappa = 1.2533141373155003f / (float)kD;  // sqrt(pi/2)/d
 
@@ -102,6 +122,7 @@ struct SplitParams {
   float scale_log2;  // softmax_scale * log2(e)
   float *scores;
   float *ws;
+  const uint4 *frag;  // query fragments, kFragWords per unit
   int64_t slot0;      // first float of the partial slots
   unsigned *cnt;      // per-unit arrival counters (zeroed by the prep kernel)
   float *out;
@@ -121,10 +142,11 @@ struct PrepParams {
   float *ws;
   unsigned *cnt;
   int units;
-  int Hq;
+  int Hq, Hkv, g, groups;
   int64_t seq_len;
   const int32_t *seq_lens;
   float *out;
+  uint32_t *frag;  // kFragWords per unit
 };
 
 
@@ -144,14 +166,24 @@ __device__ __forceinline__ uint32_t movmatrix_trans(uint32_t x) {
   return y;
 }
 
-// table entry at byte offset `off` of a shared table
-__device__ __forceinline__ uint32_t lut(const char *tab, uint32_t off) {
-  return *reinterpret_cast<const uint32_t *>(tab + off);
+// table entry at shared-window address `addr` (written once, before the
+// barrier that precedes every lookup)
+__device__ __forceinline__ uint32_t lut(uint32_t addr) {
+  uint32_t v;
+  asm("ld.shared.b32 %0, [%1];\n" : "=r"(v) : "r"(addr));
+  return v;
 }
 
 __device__ __forceinline__ uint32_t pack_half2(float lo, float hi) {
   const __half2 h = __floats2half2_rn(lo, hi);
   return *reinterpret_cast<const uint32_t *>(&h);
+}
+
+// fp16 (hi, lo) halves of the pair (a, b): hi = fp16(x), lo = fp16(x - hi)
+__device__ __forceinline__ void split_pair(float a, float b, uint32_t &hi, uint32_t &lo) {
+  hi = pack_half2(a, b);
+  const float2 f = __half22float2(*reinterpret_cast<const __half2 *>(&hi));
+  lo = pack_half2(a - f.x, b - f.y);
 }
 
 // hi = fp16(x), lo = fp16(x - hi): x to ~22 significant bits
@@ -353,6 +385,9 @@ __device__ void scale_and_table(const float *cent, int bm, float *inv_scale, uin
 // q' = H(sigma q)/sqrt(d) and q_s = S q'.  The last two blocks: the K and
 // V scale and pair table.
 __global__ void __launch_bounds__(256) decode_prep_kernel(PrepParams p) {
+  // the split kernel may be scheduled now: it waits for this grid to finish
+  // (griddepcontrol.wait) before it reads anything written here
+  asm volatile("griddepcontrol.launch_dependents;\n" ::: "memory");
   const int nqb = (p.nheads + 1) / 2;
   for (int i = blockIdx.x * blockDim.x + threadIdx.x; i < p.units; i += gridDim.x * blockDim.x) p.cnt[i] = 0u;
   if ((int)blockIdx.x >= nqb) {
@@ -364,7 +399,7 @@ __global__ void __launch_bounds__(256) decode_prep_kernel(PrepParams p) {
     }
     return;
   }
-  __shared__ float s_q[2][kD];
+  __shared__ float s_q[2][kD], s_qs[2][kD];
   const int half = threadIdx.x >> 7, t = threadIdx.x & 127;
   const int head = blockIdx.x * 2 + half;
   const bool valid = head < p.nheads;
@@ -396,10 +431,7 @@ __global__ void __launch_bounds__(256) decode_prep_kernel(PrepParams p) {
     for (int i = 0; i < 4; ++i) s_q[half][lane * 4 + i] = a[i] * 0.08838834764831845f;
   }
   __syncthreads();
-  if (!valid) return;
-  float *qo = p.ws + kHdr + (int64_t)head * kD;
-  qo[t] = s_q[half][t];
-  if (p.kS) {
+  if (valid && p.kS) {
     const float4 *Sk = reinterpret_cast<const float4 *>(p.kS + (size_t)t * kD);
     float acc = 0.f;
 #pragma unroll 8
@@ -410,7 +442,37 @@ __global__ void __launch_bounds__(256) decode_prep_kernel(PrepParams p) {
       acc = fmaf(sv.z, s_q[half][4 * i + 2], acc);
       acc = fmaf(sv.w, s_q[half][4 * i + 3], acc);
     }
-    p.ws[kHdr + (int64_t)p.nheads * kD + (int64_t)head * kD + t] = acc;
+    s_qs[half][t] = acc;
+  }
+  __syncthreads();
+  if (!valid) return;
+  // this head's fragment words (the layout of kFragWords above)
+  const int b = head / p.Hq, hq = head % p.Hq;
+  const int kvh = hq / p.g, grp = (hq % p.g) / 8, hh = (hq % p.g) % 8;
+  const int64_t u = ((int64_t)b * p.Hkv + kvh) * p.groups + grp;
+  uint32_t *fu = p.frag + u * kFragWords;
+  auto put = [&](int ln, int w, uint32_t v) { fu[((w >> 2) * 32 + ln) * 4 + (w & 3)] = v; };
+  const float *qv = s_q[half], *sv = s_qs[half];
+  if (p.g <= 4) {
+    const int ls = t >> 4, w = t & 15, sidx = w >> 1, j = w & 1;
+    const int g8 = hh + 4 * (ls >> 2), tig = ls & 3, ln = g8 * 4 + tig;
+    const bool lo = g8 >= 4;
+    const int d0 = 32 * tig + 4 * sidx + 2 * j;
+    put(ln, w, lo ? pack_lo(qv[d0], qv[d0 + 1]) : pack_hi(qv[d0], qv[d0 + 1]));
+    if (p.kS) {
+      const int e = 32 * tig + 15 - 2 * sidx - j;
+      put(ln, 16 + w, lo ? pack_lo(sv[e], sv[e + 16]) : pack_hi(sv[e], sv[e + 16]));
+    }
+  } else {
+    const int tig = t >> 5, w = t & 31, sidx = (w & 15) >> 1, j = w & 1;
+    const int ln = hh * 4 + tig;
+    const bool lo = w >= 16;
+    const int d0 = 32 * tig + 4 * sidx + 2 * j;
+    put(ln, w, lo ? pack_lo(qv[d0], qv[d0 + 1]) : pack_hi(qv[d0], qv[d0 + 1]));
+    if (p.kS) {
+      const int e = 32 * tig + 15 - 2 * sidx - j;
+      put(ln, 32 + w, lo ? pack_lo(sv[e], sv[e + 16]) : pack_hi(sv[e], sv[e + 16]));
+    }
   }
 }
 
@@ -433,45 +495,20 @@ struct VBuf {
   uint32_t w[2][4][VChunk<VBM>::NW];
 };
 
-// Per-piece row offsets (in records) of the lane's tokens inside a chunk.
-struct RowOffs {
-  int32_t k[2][2], kv[2][2], v[2][4];  // K rows, V records of the K rows, V tokens
-  int32_t rk[2][2], rv[2][4];          // token index inside the chunk
-};
-
-// Loads the key side of one chunk.  FAST: unit record strides and a full
-// chunk, so every address is a per-lane base plus a compile-time offset.
-template <bool FAST, int KBM, bool KPROD>
-__device__ __forceinline__ void load_k(KBuf<KBM, KPROD> &c, const SplitParams &p, int64_t krec0, int64_t vrec0,
-                                       int nvalid, const RowOffs &o, int tig, int g8) {
+// Loads the key side of one chunk with any record strides and nvalid <= 32
+// valid tokens (rows past nvalid are masked: norm -1).  Row offsets are
+// computed here, so nothing of this path stays live across the main loop.
+template <int KBM, bool KPROD>
+__device__ __forceinline__ void load_k_slow(KBuf<KBM, KPROD> &c, const SplitParams &p, int64_t krec0, int64_t vrec0,
+                                            int nvalid, int tig, int g8) {
   constexpr int KCB = kD * KBM / 8;
-  if constexpr (FAST) {
-    const int64_t kr0 = krec0 + g8, vr0 = vrec0 + g8;
-    const uint8_t *kcp = p.kc + kr0 * KCB + tig * (4 * KBM);
-    const uint32_t *kjp = KPROD ? reinterpret_cast<const uint32_t *>(p.kj + kr0 * (kD / 8)) + tig : nullptr;
-    const float *knp = p.kn + kr0, *krp = KPROD ? p.kr + kr0 : nullptr, *vnp = p.vn + vr0;
-#pragma unroll
-    for (int ms = 0; ms < 2; ++ms) {
-#pragma unroll
-      for (int r = 0; r < 2; ++r) {
-        const int t = 16 * ms + 8 * r;  // compile-time after unrolling
-        if constexpr (KBM > 0) load_k32<KBM>(kcp + t * KCB, c.w[ms][r]);
-        if constexpr (KPROD) {
-          c.qj[ms][r] = __ldg(kjp + t * (kD / 32));
-          c.kr[ms][r] = __ldg(krp + t);
-        }
-        c.kn[ms][r] = __ldg(knp + t);
-        c.vn[ms][r] = __ldg(vnp + t);
-      }
-    }
-    return;
-  }
 #pragma unroll
   for (int ms = 0; ms < 2; ++ms) {
 #pragma unroll
     for (int r = 0; r < 2; ++r) {
-      const bool ok = o.rk[ms][r] < nvalid;
-      const int64_t rec = krec0 + o.k[ms][r];
+      const int t = 16 * ms + 8 * r + g8;
+      const bool ok = t < nvalid;
+      const int64_t rec = krec0 + (int64_t)t * p.ksn;
       if constexpr (KBM > 0) {
         if (ok) {
           load_k32<KBM>(p.kc + rec * KCB + tig * (4 * KBM), c.w[ms][r]);
@@ -485,31 +522,84 @@ __device__ __forceinline__ void load_k(KBuf<KBM, KPROD> &c, const SplitParams &p
         c.kr[ms][r] = ok ? __ldg(p.kr + rec) : 0.f;
       }
       c.kn[ms][r] = ok ? __ldg(p.kn + rec) : -1.f;  // -1 marks a masked row
-      c.vn[ms][r] = ok ? __ldg(p.vn + vrec0 + o.kv[ms][r]) : 1.f;
+      c.vn[ms][r] = ok ? __ldg(p.vn + vrec0 + (int64_t)t * p.vsn) : 1.f;
     }
   }
 }
 
-template <bool FAST, int VBM>
-__device__ __forceinline__ void load_v(VBuf<VBM> &c, const SplitParams &p, int64_t vrec0, int nvalid,
-                                       const RowOffs &o, int g8, int tig) {
+// Per-lane pointers of the fast path (unit record strides) at chunk 0 of a
+// piece; chunk c adds c * kChunk records.
+template <int KBM, bool KPROD, int VBM>
+struct FastPtrs {
+  const uint8_t *kc;
+  const uint32_t *kj;
+  const float *kn, *kr, *vn;
+  const uint8_t *vc;
+};
+
+template <int KBM, bool KPROD, int VBM>
+__device__ __forceinline__ FastPtrs<KBM, KPROD, VBM> fast_ptrs(const SplitParams &p, int64_t krec0, int64_t vrec0,
+                                                               int tig, int g8) {
+  constexpr int KCB = kD * KBM / 8, VCB = kD * VBM / 8;
+  FastPtrs<KBM, KPROD, VBM> f;
+  const int64_t kr0 = krec0 + g8, vr0 = vrec0 + g8;
+  f.kc = p.kc + kr0 * KCB + tig * (4 * KBM);
+  f.kj = KPROD ? reinterpret_cast<const uint32_t *>(p.kj + kr0 * (kD / 8)) + tig : nullptr;
+  f.kn = p.kn + kr0;
+  f.kr = KPROD ? p.kr + kr0 : nullptr;
+  f.vn = p.vn + vr0;
+  f.vc = p.vc + (vrec0 + 2 * tig) * VCB + g8 * (2 * VBM);
+  return f;
+}
+
+// Key side of full chunk c through the fast-path pointers.
+template <int KBM, bool KPROD, int VBM>
+__device__ __forceinline__ void load_k_fast(KBuf<KBM, KPROD> &c, const FastPtrs<KBM, KPROD, VBM> &f, int ci) {
+  constexpr int KCB = kD * KBM / 8;
+  const int64_t r0 = (int64_t)ci * kChunk;
+#pragma unroll
+  for (int ms = 0; ms < 2; ++ms) {
+#pragma unroll
+    for (int r = 0; r < 2; ++r) {
+      const int t = 16 * ms + 8 * r;
+      if constexpr (KBM > 0) load_k32<KBM>(f.kc + (r0 + t) * KCB, c.w[ms][r]);
+      if constexpr (KPROD) {
+        c.qj[ms][r] = __ldg(f.kj + (r0 + t) * (kD / 32));
+        c.kr[ms][r] = __ldg(f.kr + r0 + t);
+      }
+      c.kn[ms][r] = __ldg(f.kn + r0 + t);
+      c.vn[ms][r] = __ldg(f.vn + r0 + t);
+    }
+  }
+}
+
+// Value side of full chunk c through the fast-path pointers.
+template <int KBM, bool KPROD, int VBM>
+__device__ __forceinline__ void load_v_fast(VBuf<VBM> &c, const FastPtrs<KBM, KPROD, VBM> &f, int ci, int g8) {
+  constexpr int VCB = kD * VBM / 8;
+  const int64_t r0 = (int64_t)ci * kChunk;
+#pragma unroll
+  for (int ms = 0; ms < 2; ++ms) {
+#pragma unroll
+    for (int q4 = 0; q4 < 4; ++q4)
+      load_v16<VBM>(f.vc + (r0 + 16 * ms + (q4 & 1) + 8 * (q4 >> 1)) * VCB, c.w[ms][q4], g8);
+  }
+}
+
+// Value side of one chunk with any record strides and nvalid <= 32 valid
+// tokens (rows past nvalid read as code 0; their weights are 0).
+template <int VBM>
+__device__ __forceinline__ void load_v_slow(VBuf<VBM> &c, const SplitParams &p, int64_t vrec0, int nvalid, int g8,
+                                            int tig) {
   constexpr int VCB = kD * VBM / 8;
   constexpr int NW = VChunk<VBM>::NW;
-  if constexpr (FAST) {
-    const uint8_t *vcp = p.vc + (vrec0 + 2 * tig) * VCB + g8 * (2 * VBM);
-#pragma unroll
-    for (int ms = 0; ms < 2; ++ms) {
-#pragma unroll
-      for (int q4 = 0; q4 < 4; ++q4) load_v16<VBM>(vcp + (16 * ms + (q4 & 1) + 8 * (q4 >> 1)) * VCB, c.w[ms][q4], g8);
-    }
-    return;
-  }
 #pragma unroll
   for (int ms = 0; ms < 2; ++ms) {
 #pragma unroll
     for (int q4 = 0; q4 < 4; ++q4) {
-      if (o.rv[ms][q4] < nvalid) {
-        load_v16<VBM>(p.vc + (vrec0 + o.v[ms][q4]) * VCB + g8 * (2 * VBM), c.w[ms][q4], g8);
+      const int t = 16 * ms + 2 * tig + (q4 & 1) + 8 * (q4 >> 1);
+      if (t < nvalid) {
+        load_v16<VBM>(p.vc + (vrec0 + (int64_t)t * p.vsn) * VCB + g8 * (2 * VBM), c.w[ms][q4], g8);
       } else {
 #pragma unroll
         for (int i = 0; i < NW; ++i) c.w[ms][q4][i] = 0u;
@@ -666,9 +756,13 @@ __global__ void __launch_bounds__((PACK && !KPROD ? 12 : 8) * 32, 1) decode_spli
   constexpr int VW = VChunk<VBM>::NW;
   extern __shared__ float4 smem4[];
   char *smem = reinterpret_cast<char *>(smem4);
-  float *s_q = reinterpret_cast<float *>(smem + kLutBytes);  // [8][kD] q'
-  float *s_qs = s_q + 8 * kD;                                // [8][kD] S q'
-  float *s_part = s_qs + 8 * kD;                             // [kWarps][8][kPW]
+  // [kLutAddr, +64 KB): the pair tables; then the warps' partials.  The
+  // host sizes the allocation to reach past kLutAddr + kLutBytes + partials
+  // from any dynamic base at or below kLutAddr.
+  const uint32_t dyn_base = static_cast<uint32_t>(__cvta_generic_to_shared(smem4));
+  if (dyn_base > kLutAddr) return;  // excluded on the host
+  char *s_lut = smem + (kLutAddr - dyn_base);
+  float *s_part = reinterpret_cast<float *>(s_lut + kLutBytes);  // [kWarps][8][kPW]
   __shared__ int s_last;
   __shared__ int64_t s_cut[kMaxCtas + 1];
 
@@ -695,6 +789,12 @@ __global__ void __launch_bounds__((PACK && !KPROD ? 12 : 8) * 32, 1) decode_spli
     }
   }
 
+  for (int c = tid; c <= p.ctas; c += kThreads) s_cut[c] = cut(T, p.ctas, c);
+  // Everything above reads only the arguments and the cache; the workspace
+  // (tables, query fragments, counters) is written by the prep kernel, which may still be
+  // running when this grid starts (programmatic dependent launch).
+  asm volatile("griddepcontrol.wait;\n" ::: "memory");
+
   // ---- once per CTA: the two pair tables (512 words), every load in
   // flight before any store, staged in shared memory, then one copy per lane
   float inv_sK, inv_sV;
@@ -710,11 +810,10 @@ __global__ void __launch_bounds__((PACK && !KPROD ? 12 : 8) * 32, 1) decode_spli
     if (i1 < 512) v1 = __ldg(vtab + (i1 - 256));
     inv_sK = __ldg(p.ws + 0);
     inv_sV = __ldg(p.ws + 1);
-    for (int c = tid; c <= p.ctas; c += kThreads) s_cut[c] = cut(T, p.ctas, c);
     if (i0 < 512) stage[i0] = v0;
     if (i1 < 512) stage[i1] = v1;
     __syncthreads();
-    uint4 *tab = reinterpret_cast<uint4 *>(smem);
+    uint4 *tab = reinterpret_cast<uint4 *>(s_lut);
     for (int i = tid; i < 256 * 16; i += kThreads) {  // 16 uint4 per 256-byte row
       const int e = i >> 4, part = i & 15;
       const uint32_t v = stage[part < 8 ? e : 256 + e];
@@ -722,28 +821,10 @@ __global__ void __launch_bounds__((PACK && !KPROD ? 12 : 8) * 32, 1) decode_spli
     }
   }
   const float sK = 1.0f / inv_sK;
-  const uint32_t koff = lane * 4;
-  const uint32_t voff = 128 + lane * 4;
+  const float kscale = inv_sK * p.scale_log2;  // logit = raw score * n_K * kscale
+  const uint32_t koff = kLutAddr + lane * 4;
+  const uint32_t voff = kLutAddr + 128 + lane * 4;
   const bool want_scores = p.scores != nullptr;
-
-  // this lane's token rows inside a chunk, in records
-  RowOffs ro;
-#pragma unroll
-  for (int ms = 0; ms < 2; ++ms) {
-#pragma unroll
-    for (int r = 0; r < 2; ++r) {
-      const int t = 16 * ms + 8 * r + g8;
-      ro.rk[ms][r] = t;
-      ro.k[ms][r] = (int32_t)(t * p.ksn);
-      ro.kv[ms][r] = (int32_t)(t * p.vsn);
-    }
-#pragma unroll
-    for (int q4 = 0; q4 < 4; ++q4) {
-      const int t = 16 * ms + 2 * tig + (q4 & 1) + 8 * (q4 >> 1);
-      ro.rv[ms][q4] = t;
-      ro.v[ms][q4] = (int32_t)(t * p.vsn);
-    }
-  }
 
   for (int64_t x = x0; x < x1;) {
     int u;
@@ -758,66 +839,30 @@ __global__ void __launch_bounds__((PACK && !KPROD ? 12 : 8) * 32, 1) decode_spli
     const int h0 = kvh * p.g + grp * 8;
     const int gh = min(8, p.g - grp * 8);
 
-    {
-      // q' (and S q') of the piece's heads: all loads in flight, then stored
-      constexpr int kQPer = (8 * kD + kThreads - 1) / kThreads;
-      float qv[kQPer], qsv[KPROD ? kQPer : 1];
-#pragma unroll
-      for (int j = 0; j < kQPer; ++j) {
-        const int o = tid + j * kThreads;
-        const bool ok = o < 8 * kD && (o / kD) < gh;
-        const int64_t qi = ((int64_t)b * p.Hq + h0) * kD + o;
-        qv[j] = ok ? __ldg(p.ws + kHdr + qi) : 0.f;
-        if constexpr (KPROD) qsv[j] = ok ? __ldg(p.ws + kHdr + (int64_t)p.B * p.Hq * kD + qi) : 0.f;
-      }
-      __syncthreads();  // tables ready / previous piece's shared data consumed
-#pragma unroll
-      for (int j = 0; j < kQPer; ++j) {
-        const int o = tid + j * kThreads;
-        if (o < 8 * kD) {
-          s_q[o] = qv[j];
-          if constexpr (KPROD) s_qs[o] = qsv[j];
-        }
-      }
-      __syncthreads();
-    }
+    __syncthreads();  // tables ready / the previous piece's shared data consumed
 
-    // ---- B fragments in this lane's dim order.  PACK: column n < 4 is the
-    // hi half of head n, n >= 4 the lo half of head n - 4.  Else qf = hi and
-    // qf2 = lo of head g8.
+    // ---- B fragments of the unit, written by the prep kernel in this
+    // lane's register order.  PACK: column n < 4 is the hi half of head n,
+    // n >= 4 the lo half of head n - 4.  Else qf = hi and qf2 = lo of head
+    // g8.  Lanes whose head is absent (fewer than 4 or 8 heads) hold zeros.
     uint32_t qf[8][2], qf2[PACK ? 1 : 8][2];
     uint32_t qsf[KPROD ? 8 : 1][2], qsf2[(KPROD && !PACK) ? 8 : 1][2];
     {
-      const int hsrc = PACK ? (g8 & 3) : g8;
-      const bool lo_col = PACK && g8 >= 4;
-      const float *qv = s_q + hsrc * kD + 32 * tig;
+      const bool has = (PACK ? (g8 & 3) : g8) < gh;
+      const uint4 *fr = p.frag + (int64_t)u * (kFragWords / 4) + lane;
+      auto ld4 = [&](int w4) { return has ? __ldg(fr + w4 * 32) : make_uint4(0u, 0u, 0u, 0u); };
+      auto put = [](uint32_t (&f)[8][2], int k, uint4 v) {
+        f[2 * k][0] = v.x;
+        f[2 * k][1] = v.y;
+        f[2 * k + 1][0] = v.z;
+        f[2 * k + 1][1] = v.w;
+      };
 #pragma unroll
-      for (int s = 0; s < 8; ++s) {
-        if constexpr (PACK) {
-          qf[s][0] = lo_col ? pack_lo(qv[4 * s], qv[4 * s + 1]) : pack_hi(qv[4 * s], qv[4 * s + 1]);
-          qf[s][1] = lo_col ? pack_lo(qv[4 * s + 2], qv[4 * s + 3]) : pack_hi(qv[4 * s + 2], qv[4 * s + 3]);
-        } else {
-          qf[s][0] = pack_hi(qv[4 * s], qv[4 * s + 1]);
-          qf[s][1] = pack_hi(qv[4 * s + 2], qv[4 * s + 3]);
-          qf2[s][0] = pack_lo(qv[4 * s], qv[4 * s + 1]);
-          qf2[s][1] = pack_lo(qv[4 * s + 2], qv[4 * s + 3]);
-        }
-      }
-      if constexpr (KPROD) {
-        const float *sv = s_qs + hsrc * kD + 32 * tig;
-#pragma unroll
-        for (int s = 0; s < 8; ++s) {
-          const float a0 = sv[15 - 2 * s], a1 = sv[31 - 2 * s], a2 = sv[14 - 2 * s], a3 = sv[30 - 2 * s];
-          if constexpr (PACK) {
-            qsf[s][0] = lo_col ? pack_lo(a0, a1) : pack_hi(a0, a1);
-            qsf[s][1] = lo_col ? pack_lo(a2, a3) : pack_hi(a2, a3);
-          } else {
-            qsf[s][0] = pack_hi(a0, a1);
-            qsf[s][1] = pack_hi(a2, a3);
-            qsf2[s][0] = pack_lo(a0, a1);
-            qsf2[s][1] = pack_lo(a2, a3);
-          }
-        }
+      for (int k = 0; k < 4; ++k) {
+        put(qf, k, ld4(k));
+        if constexpr (!PACK) put(qf2, k, ld4(4 + k));
+        if constexpr (KPROD) put(qsf, k, ld4((PACK ? 4 : 8) + k));
+        if constexpr (KPROD && !PACK) put(qsf2, k, ld4(12 + k));
       }
     }
 
@@ -829,63 +874,70 @@ __global__ void __launch_bounds__((PACK && !KPROD ? 12 : 8) * 32, 1) decode_spli
 
     const int64_t kbase = (int64_t)b * p.ksb + (int64_t)kvh * p.ksh;
     const int64_t vbase = (int64_t)b * p.vsb + (int64_t)kvh * p.vsh;
-    const int64_t nchunks = (t1 - t0 + kChunk - 1) / kChunk;
-    const int64_t per_warp = (nchunks + kWarps - 1) / kWarps;
-    const int64_t c_begin = min(nchunks, (int64_t)warp * per_warp);
-    const int64_t c_end = min(nchunks, c_begin + per_warp);
+    // the piece's chunks [0, nch), of which [0, nfull) are full; this warp
+    // takes [c_begin, c_end).  A piece is shorter than 2^31 tokens.
+    const int nch = (int)((t1 - t0 + kChunk - 1) / kChunk);
+    const int nfull = (int)((t1 - t0) / kChunk);
+    const int per_warp = (nch + kWarps - 1) / kWarps;
+    const int c_begin = min(nch, warp * per_warp);
+    const int c_end = min(nch, c_begin + per_warp);
+    const FastPtrs<KBM, KPROD, VBM> fp = fast_ptrs<KBM, KPROD, VBM>(p, kbase + t0, vbase + t0, tig, g8);
 
     KBuf<KBM, KPROD> kb;
     VBuf<VBM> vb;
-    // warm L2 one chunk beyond the register prefetch
+    // warm L2 up to the end of the first prefetch window
     if (unit && lane == 0 && c_begin + 1 < c_end) {
-      const int64_t jp = t0 + (c_begin + 1) * kChunk;
-      prefetch_chunk<KBM, KPROD, VBM>(p, kbase + jp, vbase + jp, min((int64_t)kChunk, t1 - jp));
+      const int64_t jp = t0 + (int64_t)(c_begin + 1) * kChunk;
+      const int pe = min(c_end, c_begin + kPfWin);
+      prefetch_chunk<KBM, KPROD, VBM>(p, kbase + jp, vbase + jp, min((int64_t)(pe - c_begin - 1) * kChunk, t1 - jp));
     }
     if (c_begin < c_end) {
-      const int64_t j0 = t0 + c_begin * kChunk;
-      const int nv = (int)min((int64_t)kChunk, t1 - j0);
-      if (unit && nv == kChunk) {
-        load_k<true>(kb, p, kbase + j0, vbase + j0, nv, ro, tig, g8);
-        load_v<true>(vb, p, vbase + j0, nv, ro, g8, tig);
+      if (unit && c_begin < nfull) {
+        load_k_fast(kb, fp, c_begin);
+        load_v_fast(vb, fp, c_begin, g8);
       } else {
-        load_k<false>(kb, p, kbase + j0 * p.ksn, vbase + j0 * p.vsn, nv, ro, tig, g8);
-        load_v<false>(vb, p, vbase + j0 * p.vsn, nv, ro, g8, tig);
+        const int64_t j0 = t0 + (int64_t)c_begin * kChunk;
+        const int nv = (int)min((int64_t)kChunk, t1 - j0);
+        load_k_slow(kb, p, kbase + j0 * p.ksn, vbase + j0 * p.vsn, nv, tig, g8);
+        load_v_slow(vb, p, vbase + j0 * p.vsn, nv, g8, tig);
       }
     }
-    for (int64_t ci = c_begin; ci < c_end; ++ci) {
-      const int64_t j0 = t0 + ci * kChunk;
-      const int64_t jn = j0 + kChunk;
-      const bool more = ci + 1 < c_end;
-      const int nvn = more ? (int)min((int64_t)kChunk, t1 - jn) : 0;
-      const bool fast_next = unit && nvn == kChunk;
-      if (unit && lane == 0 && ci + 2 < c_end) {
-        const int64_t jp = jn + kChunk;
-        prefetch_chunk<KBM, KPROD, VBM>(p, kbase + jp, vbase + jp, min((int64_t)kChunk, t1 - jp));
+    for (int ci = c_begin; ci < c_end; ++ci) {
+      const int cn = ci + 1;
+      const bool more = cn < c_end;
+      const bool fast_next = unit && cn < nfull;
+      // every kPfWin chunks, warm L2 with the window after the next one
+      if (unit && lane == 0 && ((ci - c_begin) % kPfWin) == 0 && ci + kPfWin < c_end) {
+        const int64_t jp = t0 + (int64_t)(ci + kPfWin) * kChunk;
+        const int pe = min(c_end, ci + 2 * kPfWin);
+        prefetch_chunk<KBM, KPROD, VBM>(p, kbase + jp, vbase + jp,
+                                        min((int64_t)(pe - ci - kPfWin) * kChunk, t1 - jp));
       }
-      // -------- scores: rows (ms, r) -> token j0 + 16 ms + 8 r + g8
+      // -------- scores: rows (ms, r) -> token 32 ci + 16 ms + 8 r + g8
       float sc[2][4];
       float nvl[2][2];  // log2 n_V of the lane's rows
 #pragma unroll
       for (int ms = 0; ms < 2; ++ms) {
         const auto &kw = kb.w[ms];
         const auto &qj = kb.qj[ms];
-        float kn[2], kr[2];
+        bool ok[2];
+        float fs[2], kr[2];
 #pragma unroll
         for (int r = 0; r < 2; ++r) {
-          const bool ok = kb.kn[ms][r] >= 0.f;
-          kn[r] = ok ? kb.kn[ms][r] * inv_sK : -1.f;
+          ok[r] = kb.kn[ms][r] >= 0.f;
+          fs[r] = kb.kn[ms][r] * kscale;
           kr[r] = KPROD ? kb.kr[ms][r] * (kKappa * sK) : 0.f;  // the table holds s_K c
-          nvl[ms][r] = ok ? __log2f(kb.vn[ms][r]) : -INFINITY;
+          nvl[ms][r] = ok[r] ? __log2f(kb.vn[ms][r]) : -INFINITY;
         }
         float cm[4] = {0.f, 0.f, 0.f, 0.f};
         if constexpr (KBM > 0) {
 #define TQ_KSTEP(S)                                                               \
   {                                                                               \
     uint32_t a[4];                                                                \
-    a[0] = lut(smem, pair_addr<KBM, 2 * (S), KW>(kw[0], koff));                   \
-    a[1] = lut(smem, pair_addr<KBM, 2 * (S), KW>(kw[1], koff));                   \
-    a[2] = lut(smem, pair_addr<KBM, 2 * (S) + 1, KW>(kw[0], koff));               \
-    a[3] = lut(smem, pair_addr<KBM, 2 * (S) + 1, KW>(kw[1], koff));               \
+    a[0] = lut(pair_addr<KBM, 2 * (S), KW>(kw[0], koff));                         \
+    a[1] = lut(pair_addr<KBM, 2 * (S), KW>(kw[1], koff));                         \
+    a[2] = lut(pair_addr<KBM, 2 * (S) + 1, KW>(kw[0], koff));                     \
+    a[3] = lut(pair_addr<KBM, 2 * (S) + 1, KW>(kw[1], koff));                     \
     mma16816(cm, a, qf[S][0], qf[S][1]);                                          \
     if constexpr (!PACK) mma16816(cm, a, qf2[S][0], qf2[S][1]);                   \
   }
@@ -909,7 +961,7 @@ __global__ void __launch_bounds__((PACK && !KPROD ? 12 : 8) * 32, 1) decode_spli
           TQ_QSTEP(4) TQ_QSTEP(5) TQ_QSTEP(6) TQ_QSTEP(7)
 #undef TQ_QSTEP
         }
-        // s = n/s_K * (main + kappa gamma s_K qjl): the table holds s_K c
+        // raw score = main + kappa gamma s_K qjl (the table holds s_K c)
 #pragma unroll
         for (int i = 0; i < 4; ++i) {
           float s = cm[i];
@@ -920,11 +972,7 @@ __global__ void __launch_bounds__((PACK && !KPROD ? 12 : 8) * 32, 1) decode_spli
 #pragma unroll
         for (int r = 0; r < 2; ++r) {
 #pragma unroll
-          for (int c = 0; c < 2; ++c) {
-            const float s = cm[2 * r + c] * kn[r];
-            cm[2 * r + c] = s;
-            sc[ms][2 * r + c] = kn[r] >= 0.f ? s * p.scale_log2 : -INFINITY;
-          }
+          for (int c = 0; c < 2; ++c) sc[ms][2 * r + c] = ok[r] ? cm[2 * r + c] * fs[r] : -INFINITY;
         }
         if (want_scores) {
 #pragma unroll
@@ -932,9 +980,10 @@ __global__ void __launch_bounds__((PACK && !KPROD ? 12 : 8) * 32, 1) decode_spli
 #pragma unroll
             for (int c = 0; c < 2; ++c) {
               const int head = PACK ? 2 * (tig & 1) + c : 2 * tig + c;
-              if (kn[r] >= 0.f && head < gh && (!PACK || tig < 2)) {
-                const int64_t j = j0 + 16 * ms + 8 * r + g8;
-                p.scores[((int64_t)b * p.Hq + h0 + head) * p.seq_len + j] = cm[2 * r + c];
+              if (ok[r] && head < gh && (!PACK || tig < 2)) {
+                const int64_t j = t0 + (int64_t)ci * kChunk + 16 * ms + 8 * r + g8;
+                p.scores[((int64_t)b * p.Hq + h0 + head) * p.seq_len + j] =
+                    cm[2 * r + c] * (kb.kn[ms][r] * inv_sK);
               }
             }
           }
@@ -942,8 +991,12 @@ __global__ void __launch_bounds__((PACK && !KPROD ? 12 : 8) * 32, 1) decode_spli
       }
       // the key registers are free: start the next chunk's key loads
       if (more) {
-        if (fast_next) load_k<true>(kb, p, kbase + jn, vbase + jn, nvn, ro, tig, g8);
-        else load_k<false>(kb, p, kbase + jn * p.ksn, vbase + jn * p.vsn, nvn, ro, tig, g8);
+        if (fast_next) {
+          load_k_fast(kb, fp, cn);
+        } else {
+          const int64_t jn = t0 + (int64_t)cn * kChunk;
+          load_k_slow(kb, p, kbase + jn * p.ksn, vbase + jn * p.vsn, (int)min((int64_t)kChunk, t1 - jn), tig, g8);
+        }
       }
 
       // -------- online softmax, per head column c
@@ -994,16 +1047,21 @@ __global__ void __launch_bounds__((PACK && !KPROD ? 12 : 8) * 32, 1) decode_spli
 #pragma unroll
       for (int ms = 0; ms < 2; ++ms) {
         uint32_t b0, b1, b2 = 0u, b3 = 0u;
-        if constexpr (PACK) {
-          // lanes tig < 2 carry the hi halves (columns 0-3), tig >= 2 the lo
-          const bool lo = tig >= 2;
-          b0 = movmatrix_trans(lo ? pack_lo(wgt[ms][0], wgt[ms][1]) : pack_hi(wgt[ms][0], wgt[ms][1]));
-          b1 = movmatrix_trans(lo ? pack_lo(wgt[ms][2], wgt[ms][3]) : pack_hi(wgt[ms][2], wgt[ms][3]));
-        } else {
-          b0 = movmatrix_trans(pack_hi(wgt[ms][0], wgt[ms][1]));
-          b1 = movmatrix_trans(pack_hi(wgt[ms][2], wgt[ms][3]));
-          b2 = movmatrix_trans(pack_lo(wgt[ms][0], wgt[ms][1]));
-          b3 = movmatrix_trans(pack_lo(wgt[ms][2], wgt[ms][3]));
+        {
+          uint32_t h01, l01, h23, l23;
+          split_pair(wgt[ms][0], wgt[ms][1], h01, l01);
+          split_pair(wgt[ms][2], wgt[ms][3], h23, l23);
+          if constexpr (PACK) {
+            // lanes tig < 2 carry the hi halves (columns 0-3), tig >= 2 the lo
+            const bool lo = tig >= 2;
+            b0 = movmatrix_trans(lo ? l01 : h01);
+            b1 = movmatrix_trans(lo ? l23 : h23);
+          } else {
+            b0 = movmatrix_trans(h01);
+            b1 = movmatrix_trans(h23);
+            b2 = movmatrix_trans(l01);
+            b3 = movmatrix_trans(l23);
+          }
         }
         const auto &vw = vb.w[ms];
         if constexpr (VBM == 4) {
@@ -1021,10 +1079,10 @@ __global__ void __launch_bounds__((PACK && !KPROD ? 12 : 8) * 32, 1) decode_spli
 #define TQ_VSTEP4(MT)                                                             \
   {                                                                               \
     uint32_t a[4];                                                                \
-    a[0] = lut(smem, pair_addr<4, MT, 2>(x0[0], voff));                           \
-    a[1] = lut(smem, pair_addr<4, MT, 2>(x1[0], voff));                           \
-    a[2] = lut(smem, pair_addr<4, MT, 2>(x0[1], voff));                           \
-    a[3] = lut(smem, pair_addr<4, MT, 2>(x1[1], voff));                           \
+    a[0] = lut(pair_addr<4, MT, 2>(x0[0], voff));                           \
+    a[1] = lut(pair_addr<4, MT, 2>(x1[0], voff));                           \
+    a[2] = lut(pair_addr<4, MT, 2>(x0[1], voff));                           \
+    a[3] = lut(pair_addr<4, MT, 2>(x1[1], voff));                           \
     mma16816(acc[MT], a, b0, b1);                                                 \
     if constexpr (!PACK) mma16816(acc[MT], a, b2, b3);                            \
   }
@@ -1034,10 +1092,10 @@ __global__ void __launch_bounds__((PACK && !KPROD ? 12 : 8) * 32, 1) decode_spli
         } else {
 #define TQ_VSTEP(MT)                                                              \
   {                                                                               \
-    const uint32_t h0_ = lut(smem, pair_addr<VBM, MT, VW>(vw[0], voff));          \
-    const uint32_t h1_ = lut(smem, pair_addr<VBM, MT, VW>(vw[1], voff));          \
-    const uint32_t h2_ = lut(smem, pair_addr<VBM, MT, VW>(vw[2], voff));          \
-    const uint32_t h3_ = lut(smem, pair_addr<VBM, MT, VW>(vw[3], voff));          \
+    const uint32_t h0_ = lut(pair_addr<VBM, MT, VW>(vw[0], voff));          \
+    const uint32_t h1_ = lut(pair_addr<VBM, MT, VW>(vw[1], voff));          \
+    const uint32_t h2_ = lut(pair_addr<VBM, MT, VW>(vw[2], voff));          \
+    const uint32_t h3_ = lut(pair_addr<VBM, MT, VW>(vw[3], voff));          \
     uint32_t a[4];                                                                \
     a[0] = __byte_perm(h0_, h1_, 0x5410);                                         \
     a[1] = __byte_perm(h0_, h1_, 0x7632);                                         \
@@ -1053,8 +1111,12 @@ __global__ void __launch_bounds__((PACK && !KPROD ? 12 : 8) * 32, 1) decode_spli
       }
       // the value registers are free: start the next chunk's value loads
       if (more) {
-        if (fast_next) load_v<true>(vb, p, vbase + jn, nvn, ro, g8, tig);
-        else load_v<false>(vb, p, vbase + jn * p.vsn, nvn, ro, g8, tig);
+        if (fast_next) {
+          load_v_fast(vb, fp, cn, g8);
+        } else {
+          const int64_t jn = t0 + (int64_t)cn * kChunk;
+          load_v_slow(vb, p, vbase + jn * p.vsn, (int)min((int64_t)kChunk, t1 - jn), g8, tig);
+        }
       }
     }
 
@@ -1159,8 +1221,26 @@ __global__ void zero_out_kernel(float *out, int64_t n) {
   if (i < n) out[i] = 0.f;
 }
 
+// Dynamic shared memory: enough to reach kLutAddr + kLutBytes + the warps'
+// partials from any dynamic base at or above 0.
 constexpr size_t split_smem_bytes(int warps) {
-  return kLutBytes + 2 * 8 * kD * sizeof(float) + (size_t)warps * 8 * kPW * sizeof(float);
+  return (size_t)kLutAddr + kLutBytes + (size_t)warps * 8 * kPW * sizeof(float);
+}
+
+// Static shared memory plus the per-block reserve must end at or below
+// kLutAddr, where the dynamic region's pair tables start.
+template <typename K>
+cudaError_t check_smem_layout(K kern) {
+  cudaFuncAttributes fa;
+  cudaError_t e = cudaFuncGetAttributes(&fa, kern);
+  if (e != cudaSuccess) return e;
+  int dev = 0, reserved = 0;
+  e = cudaGetDevice(&dev);
+  if (e != cudaSuccess) return e;
+  e = cudaDeviceGetAttribute(&reserved, cudaDevAttrReservedSharedMemoryPerBlock, dev);
+  if (e != cudaSuccess) return e;
+  if ((size_t)reserved + fa.sharedSizeBytes > kLutAddr) return cudaErrorInvalidConfiguration;
+  return cudaSuccess;
 }
 
 template <int KBM, bool KPROD, int VBM, bool PACK>
@@ -1168,9 +1248,25 @@ cudaError_t run_split(const SplitParams &sp, cudaStream_t s) {
   auto kern = decode_split_kernel<KBM, KPROD, VBM, PACK>;
   const int warps = PACK && !KPROD ? 12 : 8;
   const size_t smem = split_smem_bytes(warps);
+  static const cudaError_t layout = check_smem_layout(kern);
+  if (layout != cudaSuccess) return layout;
   cudaError_t e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
   if (e != cudaSuccess) return e;
-  kern<<<sp.ctas, warps * 32, smem, s>>>(sp);
+  // programmatic dependent launch: the grid may start while the prep kernel
+  // before it in the stream is still running (the kernel waits for it with
+  // griddepcontrol.wait before touching the workspace)
+  cudaLaunchConfig_t cfg = {};
+  cfg.gridDim = dim3((unsigned)sp.ctas);
+  cfg.blockDim = dim3((unsigned)(warps * 32));
+  cfg.dynamicSmemBytes = smem;
+  cfg.stream = s;
+  cudaLaunchAttribute attr[1];
+  attr[0].id = cudaLaunchAttributeProgrammaticStreamSerialization;
+  attr[0].val.programmaticStreamSerializationAllowed = 1;
+  cfg.attrs = attr;
+  cfg.numAttrs = 1;
+  e = cudaLaunchKernelEx(&cfg, kern, sp);
+  if (e != cudaSuccess) return e;
   return cudaGetLastError();
 }
 
@@ -1200,7 +1296,8 @@ bool decode_supported(int d, int kbm, bool kprod, int vbm, bool vprod) {
 
 size_t decode_workspace_floats(int B, int Hq, int Hkv, bool prod, int ctas) {
   const int64_t units = (int64_t)B * Hkv * ((Hq / Hkv + 7) / 8);
-  return (size_t)kHdr + (size_t)B * Hq * kD * (prod ? 2 : 1) + (size_t)(units + ctas) * kSlot + (size_t)units;
+  (void)prod;  // the fragment block has room for the prod words either way
+  return (size_t)kHdr + (size_t)units * kFragWords + (size_t)(units + ctas) * kSlot + (size_t)units;
 }
 
 cudaError_t static_scratch(void **ptr) {
@@ -1270,14 +1367,16 @@ cudaError_t launch_decode(const DecodeArgs &a, cudaStream_t s) {
   sp.scale_log2 = a.scale * kLog2e;
   sp.scores = a.scores;
   sp.ws = a.ws;
-  sp.slot0 = (int64_t)kHdr + (int64_t)a.B * a.Hq * kD * (a.kq.prod ? 2 : 1);
   const int units = a.B * a.Hkv * sp.groups;
+  sp.frag = reinterpret_cast<const uint4 *>(a.ws + kHdr);
+  sp.slot0 = (int64_t)kHdr + (int64_t)units * kFragWords;
   sp.cnt = reinterpret_cast<unsigned *>(a.ws + sp.slot0 + (int64_t)(units + sp.ctas) * kSlot);
   sp.out = a.out;
   sp.vsign = a.vq.signs;
   PrepParams pp{a.q, a.q_dtype, a.B * a.Hq, a.kq.signs, a.kq.prod ? a.kq.S : nullptr,
                 a.kq.centroids, a.kq.bm, a.vq.centroids, a.vq.bm, a.ws, sp.cnt, units,
-                a.Hq, a.seq_len, a.seq_lens, a.out};
+                a.Hq, a.Hkv, sp.g, sp.groups, a.seq_len, a.seq_lens, a.out,
+                reinterpret_cast<uint32_t *>(a.ws + kHdr)};
   decode_prep_kernel<<<(a.B * a.Hq + 1) / 2 + 2, 256, 0, s>>>(pp);
   cudaError_t pe = cudaGetLastError();
   if (pe != cudaSuccess) return pe;

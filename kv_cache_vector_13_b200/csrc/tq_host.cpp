@@ -27,6 +27,7 @@
 
 #include <algorithm>
 #include <cmath>
+#include <cstdint>
 #include <cstdarg>
 #include <cstdio>
 #include <cstring>
@@ -379,6 +380,8 @@ tq_status tq_decode_attention(const tq_quantizer *kq, const tq_quantizer *vq, co
   if (q_dtype != TQ_F32 && q_dtype != TQ_BF16 && q_dtype != TQ_F16)
     return fail(TQ_EINVAL, "tq_decode_attention: q_dtype=%d", (int)q_dtype);
   if (B < 0 || Hq < 0 || Hkv < 0 || seq_len < 0) return fail(TQ_EINVAL, "tq_decode_attention: negative size");
+  if (seq_len > INT32_MAX)
+    return fail(TQ_EINVAL, "tq_decode_attention: seq_len=%lld is 2^31 or more", (long long)seq_len);
   if (Hkv == 0 || Hq % Hkv) return fail(TQ_EINVAL, "tq_decode_attention: Hq=%d not a multiple of Hkv=%d", Hq, Hkv);
   if (!std::isfinite(softmax_scale)) return fail(TQ_EINVAL, "tq_decode_attention: softmax_scale not finite");
   if (B == 0 || Hq == 0) return TQ_OK;
