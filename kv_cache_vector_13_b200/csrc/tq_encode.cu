@@ -19,6 +19,8 @@
 #include "tq_device.cuh"
 #include "tq_internal.h"
 
+#include <cuda_fp16.h>
+
 namespace tq {
 namespace {
 
@@ -79,54 +81,28 @@ __device__ __forceinline__ void store_bytes(uint8_t *dst, const uint32_t (&W)[NW
   }
 }
 
-template <int D, int BM, bool PROD, int DT, int EE>
-__global__ void __launch_bounds__(kEncThreads) encode_kernel(EncParams p) {
-  using Sh = Shape<D, EE>;
-  constexpr int T = Sh::T, E = Sh::E, VPB = Sh::VPB, RS = Sh::RS;
-  constexpr int K = 1 << BM;
-  constexpr int NWC = BM > 0 ? (E * BM + 31) / 32 : 1;  // code words per lane
-  constexpr int NWQ = (E + 31) / 32;                    // qjl words per lane
-
-  __shared__ uint32_t s_sign[D / 32];
-  __shared__ float s_cent[16];
-  extern __shared__ float4 s_dyn4[];
-  float *s_dyn = reinterpret_cast<float *>(s_dyn4);
-  float *s_r = s_dyn;                   // [VPB][RS] residuals (prod)
-  float *s_S = s_dyn + (size_t)VPB * RS;  // [D][RS] projection (prod, if it fits)
-
-  const int tid = threadIdx.x;
-  if (tid < 32) {  // sign bit masks, one ballot per 32 coordinates
+// Sign-flip masks (one ballot per 32 coordinates) into s_sign; the calling
+// block's first warp does it.
+template <int D>
+__device__ __forceinline__ void load_sign_masks(const int8_t *signs, uint32_t *s_sign, int tid) {
+  if (tid < 32) {
 #pragma unroll
     for (int w = 0; w < D / 32; ++w) {
-      const unsigned m = __ballot_sync(dev::kFull, p.signs[32 * w + tid] < 0);
+      const unsigned m = __ballot_sync(dev::kFull, signs[32 * w + tid] < 0);
       if (tid == 0) s_sign[w] = m;
     }
   }
-  if constexpr (PROD && BM > 0) {
-    if (tid < K) s_cent[tid] = p.cent[tid];
-  }
-  if constexpr (PROD && Sh::kSmemS) {
-    for (int i = tid; i < D * D; i += blockDim.x) s_S[(i / D) * RS + (i % D)] = p.S[i];
-  }
-  uint32_t P[K / 2 > 0 ? K / 2 : 1];
-#pragma unroll
-  for (int m = 0; m + 1 < K / 2; ++m) P[m] = __float_as_uint(__ldg(p.thr + K / 2 + m));
-  __syncthreads();
+}
 
-  const int t = tid % T;
-  const int vl = tid / T;
-  int64_t v = (int64_t)blockIdx.x * VPB + vl;
-  const bool active = v < p.nvec;
-  if (!active) v = p.nvec - 1;  // idle lanes still take part in the shuffles
-  const int64_t n = v % p.N;
-  const int64_t bh = v / p.N;
-  const int64_t h = bh % p.H;
-  const int64_t b = bh / p.H;
-  const int64_t xoff = b * p.xsb + h * p.xsh + n * p.xsn + (int64_t)t * E;
-  const int64_t rec = b * p.osb + h * p.osh + n * p.osn;
+// Per-vector front half, in the canonical fp32 order: load, norm (fold-halves
+// sum of squares, sqrt_rn), sign flips + unnormalised FWHT, scale by
+// fl(1 / fl(n * fl(sqrt d))), quantize and pack into W.  Returns the norm;
+// a[] ends as the residual (prod) or the scaled rotation (mse).
+template <int D, int BM, bool PROD, int DT, int T, int E, int NWC, int NP>
+__device__ __forceinline__ float encode_front(const EncParams &p, int64_t xoff, int t, const uint32_t *s_sign,
+                                              const float *s_cent, const uint32_t (&P)[NP], float (&a)[E],
+                                              uint32_t (&W)[NWC]) {
   constexpr int ES = DT == 0 ? 4 : 2;
-
-  float a[E];
   dev::load_block<DT, E>(static_cast<const char *>(p.x) + xoff * ES, a);
 
   // norm: fold-halves sum of squares, then sqrt_rn
@@ -151,7 +127,6 @@ __global__ void __launch_bounds__(kEncThreads) encode_kernel(EncParams p) {
   for (int i = 0; i < E; ++i) a[i] = __fmul_rn(a[i], inv);
 
   // quantize and pack; prod keeps the residual in a[]
-  uint32_t W[NWC];
 #pragma unroll
   for (int w = 0; w < NWC; ++w) W[w] = 0u;
   if constexpr (BM > 0) {
@@ -166,6 +141,54 @@ __global__ void __launch_bounds__(kEncThreads) encode_kernel(EncParams p) {
       dev::put_field<BM>(W, i, (uint32_t)idx);
       if constexpr (PROD) a[i] = __fsub_rn(a[i], s_cent[idx]);
     }
+  }
+  return nrm;
+}
+
+template <int D, int BM, bool PROD, int DT, int EE>
+__global__ void __launch_bounds__(kEncThreads) encode_kernel(EncParams p) {
+  using Sh = Shape<D, EE>;
+  constexpr int T = Sh::T, E = Sh::E, VPB = Sh::VPB, RS = Sh::RS;
+  constexpr int K = 1 << BM;
+  constexpr int NWC = BM > 0 ? (E * BM + 31) / 32 : 1;  // code words per lane
+  constexpr int NWQ = (E + 31) / 32;                    // qjl words per lane
+
+  __shared__ uint32_t s_sign[D / 32];
+  __shared__ float s_cent[16];
+  extern __shared__ float4 s_dyn4[];
+  float *s_dyn = reinterpret_cast<float *>(s_dyn4);
+  float *s_r = s_dyn;                   // [VPB][RS] residuals (prod)
+  float *s_S = s_dyn + (size_t)VPB * RS;  // [D][RS] projection (prod, if it fits)
+
+  const int tid = threadIdx.x;
+  load_sign_masks<D>(p.signs, s_sign, tid);
+  if constexpr (PROD && BM > 0) {
+    if (tid < K) s_cent[tid] = p.cent[tid];
+  }
+  if constexpr (PROD && Sh::kSmemS) {
+    for (int i = tid; i < D * D; i += blockDim.x) s_S[(i / D) * RS + (i % D)] = p.S[i];
+  }
+  uint32_t P[K / 2 > 0 ? K / 2 : 1];
+#pragma unroll
+  for (int m = 0; m + 1 < K / 2; ++m) P[m] = __float_as_uint(__ldg(p.thr + K / 2 + m));
+  __syncthreads();
+
+  const int t = tid % T;
+  const int vl = tid / T;
+  int64_t v = (int64_t)blockIdx.x * VPB + vl;
+  const bool active = v < p.nvec;
+  if (!active) v = p.nvec - 1;  // idle lanes still take part in the shuffles
+  const int64_t n = v % p.N;
+  const int64_t bh = v / p.N;
+  const int64_t h = bh % p.H;
+  const int64_t b = bh / p.H;
+  const int64_t xoff = b * p.xsb + h * p.xsh + n * p.xsn + (int64_t)t * E;
+  const int64_t rec = b * p.osb + h * p.osh + n * p.osn;
+
+  float a[E];
+  uint32_t W[NWC];
+  const float nrm = encode_front<D, BM, PROD, DT, T, E>(p, xoff, t, s_sign, s_cent, P, a, W);
+  if constexpr (BM > 0) {
     if (active) store_bytes<E * BM / 8>(p.codes + rec * (D * BM / 8) + t * (E * BM / 8), W);
   }
   if (active && t == 0) p.norms[rec] = nrm;
@@ -214,6 +237,231 @@ __global__ void __launch_bounds__(kEncThreads) encode_kernel(EncParams p) {
   }
 }
 
+// ------------------------------------------------ prod, d = 128: tensor cores
+//
+// The QJL projection z = S r is a dense 128 x 128 contraction per vector; for
+// a batch it is Z = R S^T, which runs here on mma.m16n8k16 (f16 x f16 ->
+// f32).  One warp owns 16 vectors (two lanes per vector in the front half),
+// exactly the M = 16 rows of an MMA tile.  Operands are split into fp16
+// halves, x = hi + lo with hi = fp16(x), lo = fp16(x - hi), and
+// z ~ Sh.rh + Sh.rl + Sl.rh (the dropped Sl.rl is below 2^-22 of
+// sum |S_ki r_i|).  Each residual row is first scaled by a power of two,
+// 2^(4 - floor(log2 ||r||)), which keeps both halves in fp16's normal range
+// and leaves every sign unchanged.  The representation, the dropped term
+// and fp32 accumulation over 24 MMA steps stay far below
+// theta_k = 2^-13 ||S_k|| ||r||; a projection with |z| <= theta_k (about
+// one in a thousand) is recomputed by a sequential fp32 dot product, so a
+// stored sign can differ from the exact one only where an fp32 summation's
+// sign could.  The block is persistent: it converts S to fp16 halves in
+// shared memory once and then walks tiles of 256 vectors.
+constexpr int kMmaThreads = 512;
+constexpr int kMmaVPB = kMmaThreads / 2;  // vectors per tile (two lanes each)
+constexpr int kSRow = 128 + 8;            // fp16 row of S halves (conflict-free B loads)
+constexpr int kRRow = 128 + 4;            // fp32 residual row (conflict-free A loads)
+
+constexpr size_t enc_mma_smem_bytes() {
+  return (size_t)2 * 128 * kSRow * 2 + (size_t)kMmaVPB * kRRow * 4;
+}
+
+__device__ __forceinline__ uint32_t h2_bits(__half2 h) { return *reinterpret_cast<const uint32_t *>(&h); }
+
+// fp16 (hi, lo) halves of the pair (x, y)
+__device__ __forceinline__ void split2(float x, float y, uint32_t &hi, uint32_t &lo) {
+  const __half2 h = __floats2half2_rn(x, y);
+  const float2 f = __half22float2(h);
+  hi = h2_bits(h);
+  lo = h2_bits(__floats2half2_rn(x - f.x, y - f.y));
+}
+
+__device__ __forceinline__ void mma_f16(float (&c)[4], const uint32_t (&a)[4], uint32_t b0, uint32_t b1) {
+  asm volatile(
+      "mma.sync.aligned.m16n8k16.row.col.f32.f16.f16.f32 {%0,%1,%2,%3}, {%4,%5,%6,%7}, {%8,%9}, "
+      "{%0,%1,%2,%3};\n"
+      : "+f"(c[0]), "+f"(c[1]), "+f"(c[2]), "+f"(c[3])
+      : "r"(a[0]), "r"(a[1]), "r"(a[2]), "r"(a[3]), "r"(b0), "r"(b1));
+}
+
+// bits 0..3 of x to bits 0, 2, 4, 6
+__device__ __forceinline__ uint32_t spread4(uint32_t x) {
+  x = (x | (x << 2)) & 0x33u;
+  return (x | (x << 1)) & 0x55u;
+}
+
+// sign of the fp32 dot product of one row of S (global) with a residual row
+__device__ __noinline__ bool qjl_recheck(const float *S_row, const float *r) {
+  float acc = 0.0f;
+  for (int i = 0; i < 128; ++i) acc = fmaf(__ldg(S_row + i), r[i], acc);
+  return acc >= 0.0f;
+}
+
+template <int BM, int DT>
+__global__ void __launch_bounds__(kMmaThreads, 1) encode_prod_mma_kernel(EncParams p, int64_t ntiles) {
+  constexpr int D = 128, T = 2, E = 64;
+  constexpr int K = 1 << BM;
+  constexpr int NWC = BM > 0 ? (E * BM + 31) / 32 : 1;
+
+  __shared__ uint32_t s_sign[D / 32];
+  __shared__ float s_cent[16];
+  __shared__ float s_snorm[D];
+  __shared__ float s_rs[kMmaVPB];  // per vector: scale of its residual row, theta factor
+  __shared__ float s_th[kMmaVPB];
+  extern __shared__ float4 s_dyn4[];
+  __half *s_sh = reinterpret_cast<__half *>(s_dyn4);          // [128][kSRow] hi(S)
+  __half *s_sl = s_sh + 128 * kSRow;                          // [128][kSRow] lo(S)
+  float *s_r = reinterpret_cast<float *>(s_sl + 128 * kSRow);  // [256][kRRow] residuals
+
+  const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
+  load_sign_masks<D>(p.signs, s_sign, tid);
+  if constexpr (BM > 0) {
+    if (tid < K) s_cent[tid] = p.cent[tid];
+  }
+  {  // S to fp16 halves, and its row norms: thread = (row, quarter of 32)
+    const int row = tid >> 2, q = tid & 3;
+    const float4 *src = reinterpret_cast<const float4 *>(p.S + row * D + 32 * q);
+    float ss = 0.0f;
+#pragma unroll
+    for (int i = 0; i < 8; ++i) {
+      const float4 v = __ldg(src + i);
+      uint32_t h0, l0, h1, l1;
+      split2(v.x, v.y, h0, l0);
+      split2(v.z, v.w, h1, l1);
+      const int k = 32 * q + 4 * i;
+      *reinterpret_cast<uint2 *>(s_sh + row * kSRow + k) = make_uint2(h0, h1);
+      *reinterpret_cast<uint2 *>(s_sl + row * kSRow + k) = make_uint2(l0, l1);
+      ss = fmaf(v.x, v.x, fmaf(v.y, v.y, fmaf(v.z, v.z, fmaf(v.w, v.w, ss))));
+    }
+    ss += __shfl_xor_sync(dev::kFull, ss, 1);
+    ss += __shfl_xor_sync(dev::kFull, ss, 2);
+    if (q == 0) s_snorm[row] = sqrtf(ss);
+  }
+  uint32_t P[K / 2 > 0 ? K / 2 : 1];
+#pragma unroll
+  for (int m = 0; m + 1 < K / 2; ++m) P[m] = __float_as_uint(__ldg(p.thr + K / 2 + m));
+  __syncthreads();
+
+  const int t = tid & 1, vl = tid >> 1;
+  const int g8 = lane >> 2, tig = lane & 3;
+  const float *rw = s_r + (size_t)(warp * 16) * kRRow;  // this warp's 16 residual rows
+  for (int64_t tile = blockIdx.x; tile < ntiles; tile += gridDim.x) {
+    int64_t v = tile * kMmaVPB + vl;
+    const bool active = v < p.nvec;
+    if (!active) v = p.nvec - 1;  // idle lanes still take part in the shuffles
+    const int64_t n = v % p.N;
+    const int64_t bh = v / p.N;
+    const int64_t h = bh % p.H;
+    const int64_t b = bh / p.H;
+    const int64_t xoff = b * p.xsb + h * p.xsh + n * p.xsn + (int64_t)t * E;
+    const int64_t rec = b * p.osb + h * p.osh + n * p.osn;
+
+    float a[E];
+    uint32_t W[NWC];
+    const float nrm = encode_front<D, BM, true, DT, T, E>(p, xoff, t, s_sign, s_cent, P, a, W);
+    if constexpr (BM > 0) {
+      if (active) store_bytes<E * BM / 8>(p.codes + rec * (D * BM / 8) + t * (E * BM / 8), W);
+    }
+    if (active && t == 0) p.norms[rec] = nrm;
+    float rr[E];
+#pragma unroll
+    for (int i = 0; i < E; ++i) rr[i] = __fmul_rn(a[i], a[i]);
+    const float gam = __fsqrt_rn(dev::fold_halves_sum<T, E>(rr));
+    float *rv = s_r + (size_t)vl * kRRow + t * E;
+#pragma unroll
+    for (int i = 0; i < E; i += 4) *reinterpret_cast<float4 *>(rv + i) = make_float4(a[i], a[i + 1], a[i + 2], a[i + 3]);
+    if (t == 0) {
+      // 2^(4 - floor(log2 gam)): |scaled r_i| <= 32; gam = 0 -> 1
+      const int ex = gam > 0.0f ? ((__float_as_int(gam) >> 23) & 0xff) - 127 : 0;
+      const float sc = __int_as_float((127 + min(4 - ex, 100)) << 23);
+      s_rs[vl] = sc;
+      s_th[vl] = gam * sc * 0x1p-13f;
+    }
+    __syncwarp();
+
+    // A fragments (16 vectors x 128 dims) as fp16 halves of the scaled rows
+    uint32_t ah[8][4], al[8][4];
+    const float sc0 = s_rs[warp * 16 + g8], sc1 = s_rs[warp * 16 + g8 + 8];
+    const float th0 = s_th[warp * 16 + g8], th1 = s_th[warp * 16 + g8 + 8];
+#pragma unroll
+    for (int ks = 0; ks < 8; ++ks) {
+      const int c = ks * 16 + 2 * tig;
+      const float2 r00 = *reinterpret_cast<const float2 *>(rw + g8 * kRRow + c);
+      const float2 r10 = *reinterpret_cast<const float2 *>(rw + (g8 + 8) * kRRow + c);
+      const float2 r01 = *reinterpret_cast<const float2 *>(rw + g8 * kRRow + c + 8);
+      const float2 r11 = *reinterpret_cast<const float2 *>(rw + (g8 + 8) * kRRow + c + 8);
+      split2(r00.x * sc0, r00.y * sc0, ah[ks][0], al[ks][0]);
+      split2(r10.x * sc1, r10.y * sc1, ah[ks][1], al[ks][1]);
+      split2(r01.x * sc0, r01.y * sc0, ah[ks][2], al[ks][2]);
+      split2(r11.x * sc1, r11.y * sc1, ah[ks][3], al[ks][3]);
+    }
+    uint32_t Q[2] = {0u, 0u};
+    const int v16 = lane >> 1;  // this lane's vector within the warp (front-half layout)
+#pragma unroll 1
+    for (int ng = 0; ng < 4; ++ng) {  // outputs [32 ng, 32 ng + 32)
+      float c[4][4];
+#pragma unroll
+      for (int j = 0; j < 4; ++j) c[j][0] = c[j][1] = c[j][2] = c[j][3] = 0.0f;
+#pragma unroll
+      for (int ks = 0; ks < 8; ++ks) {
+#pragma unroll
+        for (int j = 0; j < 4; ++j) {
+          const int row = (4 * ng + j) * 8 + g8;
+          const __half *ph = s_sh + row * kSRow + ks * 16 + 2 * tig;
+          const __half *pl = s_sl + row * kSRow + ks * 16 + 2 * tig;
+          const uint32_t bh0 = *reinterpret_cast<const uint32_t *>(ph);
+          const uint32_t bh1 = *reinterpret_cast<const uint32_t *>(ph + 8);
+          const uint32_t bl0 = *reinterpret_cast<const uint32_t *>(pl);
+          const uint32_t bl1 = *reinterpret_cast<const uint32_t *>(pl + 8);
+          mma_f16(c[j], ah[ks], bh0, bh1);
+          mma_f16(c[j], al[ks], bh0, bh1);
+          mma_f16(c[j], ah[ks], bl0, bl1);
+        }
+      }
+      // signs: C element e of tile j is (row g8 + 8 (e >> 1), output
+      // 8 (4 ng + j) + 2 tig + (e & 1))
+      uint32_t bal[4][4];
+#pragma unroll
+      for (int j = 0; j < 4; ++j) {
+#pragma unroll
+        for (int e = 0; e < 4; ++e) {
+          const int out = 8 * (4 * ng + j) + 2 * tig + (e & 1);
+          const int rl = g8 + 8 * (e >> 1);
+          const float z = c[j][e];
+          bool pos = z >= 0.0f;
+          if (!(fabsf(z) > (e >> 1 ? th1 : th0) * s_snorm[out])) pos = qjl_recheck(p.S + out * D, rw + rl * kRRow);
+          bal[j][e] = __ballot_sync(dev::kFull, pos);
+        }
+      }
+      // lane (v16, t) keeps outputs [64 t, 64 t + 64): groups 2t and 2t + 1
+      if ((ng >> 1) == t) {
+        const int e0 = v16 < 8 ? 0 : 2, sh = 4 * (v16 & 7);
+        uint32_t word = 0u;
+#pragma unroll
+        for (int j = 0; j < 4; ++j) {
+          const uint32_t ev = (bal[j][e0] >> sh) & 0xfu, od = (bal[j][e0 + 1] >> sh) & 0xfu;
+          word |= (spread4(ev) | (spread4(od) << 1)) << (8 * j);
+        }
+        Q[ng & 1] = word;
+      }
+    }
+    if (active) {
+      store_bytes<8>(p.qjl + rec * (D / 8) + t * 8, Q);
+      if (t == 0) p.rnorms[rec] = gam;
+    }
+    __syncwarp();  // this warp's residual rows are read before the next tile writes them
+  }
+}
+
+template <int BM, int DT>
+cudaError_t run_prod_mma(const EncParams &p, cudaStream_t s) {
+  auto kern = encode_prod_mma_kernel<BM, DT>;
+  const size_t smem = enc_mma_smem_bytes();
+  cudaError_t e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
+  if (e != cudaSuccess) return e;
+  const int64_t ntiles = (p.nvec + kMmaVPB - 1) / kMmaVPB;
+  const int64_t grid = ntiles < decode_ctas() ? ntiles : decode_ctas();
+  kern<<<(unsigned)grid, kMmaThreads, smem, s>>>(p, ntiles);
+  return cudaGetLastError();
+}
+
 template <int D, int BM, bool PROD, int DT, int EE>
 cudaError_t run_e(const EncodeArgs &a, cudaStream_t s) {
   using Sh = Shape<D, EE>;
@@ -237,6 +485,7 @@ cudaError_t run_e(const EncodeArgs &a, cudaStream_t s) {
   p.signs = a.q.signs;
   p.S = a.q.S;
   p.sqrt_d = a.q.sqrt_d;
+  if constexpr (PROD && D == 128 && EE == 64) return run_prod_mma<BM, DT>(p, s);
   const size_t smem = enc_smem_bytes<D, PROD, EE>();
   auto kern = encode_kernel<D, BM, PROD, DT, EE>;
   if (smem > 48 * 1024) {

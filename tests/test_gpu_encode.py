@@ -128,3 +128,24 @@ def test_zero_and_empty_inputs():
     empty = api.encode(qz, torch.zeros((0, 128), device=DEV))
     assert empty.norms.numel() == 0
     torch.cuda.synchronize()
+
+
+@pytest.mark.parametrize("dtype", [torch.float32, torch.bfloat16])
+@pytest.mark.parametrize("bits", [1, 2, 4])
+def test_encode_prod_large_batch_projection(dtype, bits):
+    # d = 128 prod batches of more than a wave take the tensor-core QJL
+    # projection; a ragged last tile, a zero row (zero residual for b = 1)
+    # and a tiny-norm row ride along.  Codes, norms and residual norms stay
+    # bit-exact; QJL signs may differ only inside the fp32 band.
+    d, n = 128, 3 * (1 << 13) + 37
+    x = inputs.unit_vectors(n, d, seed=bits, device=DEV)
+    x[5] = 0.0
+    x[6] *= 1e-30
+    x = x.to(dtype)
+    qz = api.Quantizer(d, bits, "prod", seed_rot=50 + bits, seed_qjl=60 + bits, device=DEV)
+    cache = api.encode(qz, x)
+    torch.cuda.synchronize()
+    oq = oracle_twin(qz)
+    enc = OQ.encode(oq, host(x))
+    nd = compare_records(qz, oq, enc, flat_host(cache))
+    assert nd <= max(2, 1e-6 * n * d)
