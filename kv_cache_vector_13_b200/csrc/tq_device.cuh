@@ -67,13 +67,15 @@ __device__ __forceinline__ void load_block(const void *p, float (&v)[E]) {
 // ------------------------------------------------------------ butterflies
 
 // One cross-lane FWHT stage: the lane whose group index has bit P clear holds
-// a (gets a+b), its partner holds b (gets a-b).
+// a (gets a+b), its partner holds b (gets a-b).  Both are one addition,
+// fl(o + a) on the low lane and fl(o + (-b)) = fl(o - b) on the high one.
 template <int E>
 __device__ __forceinline__ void fwht_cross(float (&a)[E], int P, bool low) {
+  const uint32_t neg = low ? 0u : 0x80000000u;
 #pragma unroll
   for (int i = 0; i < E; ++i) {
     const float o = __shfl_xor_sync(kFull, a[i], P);
-    a[i] = low ? __fadd_rn(a[i], o) : __fsub_rn(o, a[i]);
+    a[i] = __fadd_rn(o, __uint_as_float(__float_as_uint(a[i]) ^ neg));
   }
 }
 
@@ -149,7 +151,8 @@ __device__ __forceinline__ int quantize_sym(float u, const uint32_t (&P)[(1 << B
     const uint32_t t2 = (k & 4) ? hi : lo;
     k += A > t2 ? 1 : 0;
   }
-  return pos ? (K / 2 + k) : (K / 2 - 1 - k);
+  // K/2 + k for u > 0, K/2 - 1 - k otherwise (k < K/2)
+  return k ^ (pos ? K / 2 : K / 2 - 1);
 }
 
 // ----------------------------------------------------------- bit packing

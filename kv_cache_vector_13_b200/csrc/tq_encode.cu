@@ -40,7 +40,39 @@ struct EncParams {
   const int8_t *signs;
   const float *S;
   float sqrt_d;
+  // v -> (n, bh) and bh -> (h, b) by multiply-shift when every index fits
+  // in 31 bits (div32): q = (x * m) >> (31 + l) with l = ceil(log2 divisor),
+  // m = floor(2^(31+l) / divisor) + 1, exact for x < 2^31 (Granlund and
+  // Montgomery, "Division by invariant integers using multiplication").
+  bool div32;
+  uint32_t mN, mH;
+  int sN, sH;
 };
+
+// Vector index v -> (b, h, n) of a [B][H][N] batch.
+__device__ __forceinline__ void split_index(const EncParams &p, int64_t v, int64_t &b, int64_t &h, int64_t &n) {
+  if (p.div32) {
+    const uint32_t x = (uint32_t)v;
+    const uint32_t bh = (uint32_t)(((uint64_t)x * p.mN) >> p.sN);
+    const uint32_t hb = (uint32_t)(((uint64_t)bh * p.mH) >> p.sH);
+    n = x - bh * (uint32_t)p.N;
+    h = bh - hb * (uint32_t)p.H;
+    b = hb;
+  } else {
+    n = v % p.N;
+    const int64_t bh = v / p.N;
+    h = bh % p.H;
+    b = bh / p.H;
+  }
+}
+
+// Magic multiplier and shift for 31-bit dividends (see EncParams).
+inline void magic31(int64_t d, uint32_t &m, int &s) {
+  int l = 0;
+  while (((int64_t)1 << l) < d) ++l;
+  m = (uint32_t)((((uint64_t)1 << (31 + l)) / (uint64_t)d) + 1);
+  s = 31 + l;
+}
 
 template <int D, int EE = 64>
 struct Shape {
@@ -145,8 +177,11 @@ __device__ __forceinline__ float encode_front(const EncParams &p, int64_t xoff, 
   return nrm;
 }
 
+// The 64-coordinate layout is held to 3 resident blocks per SM (at most 85
+// registers a thread): more blocks in flight hide the load latency better
+// than the extra registers would help.
 template <int D, int BM, bool PROD, int DT, int EE>
-__global__ void __launch_bounds__(kEncThreads) encode_kernel(EncParams p) {
+__global__ void __launch_bounds__(kEncThreads, EE == 64 ? 3 : 1) encode_kernel(EncParams p) {
   using Sh = Shape<D, EE>;
   constexpr int T = Sh::T, E = Sh::E, VPB = Sh::VPB, RS = Sh::RS;
   constexpr int K = 1 << BM;
@@ -178,10 +213,8 @@ __global__ void __launch_bounds__(kEncThreads) encode_kernel(EncParams p) {
   int64_t v = (int64_t)blockIdx.x * VPB + vl;
   const bool active = v < p.nvec;
   if (!active) v = p.nvec - 1;  // idle lanes still take part in the shuffles
-  const int64_t n = v % p.N;
-  const int64_t bh = v / p.N;
-  const int64_t h = bh % p.H;
-  const int64_t b = bh / p.H;
+  int64_t b, h, n;
+  split_index(p, v, b, h, n);
   const int64_t xoff = b * p.xsb + h * p.xsh + n * p.xsn + (int64_t)t * E;
   const int64_t rec = b * p.osb + h * p.osh + n * p.osn;
 
@@ -346,10 +379,8 @@ __global__ void __launch_bounds__(kMmaThreads, 1) encode_prod_mma_kernel(EncPara
     int64_t v = tile * kMmaVPB + vl;
     const bool active = v < p.nvec;
     if (!active) v = p.nvec - 1;  // idle lanes still take part in the shuffles
-    const int64_t n = v % p.N;
-    const int64_t bh = v / p.N;
-    const int64_t h = bh % p.H;
-    const int64_t b = bh / p.H;
+    int64_t b, h, n;
+    split_index(p, v, b, h, n);
     const int64_t xoff = b * p.xsb + h * p.xsh + n * p.xsn + (int64_t)t * E;
     const int64_t rec = b * p.osb + h * p.osh + n * p.osn;
 
@@ -446,7 +477,10 @@ __global__ void __launch_bounds__(kMmaThreads, 1) encode_prod_mma_kernel(EncPara
       store_bytes<8>(p.qjl + rec * (D / 8) + t * 8, Q);
       if (t == 0) p.rnorms[rec] = gam;
     }
-    __syncwarp();  // this warp's residual rows are read before the next tile writes them
+    // keep the block's warps in step (they run the same long straight-line
+    // code, which then stays in the instruction cache); also orders this
+    // warp's residual-row reads before the next tile's writes
+    __syncthreads();
   }
 }
 
@@ -485,6 +519,13 @@ cudaError_t run_e(const EncodeArgs &a, cudaStream_t s) {
   p.signs = a.q.signs;
   p.S = a.q.S;
   p.sqrt_d = a.q.sqrt_d;
+  p.div32 = p.nvec < ((int64_t)1 << 31) && a.N > 0 && a.H > 0;
+  p.mN = p.mH = 0u;
+  p.sN = p.sH = 0;
+  if (p.div32) {
+    magic31(a.N, p.mN, p.sN);
+    magic31(a.H, p.mH, p.sH);
+  }
   if constexpr (PROD && D == 128 && EE == 64) return run_prod_mma<BM, DT>(p, s);
   const size_t smem = enc_smem_bytes<D, PROD, EE>();
   auto kern = encode_kernel<D, BM, PROD, DT, EE>;
