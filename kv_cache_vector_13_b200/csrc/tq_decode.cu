@@ -78,6 +78,10 @@ constexpr int kLutBytes = 256 * 256;     // K and V pair tables, per-lane copies
 // complete shared address of a lookup.
 constexpr uint32_t kLutAddr = 0x10000;
 constexpr int kPfWin = 4;                // chunks per L2 prefetch window
+// The PV weights' reference maximum M moves only when a chunk's maximum of
+// logit + log2 n_V passes it by more than kLazy (log2 units); the weights
+// then stay below 2^kLazy and most rescales of the accumulators are skipped.
+constexpr float kLazy = 8.0f;
 constexpr int kPW = kD + 4;              // floats per head in a partial: m, l, M, pad, o'[d]
 constexpr int kSlot = 8 * kPW;           // floats per partial slot (8 heads)
 constexpr int kScaleCands = 4096;
@@ -653,6 +657,10 @@ __device__ void merge_unit(const SplitParams &p, const int64_t *cuts, int u, int
                            int gh, int warp, int nwarps, int lane, float *s_m) {
   const int n = c1 - c0 + 1;
   const int parts = nwarps / gh;  // gh <= 8 <= nwarps
+  // the value rotation's signs for this lane's 4 dims, loaded alongside the
+  // slots (byte loads: the sign array carries no alignment promise)
+  const int8_t sg0 = p.vsign[lane * 4], sg1 = p.vsign[lane * 4 + 1];
+  const int8_t sg2 = p.vsign[lane * 4 + 2], sg3 = p.vsign[lane * 4 + 3];
   if (warp < gh * parts) {
     const int hh = warp % gh, part = warp / gh;
     const int i_lo = part * n / parts, i_hi = (part + 1) * n / parts;
@@ -729,8 +737,10 @@ __device__ void merge_unit(const SplitParams &p, const int64_t *cuts, int u, int
       for (int i = 0; i < 4; ++i) a[i] *= f;
       dev::fwht<32, 4>(a, lane);
       float o4[4];
-#pragma unroll
-      for (int i = 0; i < 4; ++i) o4[i] = p.vsign[lane * 4 + i] < 0 ? -a[i] : a[i];
+      o4[0] = sg0 < 0 ? -a[0] : a[0];
+      o4[1] = sg1 < 0 ? -a[1] : a[1];
+      o4[2] = sg2 < 0 ? -a[2] : a[2];
+      o4[3] = sg3 < 0 ? -a[3] : a[3];
       *reinterpret_cast<float4 *>(out) = make_float4(o4[0], o4[1], o4[2], o4[3]);
     }
   }
@@ -1013,7 +1023,8 @@ __global__ void __launch_bounds__((PACK && !KPROD ? 12 : 8) * 32, 1) decode_spli
           mx = fmaxf(mx, __shfl_xor_sync(dev::kFull, mx, o));
           Mx = fmaxf(Mx, __shfl_xor_sync(dev::kFull, Mx, o));
         }
-        const float mn = fmaxf(m_run[c], mx), Mn = fmaxf(M_run[c], Mx);
+        const float mn = fmaxf(m_run[c], mx);
+        const float Mn = Mx > M_run[c] + kLazy ? Mx : M_run[c];
         const float ms_ = mn == -INFINITY ? 0.f : mn;
         const float Ms_ = Mn == -INFINITY ? 0.f : Mn;
         const float al = ex2(m_run[c] - ms_);
