@@ -280,12 +280,14 @@ __global__ void __launch_bounds__(kEncThreads, EE == 64 ? 3 : 1) encode_kernel(E
 // z ~ Sh.rh + Sh.rl + Sl.rh (the dropped Sl.rl is below 2^-22 of
 // sum |S_ki r_i|).  Each residual row is first scaled by a power of two,
 // 2^(4 - floor(log2 ||r||)), which keeps both halves in fp16's normal range
-// and leaves every sign unchanged.  The representation, the dropped term
-// and fp32 accumulation over 24 MMA steps stay far below
-// theta_k = 2^-13 ||S_k|| ||r||; a projection with |z| <= theta_k (about
-// one in a thousand) is recomputed by a sequential fp32 dot product, so a
-// stored sign can differ from the exact one only where an fp32 summation's
-// sign could.  The block is persistent: it converts S to fp16 halves in
+// and leaves every sign unchanged.  The representation (about 3 * 2^-22
+// per product), the dropped term and the fp32 accumulation over 24 MMA
+// steps (at most 24 * 2^-23 of sum |S_ki r_i|) stay below 2^-17.4
+// sum |S_ki r_i| <= 2^-17.4 ||S_k|| ||r||, a fifth of
+// theta_k = 2^-15 ||S_k|| ||r||; a projection with |z| <= theta_k (about
+// three in ten thousand) is recomputed by an fp32 dot product, so a stored
+// sign can differ from the exact one only where an fp32 summation's sign
+// could.  The block is persistent: it converts S to fp16 halves in
 // shared memory once and then walks tiles of 256 vectors.
 constexpr int kMmaThreads = 512;
 constexpr int kMmaVPB = kMmaThreads / 2;  // vectors per tile (two lanes each)
@@ -320,10 +322,20 @@ __device__ __forceinline__ uint32_t spread4(uint32_t x) {
   return (x | (x << 1)) & 0x55u;
 }
 
-// sign of the fp32 dot product of one row of S (global) with a residual row
+// sign of the fp32 dot product of one row of S (global, 16-byte aligned)
+// with a residual row (shared, 16-byte aligned)
 __device__ __noinline__ bool qjl_recheck(const float *S_row, const float *r) {
+  const float4 *s4 = reinterpret_cast<const float4 *>(S_row);
+  const float4 *r4 = reinterpret_cast<const float4 *>(r);
   float acc = 0.0f;
-  for (int i = 0; i < 128; ++i) acc = fmaf(__ldg(S_row + i), r[i], acc);
+#pragma unroll 8
+  for (int i = 0; i < 32; ++i) {
+    const float4 a = __ldg(s4 + i), b = r4[i];
+    acc = fmaf(a.x, b.x, acc);
+    acc = fmaf(a.y, b.y, acc);
+    acc = fmaf(a.z, b.z, acc);
+    acc = fmaf(a.w, b.w, acc);
+  }
   return acc >= 0.0f;
 }
 
@@ -403,7 +415,7 @@ __global__ void __launch_bounds__(kMmaThreads, 1) encode_prod_mma_kernel(EncPara
       const int ex = gam > 0.0f ? ((__float_as_int(gam) >> 23) & 0xff) - 127 : 0;
       const float sc = __int_as_float((127 + min(4 - ex, 100)) << 23);
       s_rs[vl] = sc;
-      s_th[vl] = gam * sc * 0x1p-13f;
+      s_th[vl] = gam * sc * 0x1p-15f;
     }
     __syncwarp();
 
