@@ -41,6 +41,17 @@ B, HQ, HKV, D, N = 1, 32, 8, 128, 32768
 KBITS, VBITS = 4, 4
 COPIES = 8
 FALLBACK_PEAKS = {"hbm_gbs": 6650.0, "bf16_tflops": 1590.0}
+# DRAM bytes (read + write) of one decode split-kernel launch on this
+# workload, from an ncu capture (dram__bytes_read.sum + dram__bytes_write.sum),
+# reported only while the decode source is the one it was taken on.
+TRAFFIC = {"bytes": 35772928, "source_sha256": "ce6c36e98f5cd495c969de6fc44d3661d6721aaf2b0fb42b437bdbedd1e46645"}
+
+
+def traffic_bytes():
+    import hashlib
+    with open(os.path.join(ROOT, "kv_cache_vector_13_b200", "csrc", "tq_decode.cu"), "rb") as f:
+        h = hashlib.sha256(f.read()).hexdigest()
+    return TRAFFIC["bytes"] if h == TRAFFIC["source_sha256"] else None
 
 
 def peaks():
@@ -99,7 +110,10 @@ class ClockSampler:
                 "reasons": reasons, "samples": len(rows)}
 
 
-def dist_setup():
+def dist_setup(backend="nccl"):
+    """(rank, local rank, world size) from the torchrun environment; joins the
+    process group when there is more than one rank (short timeout, so ranks
+    that wait on a missing peer end with an error)."""
     ws = int(os.environ.get("WORLD_SIZE", "1"))
     if ws == 1:
         return 0, 0, 1
@@ -107,8 +121,25 @@ def dist_setup():
     import torch.distributed as dist
     rank = int(os.environ["RANK"])
     local = int(os.environ.get("LOCAL_RANK", rank))
-    dist.init_process_group("nccl", timeout=datetime.timedelta(seconds=120), device_id=None)
+    dist.init_process_group(backend, timeout=datetime.timedelta(seconds=120), device_id=None)
     return rank, local, ws
+
+
+def max_over_ranks(times, dist, device):
+    """Element-wise maximum of a list of times over all ranks (every rank
+    gets the result); the identity without a process group."""
+    if dist is None:
+        return list(times)
+    import torch
+    tt = torch.tensor(times, device=device, dtype=torch.float64)
+    dist.all_reduce(tt, op=dist.ReduceOp.MAX)
+    return tt.tolist()
+
+
+def job_value(world_size, ms_per_step):
+    """Whole-job KV-tokens/s: every rank decodes B * N tokens per step, and
+    the job's step time is the slowest rank's."""
+    return world_size * B * N / (ms_per_step * 1e-3)
 
 
 # ------------------------------------------------------------------ our leg
@@ -224,14 +255,9 @@ def run_ours(args):
     e2e_s = time.perf_counter() - t0
     barrier()
 
-    times = [t_ms, dec_ms, e2e_s]
-    if dist is not None:
-        tt = torch.tensor(times, device=dev, dtype=torch.float64)
-        dist.all_reduce(tt, op=dist.ReduceOp.MAX)
-        times = tt.tolist()
-    t_ms, dec_ms, e2e_s = times
+    t_ms, dec_ms, e2e_s = max_over_ranks([t_ms, dec_ms, e2e_s], dist, dev)
 
-    enc_info = bench_encode(api, inputs, torch, dev, stream) if rank == 0 else None
+    enc_info = bench_encode(api, inputs, torch, dev, stream, args.encode_variant) if rank == 0 else None
     base = None
     if rank == 0 and not args.no_cpu_baseline:
         base = cpu_baseline_decode(budget_s=args.cpu_seconds)
@@ -240,7 +266,7 @@ def run_ours(args):
         dec_bytes = B * HKV * N * (kq.record_bytes + vq.record_bytes) + q.numel() * 2 + B * HQ * D * 4
         achieved = dec_bytes / (dec_ms * 1e-3) / 1e9
         ms_step = t_ms / K_steps
-        val = ws * B * N / (ms_step * 1e-3)
+        val = job_value(ws, ms_step)
         line = {
             "metric": METRIC, "value": val, "unit": "KV-tokens/s", "n_gpus": ws, "steps": K_steps,
             "warmup": max(args.warmup, 3), "ms_per_step": ms_step, "higher_is_better": True,
@@ -254,7 +280,7 @@ def run_ours(args):
                          "achieved": achieved, "peak": pk["hbm_gbs"], "unit": "GB/s",
                          "frac": achieved / pk["hbm_gbs"], "peak_kind": pk_kind,
                          "bytes_per_launch": dec_bytes, "ms_per_launch": dec_ms,
-                         "traffic": args.traffic},
+                         "traffic": args.traffic if args.traffic is not None else traffic_bytes()},
             "encode": enc_info,
             "cpu_baseline": base,
             "e2e": {"value": ws * B * N * e2e_steps / e2e_s, "unit": "KV-tokens/s",
@@ -270,11 +296,15 @@ def run_ours(args):
         dist.destroy_process_group()
 
 
-def bench_encode(api, inputs, torch, dev, stream):
-    """Encode throughput: 2^20 unit vectors, d=128, TurboQuant_mse b=4, fp32
-    input (the encode sweep's d=128 cell), 4 rotating input copies > L2."""
+def bench_encode(api, inputs, torch, dev, stream, variant="mse4"):
+    """Encode throughput: 2^20 unit vectors, d=128, fp32 input (the encode
+    sweep's d=128 cell), TurboQuant_mse b=4 (or TurboQuant_prod b=3 with
+    variant="prod3"), 2 rotating input copies (1 GB > L2)."""
     n, d = 1 << 20, 128
-    qz = api.Quantizer(d, 4, "mse", seed_rot=0, device=dev)
+    if variant == "prod3":
+        qz = api.Quantizer(d, 3, "prod", seed_rot=0, seed_qjl=1, device=dev)
+    else:
+        qz = api.Quantizer(d, 4, "mse", seed_rot=0, device=dev)
     xs = [inputs.unit_vectors(n, d, seed=i, device=dev) for i in range(2)]
     outs = [api.empty_cache(qz, 1, 1, n, dev) for _ in range(2)]
     with torch.cuda.stream(stream):
@@ -292,7 +322,8 @@ def bench_encode(api, inputs, torch, dev, stream):
     byts = n * (d * 4 + qz.record_bytes)
     pk, _ = peaks()
     gbs = byts / (ms * 1e-3) / 1e9
-    return {"workload": "2^20 unit vectors d=128 fp32, TurboQuant_mse b=4", "vectors_per_s": n / (ms * 1e-3),
+    name = "TurboQuant_prod b=3" if variant == "prod3" else "TurboQuant_mse b=4"
+    return {"workload": f"2^20 unit vectors d=128 fp32, {name}", "vectors_per_s": n / (ms * 1e-3),
             "ms_per_launch": ms, "bytes_per_launch": byts, "achieved_gbs": gbs, "frac": gbs / pk["hbm_gbs"]}
 
 
@@ -379,6 +410,8 @@ def main():
     ap.add_argument("--ref-steps", type=int, default=0)
     ap.add_argument("--traffic", type=float, default=None,
                     help="dram bytes per decode call from an ncu capture of this build, if any")
+    ap.add_argument("--encode-variant", default="mse4", choices=["mse4", "prod3"],
+                    help="codec of the encode-throughput measurement")
     args = ap.parse_args()
     if args.impl == "reference":
         run_reference(args)
