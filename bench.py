@@ -5,11 +5,12 @@ metric is quoted on): batch 1, 32 query heads / 8 KV heads, head_dim 128,
 32768 cached tokens; K and V are bf16 N(0,1) times a per-(head, channel)
 LogNormal(0, 0.5) scale, compressed with TurboQuant_mse b=4.
 
-A step is the whole hot path for one new token: encode the new token's K and
-V (norm, sign flips + FWHT, Lloyd-Max indices, bit-packing) into the cache
-tail, then decode attention over all 32768 packed tokens (query rotation,
-scores from the codes, online softmax, PV in the rotated basis, split merge,
-one inverse rotation).  value = KV-tokens/s = B * N / step time.
+A step is the whole hot path for one new token, one tq_append_decode_attention
+call: encode the new token's K and V (norm, sign flips + FWHT, Lloyd-Max
+indices, bit-packing) into the cache tail, then decode attention over all
+32768 packed tokens (query rotation, scores from the codes, online softmax, PV
+in the rotated basis, split merge, one inverse rotation).  value =
+KV-tokens/s = B * N / step time.
 
 The cache is replicated 8x (8 x 35.7 MB > 126 MB L2) and step s uses copy
 s % 8, so every step streams its cache from HBM.  Steps are replayed from a
@@ -180,10 +181,13 @@ def run_ours(args):
     stream = torch.cuda.Stream(device=dev)
 
     def step(c, decode_only=False):
-        if not decode_only:
-            api.encode(kq, k_new, out=tails[c][0], stream=stream)
-            api.encode(vq, v_new, out=tails[c][1], stream=stream)
-        op(q, kcs[c], vcs[c], stream=stream)
+        # one decode step: tq_append_decode_attention encodes the new token's
+        # K and V into the cache tail and attends over the cache (four
+        # kernels, each allowed to start while the one before it finishes)
+        if decode_only:
+            op(q, kcs[c], vcs[c], stream=stream)
+        else:
+            op.append_step(q, k_new, v_new, tails[c][0], tails[c][1], kcs[c], vcs[c], stream=stream)
 
     with torch.cuda.stream(stream):
         for s in range(max(args.warmup, 3)):

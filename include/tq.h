@@ -175,6 +175,33 @@ tq_status tq_decode_attention(const tq_quantizer *kq, const tq_quantizer *vq,
                               float *out, float *scores_out, void *workspace,
                               size_t workspace_bytes, tq_stream_t stream);
 
+/* One decode step: compress the new token's key and value into the cache,
+ * then attend over the cache ("I Spent 31 Hours On The Math Behind
+ * Turboquant", section "KV Cache: The problem": each generated token appends
+ * its K and V, and the next query attends over all of them).
+ * Equivalent to tq_encode(kq, k_new -> k_tail), tq_encode(vq, v_new ->
+ * v_tail), then tq_decode_attention(...) with the remaining arguments, with
+ * identical results, as one call: the four kernels run as a chain in which
+ * each may start while the one before it finishes.
+ *   k_new, v_new: [B][Hkv][d] (kv_dtype, DEVICE), element strides
+ *                 new_stride_b, new_stride_h (16-byte multiples), unit stride
+ *                 along d.
+ *   k_tail, v_tail: views of the B x Hkv records that receive them (usually
+ *                 token L_b - 1 of k and v, so the new token is attended).
+ *   The rest as for tq_decode_attention.  All arguments are validated before
+ *   any launch.  The chain's first kernel starts after everything already in
+ *   the stream, like any launch; inputs must not be written by later work
+ *   until the call's work completes. */
+tq_status tq_append_decode_attention(const tq_quantizer *kq, const tq_quantizer *vq,
+                                     const void *k_new, const void *v_new, tq_dtype kv_dtype,
+                                     int64_t new_stride_b, int64_t new_stride_h,
+                                     const tq_cache_view *k_tail, const tq_cache_view *v_tail,
+                                     const void *q, tq_dtype q_dtype, int32_t B, int32_t Hq,
+                                     int32_t Hkv, int64_t seq_len, const int32_t *seq_lens,
+                                     const tq_cache_view *k, const tq_cache_view *v,
+                                     float softmax_scale, float *out, float *scores_out,
+                                     void *workspace, size_t workspace_bytes, tq_stream_t stream);
+
 /* Decode attention without a caller workspace.  The pages have no
  * counterpart to this call: it exists for callers that cannot allocate
  * device memory at run time, such as a plugin whose enqueue runs inside

@@ -21,7 +21,7 @@ TQ_NOALLOC_SCRATCH_BYTES = 16 << 20  # include/tq.h
 EXPORTS = (
     "tq_make_codebook", "tq_make_signs", "tq_make_qjl", "tq_code_bytes", "tq_qjl_bytes",
     "tq_encode", "tq_dequant", "tq_decode_workspace_bytes", "tq_decode_attention",
-    "tq_decode_attention_noalloc",
+    "tq_append_decode_attention", "tq_decode_attention_noalloc",
     "tq_check", "tq_status_string", "tq_last_error", "tq_version",
 )
 
@@ -81,6 +81,12 @@ def lib() -> ctypes.CDLL:
         c_int64, c_void_p, POINTER(TqCacheView), POINTER(TqCacheView), c_float, c_void_p, c_void_p,
         c_void_p, c_size_t, c_void_p]
     L.tq_decode_attention.restype = c_int32
+    L.tq_append_decode_attention.argtypes = [
+        POINTER(TqQuantizer), POINTER(TqQuantizer), c_void_p, c_void_p, c_int32, c_int64, c_int64,
+        POINTER(TqCacheView), POINTER(TqCacheView), c_void_p, c_int32, c_int32, c_int32, c_int32, c_int64,
+        c_void_p, POINTER(TqCacheView), POINTER(TqCacheView), c_float, c_void_p, c_void_p, c_void_p, c_size_t,
+        c_void_p]
+    L.tq_append_decode_attention.restype = c_int32
     L.tq_decode_attention_noalloc.argtypes = [
         POINTER(TqQuantizer), POINTER(TqQuantizer), c_void_p, c_int32, c_int32, c_int32, c_int32,
         c_int64, c_void_p, POINTER(TqCacheView), POINTER(TqCacheView), c_float, c_void_p, c_void_p,

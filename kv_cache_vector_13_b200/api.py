@@ -203,6 +203,35 @@ class DecodeAttention:
             out.data_ptr(), _ptr(scores), self.workspace.data_ptr(), self.ws_bytes, _stream(stream)))
         return out
 
+    def append_step(self, q: torch.Tensor, k_new: torch.Tensor, v_new: torch.Tensor, k_tail: PackedCache,
+                    v_tail: PackedCache, kcache: PackedCache, vcache: PackedCache, scale: Optional[float] = None,
+                    seq_lens: Optional[torch.Tensor] = None, scores: Optional[torch.Tensor] = None,
+                    out: Optional[torch.Tensor] = None, stream=None) -> torch.Tensor:
+        """tq_append_decode_attention: encode the new token's K and V
+        ([B, Hkv, d] or [B, Hkv, 1, d], same dtype) into the tail records
+        k_tail / v_tail ([B, Hkv, 1] views, usually the last token of
+        kcache / vcache), then attend over kcache / vcache."""
+        B, Hq, d = q.shape
+        assert (B, Hq) == (self.B, self.Hq) and q.is_contiguous() and q.dtype in _DTYPES
+        if k_new.dim() == 4:
+            k_new, v_new = k_new[:, :, 0], v_new[:, :, 0]
+        assert k_new.shape == (B, self.Hkv, d) and v_new.shape == k_new.shape
+        assert k_new.dtype == v_new.dtype and k_new.dtype in _DTYPES
+        assert k_new.stride() == v_new.stride() and k_new.stride(2) == 1
+        if scale is None:
+            scale = 1.0 / math.sqrt(d)
+        out = self.out if out is None else out
+        kv, vv, kt, vt = kcache.view(), vcache.view(), k_tail.view(), v_tail.view()
+        if seq_lens is not None:
+            assert seq_lens.dtype == torch.int32 and seq_lens.is_contiguous()
+        L.check(L.lib().tq_append_decode_attention(
+            ctypes.byref(self.kq.c_struct()), ctypes.byref(self.vq.c_struct()), k_new.data_ptr(), v_new.data_ptr(),
+            _DTYPES[k_new.dtype], k_new.stride(0), k_new.stride(1), ctypes.byref(kt), ctypes.byref(vt),
+            q.data_ptr(), _DTYPES[q.dtype], B, Hq, self.Hkv, self.seq_len, _ptr(seq_lens), ctypes.byref(kv),
+            ctypes.byref(vv), float(scale), out.data_ptr(), _ptr(scores), self.workspace.data_ptr(), self.ws_bytes,
+            _stream(stream)))
+        return out
+
 
 def decode_attention(kq: Quantizer, vq: Quantizer, q: torch.Tensor, kcache: PackedCache, vcache: PackedCache,
                      scale: Optional[float] = None, seq_lens: Optional[torch.Tensor] = None,

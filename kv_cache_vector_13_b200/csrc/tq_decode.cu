@@ -478,6 +478,12 @@ __global__ void __launch_bounds__(256) decode_prep_kernel(PrepParams p) {
       put(ln, 32 + w, lo ? pack_lo(sv[e], sv[e + 16]) : pack_hi(sv[e], sv[e + 16]));
     }
   }
+  // When this grid was launched early after the new tokens' encode (the
+  // fused append + decode chain), one thread waits for that grid, so this
+  // grid completes after it and the split kernel's wait covers both.  Head 0
+  // (block 0, thread 0) always reaches this point.  Without such a launch
+  // the wait returns at once.
+  if (blockIdx.x == 0 && threadIdx.x == 0) asm volatile("griddepcontrol.wait;\n" ::: "memory");
 }
 
 // ------------------------------------------------------------ split kernel
@@ -1388,8 +1394,21 @@ cudaError_t launch_decode(const DecodeArgs &a, cudaStream_t s) {
                 a.kq.centroids, a.kq.bm, a.vq.centroids, a.vq.bm, a.ws, sp.cnt, units,
                 a.Hq, a.Hkv, sp.g, sp.groups, a.seq_len, a.seq_lens, a.out,
                 reinterpret_cast<uint32_t *>(a.ws + kHdr)};
-  decode_prep_kernel<<<(a.B * a.Hq + 1) / 2 + 2, 256, 0, s>>>(pp);
-  cudaError_t pe = cudaGetLastError();
+  cudaError_t pe;
+  {
+    cudaLaunchConfig_t cfg = {};
+    cfg.gridDim = dim3((unsigned)((a.B * a.Hq + 1) / 2 + 2));
+    cfg.blockDim = dim3(256);
+    cfg.stream = s;
+    cudaLaunchAttribute attr[1];
+    attr[0].id = cudaLaunchAttributeProgrammaticStreamSerialization;
+    attr[0].val.programmaticStreamSerializationAllowed = a.prep_pdl ? 1 : 0;
+    cfg.attrs = attr;
+    cfg.numAttrs = 1;
+    pe = cudaLaunchKernelEx(&cfg, decode_prep_kernel, pp);
+  }
+  if (pe != cudaSuccess) return pe;
+  pe = cudaGetLastError();
   if (pe != cudaSuccess) return pe;
   const bool pack = sp.g <= 4;
   cudaError_t e = cudaErrorInvalidValue;

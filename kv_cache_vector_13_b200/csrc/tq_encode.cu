@@ -47,7 +47,17 @@ struct EncParams {
   bool div32;
   uint32_t mN, mH;
   int sN, sH;
+  bool pdl;  // launched programmatically after the kernel before it
 };
+
+// Programmatic dependent launch.  Every encode grid lets the next kernel in
+// the stream start early; a grid that was itself launched early (pdl) keeps
+// one thread waiting for the grid before it, so it cannot complete first and
+// a chain of such grids completes in stream order.
+__device__ __forceinline__ void pdl_open() { asm volatile("griddepcontrol.launch_dependents;\n" ::: "memory"); }
+__device__ __forceinline__ void pdl_close(bool pdl) {
+  if (pdl && blockIdx.x == 0 && threadIdx.x == 0) asm volatile("griddepcontrol.wait;\n" ::: "memory");
+}
 
 // Vector index v -> (b, h, n) of a [B][H][N] batch.
 __device__ __forceinline__ void split_index(const EncParams &p, int64_t v, int64_t &b, int64_t &h, int64_t &n) {
@@ -196,6 +206,7 @@ __global__ void __launch_bounds__(kEncThreads, EE == 64 ? 3 : 1) encode_kernel(E
   float *s_S = s_dyn + (size_t)VPB * RS;  // [D][RS] projection (prod, if it fits)
 
   const int tid = threadIdx.x;
+  pdl_open();
   load_sign_masks<D>(p.signs, s_sign, tid);
   if constexpr (PROD && BM > 0) {
     if (tid < K) s_cent[tid] = p.cent[tid];
@@ -268,6 +279,7 @@ __global__ void __launch_bounds__(kEncThreads, EE == 64 ? 3 : 1) encode_kernel(E
       if (t == 0) p.rnorms[rec] = gam;
     }
   }
+  pdl_close(p.pdl);
 }
 
 // ------------------------------------------------ prod, d = 128: tensor cores
@@ -356,6 +368,7 @@ __global__ void __launch_bounds__(kMmaThreads, 1) encode_prod_mma_kernel(EncPara
   float *s_r = reinterpret_cast<float *>(s_sl + 128 * kSRow);  // [256][kRRow] residuals
 
   const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
+  pdl_open();
   load_sign_masks<D>(p.signs, s_sign, tid);
   if constexpr (BM > 0) {
     if (tid < K) s_cent[tid] = p.cent[tid];
@@ -494,6 +507,23 @@ __global__ void __launch_bounds__(kMmaThreads, 1) encode_prod_mma_kernel(EncPara
     // warp's residual-row reads before the next tile's writes
     __syncthreads();
   }
+  pdl_close(p.pdl);
+}
+
+// A launch, with programmatic stream serialization when pdl is set.
+template <typename K, typename... Args>
+cudaError_t launch_maybe_pdl(K kern, dim3 grid, dim3 block, size_t smem, cudaStream_t s, bool pdl, Args... args) {
+  cudaLaunchConfig_t cfg = {};
+  cfg.gridDim = grid;
+  cfg.blockDim = block;
+  cfg.dynamicSmemBytes = smem;
+  cfg.stream = s;
+  cudaLaunchAttribute attr[1];
+  attr[0].id = cudaLaunchAttributeProgrammaticStreamSerialization;
+  attr[0].val.programmaticStreamSerializationAllowed = pdl ? 1 : 0;
+  cfg.attrs = attr;
+  cfg.numAttrs = 1;
+  return cudaLaunchKernelEx(&cfg, kern, args...);
 }
 
 template <int BM, int DT>
@@ -504,7 +534,8 @@ cudaError_t run_prod_mma(const EncParams &p, cudaStream_t s) {
   if (e != cudaSuccess) return e;
   const int64_t ntiles = (p.nvec + kMmaVPB - 1) / kMmaVPB;
   const int64_t grid = ntiles < decode_ctas() ? ntiles : decode_ctas();
-  kern<<<(unsigned)grid, kMmaThreads, smem, s>>>(p, ntiles);
+  e = launch_maybe_pdl(kern, dim3((unsigned)grid), dim3(kMmaThreads), smem, s, p.pdl, p, ntiles);
+  if (e != cudaSuccess) return e;
   return cudaGetLastError();
 }
 
@@ -531,6 +562,7 @@ cudaError_t run_e(const EncodeArgs &a, cudaStream_t s) {
   p.signs = a.q.signs;
   p.S = a.q.S;
   p.sqrt_d = a.q.sqrt_d;
+  p.pdl = a.pdl;
   p.div32 = p.nvec < ((int64_t)1 << 31) && a.N > 0 && a.H > 0;
   p.mN = p.mH = 0u;
   p.sN = p.sH = 0;
@@ -546,7 +578,8 @@ cudaError_t run_e(const EncodeArgs &a, cudaStream_t s) {
     if (e != cudaSuccess) return e;
   }
   const int64_t blocks = (p.nvec + Sh::VPB - 1) / Sh::VPB;
-  kern<<<(unsigned)blocks, kEncThreads, smem, s>>>(p);
+  const cudaError_t e = launch_maybe_pdl(kern, dim3((unsigned)blocks), dim3(kEncThreads), smem, s, p.pdl, p);
+  if (e != cudaSuccess) return e;
   return cudaGetLastError();
 }
 

@@ -305,35 +305,59 @@ size_t tq_code_bytes(int32_t d, int32_t bits, int32_t variant) {
 
 size_t tq_qjl_bytes(int32_t d, int32_t variant) { return variant == TQ_PROD ? (size_t)d / 8 : 0; }
 
+}  // extern "C"
+
+namespace {
+
+// Validates an encode call into *a.  TQ_OK with *empty set means there is
+// nothing to launch.
+tq_status prepare_encode(const char *name, const char *out_name, const tq_quantizer *q, const void *x,
+                         tq_dtype x_dtype, int64_t B, int64_t H, int64_t N, int64_t x_stride_b, int64_t x_stride_h,
+                         int64_t x_stride_n, const tq_cache_view *out, tq::EncodeArgs *a, bool *empty) {
+  *a = tq::EncodeArgs{};
+  *empty = false;
+  tq_status st = check_quantizer(q, name, &a->q);
+  if (st != TQ_OK) return st;
+  if (x_dtype != TQ_F32 && x_dtype != TQ_BF16 && x_dtype != TQ_F16)
+    return fail(TQ_EINVAL, "%s: x_dtype=%d", name, (int)x_dtype);
+  if (B < 0 || H < 0 || N < 0) return fail(TQ_EINVAL, "%s: negative size", name);
+  if (x_stride_b < 0 || x_stride_h < 0 || x_stride_n < 0) return fail(TQ_EINVAL, "%s: negative stride", name);
+  if (B == 0 || H == 0 || N == 0) {
+    *empty = true;
+    return TQ_OK;
+  }
+  st = check_view(out, a->q, (std::string(name) + "(" + out_name + ")").c_str(), true, &a->out);
+  if (st != TQ_OK) return st;
+  if (!x) return fail(TQ_EINVAL, "%s: x is NULL", name);
+  const size_t es = dtype_size(x_dtype);
+  if (!aligned(x, 16) || (x_stride_b * es) % 16 || (x_stride_h * es) % 16 || (x_stride_n * es) % 16)
+    return fail(TQ_EINVAL, "%s: x and its strides must be 16-byte aligned", name);
+  if (!tq::encode_supported(a->q.d, a->q.bm, a->q.prod, x_dtype))
+    return fail(TQ_EUNSUPPORTED, "%s: d=%d b_m=%d prod=%d dtype=%d not built", name, a->q.d, a->q.bm,
+                (int)a->q.prod, (int)x_dtype);
+  a->x = x;
+  a->dtype = x_dtype;
+  a->B = B;
+  a->H = H;
+  a->N = N;
+  a->xsb = x_stride_b;
+  a->xsh = x_stride_h;
+  a->xsn = x_stride_n;
+  return TQ_OK;
+}
+
+}  // namespace
+
+extern "C" {
+
 tq_status tq_encode(const tq_quantizer *q, const void *x, tq_dtype x_dtype, int64_t B, int64_t H,
                     int64_t N, int64_t x_stride_b, int64_t x_stride_h, int64_t x_stride_n,
                     const tq_cache_view *out, tq_stream_t stream) {
-  tq::EncodeArgs a{};
-  tq_status st = check_quantizer(q, "tq_encode", &a.q);
-  if (st != TQ_OK) return st;
-  if (x_dtype != TQ_F32 && x_dtype != TQ_BF16 && x_dtype != TQ_F16)
-    return fail(TQ_EINVAL, "tq_encode: x_dtype=%d", (int)x_dtype);
-  if (B < 0 || H < 0 || N < 0) return fail(TQ_EINVAL, "tq_encode: negative size");
-  if (x_stride_b < 0 || x_stride_h < 0 || x_stride_n < 0)
-    return fail(TQ_EINVAL, "tq_encode: negative stride");
-  if (B == 0 || H == 0 || N == 0) return TQ_OK;
-  st = check_view(out, a.q, "tq_encode(out)", true, &a.out);
-  if (st != TQ_OK) return st;
-  if (!x) return fail(TQ_EINVAL, "tq_encode: x is NULL");
-  const size_t es = dtype_size(x_dtype);
-  if (!aligned(x, 16) || (x_stride_b * es) % 16 || (x_stride_h * es) % 16 || (x_stride_n * es) % 16)
-    return fail(TQ_EINVAL, "tq_encode: x and its strides must be 16-byte aligned");
-  if (!tq::encode_supported(a.q.d, a.q.bm, a.q.prod, x_dtype))
-    return fail(TQ_EUNSUPPORTED, "tq_encode: d=%d b_m=%d prod=%d dtype=%d not built", a.q.d, a.q.bm,
-                (int)a.q.prod, (int)x_dtype);
-  a.x = x;
-  a.dtype = x_dtype;
-  a.B = B;
-  a.H = H;
-  a.N = N;
-  a.xsb = x_stride_b;
-  a.xsh = x_stride_h;
-  a.xsn = x_stride_n;
+  tq::EncodeArgs a;
+  bool empty;
+  const tq_status st =
+      prepare_encode("tq_encode", "out", q, x, x_dtype, B, H, N, x_stride_b, x_stride_h, x_stride_n, out, &a, &empty);
+  if (st != TQ_OK || empty) return st;
   cudaError_t e = tq::launch_encode(a, (cudaStream_t)stream);
   if (e != cudaSuccess) return cuda_fail(e, "tq_encode launch");
   return TQ_OK;
@@ -364,57 +388,127 @@ size_t tq_decode_workspace_bytes(int32_t B, int32_t Hq, int32_t Hkv, int64_t seq
   return tq::decode_workspace_floats(B, Hq, Hkv, true, tq::decode_ctas()) * sizeof(float);
 }
 
+}  // extern "C"
+
+namespace {
+
+// Validates a decode call into *a.  TQ_OK with *empty set means there is
+// nothing to launch (B == 0 or Hq == 0).
+tq_status prepare_decode(const char *name, const tq_quantizer *kq, const tq_quantizer *vq, const void *q,
+                         tq_dtype q_dtype, int32_t B, int32_t Hq, int32_t Hkv, int64_t seq_len,
+                         const int32_t *seq_lens, const tq_cache_view *k, const tq_cache_view *v,
+                         float softmax_scale, float *out, float *scores_out, void *workspace,
+                         size_t workspace_bytes, tq::DecodeArgs *a, bool *empty) {
+  *a = tq::DecodeArgs{};
+  *empty = false;
+  const std::string nm(name);
+  tq_status st = check_quantizer(kq, (nm + "(kq)").c_str(), &a->kq);
+  if (st != TQ_OK) return st;
+  st = check_quantizer(vq, (nm + "(vq)").c_str(), &a->vq);
+  if (st != TQ_OK) return st;
+  if (a->kq.d != a->vq.d) return fail(TQ_EINVAL, "%s: K d=%d but V d=%d", name, a->kq.d, a->vq.d);
+  if (a->vq.prod) return fail(TQ_EUNSUPPORTED, "%s: prod values are not implemented", name);
+  if (q_dtype != TQ_F32 && q_dtype != TQ_BF16 && q_dtype != TQ_F16)
+    return fail(TQ_EINVAL, "%s: q_dtype=%d", name, (int)q_dtype);
+  if (B < 0 || Hq < 0 || Hkv < 0 || seq_len < 0) return fail(TQ_EINVAL, "%s: negative size", name);
+  if (seq_len > INT32_MAX) return fail(TQ_EINVAL, "%s: seq_len=%lld is 2^31 or more", name, (long long)seq_len);
+  if (Hkv == 0 || Hq % Hkv) return fail(TQ_EINVAL, "%s: Hq=%d not a multiple of Hkv=%d", name, Hq, Hkv);
+  if (!std::isfinite(softmax_scale)) return fail(TQ_EINVAL, "%s: softmax_scale not finite", name);
+  if (B == 0 || Hq == 0) {
+    *empty = true;
+    return TQ_OK;
+  }
+  st = check_view(k, a->kq, (nm + "(k)").c_str(), seq_len > 0, &a->k);
+  if (st != TQ_OK) return st;
+  st = check_view(v, a->vq, (nm + "(v)").c_str(), seq_len > 0, &a->v);
+  if (st != TQ_OK) return st;
+  if (!q || !aligned(q, 16)) return fail(TQ_EINVAL, "%s: q NULL or not 16-byte aligned", name);
+  if (!out || !aligned(out, 16)) return fail(TQ_EINVAL, "%s: out NULL or not 16-byte aligned", name);
+  if (scores_out && !aligned(scores_out, 4)) return fail(TQ_EINVAL, "%s: scores_out misaligned", name);
+  if (!tq::decode_supported(a->kq.d, a->kq.bm, a->kq.prod, a->vq.bm, a->vq.prod))
+    return fail(TQ_EUNSUPPORTED, "%s: d=%d K b_m=%d prod=%d V b_m=%d not built", name, a->kq.d, a->kq.bm,
+                (int)a->kq.prod, a->vq.bm);
+  a->q = q;
+  a->q_dtype = q_dtype;
+  a->B = B;
+  a->Hq = Hq;
+  a->Hkv = Hkv;
+  a->seq_len = seq_len;
+  a->seq_lens = seq_lens;
+  a->scale = softmax_scale;
+  a->out = out;
+  a->scores = scores_out;
+  if (seq_len > 0) {
+    const size_t need = tq_decode_workspace_bytes(B, Hq, Hkv, seq_len, a->kq.d);
+    if (workspace_bytes < need || !workspace || !aligned(workspace, 16))
+      return fail(TQ_EWORKSPACE, "%s: workspace %zu bytes, need %zu (16-byte aligned)", name, workspace_bytes,
+                  need);
+    a->splits = tq::decode_ctas();
+    a->ws = (float *)workspace;
+  }
+  return TQ_OK;
+}
+
+}  // namespace
+
+extern "C" {
+
 tq_status tq_decode_attention(const tq_quantizer *kq, const tq_quantizer *vq, const void *q,
                               tq_dtype q_dtype, int32_t B, int32_t Hq, int32_t Hkv, int64_t seq_len,
                               const int32_t *seq_lens, const tq_cache_view *k,
                               const tq_cache_view *v, float softmax_scale, float *out,
                               float *scores_out, void *workspace, size_t workspace_bytes,
                               tq_stream_t stream) {
-  tq::DecodeArgs a{};
-  tq_status st = check_quantizer(kq, "tq_decode_attention(kq)", &a.kq);
-  if (st != TQ_OK) return st;
-  st = check_quantizer(vq, "tq_decode_attention(vq)", &a.vq);
-  if (st != TQ_OK) return st;
-  if (a.kq.d != a.vq.d) return fail(TQ_EINVAL, "tq_decode_attention: K d=%d but V d=%d", a.kq.d, a.vq.d);
-  if (a.vq.prod) return fail(TQ_EUNSUPPORTED, "tq_decode_attention: prod values are not implemented");
-  if (q_dtype != TQ_F32 && q_dtype != TQ_BF16 && q_dtype != TQ_F16)
-    return fail(TQ_EINVAL, "tq_decode_attention: q_dtype=%d", (int)q_dtype);
-  if (B < 0 || Hq < 0 || Hkv < 0 || seq_len < 0) return fail(TQ_EINVAL, "tq_decode_attention: negative size");
-  if (seq_len > INT32_MAX)
-    return fail(TQ_EINVAL, "tq_decode_attention: seq_len=%lld is 2^31 or more", (long long)seq_len);
-  if (Hkv == 0 || Hq % Hkv) return fail(TQ_EINVAL, "tq_decode_attention: Hq=%d not a multiple of Hkv=%d", Hq, Hkv);
-  if (!std::isfinite(softmax_scale)) return fail(TQ_EINVAL, "tq_decode_attention: softmax_scale not finite");
-  if (B == 0 || Hq == 0) return TQ_OK;
-  st = check_view(k, a.kq, "tq_decode_attention(k)", seq_len > 0, &a.k);
-  if (st != TQ_OK) return st;
-  st = check_view(v, a.vq, "tq_decode_attention(v)", seq_len > 0, &a.v);
-  if (st != TQ_OK) return st;
-  if (!q || !aligned(q, 16)) return fail(TQ_EINVAL, "tq_decode_attention: q NULL or not 16-byte aligned");
-  if (!out || !aligned(out, 16)) return fail(TQ_EINVAL, "tq_decode_attention: out NULL or not 16-byte aligned");
-  if (scores_out && !aligned(scores_out, 4)) return fail(TQ_EINVAL, "tq_decode_attention: scores_out misaligned");
-  if (!tq::decode_supported(a.kq.d, a.kq.bm, a.kq.prod, a.vq.bm, a.vq.prod))
-    return fail(TQ_EUNSUPPORTED, "tq_decode_attention: d=%d K b_m=%d prod=%d V b_m=%d not built", a.kq.d,
-                a.kq.bm, (int)a.kq.prod, a.vq.bm);
-  a.q = q;
-  a.q_dtype = q_dtype;
-  a.B = B;
-  a.Hq = Hq;
-  a.Hkv = Hkv;
-  a.seq_len = seq_len;
-  a.seq_lens = seq_lens;
-  a.scale = softmax_scale;
-  a.out = out;
-  a.scores = scores_out;
-  if (seq_len > 0) {
-    const size_t need = tq_decode_workspace_bytes(B, Hq, Hkv, seq_len, a.kq.d);
-    if (workspace_bytes < need || !workspace || !aligned(workspace, 16))
-      return fail(TQ_EWORKSPACE, "tq_decode_attention: workspace %zu bytes, need %zu (16-byte aligned)",
-                  workspace_bytes, need);
-    a.splits = tq::decode_ctas();
-    a.ws = (float *)workspace;
-  }
+  tq::DecodeArgs a;
+  bool empty;
+  const tq_status st = prepare_decode("tq_decode_attention", kq, vq, q, q_dtype, B, Hq, Hkv, seq_len, seq_lens, k,
+                                      v, softmax_scale, out, scores_out, workspace, workspace_bytes, &a, &empty);
+  if (st != TQ_OK || empty) return st;
   cudaError_t e = tq::launch_decode(a, (cudaStream_t)stream);
   if (e != cudaSuccess) return cuda_fail(e, "tq_decode_attention launch");
+  return TQ_OK;
+}
+
+tq_status tq_append_decode_attention(const tq_quantizer *kq, const tq_quantizer *vq, const void *k_new,
+                                     const void *v_new, tq_dtype kv_dtype, int64_t new_stride_b,
+                                     int64_t new_stride_h, const tq_cache_view *k_tail,
+                                     const tq_cache_view *v_tail, const void *q, tq_dtype q_dtype, int32_t B,
+                                     int32_t Hq, int32_t Hkv, int64_t seq_len, const int32_t *seq_lens,
+                                     const tq_cache_view *k, const tq_cache_view *v, float softmax_scale,
+                                     float *out, float *scores_out, void *workspace, size_t workspace_bytes,
+                                     tq_stream_t stream) {
+  const char *name = "tq_append_decode_attention";
+  tq::EncodeArgs ak, av;
+  tq::DecodeArgs ad;
+  bool ek, ev, ed;
+  tq_status st = prepare_encode(name, "k_tail", kq, k_new, kv_dtype, B, Hkv, 1, new_stride_b, new_stride_h, 0,
+                                k_tail, &ak, &ek);
+  if (st != TQ_OK) return st;
+  st = prepare_encode(name, "v_tail", vq, v_new, kv_dtype, B, Hkv, 1, new_stride_b, new_stride_h, 0, v_tail, &av,
+                      &ev);
+  if (st != TQ_OK) return st;
+  st = prepare_decode(name, kq, vq, q, q_dtype, B, Hq, Hkv, seq_len, seq_lens, k, v, softmax_scale, out,
+                      scores_out, workspace, workspace_bytes, &ad, &ed);
+  if (st != TQ_OK) return st;
+  if (ed) return TQ_OK;  // B == 0 or Hq == 0: no tokens and no heads
+  // K append (an ordinary launch: everything before it in the stream has
+  // finished), then the V append, the prep kernel and the split kernel, each
+  // allowed to start while the one before it runs.  The V append and prep
+  // only read inputs that existed before the chain began; each keeps one
+  // thread waiting for its predecessor, so the chain completes in order and
+  // the split kernel reads the cache only after both appends.
+  const cudaStream_t s = (cudaStream_t)stream;
+  cudaError_t e = cudaSuccess;
+  if (!ek) e = tq::launch_encode(ak, s);
+  if (e == cudaSuccess && !ev) {
+    av.pdl = !ek;
+    e = tq::launch_encode(av, s);
+  }
+  if (e == cudaSuccess) {
+    ad.prep_pdl = !(ek && ev);
+    e = tq::launch_decode(ad, s);
+  }
+  if (e != cudaSuccess) return cuda_fail(e, "tq_append_decode_attention launch");
   return TQ_OK;
 }
 

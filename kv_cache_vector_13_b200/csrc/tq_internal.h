@@ -34,6 +34,10 @@ struct EncodeArgs {
   int64_t B, H, N;
   int64_t xsb, xsh, xsn;  // element strides
   CacheView out;
+  // launched with programmatic stream serialization after the kernel before
+  // it (the fused append + decode chain); the grid then waits for that
+  // kernel before it completes
+  bool pdl = false;
 };
 
 struct DequantArgs {
@@ -56,6 +60,9 @@ struct DecodeArgs {
   float *scores;
   float *ws;           // partial slots
   int splits;          // persistent CTAs of the split kernel
+  // the prep kernel is launched with programmatic stream serialization after
+  // the kernel before it (the fused append + decode chain)
+  bool prep_pdl = false;
 };
 
 // Decode work split shared by the workspace query and the launch: the number

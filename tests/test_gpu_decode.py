@@ -10,6 +10,7 @@ import numpy as np
 import pytest
 import torch
 
+from kv_cache_vector_13_b200 import _lib as L
 from kv_cache_vector_13_b200 import api, inputs
 from oracle import attention as OA
 
@@ -176,3 +177,59 @@ def test_decode_repeated_calls_reuse_workspace():
     assert torch.equal(outs[0], outs[1]) and torch.equal(outs[1], outs[2])
     ref = api.decode_attention(kq, vq, q, kc, vc)
     assert torch.equal(outs[0], ref)
+
+
+@pytest.mark.parametrize("Hq,Hkv,kspec,vspec,dtype", [
+    (8, 2, (4, "mse"), (4, "mse"), torch.bfloat16),
+    (8, 2, (3, "prod"), (3, "mse"), torch.float32),
+    (16, 2, (4, "prod"), (2, "mse"), torch.float16),
+])
+def test_append_decode_matches_separate_calls(Hq, Hkv, kspec, vspec, dtype):
+    # tq_append_decode_attention = tq_encode of the new K and V into the tail
+    # records + tq_decode_attention: same tail records and the same output
+    # bits, over two steps in a row through one workspace
+    B, N, d = 2, 1000, 128
+    g = torch.Generator(device=DEV).manual_seed(71)
+    kq = api.Quantizer(d, kspec[0], kspec[1], seed_rot=72, seed_qjl=73, device=DEV)
+    vq = api.Quantizer(d, vspec[0], vspec[1], seed_rot=74, device=DEV)
+    K = torch.randn((B, Hkv, N, d), generator=g, device=DEV).to(dtype)
+    V = torch.randn((B, Hkv, N, d), generator=g, device=DEV).to(dtype)
+    ka, va = api.encode(kq, K), api.encode(vq, V)
+    kb = api.PackedCache(*(None if t is None else t.clone() for t in (ka.codes, ka.norms, ka.qjl, ka.rnorms)))
+    vb = api.PackedCache(*(None if t is None else t.clone() for t in (va.codes, va.norms, va.qjl, va.rnorms)))
+
+    def tail(c, n):
+        return api.PackedCache(*(None if t is None else t[:, :, n:n + 1] for t in (c.codes, c.norms, c.qjl, c.rnorms)))
+
+    op = api.DecodeAttention(kq, vq, B, Hq, Hkv, N, device=DEV)
+    for step, n in enumerate((N - 1, N - 2)):
+        q = torch.randn((B, Hq, d), generator=g, device=DEV).to(dtype)
+        k_new = torch.randn((B, Hkv, d), generator=g, device=DEV).to(dtype)
+        v_new = torch.randn((B, Hkv, d), generator=g, device=DEV).to(dtype)
+        api.encode(kq, k_new[:, :, None], out=tail(ka, n))
+        api.encode(vq, v_new[:, :, None], out=tail(va, n))
+        ref = api.decode_attention(kq, vq, q, ka, va)
+        got = op.append_step(q, k_new, v_new, tail(kb, n), tail(vb, n), kb, vb).clone()
+        torch.cuda.synchronize()
+        for a_, b_ in ((ka, kb), (va, vb)):
+            for t1, t2 in zip((a_.codes, a_.norms, a_.qjl, a_.rnorms), (b_.codes, b_.norms, b_.qjl, b_.rnorms)):
+                if t1 is not None:
+                    assert torch.equal(t1, t2), f"step {step}: cache records differ"
+        assert torch.equal(ref, got), f"step {step}: max diff {(ref - got).abs().max().item()}"
+
+
+def test_append_decode_rejects_bad_tail_before_any_launch():
+    # a misaligned new-token stride is refused with TQ_EINVAL and nothing runs
+    B, Hq, Hkv, N, d = 1, 4, 1, 64, 128
+    kq = api.Quantizer(d, 4, "mse", seed_rot=1, device=DEV)
+    vq = api.Quantizer(d, 4, "mse", seed_rot=2, device=DEV)
+    kc, vc = api.empty_cache(kq, B, Hkv, N, DEV), api.empty_cache(vq, B, Hkv, N, DEV)
+    op = api.DecodeAttention(kq, vq, B, Hq, Hkv, N, device=DEV)
+    q = torch.zeros((B, Hq, d), device=DEV)
+    buf = torch.zeros((B, Hkv, d + 1), device=DEV)  # row stride d + 1 floats: not a 16-byte multiple
+    k_new = buf[:, :, :d]
+    tk = api.PackedCache(kc.codes[:, :, -1:], kc.norms[:, :, -1:])
+    tv = api.PackedCache(vc.codes[:, :, -1:], vc.norms[:, :, -1:])
+    with pytest.raises(L.TqError) as e:
+        op.append_step(q, k_new, k_new, tk, tv, kc, vc)
+    assert e.value.status == L.TQ_EINVAL
