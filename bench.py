@@ -45,7 +45,7 @@ FALLBACK_PEAKS = {"hbm_gbs": 6650.0, "bf16_tflops": 1590.0}
 # DRAM bytes (read + write) of one decode split-kernel launch on this
 # workload, from an ncu capture (dram__bytes_read.sum + dram__bytes_write.sum),
 # reported only while the decode source is the one it was taken on.
-TRAFFIC = {"bytes": 35772928, "source_sha256": "ce6c36e98f5cd495c969de6fc44d3661d6721aaf2b0fb42b437bdbedd1e46645"}
+TRAFFIC = {"bytes": 35773184, "source_sha256": "07fdf59836888a13898866f28425838d6154c2e64d8a5bf02fa3304648e29a19"}
 
 
 def traffic_bytes():
