@@ -115,12 +115,19 @@ class PackedCache:
         return tuple(self.norms.shape)
 
     def view(self) -> L.TqCacheView:
-        sb, sh, sn = self.norms.stride()
+        # built once per (arrays, layout): a decode step passes the same views
+        key = (_ptr(self.codes), _ptr(self.qjl), _ptr(self.norms), _ptr(self.rnorms), self.norms.stride())
+        cached = self.__dict__.get("_view")
+        if cached is not None and cached[0] == key:
+            return cached[1]
+        sb, sh, sn = key[4]
         for t in (self.codes, self.qjl, self.rnorms):
             if t is not None:
                 w = t.shape[3] if t.dim() == 4 else 1
                 assert t.stride()[:3] == (sb * w, sh * w, sn * w), "all arrays must share one record layout"
-        return L.TqCacheView(_ptr(self.codes), _ptr(self.qjl), _ptr(self.norms), _ptr(self.rnorms), sb, sh, sn)
+        v = L.TqCacheView(key[0], key[1], key[2], key[3], sb, sh, sn)
+        self.__dict__["_view"] = (key, v)
+        return v
 
     def nbytes(self) -> int:
         return sum(t.numel() * t.element_size() for t in (self.codes, self.qjl, self.norms, self.rnorms)

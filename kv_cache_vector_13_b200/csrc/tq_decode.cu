@@ -57,6 +57,7 @@
 
 #include <math.h>
 
+#include <atomic>
 #include <mutex>
 
 // Scratch for tq_decode_attention_noalloc: a fixed array in device memory,
@@ -1260,6 +1261,21 @@ cudaError_t check_smem_layout(K kern) {
   return cudaSuccess;
 }
 
+// Raises a kernel's dynamic shared memory limit once per device (the
+// setting belongs to the kernel, so later launches skip the driver call).
+template <auto Kern>
+cudaError_t set_smem_once(size_t smem) {
+  static std::atomic<uint64_t> done{0};
+  int dev = 0;
+  cudaError_t e = cudaGetDevice(&dev);
+  if (e != cudaSuccess) return e;
+  const uint64_t bit = dev >= 0 && dev < 64 ? (uint64_t)1 << dev : 0;
+  if (bit && (done.load(std::memory_order_acquire) & bit)) return cudaSuccess;
+  e = cudaFuncSetAttribute(Kern, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
+  if (e == cudaSuccess && bit) done.fetch_or(bit, std::memory_order_release);
+  return e;
+}
+
 template <int KBM, bool KPROD, int VBM, bool PACK>
 cudaError_t run_split(const SplitParams &sp, cudaStream_t s) {
   auto kern = decode_split_kernel<KBM, KPROD, VBM, PACK>;
@@ -1267,7 +1283,7 @@ cudaError_t run_split(const SplitParams &sp, cudaStream_t s) {
   const size_t smem = split_smem_bytes(warps);
   static const cudaError_t layout = check_smem_layout(kern);
   if (layout != cudaSuccess) return layout;
-  cudaError_t e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
+  cudaError_t e = set_smem_once<decode_split_kernel<KBM, KPROD, VBM, PACK>>(smem);
   if (e != cudaSuccess) return e;
   // programmatic dependent launch: the grid may start while the prep kernel
   // before it in the stream is still running (the kernel waits for it with
