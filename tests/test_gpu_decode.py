@@ -233,3 +233,36 @@ def test_append_decode_rejects_bad_tail_before_any_launch():
     with pytest.raises(L.TqError) as e:
         op.append_step(q, k_new, k_new, tk, tv, kc, vc)
     assert e.value.status == L.TQ_EINVAL
+
+
+def test_append_decode_with_batch_lengths_and_scores():
+    # ragged per-batch lengths and the scores output through the fused step:
+    # identical to the separate calls (tail at a position every batch attends)
+    B, Hq, Hkv, N, d = 2, 8, 2, 700, 128
+    g = torch.Generator(device=DEV).manual_seed(81)
+    kq = api.Quantizer(d, 3, "prod", seed_rot=82, seed_qjl=83, device=DEV)
+    vq = api.Quantizer(d, 4, "mse", seed_rot=84, device=DEV)
+    K = torch.randn((B, Hkv, N, d), generator=g, device=DEV).to(torch.bfloat16)
+    V = torch.randn((B, Hkv, N, d), generator=g, device=DEV).to(torch.bfloat16)
+    ka, va = api.encode(kq, K), api.encode(vq, V)
+    kb = api.PackedCache(*(None if t is None else t.clone() for t in (ka.codes, ka.norms, ka.qjl, ka.rnorms)))
+    vb = api.PackedCache(*(None if t is None else t.clone() for t in (va.codes, va.norms, va.qjl, va.rnorms)))
+    lens = torch.tensor([N, N - 37], dtype=torch.int32, device=DEV)
+    n = N - 40
+
+    def tail(c):
+        return api.PackedCache(*(None if t is None else t[:, :, n:n + 1] for t in (c.codes, c.norms, c.qjl, c.rnorms)))
+
+    q = torch.randn((B, Hq, d), generator=g, device=DEV).to(torch.bfloat16)
+    k_new = torch.randn((B, Hkv, d), generator=g, device=DEV).to(torch.bfloat16)
+    v_new = torch.randn((B, Hkv, d), generator=g, device=DEV).to(torch.bfloat16)
+    api.encode(kq, k_new[:, :, None], out=tail(ka))
+    api.encode(vq, v_new[:, :, None], out=tail(va))
+    s_ref = torch.full((B, Hq, N), -7.0, device=DEV)
+    ref = api.decode_attention(kq, vq, q, ka, va, seq_lens=lens, scores=s_ref)
+    s_got = torch.full((B, Hq, N), -7.0, device=DEV)
+    op = api.DecodeAttention(kq, vq, B, Hq, Hkv, N, device=DEV)
+    got = op.append_step(q, k_new, v_new, tail(kb), tail(vb), kb, vb, seq_lens=lens, scores=s_got).clone()
+    torch.cuda.synchronize()
+    assert torch.equal(ref, got)
+    assert torch.equal(s_ref, s_got)
