@@ -1,21 +1,27 @@
 """Benchmark: one TurboQuant decode step per step, on B200.
 
-Workload (Llama-3.1-8B-shaped single layer, the configuration the headline
-metric is quoted on): batch 1, 32 query heads / 8 KV heads, head_dim 128,
-32768 cached tokens; K and V are bf16 N(0,1) times a per-(head, channel)
-LogNormal(0, 0.5) scale, compressed with TurboQuant_mse b=4.
+Workload (the largest decode configuration that fits one GPU): batched
+decode, batch 16, 32 query heads / 8 KV heads, head_dim 128, 131072 cached
+tokens per sequence; K, V bf16 N(0,1) with 3 seeded channels per KV head
+(2% of 128) scaled x8; keys TurboQuant_prod b=3 (2-bit Lloyd-Max codes +
+1-bit QJL sketch of the residual), values TurboQuant_mse b=3.  The packed
+cache is 1.81 GB, far larger than the 126 MB L2, so every step streams it
+from HBM.
 
-A step is the whole hot path for one new token, one tq_append_decode_attention
-call: encode the new token's K and V (norm, sign flips + FWHT, Lloyd-Max
-indices, bit-packing) into the cache tail, then decode attention over all
-32768 packed tokens (query rotation, scores from the codes, online softmax, PV
-in the rotated basis, split merge, one inverse rotation).  value =
-KV-tokens/s = B * N / step time.
+A step is the whole hot path for one new token per sequence, one
+tq_append_decode_attention call: encode the new token's K and V (norm, sign
+flips + FWHT, Lloyd-Max indices, bit-packing, residual + QJL signs) into the
+cache tail, then decode attention over all 131072 packed tokens of all 16
+sequences (query rotation, scores from the codes, online softmax, PV in the
+rotated basis, split merge, one inverse rotation).  value = KV-tokens/s =
+B * N / step time.  Steps are timed with CUDA events on the launching stream,
+bracketed by a barrier and a device synchronize, max over ranks.
 
-The cache is replicated 8x (8 x 35.7 MB > 126 MB L2) and step s uses copy
-s % 8, so every step streams its cache from HBM.  Steps are replayed from a
-CUDA graph of 8 steps; the time is taken with CUDA events on the launching
-stream, bracketed by a barrier and a device synchronize, max over ranks.
+The line also carries, as extra keys, the decode call on the 70B-shaped
+long-context configuration (B=1, 64/8 heads, N=2^20, prod-4 K, mse-4 V) and
+on the Llama-3.1-8B-shaped one (B=1, 32/8 heads, N=32768, mse-4 K and V; 8
+rotating cache copies so that it does not sit in L2), and the encode
+throughput on the encode sweep's d=128 cells.
 
 --impl reference times the CPU oracle (oracle/, NumPy) on a bounded sample of
 the same step; that leg is the reported baseline, not the optimisation target.
@@ -26,8 +32,8 @@ scaling is weak and value sums the ranks' tokens over the slowest rank's time.
 """
 
 import argparse
+import hashlib
 import json
-import math
 import os
 import statistics
 import subprocess
@@ -38,18 +44,34 @@ ROOT = os.path.dirname(os.path.abspath(__file__))
 sys.path.insert(0, ROOT)
 
 METRIC = "decode attention KV-tokens/s and encode vectors/s on 1 B200; % of HBM roofline"
-B, HQ, HKV, D, N = 1, 32, 8, 128, 32768
-KBITS, VBITS = 4, 4
-COPIES = 8
+D = 128
+# workloads: sizes, quantizers (bits, variant, seed_rot[, seed_qjl]) and the
+# seeded generator of their K/V (kv_cache_vector_13_b200.inputs)
+WORKLOADS = {
+    "batched": dict(
+        B=16, Hq=32, Hkv=8, N=131072, k=(3, "prod", 20, 21), v=(3, "mse", 22), gen="outlier_kv", seed=3, copies=1,
+        name="batched decode step (append 1 token + attend): B=16 Hq=32 Hkv=8 d=128 N=131072, bf16 K,V "
+             "N(0,1) with 2% outlier channels x8; K TurboQuant_prod b=3, V TurboQuant_mse b=3, "
+             "randomized Hadamard"),
+    "long70b": dict(
+        B=1, Hq=64, Hkv=8, N=1 << 20, k=(4, "prod", 30, 31), v=(4, "mse", 32), gen="student_kv", seed=5, copies=1,
+        name="70B-shaped long-context decode: B=1 Hq=64 Hkv=8 d=128 N=2^20, bf16 K,V 0.5*StudentT(3)*"
+             "LogNormal(0,1) channel scales; K TurboQuant_prod b=4, V TurboQuant_mse b=4"),
+    "llama8b": dict(
+        B=1, Hq=32, Hkv=8, N=32768, k=(4, "mse", 10), v=(4, "mse", 11), gen="llama8b_kv", seed=2, copies=8,
+        name="Llama-3.1-8B-shaped decode: B=1 Hq=32 Hkv=8 d=128 N=32768, bf16 K,V N(0,1)*LogNormal(0,0.5) "
+             "channel scales; K,V TurboQuant_mse b=4"),
+}
+HEADLINE = "batched"
+B, N = WORKLOADS[HEADLINE]["B"], WORKLOADS[HEADLINE]["N"]
 FALLBACK_PEAKS = {"hbm_gbs": 6650.0, "bf16_tflops": 1590.0}
-# DRAM bytes (read + write) of one decode split-kernel launch on this
+# DRAM bytes (read + write) of one decode split-kernel launch on the headline
 # workload, from an ncu capture (dram__bytes_read.sum + dram__bytes_write.sum),
 # reported only while the decode source is the one it was taken on.
-TRAFFIC = {"bytes": 35774976, "source_sha256": "f9f3e6ad80b24e86ffc882a923d0c951bb453cd93ac53a7431e927a72c738390"}
+TRAFFIC = {"bytes": None, "source_sha256": None}
 
 
 def traffic_bytes():
-    import hashlib
     with open(os.path.join(ROOT, "kv_cache_vector_13_b200", "csrc", "tq_decode.cu"), "rb") as f:
         h = hashlib.sha256(f.read()).hexdigest()
     return TRAFFIC["bytes"] if h == TRAFFIC["source_sha256"] else None
@@ -64,7 +86,8 @@ def peaks():
 
 
 class ClockSampler:
-    """nvidia-smi clocks and throttle reasons sampled during the timed region."""
+    """nvidia-smi clocks and throttle reasons, sampled every 20 ms while the
+    GPU runs the warm-up and timed steps."""
 
     Q = ("index,clocks.sm,clocks.max.sm,power.draw,clocks_event_reasons.active,"
          "clocks_event_reasons.hw_slowdown,clocks_event_reasons.hw_thermal_slowdown,"
@@ -78,16 +101,14 @@ class ClockSampler:
         try:
             self.proc = subprocess.Popen(
                 ["nvidia-smi", "-i", str(self.index), f"--query-gpu={self.Q}", "--format=csv,noheader,nounits",
-                 "-lms", "100"], stdout=subprocess.PIPE, stderr=subprocess.DEVNULL, text=True)
+                 "-lms", "20"], stdout=subprocess.PIPE, stderr=subprocess.DEVNULL, text=True)
         except OSError:
             self.proc = None
-        time.sleep(0.3)
         return self
 
     def __exit__(self, *a):
         self.out = ""
         if self.proc is not None:
-            time.sleep(0.2)
             self.proc.terminate()
             try:
                 self.out, _ = self.proc.communicate(timeout=5)
@@ -145,6 +166,78 @@ def job_value(world_size, ms_per_step):
 
 # ------------------------------------------------------------------ our leg
 
+class Setup:
+    """One workload on the device: quantizers, packed caches (encoded by
+    tq_encode from the seeded bf16 K/V, then the inputs are freed), the
+    decode operator and the tail views of token N-1."""
+
+    def __init__(self, api, inputs, torch, dev, key, seed_shift=0):
+        w = WORKLOADS[key]
+        self.w, self.key = w, key
+        self.B, self.Hq, self.Hkv, self.N = w["B"], w["Hq"], w["Hkv"], w["N"]
+        kb, kvar, ksr, *kqs = w["k"]
+        vb, vvar, vsr = w["v"]
+        self.kq = api.Quantizer(D, kb, kvar, seed_rot=ksr, seed_qjl=kqs[0] if kqs else 1, device=dev)
+        self.vq = api.Quantizer(D, vb, vvar, seed_rot=vsr, device=dev)
+        K, V = getattr(inputs, w["gen"])(N=self.N, B=self.B, seed=w["seed"] + seed_shift, device=dev)
+        kc0, vc0 = api.encode(self.kq, K), api.encode(self.vq, V)
+        del K, V
+        torch.cuda.synchronize()
+
+        def clone(c):
+            return api.PackedCache(*(None if t is None else t.clone() for t in (c.codes, c.norms, c.qjl, c.rnorms)))
+
+        self.kcs = [kc0] + [clone(kc0) for _ in range(w["copies"] - 1)]
+        self.vcs = [vc0] + [clone(vc0) for _ in range(w["copies"] - 1)]
+        g = torch.Generator(device=dev).manual_seed(100 + seed_shift)
+        self.q = torch.randn((self.B, self.Hq, D), generator=g, device=dev).to(torch.bfloat16)
+        self.k_new = torch.randn((self.B, self.Hkv, D), generator=g, device=dev).to(torch.bfloat16)
+        self.v_new = torch.randn((self.B, self.Hkv, D), generator=g, device=dev).to(torch.bfloat16)
+        self.op = api.DecodeAttention(self.kq, self.vq, self.B, self.Hq, self.Hkv, self.N, device=dev)
+
+        def tail(c):
+            return api.PackedCache(*(None if t is None else t[:, :, self.N - 1:self.N]
+                                     for t in (c.codes, c.norms, c.qjl, c.rnorms)))
+
+        self.tails = [(tail(kc), tail(vc)) for kc, vc in zip(self.kcs, self.vcs)]
+
+    @property
+    def copies(self):
+        return len(self.kcs)
+
+    def decode_bytes(self):
+        """Algorithmic bytes of one decode call: the packed K and V records of
+        every cached token, the bf16 query and the fp32 output."""
+        return (self.B * self.Hkv * self.N * (self.kq.record_bytes + self.vq.record_bytes)
+                + self.q.numel() * 2 + self.B * self.Hq * D * 4)
+
+    def step(self, c, stream, q=None, k_new=None, v_new=None):
+        # one decode step: tq_append_decode_attention encodes the new token's
+        # K and V into the cache tail and attends over the cache (four
+        # kernels, each allowed to start while the one before it finishes)
+        self.op.append_step(self.q if q is None else q, self.k_new if k_new is None else k_new,
+                            self.v_new if v_new is None else v_new, self.tails[c][0], self.tails[c][1],
+                            self.kcs[c], self.vcs[c], stream=stream)
+
+    def decode(self, c, stream):
+        self.op(self.q, self.kcs[c], self.vcs[c], stream=stream)
+
+
+def time_decode_calls(torch, s, stream, reps):
+    """Live CUDA-event time of one tq_decode_attention call (ms), averaged
+    over `reps` back-to-back calls that cycle through the cache copies."""
+    with torch.cuda.stream(stream):
+        for c in range(max(3, s.copies)):
+            s.decode(c % s.copies, stream)
+        e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+        e0.record(stream)
+        for i in range(reps):
+            s.decode(i % s.copies, stream)
+        e1.record(stream)
+    torch.cuda.synchronize()
+    return e0.elapsed_time(e1) / reps
+
+
 def run_ours(args):
     import torch
     from kv_cache_vector_13_b200 import api, inputs
@@ -160,224 +253,176 @@ def run_ours(args):
         if dist is not None:
             dist.barrier()
 
-    kq = api.Quantizer(D, KBITS, "mse", seed_rot=10, device=dev)
-    vq = api.Quantizer(D, VBITS, "mse", seed_rot=11, device=dev)
-    K, V = inputs.llama8b_kv(N=N, seed=2 + rank, device=dev)
-    kc0, vc0 = api.encode(kq, K), api.encode(vq, V)
-    del K, V
-
-    def clone(c):
-        return api.PackedCache(*(None if t is None else t.clone() for t in (c.codes, c.norms, c.qjl, c.rnorms)))
-
-    kcs = [kc0] + [clone(kc0) for _ in range(COPIES - 1)]
-    vcs = [vc0] + [clone(vc0) for _ in range(COPIES - 1)]
-    g = torch.Generator(device=dev).manual_seed(100 + rank)
-    q = torch.randn((B, HQ, D), generator=g, device=dev).to(torch.bfloat16)
-    k_new = torch.randn((B, HKV, 1, D), generator=g, device=dev).to(torch.bfloat16)
-    v_new = torch.randn((B, HKV, 1, D), generator=g, device=dev).to(torch.bfloat16)
-    op = api.DecodeAttention(kq, vq, B, HQ, HKV, N, device=dev)
-    tails = [(api.PackedCache(kc.codes[:, :, N - 1:N], kc.norms[:, :, N - 1:N]),
-              api.PackedCache(vc.codes[:, :, N - 1:N], vc.norms[:, :, N - 1:N])) for kc, vc in zip(kcs, vcs)]
     stream = torch.cuda.Stream(device=dev)
-
-    def step(c, decode_only=False):
-        # one decode step: tq_append_decode_attention encodes the new token's
-        # K and V into the cache tail and attends over the cache (four
-        # kernels, each allowed to start while the one before it finishes)
-        if decode_only:
-            op(q, kcs[c], vcs[c], stream=stream)
-        else:
-            op.append_step(q, k_new, v_new, tails[c][0], tails[c][1], kcs[c], vcs[c], stream=stream)
-
-    with torch.cuda.stream(stream):
-        for s in range(max(args.warmup, 3)):
-            step(s % COPIES)
-        torch.cuda.synchronize()
-        graph = torch.cuda.CUDAGraph()
-        with torch.cuda.graph(graph, stream=stream):
-            for c in range(COPIES):
-                step(c)
-        graph_dec = torch.cuda.CUDAGraph()
-        with torch.cuda.graph(graph_dec, stream=stream):
-            for c in range(COPIES):
-                step(c, decode_only=True)
-        for _ in range(2):
-            graph.replay()
-            graph_dec.replay()
-        torch.cuda.synchronize()
-
+    s = Setup(api, inputs, torch, dev, HEADLINE, seed_shift=rank)
     K_steps = args.steps
-    reps, rem = divmod(K_steps, COPIES)
-    ev0, ev1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+
+    # warm-up: at least W steps, and at least half a second of them, while the
+    # clock sampler already runs (so its samples see the GPU under load)
     clocks = ClockSampler(local)
     with clocks:
+        with torch.cuda.stream(stream):
+            t_w = time.perf_counter()
+            n_warm = 0
+            while n_warm < max(args.warmup, 3) or time.perf_counter() - t_w < 0.5:
+                s.step(n_warm % s.copies, stream)
+                n_warm += 1
+                if n_warm % 8 == 0:
+                    torch.cuda.synchronize()
         barrier()
         torch.cuda.synchronize()
+        ev0, ev1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
         with torch.cuda.stream(stream):
             ev0.record(stream)
-            for _ in range(reps):
-                graph.replay()
-            for c in range(rem):
-                step(c)
+            for i in range(K_steps):
+                s.step(i % s.copies, stream)
             ev1.record(stream)
         torch.cuda.synchronize()
         barrier()
     t_ms = ev0.elapsed_time(ev1)
 
     # the dominant kernels (prep + split of tq_decode_attention), live
-    d_reps = max(1, reps)
-    e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
-    with torch.cuda.stream(stream):
-        e0.record(stream)
-        for _ in range(d_reps):
-            graph_dec.replay()
-        e1.record(stream)
-    torch.cuda.synchronize()
-    dec_ms = e0.elapsed_time(e1) / (d_reps * COPIES)
+    dec_ms = time_decode_calls(torch, s, stream, max(10, min(K_steps, 200)))
 
-    # end to end through the public API with host buffers (pinned), per step:
-    # H2D of the step's inputs (q, k_new, v_new), the step, D2H of the output
-    # the step's inputs (q, k_new, v_new, all bf16) staged in one pinned host
-    # buffer and one device buffer, so each step copies them with one H2D copy
-    parts = (q, k_new, v_new)
+    # end to end through the public API with host buffers, every step: H2D of
+    # the step's inputs (q, k_new, v_new, bf16, one pinned buffer), the step,
+    # D2H of the fp32 output, host synchronize
+    parts = (s.q, s.k_new, s.v_new)
     sizes = [t.numel() for t in parts]
     hin = torch.empty(sum(sizes), dtype=torch.bfloat16).pin_memory()
     din = torch.empty(sum(sizes), dtype=torch.bfloat16, device=dev)
-    off = 0
-    views = []
+    off, views = 0, []
     for t, n in zip(parts, sizes):
         hin[off:off + n].copy_(t.reshape(-1).cpu())
         views.append(din[off:off + n].view(t.shape))
         off += n
     dq, dk, dv = views
-    hout = torch.empty((B, HQ, D), dtype=torch.float32).pin_memory()
-    e2e_steps = min(K_steps, 2000)
+    hout = torch.empty((s.B, s.Hq, D), dtype=torch.float32).pin_memory()
 
     def e2e_step(c):
         din.copy_(hin, non_blocking=True)
-        op.append_step(dq, dk, dv, tails[c][0], tails[c][1], kcs[c], vcs[c], stream=stream)
-        hout.copy_(op.out, non_blocking=True)
+        s.step(c, stream, dq, dk, dv)
+        hout.copy_(s.op.out, non_blocking=True)
+        stream.synchronize()
 
-    # e2e: each step is one CUDA-graph replay of [H2D copy of the inputs from
-    # pinned memory, tq_append_decode_attention, D2H copy of the output],
-    # then a host synchronize (how a serving loop runs a decode step);
-    # e2e_eager issues the same three calls without a graph
     with torch.cuda.stream(stream):
-        for c in range(COPIES):
-            e2e_step(c)
-        torch.cuda.synchronize()
-        e2e_graphs = []
-        for c in range(COPIES):
-            gph = torch.cuda.CUDAGraph()
-            with torch.cuda.graph(gph, stream=stream):
-                e2e_step(c)
-            e2e_graphs.append(gph)
-        for gph in e2e_graphs:
-            gph.replay()
-        torch.cuda.synchronize()
+        for c in range(3):
+            e2e_step(c % s.copies)
     barrier()
     torch.cuda.synchronize()
     t0 = time.perf_counter()
     with torch.cuda.stream(stream):
-        for s in range(e2e_steps):
-            e2e_graphs[s % COPIES].replay()
-            stream.synchronize()
+        for i in range(K_steps):
+            e2e_step(i % s.copies)
     e2e_s = time.perf_counter() - t0
     barrier()
-    torch.cuda.synchronize()
-    t0 = time.perf_counter()
-    with torch.cuda.stream(stream):
-        for s in range(e2e_steps):
-            e2e_step(s % COPIES)
-            stream.synchronize()
-    e2e_eager_s = time.perf_counter() - t0
-    barrier()
 
-    t_ms, dec_ms, e2e_s, e2e_eager_s = max_over_ranks([t_ms, dec_ms, e2e_s, e2e_eager_s], dist, dev)
-
-    enc_info = bench_encode(api, inputs, torch, dev, stream, args.encode_variant) if rank == 0 else None
-    base = None
-    if rank == 0 and not args.no_cpu_baseline:
-        base = cpu_baseline_decode(budget_s=args.cpu_seconds)
+    t_ms, dec_ms, e2e_s = max_over_ranks([t_ms, dec_ms, e2e_s], dist, dev)
+    line = None
     if rank == 0:
         pk, pk_kind = peaks()
-        dec_bytes = B * HKV * N * (kq.record_bytes + vq.record_bytes) + q.numel() * 2 + B * HQ * D * 4
-        achieved = dec_bytes / (dec_ms * 1e-3) / 1e9
         ms_step = t_ms / K_steps
-        val = job_value(ws, ms_step)
+        dec_bytes = s.decode_bytes()
+        achieved = dec_bytes / (dec_ms * 1e-3) / 1e9
         line = {
-            "metric": METRIC, "value": val, "unit": "KV-tokens/s", "n_gpus": ws, "steps": K_steps,
-            "warmup": max(args.warmup, 3), "ms_per_step": ms_step, "higher_is_better": True,
+            "metric": METRIC, "value": job_value(ws, ms_step), "unit": "KV-tokens/s", "n_gpus": ws,
+            "steps": K_steps, "warmup": n_warm, "ms_per_step": ms_step, "higher_is_better": True,
             "scaling": "weak", "vs_baseline": None, "dtype": "f32 encode; f16xf16->f32 mma decode",
             "data": "synthetic",
-            "config": {"workload": "llama3.1-8b-shaped decode step (append 1 token + attend): B=1 Hq=32 Hkv=8 "
-                                   "d=128 N=32768, K/V TurboQuant_mse b=4, randomized Hadamard",
-                       "global_batch": B * ws, "seq_len": N, "parallelism": f"replicas x{ws}",
-                       "l2": f"{COPIES} rotating cache copies ({COPIES * dec_bytes / 1e6:.0f} MB > 126 MB L2)"},
+            "config": {"workload": s.w["name"], "global_batch": s.B * ws, "seq_len": s.N,
+                       "parallelism": f"replicas x{ws}",
+                       "l2": f"packed cache {dec_bytes / 1e9:.2f} GB per step, larger than the 126 MB L2"},
             "roofline": {"kernel": "tq_decode_attention (prep + split)", "bound": "hbm",
                          "achieved": achieved, "peak": pk["hbm_gbs"], "unit": "GB/s",
                          "frac": achieved / pk["hbm_gbs"], "peak_kind": pk_kind,
                          "bytes_per_launch": dec_bytes, "ms_per_launch": dec_ms,
                          "traffic": args.traffic if args.traffic is not None else traffic_bytes()},
-            "encode": enc_info,
-            "cpu_baseline": base,
-            "e2e": {"value": ws * B * N * e2e_steps / e2e_s, "unit": "KV-tokens/s",
+            "e2e": {"value": ws * s.B * s.N * K_steps / e2e_s, "unit": "KV-tokens/s",
                     "h2d_bytes_per_step": hin.numel() * hin.element_size(),
-                    "d2h_bytes_per_step": hout.numel() * 4, "steps": e2e_steps,
-                    "mode": "per step: CUDA-graph replay of (H2D copy, tq_append_decode_attention, D2H copy), "
-                            "host synchronize"},
-            "e2e_eager": {"value": ws * B * N * e2e_steps / e2e_eager_s, "unit": "KV-tokens/s",
-                          "mode": "the same three calls issued per step without a graph"},
+                    "d2h_bytes_per_step": hout.numel() * 4, "steps": K_steps,
+                    "mode": "per step: H2D copy of (q, k_new, v_new) from pinned memory, "
+                            "tq_append_decode_attention, D2H copy of the output, host synchronize"},
             "gpu_launches": 4 * K_steps,
             "clocks": clocks.summary(),
         }
+    del s
+    torch.cuda.empty_cache()
+
+    if rank == 0:
+        pk, _ = peaks()
+        if not args.no_extras and ws == 1:
+            extras = {}
+            for key in ("long70b", "llama8b"):
+                e = Setup(api, inputs, torch, dev, key)
+                ms = time_decode_calls(torch, e, stream, 40)
+                by = e.decode_bytes()
+                extras[key] = {"workload": e.w["name"], "ms_per_call": ms, "kv_tokens_per_s": e.B * e.N / (ms * 1e-3),
+                               "bytes_per_call": by, "achieved_gbs": by / (ms * 1e-3) / 1e9,
+                               "frac": by / (ms * 1e-3) / 1e9 / pk["hbm_gbs"]}
+                del e
+                torch.cuda.empty_cache()
+            line["decode_other_workloads"] = extras
+            line["encode"] = [bench_encode(api, inputs, torch, dev, stream, v) for v in ("mse4", "prod3", "mse3_bf16")]
+        if not args.no_cpu_baseline and ws == 1:
+            line["cpu_baseline"] = cpu_baseline_decode(budget_s=args.cpu_seconds)
         print(json.dumps(line), flush=True)
     if dist is not None:
-        del graph, graph_dec
         dist.barrier()
         dist.destroy_process_group()
 
 
 def bench_encode(api, inputs, torch, dev, stream, variant="mse4"):
-    """Encode throughput: 2^20 unit vectors, d=128, fp32 input (the encode
-    sweep's d=128 cell), TurboQuant_mse b=4 (or TurboQuant_prod b=3 with
-    variant="prod3"), 2 rotating input copies (1 GB > L2)."""
+    """Encode throughput on 2^20 vectors, d=128, 2 rotating inputs (larger
+    than L2 together): "mse4" / "prod3" are the encode sweep's d=128 cells
+    (unit vectors, fp32, TurboQuant_mse b=4 / TurboQuant_prod b=3);
+    "mse3_bf16" encodes bf16 rows like the decode workloads' values."""
     n, d = 1 << 20, 128
     if variant == "prod3":
         qz = api.Quantizer(d, 3, "prod", seed_rot=0, seed_qjl=1, device=dev)
+    elif variant == "mse3_bf16":
+        qz = api.Quantizer(d, 3, "mse", seed_rot=0, device=dev)
     else:
         qz = api.Quantizer(d, 4, "mse", seed_rot=0, device=dev)
-    xs = [inputs.unit_vectors(n, d, seed=i, device=dev) for i in range(2)]
-    outs = [api.empty_cache(qz, 1, 1, n, dev) for _ in range(2)]
+    if variant == "mse3_bf16":
+        xs = [inputs.vectors(n, d, seed=i, device=dev).to(torch.bfloat16) for i in range(4)]
+    else:
+        xs = [inputs.unit_vectors(n, d, seed=i, device=dev) for i in range(2)]
+    outs = [api.empty_cache(qz, 1, 1, n, dev) for _ in range(len(xs))]
     with torch.cuda.stream(stream):
         for i in range(3):
-            api.encode(qz, xs[i % 2], out=outs[i % 2], stream=stream)
+            api.encode(qz, xs[i % len(xs)], out=outs[i % len(xs)], stream=stream)
         torch.cuda.synchronize()
         e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
         reps = 50
         e0.record(stream)
         for i in range(reps):
-            api.encode(qz, xs[i % 2], out=outs[i % 2], stream=stream)
+            api.encode(qz, xs[i % len(xs)], out=outs[i % len(xs)], stream=stream)
         e1.record(stream)
     torch.cuda.synchronize()
     ms = e0.elapsed_time(e1) / reps
-    byts = n * (d * 4 + qz.record_bytes)
+    byts = n * (d * xs[0].element_size() + qz.record_bytes)
     pk, _ = peaks()
     gbs = byts / (ms * 1e-3) / 1e9
-    name = "TurboQuant_prod b=3" if variant == "prod3" else "TurboQuant_mse b=4"
-    return {"workload": f"2^20 unit vectors d=128 fp32, {name}", "vectors_per_s": n / (ms * 1e-3),
-            "ms_per_launch": ms, "bytes_per_launch": byts, "achieved_gbs": gbs, "frac": gbs / pk["hbm_gbs"]}
+    names = {"mse4": "2^20 unit vectors d=128 fp32, TurboQuant_mse b=4",
+             "prod3": "2^20 unit vectors d=128 fp32, TurboQuant_prod b=3",
+             "mse3_bf16": "2^20 N(0,1) vectors d=128 bf16, TurboQuant_mse b=3"}
+    return {"workload": names[variant], "vectors_per_s": n / (ms * 1e-3), "ms_per_launch": ms,
+            "bytes_per_launch": byts, "achieved_gbs": gbs, "frac": gbs / pk["hbm_gbs"]}
 
 
 # ------------------------------------------------------------- CPU oracle
 
+CPU_TOKENS = 8192  # cached tokens of the oracle's sample slice
+
+
 def cpu_baseline_decode(budget_s=15.0, steps=None):
-    """Time the oracle on a bounded sample of the step: for one KV head (4
-    query heads) of the 8, encode the new token and attend over the 32768
-    tokens; repeat over KV heads until ``budget_s`` of CPU work, and scale
-    the rate to the full layer (8 KV heads)."""
+    """Time the oracle on a bounded sample of the headline step: one (batch,
+    KV head) slice of CPU_TOKENS cached tokens drawn like the headline's
+    (outlier channels, prod-3 keys, mse-3 values); a sample step encodes the
+    new token's K and V and attends the slice's 4 query heads over it.  The
+    rate in token-heads/s is scaled to the headline's KV-tokens/s (a step
+    processes B * Hkv * N token-heads)."""
     import numpy as np
-    import torch
     from kv_cache_vector_13_b200 import inputs
     from oracle import attention as OA
     from oracle import quantizer as OQ
@@ -386,35 +431,35 @@ def cpu_baseline_decode(budget_s=15.0, steps=None):
         blas_threads = max([i.get("num_threads", 1) for i in threadpool_info()] or [1])
     except Exception:  # pragma: no cover
         blas_threads = 1
+    w = WORKLOADS[HEADLINE]
     cores = len(os.sched_getaffinity(0))
-    kq = OQ.Quantizer(D, KBITS, "mse", seed_rot=10)
-    vq = OQ.Quantizer(D, VBITS, "mse", seed_rot=11)
-    K, V = inputs.llama8b_kv(N=N, seed=2, H=1, device="cpu")
-    Kh = K[0, 0].float().numpy()
-    Vh = V[0, 0].float().numpy()
-    kc = {k: v[None, None] for k, v in OQ.encode(kq, Kh, aux=False).items()}
-    vc = {k: v[None, None] for k, v in OQ.encode(vq, Vh, aux=False).items()}
+    kb, kvar, ksr, kqs = w["k"]
+    vb, vvar, vsr = w["v"]
+    kq = OQ.Quantizer(D, kb, kvar, seed_rot=ksr, seed_qjl=kqs)
+    vq = OQ.Quantizer(D, vb, vvar, seed_rot=vsr)
+    K, V = getattr(inputs, w["gen"])(N=CPU_TOKENS, B=1, seed=w["seed"], device="cpu")
+    kc = {k: v[None, None] for k, v in OQ.encode(kq, K[0, 0].float().numpy(), aux=False).items()}
+    vc = {k: v[None, None] for k, v in OQ.encode(vq, V[0, 0].float().numpy(), aux=False).items()}
+    g = w["Hq"] // w["Hkv"]
     rng = np.random.default_rng(0)
-    q = rng.standard_normal((1, HQ // HKV, D)).astype(np.float32)
+    q = rng.standard_normal((1, g, D)).astype(np.float32)
     knew = rng.standard_normal((1, D)).astype(np.float32)
     done, t0 = 0, time.perf_counter()
-    n_steps = 0
     while True:
         OQ.encode(kq, knew, aux=False)
         OQ.encode(vq, knew, aux=False)
         OA.decode_attention(kq, vq, q, kc, vc)
         done += 1
-        n_steps += 1
         el = time.perf_counter() - t0
-        if (steps is not None and n_steps >= steps) or (steps is None and el >= budget_s):
+        if (steps is not None and done >= steps) or (steps is None and el >= budget_s):
             break
-    per_kv_head = el / done
-    step_s = per_kv_head * HKV
-    return {"value": B * N / step_s, "unit": "KV-tokens/s", "cores": cores, "blas_threads": blas_threads,
-            "kind": "oracle",
-            "sample": f"{done} x (1 of 8 KV heads: oracle encode of the new K,V token + float64 decode attention "
-                      f"of 4 query heads over N=32768 TurboQuant_mse b=4 tokens), scaled x8 to the layer; "
-                      f"{el:.1f} s of CPU time"}
+    token_heads_per_s = done * CPU_TOKENS / el
+    return {"value": token_heads_per_s / w["Hkv"], "unit": "KV-tokens/s", "cores": cores,
+            "blas_threads": blas_threads, "kind": "oracle",
+            "sample": f"{done} x (one (batch, KV head) slice of {CPU_TOKENS} tokens drawn like the workload: "
+                      f"oracle encode of the new K,V token + float64 decode attention of {g} query heads, "
+                      f"prod-3 keys, mse-3 values), scaled by token-heads to B={w['B']} x Hkv={w['Hkv']} x "
+                      f"N={w['N']}; {el:.1f} s of CPU time"}
 
 
 def run_reference(args):
@@ -423,17 +468,18 @@ def run_reference(args):
         return
     warm = max(args.warmup, 3)
     cpu_baseline_decode(steps=warm)
+    n = args.ref_steps or min(args.steps, 20)
     t0 = time.perf_counter()
-    base = cpu_baseline_decode(steps=args.ref_steps or min(args.steps, 20))
+    base = cpu_baseline_decode(steps=n)
     el = time.perf_counter() - t0
     ws = int(os.environ.get("WORLD_SIZE", "1"))
+    w = WORKLOADS[HEADLINE]
     line = {"impl": "reference", "metric": METRIC, "value": base["value"], "unit": "KV-tokens/s",
-            "n_gpus": ws, "steps": args.ref_steps or min(args.steps, 20), "warmup": warm,
-            "ms_per_step": B * N / base["value"] * 1e3, "higher_is_better": True, "scaling": "weak",
+            "n_gpus": ws, "steps": n, "warmup": warm,
+            "ms_per_step": w["B"] * w["N"] / base["value"] * 1e3, "higher_is_better": True, "scaling": "weak",
             "vs_baseline": None, "dtype": "f64", "data": "synthetic",
-            "config": {"workload": "llama3.1-8b-shaped decode step (append 1 token + attend): B=1 Hq=32 Hkv=8 "
-                                   "d=128 N=32768, K/V TurboQuant_mse b=4, randomized Hadamard",
-                       "global_batch": B, "seq_len": N, "parallelism": "cpu oracle"},
+            "config": {"workload": w["name"], "global_batch": w["B"], "seq_len": w["N"],
+                       "parallelism": "cpu oracle"},
             "cpu_baseline": base,
             "e2e": {"value": base["value"], "unit": "KV-tokens/s", "h2d_bytes_per_step": 0,
                     "d2h_bytes_per_step": 0},
@@ -444,16 +490,16 @@ def run_reference(args):
 def main():
     ap = argparse.ArgumentParser()
     ap.add_argument("--gpus", type=int, default=1)
-    ap.add_argument("--steps", type=int, default=40000)
-    ap.add_argument("--warmup", type=int, default=16)
+    ap.add_argument("--steps", type=int, default=200)
+    ap.add_argument("--warmup", type=int, default=10)
     ap.add_argument("--impl", default="ours", choices=["ours", "reference"])
     ap.add_argument("--cpu-seconds", type=float, default=15.0)
     ap.add_argument("--no-cpu-baseline", action="store_true")
+    ap.add_argument("--no-extras", action="store_true",
+                    help="skip the other decode workloads and the encode measurements")
     ap.add_argument("--ref-steps", type=int, default=0)
     ap.add_argument("--traffic", type=float, default=None,
                     help="dram bytes per decode call from an ncu capture of this build, if any")
-    ap.add_argument("--encode-variant", default="mse4", choices=["mse4", "prod3"],
-                    help="codec of the encode-throughput measurement")
     args = ap.parse_args()
     if args.impl == "reference":
         run_reference(args)

@@ -58,7 +58,7 @@ typedef enum {
   TQ_EUNSUPPORTED = 2,  /* valid request this build does not implement */
   TQ_ECUDA = 3,         /* a CUDA runtime call or launch failed */
   TQ_EWORKSPACE = 4,    /* workspace smaller than tq_decode_workspace_bytes */
-  TQ_ETIMEOUT = 5       /* reserved: a bounded device-side wait expired */
+  TQ_ETIMEOUT = 5       /* a kernel gave up a bounded wait (reported by tq_check) */
 } tq_status;
 
 typedef enum { TQ_MSE = 0, TQ_PROD = 1 } tq_variant;
@@ -231,7 +231,13 @@ tq_status tq_decode_attention_noalloc(const tq_quantizer *kq, const tq_quantizer
                                       float softmax_scale, float *out,
                                       float *scores_out, tq_stream_t stream);
 
-/* Synchronize `stream` and report any asynchronous CUDA error. */
+/* Synchronize `stream` and report any asynchronous CUDA error, then read and
+ * clear the current GPU's fault word, which the kernels set themselves
+ * instead of trapping: TQ_ETIMEOUT when a kernel gave up a bounded wait on
+ * data that never arrived (about a second; the outputs of that call are not
+ * valid), TQ_ECUDA when a decode launch found its shared-memory layout
+ * invalid and wrote nothing.  The word is per GPU, not per stream: it
+ * reports every such fault on the device since the last tq_check. */
 tq_status tq_check(tq_stream_t stream);
 
 const char *tq_status_string(tq_status s);

@@ -66,6 +66,10 @@
 // from cudaGetSymbolAddress (static_scratch below).
 static __device__ __align__(256) unsigned char g_tq_noalloc_scratch[TQ_NOALLOC_SCRATCH_BYTES];
 
+// Faults a kernel detects on its own, one word per GPU (tq::kFault* bits),
+// set with atomicOr and read back and cleared by tq_check.
+static __device__ unsigned int g_tq_faults;
+
 namespace tq {
 namespace {
 
@@ -777,7 +781,10 @@ __global__ void __launch_bounds__((PACK && !KPROD ? 12 : 8) * 32, 1) decode_spli
   // host sizes the allocation to reach past kLutAddr + kLutBytes + partials
   // from any dynamic base at or below kLutAddr.
   const uint32_t dyn_base = static_cast<uint32_t>(__cvta_generic_to_shared(smem4));
-  if (dyn_base > kLutAddr) return;  // excluded on the host
+  if (dyn_base > kLutAddr) {  // excluded on the host; reported, never silent
+    if (threadIdx.x == 0) atomicOr(&g_tq_faults, kFaultSmemLayout);
+    return;
+  }
   char *s_lut = smem + (kLutAddr - dyn_base);
   float *s_part = reinterpret_cast<float *>(s_lut + kLutBytes);  // [kWarps][8][kPW]
   __shared__ int s_last;
@@ -1331,6 +1338,18 @@ size_t decode_workspace_floats(int B, int Hq, int Hkv, bool prod, int ctas) {
   const int64_t units = (int64_t)B * Hkv * ((Hq / Hkv + 7) / 8);
   (void)prod;  // the fragment block has room for the prod words either way
   return (size_t)kHdr + (size_t)units * kFragWords + (size_t)(units + ctas) * kSlot + (size_t)units;
+}
+
+cudaError_t take_device_faults(unsigned *faults) {
+  unsigned w = 0;
+  cudaError_t e = cudaMemcpyFromSymbol(&w, g_tq_faults, sizeof(w));
+  if (e != cudaSuccess) return e;
+  *faults = w;
+  if (w) {
+    const unsigned zero = 0;
+    e = cudaMemcpyToSymbol(g_tq_faults, &zero, sizeof(zero));
+  }
+  return e;
 }
 
 cudaError_t static_scratch(void **ptr) {

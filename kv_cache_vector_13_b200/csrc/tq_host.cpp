@@ -536,6 +536,14 @@ tq_status tq_check(tq_stream_t stream) {
   if (e != cudaSuccess) return cuda_fail(e, "tq_check");
   e = cudaGetLastError();
   if (e != cudaSuccess) return cuda_fail(e, "tq_check");
+  unsigned faults = 0;
+  e = tq::take_device_faults(&faults);
+  if (e != cudaSuccess) return cuda_fail(e, "tq_check: reading the device fault word");
+  if (faults & tq::kFaultTimeout)
+    return fail(TQ_ETIMEOUT, "tq_check: a kernel gave up a bounded wait on data that never arrived; "
+                             "its outputs are not valid");
+  if (faults & tq::kFaultSmemLayout)
+    return fail(TQ_ECUDA, "tq_check: a decode kernel found its shared-memory layout invalid and wrote nothing");
   return TQ_OK;
 }
 

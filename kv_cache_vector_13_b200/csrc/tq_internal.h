@@ -72,6 +72,15 @@ struct DecodeArgs {
 int decode_ctas();
 size_t decode_workspace_floats(int B, int Hq, int Hkv, bool prod, int ctas);
 
+// Faults the kernels detect themselves (bits of a per-GPU word): a bounded
+// wait that expired, and a launch whose shared-memory layout check failed
+// (the kernel then writes nothing).
+constexpr unsigned kFaultTimeout = 1u;
+constexpr unsigned kFaultSmemLayout = 2u;
+
+// Reads the current device's fault word and clears it (synchronous).
+cudaError_t take_device_faults(unsigned *faults);
+
 // Device address of the allocation-free decode's fixed scratch array on
 // the current device (looked up once per device with cudaGetSymbolAddress).
 cudaError_t static_scratch(void **ptr);

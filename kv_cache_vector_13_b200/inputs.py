@@ -20,8 +20,6 @@ The K/V tensors are returned as [B, Hkv, N, d] views of a [B, N, Hkv, d]
 buffer, the layout a fused QKV projection writes.
 """
 
-import math
-
 import torch
 
 
@@ -106,12 +104,3 @@ def outlier_channels(seed: int = 3, H: int = 8, d: int = 128, frac: float = 0.02
     g = _gen(seed, "cpu")
     n_out = int(round(frac * d))
     return [torch.randperm(d, generator=g)[:n_out].tolist() for _ in range(H)]
-
-
-def flush_l2(buf: torch.Tensor) -> None:
-    """Overwrite a buffer larger than L2 so the next kernel starts cold."""
-    buf.add_(1)
-
-
-def math_sqrt(d: int) -> float:
-    return math.sqrt(d)

@@ -1,8 +1,6 @@
 """Shared helpers for the GPU parity tests: oracle twins of device
 quantizers, and record comparison with the QJL boundary allowance."""
 
-import math
-
 import numpy as np
 import torch
 
@@ -93,5 +91,17 @@ def oracle_attention(kq, vq, q, kc, vc, heads=None, scale=None):
                                heads=heads)
 
 
-def sqrt_d(d):
-    return math.sqrt(d)
+def compare_slice_records(qz, oq, X: np.ndarray, cache, b: int, h: int, chunk: int = 1 << 16) -> int:
+    """Oracle-encode the rows X [N, d] of one (batch, kv head) slice chunk by
+    chunk (with the auxiliary u and z the QJL band needs) and compare them
+    with the device cache's records of slice (b, h).  Returns the number of
+    QJL bits that differ (all inside the fp32 band)."""
+    got_all = flat_host(cache, sl=(b, h))
+    n = X.shape[0]
+    nd = 0
+    for lo in range(0, n, chunk):
+        hi = min(n, lo + chunk)
+        enc = OQ.encode(oq, X[lo:hi], chunk=chunk)
+        got = {k: v[lo:hi] for k, v in got_all.items()}
+        nd += compare_records(qz, oq, enc, got)
+    return nd

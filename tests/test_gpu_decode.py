@@ -13,8 +13,11 @@ import torch
 from kv_cache_vector_13_b200 import _lib as L
 from kv_cache_vector_13_b200 import api, inputs
 from oracle import attention as OA
+from oracle import metrics as OM
+from oracle import quantizer as OQ
 
-from helpers import host, oracle_attention, oracle_cache_slices, oracle_twin, rel_err
+from helpers import (compare_records, compare_slice_records, flat_host, host, oracle_attention,
+                     oracle_cache_slices, oracle_twin, rel_err)
 
 pytestmark = pytest.mark.gpu
 DEV = "cuda"
@@ -118,21 +121,32 @@ def test_decode_config2_full_size():
     kc, vc = api.encode(kq, K), api.encode(vq, V)
     out = host(api.decode_attention(kq, vq, q, kc, vc))
     okq, ovq = oracle_twin(kq), oracle_twin(vq)
-    okc, _ = oracle_cache_slices(okq, host(K))
-    ovc, _ = oracle_cache_slices(ovq, host(V))
+    okc, kenc = oracle_cache_slices(okq, host(K))
+    ovc, venc = oracle_cache_slices(ovq, host(V))
+    # the packed records of all 8 KV heads, bit for bit
+    compare_records(kq, okq, kenc, flat_host(kc))
+    compare_records(vq, ovq, venc, flat_host(vc))
     ref = oracle_attention(okq, ovq, host(q), okc, ovc)
     e = rel_err(out, ref)
     assert e.max() <= TOL, e.max()
 
 
 def sampled_decode(K, V, q, kq, vq, kv_heads):
+    """Decode the whole cache on the GPU; for the sampled (batch, kv head)
+    slices, compare every packed record with the oracle's (codes, norms and
+    residual norms bit for bit, QJL signs up to the fp32 band, at most a
+    1e-6 fraction of them) and the attention outputs of the slice's query
+    heads with the fp32 oracle."""
     kc, vc = api.encode(kq, K), api.encode(vq, V)
     out = host(api.decode_attention(kq, vq, q, kc, vc))
     okq, ovq = oracle_twin(kq), oracle_twin(vq)
-    Hq, Hkv = q.shape[1], K.shape[1]
+    Hq, Hkv, N, d = q.shape[1], K.shape[1], K.shape[2], K.shape[3]
     g = Hq // Hkv
     worst = 0.0
     for (b, h) in kv_heads:
+        nk = compare_slice_records(kq, okq, host(K[b, h]), kc, b, h)
+        assert nk <= max(2, 1e-6 * N * d), f"slice ({b}, {h}): {nk} QJL bits differ"
+        compare_slice_records(vq, ovq, host(V[b, h]), vc, b, h)
         okc, _ = oracle_cache_slices(okq, host(K[b:b + 1, h:h + 1]))
         ovc, _ = oracle_cache_slices(ovq, host(V[b:b + 1, h:h + 1]))
         qb = host(q[b:b + 1, h * g:(h + 1) * g])
@@ -159,6 +173,91 @@ def test_decode_config5_sampled():
     kq = api.Quantizer(128, 4, "prod", seed_rot=30, seed_qjl=31, device=DEV)
     vq = api.Quantizer(128, 4, "mse", seed_rot=32, device=DEV)
     sampled_decode(K, V, q, kq, vq, [(0, 0), (0, 5)])
+
+
+def test_decode_config1_codes_norms_and_mse():
+    # config 1's remaining outputs: the packed codes and norms of the 4096
+    # keys (bit for bit), and the MSE on unit-normalised vectors, measured
+    # through the GPU encode + dequant and equal to the oracle's
+    d, N = 128, 4096
+    x = inputs.vectors(N, d, seed=0, device=DEV)
+    kq = api.Quantizer(d, 3, "mse", seed_rot=0, device=DEV)
+    kc = api.encode(kq, x)
+    okq = oracle_twin(kq)
+    enc = OQ.encode(okq, host(x))
+    compare_records(kq, okq, enc, flat_host(kc))
+    xu = x / x.norm(dim=1, keepdim=True)
+    cu = api.encode(kq, xu)
+    xh = api.dequant(kq, cu)[0, 0].double()
+    mse_gpu = float(((xu.double() - xh) ** 2).sum(dim=1).mean())
+    mse_ref, se = OM.mse(okq, host(xu))
+    compare_records(kq, okq, OQ.encode(okq, host(xu)), flat_host(cu))
+    assert abs(mse_gpu - mse_ref) <= 1e-5 * mse_ref, (mse_gpu, mse_ref)
+    # the sphere value for b = 3 at d = 128 is 0.0340, within sampling error
+    assert abs(mse_gpu - 0.0340) <= 4 * se + 5e-4, (mse_gpu, se)
+
+
+@pytest.mark.parametrize("kspec", [(4, "mse"), (3, "prod")])
+def test_decode_token_major_cache(kspec):
+    # a [B, N, Hkv]-major cache (stride_n = Hkv records): the kernel's general
+    # record addressing; the cache is written by tq_encode through the same
+    # strided view
+    B, Hq, Hkv, N, d = 2, 8, 2, 777, 128
+    g = torch.Generator(device=DEV).manual_seed(41)
+    K = torch.randn((B, Hkv, N, d), generator=g, device=DEV)
+    V = torch.randn((B, Hkv, N, d), generator=g, device=DEV)
+    q = torch.randn((B, Hq, d), generator=g, device=DEV).to(torch.bfloat16)
+    kq = api.Quantizer(d, kspec[0], kspec[1], seed_rot=42, seed_qjl=43, device=DEV)
+    vq = api.Quantizer(d, 3, "mse", seed_rot=44, device=DEV)
+
+    def token_major(qz):
+        def arr(w, dt):
+            t = torch.empty((B, N, Hkv, w), dtype=dt, device=DEV).permute(0, 2, 1, 3)
+            return t if w > 1 else t[..., 0]
+        return api.PackedCache(arr(qz.code_bytes, torch.uint8) if qz.bm else None, arr(1, torch.float32),
+                               arr(qz.qjl_bytes, torch.uint8) if qz.prod else None,
+                               arr(1, torch.float32) if qz.prod else None)
+
+    kc, vc = token_major(kq), token_major(vq)
+    assert kc.view().stride_n == Hkv and kc.view().stride_h == 1
+    api.encode(kq, K, out=kc)
+    api.encode(vq, V, out=vc)
+    sl = torch.tensor([N, N - 300], dtype=torch.int32, device=DEV)
+    out = host(api.decode_attention(kq, vq, q, kc, vc, seq_lens=sl))
+    okq, ovq = oracle_twin(kq), oracle_twin(vq)
+    okc, _ = oracle_cache_slices(okq, host(K))
+    ovc, _ = oracle_cache_slices(ovq, host(V))
+    for b in range(B):
+        L = int(sl[b])
+        kcs = {k: v[b:b + 1, :, :L] for k, v in okc.items()}
+        vcs = {k: v[b:b + 1, :, :L] for k, v in ovc.items()}
+        ref = oracle_attention(okq, ovq, host(q)[b:b + 1], kcs, vcs)
+        e = rel_err(out[b], ref[0]).max()
+        assert e <= TOL, (b, e)
+
+
+def test_decode_zero_norm_rows():
+    # zero key and value vectors: n = 0, so the key's score is 0 and the
+    # value's weight p_j n_j is 0 (log2 n = -inf inside the kernel)
+    B, Hq, Hkv, N, d = 1, 8, 2, 1500, 128
+    g = torch.Generator(device=DEV).manual_seed(51)
+    K = torch.randn((B, Hkv, N, d), generator=g, device=DEV)
+    V = torch.randn((B, Hkv, N, d), generator=g, device=DEV)
+    K[:, :, 3::11] = 0.0
+    V[:, :, ::7] = 0.0
+    V[:, 1, :64] = 0.0  # a whole chunk of zero values on one head
+    q = torch.randn((B, Hq, d), generator=g, device=DEV).to(torch.bfloat16)
+    kq = api.Quantizer(d, 4, "prod", seed_rot=52, seed_qjl=53, device=DEV)
+    vq = api.Quantizer(d, 4, "mse", seed_rot=54, device=DEV)
+    kc, vc = api.encode(kq, K), api.encode(vq, V)
+    assert int((vc.norms == 0).sum()) > 0
+    out = host(api.decode_attention(kq, vq, q, kc, vc))
+    assert np.all(np.isfinite(out))
+    okq, ovq = oracle_twin(kq), oracle_twin(vq)
+    okc, _ = oracle_cache_slices(okq, host(K))
+    ovc, _ = oracle_cache_slices(ovq, host(V))
+    ref = oracle_attention(okq, ovq, host(q), okc, ovc)
+    assert rel_err(out, ref).max() <= TOL
 
 
 def test_decode_repeated_calls_reuse_workspace():
@@ -202,6 +301,8 @@ def test_append_decode_matches_separate_calls(Hq, Hkv, kspec, vspec, dtype):
         return api.PackedCache(*(None if t is None else t[:, :, n:n + 1] for t in (c.codes, c.norms, c.qjl, c.rnorms)))
 
     op = api.DecodeAttention(kq, vq, B, Hq, Hkv, N, device=DEV)
+    okq, ovq = oracle_twin(kq), oracle_twin(vq)
+    Kh, Vh = host(K), host(V)
     for step, n in enumerate((N - 1, N - 2)):
         q = torch.randn((B, Hq, d), generator=g, device=DEV).to(dtype)
         k_new = torch.randn((B, Hkv, d), generator=g, device=DEV).to(dtype)
@@ -216,6 +317,13 @@ def test_append_decode_matches_separate_calls(Hq, Hkv, kspec, vspec, dtype):
                 if t1 is not None:
                     assert torch.equal(t1, t2), f"step {step}: cache records differ"
         assert torch.equal(ref, got), f"step {step}: max diff {(ref - got).abs().max().item()}"
+        # and the fused step against the oracle: the cache with the new
+        # token written at n, encoded and attended by the oracle
+        Kh[:, :, n], Vh[:, :, n] = host(k_new), host(v_new)
+        okc, _ = oracle_cache_slices(okq, Kh)
+        ovc, _ = oracle_cache_slices(ovq, Vh)
+        e = rel_err(host(got), oracle_attention(okq, ovq, host(q), okc, ovc)).max()
+        assert e <= TOL, f"step {step}: fused step vs oracle {e:.2e}"
 
 
 def test_append_decode_rejects_bad_tail_before_any_launch():

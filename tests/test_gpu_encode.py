@@ -58,6 +58,39 @@ def test_encode_bit_exact_half_inputs_strided(dtype, bits, variant):
     compare_records(qz, oq, enc, flat_host(cache))
 
 
+@pytest.mark.parametrize("bits", [3, 4])
+def test_encode_bit_exact_bf16_large_batch_strided(bits):
+    # more than 18944 vectors take the 64-coordinates-per-lane layout: the
+    # one that encodes the decode workloads' bf16 K and V from a
+    # [B, N, H, d] projection buffer through a [B, H, N, d] view
+    B, N, H, d = 2, (1 << 15) + 17, 2, 128
+    g = torch.Generator(device=DEV).manual_seed(60 + bits)
+    buf = (torch.randn((B, N, H, d), generator=g, device=DEV) * 2).to(torch.bfloat16)
+    buf[:, ::1001] = 0
+    x = buf.permute(0, 2, 1, 3)
+    qz = api.Quantizer(d, bits, "mse", seed_rot=61, device=DEV)
+    cache = api.encode(qz, x)
+    torch.cuda.synchronize()
+    oq = oracle_twin(qz)
+    enc = OQ.encode(oq, host(x).reshape(-1, d), chunk=1 << 15, aux=False)
+    compare_records(qz, oq, enc, flat_host(cache))
+
+
+@pytest.mark.parametrize("d", [64, 128, 256])
+@pytest.mark.parametrize("bits", [1, 3])
+def test_encode_bit_exact_fp32_large_batch(d, bits):
+    # the large-batch layout at every d, for the b_m values the other large
+    # tests leave out (1: the sign bit alone; 3: fields that straddle words)
+    n = (1 << 16) + 37
+    x = sample_vectors(n, d, 7 * d + bits, torch.float32)
+    qz = api.Quantizer(d, bits, "mse", seed_rot=70 + bits, device=DEV)
+    cache = api.encode(qz, x.to(DEV))
+    torch.cuda.synchronize()
+    oq = oracle_twin(qz)
+    enc = OQ.encode(oq, host(x), chunk=1 << 15, aux=False)
+    compare_records(qz, oq, enc, flat_host(cache))
+
+
 def test_encode_into_strided_cache_and_tail_append():
     # cache layout [B, H, Ncap] written one token at a time (decode-step append)
     B, H, Ncap, d = 2, 4, 40, 128

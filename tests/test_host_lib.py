@@ -137,6 +137,14 @@ def test_workspace_query_edges():
     assert f(1, 32, 8, 1 << 20, 128) >= f(1, 32, 8, 1 << 10, 128)
 
 
+def test_noalloc_scratch_size_matches_header():
+    # the binding's copy of TQ_NOALLOC_SCRATCH_BYTES is the header's value
+    src = open(os.path.join(ROOT, "include", "tq.h")).read()
+    m = re.search(r"#define\s+TQ_NOALLOC_SCRATCH_BYTES\s+\(\(size_t\)(\d+)\s*<<\s*(\d+)\)", src)
+    assert m, "TQ_NOALLOC_SCRATCH_BYTES not found in include/tq.h"
+    assert L.TQ_NOALLOC_SCRATCH_BYTES == int(m.group(1)) << int(m.group(2))
+
+
 def test_status_strings():
     assert L.status_name(L.TQ_EWORKSPACE) == "TQ_EWORKSPACE"
     assert L.status_name(99) == "TQ_UNKNOWN"
