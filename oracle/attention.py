@@ -11,7 +11,8 @@ function asymmetric_attention_score), i.e. for key j
     est_j = n_j * ( <q', c[idx_j]> + gamma_j * sqrt(pi/2)/d * <S q', sign_j> )
 
 with q' = Pi q the query in the rotated basis (the prod term only for
-TurboQuant_prod keys).  Reading: the pseudocode's correction has no scale and
+TurboQuant_prod keys; Pi is the randomized Hadamard map or, for the dense
+option, the stored Haar matrix).  Reading: the pseudocode's correction has no scale and
 no ||r||; the scale sqrt(pi/2)/d * ||r|| that makes the QJL estimate unbiased
 for m = d projections is used instead ("TurboQuant của Google", section "Vấn
 đề của inner product", the unbiased QJL estimator).
@@ -44,7 +45,9 @@ def _scores_one(qz, q, cache, dtype=np.float64):
     d = qz.d
     N = cache["norms"].shape[0]
     sig = qz.signs.astype(f)
-    if f == np.float64:
+    if qz.dense:
+        qp = qz.Pi.astype(f) @ np.asarray(q, f)
+    elif f == np.float64:
         qp = _rot.rotate_f64(q, qz.signs)
     else:
         qp = _rot.fwht_f32((np.asarray(q, np.float32) * sig)[None, :])[0] / np.float32(math.sqrt(d))
@@ -82,6 +85,8 @@ def _values_one(vq, p, cache, dtype=np.float64):
             sg = (2 * _qz.unpack_bits(cache["qjl"][lo:hi], d, 1) - 1).astype(f)
             gam = cache["rnorms"][lo:hi].astype(f)
             op = op + ((w * gam) @ sg) @ vq.S.astype(f) * f(_qz.SQRT_HALF_PI / d)
+    if vq.dense:
+        return op.astype(f) @ vq.Pi.astype(f)          # Pi^T o'
     if f == np.float64:
         return _rot.unrotate_f64(op, vq.signs)
     sig = vq.signs.astype(np.float32)

@@ -16,6 +16,9 @@ clear, else -1.  S: row-major, entry e from the Box-Muller pair of outputs
 (2*(e//2), 2*(e//2)+1), each mapped to (out >> 11) * 2^-53, the first one
 replaced by 1-u so the log never sees zero; cos for even e, sin for odd e;
 float64 arithmetic rounded once to fp32.
+
+The dense rotation's Gaussian matrix G (oracle.rotation.haar_matrix) is the
+same stream, kept in float64.
 """
 
 import math
@@ -46,16 +49,21 @@ def _unit53(v: int) -> float:
     return (v >> 11) * (1.0 / 9007199254740992.0)
 
 
-def gaussian_matrix(seed: int, d: int) -> np.ndarray:
-    """QJL projection S in R^{d x d}, i.i.d. N(0,1), row-major, fp32."""
+def gaussian_matrix_f64(seed: int, d: int) -> np.ndarray:
+    """d x d i.i.d. N(0,1) entries, row-major, float64 (Box-Muller, unrounded)."""
     n = d * d
-    out = np.empty(n, dtype=np.float32)
+    out = np.empty(n, dtype=np.float64)
     for p in range((n + 1) // 2):
         u1 = 1.0 - _unit53(splitmix64(seed, 2 * p))
         u2 = _unit53(splitmix64(seed, 2 * p + 1))
         r = math.sqrt(-2.0 * math.log(u1))
         ang = 2.0 * math.pi * u2
-        out[2 * p] = np.float32(r * math.cos(ang))
+        out[2 * p] = r * math.cos(ang)
         if 2 * p + 1 < n:
-            out[2 * p + 1] = np.float32(r * math.sin(ang))
+            out[2 * p + 1] = r * math.sin(ang)
     return out.reshape(d, d)
+
+
+def gaussian_matrix(seed: int, d: int) -> np.ndarray:
+    """QJL projection S in R^{d x d}, i.i.d. N(0,1), row-major, fp32."""
+    return gaussian_matrix_f64(seed, d).astype(np.float32)

@@ -17,6 +17,7 @@ NumPy float32 element-wise ops round to nearest even and never fuse):
   x_f  = fp32(x)                      (bf16 / fp16 widen exactly)
   s    = fold-halves sum of fl(x_i^2): for h = d/2, d/4, ..., 1,
          a_i <- fl(a_i + a_{i+h}) for i < h;    n = sqrt_rn(s)
+         (a d that is not a power of two is zero-padded to one first)
   y    = FWHT_f32(sigma * x_f)        (oracle.rotation.fwht_f32)
   w    = fl(n * fp32(sqrt(d)));  inv = fl(1/w) if w > 0 else 0
   u_i  = fl(y_i * inv)                (= (Pi x / ||x||)_i up to rounding)
@@ -27,6 +28,11 @@ NumPy float32 element-wise ops round to nearest even and never fuse):
 Readings (the pages are silent): the residual is taken in the rotated basis
 (the norm and the law of S Pi are unchanged, so the estimator is the same in
 distribution); sign(0) = +1; n = 0 gives inv = 0.
+
+Dense rotation (the Haar-random Pi of oracle.rotation.haar_matrix, stored in
+fp32): the norm is the same canonical fp32 value, and the rotation is the plain
+definition evaluated in float64, u = (Pi_f32 x_f) / n (0 when n = 0); indices
+and residual follow from that u.  Any d that is a multiple of 8 works.
 
 Layout: codes are an LSB-first bitstream per vector, index i's bit k at
 stream bit i*b_m + k (byte p >> 3, bit p & 7); the QJL sketch puts bit k at
@@ -54,17 +60,28 @@ class Quantizer:
     seed_rot: int = 0
     seed_qjl: int = 1
     dist: str = "gauss"
+    rotation: str = "hadamard"    # "hadamard" (sign flips + FWHT) or "dense" (Haar)
     centroids: np.ndarray = field(init=False)
     thresholds: np.ndarray = field(init=False)
     signs: np.ndarray = field(init=False)
     S: np.ndarray = field(init=False)
+    Pi: np.ndarray = field(init=False)
 
     def __post_init__(self):
         assert self.variant in ("mse", "prod")
-        assert self.d >= 2 and self.d & (self.d - 1) == 0
+        assert self.rotation in ("hadamard", "dense")
+        if self.dense:
+            assert self.d >= 8 and self.d % 8 == 0
+        else:
+            assert self.d >= 2 and self.d & (self.d - 1) == 0
         self.centroids, self.thresholds, _, _ = _cb.codebook(self.d, self.bm, self.dist)
         self.signs = _prng.signs(self.seed_rot, self.d)
+        self.Pi = _rot.haar_matrix(self.seed_rot, self.d).astype(np.float32) if self.dense else None
         self.S = _prng.gaussian_matrix(self.seed_qjl, self.d) if self.prod else None
+
+    @property
+    def dense(self) -> bool:
+        return self.rotation == "dense"
 
     @property
     def prod(self) -> bool:
@@ -85,9 +102,15 @@ class Quantizer:
 
 
 def fold_halves_sum_f32(a: np.ndarray) -> np.ndarray:
-    """Row sums of [n, d] float32 in the canonical fold-halves order."""
+    """Row sums of [n, d] float32 in the canonical fold-halves order; a d that
+    is not a power of two (the dense rotation's) is first padded with zeros
+    to the next power of two, which changes no partial sum."""
     assert a.dtype == np.float32
     d = a.shape[1]
+    p2 = 1 << max(0, (d - 1).bit_length())
+    if p2 != d:
+        a = np.concatenate([a, np.zeros((a.shape[0], p2 - d), np.float32)], axis=1)
+        d = p2
     h = d // 2
     while h >= 1:
         a = a[:, :h] + a[:, h:2 * h]
@@ -120,9 +143,9 @@ def encode(qz: Quantizer, x: np.ndarray, chunk: int = 8192, aux: bool = True) ->
     """Encode rows of ``x`` ([n, d], any float dtype holding the input values).
 
     Returns dict(codes [n, code_bytes] u8, norms [n] f32, and for prod
-    qjl [n, d/8] u8, rnorms [n] f32); with ``aux`` also u [n, d] f32 and, for
-    prod, z [n, d] f64 (the projections, kept so tests can measure the
-    distance to the sign boundary).
+    qjl [n, d/8] u8, rnorms [n] f32); with ``aux`` also u [n, d] (f32; f64
+    for the dense rotation) and, for prod, z [n, d] f64 (the projections,
+    kept so tests can measure the distance to the sign boundary).
     """
     x = np.ascontiguousarray(x, dtype=np.float32)
     n, d = x.shape
@@ -135,11 +158,17 @@ def encode(qz: Quantizer, x: np.ndarray, chunk: int = 8192, aux: bool = True) ->
     for s in range(0, n, chunk):
         xb = x[s:s + chunk]
         nrm = np.sqrt(fold_halves_sum_f32(xb * xb))
-        y = _rot.fwht_f32(xb * sig[None, :])
-        w = nrm * sqrt_d
-        inv = np.zeros_like(w)
-        np.divide(np.float32(1.0), w, out=inv, where=w > 0)
-        u = y * inv[:, None]
+        if qz.dense:
+            y = xb.astype(np.float64) @ qz.Pi.astype(np.float64).T
+            n64 = nrm.astype(np.float64)[:, None]
+            u = np.zeros_like(y)
+            np.divide(y, n64, out=u, where=n64 > 0)
+        else:
+            y = _rot.fwht_f32(xb * sig[None, :])
+            w = nrm * sqrt_d
+            inv = np.zeros_like(w)
+            np.divide(np.float32(1.0), w, out=inv, where=w > 0)
+            u = y * inv[:, None]
         if qz.bm > 0:
             idx = (u[:, :, None] > qz.thresholds[None, None, :]).sum(axis=2)
         else:
@@ -150,7 +179,10 @@ def encode(qz: Quantizer, x: np.ndarray, chunk: int = 8192, aux: bool = True) ->
             out["u"].append(u)
         if qz.prod:
             r = u - qz.centroids[idx] if qz.bm > 0 else u.copy()
-            gam = np.sqrt(fold_halves_sum_f32(r * r))
+            if qz.dense:
+                gam = np.sqrt(np.sum(r * r, axis=1)).astype(np.float32)
+            else:
+                gam = np.sqrt(fold_halves_sum_f32(r * r))
             z = r.astype(np.float64) @ qz.S.astype(np.float64).T
             out["qjl"].append(pack_bits((z >= 0).astype(np.int64), 1))
             out["rnorms"].append(gam)
@@ -177,4 +209,8 @@ def dequant(qz: Quantizer, enc: dict) -> np.ndarray:
     """x_hat = ||x|| * Pi^T u_hat, float64 ("内存厂商的噩梦来了", section 4
     pseudocode, dequant)."""
     uh = rotated_estimate(qz, enc)
-    return enc["norms"].astype(np.float64)[:, None] * _rot.unrotate_f64(uh, qz.signs)
+    if qz.dense:
+        back = uh @ qz.Pi.astype(np.float64)          # Pi^T u_hat, row by row
+    else:
+        back = _rot.unrotate_f64(uh, qz.signs)
+    return enc["norms"].astype(np.float64)[:, None] * back
