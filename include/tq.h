@@ -65,8 +65,12 @@ typedef enum { TQ_MSE = 0, TQ_PROD = 1 } tq_variant;
 
 /* TQ_ROT_HADAMARD: Pi = H diag(sigma) / sqrt(d), H the Sylvester Hadamard
  * matrix, sigma the seeded signs ("内存厂商的噩梦来了", the note after the
- * section-4 pseudocode: WHT instead of the dense product).
- * TQ_ROT_DENSE (a Haar-random d x d matrix) returns TQ_EUNSUPPORTED. */
+ * section-4 pseudocode: WHT instead of the dense product); d is 64, 128 or
+ * 256.
+ * TQ_ROT_DENSE: Pi is a Haar-random d x d orthogonal matrix, the Q factor of
+ * the QR decomposition of a seeded Gaussian matrix ("TurboQuant của Google",
+ * section "Trick đầu tiên"), passed as tq_quantizer.rot (tq_make_rotation);
+ * d is any multiple of 8 from 8 to 256. */
 typedef enum { TQ_ROT_HADAMARD = 0, TQ_ROT_DENSE = 1 } tq_rotation;
 
 /* Density the codebook is fitted to: N(0, 1/d) (default), or the exact law
@@ -88,8 +92,10 @@ typedef struct {
   int32_t rotation;        /* tq_rotation */
   const float *centroids;  /* 2^b_m fp32 (unused when b_m == 0) */
   const float *thresholds; /* 2^b_m - 1 fp32 */
-  const int8_t *signs;     /* d entries, each +1 or -1 */
+  const int8_t *signs;     /* d entries, each +1 or -1 (Hadamard rotation) */
   const float *qjl_S;      /* d*d fp32 row-major, prod only, else NULL */
+  const float *rot;        /* d*d fp32 row-major Pi, 16-byte aligned (dense
+                              rotation only, else NULL): y = Pi x */
 } tq_quantizer;
 
 /* A packed cache: records addressed as
@@ -107,8 +113,9 @@ typedef struct {
 
 /* ---- host, synchronous, pure ------------------------------------------ */
 
-/* Lloyd-Max codebook for d and b_m = bits_mse (1..4): 2^b_m centroids and
- * 2^b_m - 1 thresholds (midpoints), fp32, written to HOST arrays.  Lloyd's
+/* Lloyd-Max codebook for d (a multiple of 8 up to 256) and b_m = bits_mse
+ * (1..4): 2^b_m centroids and 2^b_m - 1 thresholds (midpoints), fp32,
+ * written to HOST arrays.  Lloyd's
  * alternation runs in double and is rounded once to fp32 ("TurboQuant của
  * Google", section "Lloyd-Max quantizer": computed once, shipped, reused). */
 tq_status tq_make_codebook(int32_t d, int32_t bits_mse, tq_codebook_dist dist,
@@ -122,6 +129,15 @@ tq_status tq_make_signs(uint64_t seed, int32_t d, int8_t *signs);
  * Box-Muller on consecutive SplitMix64 output pairs ("TurboQuant của
  * Google", section "Vấn đề của inner product": QJL's random projection). */
 tq_status tq_make_qjl(uint64_t seed, int32_t d, float *S);
+
+/* Seeded dense rotation Pi (d x d fp32, row-major, HOST array), d a
+ * multiple of 8 from 8 to 256: G = the seeded Gaussian matrix of
+ * tq_make_qjl's generator in double (unrounded), G = Q R by Householder
+ * reflections in double, Q's columns negated where R's diagonal is negative
+ * (R then has a positive diagonal, which makes Q Haar-distributed),
+ * Pi = Q rounded once to fp32 ("TurboQuant của Google", section "Trick đầu
+ * tiên": the rotation is the Q of a Gaussian matrix's QR). */
+tq_status tq_make_rotation(uint64_t seed, int32_t d, float *rot);
 
 /* Bytes of one record's codes (d*b_m/8) and QJL sketch (d/8 or 0). */
 size_t tq_code_bytes(int32_t d, int32_t bits, int32_t variant);

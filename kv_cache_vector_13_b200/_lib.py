@@ -19,7 +19,7 @@ TQ_NOALLOC_SCRATCH_BYTES = 16 << 20  # include/tq.h
 
 # every symbol include/tq.h declares
 EXPORTS = (
-    "tq_make_codebook", "tq_make_signs", "tq_make_qjl", "tq_code_bytes", "tq_qjl_bytes",
+    "tq_make_codebook", "tq_make_signs", "tq_make_qjl", "tq_make_rotation", "tq_code_bytes", "tq_qjl_bytes",
     "tq_encode", "tq_dequant", "tq_decode_workspace_bytes", "tq_decode_attention",
     "tq_append_decode_attention", "tq_decode_attention_noalloc",
     "tq_check", "tq_status_string", "tq_last_error", "tq_version",
@@ -30,6 +30,7 @@ class TqQuantizer(ctypes.Structure):
     _fields_ = [
         ("d", c_int32), ("bits", c_int32), ("variant", c_int32), ("rotation", c_int32),
         ("centroids", c_void_p), ("thresholds", c_void_p), ("signs", c_void_p), ("qjl_S", c_void_p),
+        ("rot", c_void_p),
     ]
 
 
@@ -64,6 +65,8 @@ def lib() -> ctypes.CDLL:
     L.tq_make_signs.restype = c_int32
     L.tq_make_qjl.argtypes = [c_uint64, c_int32, POINTER(c_float)]
     L.tq_make_qjl.restype = c_int32
+    L.tq_make_rotation.argtypes = [c_uint64, c_int32, POINTER(c_float)]
+    L.tq_make_rotation.restype = c_int32
     L.tq_code_bytes.argtypes = [c_int32, c_int32, c_int32]
     L.tq_code_bytes.restype = c_size_t
     L.tq_qjl_bytes.argtypes = [c_int32, c_int32]

@@ -50,6 +50,13 @@ def make_qjl(seed: int, d: int) -> np.ndarray:
     return S
 
 
+def make_rotation(seed: int, d: int) -> np.ndarray:
+    """Dense Haar rotation Pi (tq_make_rotation), numpy fp32 [d, d]."""
+    R = np.empty((d, d), np.float32)
+    L.check(L.lib().tq_make_rotation(seed, d, R.ctypes.data_as(ctypes.POINTER(ctypes.c_float))))
+    return R
+
+
 def code_bytes(d: int, bits: int, variant: str) -> int:
     return int(L.lib().tq_code_bytes(d, bits, L.TQ_PROD if variant == "prod" else L.TQ_MSE))
 
@@ -64,10 +71,10 @@ class Quantizer:
     """Device-resident parameters of one TurboQuant quantizer."""
 
     def __init__(self, d: int, bits: int, variant: str = "mse", seed_rot: int = 0,
-                 seed_qjl: int = 1, dist: str = "gauss", device="cuda"):
-        assert variant in ("mse", "prod")
+                 seed_qjl: int = 1, dist: str = "gauss", device="cuda", rotation: str = "hadamard"):
+        assert variant in ("mse", "prod") and rotation in ("hadamard", "dense")
         self.d, self.bits, self.variant = d, bits, variant
-        self.seed_rot, self.seed_qjl, self.dist = seed_rot, seed_qjl, dist
+        self.seed_rot, self.seed_qjl, self.dist, self.rotation = seed_rot, seed_qjl, dist, rotation
         self.bm = bits - 1 if variant == "prod" else bits
         dev = torch.device(device)
         if self.bm > 0:
@@ -78,8 +85,11 @@ class Quantizer:
             self.centroids = self.thresholds = None
         self.signs = torch.from_numpy(make_signs(seed_rot, d)).to(dev)
         self.S = torch.from_numpy(make_qjl(seed_qjl, d)).to(dev) if variant == "prod" else None
-        self._c = L.TqQuantizer(d, bits, L.TQ_PROD if variant == "prod" else L.TQ_MSE, L.TQ_ROT_HADAMARD,
-                                _ptr(self.centroids), _ptr(self.thresholds), _ptr(self.signs), _ptr(self.S))
+        self.rot = torch.from_numpy(make_rotation(seed_rot, d)).to(dev) if rotation == "dense" else None
+        self._c = L.TqQuantizer(d, bits, L.TQ_PROD if variant == "prod" else L.TQ_MSE,
+                                L.TQ_ROT_DENSE if rotation == "dense" else L.TQ_ROT_HADAMARD,
+                                _ptr(self.centroids), _ptr(self.thresholds), _ptr(self.signs), _ptr(self.S),
+                                _ptr(self.rot))
 
     @property
     def prod(self) -> bool:

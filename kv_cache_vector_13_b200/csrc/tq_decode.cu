@@ -185,7 +185,8 @@ __global__ void __launch_bounds__(256) decode_prep_kernel(PrepParams p) {
 }  // namespace
 
 
-bool decode_supported(int d, int kbm, bool kprod, int vbm, bool vprod) {
+bool decode_supported(int d, int kbm, bool kprod, int vbm, bool vprod, bool kdense, bool vdense) {
+  if (kdense || vdense) return false;
   return d == kD && !vprod && vbm >= 1 && vbm <= 4 && kbm >= (kprod ? 0 : 1) && kbm <= 4;
 }
 

@@ -123,6 +123,11 @@ cudaError_t by_variant(const DequantArgs &a, cudaStream_t s) {
 
 }  // namespace
 
+bool dequant_supported(int d, int bm, bool prod, bool dense) {
+  if (dense) return false;
+  return (d == 64 || d == 128 || d == 256) && bm >= (prod ? 0 : 1) && bm <= 4;
+}
+
 cudaError_t launch_dequant(const DequantArgs &a, cudaStream_t s) {
   switch (a.q.d) {
     case 64: return by_variant<64>(a, s);

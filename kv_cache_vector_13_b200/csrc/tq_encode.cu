@@ -621,7 +621,8 @@ cudaError_t by_variant(const EncodeArgs &a, cudaStream_t s) {
 
 }  // namespace
 
-bool encode_supported(int d, int bm, bool prod, int dtype) {
+bool encode_supported(int d, int bm, bool prod, int dtype, bool dense) {
+  if (dense) return false;
   return (d == 64 || d == 128 || d == 256) && bm >= (prod ? 0 : 1) && bm <= 4 && dtype >= 0 && dtype <= 2;
 }
 

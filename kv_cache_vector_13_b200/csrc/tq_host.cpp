@@ -168,24 +168,90 @@ uint64_t splitmix64(uint64_t seed, uint64_t k) {
 
 double unit53(uint64_t v) { return (double)(v >> 11) * (1.0 / 9007199254740992.0); }
 
+// Entry e of the seeded d x d Gaussian matrix (row-major), float64: the
+// Box-Muller pair of outputs 2(e/2), 2(e/2)+1, cos for even e, sin for odd.
+void gaussian_f64(uint64_t seed, int d, std::vector<double> &g) {
+  const int64_t n = (int64_t)d * d;
+  g.assign((size_t)n, 0.0);
+  for (int64_t p = 0; p < (n + 1) / 2; ++p) {
+    const double u1 = 1.0 - unit53(splitmix64(seed, 2 * p));
+    const double u2 = unit53(splitmix64(seed, 2 * p + 1));
+    const double r = std::sqrt(-2.0 * std::log(u1));
+    const double ang = 2.0 * M_PI * u2;
+    g[2 * p] = r * std::cos(ang);
+    if (2 * p + 1 < n) g[2 * p + 1] = r * std::sin(ang);
+  }
+}
+
+// Q of G = Q R (Householder, in double) with the columns' signs chosen so
+// that diag(R) > 0; Q written row-major into q.
+void haar_q(std::vector<double> a, int d, std::vector<double> &q) {
+  // a: row-major d x d, overwritten by R; reflectors kept in v[k]
+  std::vector<std::vector<double>> v((size_t)d);
+  for (int k = 0; k < d; ++k) {
+    double nx = 0.0;
+    for (int i = k; i < d; ++i) nx += a[(size_t)i * d + k] * a[(size_t)i * d + k];
+    nx = std::sqrt(nx);
+    std::vector<double> w((size_t)(d - k), 0.0);
+    const double x0 = a[(size_t)k * d + k];
+    const double alpha = x0 >= 0.0 ? -nx : nx;
+    for (int i = k; i < d; ++i) w[(size_t)(i - k)] = a[(size_t)i * d + k];
+    w[0] -= alpha;
+    double nw = 0.0;
+    for (double t : w) nw += t * t;
+    nw = std::sqrt(nw);
+    if (nw > 0.0) {
+      for (double &t : w) t /= nw;
+      for (int j = k; j < d; ++j) {  // A[k:, j] -= 2 w (w . A[k:, j])
+        double dot = 0.0;
+        for (int i = k; i < d; ++i) dot += w[(size_t)(i - k)] * a[(size_t)i * d + j];
+        for (int i = k; i < d; ++i) a[(size_t)i * d + j] -= 2.0 * w[(size_t)(i - k)] * dot;
+      }
+    }
+    v[(size_t)k] = w;
+  }
+  // Q = H_0 H_1 ... H_{d-1} I, applied right to left
+  q.assign((size_t)d * d, 0.0);
+  for (int i = 0; i < d; ++i) q[(size_t)i * d + i] = 1.0;
+  for (int k = d - 1; k >= 0; --k) {
+    const std::vector<double> &w = v[(size_t)k];
+    for (int j = 0; j < d; ++j) {
+      double dot = 0.0;
+      for (int i = k; i < d; ++i) dot += w[(size_t)(i - k)] * q[(size_t)i * d + j];
+      for (int i = k; i < d; ++i) q[(size_t)i * d + j] -= 2.0 * w[(size_t)(i - k)] * dot;
+    }
+  }
+  // sign fix: column j times sign(R_jj)
+  for (int j = 0; j < d; ++j) {
+    if (a[(size_t)j * d + j] < 0.0)
+      for (int i = 0; i < d; ++i) q[(size_t)i * d + j] = -q[(size_t)i * d + j];
+  }
+}
+
 // ------------------------------------------------------------- validation
 
 bool valid_d(int d) { return d == 64 || d == 128 || d == 256; }
+// the dense rotation takes any multiple of 8 up to 256
+bool valid_dense_d(int d) { return d >= 8 && d <= 256 && d % 8 == 0; }
 
 tq_status check_quantizer(const tq_quantizer *q, const char *name, tq::QuantParams *out) {
   if (!q) return fail(TQ_EINVAL, "%s: quantizer is NULL", name);
-  if (!valid_d(q->d)) return fail(TQ_EINVAL, "%s: d=%d (expected 64, 128 or 256)", name, q->d);
+  if (q->rotation != TQ_ROT_HADAMARD && q->rotation != TQ_ROT_DENSE)
+    return fail(TQ_EINVAL, "%s: rotation=%d", name, q->rotation);
+  const bool dense = q->rotation == TQ_ROT_DENSE;
+  if (dense ? !valid_dense_d(q->d) : !valid_d(q->d))
+    return fail(TQ_EINVAL, "%s: d=%d (expected %s)", name, q->d,
+                dense ? "a multiple of 8 from 8 to 256" : "64, 128 or 256");
   if (q->bits < 1 || q->bits > 4) return fail(TQ_EINVAL, "%s: bits=%d (expected 1..4)", name, q->bits);
   if (q->variant != TQ_MSE && q->variant != TQ_PROD)
     return fail(TQ_EINVAL, "%s: variant=%d", name, q->variant);
-  if (q->rotation == TQ_ROT_DENSE)
-    return fail(TQ_EUNSUPPORTED, "%s: dense rotation is not implemented", name);
-  if (q->rotation != TQ_ROT_HADAMARD) return fail(TQ_EINVAL, "%s: rotation=%d", name, q->rotation);
+  if (dense && (!q->rot || (uintptr_t)q->rot % 16))
+    return fail(TQ_EINVAL, "%s: dense rotation without a 16-byte aligned rot matrix", name);
   const bool prod = q->variant == TQ_PROD;
   const int bm = prod ? q->bits - 1 : q->bits;
   if (bm > 0 && (!q->centroids || !q->thresholds))
     return fail(TQ_EINVAL, "%s: centroids/thresholds are NULL", name);
-  if (!q->signs) return fail(TQ_EINVAL, "%s: signs are NULL", name);
+  if (!dense && !q->signs) return fail(TQ_EINVAL, "%s: signs are NULL", name);
   if (prod && !q->qjl_S) return fail(TQ_EINVAL, "%s: prod quantizer without qjl_S", name);
   if (prod && (uintptr_t)q->qjl_S % 16) return fail(TQ_EINVAL, "%s: qjl_S not 16-byte aligned", name);
   out->d = q->d;
@@ -195,6 +261,7 @@ tq_status check_quantizer(const tq_quantizer *q, const char *name, tq::QuantPara
   out->thresholds = q->thresholds;
   out->signs = q->signs;
   out->S = q->qjl_S;
+  out->rot = dense ? q->rot : nullptr;
   out->sqrt_d = (float)std::sqrt((double)q->d);
   return TQ_OK;
 }
@@ -257,7 +324,7 @@ extern "C" {
 
 tq_status tq_make_codebook(int32_t d, int32_t bits_mse, tq_codebook_dist dist, float *centroids,
                            float *thresholds) {
-  if (!valid_d(d)) return fail(TQ_EINVAL, "tq_make_codebook: d=%d", d);
+  if (!valid_dense_d(d)) return fail(TQ_EINVAL, "tq_make_codebook: d=%d", d);
   if (bits_mse < 1 || bits_mse > 4) return fail(TQ_EINVAL, "tq_make_codebook: bits_mse=%d", bits_mse);
   if (!centroids || !thresholds) return fail(TQ_EINVAL, "tq_make_codebook: NULL output");
   const int K = 1 << bits_mse;
@@ -277,24 +344,28 @@ tq_status tq_make_codebook(int32_t d, int32_t bits_mse, tq_codebook_dist dist, f
 }
 
 tq_status tq_make_signs(uint64_t seed, int32_t d, int8_t *signs) {
-  if (!valid_d(d)) return fail(TQ_EINVAL, "tq_make_signs: d=%d", d);
+  if (!valid_dense_d(d)) return fail(TQ_EINVAL, "tq_make_signs: d=%d", d);
   if (!signs) return fail(TQ_EINVAL, "tq_make_signs: NULL output");
   for (int i = 0; i < d; ++i) signs[i] = (splitmix64(seed, (uint64_t)i) >> 63) ? -1 : 1;
   return TQ_OK;
 }
 
 tq_status tq_make_qjl(uint64_t seed, int32_t d, float *S) {
-  if (!valid_d(d)) return fail(TQ_EINVAL, "tq_make_qjl: d=%d", d);
+  if (!valid_dense_d(d)) return fail(TQ_EINVAL, "tq_make_qjl: d=%d", d);
   if (!S) return fail(TQ_EINVAL, "tq_make_qjl: NULL output");
-  const int64_t n = (int64_t)d * d;
-  for (int64_t p = 0; p < (n + 1) / 2; ++p) {
-    const double u1 = 1.0 - unit53(splitmix64(seed, 2 * p));
-    const double u2 = unit53(splitmix64(seed, 2 * p + 1));
-    const double r = std::sqrt(-2.0 * std::log(u1));
-    const double ang = 2.0 * M_PI * u2;
-    S[2 * p] = (float)(r * std::cos(ang));
-    if (2 * p + 1 < n) S[2 * p + 1] = (float)(r * std::sin(ang));
-  }
+  std::vector<double> g;
+  gaussian_f64(seed, d, g);
+  for (size_t i = 0; i < g.size(); ++i) S[i] = (float)g[i];
+  return TQ_OK;
+}
+
+tq_status tq_make_rotation(uint64_t seed, int32_t d, float *rot) {
+  if (!valid_dense_d(d)) return fail(TQ_EINVAL, "tq_make_rotation: d=%d (expected a multiple of 8 from 8 to 256)", d);
+  if (!rot) return fail(TQ_EINVAL, "tq_make_rotation: NULL output");
+  std::vector<double> g, q;
+  gaussian_f64(seed, d, g);
+  haar_q(g, d, q);
+  for (size_t i = 0; i < q.size(); ++i) rot[i] = (float)q[i];
   return TQ_OK;
 }
 
@@ -332,7 +403,7 @@ tq_status prepare_encode(const char *name, const char *out_name, const tq_quanti
   const size_t es = dtype_size(x_dtype);
   if (!aligned(x, 16) || (x_stride_b * es) % 16 || (x_stride_h * es) % 16 || (x_stride_n * es) % 16)
     return fail(TQ_EINVAL, "%s: x and its strides must be 16-byte aligned", name);
-  if (!tq::encode_supported(a->q.d, a->q.bm, a->q.prod, x_dtype))
+  if (!tq::encode_supported(a->q.d, a->q.bm, a->q.prod, x_dtype, a->q.rot != nullptr))
     return fail(TQ_EUNSUPPORTED, "%s: d=%d b_m=%d prod=%d dtype=%d not built", name, a->q.d, a->q.bm,
                 (int)a->q.prod, (int)x_dtype);
   a->x = x;
@@ -373,6 +444,9 @@ tq_status tq_dequant(const tq_quantizer *q, const tq_cache_view *in, int64_t B, 
   st = check_view(in, a.q, "tq_dequant(in)", true, &a.in);
   if (st != TQ_OK) return st;
   if (!out || !aligned(out, 16)) return fail(TQ_EINVAL, "tq_dequant: out NULL or not 16-byte aligned");
+  if (!tq::dequant_supported(a.q.d, a.q.bm, a.q.prod, a.q.rot != nullptr))
+    return fail(TQ_EUNSUPPORTED, "tq_dequant: d=%d b_m=%d prod=%d rotation=%s not built", a.q.d, a.q.bm,
+                (int)a.q.prod, a.q.rot ? "dense" : "hadamard");
   a.B = B;
   a.H = H;
   a.N = N;
@@ -383,7 +457,7 @@ tq_status tq_dequant(const tq_quantizer *q, const tq_cache_view *in, int64_t B, 
 }
 
 size_t tq_decode_workspace_bytes(int32_t B, int32_t Hq, int32_t Hkv, int64_t seq_len, int32_t d) {
-  if (B <= 0 || Hq <= 0 || Hkv <= 0 || seq_len <= 0 || Hq % Hkv || !valid_d(d)) return 0;
+  if (B <= 0 || Hq <= 0 || Hkv <= 0 || seq_len <= 0 || Hq % Hkv || !valid_dense_d(d)) return 0;
   // sized for TurboQuant_prod keys (the larger case) so the query needs no quantizer
   return tq::decode_workspace_floats(B, Hq, Hkv, true, tq::decode_ctas()) * sizeof(float);
 }
@@ -425,7 +499,8 @@ tq_status prepare_decode(const char *name, const tq_quantizer *kq, const tq_quan
   if (!q || !aligned(q, 16)) return fail(TQ_EINVAL, "%s: q NULL or not 16-byte aligned", name);
   if (!out || !aligned(out, 16)) return fail(TQ_EINVAL, "%s: out NULL or not 16-byte aligned", name);
   if (scores_out && !aligned(scores_out, 4)) return fail(TQ_EINVAL, "%s: scores_out misaligned", name);
-  if (!tq::decode_supported(a->kq.d, a->kq.bm, a->kq.prod, a->vq.bm, a->vq.prod))
+  if (!tq::decode_supported(a->kq.d, a->kq.bm, a->kq.prod, a->vq.bm, a->vq.prod, a->kq.rot != nullptr,
+                            a->vq.rot != nullptr))
     return fail(TQ_EUNSUPPORTED, "%s: d=%d K b_m=%d prod=%d V b_m=%d not built", name, a->kq.d, a->kq.bm,
                 (int)a->kq.prod, a->vq.bm);
   a->q = q;

@@ -16,6 +16,7 @@ struct QuantParams {
   const float *thresholds;  // 2^bm - 1
   const int8_t *signs;      // d
   const float *S;           // d*d (prod)
+  const float *rot;         // d*d row-major Pi (dense rotation), else NULL
   float sqrt_d;             // fl32(sqrt(d)) (double sqrt rounded once)
 };
 
@@ -89,8 +90,9 @@ cudaError_t launch_encode(const EncodeArgs &a, cudaStream_t s);
 cudaError_t launch_dequant(const DequantArgs &a, cudaStream_t s);
 cudaError_t launch_decode(const DecodeArgs &a, cudaStream_t s);
 
-// Whether a (d, bm, prod, dtype) encode instantiation exists.
-bool encode_supported(int d, int bm, bool prod, int dtype);
-bool decode_supported(int d, int kbm, bool kprod, int vbm, bool vprod);
+// Whether a (d, bm, prod, dtype, rotation) instantiation exists.
+bool encode_supported(int d, int bm, bool prod, int dtype, bool dense);
+bool dequant_supported(int d, int bm, bool prod, bool dense);
+bool decode_supported(int d, int kbm, bool kprod, int vbm, bool vprod, bool kdense, bool vdense);
 
 }  // namespace tq

@@ -10,7 +10,8 @@ from oracle import quantizer as OQ
 
 def oracle_twin(qz) -> OQ.Quantizer:
     """The oracle's own quantizer with the same (d, bits, variant, seeds)."""
-    return OQ.Quantizer(qz.d, qz.bits, qz.variant, seed_rot=qz.seed_rot, seed_qjl=qz.seed_qjl, dist=qz.dist)
+    return OQ.Quantizer(qz.d, qz.bits, qz.variant, seed_rot=qz.seed_rot, seed_qjl=qz.seed_qjl, dist=qz.dist,
+                        rotation=qz.rotation)
 
 
 def host(t: torch.Tensor) -> np.ndarray:

@@ -50,6 +50,18 @@ def test_beta_codebook_bit_exact_with_oracle(b):
     np.testing.assert_array_equal(t, t2)
 
 
+@pytest.mark.parametrize("d", [8, 64, 128, 200, 256])
+def test_dense_rotation_matches_oracle_within_one_ulp(d):
+    # the library's Householder QR and the oracle's LAPACK QR, both in double
+    # with the same sign fix, agree to within one fp32 rounding step
+    from oracle import rotation as rot
+    P = api.make_rotation(12345 + d, d)
+    Q = rot.haar_matrix(12345 + d, d).astype(np.float32)
+    ulp = np.abs(P.view(np.int32).astype(np.int64) - Q.view(np.int32).astype(np.int64))
+    assert ulp.max() <= 1
+    assert (ulp > 0).mean() < 1e-3
+
+
 @pytest.mark.parametrize("seed", [0, 1, 7, 2 ** 40 + 3, 2 ** 64 - 1])
 def test_seeded_parameters_bit_exact_with_oracle(seed):
     np.testing.assert_array_equal(api.make_signs(seed, 256), prng.signs(seed, 256))
@@ -68,9 +80,9 @@ def test_record_sizes():
 FAKE = 0x10000  # a 64 KiB-aligned address that is never dereferenced
 
 
-def quant(d=128, bits=4, variant=L.TQ_MSE, rot=L.TQ_ROT_HADAMARD, ptrs=True):
+def quant(d=128, bits=4, variant=L.TQ_MSE, rot=L.TQ_ROT_HADAMARD, ptrs=True, rot_matrix=None):
     p = FAKE if ptrs else None
-    return L.TqQuantizer(d, bits, variant, rot, p, p, p, p)
+    return L.TqQuantizer(d, bits, variant, rot, p, p, p, p, rot_matrix)
 
 
 def view(codes=FAKE, norms=FAKE, qjl=FAKE, rnorms=FAKE, sb=0, sh=0, sn=1):
@@ -89,7 +101,10 @@ def test_encode_argument_checks():
     assert enc(quant(bits=5)) == L.TQ_EINVAL
     assert enc(quant(bits=0)) == L.TQ_EINVAL
     assert enc(quant(variant=7)) == L.TQ_EINVAL
-    assert enc(quant(rot=L.TQ_ROT_DENSE)) == L.TQ_EUNSUPPORTED
+    assert enc(quant(rot=L.TQ_ROT_DENSE)) == L.TQ_EINVAL                        # no rot matrix
+    assert enc(quant(rot=L.TQ_ROT_DENSE, rot_matrix=FAKE + 4)) == L.TQ_EINVAL   # misaligned
+    assert enc(quant(d=100, rot=L.TQ_ROT_DENSE, rot_matrix=FAKE)) == L.TQ_EINVAL  # d not a multiple of 8
+    assert enc(quant(d=200)) == L.TQ_EINVAL                                     # Hadamard needs 2^k
     assert enc(quant(ptrs=False)) == L.TQ_EINVAL
     assert enc(quant(), dtype=9) == L.TQ_EINVAL
     assert enc(quant(), B=-1) == L.TQ_EINVAL
