@@ -121,15 +121,39 @@ __global__ void __launch_bounds__(256) decode_prep_kernel(PrepParams p) {
           a[0] = dev::f16lo(v.x); a[1] = dev::f16hi(v.x); a[2] = dev::f16lo(v.y); a[3] = dev::f16hi(v.y);
         }
       }
+      if (!p.krot) {
 #pragma unroll
-      for (int i = 0; i < 4; ++i)
-        if (p.ksign[lane * 4 + i] < 0) a[i] = -a[i];
+        for (int i = 0; i < 4; ++i)
+          if (p.ksign[lane * 4 + i] < 0) a[i] = -a[i];
+      }
     }
-    dev::fwht<32, 4>(a, lane);
+    if (p.krot) {  // dense rotation: stage q, the product follows below
 #pragma unroll
-    for (int i = 0; i < 4; ++i) s_q[half][lane * 4 + i] = a[i] * 0.08838834764831845f;
+      for (int i = 0; i < 4; ++i) s_qs[half][lane * 4 + i] = a[i];
+    } else {
+      dev::fwht<32, 4>(a, lane);
+#pragma unroll
+      for (int i = 0; i < 4; ++i) s_q[half][lane * 4 + i] = a[i] * 0.08838834764831845f;
+    }
   }
   __syncthreads();
+  if (p.krot) {  // q' = Pi q, one output per thread
+    float acc = 0.f;
+    if (valid) {
+      const float4 *R = reinterpret_cast<const float4 *>(p.krot + (size_t)t * kD);
+#pragma unroll 8
+      for (int i = 0; i < kD / 4; ++i) {
+        const float4 r = __ldg(R + i);
+        acc = fmaf(r.x, s_qs[half][4 * i], acc);
+        acc = fmaf(r.y, s_qs[half][4 * i + 1], acc);
+        acc = fmaf(r.z, s_qs[half][4 * i + 2], acc);
+        acc = fmaf(r.w, s_qs[half][4 * i + 3], acc);
+      }
+    }
+    __syncthreads();
+    s_q[half][t] = acc;
+    __syncthreads();
+  }
   if (valid && p.kS) {
     const float4 *Sk = reinterpret_cast<const float4 *>(p.kS + (size_t)t * kD);
     float acc = 0.f;
@@ -186,7 +210,8 @@ __global__ void __launch_bounds__(256) decode_prep_kernel(PrepParams p) {
 
 
 bool decode_supported(int d, int kbm, bool kprod, int vbm, bool vprod, bool kdense, bool vdense) {
-  if (kdense || vdense) return false;
+  (void)kdense;
+  (void)vdense;  // either rotation: only the query's and the output's rotation differ
   return d == kD && !vprod && vbm >= 1 && vbm <= 4 && kbm >= (kprod ? 0 : 1) && kbm <= 4;
 }
 
@@ -292,6 +317,7 @@ cudaError_t launch_decode(const DecodeArgs &a, cudaStream_t s) {
   sp.cnt = reinterpret_cast<unsigned *>(a.ws + sp.slot0 + (int64_t)(units + sp.ctas) * kSlot);
   sp.out = a.out;
   sp.vsign = a.vq.signs;
+  sp.vrot = a.vq.rot;
   {
     void *fw = nullptr;
     const cudaError_t fe = symbol_address(g_tq_faults, &fw);
@@ -301,7 +327,7 @@ cudaError_t launch_decode(const DecodeArgs &a, cudaStream_t s) {
   // without an append before it in the chain, the cache is complete when the
   // split grid starts, so its first bulk copies may precede the prep kernel
   sp.early = !a.prep_pdl;
-  PrepParams pp{a.q, a.q_dtype, a.B * a.Hq, a.kq.signs, a.kq.prod ? a.kq.S : nullptr,
+  PrepParams pp{a.q, a.q_dtype, a.B * a.Hq, a.kq.signs, a.kq.rot, a.kq.prod ? a.kq.S : nullptr,
                 a.kq.centroids, a.kq.bm, a.vq.centroids, a.vq.bm, a.ws, sp.cnt, units,
                 a.Hq, a.Hkv, sp.g, sp.groups, a.seq_len, a.seq_lens, a.out,
                 reinterpret_cast<uint32_t *>(a.ws + kHdr)};

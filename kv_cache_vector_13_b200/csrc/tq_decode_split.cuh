@@ -133,6 +133,7 @@ struct SplitParams {
   unsigned *cnt;      // per-unit arrival counters (zeroed by the prep kernel)
   float *out;
   const int8_t *vsign;
+  const float *vrot;  // dense value rotation Pi_V (row-major), else NULL
   unsigned *faults;   // the GPU's fault word (kFault* bits)
   int dyn_bytes;      // dynamic shared memory of the launch
   bool early;         // the cache is complete when the grid starts (no append before it)
@@ -143,6 +144,7 @@ struct PrepParams {
   int q_dtype;
   int nheads;  // B * Hq
   const int8_t *ksign;
+  const float *krot;  // dense key rotation Pi_K (row-major), else NULL
   const float *kS;  // prod keys only
   const float *kcent;
   int kbm;
@@ -538,8 +540,9 @@ __device__ void merge_unit(const SplitParams &p, const int64_t *cuts, int u, int
   const int parts = nwarps / gh;  // gh <= 8 <= nwarps
   // the value rotation's signs for this lane's 4 dims, loaded alongside the
   // slots (byte loads: the sign array carries no alignment promise)
-  const int8_t sg0 = p.vsign[lane * 4], sg1 = p.vsign[lane * 4 + 1];
-  const int8_t sg2 = p.vsign[lane * 4 + 2], sg3 = p.vsign[lane * 4 + 3];
+  const bool had = p.vrot == nullptr;
+  const int8_t sg0 = had ? p.vsign[lane * 4] : 1, sg1 = had ? p.vsign[lane * 4 + 1] : 1;
+  const int8_t sg2 = had ? p.vsign[lane * 4 + 2] : 1, sg3 = had ? p.vsign[lane * 4 + 3] : 1;
   if (warp < gh * parts) {
     const int hh = warp % gh, part = warp / gh;
     const int i_lo = part * n / parts, i_hi = (part + 1) * n / parts;
@@ -611,16 +614,36 @@ __device__ void merge_unit(const SplitParams &p, const int64_t *cuts, int u, int
         a[2] = fmaf(v.z, w, a[2]);
         a[3] = fmaf(v.w, w, a[3]);
       }
-      const float f = ex2(Ms - m_all) / l * 0.08838834764831845f;
+      if (p.vrot) {
+        // o = Pi_V^T (o' / l): stage o' in this head's own row of s_m (read
+        // only by this warp), then out_j = sum_k Pi[k][j] o'_k
+        const float f = ex2(Ms - m_all) / l;
+        float *st = s_m + hh * kPW + 4;
+        *reinterpret_cast<float4 *>(st + lane * 4) = make_float4(a[0] * f, a[1] * f, a[2] * f, a[3] * f);
+        __syncwarp();
+        float o4[4] = {0.f, 0.f, 0.f, 0.f};
+        const float4 *R = reinterpret_cast<const float4 *>(p.vrot) + lane;
+        for (int k = 0; k < kD; ++k) {
+          const float4 r = __ldg(R + k * (kD / 4));
+          const float ok = st[k];
+          o4[0] = fmaf(r.x, ok, o4[0]);
+          o4[1] = fmaf(r.y, ok, o4[1]);
+          o4[2] = fmaf(r.z, ok, o4[2]);
+          o4[3] = fmaf(r.w, ok, o4[3]);
+        }
+        *reinterpret_cast<float4 *>(out) = make_float4(o4[0], o4[1], o4[2], o4[3]);
+      } else {
+        const float f = ex2(Ms - m_all) / l * 0.08838834764831845f;
 #pragma unroll
-      for (int i = 0; i < 4; ++i) a[i] *= f;
-      dev::fwht<32, 4>(a, lane);
-      float o4[4];
-      o4[0] = sg0 < 0 ? -a[0] : a[0];
-      o4[1] = sg1 < 0 ? -a[1] : a[1];
-      o4[2] = sg2 < 0 ? -a[2] : a[2];
-      o4[3] = sg3 < 0 ? -a[3] : a[3];
-      *reinterpret_cast<float4 *>(out) = make_float4(o4[0], o4[1], o4[2], o4[3]);
+        for (int i = 0; i < 4; ++i) a[i] *= f;
+        dev::fwht<32, 4>(a, lane);
+        float o4[4];
+        o4[0] = sg0 < 0 ? -a[0] : a[0];
+        o4[1] = sg1 < 0 ? -a[1] : a[1];
+        o4[2] = sg2 < 0 ? -a[2] : a[2];
+        o4[3] = sg3 < 0 ? -a[3] : a[3];
+        *reinterpret_cast<float4 *>(out) = make_float4(o4[0], o4[1], o4[2], o4[3]);
+      }
     }
   }
 }

@@ -124,11 +124,12 @@ cudaError_t by_variant(const DequantArgs &a, cudaStream_t s) {
 }  // namespace
 
 bool dequant_supported(int d, int bm, bool prod, bool dense) {
-  if (dense) return false;
+  if (dense) return d >= 8 && d <= 256 && d % 8 == 0 && bm >= (prod ? 0 : 1) && bm <= 4;
   return (d == 64 || d == 128 || d == 256) && bm >= (prod ? 0 : 1) && bm <= 4;
 }
 
 cudaError_t launch_dequant(const DequantArgs &a, cudaStream_t s) {
+  if (a.q.rot) return launch_dequant_dense(a, s);
   switch (a.q.d) {
     case 64: return by_variant<64>(a, s);
     case 128: return by_variant<128>(a, s);

@@ -622,12 +622,13 @@ cudaError_t by_variant(const EncodeArgs &a, cudaStream_t s) {
 }  // namespace
 
 bool encode_supported(int d, int bm, bool prod, int dtype, bool dense) {
-  if (dense) return false;
+  if (dense) return d >= 8 && d <= 256 && d % 8 == 0 && bm >= (prod ? 0 : 1) && bm <= 4 && dtype >= 0 && dtype <= 2;
   return (d == 64 || d == 128 || d == 256) && bm >= (prod ? 0 : 1) && bm <= 4 && dtype >= 0 && dtype <= 2;
 }
 
 cudaError_t launch_encode(const EncodeArgs &a, cudaStream_t s) {
   if (a.B * a.H * a.N >= (int64_t)1 << 40) return cudaErrorInvalidValue;
+  if (a.q.rot) return launch_encode_dense(a, s);
   switch (a.q.d) {
     case 64: return by_variant<64>(a, s);
     case 128: return by_variant<128>(a, s);

@@ -87,6 +87,9 @@ cudaError_t take_device_faults(unsigned *faults);
 cudaError_t static_scratch(void **ptr);
 
 cudaError_t launch_encode(const EncodeArgs &a, cudaStream_t s);
+// the dense (Haar) rotation, any d that is a multiple of 8 up to 256
+cudaError_t launch_encode_dense(const EncodeArgs &a, cudaStream_t s);
+cudaError_t launch_dequant_dense(const DequantArgs &a, cudaStream_t s);
 cudaError_t launch_dequant(const DequantArgs &a, cudaStream_t s);
 cudaError_t launch_decode(const DecodeArgs &a, cudaStream_t s);
 
