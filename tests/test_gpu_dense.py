@@ -107,12 +107,18 @@ def test_dense_dequant_matches_oracle(d, bits, variant):
     cache = api.encode(qz, x.to(DEV))
     xh = host(api.dequant(qz, cache)).reshape(n, d)
     oq = oracle_twin(qz)
-    # dequantize the device's own records with the oracle (same codes)
-    got = flat_host(cache)
-    enc = {k: v.reshape((n,) + v.shape[1:]) if v.ndim > 1 else v.reshape(n) for k, v in got.items()}
+    enc = OQ.encode(oq, host(x))
     ref = OQ.dequant(oq, enc)
+    # rows whose records equal the oracle's (all but the few with a code or
+    # sign inside the rounding band) reconstruct to the same vector
+    got = flat_host(cache)
+    same = np.ones(n, bool)
+    for k in ("codes", "qjl"):
+        if k in enc:
+            same &= np.all(got[k].reshape(enc[k].shape) == enc[k], axis=1)
+    assert same.mean() > 0.99
     nrm = enc["norms"].astype(np.float64)[:, None]
-    assert np.all(np.abs(xh - ref) <= 4 * d * 2.0 ** -24 * nrm + 1e-30)
+    assert np.all((np.abs(xh - ref) <= 4 * d * 2.0 ** -24 * nrm + 1e-30)[same])
 
 
 @pytest.mark.parametrize("kspec,vspec", [((4, "mse"), (4, "mse")), ((3, "prod"), (3, "mse"))])
@@ -127,9 +133,7 @@ def test_dense_decode_matches_oracle(kspec, vspec):
     kc, vc = api.encode(kq, K), api.encode(vq, V)
     out = host(api.decode_attention(kq, vq, q, kc, vc))
     okq, ovq = oracle_twin(kq), oracle_twin(vq)
-    # the oracle attends over the device's own records (codes equal except in
-    # the rounding band, which the encode tests cover)
-    def recs(c):
-        return {k: host(getattr(c, k)) for k in ("codes", "norms", "qjl", "rnorms") if getattr(c, k) is not None}
-    ref = oracle_attention(okq, ovq, host(q), recs(kc), recs(vc))
+    okc, _ = oracle_cache_slices(okq, host(K))
+    ovc, _ = oracle_cache_slices(ovq, host(V))
+    ref = oracle_attention(okq, ovq, host(q), okc, ovc)
     assert rel_err(out, ref).max() <= 2e-3
