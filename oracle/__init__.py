@@ -13,15 +13,18 @@ Modules
   prng       SplitMix64 counter generator, Rademacher signs, Gaussian S
   codebook   Lloyd-Max centroids/thresholds for N(0,1/d) and the exact
              sphere-coordinate (Beta) density
-  rotation   Sylvester-Hadamard rotation, canonical fp32 FWHT
+  rotation   Sylvester-Hadamard rotation, canonical fp32 FWHT; the dense
+             Haar rotation (Q of a seeded Gaussian's QR)
   quantizer  encode (TurboQuant_mse / TurboQuant_prod), bit packing, dequant
   attention  decode attention on the packed cache (float64 and fp32)
+  search     top-k vector search by the estimated inner product
   metrics    distortion (MSE) and inner-product bias
 
 Parity unpinned: the GPU's fp32 summation order for the QJL projection
-S.r (the oracle takes it in float64; sign decisions within rounding of zero
-may differ and are counted by the tests), and the Beta-codebook distortion
-values (the pages print none; only the numerical integral pins them).
+S.r and for the dense rotation's product Pi.x (the oracle takes both in
+float64; decisions within rounding of a threshold or of zero may differ and
+are counted by the tests), and the Beta-codebook distortion values (the
+pages print none; only the numerical integral pins them).
 """
 
-from . import prng, codebook, rotation, quantizer, attention, metrics  # noqa: F401
+from . import prng, codebook, rotation, quantizer, attention, metrics, search  # noqa: F401
