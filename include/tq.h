@@ -247,6 +247,27 @@ tq_status tq_decode_attention_noalloc(const tq_quantizer *kq, const tq_quantizer
                                       float softmax_scale, float *out,
                                       float *scores_out, tq_stream_t stream);
 
+/* Workspace of tq_search_topk, in bytes (0 when a size is out of range). */
+size_t tq_search_workspace_bytes(int32_t n_q, int64_t n_db, int32_t d);
+
+/* Top-k vector search over a packed database ("内存厂商的噩梦来了", section
+ * 6.4: TurboQuant as a nearest-neighbour index, database quantized online,
+ * full-precision queries).  For each query i (queries: [n_q][d], q_dtype,
+ * DEVICE) the k records j < n_db of `db` (record n at n * db->stride_n; the
+ * batch and head strides are not used) with the largest estimated inner
+ * product
+ *   est_j = n_j (<q', c[idx_j]> + [prod] ||r_j|| sqrt(pi/2)/d <S q', sign_j>),
+ * q' = Pi q: the decode scores' estimator, computed the same way.  Order:
+ * est descending, ties by record index ascending.  top_scores: [n_q][k]
+ * fp32, top_index: [n_q][k] int64 (DEVICE); when k > n_db the last k - n_db
+ * entries are -inf and -1.  d must be 128 and 1 <= k <= 32; n_db < 2^31.
+ * workspace: DEVICE, at least tq_search_workspace_bytes(n_q, n_db, d)
+ * bytes, 16-byte aligned, else TQ_EWORKSPACE. */
+tq_status tq_search_topk(const tq_quantizer *q, const tq_cache_view *db, int64_t n_db,
+                         const void *queries, tq_dtype q_dtype, int32_t n_q, int32_t k,
+                         float *top_scores, int64_t *top_index, void *workspace,
+                         size_t workspace_bytes, tq_stream_t stream);
+
 /* Synchronize `stream` and report any asynchronous CUDA error, then read and
  * clear the current GPU's fault word, which the kernels set themselves
  * instead of trapping: TQ_ETIMEOUT when a kernel gave up a bounded wait on

@@ -22,6 +22,7 @@ EXPORTS = (
     "tq_make_codebook", "tq_make_signs", "tq_make_qjl", "tq_make_rotation", "tq_code_bytes", "tq_qjl_bytes",
     "tq_encode", "tq_dequant", "tq_decode_workspace_bytes", "tq_decode_attention",
     "tq_append_decode_attention", "tq_decode_attention_noalloc",
+    "tq_search_workspace_bytes", "tq_search_topk",
     "tq_check", "tq_status_string", "tq_last_error", "tq_version",
 )
 
@@ -95,6 +96,11 @@ def lib() -> ctypes.CDLL:
         c_int64, c_void_p, POINTER(TqCacheView), POINTER(TqCacheView), c_float, c_void_p, c_void_p,
         c_void_p]
     L.tq_decode_attention_noalloc.restype = c_int32
+    L.tq_search_workspace_bytes.argtypes = [c_int32, c_int64, c_int32]
+    L.tq_search_workspace_bytes.restype = c_size_t
+    L.tq_search_topk.argtypes = [POINTER(TqQuantizer), POINTER(TqCacheView), c_int64, c_void_p, c_int32, c_int32,
+                                 c_int32, c_void_p, c_void_p, c_void_p, c_size_t, c_void_p]
+    L.tq_search_topk.restype = c_int32
     L.tq_check.argtypes = [c_void_p]
     L.tq_check.restype = c_int32
     L.tq_status_string.argtypes = [c_int32]

@@ -260,5 +260,38 @@ def decode_attention(kq: Quantizer, vq: Quantizer, q: torch.Tensor, kcache: Pack
     return op(q, kcache, vcache, scale=scale, seq_lens=seq_lens, scores=scores).clone()
 
 
+class Search:
+    """Reusable tq_search_topk call over a packed database of n_db records
+    (its workspace allocated once)."""
+
+    def __init__(self, qz: Quantizer, n_q: int, n_db: int, device="cuda"):
+        self.qz, self.n_q, self.n_db = qz, n_q, n_db
+        nb = int(L.lib().tq_search_workspace_bytes(n_q, n_db, qz.d))
+        self.workspace = torch.empty(max(nb, 16), dtype=torch.uint8, device=device)
+        self.ws_bytes = nb
+
+    def __call__(self, queries: torch.Tensor, db: PackedCache, k: int, stream=None):
+        """(top scores [n_q, k] fp32, top indices [n_q, k] int64) of the
+        queries [n_q, d] against the n_db records of db (shaped [1, 1, n_db]
+        or [n_db], any record stride)."""
+        n_q, d = queries.shape
+        assert n_q == self.n_q and d == self.qz.d and queries.is_contiguous() and queries.dtype in _DTYPES
+        dev = queries.device
+        top_v = torch.empty((n_q, k), dtype=torch.float32, device=dev)
+        top_i = torch.empty((n_q, k), dtype=torch.int64, device=dev)
+        v = db.view()
+        L.check(L.lib().tq_search_topk(ctypes.byref(self.qz.c_struct()), ctypes.byref(v), self.n_db,
+                                       queries.data_ptr(), _DTYPES[queries.dtype], n_q, k, top_v.data_ptr(),
+                                       top_i.data_ptr(), self.workspace.data_ptr(), self.ws_bytes,
+                                       _stream(stream)))
+        return top_v, top_i
+
+
+def search_topk(qz: Quantizer, queries: torch.Tensor, db: PackedCache, k: int):
+    """One-shot tq_search_topk (allocates its workspace and outputs)."""
+    n_db = db.norms.numel()
+    return Search(qz, queries.shape[0], n_db, device=queries.device)(queries, db, k)
+
+
 def check(stream=None) -> None:
     L.check(L.lib().tq_check(_stream(stream)))

@@ -93,8 +93,10 @@ __global__ void __launch_bounds__(256) decode_prep_kernel(PrepParams p) {
     if (blockIdx.x == (unsigned)nqb) {
       if (p.kbm > 0) scale_and_table(p.kcent, p.kbm, p.ws + 0, reinterpret_cast<uint32_t *>(p.ws + 64));
       else if (threadIdx.x == 0) p.ws[0] = 1.0f;
-    } else {
+    } else if (p.vbm > 0) {
       scale_and_table(p.vcent, p.vbm, p.ws + 1, reinterpret_cast<uint32_t *>(p.ws + 320));
+    } else if (threadIdx.x == 0) {
+      p.ws[1] = 1.0f;
     }
     return;
   }
@@ -264,6 +266,25 @@ cudaError_t static_scratch(void **ptr) {
   return symbol_address(g_tq_noalloc_scratch, ptr);
 }
 
+namespace dec {
+
+// The prep kernel: (nheads + 1) / 2 blocks of two query heads, then the key
+// and value table blocks.
+cudaError_t launch_prep(const PrepParams &pp, bool pdl, cudaStream_t s) {
+  cudaLaunchConfig_t cfg = {};
+  cfg.gridDim = dim3((unsigned)((pp.nheads + 1) / 2 + 2));
+  cfg.blockDim = dim3(256);
+  cfg.stream = s;
+  cudaLaunchAttribute attr[1];
+  attr[0].id = cudaLaunchAttributeProgrammaticStreamSerialization;
+  attr[0].val.programmaticStreamSerializationAllowed = pdl ? 1 : 0;
+  cfg.attrs = attr;
+  cfg.numAttrs = 1;
+  return cudaLaunchKernelEx(&cfg, decode_prep_kernel, pp);
+}
+
+}  // namespace dec
+
 cudaError_t launch_decode(const DecodeArgs &a, cudaStream_t s) {
   const int64_t outn = (int64_t)a.B * a.Hq * kD;
   if (a.seq_len == 0) {
@@ -331,19 +352,7 @@ cudaError_t launch_decode(const DecodeArgs &a, cudaStream_t s) {
                 a.kq.centroids, a.kq.bm, a.vq.centroids, a.vq.bm, a.ws, sp.cnt, units,
                 a.Hq, a.Hkv, sp.g, sp.groups, a.seq_len, a.seq_lens, a.out,
                 reinterpret_cast<uint32_t *>(a.ws + kHdr)};
-  cudaError_t pe;
-  {
-    cudaLaunchConfig_t cfg = {};
-    cfg.gridDim = dim3((unsigned)((a.B * a.Hq + 1) / 2 + 2));
-    cfg.blockDim = dim3(256);
-    cfg.stream = s;
-    cudaLaunchAttribute attr[1];
-    attr[0].id = cudaLaunchAttributeProgrammaticStreamSerialization;
-    attr[0].val.programmaticStreamSerializationAllowed = a.prep_pdl ? 1 : 0;
-    cfg.attrs = attr;
-    cfg.numAttrs = 1;
-    pe = cudaLaunchKernelEx(&cfg, decode_prep_kernel, pp);
-  }
+  cudaError_t pe = dec::launch_prep(pp, a.prep_pdl, s);
   if (pe != cudaSuccess) return pe;
   pe = cudaGetLastError();
   if (pe != cudaSuccess) return pe;

@@ -160,6 +160,10 @@ struct PrepParams {
   uint32_t *frag;  // kFragWords per unit
 };
 
+// The prep kernel (tq_decode.cu): query rotation and fragments of every
+// unit, the pair tables, the units' counters zeroed.
+cudaError_t launch_prep(const PrepParams &pp, bool pdl, cudaStream_t s);
+
 // Split-kernel launchers of the two variants (one translation unit each).
 // Each picks the instantiation for (K b_m, K prod, V b_m, <= 4 heads per kv
 // head) and launches it with programmatic stream serialization.

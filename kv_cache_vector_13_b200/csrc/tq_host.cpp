@@ -606,6 +606,59 @@ tq_status tq_decode_attention_noalloc(const tq_quantizer *kq, const tq_quantizer
                              scores_out, ws, need, stream);
 }
 
+size_t tq_search_workspace_bytes(int32_t n_q, int64_t n_db, int32_t d) {
+  if (n_q <= 0 || n_db <= 0 || n_db >= ((int64_t)1 << 31) || d != 128) return 0;
+  return tq::search_workspace_floats(n_q, n_db) * sizeof(float);
+}
+
+tq_status tq_search_topk(const tq_quantizer *q, const tq_cache_view *db, int64_t n_db, const void *queries,
+                         tq_dtype q_dtype, int32_t n_q, int32_t k, float *top_scores, int64_t *top_index,
+                         void *workspace, size_t workspace_bytes, tq_stream_t stream) {
+  const char *name = "tq_search_topk";
+  tq::SearchArgs a{};
+  tq_status st = check_quantizer(q, "tq_search_topk(q)", &a.q);
+  if (st != TQ_OK) return st;
+  if (a.q.d != 128) return fail(TQ_EUNSUPPORTED, "%s: d=%d (only 128 is built)", name, a.q.d);
+  if (q_dtype != TQ_F32 && q_dtype != TQ_BF16 && q_dtype != TQ_F16)
+    return fail(TQ_EINVAL, "%s: q_dtype=%d", name, (int)q_dtype);
+  if (n_q < 0 || n_db < 0) return fail(TQ_EINVAL, "%s: negative size", name);
+  if (n_db >= ((int64_t)1 << 31)) return fail(TQ_EINVAL, "%s: n_db=%lld is 2^31 or more", name, (long long)n_db);
+  if (k < 1 || k > 32) return fail(TQ_EINVAL, "%s: k=%d (expected 1..32)", name, k);
+  if (n_q == 0) return TQ_OK;
+  if (!top_scores || !top_index || !aligned(top_scores, 4) || !aligned(top_index, 8))
+    return fail(TQ_EINVAL, "%s: outputs NULL or misaligned", name);
+  if (!queries || !aligned(queries, 16)) return fail(TQ_EINVAL, "%s: queries NULL or not 16-byte aligned", name);
+  if (n_db == 0) {
+    // nothing to rank: every entry is empty
+    std::vector<float> v((size_t)n_q * k, -INFINITY);
+    std::vector<int64_t> ix((size_t)n_q * k, -1);
+    cudaError_t e = cudaMemcpyAsync(top_scores, v.data(), v.size() * sizeof(float), cudaMemcpyHostToDevice,
+                                    (cudaStream_t)stream);
+    if (e == cudaSuccess)
+      e = cudaMemcpyAsync(top_index, ix.data(), ix.size() * sizeof(int64_t), cudaMemcpyHostToDevice,
+                          (cudaStream_t)stream);
+    if (e == cudaSuccess) e = cudaStreamSynchronize((cudaStream_t)stream);
+    if (e != cudaSuccess) return cuda_fail(e, name);
+    return TQ_OK;
+  }
+  st = check_view(db, a.q, "tq_search_topk(db)", true, &a.db);
+  if (st != TQ_OK) return st;
+  const size_t need = tq_search_workspace_bytes(n_q, n_db, 128);
+  if (workspace_bytes < need || !workspace || !aligned(workspace, 16))
+    return fail(TQ_EWORKSPACE, "%s: workspace %zu bytes, need %zu (16-byte aligned)", name, workspace_bytes, need);
+  a.n_db = n_db;
+  a.queries = queries;
+  a.q_dtype = q_dtype;
+  a.nq = n_q;
+  a.k = k;
+  a.top_v = top_scores;
+  a.top_i = top_index;
+  a.ws = (float *)workspace;
+  const cudaError_t e = tq::launch_search(a, (cudaStream_t)stream);
+  if (e != cudaSuccess) return cuda_fail(e, "tq_search_topk launch");
+  return TQ_OK;
+}
+
 tq_status tq_check(tq_stream_t stream) {
   cudaError_t e = cudaStreamSynchronize((cudaStream_t)stream);
   if (e != cudaSuccess) return cuda_fail(e, "tq_check");

@@ -66,6 +66,22 @@ struct DecodeArgs {
   bool prep_pdl = false;
 };
 
+struct SearchArgs {
+  QuantParams q;
+  CacheView db;   // records n * db.sn, n < n_db
+  int64_t n_db;
+  const void *queries;
+  int q_dtype;
+  int nq, k;
+  float *top_v;
+  int64_t *top_i;
+  float *ws;
+};
+
+// Workspace of a search, in floats.
+size_t search_workspace_floats(int nq, int64_t n_db);
+cudaError_t launch_search(const SearchArgs &a, cudaStream_t s);
+
 // Decode work split shared by the workspace query and the launch: the number
 // of persistent CTAs, and the workspace size in floats (a header with the
 // centroid tables, the rotated queries, and (units + CTAs) partial slots,
