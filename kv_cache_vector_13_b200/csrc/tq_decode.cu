@@ -21,6 +21,12 @@
 
 #include <mutex>
 
+// Which split-kernel variant feeds unit-stride caches: the register-fed one
+// (0, the faster one measured on B200) or the bulk-copy ring (1).
+#ifndef TQ_DECODE_STAGED
+#define TQ_DECODE_STAGED 0
+#endif
+
 // Scratch for tq_decode_attention_noalloc: a fixed array in device memory,
 // one copy per GPU that loads the library, held until the process exits.
 // Host code must not use its name as a device address; the address comes
@@ -261,6 +267,13 @@ cudaError_t symbol_address(const Sym &sym, void **ptr) {
 
 }  // namespace
 
+cudaError_t fault_word(unsigned **ptr) {
+  void *a = nullptr;
+  const cudaError_t e = symbol_address(g_tq_faults, &a);
+  *ptr = static_cast<unsigned *>(a);
+  return e;
+}
+
 cudaError_t static_scratch(void **ptr) {
   // looked up once per device, with that device current, and cached
   return symbol_address(g_tq_noalloc_scratch, ptr);
@@ -362,7 +375,7 @@ cudaError_t launch_decode(const DecodeArgs &a, cudaStream_t s) {
   auto rows16 = [&](const void *ptr, int64_t sb, int64_t sh) {
     return ptr == nullptr || (((uintptr_t)ptr % 16) == 0 && (a.B == 1 || sb % 4 == 0) && (a.Hkv == 1 || sh % 4 == 0));
   };
-  const bool staged = a.k.sn == 1 && a.v.sn == 1 && rows16(a.k.norms, a.k.sb, a.k.sh) &&
+  const bool staged = TQ_DECODE_STAGED && a.k.sn == 1 && a.v.sn == 1 && rows16(a.k.norms, a.k.sb, a.k.sh) &&
                       rows16(a.k.rnorms, a.k.sb, a.k.sh) && rows16(a.v.norms, a.v.sb, a.v.sh);
   cudaError_t e = cudaErrorInvalidValue;
   if (staged) e = dec::launch_split_staged(a.kq.bm, a.kq.prod, a.vq.bm, pack, sp, s);

@@ -21,6 +21,8 @@
 #include "tq_device.cuh"
 #include "tq_internal.h"
 
+#include <cuda_fp16.h>
+
 namespace tq {
 namespace {
 
@@ -205,6 +207,309 @@ __global__ void __launch_bounds__(kDnWarps * 32) dequant_dense_kernel(DenseParam
   }
 }
 
+
+// ------------------------------------------------ tensor cores (tcgen05)
+//
+// d = 64 or 128, TurboQuant_mse, large batches: the rotation of a tile of
+// 128 vectors is the GEMM Y = X Pi^T (M = 128 vectors, N = K = d) on the
+// fifth-generation tensor cores.  fp32 is carried by fp16 halves: each row
+// of X is first scaled by 2^(13 - floor(log2 ||x||)) (exact; the row then
+// lies within [-2^14, 2^14]) and Pi by 16 (exact), and x = hi + lo with
+// hi = fp16(x), lo = fp16(x - hi), likewise Pi; the product is
+// Xh Ph + Xh Pl + Xl Ph (the dropped Xl Pl is below 2^-22 of the terms),
+// accumulated in fp32 in tensor memory.  u = y_scaled * fl(1 / fl(16 s n)).
+// Per CTA (persistent, one per SM, 256 threads):
+//   * once: Pi's halves into shared memory in the K-major, no-swizzle
+//     canonical layout (8 x 16-byte core matrices), and d TMEM columns;
+//   * per tile: the warps load 16 rows each (all loads in flight first),
+//     take each row's canonical norm (fold-halves: in-register stages, then
+//     shuffles), scale, split and store the halves -- the A tile's core
+//     matrices are 144 bytes apart along K so that a warp's 2-byte stores of
+//     one row hit 32 different banks;
+//   * one thread issues the 3 d/16 tcgen05.mma and a tcgen05.commit to an
+//     mbarrier; every thread waits on it (bounded);
+//   * the epilogue: warp w reads TMEM lanes 32 (w % 4) + [0, 32) (its rows)
+//     and columns (w / 4) d/2 + [0, d/2) with tcgen05.ld, scales, quantizes
+//     and packs half a record per thread.
+
+constexpr int kTcThreads = 256;
+constexpr int kTcM = 128;          // vectors per tile
+constexpr int kTcLboA = 144;       // bytes between K-adjacent core matrices of A
+constexpr int kTcLboB = 128;
+
+template <int D>
+struct TcLayout {
+  static constexpr int SBO_A = (D / 8) * kTcLboA;  // bytes between 8-row groups of A
+  static constexpr int SBO_B = (D / 8) * kTcLboB;
+  static constexpr int A_BYTES = (kTcM / 8) * SBO_A;
+  static constexpr int B_BYTES = (D / 8) * SBO_B;
+  static constexpr int oBh = 0, oBl = B_BYTES, oAh = 2 * B_BYTES, oAl = 2 * B_BYTES + A_BYTES;
+  static constexpr int oInv = 2 * B_BYTES + 2 * A_BYTES;  // kTcM floats
+  static constexpr int kBytes = oInv + kTcM * 4;
+};
+
+__device__ __forceinline__ uint32_t a_off(int m, int k, int sbo, int lbo) {
+  return (uint32_t)((m >> 3) * sbo + (k >> 3) * lbo + (m & 7) * 16 + (k & 7) * 2);
+}
+
+// UMMA shared-memory descriptor: K-major, no swizzle (canonical layout of
+// 8-row x 16-byte core matrices; LBO = distance between K-adjacent core
+// matrices, SBO = distance between M/N-adjacent 8-row groups), version 1.
+__device__ __forceinline__ uint64_t umma_desc(uint32_t saddr, uint32_t lbo, uint32_t sbo) {
+  uint64_t d = (uint64_t)((saddr >> 4) & 0x3FFFu);
+  d |= (uint64_t)((lbo >> 4) & 0x3FFFu) << 16;
+  d |= (uint64_t)((sbo >> 4) & 0x3FFFu) << 32;
+  d |= (uint64_t)1 << 46;
+  return d;
+}
+
+__device__ __forceinline__ void umma_f16(uint32_t tmem, uint64_t adesc, uint64_t bdesc, uint32_t idesc,
+                                         uint32_t accum) {
+  const uint32_t z = 0u;
+  asm volatile(
+      "{\n .reg .pred p;\n setp.ne.b32 p, %4, 0;\n"
+      " tcgen05.mma.cta_group::1.kind::f16 [%0], %1, %2, %3, {%5, %6, %7, %8}, p;\n}\n" ::"r"(tmem),
+      "l"(adesc), "l"(bdesc), "r"(idesc), "r"(accum), "r"(z), "r"(z), "r"(z), "r"(z));
+}
+
+__device__ __forceinline__ void tmem_ld32(uint32_t taddr, uint32_t (&v)[32]) {
+  asm volatile(
+      "tcgen05.ld.sync.aligned.32x32b.x32.b32 {%0, %1, %2, %3, %4, %5, %6, %7, %8, %9, %10, %11, %12, %13, "
+      "%14, %15, %16, %17, %18, %19, %20, %21, %22, %23, %24, %25, %26, %27, %28, %29, %30, %31}, [%32];\n"
+      : "=r"(v[0]), "=r"(v[1]), "=r"(v[2]), "=r"(v[3]), "=r"(v[4]), "=r"(v[5]), "=r"(v[6]), "=r"(v[7]),
+        "=r"(v[8]), "=r"(v[9]), "=r"(v[10]), "=r"(v[11]), "=r"(v[12]), "=r"(v[13]), "=r"(v[14]), "=r"(v[15]),
+        "=r"(v[16]), "=r"(v[17]), "=r"(v[18]), "=r"(v[19]), "=r"(v[20]), "=r"(v[21]), "=r"(v[22]), "=r"(v[23]),
+        "=r"(v[24]), "=r"(v[25]), "=r"(v[26]), "=r"(v[27]), "=r"(v[28]), "=r"(v[29]), "=r"(v[30]), "=r"(v[31])
+      : "r"(taddr));
+}
+
+__device__ __forceinline__ bool mbar_try(uint32_t bar, uint32_t parity) {
+  uint32_t ok;
+  asm volatile(
+      "{\n .reg .pred p;\n mbarrier.try_wait.parity.shared::cta.b64 p, [%1], %2;\n selp.u32 %0, 1, 0, p;\n}\n"
+      : "=r"(ok)
+      : "r"(bar), "r"(parity)
+      : "memory");
+  return ok != 0;
+}
+
+template <int D, int BM, int DT>
+__global__ void __launch_bounds__(kTcThreads, 1) encode_dense_tc_kernel(DenseParams p, unsigned *faults,
+                                                                        int64_t ntiles) {
+  using L = TcLayout<D>;
+  constexpr int J = D / 32;          // elements per lane per row in the loads
+  constexpr int HALF = D / 2;        // columns per epilogue thread
+  constexpr int K = 1 << BM;
+  extern __shared__ __align__(1024) unsigned char smem[];
+  __shared__ __align__(8) uint64_t s_bar;
+  __shared__ uint32_t s_tmem;
+  const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
+  const uint32_t sbase = (uint32_t)__cvta_generic_to_shared(smem);
+  const uint32_t bar = (uint32_t)__cvta_generic_to_shared(&s_bar);
+  float *s_inv = reinterpret_cast<float *>(smem + L::oInv);
+
+  // ---- once: TMEM columns, the mbarrier, Pi's halves (scaled by 16)
+  if (warp == 0) {
+    const uint32_t dst = (uint32_t)__cvta_generic_to_shared(&s_tmem);
+    asm volatile("tcgen05.alloc.cta_group::1.sync.aligned.shared::cta.b32 [%0], %1;\n" ::"r"(dst), "r"((uint32_t)D)
+                 : "memory");
+    asm volatile("tcgen05.relinquish_alloc_permit.cta_group::1.sync.aligned;\n" ::: "memory");
+  }
+  if (tid == 0) {
+    asm volatile("mbarrier.init.shared::cta.b64 [%0], 1;\n" ::"r"(bar) : "memory");
+    asm volatile("fence.mbarrier_init.release.cluster;\n" ::: "memory");
+  }
+  for (int i = tid; i < D * D; i += kTcThreads) {
+    const int n = i / D, k = i % D;
+    const float v = 16.0f * __ldg(p.rot + i);
+    const __half h = __float2half_rn(v);
+    const __half l = __float2half_rn(v - __half2float(h));
+    const uint32_t o = a_off(n, k, L::SBO_B, kTcLboB);
+    *reinterpret_cast<__half *>(smem + L::oBh + o) = h;
+    *reinterpret_cast<__half *>(smem + L::oBl + o) = l;
+  }
+  uint32_t P[K / 2 > 0 ? K / 2 : 1];
+#pragma unroll
+  for (int m = 0; m + 1 < K / 2; ++m) P[m] = __float_as_uint(__ldg(p.thr + K / 2 + m));
+  asm volatile("fence.proxy.async.shared::cta;\n" ::: "memory");
+  asm volatile("tcgen05.fence::before_thread_sync;\n" ::: "memory");
+  __syncthreads();
+  asm volatile("tcgen05.fence::after_thread_sync;\n" ::: "memory");
+  const uint32_t tmem = s_tmem;
+  const uint32_t idesc = (1u << 4) | ((uint32_t)(D >> 3) << 17) | ((uint32_t)(kTcM >> 4) << 24);
+  bool dead = false;
+
+  for (int64_t tile = blockIdx.x, it = 0; tile < ntiles; tile += gridDim.x, ++it) {
+    // ---- phase 1: rows warp * 16 + [0, 16), in two batches of 8 whose
+    // loads are all in flight before the first row is used
+#pragma unroll 1
+    for (int rb = 0; rb < 16; rb += 8) {
+      float xr[8][J];
+#pragma unroll
+      for (int r = 0; r < 8; ++r) {
+        const int64_t v = tile * kTcM + warp * 16 + rb + r;
+        int64_t b, h, n;
+        bhn(p, v < p.nvec ? v : 0, b, h, n);
+        const int64_t xoff = b * p.xsb + h * p.xsh + n * p.xsn;
+#pragma unroll
+        for (int j = 0; j < J; ++j) xr[r][j] = v < p.nvec ? load_elem(p.x, DT, xoff + lane + 32 * j) : 0.0f;
+      }
+#pragma unroll
+      for (int r = 0; r < 8; ++r) {
+        const int m = warp * 16 + rb + r;
+        const int64_t v = tile * kTcM + m;
+        float sq[J];
+#pragma unroll
+        for (int j = 0; j < J; ++j) sq[j] = __fmul_rn(xr[r][j], xr[r][j]);
+#pragma unroll
+        for (int st = J / 2; st >= 1; st >>= 1) {
+#pragma unroll
+          for (int j = 0; j < st; ++j) sq[j] = __fadd_rn(sq[j], sq[j + st]);
+        }
+        float s = sq[0];
+#pragma unroll
+        for (int hh = 16; hh >= 1; hh >>= 1) s = __fadd_rn(s, __shfl_down_sync(dev::kFull, s, hh));
+        const float nrm = __fsqrt_rn(__shfl_sync(dev::kFull, s, 0));
+        // 2^(13 - floor(log2 n)) for a normal n > 0, else 1
+        const int ex = ((__float_as_int(nrm) >> 23) & 0xff) - 127;
+        const bool normal = nrm > 0.0f && ex > -127;
+        const float sc = normal ? __int_as_float((127 + 13 - ex) << 23) : 1.0f;
+#pragma unroll
+        for (int j = 0; j < J; ++j) {
+          const int k = lane + 32 * j;
+          const float xs = xr[r][j] * sc;
+          const __half hi = __float2half_rn(xs);
+          const __half lo = __float2half_rn(xs - __half2float(hi));
+          const uint32_t o = a_off(m, k, L::SBO_A, kTcLboA);
+          *reinterpret_cast<__half *>(smem + L::oAh + o) = hi;
+          *reinterpret_cast<__half *>(smem + L::oAl + o) = lo;
+        }
+        if (lane == 0) {
+          s_inv[m] = normal ? __frcp_rn(__fmul_rn(16.0f * sc, nrm)) : 0.0f;
+          if (v < p.nvec) {
+            int64_t b, h, n;
+            bhn(p, v, b, h, n);
+            p.norms[b * p.osb + h * p.osh + n * p.osn] = nrm;
+          }
+        }
+      }
+    }
+    asm volatile("fence.proxy.async.shared::cta;\n" ::: "memory");
+    __syncthreads();
+
+    // ---- phase 2: Y = Xh Ph + Xh Pl + Xl Ph into TMEM
+    if (tid == 0) {
+      asm volatile("tcgen05.fence::after_thread_sync;\n" ::: "memory");
+#pragma unroll 1
+      for (int ks = 0; ks < D / 16; ++ks) {
+        const uint64_t ah = umma_desc(sbase + L::oAh + ks * 2 * kTcLboA, kTcLboA, L::SBO_A);
+        const uint64_t al = umma_desc(sbase + L::oAl + ks * 2 * kTcLboA, kTcLboA, L::SBO_A);
+        const uint64_t bh = umma_desc(sbase + L::oBh + ks * 2 * kTcLboB, kTcLboB, L::SBO_B);
+        const uint64_t bl = umma_desc(sbase + L::oBl + ks * 2 * kTcLboB, kTcLboB, L::SBO_B);
+        umma_f16(tmem, ah, bh, idesc, ks > 0 ? 1u : 0u);
+        umma_f16(tmem, ah, bl, idesc, 1u);
+        umma_f16(tmem, al, bh, idesc, 1u);
+      }
+      asm volatile("tcgen05.commit.cta_group::1.mbarrier::arrive::one.shared::cluster.b64 [%0];\n" ::"r"(bar)
+                   : "memory");
+    }
+    // bounded wait for the MMAs (phase parity = tile count & 1)
+    if (!dead) {
+      const uint32_t par = (uint32_t)(it & 1);
+      uint64_t t0 = 0;
+      for (uint32_t spin = 0; !mbar_try(bar, par); ++spin) {
+        if ((spin & 255u) == 255u) {
+          uint64_t now;
+          asm volatile("mov.u64 %0, %%globaltimer;\n" : "=l"(now));
+          if (t0 == 0) {
+            t0 = now;
+          } else if (now - t0 > 1000000000ull) {
+            atomicOr(faults, kFaultTimeout);
+            dead = true;
+            break;
+          }
+        }
+      }
+    }
+    asm volatile("tcgen05.fence::after_thread_sync;\n" ::: "memory");
+
+    // ---- phase 3: half a record per thread, 32 columns (BM words of
+    // codes) at a time
+    {
+      const int q4 = warp & 3, hf = warp >> 2;
+      const int m = 32 * q4 + lane;
+      const int64_t v = tile * kTcM + m;
+      const float inv = s_inv[m];
+      uint8_t *dst = nullptr;
+      if (v < p.nvec) {
+        int64_t b, h, n;
+        bhn(p, v, b, h, n);
+        dst = p.codes + (b * p.osb + h * p.osh + n * p.osn) * (D * BM / 8) + hf * (HALF * BM / 8);
+      }
+#pragma unroll 1
+      for (int c = 0; c < HALF / 32; ++c) {
+        uint32_t y[32];
+        tmem_ld32(tmem + ((uint32_t)(32 * q4) << 16) + (uint32_t)(hf * HALF + 32 * c), y);
+        asm volatile("tcgen05.wait::ld.sync.aligned;\n" ::: "memory");
+        uint32_t W[BM];
+#pragma unroll
+        for (int w = 0; w < BM; ++w) W[w] = 0u;
+#pragma unroll
+        for (int i = 0; i < 32; ++i) {
+          const float u = __fmul_rn(__uint_as_float(y[i]), inv);
+          int idx;
+          if constexpr (BM == 1) {
+            idx = u > 0.0f ? 1 : 0;
+          } else {
+            idx = dev::quantize_sym<BM>(u, P);
+          }
+          dev::put_field<BM>(W, i, (uint32_t)idx);
+        }
+        if (dst) dev::store_words<BM>(dst + c * 4 * BM, W);
+      }
+    }
+    asm volatile("tcgen05.fence::before_thread_sync;\n" ::: "memory");
+    __syncthreads();
+  }
+  if (warp == 0) {
+    asm volatile("tcgen05.fence::after_thread_sync;\n" ::: "memory");
+    asm volatile("tcgen05.dealloc.cta_group::1.sync.aligned.b32 %0, %1;\n" ::"r"(tmem), "r"((uint32_t)D) : "memory");
+  }
+}
+
+template <int D, int BM, int DT>
+cudaError_t run_dense_tc(const DenseParams &p, unsigned *faults, cudaStream_t s) {
+  auto kern = encode_dense_tc_kernel<D, BM, DT>;
+  constexpr int smem = TcLayout<D>::kBytes;
+  cudaError_t e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, smem);
+  if (e != cudaSuccess) return e;
+  const int64_t ntiles = (p.nvec + kTcM - 1) / kTcM;
+  const int64_t grid = ntiles < decode_ctas() ? ntiles : decode_ctas();
+  kern<<<(unsigned)grid, kTcThreads, smem, s>>>(p, faults, ntiles);
+  return cudaGetLastError();
+}
+
+template <int D, int DT>
+cudaError_t dense_tc_bits(const DenseParams &p, unsigned *faults, cudaStream_t s) {
+  switch (p.bm) {
+    case 1: return run_dense_tc<D, 1, DT>(p, faults, s);
+    case 2: return run_dense_tc<D, 2, DT>(p, faults, s);
+    case 3: return run_dense_tc<D, 3, DT>(p, faults, s);
+    case 4: return run_dense_tc<D, 4, DT>(p, faults, s);
+  }
+  return cudaErrorInvalidValue;
+}
+
+template <int D>
+cudaError_t dense_tc_dtype(const DenseParams &p, unsigned *faults, cudaStream_t s) {
+  switch (p.dtype) {
+    case TQ_F32: return dense_tc_bits<D, TQ_F32>(p, faults, s);
+    case TQ_BF16: return dense_tc_bits<D, TQ_BF16>(p, faults, s);
+    case TQ_F16: return dense_tc_bits<D, TQ_F16>(p, faults, s);
+  }
+  return cudaErrorInvalidValue;
+}
+
 }  // namespace
 
 cudaError_t launch_encode_dense(const EncodeArgs &a, cudaStream_t s) {
@@ -233,6 +538,13 @@ cudaError_t launch_encode_dense(const EncodeArgs &a, cudaStream_t s) {
   p.bm = a.q.bm;
   p.kcb = a.q.d * a.q.bm / 8;
   p.prod = a.q.prod;
+  // large TurboQuant_mse batches at d = 64 / 128: the rotation on tcgen05
+  if (!p.prod && (p.d == 64 || p.d == 128) && p.nvec >= 8 * kTcM) {
+    unsigned *faults = nullptr;
+    cudaError_t e = fault_word(&faults);
+    if (e != cudaSuccess) return e;
+    return p.d == 64 ? dense_tc_dtype<64>(p, faults, s) : dense_tc_dtype<128>(p, faults, s);
+  }
   const int64_t blocks = (p.nvec + kDnWarps - 1) / kDnWarps;
   encode_dense_kernel<<<(unsigned)blocks, kDnWarps * 32, 0, s>>>(p);
   return cudaGetLastError();

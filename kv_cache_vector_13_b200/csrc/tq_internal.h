@@ -95,6 +95,10 @@ size_t decode_workspace_floats(int B, int Hq, int Hkv, bool prod, int ctas);
 constexpr unsigned kFaultTimeout = 1u;
 constexpr unsigned kFaultSmemLayout = 2u;
 
+// Device address of the current device's fault word (for kernels that set
+// bits in it).
+cudaError_t fault_word(unsigned **ptr);
+
 // Reads the current device's fault word and clears it (synchronous).
 cudaError_t take_device_faults(unsigned *faults);
 

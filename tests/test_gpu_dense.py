@@ -5,10 +5,11 @@ the exact product in float64.  So:
 - norms are bit-exact (the same canonical fp32 fold-halves sum);
 - a code may differ from the oracle's only for a coordinate whose exact u
   lies within the device's rounding band of a threshold,
-  band = (d + 2) 2^-24 sum_k |Pi_jk x_k| / n + 2^-23 |u|
-  (Higham's bound for a d-term dot product, plus the scale and the
-  product's rounding); every such difference is checked against it and the
-  count is reported;
+  band = (6 d + 16) 2^-24 sum_k |Pi_jk x_k| / n + 2^-22 |u|
+  (the tensor-core path: x and Pi each carried to 22 bits by fp16 halves,
+  three products, 3d fp32 additions that may truncate; the CUDA-core path's
+  fp32 dot product is well inside it); every such difference is checked
+  against it and the count is reported;
 - prod: ||r|| within 1e-5 relative, and a QJL sign may differ only where
   |(S r)_k| is within the fp32 dot-product band plus what the residual's
   own band can move it.
@@ -35,7 +36,7 @@ def u_band(oq, x):
     P = oq.Pi.astype(np.float64)
     absdot = np.abs(x) @ np.abs(P).T
     u = (x @ P.T) / np.where(n > 0, n, 1.0)[:, None]
-    band = (oq.d + 2) * 2.0 ** -24 * absdot / np.where(n > 0, n, 1.0)[:, None] + 2.0 ** -23 * np.abs(u)
+    band = (6 * oq.d + 16) * 2.0 ** -24 * absdot / np.where(n > 0, n, 1.0)[:, None] + 2.0 ** -22 * np.abs(u)
     return band
 
 
