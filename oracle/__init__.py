@@ -18,6 +18,7 @@ Modules
   quantizer  encode (TurboQuant_mse / TurboQuant_prod), bit packing, dequant
   attention  decode attention on the packed cache (float64 and fp32)
   search     top-k vector search by the estimated inner product
+  split      outlier-channel split: two channel groups at two bit widths
   metrics    distortion (MSE) and inner-product bias
 
 Parity unpinned: the GPU's fp32 summation order for the QJL projection
@@ -27,4 +28,4 @@ are counted by the tests), and the Beta-codebook distortion values (the
 pages print none; only the numerical integral pins them).
 """
 
-from . import prng, codebook, rotation, quantizer, attention, metrics, search  # noqa: F401
+from . import prng, codebook, rotation, quantizer, attention, metrics, search, split  # noqa: F401
