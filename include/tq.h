@@ -96,6 +96,11 @@ typedef struct {
   const float *qjl_S;      /* d*d fp32 row-major, prod only, else NULL */
   const float *rot;        /* d*d fp32 row-major Pi, 16-byte aligned (dense
                               rotation only, else NULL): y = Pi x */
+  const int32_t *channels; /* DEVICE, d entries or NULL: coordinate i of the
+                              quantized vector is element channels[i] of the
+                              input row (a channel group of a wider head,
+                              the outlier-channel split); dense rotation
+                              only.  NULL = elements 0..d-1. */
 } tq_quantizer;
 
 /* A packed cache: records addressed as
@@ -246,6 +251,30 @@ tq_status tq_decode_attention_noalloc(const tq_quantizer *kq, const tq_quantizer
                                       const tq_cache_view *k, const tq_cache_view *v,
                                       float softmax_scale, float *out,
                                       float *scores_out, tq_stream_t stream);
+
+/* Decode attention over an outlier-channel split cache ("TurboQuant của
+ * Google", the correction in the experiments section: a head's channels in
+ * two groups, the outlier channels at a higher bit width).  Each cache is
+ * two caches, one per channel group: group 0 of the keys is quantized by
+ * kq[0] (its channels list gives the group's head-dim channels), group 1 by
+ * kq[1], likewise the values; both groups use the dense rotation and
+ * together cover the d = kq[0].d + kq[1].d channels of the head once.
+ * Scores are the two groups' asymmetric estimates added,
+ *   s_j = est_0(q[ch_0], k_0j) + est_1(q[ch_1], k_1j),
+ * the softmax is over all L_b tokens, and each value group is summed in its
+ * own rotated basis and rotated back into its channels of out[B][Hq][d].
+ * The rest as for tq_decode_attention (q: [B][Hq][d]; GQA; seq_lens;
+ * softmax_scale); d <= 256.  workspace: DEVICE, at least
+ * tq_decode_split_workspace_bytes(B, Hq, seq_len) bytes, 16-byte aligned.
+ * Plain CUDA-core kernels (one pass for the scores, one for softmax and
+ * values). */
+size_t tq_decode_split_workspace_bytes(int32_t B, int32_t Hq, int64_t seq_len);
+tq_status tq_decode_attention_split(const tq_quantizer kq[2], const tq_quantizer vq[2],
+                                    const void *q, tq_dtype q_dtype, int32_t B, int32_t Hq,
+                                    int32_t Hkv, int64_t seq_len, const int32_t *seq_lens,
+                                    const tq_cache_view k[2], const tq_cache_view v[2],
+                                    float softmax_scale, float *out, void *workspace,
+                                    size_t workspace_bytes, tq_stream_t stream);
 
 /* Workspace of tq_search_topk, in bytes (0 when a size is out of range). */
 size_t tq_search_workspace_bytes(int32_t n_q, int64_t n_db, int32_t d);

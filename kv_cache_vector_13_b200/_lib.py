@@ -23,6 +23,7 @@ EXPORTS = (
     "tq_encode", "tq_dequant", "tq_decode_workspace_bytes", "tq_decode_attention",
     "tq_append_decode_attention", "tq_decode_attention_noalloc",
     "tq_search_workspace_bytes", "tq_search_topk",
+    "tq_decode_split_workspace_bytes", "tq_decode_attention_split",
     "tq_check", "tq_status_string", "tq_last_error", "tq_version",
 )
 
@@ -31,7 +32,7 @@ class TqQuantizer(ctypes.Structure):
     _fields_ = [
         ("d", c_int32), ("bits", c_int32), ("variant", c_int32), ("rotation", c_int32),
         ("centroids", c_void_p), ("thresholds", c_void_p), ("signs", c_void_p), ("qjl_S", c_void_p),
-        ("rot", c_void_p),
+        ("rot", c_void_p), ("channels", c_void_p),
     ]
 
 
@@ -101,6 +102,12 @@ def lib() -> ctypes.CDLL:
     L.tq_search_topk.argtypes = [POINTER(TqQuantizer), POINTER(TqCacheView), c_int64, c_void_p, c_int32, c_int32,
                                  c_int32, c_void_p, c_void_p, c_void_p, c_size_t, c_void_p]
     L.tq_search_topk.restype = c_int32
+    L.tq_decode_split_workspace_bytes.argtypes = [c_int32, c_int32, c_int64]
+    L.tq_decode_split_workspace_bytes.restype = c_size_t
+    L.tq_decode_attention_split.argtypes = [
+        POINTER(TqQuantizer), POINTER(TqQuantizer), c_void_p, c_int32, c_int32, c_int32, c_int32, c_int64,
+        c_void_p, POINTER(TqCacheView), POINTER(TqCacheView), c_float, c_void_p, c_void_p, c_size_t, c_void_p]
+    L.tq_decode_attention_split.restype = c_int32
     L.tq_check.argtypes = [c_void_p]
     L.tq_check.restype = c_int32
     L.tq_status_string.argtypes = [c_int32]

@@ -71,7 +71,8 @@ class Quantizer:
     """Device-resident parameters of one TurboQuant quantizer."""
 
     def __init__(self, d: int, bits: int, variant: str = "mse", seed_rot: int = 0,
-                 seed_qjl: int = 1, dist: str = "gauss", device="cuda", rotation: str = "hadamard"):
+                 seed_qjl: int = 1, dist: str = "gauss", device="cuda", rotation: str = "hadamard",
+                 channels: Optional[torch.Tensor] = None):
         assert variant in ("mse", "prod") and rotation in ("hadamard", "dense")
         self.d, self.bits, self.variant = d, bits, variant
         self.seed_rot, self.seed_qjl, self.dist, self.rotation = seed_rot, seed_qjl, dist, rotation
@@ -86,10 +87,11 @@ class Quantizer:
         self.signs = torch.from_numpy(make_signs(seed_rot, d)).to(dev)
         self.S = torch.from_numpy(make_qjl(seed_qjl, d)).to(dev) if variant == "prod" else None
         self.rot = torch.from_numpy(make_rotation(seed_rot, d)).to(dev) if rotation == "dense" else None
+        self.channels = None if channels is None else channels.to(device=dev, dtype=torch.int32).contiguous()
         self._c = L.TqQuantizer(d, bits, L.TQ_PROD if variant == "prod" else L.TQ_MSE,
                                 L.TQ_ROT_DENSE if rotation == "dense" else L.TQ_ROT_HADAMARD,
                                 _ptr(self.centroids), _ptr(self.thresholds), _ptr(self.signs), _ptr(self.S),
-                                _ptr(self.rot))
+                                _ptr(self.rot), _ptr(self.channels))
 
     @property
     def prod(self) -> bool:
@@ -258,6 +260,60 @@ def decode_attention(kq: Quantizer, vq: Quantizer, q: torch.Tensor, kcache: Pack
     _, Hkv, N = kcache.shape
     op = DecodeAttention(kq, vq, B, Hq, Hkv, N, device=q.device)
     return op(q, kcache, vcache, scale=scale, seq_lens=seq_lens, scores=scores).clone()
+
+
+class SplitQuantizer:
+    """Outlier-channel split of a d-channel head: group 0 (the outlier
+    channels, ascending) at bits_o, group 1 (the rest) at bits_r, each its
+    own dense-rotation quantizer reading its channels of the head."""
+
+    def __init__(self, d: int, channels, bits_o: int, bits_r: int, variant: str = "mse", seed_rot: int = 0,
+                 seed_qjl: int = 1, device="cuda"):
+        ch = torch.as_tensor(channels, dtype=torch.int64).sort().values
+        mask = torch.ones(d, dtype=torch.bool)
+        mask[ch] = False
+        rest = torch.nonzero(mask)[:, 0]
+        self.d, self.channels, self.rest = d, ch, rest
+        self.groups = (
+            Quantizer(ch.numel(), bits_o, variant, seed_rot=seed_rot, seed_qjl=seed_qjl, device=device,
+                      rotation="dense", channels=ch),
+            Quantizer(rest.numel(), bits_r, variant, seed_rot=seed_rot + 1, seed_qjl=seed_qjl + 1, device=device,
+                      rotation="dense", channels=rest))
+
+    def c_array(self):
+        return (L.TqQuantizer * 2)(self.groups[0].c_struct(), self.groups[1].c_struct())
+
+
+def encode_split(sq: SplitQuantizer, x: torch.Tensor, stream=None):
+    """tq_encode of both channel groups of x ([B, H, N, d] or fewer dims):
+    (cache of group 0, cache of group 1)."""
+    return tuple(encode(g, x, stream=stream) for g in sq.groups)
+
+
+class DecodeAttentionSplit:
+    """tq_decode_attention_split with its workspace allocated once."""
+
+    def __init__(self, kq: SplitQuantizer, vq: SplitQuantizer, B: int, Hq: int, Hkv: int, seq_len: int,
+                 device="cuda"):
+        self.kq, self.vq, self.B, self.Hq, self.Hkv, self.seq_len = kq, vq, B, Hq, Hkv, seq_len
+        nb = int(L.lib().tq_decode_split_workspace_bytes(B, Hq, seq_len))
+        self.workspace = torch.empty(max(nb, 16), dtype=torch.uint8, device=device)
+        self.ws_bytes = nb
+        self.out = torch.empty((B, Hq, kq.d), dtype=torch.float32, device=device)
+
+    def __call__(self, q: torch.Tensor, kcaches, vcaches, scale: Optional[float] = None,
+                 seq_lens: Optional[torch.Tensor] = None, stream=None) -> torch.Tensor:
+        B, Hq, d = q.shape
+        assert (B, Hq, d) == (self.B, self.Hq, self.kq.d) and q.is_contiguous() and q.dtype in _DTYPES
+        if scale is None:
+            scale = 1.0 / math.sqrt(d)
+        kv = (L.TqCacheView * 2)(kcaches[0].view(), kcaches[1].view())
+        vv = (L.TqCacheView * 2)(vcaches[0].view(), vcaches[1].view())
+        ka, va = self.kq.c_array(), self.vq.c_array()
+        L.check(L.lib().tq_decode_attention_split(
+            ka, va, q.data_ptr(), _DTYPES[q.dtype], B, Hq, self.Hkv, self.seq_len, _ptr(seq_lens), kv, vv,
+            float(scale), self.out.data_ptr(), self.workspace.data_ptr(), self.ws_bytes, _stream(stream)))
+        return self.out
 
 
 class Search:

@@ -44,6 +44,7 @@ struct DenseParams {
   const float *thr;
   const float *rot;
   const float *S;
+  const int32_t *chan;  // input element of each coordinate, or NULL
   int d, bm, kcb;
   bool prod;
   float *out;  // dequant
@@ -102,7 +103,7 @@ __global__ void __launch_bounds__(kDnWarps * 32) encode_dense_kernel(DenseParams
 #pragma unroll
   for (int j = 0; j < kDnJ; ++j) {
     const int k = lane + 32 * j;
-    const float a = k < d ? load_elem(p.x, p.dtype, xoff + k) : 0.0f;
+    const float a = k < d ? load_elem(p.x, p.dtype, xoff + (p.chan ? __ldg(p.chan + k) : k)) : 0.0f;
     if (k < d) xs[k] = a;
     sq[j] = __fmul_rn(a, a);
   }
@@ -534,12 +535,13 @@ cudaError_t launch_encode_dense(const EncodeArgs &a, cudaStream_t s) {
   p.thr = a.q.thresholds;
   p.rot = a.q.rot;
   p.S = a.q.S;
+  p.chan = a.q.channels;
   p.d = a.q.d;
   p.bm = a.q.bm;
   p.kcb = a.q.d * a.q.bm / 8;
   p.prod = a.q.prod;
   // large TurboQuant_mse batches at d = 64 / 128: the rotation on tcgen05
-  if (!p.prod && (p.d == 64 || p.d == 128) && p.nvec >= 8 * kTcM) {
+  if (!p.prod && !p.chan && (p.d == 64 || p.d == 128) && p.nvec >= 8 * kTcM) {
     unsigned *faults = nullptr;
     cudaError_t e = fault_word(&faults);
     if (e != cudaSuccess) return e;

@@ -262,6 +262,9 @@ tq_status check_quantizer(const tq_quantizer *q, const char *name, tq::QuantPara
   out->signs = q->signs;
   out->S = q->qjl_S;
   out->rot = dense ? q->rot : nullptr;
+  if (q->channels && !dense)
+    return fail(TQ_EUNSUPPORTED, "%s: a channel list needs the dense rotation", name);
+  out->channels = q->channels;
   out->sqrt_d = (float)std::sqrt((double)q->d);
   return TQ_OK;
 }
@@ -604,6 +607,68 @@ tq_status tq_decode_attention_noalloc(const tq_quantizer *kq, const tq_quantizer
   }
   return tq_decode_attention(kq, vq, q, q_dtype, B, Hq, Hkv, seq_len, seq_lens, k, v, softmax_scale, out,
                              scores_out, ws, need, stream);
+}
+
+size_t tq_decode_split_workspace_bytes(int32_t B, int32_t Hq, int64_t seq_len) {
+  if (B <= 0 || Hq <= 0 || seq_len <= 0) return 0;
+  return (size_t)B * Hq * (size_t)seq_len * sizeof(float);
+}
+
+tq_status tq_decode_attention_split(const tq_quantizer kq[2], const tq_quantizer vq[2], const void *q,
+                                    tq_dtype q_dtype, int32_t B, int32_t Hq, int32_t Hkv, int64_t seq_len,
+                                    const int32_t *seq_lens, const tq_cache_view k[2], const tq_cache_view v[2],
+                                    float softmax_scale, float *out, void *workspace, size_t workspace_bytes,
+                                    tq_stream_t stream) {
+  const char *name = "tq_decode_attention_split";
+  if (!kq || !vq || !k || !v) return fail(TQ_EINVAL, "%s: NULL quantizer or cache array", name);
+  tq::SplitDecodeArgs a{};
+  for (int g = 0; g < 2; ++g) {
+    tq_status st = check_quantizer(&kq[g], name, &a.kq[g]);
+    if (st != TQ_OK) return st;
+    st = check_quantizer(&vq[g], name, &a.vq[g]);
+    if (st != TQ_OK) return st;
+    if (!a.kq[g].rot || !a.kq[g].channels || !a.vq[g].rot || !a.vq[g].channels)
+      return fail(TQ_EINVAL, "%s: every group needs the dense rotation and a channel list", name);
+    if (a.vq[g].prod && a.vq[g].bm == 0 && !a.vq[g].S) return fail(TQ_EINVAL, "%s: prod value group without S", name);
+  }
+  const int d = a.kq[0].d + a.kq[1].d;
+  if (a.vq[0].d + a.vq[1].d != d) return fail(TQ_EINVAL, "%s: key groups cover %d channels, value groups %d", name, d,
+                                               a.vq[0].d + a.vq[1].d);
+  if (d > 256) return fail(TQ_EINVAL, "%s: d=%d (at most 256)", name, d);
+  if (q_dtype != TQ_F32 && q_dtype != TQ_BF16 && q_dtype != TQ_F16)
+    return fail(TQ_EINVAL, "%s: q_dtype=%d", name, (int)q_dtype);
+  if (B < 0 || Hq < 0 || Hkv <= 0 || seq_len < 0 || Hq % Hkv) return fail(TQ_EINVAL, "%s: bad sizes", name);
+  if (Hq / Hkv > 8) return fail(TQ_EUNSUPPORTED, "%s: %d query heads per kv head (at most 8)", name, Hq / Hkv);
+  if (!std::isfinite(softmax_scale)) return fail(TQ_EINVAL, "%s: softmax_scale not finite", name);
+  if (B == 0 || Hq == 0) return TQ_OK;
+  if (!q || !out) return fail(TQ_EINVAL, "%s: q or out is NULL", name);
+  for (int g = 0; g < 2; ++g) {
+    tq_status st = check_view(&k[g], a.kq[g], name, seq_len > 0, &a.k[g]);
+    if (st != TQ_OK) return st;
+    st = check_view(&v[g], a.vq[g], name, seq_len > 0, &a.v[g]);
+    if (st != TQ_OK) return st;
+  }
+  if (seq_len == 0) {
+    const cudaError_t e = cudaMemsetAsync(out, 0, (size_t)B * Hq * d * sizeof(float), (cudaStream_t)stream);
+    return e == cudaSuccess ? TQ_OK : cuda_fail(e, name);
+  }
+  const size_t need = tq_decode_split_workspace_bytes(B, Hq, seq_len);
+  if (workspace_bytes < need || !workspace || !aligned(workspace, 16))
+    return fail(TQ_EWORKSPACE, "%s: workspace %zu bytes, need %zu", name, workspace_bytes, need);
+  a.q = q;
+  a.q_dtype = q_dtype;
+  a.B = B;
+  a.Hq = Hq;
+  a.Hkv = Hkv;
+  a.d = d;
+  a.seq_len = seq_len;
+  a.seq_lens = seq_lens;
+  a.scale = softmax_scale;
+  a.out = out;
+  a.ws = (float *)workspace;
+  const cudaError_t e = tq::launch_decode_split(a, (cudaStream_t)stream);
+  if (e != cudaSuccess) return cuda_fail(e, "tq_decode_attention_split launch");
+  return TQ_OK;
 }
 
 size_t tq_search_workspace_bytes(int32_t n_q, int64_t n_db, int32_t d) {

@@ -17,6 +17,7 @@ struct QuantParams {
   const int8_t *signs;      // d
   const float *S;           // d*d (prod)
   const float *rot;         // d*d row-major Pi (dense rotation), else NULL
+  const int32_t *channels;  // d input-element indices (channel group), else NULL
   float sqrt_d;             // fl32(sqrt(d)) (double sqrt rounded once)
 };
 
@@ -77,6 +78,20 @@ struct SearchArgs {
   int64_t *top_i;
   float *ws;
 };
+
+struct SplitDecodeArgs {
+  QuantParams kq[2], vq[2];
+  const void *q;
+  int q_dtype;
+  int B, Hq, Hkv, d;
+  int64_t seq_len;
+  const int32_t *seq_lens;
+  CacheView k[2], v[2];
+  float scale;
+  float *out;
+  float *ws;  // logits [B * Hq][seq_len], then per-head (max, sum)
+};
+cudaError_t launch_decode_split(const SplitDecodeArgs &a, cudaStream_t s);
 
 // Workspace of a search, in floats.
 size_t search_workspace_floats(int nq, int64_t n_db);
