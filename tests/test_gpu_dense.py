@@ -10,9 +10,11 @@ the exact product in float64.  So:
   three products, 3d fp32 additions that may truncate; the CUDA-core path's
   fp32 dot product is well inside it); every such difference is checked
   against it and the count is reported;
-- prod: ||r|| within 1e-5 relative, and a QJL sign may differ only where
-  |(S r)_k| is within the fp32 dot-product band plus what the residual's
-  own band can move it.
+- prod: the residual is the one the device's own indices give (an index
+  that flipped inside the band moves its coordinate of r by a centroid
+  step); ||r|| within 1e-5 relative of that residual's norm, and a QJL sign
+  may differ only where |(S r)_k| is within the fp32 dot-product band plus
+  what the residual's band and flipped indices can move it.
 Decode attention with dense keys and values (d = 128) is compared with the
 fp32 oracle at the 2e-3 tolerance of the other decode tests.
 """
@@ -57,18 +59,26 @@ def check_dense_records(qz, oq, x, got):
             assert np.all(gap[diff] <= band[diff]), "a code differs outside the rounding band"
     nq = 0
     if qz.prod:
+        # the residual the device formed: the exact u with the device's own
+        # indices (they differ from the oracle's only inside the band above,
+        # and a flipped index moves that coordinate of r by a centroid step)
+        gidx = (OQ.unpack_bits(got["codes"].reshape(enc["codes"].shape), d, qz.bm) if qz.bm else
+                np.zeros((n, d), np.int64))
+        c64 = oq.centroids.astype(np.float64)
+        r = enc["u"] - (c64[OQ.unpack_bits(enc["codes"], d, oq.bm)] if oq.bm else 0.0)
+        r_dev = enc["u"] - (c64[gidx] if oq.bm else 0.0)
         g = got["rnorms"].reshape(-1).astype(np.float64)
-        o = enc["rnorms"].astype(np.float64)
-        assert np.all(np.abs(g - o) <= 1e-5 * np.maximum(o, 1e-30))
+        want = np.sqrt(np.sum(r_dev ** 2, axis=1))
+        assert np.all(np.abs(g - want) <= 1e-5 * np.maximum(want, 1e-30) + 4 * d * 2.0 ** -24 * np.sqrt(
+            np.sum(band ** 2, axis=1)))
         gq = OQ.unpack_bits(got["qjl"].reshape(enc["qjl"].shape), d, 1)
         oqb = OQ.unpack_bits(enc["qjl"], d, 1)
         qd = gq != oqb
         nq = int(qd.sum())
         if nq:
-            idx = OQ.unpack_bits(enc["codes"], d, oq.bm)
-            r = enc["u"] - (oq.centroids.astype(np.float64)[idx] if oq.bm else 0.0)
             S = np.abs(oq.S.astype(np.float64))
-            zb = (d + 2) * 2.0 ** -24 * (np.abs(r) @ S.T) + (band + 2.0 ** -23 * np.abs(r)) @ S.T
+            zb = ((d + 2) * 2.0 ** -24 * (np.abs(r) @ S.T)
+                  + (band + 2.0 ** -23 * np.abs(r) + np.abs(r_dev - r)) @ S.T)
             assert np.all(np.abs(enc["z"])[qd] <= zb[qd]), "a QJL sign differs outside its band"
     return nd, nq
 
