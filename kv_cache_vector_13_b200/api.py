@@ -169,7 +169,8 @@ def encode(qz: Quantizer, x: torch.Tensor, out: Optional[PackedCache] = None, st
     dim must be contiguous; out defaults to a new [B, H, N] cache."""
     x4 = _as_bhn(x)
     B, H, N, d = x4.shape
-    assert d == qz.d and x4.stride(3) == 1 and x4.dtype in _DTYPES
+    # a channel-group quantizer reads its channels of a wider row
+    assert (d == qz.d if qz.channels is None else d >= qz.d) and x4.stride(3) == 1 and x4.dtype in _DTYPES
     if out is None:
         out = empty_cache(qz, B, H, N, x.device)
     v = out.view()

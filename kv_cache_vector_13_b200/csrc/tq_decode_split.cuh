@@ -416,62 +416,51 @@ __device__ __forceinline__ void load_k_slow(KBuf<KBM, KPROD> &c, const SplitPara
   }
 }
 
-// Per-lane pointers of the fast path (unit record strides) at chunk 0 of a
-// piece; chunk c adds c * kChunk records.
-template <int KBM, bool KPROD, int VBM>
+// The lane's record indices of the fast path (unit record strides) at chunk
+// 0 of a piece: the key rows' (token g8) and the value rows' (token 2 tig);
+// chunk c adds c * kChunk records.  The array bases stay in the kernel
+// parameters, so a piece keeps two indices live rather than six pointers.
 struct FastPtrs {
-  const uint8_t *kc;
-  const uint32_t *kj;
-  const float *kn, *kr, *vn;
-  const uint8_t *vc;
+  int64_t kr0, vr0;
 };
 
-template <int KBM, bool KPROD, int VBM>
-__device__ __forceinline__ FastPtrs<KBM, KPROD, VBM> fast_ptrs(const SplitParams &p, int64_t krec0, int64_t vrec0,
-                                                               int tig, int g8) {
-  constexpr int KCB = kD * KBM / 8, VCB = kD * VBM / 8;
-  FastPtrs<KBM, KPROD, VBM> f;
-  const int64_t kr0 = krec0 + g8, vr0 = vrec0 + g8;
-  f.kc = p.kc + kr0 * KCB + tig * (4 * KBM);
-  f.kj = KPROD ? reinterpret_cast<const uint32_t *>(p.kj + kr0 * (kD / 8)) + tig : nullptr;
-  f.kn = p.kn + kr0;
-  f.kr = KPROD ? p.kr + kr0 : nullptr;
-  f.vn = p.vn + vr0;
-  f.vc = p.vc + (vrec0 + 2 * tig) * VCB + g8 * (2 * VBM);
-  return f;
+__device__ __forceinline__ FastPtrs fast_ptrs(int64_t krec0, int64_t vrec0, int tig, int g8) {
+  return FastPtrs{krec0 + g8, vrec0 + 2 * tig};
 }
 
-// Key side of full chunk c through the fast-path pointers.
+// Key side of full chunk c through the fast-path indices.
 template <int KBM, bool KPROD, int VBM>
-__device__ __forceinline__ void load_k_fast(KBuf<KBM, KPROD> &c, const FastPtrs<KBM, KPROD, VBM> &f, int ci) {
+__device__ __forceinline__ void load_k_fast(KBuf<KBM, KPROD> &c, const SplitParams &p, const FastPtrs &f, int ci,
+                                            int tig, int g8) {
   constexpr int KCB = kD * KBM / 8;
-  const int64_t r0 = (int64_t)ci * kChunk;
+  const int64_t r0 = f.kr0 + (int64_t)ci * kChunk;
+  const int64_t v0 = f.vr0 - 2 * tig + g8 + (int64_t)ci * kChunk;  // the key rows' value norms
 #pragma unroll
   for (int ms = 0; ms < 2; ++ms) {
 #pragma unroll
     for (int r = 0; r < 2; ++r) {
       const int t = 16 * ms + 8 * r;
-      if constexpr (KBM > 0) load_k32<KBM>(f.kc + (r0 + t) * KCB, c.w[ms][r]);
+      if constexpr (KBM > 0) load_k32<KBM>(p.kc + (r0 + t) * KCB + tig * (4 * KBM), c.w[ms][r]);
       if constexpr (KPROD) {
-        c.qj[ms][r] = __ldg(f.kj + (r0 + t) * (kD / 32));
-        c.kr[ms][r] = __ldg(f.kr + r0 + t);
+        c.qj[ms][r] = __ldg(reinterpret_cast<const uint32_t *>(p.kj + (r0 + t) * (kD / 8)) + tig);
+        c.kr[ms][r] = __ldg(p.kr + r0 + t);
       }
-      c.kn[ms][r] = __ldg(f.kn + r0 + t);
-      c.vn[ms][r] = __ldg(f.vn + r0 + t);
+      c.kn[ms][r] = __ldg(p.kn + r0 + t);
+      c.vn[ms][r] = __ldg(p.vn + v0 + t);
     }
   }
 }
 
-// Value side of full chunk c through the fast-path pointers.
+// Value side of full chunk c through the fast-path indices.
 template <int KBM, bool KPROD, int VBM>
-__device__ __forceinline__ void load_v_fast(VBuf<VBM> &c, const FastPtrs<KBM, KPROD, VBM> &f, int ci, int g8) {
+__device__ __forceinline__ void load_v_fast(VBuf<VBM> &c, const SplitParams &p, const FastPtrs &f, int ci, int g8) {
   constexpr int VCB = kD * VBM / 8;
-  const int64_t r0 = (int64_t)ci * kChunk;
+  const int64_t r0 = f.vr0 + (int64_t)ci * kChunk;
 #pragma unroll
   for (int ms = 0; ms < 2; ++ms) {
 #pragma unroll
     for (int q4 = 0; q4 < 4; ++q4)
-      load_v16<VBM>(f.vc + (r0 + 16 * ms + (q4 & 1) + 8 * (q4 >> 1)) * VCB, c.w[ms][q4], g8);
+      load_v16<VBM>(p.vc + (r0 + 16 * ms + (q4 & 1) + 8 * (q4 >> 1)) * VCB + g8 * (2 * VBM), c.w[ms][q4], g8);
   }
 }
 
@@ -853,10 +842,17 @@ __device__ __forceinline__ void load_v_ring(VBuf<VBM> &c, const char *slot, int 
 
 // Warps per CTA: 12 with <= 4 query heads per kv head (the hi and lo query
 // halves share one MMA); 8 with more, whose extra fragments need the
-// registers.
+// registers.  The register-fed variant keeps the QJL term's query fragments
+// (S q') in shared memory, which leaves room for 12 warps with prod keys.
 template <bool PACK, bool KPROD, bool STAGED>
 __host__ __device__ constexpr int split_warps() {
-  return PACK ? (STAGED || !KPROD ? 12 : 8) : 8;
+  return PACK ? 12 : 8;
+}
+
+// Whether the QJL term's query fragments are read from shared memory.
+template <bool KPROD, bool STAGED>
+__host__ __device__ constexpr bool qs_in_smem() {
+  return KPROD && !STAGED;
 }
 
 template <int KBM, bool KPROD, int VBM, bool PACK, bool STAGED>
@@ -1033,8 +1029,12 @@ __global__ void __launch_bounds__(split_warps<PACK, KPROD, STAGED>() * 32, 1) de
     // lane's register order.  PACK: column n < 4 is the hi half of head n,
     // n >= 4 the lo half of head n - 4.  Else qf = hi and qf2 = lo of head
     // g8.  Lanes whose head is absent (fewer than 4 or 8 heads) hold zeros.
+    constexpr bool QS_SMEM = qs_in_smem<KPROD, STAGED>();
     uint32_t qf[8][2], qf2[PACK ? 1 : 8][2];
-    uint32_t qsf[KPROD ? 8 : 1][2], qsf2[(KPROD && !PACK) ? 8 : 1][2];
+    uint32_t qsf[(KPROD && !QS_SMEM) ? 8 : 1][2], qsf2[(KPROD && !PACK && !QS_SMEM) ? 8 : 1][2];
+    // QS_SMEM: the unit's S q' fragments at the start of the dynamic region,
+    // [S][hi 0 / lo 1][lane] words pairs (one 8-byte load per lane and step)
+    const uint2 *s_qs = reinterpret_cast<const uint2 *>(smem + (((dyn_base + 15u) & ~15u) - dyn_base));
     {
       const bool has = (PACK ? (g8 & 3) : g8) < gh;
       const uint4 *fr = p.frag + (int64_t)u * (kFragWords / 4) + lane;
@@ -1049,8 +1049,22 @@ __global__ void __launch_bounds__(split_warps<PACK, KPROD, STAGED>() * 32, 1) de
       for (int k = 0; k < 4; ++k) {
         put(qf, k, ld4(k));
         if constexpr (!PACK) put(qf2, k, ld4(4 + k));
-        if constexpr (KPROD) put(qsf, k, ld4((PACK ? 4 : 8) + k));
-        if constexpr (KPROD && !PACK) put(qsf2, k, ld4(12 + k));
+        if constexpr (KPROD && !QS_SMEM) put(qsf, k, ld4((PACK ? 4 : 8) + k));
+        if constexpr (KPROD && !PACK && !QS_SMEM) put(qsf2, k, ld4(12 + k));
+      }
+      if constexpr (QS_SMEM) {
+        // every thread copies its share; the barrier below (before the
+        // chunk loop) publishes them
+        uint2 *dst = const_cast<uint2 *>(s_qs);
+        for (int i = tid; i < 2 * 8 * 32; i += kThreads) {
+          const int ln = i & 31, S = (i >> 5) & 7, j2 = i >> 8;
+          if (PACK && j2 == 1) continue;
+          const bool h = (PACK ? ((ln >> 2) & 3) : (ln >> 2)) < gh;
+          const int w4 = (PACK ? 4 : (j2 ? 12 : 8)) + (S >> 1);
+          uint4 v = h ? __ldg(p.frag + (int64_t)u * (kFragWords / 4) + ln + w4 * 32) : make_uint4(0u, 0u, 0u, 0u);
+          dst[(S * 2 + j2) * 32 + ln] = (S & 1) ? make_uint2(v.z, v.w) : make_uint2(v.x, v.y);
+        }
+        __syncthreads();
       }
     }
 
@@ -1070,9 +1084,9 @@ __global__ void __launch_bounds__(split_warps<PACK, KPROD, STAGED>() * 32, 1) de
 
     KBuf<KBM, KPROD> kb;
     VBuf<VBM> vb;
-    FastPtrs<KBM, KPROD, VBM> fp{};
+    FastPtrs fp{};
     if constexpr (!STAGED) {
-      fp = fast_ptrs<KBM, KPROD, VBM>(p, kbase + t0, vbase + t0, tig, g8);
+      fp = fast_ptrs(kbase + t0, vbase + t0, tig, g8);
       // warm L2 up to the end of the first prefetch window
       if (unit && lane == 0 && c_begin + 1 < c_end) {
         const int64_t jp = t0 + (int64_t)(c_begin + 1) * kChunk;
@@ -1082,8 +1096,8 @@ __global__ void __launch_bounds__(split_warps<PACK, KPROD, STAGED>() * 32, 1) de
       }
       if (c_begin < c_end) {
         if (unit && c_begin < nfull) {
-          load_k_fast(kb, fp, c_begin);
-          load_v_fast(vb, fp, c_begin, g8);
+          load_k_fast<KBM, KPROD, VBM>(kb, p, fp, c_begin, tig, g8);
+          load_v_fast<KBM, KPROD, VBM>(vb, p, fp, c_begin, g8);
         } else {
           const int64_t j0 = t0 + (int64_t)c_begin * kChunk;
           const int nv = (int)min((int64_t)kChunk, t1 - j0);
@@ -1157,8 +1171,17 @@ __global__ void __launch_bounds__(split_warps<PACK, KPROD, STAGED>() * 32, 1) de
     a[1] = qjl_half2<2 * (S)>(qj[1]);                                             \
     a[2] = qjl_half2<2 * (S) + 1>(qj[0]);                                         \
     a[3] = qjl_half2<2 * (S) + 1>(qj[1]);                                         \
-    mma16816(cq, a, qsf[S][0], qsf[S][1]);                                        \
-    if constexpr (!PACK) mma16816(cq, a, qsf2[S][0], qsf2[S][1]);                 \
+    if constexpr (QS_SMEM) {                                                      \
+      const uint2 f = s_qs[((S) * 2) * 32 + lane];                                \
+      mma16816(cq, a, f.x, f.y);                                                  \
+      if constexpr (!PACK) {                                                      \
+        const uint2 f2 = s_qs[((S) * 2 + 1) * 32 + lane];                         \
+        mma16816(cq, a, f2.x, f2.y);                                              \
+      }                                                                           \
+    } else {                                                                      \
+      mma16816(cq, a, qsf[S][0], qsf[S][1]);                                      \
+      if constexpr (!PACK) mma16816(cq, a, qsf2[S][0], qsf2[S][1]);               \
+    }                                                                             \
   }
           TQ_QSTEP(0) TQ_QSTEP(1) TQ_QSTEP(2) TQ_QSTEP(3)
           TQ_QSTEP(4) TQ_QSTEP(5) TQ_QSTEP(6) TQ_QSTEP(7)
@@ -1196,7 +1219,7 @@ __global__ void __launch_bounds__(split_warps<PACK, KPROD, STAGED>() * 32, 1) de
       if constexpr (!STAGED) {
         if (more) {
           if (fast_next) {
-            load_k_fast(kb, fp, cn);
+            load_k_fast<KBM, KPROD, VBM>(kb, p, fp, cn, tig, g8);
           } else {
             const int64_t jn = t0 + (int64_t)cn * kChunk;
             load_k_slow(kb, p, kbase + jn * p.ksn, vbase + jn * p.vsn, (int)min((int64_t)kChunk, t1 - jn), tig,
@@ -1325,7 +1348,7 @@ __global__ void __launch_bounds__(split_warps<PACK, KPROD, STAGED>() * 32, 1) de
         // the value registers are free: start the next chunk's value loads
         if (more) {
           if (fast_next) {
-            load_v_fast(vb, fp, cn, g8);
+            load_v_fast<KBM, KPROD, VBM>(vb, p, fp, cn, g8);
           } else {
             const int64_t jn = t0 + (int64_t)cn * kChunk;
             load_v_slow(vb, p, vbase + jn * p.vsn, (int)min((int64_t)kChunk, t1 - jn), g8, tig);
