@@ -20,6 +20,7 @@
 #include "../../include/tq.h"
 #include "tq_device.cuh"
 #include "tq_internal.h"
+#include "tq_umma.cuh"
 
 #include <cuda_fp16.h>
 
@@ -249,51 +250,6 @@ struct TcLayout {
   static constexpr int kBytes = oInv + kTcM * 4;
 };
 
-__device__ __forceinline__ uint32_t a_off(int m, int k, int sbo, int lbo) {
-  return (uint32_t)((m >> 3) * sbo + (k >> 3) * lbo + (m & 7) * 16 + (k & 7) * 2);
-}
-
-// UMMA shared-memory descriptor: K-major, no swizzle (canonical layout of
-// 8-row x 16-byte core matrices; LBO = distance between K-adjacent core
-// matrices, SBO = distance between M/N-adjacent 8-row groups), version 1.
-__device__ __forceinline__ uint64_t umma_desc(uint32_t saddr, uint32_t lbo, uint32_t sbo) {
-  uint64_t d = (uint64_t)((saddr >> 4) & 0x3FFFu);
-  d |= (uint64_t)((lbo >> 4) & 0x3FFFu) << 16;
-  d |= (uint64_t)((sbo >> 4) & 0x3FFFu) << 32;
-  d |= (uint64_t)1 << 46;
-  return d;
-}
-
-__device__ __forceinline__ void umma_f16(uint32_t tmem, uint64_t adesc, uint64_t bdesc, uint32_t idesc,
-                                         uint32_t accum) {
-  const uint32_t z = 0u;
-  asm volatile(
-      "{\n .reg .pred p;\n setp.ne.b32 p, %4, 0;\n"
-      " tcgen05.mma.cta_group::1.kind::f16 [%0], %1, %2, %3, {%5, %6, %7, %8}, p;\n}\n" ::"r"(tmem),
-      "l"(adesc), "l"(bdesc), "r"(idesc), "r"(accum), "r"(z), "r"(z), "r"(z), "r"(z));
-}
-
-__device__ __forceinline__ void tmem_ld32(uint32_t taddr, uint32_t (&v)[32]) {
-  asm volatile(
-      "tcgen05.ld.sync.aligned.32x32b.x32.b32 {%0, %1, %2, %3, %4, %5, %6, %7, %8, %9, %10, %11, %12, %13, "
-      "%14, %15, %16, %17, %18, %19, %20, %21, %22, %23, %24, %25, %26, %27, %28, %29, %30, %31}, [%32];\n"
-      : "=r"(v[0]), "=r"(v[1]), "=r"(v[2]), "=r"(v[3]), "=r"(v[4]), "=r"(v[5]), "=r"(v[6]), "=r"(v[7]),
-        "=r"(v[8]), "=r"(v[9]), "=r"(v[10]), "=r"(v[11]), "=r"(v[12]), "=r"(v[13]), "=r"(v[14]), "=r"(v[15]),
-        "=r"(v[16]), "=r"(v[17]), "=r"(v[18]), "=r"(v[19]), "=r"(v[20]), "=r"(v[21]), "=r"(v[22]), "=r"(v[23]),
-        "=r"(v[24]), "=r"(v[25]), "=r"(v[26]), "=r"(v[27]), "=r"(v[28]), "=r"(v[29]), "=r"(v[30]), "=r"(v[31])
-      : "r"(taddr));
-}
-
-__device__ __forceinline__ bool mbar_try(uint32_t bar, uint32_t parity) {
-  uint32_t ok;
-  asm volatile(
-      "{\n .reg .pred p;\n mbarrier.try_wait.parity.shared::cta.b64 p, [%1], %2;\n selp.u32 %0, 1, 0, p;\n}\n"
-      : "=r"(ok)
-      : "r"(bar), "r"(parity)
-      : "memory");
-  return ok != 0;
-}
-
 template <int D, int BM, int DT>
 __global__ void __launch_bounds__(kTcThreads, 1) encode_dense_tc_kernel(DenseParams p, unsigned *faults,
                                                                         int64_t ntiles) {
@@ -310,34 +266,26 @@ __global__ void __launch_bounds__(kTcThreads, 1) encode_dense_tc_kernel(DensePar
   float *s_inv = reinterpret_cast<float *>(smem + L::oInv);
 
   // ---- once: TMEM columns, the mbarrier, Pi's halves (scaled by 16)
-  if (warp == 0) {
-    const uint32_t dst = (uint32_t)__cvta_generic_to_shared(&s_tmem);
-    asm volatile("tcgen05.alloc.cta_group::1.sync.aligned.shared::cta.b32 [%0], %1;\n" ::"r"(dst), "r"((uint32_t)D)
-                 : "memory");
-    asm volatile("tcgen05.relinquish_alloc_permit.cta_group::1.sync.aligned;\n" ::: "memory");
-  }
-  if (tid == 0) {
-    asm volatile("mbarrier.init.shared::cta.b64 [%0], 1;\n" ::"r"(bar) : "memory");
-    asm volatile("fence.mbarrier_init.release.cluster;\n" ::: "memory");
-  }
+  if (warp == 0) umma::alloc(&s_tmem, (uint32_t)D);
+  if (tid == 0) umma::mbar_init(bar, 1);
   for (int i = tid; i < D * D; i += kTcThreads) {
     const int n = i / D, k = i % D;
     const float v = 16.0f * __ldg(p.rot + i);
     const __half h = __float2half_rn(v);
     const __half l = __float2half_rn(v - __half2float(h));
-    const uint32_t o = a_off(n, k, L::SBO_B, kTcLboB);
+    const uint32_t o = umma::off(n, k, L::SBO_B, kTcLboB);
     *reinterpret_cast<__half *>(smem + L::oBh + o) = h;
     *reinterpret_cast<__half *>(smem + L::oBl + o) = l;
   }
   uint32_t P[K / 2 > 0 ? K / 2 : 1];
 #pragma unroll
   for (int m = 0; m + 1 < K / 2; ++m) P[m] = __float_as_uint(__ldg(p.thr + K / 2 + m));
-  asm volatile("fence.proxy.async.shared::cta;\n" ::: "memory");
-  asm volatile("tcgen05.fence::before_thread_sync;\n" ::: "memory");
+  umma::fence_async_smem();
+  umma::fence_before();
   __syncthreads();
-  asm volatile("tcgen05.fence::after_thread_sync;\n" ::: "memory");
+  umma::fence_after();
   const uint32_t tmem = s_tmem;
-  const uint32_t idesc = (1u << 4) | ((uint32_t)(D >> 3) << 17) | ((uint32_t)(kTcM >> 4) << 24);
+  constexpr uint32_t idesc = umma::idesc_f16(kTcM, D);
   bool dead = false;
 
   for (int64_t tile = blockIdx.x, it = 0; tile < ntiles; tile += gridDim.x, ++it) {
@@ -381,7 +329,7 @@ __global__ void __launch_bounds__(kTcThreads, 1) encode_dense_tc_kernel(DensePar
           const float xs = xr[r][j] * sc;
           const __half hi = __float2half_rn(xs);
           const __half lo = __float2half_rn(xs - __half2float(hi));
-          const uint32_t o = a_off(m, k, L::SBO_A, kTcLboA);
+          const uint32_t o = umma::off(m, k, L::SBO_A, kTcLboA);
           *reinterpret_cast<__half *>(smem + L::oAh + o) = hi;
           *reinterpret_cast<__half *>(smem + L::oAl + o) = lo;
         }
@@ -395,44 +343,27 @@ __global__ void __launch_bounds__(kTcThreads, 1) encode_dense_tc_kernel(DensePar
         }
       }
     }
-    asm volatile("fence.proxy.async.shared::cta;\n" ::: "memory");
+    umma::fence_async_smem();
     __syncthreads();
 
     // ---- phase 2: Y = Xh Ph + Xh Pl + Xl Ph into TMEM
     if (tid == 0) {
-      asm volatile("tcgen05.fence::after_thread_sync;\n" ::: "memory");
+      umma::fence_after();
 #pragma unroll 1
       for (int ks = 0; ks < D / 16; ++ks) {
-        const uint64_t ah = umma_desc(sbase + L::oAh + ks * 2 * kTcLboA, kTcLboA, L::SBO_A);
-        const uint64_t al = umma_desc(sbase + L::oAl + ks * 2 * kTcLboA, kTcLboA, L::SBO_A);
-        const uint64_t bh = umma_desc(sbase + L::oBh + ks * 2 * kTcLboB, kTcLboB, L::SBO_B);
-        const uint64_t bl = umma_desc(sbase + L::oBl + ks * 2 * kTcLboB, kTcLboB, L::SBO_B);
-        umma_f16(tmem, ah, bh, idesc, ks > 0 ? 1u : 0u);
-        umma_f16(tmem, ah, bl, idesc, 1u);
-        umma_f16(tmem, al, bh, idesc, 1u);
+        const uint64_t ah = umma::desc(sbase + L::oAh + ks * 2 * kTcLboA, kTcLboA, L::SBO_A);
+        const uint64_t al = umma::desc(sbase + L::oAl + ks * 2 * kTcLboA, kTcLboA, L::SBO_A);
+        const uint64_t bh = umma::desc(sbase + L::oBh + ks * 2 * kTcLboB, kTcLboB, L::SBO_B);
+        const uint64_t bl = umma::desc(sbase + L::oBl + ks * 2 * kTcLboB, kTcLboB, L::SBO_B);
+        umma::mma_f16(tmem, ah, bh, idesc, ks > 0 ? 1u : 0u);
+        umma::mma_f16(tmem, ah, bl, idesc, 1u);
+        umma::mma_f16(tmem, al, bh, idesc, 1u);
       }
-      asm volatile("tcgen05.commit.cta_group::1.mbarrier::arrive::one.shared::cluster.b64 [%0];\n" ::"r"(bar)
-                   : "memory");
+      umma::commit(bar);
     }
     // bounded wait for the MMAs (phase parity = tile count & 1)
-    if (!dead) {
-      const uint32_t par = (uint32_t)(it & 1);
-      uint64_t t0 = 0;
-      for (uint32_t spin = 0; !mbar_try(bar, par); ++spin) {
-        if ((spin & 255u) == 255u) {
-          uint64_t now;
-          asm volatile("mov.u64 %0, %%globaltimer;\n" : "=l"(now));
-          if (t0 == 0) {
-            t0 = now;
-          } else if (now - t0 > 1000000000ull) {
-            atomicOr(faults, kFaultTimeout);
-            dead = true;
-            break;
-          }
-        }
-      }
-    }
-    asm volatile("tcgen05.fence::after_thread_sync;\n" ::: "memory");
+    if (!dead) dead = !umma::mbar_wait_bounded(bar, (uint32_t)(it & 1), faults, kFaultTimeout);
+    umma::fence_after();
 
     // ---- phase 3: half a record per thread, 32 columns (BM words of
     // codes) at a time
@@ -450,8 +381,8 @@ __global__ void __launch_bounds__(kTcThreads, 1) encode_dense_tc_kernel(DensePar
 #pragma unroll 1
       for (int c = 0; c < HALF / 32; ++c) {
         uint32_t y[32];
-        tmem_ld32(tmem + ((uint32_t)(32 * q4) << 16) + (uint32_t)(hf * HALF + 32 * c), y);
-        asm volatile("tcgen05.wait::ld.sync.aligned;\n" ::: "memory");
+        umma::ld32(tmem + ((uint32_t)(32 * q4) << 16) + (uint32_t)(hf * HALF + 32 * c), y);
+        umma::wait_ld();
         uint32_t W[BM];
 #pragma unroll
         for (int w = 0; w < BM; ++w) W[w] = 0u;
@@ -469,12 +400,12 @@ __global__ void __launch_bounds__(kTcThreads, 1) encode_dense_tc_kernel(DensePar
         if (dst) dev::store_words<BM>(dst + c * 4 * BM, W);
       }
     }
-    asm volatile("tcgen05.fence::before_thread_sync;\n" ::: "memory");
+    umma::fence_before();
     __syncthreads();
   }
   if (warp == 0) {
-    asm volatile("tcgen05.fence::after_thread_sync;\n" ::: "memory");
-    asm volatile("tcgen05.dealloc.cta_group::1.sync.aligned.b32 %0, %1;\n" ::"r"(tmem), "r"((uint32_t)D) : "memory");
+    umma::fence_after();
+    umma::dealloc(tmem, (uint32_t)D);
   }
 }
 

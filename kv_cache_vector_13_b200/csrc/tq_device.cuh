@@ -121,6 +121,29 @@ __device__ __forceinline__ float fold_halves_sum(float (&a)[E]) {
   return a[0];
 }
 
+// The same fold-halves sum of the squares fl(a_i * a_i), without a second
+// array: after the cross-lane stages, element i after in-register stage h is
+// W(i, h) = W(i, 2h) + W(i + h, 2h), with W(i, E) the squared element; the
+// recursion visits the leaves depth first, so only log2(E) partial sums are
+// live at a time.  Bit-identical to fold_halves_sum of the squares.
+template <int T, int E, int I, int H>
+__device__ __forceinline__ float fold_sumsq_node(const float (&a)[E]) {
+  if constexpr (H == E) {
+    float s = __fmul_rn(a[I], a[I]);
+#pragma unroll
+    for (int P = T / 2; P >= 1; P >>= 1) s = __fadd_rn(s, __shfl_xor_sync(kFull, s, P));
+    return s;
+  } else {
+    const float lo = fold_sumsq_node<T, E, I, 2 * H>(a);
+    return __fadd_rn(lo, fold_sumsq_node<T, E, I + H, 2 * H>(a));
+  }
+}
+
+template <int T, int E>
+__device__ __forceinline__ float fold_halves_sumsq(const float (&a)[E]) {
+  return fold_sumsq_node<T, E, 0, 1>(a);
+}
+
 // -------------------------------------------------------------- quantize
 
 // idx = #{j : u > t_j} for an antisymmetric codebook with K = 2^BM levels,

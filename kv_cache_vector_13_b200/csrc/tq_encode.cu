@@ -18,6 +18,7 @@
 #include "../../include/tq.h"
 #include "tq_device.cuh"
 #include "tq_internal.h"
+#include "tq_umma.cuh"
 
 #include <cuda_fp16.h>
 
@@ -282,230 +283,347 @@ __global__ void __launch_bounds__(kEncThreads, EE == 64 ? 3 : 1) encode_kernel(E
   pdl_close(p.pdl);
 }
 
-// ------------------------------------------------ prod, d = 128: tensor cores
+// ------------------------------------------------ prod, d = 128: tcgen05
 //
 // The QJL projection z = S r is a dense 128 x 128 contraction per vector; for
-// a batch it is Z = R S^T, which runs here on mma.m16n8k16 (f16 x f16 ->
-// f32).  One warp owns 16 vectors (two lanes per vector in the front half),
-// exactly the M = 16 rows of an MMA tile.  Operands are split into fp16
-// halves, x = hi + lo with hi = fp16(x), lo = fp16(x - hi), and
-// z ~ Sh.rh + Sh.rl + Sl.rh (the dropped Sl.rl is below 2^-22 of
-// sum |S_ki r_i|).  Each residual row is first scaled by a power of two,
-// 2^(4 - floor(log2 ||r||)), which keeps both halves in fp16's normal range
-// and leaves every sign unchanged.  The representation (about 3 * 2^-22
-// per product), the dropped term and the fp32 accumulation over 24 MMA
-// steps (at most 24 * 2^-23 of sum |S_ki r_i|) stay below 2^-17.4
-// sum |S_ki r_i| <= 2^-17.4 ||S_k|| ||r||, a fifth of
-// theta_k = 2^-15 ||S_k|| ||r||; a projection with |z| <= theta_k (about
-// three in ten thousand) is recomputed by an fp32 dot product, so a stored
-// sign can differ from the exact one only where an fp32 summation's sign
-// could.  The block is persistent: it converts S to fp16 halves in
-// shared memory once and then walks tiles of 256 vectors.
-constexpr int kMmaThreads = 512;
-constexpr int kMmaVPB = kMmaThreads / 2;  // vectors per tile (two lanes each)
-constexpr int kSRow = 128 + 8;            // fp16 row of S halves (conflict-free B loads)
-constexpr int kRRow = 128 + 4;            // fp32 residual row (conflict-free A loads)
+// a tile of 128 vectors it is Z = R S^T (M = N = K = 128), which runs here on
+// the fifth-generation tensor cores with the accumulator in tensor memory.
+// fp32 is carried by fp16 halves, x = hi + lo with hi = fp16(x),
+// lo = fp16(x - hi), and Z ~ Rh Sh + Rh Sl + Rl Sh (the dropped Rl Sl is
+// below 2^-22 of sum |S_ki r_i|).  Scalings that keep every half in fp16's
+// normal range and leave every sign unchanged: each row of S by
+// 16 / ||S_k||, each residual row by sc = 2^(4 - floor(log2 ||r||)).  The
+// representation (about 3 * 2^-22 per product), the dropped term and the
+// fp32 accumulation stay below 2^-17.4 sum |S_ki r_i| <= 2^-17.4 ||S_k||
+// ||r||, a fifth of theta_k = 2^-15 ||S_k|| ||r||; in the scaled units the
+// test is |z'_k| <= sc ||r|| 2^-11 for every k.  Such a projection (about
+// three in ten thousand) is recomputed exactly: the warp re-encodes the
+// vector from its input in the canonical fp32 order (four coordinates a
+// lane) and forms z_k = sum_i S_ki r_i in fp32, so a stored sign can differ
+// from the exact one only where an fp32 summation's sign could.
+//
+// Per CTA (persistent, one per SM): two groups of 8 warps, each with its own
+// A operand, TMEM accumulator and mbarrier, walk alternate tiles, so one
+// group's loads and front half overlap the other's MMAs and epilogue.
+//   * once: S's scaled halves into shared memory (the B operand, K-major, no
+//     swizzle), 2 x 128 TMEM columns;
+//   * front half (two lanes per vector, 64 coordinates each): norm, sign
+//     flips + FWHT, scale, codes, residual, ||r||; the scaled residual's
+//     halves go into the group's A operand as 16-byte core-matrix rows;
+//   * one thread issues the 3 x 8 tcgen05.mma and commits to the group's
+//     mbarrier; the group waits on it (bounded);
+//   * epilogue: warp w of the group reads TMEM lanes 32 (w % 4) + [0, 32)
+//     (one vector each) and 64 of the 128 columns; a sign bit is the fp32
+//     sign of z', gathered by funnel shifts.
+constexpr int kPtGroups = 2;                 // tiles in flight per CTA
+constexpr int kPtGroupThreads = 256;         // 8 warps a group
+constexpr int kPtThreads = kPtGroups * kPtGroupThreads;
+constexpr int kPtM = 128;                    // vectors per tile
+constexpr int kPtLbo = 128;                  // bytes between K-adjacent core matrices
+constexpr int kPtSbo = 16 * kPtLbo;          // bytes between 8-row groups (K = 128)
+constexpr int kPtOp = 16 * kPtSbo;           // one 128 x 128 fp16 operand: 32 KiB
+constexpr size_t kPtSmem = (size_t)(2 + 2 * kPtGroups) * kPtOp;  // S hi, S lo, then A hi, A lo per group
 
-constexpr size_t enc_mma_smem_bytes() {
-  return (size_t)2 * 128 * kSRow * 2 + (size_t)kMmaVPB * kRRow * 4;
+__device__ __forceinline__ uint32_t pack_h2(float a, float b) {
+  const __half2 h = __floats2half2_rn(a, b);
+  return *reinterpret_cast<const uint32_t *>(&h);
 }
 
-__device__ __forceinline__ uint32_t h2_bits(__half2 h) { return *reinterpret_cast<const uint32_t *>(&h); }
-
-// fp16 (hi, lo) halves of the pair (x, y)
-__device__ __forceinline__ void split2(float x, float y, uint32_t &hi, uint32_t &lo) {
-  const __half2 h = __floats2half2_rn(x, y);
-  const float2 f = __half22float2(h);
-  hi = h2_bits(h);
-  lo = h2_bits(__floats2half2_rn(x - f.x, y - f.y));
-}
-
-__device__ __forceinline__ void mma_f16(float (&c)[4], const uint32_t (&a)[4], uint32_t b0, uint32_t b1) {
-  asm volatile(
-      "mma.sync.aligned.m16n8k16.row.col.f32.f16.f16.f32 {%0,%1,%2,%3}, {%4,%5,%6,%7}, {%8,%9}, "
-      "{%0,%1,%2,%3};\n"
-      : "+f"(c[0]), "+f"(c[1]), "+f"(c[2]), "+f"(c[3])
-      : "r"(a[0]), "r"(a[1]), "r"(a[2]), "r"(a[3]), "r"(b0), "r"(b1));
-}
-
-// bits 0..3 of x to bits 0, 2, 4, 6
-__device__ __forceinline__ uint32_t spread4(uint32_t x) {
-  x = (x | (x << 2)) & 0x33u;
-  return (x | (x << 1)) & 0x55u;
-}
-
-// sign of the fp32 dot product of one row of S (global, 16-byte aligned)
-// with a residual row (shared, 16-byte aligned)
-__device__ __noinline__ bool qjl_recheck(const float *S_row, const float *r) {
-  const float4 *s4 = reinterpret_cast<const float4 *>(S_row);
-  const float4 *r4 = reinterpret_cast<const float4 *>(r);
-  float acc = 0.0f;
-#pragma unroll 8
-  for (int i = 0; i < 32; ++i) {
-    const float4 a = __ldg(s4 + i), b = r4[i];
-    acc = fmaf(a.x, b.x, acc);
-    acc = fmaf(a.y, b.y, acc);
-    acc = fmaf(a.z, b.z, acc);
-    acc = fmaf(a.w, b.w, acc);
+// fp16 halves of 8 consecutive values: hi into H, lo into L (as uint4 rows
+// of a core matrix)
+__device__ __forceinline__ void split8(const float (&x)[8], uint4 &H, uint4 &L) {
+  uint32_t h[4], l[4];
+#pragma unroll
+  for (int i = 0; i < 4; ++i) {
+    h[i] = pack_h2(x[2 * i], x[2 * i + 1]);
+    const float2 f = __half22float2(*reinterpret_cast<const __half2 *>(&h[i]));
+    l[i] = pack_h2(x[2 * i] - f.x, x[2 * i + 1] - f.y);
   }
-  return acc >= 0.0f;
+  H = make_uint4(h[0], h[1], h[2], h[3]);
+  L = make_uint4(l[0], l[1], l[2], l[3]);
+}
+
+__device__ __forceinline__ void group_sync(int grp) {
+  asm volatile("bar.sync %0, %1;\n" ::"r"(1 + grp), "r"(kPtGroupThreads) : "memory");
+}
+
+// The exact fp32 residual of vector v, re-encoded by the whole warp in the
+// canonical order: lane l holds coordinates 4l + j.  Every step is the same
+// IEEE operation on the same operands as the two-lane front half (the
+// butterfly and the fold-halves sum pair the same coordinates whatever the
+// layout), so r[] equals the residual the front half formed.
+template <int BM, int DT>
+__device__ __forceinline__ void residual_exact(const EncParams &p, int64_t v, const uint32_t *s_sign, const float *s_cent,
+                                               float (&r)[4]) {
+  constexpr int K = 1 << BM;
+  const int lane = threadIdx.x & 31;
+  int64_t b, h, n;
+  split_index(p, v, b, h, n);
+  const int64_t xoff = b * p.xsb + h * p.xsh + n * p.xsn + 4 * lane;
+  float x[4];
+  if constexpr (DT == 0) {
+    const float4 t = __ldg(reinterpret_cast<const float4 *>(static_cast<const float *>(p.x) + xoff));
+    x[0] = t.x, x[1] = t.y, x[2] = t.z, x[3] = t.w;
+  } else {
+    const uint2 t = __ldg(reinterpret_cast<const uint2 *>(static_cast<const unsigned short *>(p.x) + xoff));
+    if constexpr (DT == 1) {
+      x[0] = dev::bf16lo(t.x), x[1] = dev::bf16hi(t.x), x[2] = dev::bf16lo(t.y), x[3] = dev::bf16hi(t.y);
+    } else {
+      x[0] = dev::f16lo(t.x), x[1] = dev::f16hi(t.x), x[2] = dev::f16lo(t.y), x[3] = dev::f16hi(t.y);
+    }
+  }
+  // norm: fold-halves over h = 64 .. 1 (lanes < h/4 hold the live partial sums)
+  float sq[4];
+#pragma unroll
+  for (int j = 0; j < 4; ++j) sq[j] = __fmul_rn(x[j], x[j]);
+#pragma unroll
+  for (int sh = 16; sh >= 1; sh >>= 1) {
+#pragma unroll
+    for (int j = 0; j < 4; ++j) sq[j] = __fadd_rn(sq[j], __shfl_down_sync(dev::kFull, sq[j], sh));
+  }
+  sq[0] = __fadd_rn(sq[0], sq[2]);
+  sq[1] = __fadd_rn(sq[1], sq[3]);
+  const float nrm = __fsqrt_rn(__shfl_sync(dev::kFull, __fadd_rn(sq[0], sq[1]), 0));
+  // sign flips, then the FWHT stages h = 64 .. 1
+  const uint32_t sw = s_sign[lane >> 3] >> (4 * (lane & 7));
+#pragma unroll
+  for (int j = 0; j < 4; ++j) x[j] = __uint_as_float(__float_as_uint(x[j]) ^ (((sw >> j) & 1u) << 31));
+#pragma unroll
+  for (int pl = 16; pl >= 1; pl >>= 1) {
+    const bool low = (lane & pl) == 0;
+#pragma unroll
+    for (int j = 0; j < 4; ++j) {
+      const float o = __shfl_xor_sync(dev::kFull, x[j], pl);
+      x[j] = low ? __fadd_rn(x[j], o) : __fsub_rn(o, x[j]);
+    }
+  }
+  {
+    const float a0 = x[0], a1 = x[1], a2 = x[2], a3 = x[3];
+    x[0] = __fadd_rn(a0, a2), x[2] = __fsub_rn(a0, a2);
+    x[1] = __fadd_rn(a1, a3), x[3] = __fsub_rn(a1, a3);
+    const float c0 = x[0], c1 = x[1], c2 = x[2], c3 = x[3];
+    x[0] = __fadd_rn(c0, c1), x[1] = __fsub_rn(c0, c1);
+    x[2] = __fadd_rn(c2, c3), x[3] = __fsub_rn(c2, c3);
+  }
+  const float wsc = __fmul_rn(nrm, p.sqrt_d);
+  const float inv = wsc > 0.0f ? __frcp_rn(wsc) : 0.0f;
+  uint32_t PP[K / 2 > 0 ? K / 2 : 1];
+#pragma unroll
+  for (int m = 0; m + 1 < K / 2; ++m) PP[m] = __float_as_uint(__ldg(p.thr + K / 2 + m));
+#pragma unroll
+  for (int j = 0; j < 4; ++j) {
+    const float u = __fmul_rn(x[j], inv);
+    if constexpr (BM == 0) {
+      r[j] = u;
+    } else {
+      const int idx = BM == 1 ? (u > 0.0f ? 1 : 0) : dev::quantize_sym<BM>(u, PP);
+      r[j] = __fsub_rn(u, s_cent[idx]);
+    }
+  }
+}
+
+// The warp's exact recheck of one 32-column chunk: lanes in `need` hold a
+// vector (v0 + lane) with near-zero projections k0 + i for the bits i of
+// their `mine`; each such sign is recomputed from the exact residual.
+// Returns the calling lane's corrected sign word.
+template <int BM, int DT>
+__device__ __noinline__ uint32_t recheck(const EncParams &p, int64_t v0, int k0, uint32_t need, uint32_t mine,
+                                         uint32_t q, const uint32_t *s_sign, const float *s_cent) {
+  const int lane = threadIdx.x & 31;
+  while (need) {
+    const int src = __ffs(need) - 1;
+    need &= need - 1;
+    uint32_t mask = __shfl_sync(dev::kFull, mine, src);
+    float r[4];
+    residual_exact<BM, DT>(p, v0 + src, s_sign, s_cent, r);
+    while (mask) {
+      const int i = __ffs(mask) - 1;
+      mask &= mask - 1;
+      const float4 sk = __ldg(reinterpret_cast<const float4 *>(p.S + (k0 + i) * 128) + lane);
+      float z = fmaf(sk.x, r[0], fmaf(sk.y, r[1], fmaf(sk.z, r[2], sk.w * r[3])));
+#pragma unroll
+      for (int o = 16; o >= 1; o >>= 1) z += __shfl_xor_sync(dev::kFull, z, o);
+      if (lane == src) q = (q & ~(1u << i)) | ((z >= 0.0f ? 1u : 0u) << i);
+    }
+  }
+  return q;
 }
 
 template <int BM, int DT>
-__global__ void __launch_bounds__(kMmaThreads, 1) encode_prod_mma_kernel(EncParams p, int64_t ntiles) {
+__global__ void __launch_bounds__(kPtThreads, 1) encode_prod_tc_kernel(EncParams p, unsigned *faults, int64_t ntiles) {
   constexpr int D = 128, T = 2, E = 64;
   constexpr int K = 1 << BM;
   constexpr int NWC = BM > 0 ? (E * BM + 31) / 32 : 1;
-
+  constexpr uint32_t kIdesc = umma::idesc_f16(kPtM, D);
+  extern __shared__ __align__(1024) unsigned char smem[];
   __shared__ uint32_t s_sign[D / 32];
   __shared__ float s_cent[16];
-  __shared__ float s_snorm[D];
-  __shared__ float s_rs[kMmaVPB];  // per vector: scale of its residual row, theta factor
-  __shared__ float s_th[kMmaVPB];
-  extern __shared__ float4 s_dyn4[];
-  __half *s_sh = reinterpret_cast<__half *>(s_dyn4);          // [128][kSRow] hi(S)
-  __half *s_sl = s_sh + 128 * kSRow;                          // [128][kSRow] lo(S)
-  float *s_r = reinterpret_cast<float *>(s_sl + 128 * kSRow);  // [256][kRRow] residuals
+  __shared__ float s_th[kPtGroups][2][kPtM];  // per tile parity: sc ||r|| 2^-11
+  __shared__ __align__(8) uint64_t s_bar[kPtGroups];
+  __shared__ uint32_t s_tmem;
 
-  const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
+  const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
+  const int grp = warp / 8, gt = tid % kPtGroupThreads, gw = warp % 8;
+  const uint32_t sbase = (uint32_t)__cvta_generic_to_shared(smem);
+  const uint32_t bar = (uint32_t)__cvta_generic_to_shared(&s_bar[grp]);
   pdl_open();
+
+  // ---- once: TMEM, mbarriers, S's scaled halves, codebook, sign masks
+  if (warp == 0) umma::alloc(&s_tmem, kPtGroups * D);
+  if (tid == 0) {
+#pragma unroll
+    for (int g = 0; g < kPtGroups; ++g) umma::mbar_init((uint32_t)__cvta_generic_to_shared(&s_bar[g]), 1);
+  }
   load_sign_masks<D>(p.signs, s_sign, tid);
   if constexpr (BM > 0) {
     if (tid < K) s_cent[tid] = p.cent[tid];
   }
-  {  // S to fp16 halves, and its row norms: thread = (row, quarter of 32)
+  {  // thread = (row of S, quarter of 32 columns)
     const int row = tid >> 2, q = tid & 3;
     const float4 *src = reinterpret_cast<const float4 *>(p.S + row * D + 32 * q);
+    float v[32];
     float ss = 0.0f;
 #pragma unroll
     for (int i = 0; i < 8; ++i) {
-      const float4 v = __ldg(src + i);
-      uint32_t h0, l0, h1, l1;
-      split2(v.x, v.y, h0, l0);
-      split2(v.z, v.w, h1, l1);
-      const int k = 32 * q + 4 * i;
-      *reinterpret_cast<uint2 *>(s_sh + row * kSRow + k) = make_uint2(h0, h1);
-      *reinterpret_cast<uint2 *>(s_sl + row * kSRow + k) = make_uint2(l0, l1);
-      ss = fmaf(v.x, v.x, fmaf(v.y, v.y, fmaf(v.z, v.z, fmaf(v.w, v.w, ss))));
+      const float4 t = __ldg(src + i);
+      v[4 * i] = t.x, v[4 * i + 1] = t.y, v[4 * i + 2] = t.z, v[4 * i + 3] = t.w;
+      ss = fmaf(t.x, t.x, fmaf(t.y, t.y, fmaf(t.z, t.z, fmaf(t.w, t.w, ss))));
     }
     ss += __shfl_xor_sync(dev::kFull, ss, 1);
     ss += __shfl_xor_sync(dev::kFull, ss, 2);
-    if (q == 0) s_snorm[row] = sqrtf(ss);
+    const float f = ss > 0.0f ? 16.0f / sqrtf(ss) : 0.0f;
+#pragma unroll
+    for (int c = 0; c < 4; ++c) {
+      float x[8];
+#pragma unroll
+      for (int i = 0; i < 8; ++i) x[i] = v[8 * c + i] * f;
+      uint4 H, L;
+      split8(x, H, L);
+      const uint32_t o = umma::off(row, 32 * q + 8 * c, kPtSbo, kPtLbo);
+      *reinterpret_cast<uint4 *>(smem + o) = H;
+      *reinterpret_cast<uint4 *>(smem + kPtOp + o) = L;
+    }
   }
   uint32_t P[K / 2 > 0 ? K / 2 : 1];
 #pragma unroll
   for (int m = 0; m + 1 < K / 2; ++m) P[m] = __float_as_uint(__ldg(p.thr + K / 2 + m));
+  umma::fence_async_smem();
+  umma::fence_before();
   __syncthreads();
+  umma::fence_after();
+  const uint32_t tmem = s_tmem + (uint32_t)(grp * D);
+  const uint32_t oAh = (uint32_t)((2 + 2 * grp) * kPtOp), oAl = oAh + kPtOp;
+  const int t = gt & 1, vl = gt >> 1;
+  bool dead = false;
 
-  const int t = tid & 1, vl = tid >> 1;
-  const int g8 = lane >> 2, tig = lane & 3;
-  const float *rw = s_r + (size_t)(warp * 16) * kRRow;  // this warp's 16 residual rows
-  for (int64_t tile = blockIdx.x; tile < ntiles; tile += gridDim.x) {
-    int64_t v = tile * kMmaVPB + vl;
-    const bool active = v < p.nvec;
-    if (!active) v = p.nvec - 1;  // idle lanes still take part in the shuffles
-    int64_t b, h, n;
-    split_index(p, v, b, h, n);
-    const int64_t xoff = b * p.xsb + h * p.xsh + n * p.xsn + (int64_t)t * E;
-    const int64_t rec = b * p.osb + h * p.osh + n * p.osn;
-
-    float a[E];
-    uint32_t W[NWC];
-    const float nrm = encode_front<D, BM, true, DT, T, E>(p, xoff, t, s_sign, s_cent, P, a, W);
-    if constexpr (BM > 0) {
-      if (active) store_bytes<E * BM / 8>(p.codes + rec * (D * BM / 8) + t * (E * BM / 8), W);
-    }
-    if (active && t == 0) p.norms[rec] = nrm;
-    float rr[E];
-#pragma unroll
-    for (int i = 0; i < E; ++i) rr[i] = __fmul_rn(a[i], a[i]);
-    const float gam = __fsqrt_rn(dev::fold_halves_sum<T, E>(rr));
-    float *rv = s_r + (size_t)vl * kRRow + t * E;
-#pragma unroll
-    for (int i = 0; i < E; i += 4) *reinterpret_cast<float4 *>(rv + i) = make_float4(a[i], a[i + 1], a[i + 2], a[i + 3]);
-    if (t == 0) {
+  int64_t it = 0;
+  for (int64_t tile = (int64_t)blockIdx.x * kPtGroups + grp; tile < ntiles;
+       tile += (int64_t)gridDim.x * kPtGroups, ++it) {
+    const int par = (int)(it & 1);
+    // ---- front half: vector vl of the tile, coordinates [64 t, 64 t + 64)
+    {
+      int64_t v = tile * kPtM + vl;
+      const bool active = v < p.nvec;
+      if (!active) v = p.nvec - 1;  // idle lanes still take part in the shuffles
+      int64_t b, h, n;
+      split_index(p, v, b, h, n);
+      const int64_t xoff = b * p.xsb + h * p.xsh + n * p.xsn + (int64_t)t * E;
+      const int64_t rec = b * p.osb + h * p.osh + n * p.osn;
+      float a[E];
+      uint32_t W[NWC];
+      const float nrm = encode_front<D, BM, true, DT, T, E>(p, xoff, t, s_sign, s_cent, P, a, W);
+      if constexpr (BM > 0) {
+        if (active) store_bytes<E * BM / 8>(p.codes + rec * (D * BM / 8) + t * (E * BM / 8), W);
+      }
+      const float gam = __fsqrt_rn(dev::fold_halves_sumsq<T, E>(a));
       // 2^(4 - floor(log2 gam)): |scaled r_i| <= 32; gam = 0 -> 1
       const int ex = gam > 0.0f ? ((__float_as_int(gam) >> 23) & 0xff) - 127 : 0;
       const float sc = __int_as_float((127 + min(4 - ex, 100)) << 23);
-      s_rs[vl] = sc;
-      s_th[vl] = gam * sc * 0x1p-15f;
+      if (t == 0) {
+        s_th[grp][par][vl] = gam * sc * 0x1p-11f;
+        if (active) {
+          p.norms[rec] = nrm;
+          p.rnorms[rec] = gam;
+        }
+      }
+#pragma unroll
+      for (int c = 0; c < E / 8; ++c) {
+        float x[8];
+#pragma unroll
+        for (int i = 0; i < 8; ++i) x[i] = a[8 * c + i] * sc;
+        uint4 H, L;
+        split8(x, H, L);
+        const uint32_t o = umma::off(vl, t * E + 8 * c, kPtSbo, kPtLbo);
+        *reinterpret_cast<uint4 *>(smem + oAh + o) = H;
+        *reinterpret_cast<uint4 *>(smem + oAl + o) = L;
+      }
     }
-    __syncwarp();
+    umma::fence_async_smem();
+    umma::fence_before();
+    group_sync(grp);
 
-    // A fragments (16 vectors x 128 dims) as fp16 halves of the scaled rows
-    uint32_t ah[8][4], al[8][4];
-    const float sc0 = s_rs[warp * 16 + g8], sc1 = s_rs[warp * 16 + g8 + 8];
-    const float th0 = s_th[warp * 16 + g8], th1 = s_th[warp * 16 + g8 + 8];
-#pragma unroll
-    for (int ks = 0; ks < 8; ++ks) {
-      const int c = ks * 16 + 2 * tig;
-      const float2 r00 = *reinterpret_cast<const float2 *>(rw + g8 * kRRow + c);
-      const float2 r10 = *reinterpret_cast<const float2 *>(rw + (g8 + 8) * kRRow + c);
-      const float2 r01 = *reinterpret_cast<const float2 *>(rw + g8 * kRRow + c + 8);
-      const float2 r11 = *reinterpret_cast<const float2 *>(rw + (g8 + 8) * kRRow + c + 8);
-      split2(r00.x * sc0, r00.y * sc0, ah[ks][0], al[ks][0]);
-      split2(r10.x * sc1, r10.y * sc1, ah[ks][1], al[ks][1]);
-      split2(r01.x * sc0, r01.y * sc0, ah[ks][2], al[ks][2]);
-      split2(r11.x * sc1, r11.y * sc1, ah[ks][3], al[ks][3]);
-    }
-    uint32_t Q[2] = {0u, 0u};
-    const int v16 = lane >> 1;  // this lane's vector within the warp (front-half layout)
+    // ---- Z' = Rh Sh + Rh Sl + Rl Sh into the group's TMEM columns
+    if (gt == 0) {
+      umma::fence_after();
 #pragma unroll 1
-    for (int ng = 0; ng < 4; ++ng) {  // outputs [32 ng, 32 ng + 32)
-      float c[4][4];
-#pragma unroll
-      for (int j = 0; j < 4; ++j) c[j][0] = c[j][1] = c[j][2] = c[j][3] = 0.0f;
-#pragma unroll
-      for (int ks = 0; ks < 8; ++ks) {
-#pragma unroll
-        for (int j = 0; j < 4; ++j) {
-          const int row = (4 * ng + j) * 8 + g8;
-          const __half *ph = s_sh + row * kSRow + ks * 16 + 2 * tig;
-          const __half *pl = s_sl + row * kSRow + ks * 16 + 2 * tig;
-          const uint32_t bh0 = *reinterpret_cast<const uint32_t *>(ph);
-          const uint32_t bh1 = *reinterpret_cast<const uint32_t *>(ph + 8);
-          const uint32_t bl0 = *reinterpret_cast<const uint32_t *>(pl);
-          const uint32_t bl1 = *reinterpret_cast<const uint32_t *>(pl + 8);
-          mma_f16(c[j], ah[ks], bh0, bh1);
-          mma_f16(c[j], al[ks], bh0, bh1);
-          mma_f16(c[j], ah[ks], bl0, bl1);
-        }
+      for (int ks = 0; ks < D / 16; ++ks) {
+        const uint32_t k0 = (uint32_t)(ks * 2 * kPtLbo);
+        const uint64_t ah = umma::desc(sbase + oAh + k0, kPtLbo, kPtSbo);
+        const uint64_t al = umma::desc(sbase + oAl + k0, kPtLbo, kPtSbo);
+        const uint64_t bh = umma::desc(sbase + k0, kPtLbo, kPtSbo);
+        const uint64_t bl = umma::desc(sbase + kPtOp + k0, kPtLbo, kPtSbo);
+        umma::mma_f16(tmem, ah, bh, kIdesc, ks > 0 ? 1u : 0u);
+        umma::mma_f16(tmem, ah, bl, kIdesc, 1u);
+        umma::mma_f16(tmem, al, bh, kIdesc, 1u);
       }
-      // signs: C element e of tile j is (row g8 + 8 (e >> 1), output
-      // 8 (4 ng + j) + 2 tig + (e & 1))
-      uint32_t bal[4][4];
+      umma::commit(bar);
+    }
+    if (!dead) dead = !umma::mbar_wait_bounded(bar, (uint32_t)par, faults, kFaultTimeout);
+    umma::fence_after();
+
+    // ---- epilogue: vector m, projections [64 hf, 64 hf + 64)
+    {
+      const int q4 = gw & 3, hf = gw >> 2;
+      const int m = 32 * q4 + lane;
+      const int64_t v = tile * kPtM + m;
+      const float th = s_th[grp][par][m];
+      uint32_t Q[2];
+#pragma unroll 1
+      for (int c = 0; c < 2; ++c) {
+        uint32_t y[32];
+        umma::ld32(tmem + ((uint32_t)(32 * q4) << 16) + (uint32_t)(hf * 64 + 32 * c), y);
+        umma::wait_ld();
+        uint32_t neg = 0u;  // bit i: the sign bit of z'_i
+        bool near = false;
 #pragma unroll
-      for (int j = 0; j < 4; ++j) {
-#pragma unroll
-        for (int e = 0; e < 4; ++e) {
-          const int out = 8 * (4 * ng + j) + 2 * tig + (e & 1);
-          const int rl = g8 + 8 * (e >> 1);
-          const float z = c[j][e];
-          bool pos = z >= 0.0f;
-          if (!(fabsf(z) > (e >> 1 ? th1 : th0) * s_snorm[out])) pos = qjl_recheck(p.S + out * D, rw + rl * kRRow);
-          bal[j][e] = __ballot_sync(dev::kFull, pos);
+        for (int i = 31; i >= 0; --i) {
+          neg = __funnelshift_l(y[i], neg, 1);
+          near |= !(fabsf(__uint_as_float(y[i])) > th);
         }
+        uint32_t q = ~neg;
+        // exact recheck of the projections too close to zero to trust
+        uint32_t need = __ballot_sync(dev::kFull, near && v < p.nvec);
+        if (need) {
+          uint32_t mine = 0u;
+#pragma unroll
+          for (int i = 0; i < 32; ++i) mine |= (!(fabsf(__uint_as_float(y[i])) > th) ? 1u : 0u) << i;
+          q = recheck<BM, DT>(p, tile * kPtM + 32 * q4, hf * 64 + 32 * c, need, mine, q, s_sign, s_cent);
+        }
+        Q[c] = q;
       }
-      // lane (v16, t) keeps outputs [64 t, 64 t + 64): groups 2t and 2t + 1
-      if ((ng >> 1) == t) {
-        const int e0 = v16 < 8 ? 0 : 2, sh = 4 * (v16 & 7);
-        uint32_t word = 0u;
-#pragma unroll
-        for (int j = 0; j < 4; ++j) {
-          const uint32_t ev = (bal[j][e0] >> sh) & 0xfu, od = (bal[j][e0 + 1] >> sh) & 0xfu;
-          word |= (spread4(ev) | (spread4(od) << 1)) << (8 * j);
-        }
-        Q[ng & 1] = word;
+      if (v < p.nvec) {
+        int64_t b, h, n;
+        split_index(p, v, b, h, n);
+        const int64_t rec = b * p.osb + h * p.osh + n * p.osn;
+        store_bytes<8>(p.qjl + rec * (D / 8) + hf * 8, Q);
       }
     }
-    if (active) {
-      store_bytes<8>(p.qjl + rec * (D / 8) + t * 8, Q);
-      if (t == 0) p.rnorms[rec] = gam;
-    }
-    // keep the block's warps in step (they run the same long straight-line
-    // code, which then stays in the instruction cache); also orders this
-    // warp's residual-row reads before the next tile's writes
-    __syncthreads();
+    umma::fence_before();
+  }
+  __syncthreads();
+  if (warp == 0) {
+    umma::fence_after();
+    umma::dealloc(s_tmem, kPtGroups * D);
   }
   pdl_close(p.pdl);
 }
@@ -527,14 +645,17 @@ cudaError_t launch_maybe_pdl(K kern, dim3 grid, dim3 block, size_t smem, cudaStr
 }
 
 template <int BM, int DT>
-cudaError_t run_prod_mma(const EncParams &p, cudaStream_t s) {
-  auto kern = encode_prod_mma_kernel<BM, DT>;
-  const size_t smem = enc_mma_smem_bytes();
-  cudaError_t e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
+cudaError_t run_prod_tc(const EncParams &p, cudaStream_t s) {
+  auto kern = encode_prod_tc_kernel<BM, DT>;
+  cudaError_t e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)kPtSmem);
   if (e != cudaSuccess) return e;
-  const int64_t ntiles = (p.nvec + kMmaVPB - 1) / kMmaVPB;
-  const int64_t grid = ntiles < decode_ctas() ? ntiles : decode_ctas();
-  e = launch_maybe_pdl(kern, dim3((unsigned)grid), dim3(kMmaThreads), smem, s, p.pdl, p, ntiles);
+  unsigned *faults = nullptr;
+  e = fault_word(&faults);
+  if (e != cudaSuccess) return e;
+  const int64_t ntiles = (p.nvec + kPtM - 1) / kPtM;
+  const int64_t pairs = (ntiles + kPtGroups - 1) / kPtGroups;
+  const int64_t grid = pairs < decode_ctas() ? pairs : decode_ctas();
+  e = launch_maybe_pdl(kern, dim3((unsigned)grid), dim3(kPtThreads), kPtSmem, s, p.pdl, p, faults, ntiles);
   if (e != cudaSuccess) return e;
   return cudaGetLastError();
 }
@@ -570,7 +691,7 @@ cudaError_t run_e(const EncodeArgs &a, cudaStream_t s) {
     magic31(a.N, p.mN, p.sN);
     magic31(a.H, p.mH, p.sH);
   }
-  if constexpr (PROD && D == 128 && EE == 64) return run_prod_mma<BM, DT>(p, s);
+  if constexpr (PROD && D == 128 && EE == 64) return run_prod_tc<BM, DT>(p, s);
   const size_t smem = enc_smem_bytes<D, PROD, EE>();
   auto kern = encode_kernel<D, BM, PROD, DT, EE>;
   if (smem > 48 * 1024) {
