@@ -184,8 +184,11 @@ size_t tq_decode_workspace_bytes(int32_t B, int32_t Hq, int32_t Hkv,
  * and rotated back once at the end.  out: [B][Hq][d] fp32 (DEVICE); a batch
  * with L_b == 0 gets zeros.  scores_out: optional [B][Hq][seq_len] fp32 of
  * the pre-scale estimator s_j (entries j >= L_b untouched), or NULL.
- * V must be mse (prod values return TQ_EUNSUPPORTED); d must be 128 (other d
- * return TQ_EUNSUPPORTED).
+ * Any valid pair of quantizers with equal d: K and V may each be mse or
+ * prod, with either rotation.  Prod values are dequantized as
+ * n_j (c_V[idx_j] + ||r_j|| sqrt(pi/2)/d S_V^T sign_j) in the rotated basis.
+ * d = 128 with mse values runs on tensor cores (fp16 hi/lo operands, fp32
+ * accumulation); every other case runs on CUDA cores in fp32.
  * workspace: DEVICE, at least tq_decode_workspace_bytes(...) bytes, 16-byte
  * aligned, else TQ_EWORKSPACE. */
 tq_status tq_decode_attention(const tq_quantizer *kq, const tq_quantizer *vq,

@@ -217,10 +217,16 @@ __global__ void __launch_bounds__(256) decode_prep_kernel(PrepParams p) {
 }  // namespace
 
 
+// The tensor-core split kernel takes d = 128 with TurboQuant_mse values
+// (either rotation: only the query's and the output's rotation differ); the
+// CUDA-core path takes every other valid pair of quantizers.
+bool decode_fast_path(int d, bool vprod) { return d == kD && !vprod; }
+
 bool decode_supported(int d, int kbm, bool kprod, int vbm, bool vprod, bool kdense, bool vdense) {
   (void)kdense;
-  (void)vdense;  // either rotation: only the query's and the output's rotation differ
-  return d == kD && !vprod && vbm >= 1 && vbm <= 4 && kbm >= (kprod ? 0 : 1) && kbm <= 4;
+  (void)vdense;
+  return d >= 8 && d <= 256 && d % 8 == 0 && vbm >= (vprod ? 0 : 1) && vbm <= 4 && kbm >= (kprod ? 0 : 1) &&
+         kbm <= 4;
 }
 
 size_t decode_workspace_floats(int B, int Hq, int Hkv, bool prod, int ctas) {
@@ -299,6 +305,7 @@ cudaError_t launch_prep(const PrepParams &pp, bool pdl, cudaStream_t s) {
 }  // namespace dec
 
 cudaError_t launch_decode(const DecodeArgs &a, cudaStream_t s) {
+  if (!decode_fast_path(a.kq.d, a.vq.prod)) return launch_decode_general(a, s);
   const int64_t outn = (int64_t)a.B * a.Hq * kD;
   if (a.seq_len == 0) {
     zero_out_kernel<<<(unsigned)((outn + 255) / 256), 256, 0, s>>>(a.out, outn);

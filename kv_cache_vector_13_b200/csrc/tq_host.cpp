@@ -461,8 +461,12 @@ tq_status tq_dequant(const tq_quantizer *q, const tq_cache_view *in, int64_t B, 
 
 size_t tq_decode_workspace_bytes(int32_t B, int32_t Hq, int32_t Hkv, int64_t seq_len, int32_t d) {
   if (B <= 0 || Hq <= 0 || Hkv <= 0 || seq_len <= 0 || Hq % Hkv || !valid_dense_d(d)) return 0;
-  // sized for TurboQuant_prod keys (the larger case) so the query needs no quantizer
-  return tq::decode_workspace_floats(B, Hq, Hkv, true, tq::decode_ctas()) * sizeof(float);
+  // enough for either decode path (the quantizers are not arguments): the
+  // tensor-core split kernel (d = 128, sized for TurboQuant_prod keys) and
+  // the CUDA-core path (any d, prod values)
+  size_t fl = tq::general_decode_workspace_floats(B, Hq, Hkv, seq_len, d);
+  if (d == 128) fl = std::max(fl, tq::decode_workspace_floats(B, Hq, Hkv, true, tq::decode_ctas()));
+  return fl * sizeof(float);
 }
 
 }  // extern "C"
@@ -484,7 +488,6 @@ tq_status prepare_decode(const char *name, const tq_quantizer *kq, const tq_quan
   st = check_quantizer(vq, (nm + "(vq)").c_str(), &a->vq);
   if (st != TQ_OK) return st;
   if (a->kq.d != a->vq.d) return fail(TQ_EINVAL, "%s: K d=%d but V d=%d", name, a->kq.d, a->vq.d);
-  if (a->vq.prod) return fail(TQ_EUNSUPPORTED, "%s: prod values are not implemented", name);
   if (q_dtype != TQ_F32 && q_dtype != TQ_BF16 && q_dtype != TQ_F16)
     return fail(TQ_EINVAL, "%s: q_dtype=%d", name, (int)q_dtype);
   if (B < 0 || Hq < 0 || Hkv < 0 || seq_len < 0) return fail(TQ_EINVAL, "%s: negative size", name);

@@ -104,6 +104,14 @@ cudaError_t launch_search(const SearchArgs &a, cudaStream_t s);
 int decode_ctas();
 size_t decode_workspace_floats(int B, int Hq, int Hkv, bool prod, int ctas);
 
+// The CUDA-core decode for what the tensor-core split kernel does not take
+// (d other than 128, prod values): its sequence splits and workspace in
+// floats (both depend only on the arguments), and the launch.
+bool decode_fast_path(int d, bool vprod);
+int general_decode_splits(int B, int Hq, int Hkv, int64_t seq_len);
+size_t general_decode_workspace_floats(int B, int Hq, int Hkv, int64_t seq_len, int d);
+cudaError_t launch_decode_general(const DecodeArgs &a, cudaStream_t s);
+
 // Faults the kernels detect themselves (bits of a per-GPU word): a bounded
 // wait that expired, and a launch whose shared-memory layout check failed
 // (the kernel then writes nothing).

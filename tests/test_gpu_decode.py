@@ -24,14 +24,15 @@ DEV = "cuda"
 TOL = 2e-3
 
 
-def run_case(B, Hq, Hkv, N, kspec, vspec, seed=0, seq_lens=None, kv_scale=1.0, heads=None, scores=False):
+def run_case(B, Hq, Hkv, N, kspec, vspec, seed=0, seq_lens=None, kv_scale=1.0, heads=None, scores=False, d=128,
+             rotation=("hadamard", "hadamard")):
     g = torch.Generator(device=DEV).manual_seed(seed)
-    d = 128
     K = torch.randn((B, Hkv, N, d), generator=g, device=DEV) * kv_scale
     V = torch.randn((B, Hkv, N, d), generator=g, device=DEV)
     q = torch.randn((B, Hq, d), generator=g, device=DEV).to(torch.bfloat16)
-    kq = api.Quantizer(d, kspec[0], kspec[1], seed_rot=seed + 1, seed_qjl=seed + 2, device=DEV)
-    vq = api.Quantizer(d, vspec[0], vspec[1], seed_rot=seed + 3, device=DEV)
+    kq = api.Quantizer(d, kspec[0], kspec[1], seed_rot=seed + 1, seed_qjl=seed + 2, device=DEV, rotation=rotation[0])
+    vq = api.Quantizer(d, vspec[0], vspec[1], seed_rot=seed + 3, seed_qjl=seed + 4, device=DEV,
+                       rotation=rotation[1])
     kc, vc = api.encode(kq, K), api.encode(vq, V)
     sl = None if seq_lens is None else torch.tensor(seq_lens, dtype=torch.int32, device=DEV)
     sc = torch.full((B, Hq, N), float("nan"), device=DEV) if scores else None
@@ -374,3 +375,27 @@ def test_append_decode_with_batch_lengths_and_scores():
     torch.cuda.synchronize()
     assert torch.equal(ref, got)
     assert torch.equal(s_ref, s_got)
+
+
+# The CUDA-core path: d other than 128, prod values, dense rotations of any
+# d; ragged lengths (one batch empty), scores, a GQA group of 12 (two head
+# groups of a block) and a long enough cache for several sequence splits.
+@pytest.mark.parametrize("d,kspec,vspec,rotation,g", [
+    (64, (3, "prod"), (3, "mse"), ("hadamard", "hadamard"), 4),
+    (256, (4, "mse"), (3, "prod"), ("hadamard", "hadamard"), 4),
+    (128, (3, "prod"), (3, "prod"), ("hadamard", "hadamard"), 12),
+    (128, (2, "mse"), (2, "prod"), ("dense", "dense"), 4),
+    (200, (3, "mse"), (4, "mse"), ("dense", "dense"), 2),
+    (64, (1, "prod"), (1, "prod"), ("hadamard", "dense"), 1),
+])
+def test_decode_cuda_core_path(d, kspec, vspec, rotation, g):
+    Hkv = 2
+    run_case(3, g * Hkv, Hkv, 1500, kspec, vspec, seed=d + 7 * g + kspec[0], seq_lens=[1500, 0, 613],
+             scores=True, d=d, rotation=rotation)
+
+
+def test_decode_cuda_core_path_long_cache():
+    # one (batch, kv head) over 40000 tokens: the sequence split across blocks
+    out = run_case(1, 4, 1, 40000, (4, "prod"), (4, "prod"), seed=77, d=256, kv_scale=3.0)
+    assert np.all(np.isfinite(out))
+

@@ -134,13 +134,16 @@ def test_decode_argument_checks():
     assert need > 0
     assert dec(Hq=6, Hkv=4) == L.TQ_EINVAL
     assert dec(Hkv=0) == L.TQ_EINVAL
-    assert dec(vq=quant(variant=L.TQ_PROD)) == L.TQ_EUNSUPPORTED
+    # prod values and d = 256 pass validation up to the workspace check (no
+    # launch happens on these fake pointers)
+    assert dec(vq=quant(variant=L.TQ_PROD), ws_bytes=need - 1) == L.TQ_EWORKSPACE
+    need256 = L.lib().tq_decode_workspace_bytes(1, 8, 2, 100, 256)
+    assert dec(kq=quant(d=256), vq=quant(d=256, variant=L.TQ_PROD), ws_bytes=need256 - 1) == L.TQ_EWORKSPACE
     assert dec(kq=quant(d=64), vq=quant(d=128)) == L.TQ_EINVAL
     assert dec(ws_bytes=need - 1) == L.TQ_EWORKSPACE
     assert dec(ws=FAKE + 4) == L.TQ_EWORKSPACE
     assert dec(q=FAKE + 2) == L.TQ_EINVAL
     assert dec(scale=float("nan")) == L.TQ_EINVAL
-    assert dec(kq=quant(d=256), vq=quant(d=256)) == L.TQ_EUNSUPPORTED
     assert dec(B=0) == L.TQ_OK
 
 

@@ -37,12 +37,19 @@ def make_cache(qz, X):
     return out, Q.dequant(qz, enc).reshape(B, H, N, d)
 
 
-@pytest.mark.parametrize("kvar,kb,vb", [("mse", 4, 4), ("prod", 3, 3), ("prod", 4, 4), ("mse", 3, 2)])
-def test_packed_attention_equals_attention_on_dequantized_cache(kvar, kb, vb):
-    rng = np.random.default_rng(kb * 10 + vb)
-    B, Hq, Hkv, N, d = 2, 8, 2, 300, 128
+@pytest.mark.parametrize("kvar,kb,vvar,vb,d", [("mse", 4, "mse", 4, 128), ("prod", 3, "mse", 3, 128),
+                                               ("prod", 4, "mse", 4, 128), ("mse", 3, "mse", 2, 128),
+                                               ("prod", 3, "prod", 3, 64), ("mse", 2, "prod", 4, 256),
+                                               ("prod", 1, "prod", 1, 64)])
+def test_packed_attention_equals_attention_on_dequantized_cache(kvar, kb, vvar, vb, d):
+    # prod values: the values are summed in the rotated basis and S^T is
+    # applied once to the weighted sign sums; the result must equal
+    # attention over the dequantized values x_hat = n Pi^T (c + gamma
+    # sqrt(pi/2)/d S^T sign)
+    rng = np.random.default_rng(kb * 10 + vb + d)
+    B, Hq, Hkv, N = 2, 8, 2, 300
     kq = Q.Quantizer(d, kb, kvar, seed_rot=1, seed_qjl=2)
-    vq = Q.Quantizer(d, vb, "mse", seed_rot=3)
+    vq = Q.Quantizer(d, vb, vvar, seed_rot=3, seed_qjl=4)
     K = (rng.standard_normal((B, Hkv, N, d)) * rng.lognormal(0, 0.5, (1, Hkv, 1, d))).astype(np.float32)
     V = rng.standard_normal((B, Hkv, N, d)).astype(np.float32)
     q = rng.standard_normal((B, Hq, d))
