@@ -50,31 +50,54 @@ D = 128
 WORKLOADS = {
     "batched": dict(
         B=16, Hq=32, Hkv=8, N=131072, k=(3, "prod", 20, 21), v=(3, "mse", 22), gen="outlier_kv", seed=3, copies=1,
-        name="batched decode step (append 1 token + attend): B=16 Hq=32 Hkv=8 d=128 N=131072, bf16 K,V "
-             "N(0,1) with 2% outlier channels x8; K TurboQuant_prod b=3, V TurboQuant_mse b=3, "
-             "randomized Hadamard"),
+        desc="batched decode step (append 1 token + attend)", data="bf16 K,V N(0,1) with 2% outlier channels x8",
+        rot="randomized Hadamard"),
     "long70b": dict(
         B=1, Hq=64, Hkv=8, N=1 << 20, k=(4, "prod", 30, 31), v=(4, "mse", 32), gen="student_kv", seed=5, copies=1,
-        name="70B-shaped long-context decode: B=1 Hq=64 Hkv=8 d=128 N=2^20, bf16 K,V 0.5*StudentT(3)*"
-             "LogNormal(0,1) channel scales; K TurboQuant_prod b=4, V TurboQuant_mse b=4"),
+        desc="70B-shaped long-context decode", data="bf16 K,V 0.5*StudentT(3)*LogNormal(0,1) channel scales",
+        rot="randomized Hadamard"),
     "llama8b": dict(
         B=1, Hq=32, Hkv=8, N=32768, k=(4, "mse", 10), v=(4, "mse", 11), gen="llama8b_kv", seed=2, copies=8,
-        name="Llama-3.1-8B-shaped decode: B=1 Hq=32 Hkv=8 d=128 N=32768, bf16 K,V N(0,1)*LogNormal(0,0.5) "
-             "channel scales; K,V TurboQuant_mse b=4"),
+        desc="Llama-3.1-8B-shaped decode", data="bf16 K,V N(0,1)*LogNormal(0,0.5) channel scales",
+        rot="randomized Hadamard"),
 }
 HEADLINE = "batched"
-B, N = WORKLOADS[HEADLINE]["B"], WORKLOADS[HEADLINE]["N"]
+
+
+def workload(key, batch=None):
+    """The workload's parameters (batch optionally overridden, for smaller
+    profiling captures) with its full name."""
+    w = dict(WORKLOADS[key])
+    if batch:
+        w["B"] = batch
+    n = w["N"]
+    nstr = f"2^{n.bit_length() - 1}" if n & (n - 1) == 0 and n >= 1 << 20 else str(n)
+    w["name"] = (f"{w['desc']}: B={w['B']} Hq={w['Hq']} Hkv={w['Hkv']} d={D} N={nstr}, {w['data']}; "
+                 f"K TurboQuant_{w['k'][1]} b={w['k'][0]}, V TurboQuant_{w['v'][1]} b={w['v'][0]}, {w['rot']}")
+    return w
+
+
 FALLBACK_PEAKS = {"hbm_gbs": 6650.0, "bf16_tflops": 1590.0}
 # DRAM bytes (read + write) of one decode split-kernel launch on the headline
 # workload, from an ncu capture (dram__bytes_read.sum + dram__bytes_write.sum),
-# reported only while the decode source is the one it was taken on.
-TRAFFIC = {"bytes": None, "source_sha256": None}
+# reported only for that workload and while the decode sources are the ones
+# it was taken on.
+TRAFFIC = {"workload": None, "bytes": None, "source_sha256": None}
+DECODE_SOURCES = ("tq_decode.cu", "tq_decode_split.cuh", "tq_decode_regs.cu")
 
 
-def traffic_bytes():
-    with open(os.path.join(ROOT, "kv_cache_vector_13_b200", "csrc", "tq_decode.cu"), "rb") as f:
-        h = hashlib.sha256(f.read()).hexdigest()
-    return TRAFFIC["bytes"] if h == TRAFFIC["source_sha256"] else None
+def decode_source_sha256():
+    h = hashlib.sha256()
+    for f in DECODE_SOURCES:
+        with open(os.path.join(ROOT, "kv_cache_vector_13_b200", "csrc", f), "rb") as fh:
+            h.update(fh.read())
+    return h.hexdigest()
+
+
+def traffic_bytes(key, B):
+    if (key, B) != TRAFFIC["workload"]:
+        return None
+    return TRAFFIC["bytes"] if decode_source_sha256() == TRAFFIC["source_sha256"] else None
 
 
 def peaks():
@@ -158,7 +181,7 @@ def max_over_ranks(times, dist, device):
     return tt.tolist()
 
 
-def job_value(world_size, ms_per_step):
+def job_value(world_size, ms_per_step, B, N):
     """Whole-job KV-tokens/s: every rank decodes B * N tokens per step, and
     the job's step time is the slowest rank's."""
     return world_size * B * N / (ms_per_step * 1e-3)
@@ -171,8 +194,8 @@ class Setup:
     tq_encode from the seeded bf16 K/V, then the inputs are freed), the
     decode operator and the tail views of token N-1."""
 
-    def __init__(self, api, inputs, torch, dev, key, seed_shift=0):
-        w = WORKLOADS[key]
+    def __init__(self, api, inputs, torch, dev, key, seed_shift=0, batch=None):
+        w = workload(key, batch)
         self.w, self.key = w, key
         self.B, self.Hq, self.Hkv, self.N = w["B"], w["Hq"], w["Hkv"], w["N"]
         kb, kvar, ksr, *kqs = w["k"]
@@ -254,7 +277,7 @@ def run_ours(args):
             dist.barrier()
 
     stream = torch.cuda.Stream(device=dev)
-    s = Setup(api, inputs, torch, dev, HEADLINE, seed_shift=rank)
+    s = Setup(api, inputs, torch, dev, args.workload, seed_shift=rank, batch=args.batch)
     K_steps = args.steps
 
     # warm-up: at least W steps, and at least half a second of them, while the
@@ -325,7 +348,7 @@ def run_ours(args):
         dec_bytes = s.decode_bytes()
         achieved = dec_bytes / (dec_ms * 1e-3) / 1e9
         line = {
-            "metric": METRIC, "value": job_value(ws, ms_step), "unit": "KV-tokens/s", "n_gpus": ws,
+            "metric": METRIC, "value": job_value(ws, ms_step, s.B, s.N), "unit": "KV-tokens/s", "n_gpus": ws,
             "steps": K_steps, "warmup": n_warm, "ms_per_step": ms_step, "higher_is_better": True,
             "scaling": "weak", "vs_baseline": None, "dtype": "f32 encode; f16xf16->f32 mma decode",
             "data": "synthetic",
@@ -336,7 +359,7 @@ def run_ours(args):
                          "achieved": achieved, "peak": pk["hbm_gbs"], "unit": "GB/s",
                          "frac": achieved / pk["hbm_gbs"], "peak_kind": pk_kind,
                          "bytes_per_launch": dec_bytes, "ms_per_launch": dec_ms,
-                         "traffic": args.traffic if args.traffic is not None else traffic_bytes()},
+                         "traffic": args.traffic if args.traffic is not None else traffic_bytes(s.key, s.B)},
             "e2e": {"value": ws * s.B * s.N * K_steps / e2e_s, "unit": "KV-tokens/s",
                     "h2d_bytes_per_step": hin.numel() * hin.element_size(),
                     "d2h_bytes_per_step": hout.numel() * 4, "steps": K_steps,
@@ -352,7 +375,7 @@ def run_ours(args):
         pk, _ = peaks()
         if not args.no_extras and ws == 1:
             extras = {}
-            for key in ("long70b", "llama8b"):
+            for key in (k for k in WORKLOADS if k != args.workload):
                 e = Setup(api, inputs, torch, dev, key)
                 ms = time_decode_calls(torch, e, stream, 40)
                 by = e.decode_bytes()
@@ -364,7 +387,7 @@ def run_ours(args):
             line["decode_other_workloads"] = extras
             line["encode"] = [bench_encode(api, inputs, torch, dev, stream, v) for v in ("mse4", "prod3", "mse3_bf16")]
         if not args.no_cpu_baseline and ws == 1:
-            line["cpu_baseline"] = cpu_baseline_decode(budget_s=args.cpu_seconds)
+            line["cpu_baseline"] = cpu_baseline_decode(args.workload, args.batch, budget_s=args.cpu_seconds)
         print(json.dumps(line), flush=True)
     if dist is not None:
         dist.barrier()
@@ -415,13 +438,13 @@ def bench_encode(api, inputs, torch, dev, stream, variant="mse4"):
 CPU_TOKENS = 8192  # cached tokens of the oracle's sample slice
 
 
-def cpu_baseline_decode(budget_s=15.0, steps=None):
-    """Time the oracle on a bounded sample of the headline step: one (batch,
-    KV head) slice of CPU_TOKENS cached tokens drawn like the headline's
-    (outlier channels, prod-3 keys, mse-3 values); a sample step encodes the
-    new token's K and V and attends the slice's 4 query heads over it.  The
-    rate in token-heads/s is scaled to the headline's KV-tokens/s (a step
-    processes B * Hkv * N token-heads)."""
+def cpu_baseline_decode(key=HEADLINE, batch=None, budget_s=15.0, steps=None):
+    """Time the oracle on a bounded sample of the workload's step: one
+    (batch, KV head) slice of CPU_TOKENS cached tokens drawn like the
+    workload's, with its quantizers; a sample step encodes the new token's K
+    and V and attends the slice's query heads over it.  The rate in
+    token-heads/s is scaled to the workload's KV-tokens/s (a step processes
+    B * Hkv * N token-heads)."""
     import numpy as np
     from kv_cache_vector_13_b200 import inputs
     from oracle import attention as OA
@@ -431,11 +454,11 @@ def cpu_baseline_decode(budget_s=15.0, steps=None):
         blas_threads = max([i.get("num_threads", 1) for i in threadpool_info()] or [1])
     except Exception:  # pragma: no cover
         blas_threads = 1
-    w = WORKLOADS[HEADLINE]
+    w = workload(key, batch)
     cores = len(os.sched_getaffinity(0))
-    kb, kvar, ksr, kqs = w["k"]
+    kb, kvar, ksr, *kqs = w["k"]
     vb, vvar, vsr = w["v"]
-    kq = OQ.Quantizer(D, kb, kvar, seed_rot=ksr, seed_qjl=kqs)
+    kq = OQ.Quantizer(D, kb, kvar, seed_rot=ksr, seed_qjl=kqs[0] if kqs else 1)
     vq = OQ.Quantizer(D, vb, vvar, seed_rot=vsr)
     K, V = getattr(inputs, w["gen"])(N=CPU_TOKENS, B=1, seed=w["seed"], device="cpu")
     kc = {k: v[None, None] for k, v in OQ.encode(kq, K[0, 0].float().numpy(), aux=False).items()}
@@ -458,7 +481,7 @@ def cpu_baseline_decode(budget_s=15.0, steps=None):
             "blas_threads": blas_threads, "kind": "oracle",
             "sample": f"{done} x (one (batch, KV head) slice of {CPU_TOKENS} tokens drawn like the workload: "
                       f"oracle encode of the new K,V token + float64 decode attention of {g} query heads, "
-                      f"prod-3 keys, mse-3 values), scaled by token-heads to B={w['B']} x Hkv={w['Hkv']} x "
+                      f"{kvar}-{kb} keys, {vvar}-{vb} values), scaled by token-heads to B={w['B']} x Hkv={w['Hkv']} x "
                       f"N={w['N']}; {el:.1f} s of CPU time"}
 
 
@@ -467,13 +490,13 @@ def run_reference(args):
     if rank != 0:
         return
     warm = max(args.warmup, 3)
-    cpu_baseline_decode(steps=warm)
+    cpu_baseline_decode(args.workload, args.batch, steps=warm)
     n = args.ref_steps or min(args.steps, 20)
     t0 = time.perf_counter()
-    base = cpu_baseline_decode(steps=n)
+    base = cpu_baseline_decode(args.workload, args.batch, steps=n)
     el = time.perf_counter() - t0
     ws = int(os.environ.get("WORLD_SIZE", "1"))
-    w = WORKLOADS[HEADLINE]
+    w = workload(args.workload, args.batch)
     line = {"impl": "reference", "metric": METRIC, "value": base["value"], "unit": "KV-tokens/s",
             "n_gpus": ws, "steps": n, "warmup": warm,
             "ms_per_step": w["B"] * w["N"] / base["value"] * 1e3, "higher_is_better": True, "scaling": "weak",
@@ -493,6 +516,10 @@ def main():
     ap.add_argument("--steps", type=int, default=200)
     ap.add_argument("--warmup", type=int, default=10)
     ap.add_argument("--impl", default="ours", choices=["ours", "reference"])
+    ap.add_argument("--workload", default=HEADLINE, choices=list(WORKLOADS),
+                    help="the timed step's workload (the others are reported as extra keys)")
+    ap.add_argument("--batch", type=int, default=None,
+                    help="override the workload's batch (smaller cases for profiler captures)")
     ap.add_argument("--cpu-seconds", type=float, default=15.0)
     ap.add_argument("--no-cpu-baseline", action="store_true")
     ap.add_argument("--no-extras", action="store_true",

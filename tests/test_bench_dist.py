@@ -28,7 +28,8 @@ def _rank(rank, ws, port, out):
     got = bench.max_over_ranks(times, dist, "cpu")
     dist.barrier()
     dist.destroy_process_group()
-    out.put((rank, got, bench.job_value(w, got[0])))
+    w0 = bench.workload(bench.HEADLINE)
+    out.put((rank, got, bench.job_value(w, got[0], w0["B"], w0["N"])))
 
 
 def test_two_gloo_ranks_take_the_max_and_sum_tokens():
@@ -44,14 +45,15 @@ def test_two_gloo_ranks_take_the_max_and_sum_tokens():
         assert p.exitcode == 0
     for rank, got, val in res:
         assert got == [2.0, 10.0, 3.0]
-        assert val == pytest.approx(2 * bench.B * bench.N / (2.0e-3))
+        w0 = bench.workload(bench.HEADLINE)
+        assert val == pytest.approx(2 * w0["B"] * w0["N"] / (2.0e-3))
 
 
 def test_single_rank_needs_no_process_group(monkeypatch):
     monkeypatch.delenv("WORLD_SIZE", raising=False)
     assert bench.dist_setup() == (0, 0, 1)
     assert bench.max_over_ranks([1.0, 2.0], None, "cpu") == [1.0, 2.0]
-    assert bench.job_value(1, 1.0) == pytest.approx(bench.B * bench.N / 1e-3)
+    assert bench.job_value(1, 1.0, 16, 131072) == pytest.approx(16 * 131072 / 1e-3)
 
 
 def test_reference_arm_nonzero_rank_exits_without_work(monkeypatch, capsys):
@@ -60,6 +62,7 @@ def test_reference_arm_nonzero_rank_exits_without_work(monkeypatch, capsys):
 
     class Args:
         steps, warmup, ref_steps, gpus, cpu_seconds = 4, 3, 0, 2, 1.0
+        workload, batch = bench.HEADLINE, None
 
     bench.run_reference(Args())
     assert capsys.readouterr().out == ""
