@@ -241,15 +241,18 @@ __device__ __forceinline__ uint32_t pack_lo(float a, float b) {
 // The byte starting `SH` bits up the little-endian word pair (w0, w1), moved
 // into byte 1 of the lane's offset (byte 0 = 4*lane, +128 for the value
 // table): the entry's byte offset inside the table.
+// The word is shifted by the bit residue s % 8 only and the byte s / 8 of
+// the result selected, so every field of a word at the same residue shares
+// one shift.
 template <int SH>
 __device__ __forceinline__ uint32_t lut_addr(uint32_t w0, uint32_t w1, uint32_t laneoff) {
-  constexpr int s = SH & 31;
-  if constexpr (s % 8 == 0) {
-    return __byte_perm(w0, laneoff, 0x7604 | ((s / 8) << 4));
+  constexpr int s = SH & 31, r = s % 8, by = s / 8;
+  if constexpr (r == 0) {
+    return __byte_perm(w0, laneoff, 0x7604 | (by << 4));
   } else if constexpr (s + 8 <= 32) {
-    return __byte_perm(w0 >> s, laneoff, 0x7604);
-  } else {
-    return __byte_perm(__funnelshift_r(w0, w1, s), laneoff, 0x7604);
+    return __byte_perm(w0 >> r, laneoff, 0x7604 | (by << 4));
+  } else {  // the byte crosses into w1 (by == 3)
+    return __byte_perm(__funnelshift_r(w0, w1, r), laneoff, 0x7604 | (by << 4));
   }
 }
 
@@ -273,6 +276,39 @@ struct VChunk {  // 16 dims of one token: 2*BM bytes
   static constexpr int NW = (2 * BM + 3) / 4;
 };
 
+// Two tokens' BM-bit streams of 16 dims (a, b) interleaved field by field:
+// field j of xe holds (a's code, b's code) of dim 2j as one 2BM-bit pair
+// index (a in the low bits: the pair tables' layout), xo the same for dim
+// 2j + 1; field j sits at bit 2 BM j, where pair j of a token's own stream
+// sits.
+template <int BM>
+__device__ __forceinline__ void interleave_tokens(const uint32_t (&a)[VChunk<BM>::NW],
+                                                  const uint32_t (&b)[VChunk<BM>::NW],
+                                                  uint32_t (&xe)[VChunk<BM>::NW], uint32_t (&xo)[VChunk<BM>::NW]) {
+  if constexpr (BM == 3) {
+    constexpr uint64_t Me = 0x1C71C71C71C7ull;  // bits [6j, 6j + 3), j < 8
+    const uint64_t A = ((uint64_t)a[1] << 32) | a[0], B = ((uint64_t)b[1] << 32) | b[0];
+    const uint64_t e = (A & Me) | ((B << 3) & (Me << 3));
+    const uint64_t o = ((A >> 3) & Me) | (B & (Me << 3));
+    xe[0] = (uint32_t)e;
+    xe[1] = (uint32_t)(e >> 32);
+    xo[0] = (uint32_t)o;
+    xo[1] = (uint32_t)(o >> 32);
+  } else if constexpr (BM == 2) {
+    xe[0] = (a[0] & 0x33333333u) | ((b[0] << 2) & 0xCCCCCCCCu);
+    xo[0] = ((a[0] >> 2) & 0x33333333u) | (b[0] & 0xCCCCCCCCu);
+  } else if constexpr (BM == 1) {
+    xe[0] = (a[0] & 0x5555u) | ((b[0] << 1) & 0xAAAAu);
+    xo[0] = ((a[0] >> 1) & 0x5555u) | (b[0] & 0xAAAAu);
+  } else {  // BM == 4: fields stay inside their bytes
+#pragma unroll
+    for (int w = 0; w < 2; ++w) {
+      xe[w] = (a[w] & 0x0F0F0F0Fu) | ((b[w] << 4) & 0xF0F0F0F0u);
+      xo[w] = ((a[w] >> 4) & 0x0F0F0F0Fu) | (b[w] & 0xF0F0F0F0u);
+    }
+  }
+}
+
 template <int BM>
 __device__ __forceinline__ void load_v16(const uint8_t *p, uint32_t (&W)[VChunk<BM>::NW], int g) {
   // bytes [2*BM*g, 2*BM*g + 2*BM) of the record, naturally aligned pieces only
@@ -284,16 +320,14 @@ __device__ __forceinline__ void load_v16(const uint8_t *p, uint32_t (&W)[VChunk<
     W[0] = __ldg(reinterpret_cast<const uint32_t *>(p));
   } else if constexpr (BM == 1) {
     W[0] = __ldg(reinterpret_cast<const unsigned short *>(p));
-  } else {  // BM == 3: 6 bytes at 6g, 2-byte aligned
-    if ((g & 1) == 0) {
-      W[0] = __ldg(reinterpret_cast<const uint32_t *>(p));
-      W[1] = __ldg(reinterpret_cast<const unsigned short *>(p + 4));
-    } else {
-      const uint32_t lo = __ldg(reinterpret_cast<const unsigned short *>(p));
-      const uint32_t hi = __ldg(reinterpret_cast<const uint32_t *>(p + 2));
-      W[0] = lo | (hi << 16);
-      W[1] = hi >> 16;
-    }
+  } else {  // BM == 3: 6 bytes at 6g of a 48-byte record, 2-byte aligned:
+    // the two words at the 4-byte boundary below (still inside the record),
+    // shifted down by 16 bits for odd g, with no branch
+    const uint32_t *q = reinterpret_cast<const uint32_t *>(p - 2 * (g & 1));
+    const uint32_t lo = __ldg(q), hi = __ldg(q + 1);
+    const int sh = 16 * (g & 1);
+    W[0] = __funnelshift_r(lo, hi, sh);
+    W[1] = (hi >> sh) & 0xFFFFu;
   }
 }
 
@@ -1295,50 +1329,24 @@ __global__ void __launch_bounds__(split_warps<PACK, KPROD, STAGED>() * 32, 1) de
           }
         }
         const auto &vw = vb.w[ms];
-        if constexpr (VBM == 4) {
-          // cross-nibble bytes: (token a, dim) | (token b, dim) << 4
-          uint32_t x0[2][2], x1[2][2];
-#pragma unroll
-          for (int pr = 0; pr < 2; ++pr) {
-#pragma unroll
-            for (int w = 0; w < 2; ++w) {
-              const uint32_t wa = vw[2 * pr][w], wb = vw[2 * pr + 1][w];
-              x0[pr][w] = (wa & 0x0F0F0F0Fu) | ((wb << 4) & 0xF0F0F0F0u);
-              x1[pr][w] = ((wa >> 4) & 0x0F0F0F0Fu) | (wb & 0xF0F0F0F0u);
-            }
-          }
-#define TQ_VSTEP4(MT)                                                             \
-  {                                                                               \
-    uint32_t a[4];                                                                \
-    a[0] = lut(pair_addr<4, MT, 2>(x0[0], voff));                           \
-    a[1] = lut(pair_addr<4, MT, 2>(x1[0], voff));                           \
-    a[2] = lut(pair_addr<4, MT, 2>(x0[1], voff));                           \
-    a[3] = lut(pair_addr<4, MT, 2>(x1[1], voff));                           \
-    mma16816(acc[MT], a, b0, b1);                                                 \
-    if constexpr (!PACK) mma16816(acc[MT], a, b2, b3);                            \
-  }
-          TQ_VSTEP4(0) TQ_VSTEP4(1) TQ_VSTEP4(2) TQ_VSTEP4(3)
-          TQ_VSTEP4(4) TQ_VSTEP4(5) TQ_VSTEP4(6) TQ_VSTEP4(7)
-#undef TQ_VSTEP4
-        } else {
+        // tokens (q4 = 0, 1) and (2, 3) interleaved into pair indices: the
+        // table then yields A's (token, token) pairs at one dim directly
+        uint32_t xe[2][VW], xo[2][VW];
+        interleave_tokens<VBM>(vw[0], vw[1], xe[0], xo[0]);
+        interleave_tokens<VBM>(vw[2], vw[3], xe[1], xo[1]);
 #define TQ_VSTEP(MT)                                                              \
   {                                                                               \
-    const uint32_t h0_ = lut(pair_addr<VBM, MT, VW>(vw[0], voff));          \
-    const uint32_t h1_ = lut(pair_addr<VBM, MT, VW>(vw[1], voff));          \
-    const uint32_t h2_ = lut(pair_addr<VBM, MT, VW>(vw[2], voff));          \
-    const uint32_t h3_ = lut(pair_addr<VBM, MT, VW>(vw[3], voff));          \
     uint32_t a[4];                                                                \
-    a[0] = __byte_perm(h0_, h1_, 0x5410);                                         \
-    a[1] = __byte_perm(h0_, h1_, 0x7632);                                         \
-    a[2] = __byte_perm(h2_, h3_, 0x5410);                                         \
-    a[3] = __byte_perm(h2_, h3_, 0x7632);                                         \
+    a[0] = lut(pair_addr<VBM, MT, VW>(xe[0], voff));                              \
+    a[1] = lut(pair_addr<VBM, MT, VW>(xo[0], voff));                              \
+    a[2] = lut(pair_addr<VBM, MT, VW>(xe[1], voff));                              \
+    a[3] = lut(pair_addr<VBM, MT, VW>(xo[1], voff));                              \
     mma16816(acc[MT], a, b0, b1);                                                 \
     if constexpr (!PACK) mma16816(acc[MT], a, b2, b3);                            \
   }
-          TQ_VSTEP(0) TQ_VSTEP(1) TQ_VSTEP(2) TQ_VSTEP(3)
-          TQ_VSTEP(4) TQ_VSTEP(5) TQ_VSTEP(6) TQ_VSTEP(7)
+        TQ_VSTEP(0) TQ_VSTEP(1) TQ_VSTEP(2) TQ_VSTEP(3)
+        TQ_VSTEP(4) TQ_VSTEP(5) TQ_VSTEP(6) TQ_VSTEP(7)
 #undef TQ_VSTEP
-        }
       }
       if constexpr (STAGED) {
         // the slot is read: refill it with the chunk R ahead
