@@ -385,7 +385,7 @@ def run_ours(args):
                 del e
                 torch.cuda.empty_cache()
             line["decode_other_workloads"] = extras
-            line["encode"] = [bench_encode(api, inputs, torch, dev, stream, v) for v in ("mse4", "prod3", "mse3_bf16")]
+            line["encode"] = [bench_encode(api, inputs, torch, dev, stream, v) for v in ENCODE_VARIANTS]
         if not args.no_cpu_baseline and ws == 1:
             line["cpu_baseline"] = cpu_baseline_decode(args.workload, args.batch, budget_s=args.cpu_seconds)
         print(json.dumps(line), flush=True)
@@ -394,19 +394,33 @@ def run_ours(args):
         dist.destroy_process_group()
 
 
+ENCODE_VARIANTS = ("mse4", "prod3", "mse3_bf16", "prod3_bf16")
+
+
+def run_encode_only(variant):
+    """Only the encode measurement of one variant (for profiler captures)."""
+    import torch
+    from kv_cache_vector_13_b200 import api, inputs
+    dev = torch.device("cuda", 0)
+    torch.cuda.set_device(dev)
+    stream = torch.cuda.Stream(device=dev)
+    print(json.dumps({"encode": bench_encode(api, inputs, torch, dev, stream, variant)}), flush=True)
+
+
 def bench_encode(api, inputs, torch, dev, stream, variant="mse4"):
     """Encode throughput on 2^20 vectors, d=128, 2 rotating inputs (larger
     than L2 together): "mse4" / "prod3" are the encode sweep's d=128 cells
     (unit vectors, fp32, TurboQuant_mse b=4 / TurboQuant_prod b=3);
-    "mse3_bf16" encodes bf16 rows like the decode workloads' values."""
+    "mse3_bf16" / "prod3_bf16" encode bf16 rows like the decode workloads'
+    values / keys."""
     n, d = 1 << 20, 128
-    if variant == "prod3":
+    if variant in ("prod3", "prod3_bf16"):
         qz = api.Quantizer(d, 3, "prod", seed_rot=0, seed_qjl=1, device=dev)
     elif variant == "mse3_bf16":
         qz = api.Quantizer(d, 3, "mse", seed_rot=0, device=dev)
     else:
         qz = api.Quantizer(d, 4, "mse", seed_rot=0, device=dev)
-    if variant == "mse3_bf16":
+    if variant.endswith("_bf16"):
         xs = [inputs.vectors(n, d, seed=i, device=dev).to(torch.bfloat16) for i in range(4)]
     else:
         xs = [inputs.unit_vectors(n, d, seed=i, device=dev) for i in range(2)]
@@ -428,7 +442,8 @@ def bench_encode(api, inputs, torch, dev, stream, variant="mse4"):
     gbs = byts / (ms * 1e-3) / 1e9
     names = {"mse4": "2^20 unit vectors d=128 fp32, TurboQuant_mse b=4",
              "prod3": "2^20 unit vectors d=128 fp32, TurboQuant_prod b=3",
-             "mse3_bf16": "2^20 N(0,1) vectors d=128 bf16, TurboQuant_mse b=3"}
+             "mse3_bf16": "2^20 N(0,1) vectors d=128 bf16, TurboQuant_mse b=3",
+             "prod3_bf16": "2^20 N(0,1) vectors d=128 bf16, TurboQuant_prod b=3"}
     return {"workload": names[variant], "vectors_per_s": n / (ms * 1e-3), "ms_per_launch": ms,
             "bytes_per_launch": byts, "achieved_gbs": gbs, "frac": gbs / pk["hbm_gbs"]}
 
@@ -527,8 +542,12 @@ def main():
     ap.add_argument("--ref-steps", type=int, default=0)
     ap.add_argument("--traffic", type=float, default=None,
                     help="dram bytes per decode call from an ncu capture of this build, if any")
+    ap.add_argument("--encode-only", default=None, choices=list(ENCODE_VARIANTS),
+                    help="measure only this encode variant (for profiler captures)")
     args = ap.parse_args()
-    if args.impl == "reference":
+    if args.encode_only:
+        run_encode_only(args.encode_only)
+    elif args.impl == "reference":
         run_reference(args)
     else:
         run_ours(args)
