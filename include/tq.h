@@ -268,10 +268,12 @@ tq_status tq_decode_attention_noalloc(const tq_quantizer *kq, const tq_quantizer
  * own rotated basis and rotated back into its channels of out[B][Hq][d].
  * The rest as for tq_decode_attention (q: [B][Hq][d]; GQA; seq_lens;
  * softmax_scale); d <= 256.  workspace: DEVICE, at least
- * tq_decode_split_workspace_bytes(B, Hq, seq_len) bytes, 16-byte aligned.
- * Plain CUDA-core kernels (one pass for the scores, one for softmax and
- * values). */
-size_t tq_decode_split_workspace_bytes(int32_t B, int32_t Hq, int64_t seq_len);
+ * tq_decode_split_workspace_bytes(B, Hq, Hkv, seq_len, d) bytes, 16-byte
+ * aligned, else TQ_EWORKSPACE.  CUDA cores in fp32: a split over the
+ * sequence (blocks of up to 8 query heads by token slices, an online
+ * softmax per head) and one merge block per query head. */
+size_t tq_decode_split_workspace_bytes(int32_t B, int32_t Hq, int32_t Hkv, int64_t seq_len,
+                                       int32_t d);
 tq_status tq_decode_attention_split(const tq_quantizer kq[2], const tq_quantizer vq[2],
                                     const void *q, tq_dtype q_dtype, int32_t B, int32_t Hq,
                                     int32_t Hkv, int64_t seq_len, const int32_t *seq_lens,

@@ -102,7 +102,7 @@ def lib() -> ctypes.CDLL:
     L.tq_search_topk.argtypes = [POINTER(TqQuantizer), POINTER(TqCacheView), c_int64, c_void_p, c_int32, c_int32,
                                  c_int32, c_void_p, c_void_p, c_void_p, c_size_t, c_void_p]
     L.tq_search_topk.restype = c_int32
-    L.tq_decode_split_workspace_bytes.argtypes = [c_int32, c_int32, c_int64]
+    L.tq_decode_split_workspace_bytes.argtypes = [c_int32, c_int32, c_int32, c_int64, c_int32]
     L.tq_decode_split_workspace_bytes.restype = c_size_t
     L.tq_decode_attention_split.argtypes = [
         POINTER(TqQuantizer), POINTER(TqQuantizer), c_void_p, c_int32, c_int32, c_int32, c_int32, c_int64,

@@ -297,7 +297,7 @@ class DecodeAttentionSplit:
     def __init__(self, kq: SplitQuantizer, vq: SplitQuantizer, B: int, Hq: int, Hkv: int, seq_len: int,
                  device="cuda"):
         self.kq, self.vq, self.B, self.Hq, self.Hkv, self.seq_len = kq, vq, B, Hq, Hkv, seq_len
-        nb = int(L.lib().tq_decode_split_workspace_bytes(B, Hq, seq_len))
+        nb = int(L.lib().tq_decode_split_workspace_bytes(B, Hq, Hkv, seq_len, kq.d))
         self.workspace = torch.empty(max(nb, 16), dtype=torch.uint8, device=device)
         self.ws_bytes = nb
         self.out = torch.empty((B, Hq, kq.d), dtype=torch.float32, device=device)

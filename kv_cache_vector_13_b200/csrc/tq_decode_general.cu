@@ -1,23 +1,28 @@
-// Decode attention on CUDA cores (sm_100a) for the quantizers the
-// tensor-core split kernel does not take: d = 64 or 256 with the Hadamard
-// rotation, dense (Haar) rotations of any supported d other than 128, and
-// TurboQuant_prod values.  Same definition as the main path ("I Spent 31
-// Hours On The Math Behind Turboquant", section "KV Cache: The problem";
-// "内存厂商的噩梦来了", section 4.2, the asymmetric score):
-//   s_j = n_j (<q', c_K[idx_j]> + [prod] ||r_j|| sqrt(pi/2)/d <S_K q', sign_j>),
-//   q' = Pi_K q, softmax over s_j * scale, and the values summed in their
-//   rotated basis, o' = sum_j p_j n_j (c_V[idx_j] + [prod] ||r_j|| sqrt(pi/2)/d
-//   S_V^T sign_j), rotated back once, o = Pi_V^T o'.
+// Decode attention on CUDA cores (sm_100a) for the caches the tensor-core
+// split kernel does not take: d = 64 or 256 with the Hadamard rotation,
+// dense (Haar) rotations of any supported d other than 128, TurboQuant_prod
+// values, and outlier-channel split caches.  Same definition as the main
+// path ("I Spent 31 Hours On The Math Behind Turboquant", section "KV Cache:
+// The problem"; "内存厂商的噩梦来了", section 4.2, the asymmetric score):
+//   s_j = sum_g n_gj (<q'_g, c_g[idx_gj]> + [prod] ||r_gj|| sqrt(pi/2)/d_g <S_g q'_g, sign_gj>),
+//   q'_g = Pi_g q[channels_g], softmax over s_j * scale, and each value group
+//   summed in its rotated basis, o'_g = sum_j p_j n_gj (c_g[idx_gj] + [prod]
+//   ||r_gj|| sqrt(pi/2)/d_g S_g^T sign_gj), rotated back once into its
+//   channels, o[channels_g] = Pi_g^T o'_g.  A plain cache is one group over
+//   all d channels; an outlier-channel split cache ("TurboQuant của Google",
+//   the correction in the experiments section) is two.
 //
 // Flash-decoding split over the sequence:
 //   general_partial_kernel, grid (splits, B * Hkv * head groups): up to 8
 //     query heads of one kv head over one token slice, in tiles of 64
-//     tokens: scores (4 threads a token), an online softmax per head, then a
-//     thread per (head, coordinate) accumulates the weighted centroids (and,
-//     for prod values, the weighted signs) of the tile; the slice's
-//     (m, l, o', signs) go to a workspace slot;
+//     tokens: scores (4 threads a token), an online softmax per head, then
+//     the values 8 tokens at a time: each (token, coordinate) decoded once
+//     into shared memory, and a thread per (head, coordinate) accumulating
+//     the weighted centroids (and, for prod values, the weighted signs); the
+//     slice's (m, l, o', signs) go to a workspace slot;
 //   general_merge_kernel, a block per (batch, query head): merges the slots,
-//   adds S_V^T of the sign sums, applies the inverse rotation and 1/l.
+//   adds S_g^T of the sign sums, applies each group's inverse rotation and
+//   1/l, and scatters the groups into their channels.
 
 #include "../../include/tq.h"
 #include "tq_device.cuh"
@@ -30,22 +35,28 @@ constexpr int kGnThreads = 256;
 constexpr int kGnMaxD = 256;
 constexpr int kGnHeads = 8;   // query heads a block
 constexpr int kGnTile = 64;   // tokens a tile
+constexpr int kGnSub = 8;     // tokens a value-decode step
 constexpr int kGnCoords = kGnHeads * kGnMaxD / kGnThreads;  // (head, coordinate) pairs a thread
 constexpr float kGnLog2e = 1.4426950408889634f;
 constexpr float kGnSqrtHalfPi = 1.2533141373155003f;
 
-struct GnSide {
-  int bm;
+// One quantizer group: its dimension and offset among the head's
+// rotated coordinates, codebook, rotation (dense Pi, or the Hadamard signs
+// when rot is NULL), channel list (NULL: channels 0..d-1), and its cache.
+struct GnGroup {
+  int d, off, bm;
   bool prod;
   const float *cent, *rot, *S;
   const int8_t *signs;
+  const int32_t *chan;
   const uint8_t *codes, *qjl;
   const float *norms, *rnorms;
   int64_t sb, sh, sn;
 };
 
 struct GnParams {
-  GnSide k, v;
+  GnGroup k[2], v[2];
+  int nk, nv;        // groups per side (1 or 2)
   const void *q;
   int q_dtype;
   int B, Hq, Hkv, g, hg, d, splits;
@@ -103,11 +114,12 @@ __device__ void gn_fwht(float *x, int nv, int d, int stride) {
 }
 
 __global__ void __launch_bounds__(kGnThreads) general_partial_kernel(GnParams p) {
-  __shared__ float s_q[kGnHeads][kGnMaxD];   // q' (rotated query)
-  __shared__ float s_qs[kGnHeads][kGnMaxD];  // S_K q' (prod keys); staging of q otherwise
+  __shared__ float s_q[kGnHeads][kGnMaxD];   // q'_g at the group's offset
+  __shared__ float s_qs[kGnHeads][kGnMaxD];  // S_g q'_g (prod groups); staging of q[channels] first
   __shared__ float s_w[kGnHeads][kGnTile];   // logits, then weights
-  __shared__ float s_vn[kGnTile], s_vr[kGnTile];
+  __shared__ float s_vn[2][kGnTile], s_vr[2][kGnTile];
   __shared__ float s_alpha[kGnHeads], s_m[kGnHeads], s_l[kGnHeads];
+  __shared__ float s_vx[2][kGnSub][kGnMaxD];  // decoded values (and prod sign terms)
   const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
   const int d = p.d;
   const int split = blockIdx.x;
@@ -120,38 +132,47 @@ __global__ void __launch_bounds__(kGnThreads) general_partial_kernel(GnParams p)
   const int64_t t0 = (int64_t)split * p.per_split;
   const int64_t t1 = min(L, t0 + p.per_split);
 
-  // ---- q' = Pi_K q for the block's heads (and S_K q' for prod keys)
-  for (int e = tid; e < nh * d; e += kGnThreads) {
-    const int hh = e / d, i = e % d;
-    const float x = gn_q(p, ((int64_t)b * p.Hq + h0 + hh) * d + i);
-    if (p.k.rot) {
-      s_qs[hh][i] = x;
-    } else {
-      s_q[hh][i] = p.k.signs[i] < 0 ? -x : x;
+  // ---- q'_g = Pi_g q[channels_g] for the block's heads (and S_g q'_g)
+  for (int gr = 0; gr < p.nk; ++gr) {
+    const GnGroup &G = p.k[gr];
+    for (int e = tid; e < nh * G.d; e += kGnThreads) {
+      const int hh = e / G.d, c = e % G.d;
+      const int ch = G.chan ? min(max(__ldg(G.chan + c), 0), d - 1) : c;
+      const float x = gn_q(p, ((int64_t)b * p.Hq + h0 + hh) * d + ch);
+      if (G.rot) {
+        s_qs[hh][G.off + c] = x;
+      } else {
+        s_q[hh][G.off + c] = G.signs[c] < 0 ? -x : x;
+      }
     }
   }
   __syncthreads();
-  if (p.k.rot) {
-    for (int e = tid; e < nh * d; e += kGnThreads) {
-      const int hh = e / d, r = e % d;
-      const float *row = p.k.rot + (int64_t)r * d;
-      float acc = 0.f;
-      for (int c = 0; c < d; ++c) acc = fmaf(__ldg(row + c), s_qs[hh][c], acc);
-      s_q[hh][r] = acc;
+  for (int gr = 0; gr < p.nk; ++gr) {
+    const GnGroup &G = p.k[gr];
+    if (G.rot) {
+      for (int e = tid; e < nh * G.d; e += kGnThreads) {
+        const int hh = e / G.d, r = e % G.d;
+        const float *row = G.rot + (int64_t)r * G.d;
+        float acc = 0.f;
+        for (int c = 0; c < G.d; ++c) acc = fmaf(__ldg(row + c), s_qs[hh][G.off + c], acc);
+        s_q[hh][G.off + r] = acc;
+      }
+    } else {  // Hadamard: a single group at offset 0
+      gn_fwht(&s_q[0][0], nh, G.d, kGnMaxD);
+      const float inv = rsqrtf((float)G.d);
+      for (int e = tid; e < nh * G.d; e += kGnThreads) s_q[e / G.d][e % G.d] *= inv;
     }
-  } else {
-    gn_fwht(&s_q[0][0], nh, d, kGnMaxD);
-    const float inv = rsqrtf((float)d);
-    for (int e = tid; e < nh * d; e += kGnThreads) s_q[e / d][e % d] *= inv;
   }
   __syncthreads();
-  if (p.k.prod) {
-    for (int e = tid; e < nh * d; e += kGnThreads) {
-      const int hh = e / d, r = e % d;
-      const float *row = p.k.S + (int64_t)r * d;
+  for (int gr = 0; gr < p.nk; ++gr) {
+    const GnGroup &G = p.k[gr];
+    if (!G.prod) continue;
+    for (int e = tid; e < nh * G.d; e += kGnThreads) {
+      const int hh = e / G.d, r = e % G.d;
+      const float *row = G.S + (int64_t)r * G.d;
       float acc = 0.f;
-      for (int c = 0; c < d; ++c) acc = fmaf(__ldg(row + c), s_q[hh][c], acc);
-      s_qs[hh][r] = acc;
+      for (int c = 0; c < G.d; ++c) acc = fmaf(__ldg(row + c), s_q[hh][G.off + c], acc);
+      s_qs[hh][G.off + r] = acc;
     }
   }
   if (tid < kGnHeads) {
@@ -162,61 +183,79 @@ __global__ void __launch_bounds__(kGnThreads) general_partial_kernel(GnParams p)
 
   // this thread's (head, coordinate) pairs: e = tid + kGnThreads * c
   float acc[kGnCoords], sacc[kGnCoords];
+  int c_h[kGnCoords], c_i[kGnCoords];
+  bool c_prod[kGnCoords];
 #pragma unroll
-  for (int c = 0; c < kGnCoords; ++c) acc[c] = sacc[c] = 0.f;
-  const int kcb = d * p.k.bm / 8, vcb = d * p.v.bm / 8;
-  const int64_t kbase = (int64_t)b * p.k.sb + (int64_t)kvh * p.k.sh;
-  const int64_t vbase = (int64_t)b * p.v.sb + (int64_t)kvh * p.v.sh;
-  const float kkap = kGnSqrtHalfPi / (float)d;
+  for (int c = 0; c < kGnCoords; ++c) {
+    acc[c] = sacc[c] = 0.f;
+    const int e = tid + kGnThreads * c;
+    c_h[c] = e < nh * d ? e / d : -1;
+    c_i[c] = e % d;
+    c_prod[c] = p.v[(p.nv == 2 && c_i[c] >= p.v[1].off) ? 1 : 0].prod;
+  }
+  // the value decode's (token, coordinate) share: coordinate dec_i of
+  // tokens dec_t, dec_t + dec_step, ...
+  const int dec_step = kGnThreads / d;
+  const int dec_i = tid < dec_step * d ? tid % d : -1;
+  const int dec_t = tid / d;
 
   for (int64_t base = t0; base < t1; base += kGnTile) {
     const int nt = (int)min((int64_t)kGnTile, t1 - base);
-    // ---- scores: 4 threads a token, d/4 coordinates each
+    // ---- scores: 4 threads a token, a quarter of every group's coordinates each
     {
       const int tt = tid >> 2, qq = tid & 3;
       const bool ok = tt < nt;
       const int64_t j = base + (ok ? tt : 0);
-      const int64_t kr = kbase + j * p.k.sn;
-      float part[kGnHeads], qpart[kGnHeads];
+      float tot[kGnHeads];
 #pragma unroll
-      for (int hh = 0; hh < kGnHeads; ++hh) part[hh] = qpart[hh] = 0.f;
+      for (int hh = 0; hh < kGnHeads; ++hh) tot[hh] = 0.f;
       if (ok) {
-        const uint8_t *kc = p.k.bm > 0 ? p.k.codes + kr * kcb : nullptr;
-        const uint8_t *kj = p.k.prod ? p.k.qjl + kr * (d / 8) : nullptr;
-        const int i0 = qq * (d / 4), i1 = i0 + d / 4;
-        for (int i = i0; i < i1; ++i) {
-          const float c = p.k.bm > 0 ? __ldg(p.k.cent + gn_field(kc, i, p.k.bm, kcb)) : 0.f;
-          const float sg = p.k.prod ? (gn_bit(kj, i) ? 1.f : -1.f) : 0.f;
+        for (int gr = 0; gr < p.nk; ++gr) {
+          const GnGroup &G = p.k[gr];
+          const int64_t kr = (int64_t)b * G.sb + (int64_t)kvh * G.sh + j * G.sn;
+          const int kcb = G.d * G.bm / 8;
+          const uint8_t *kc = G.bm > 0 ? G.codes + kr * kcb : nullptr;
+          const uint8_t *kj = G.prod ? G.qjl + kr * (G.d / 8) : nullptr;
+          float part[kGnHeads], qpart[kGnHeads];
 #pragma unroll
-          for (int hh = 0; hh < kGnHeads; ++hh) {
-            if (hh < nh) {
-              part[hh] = fmaf(c, s_q[hh][i], part[hh]);
-              if (p.k.prod) qpart[hh] = fmaf(sg, s_qs[hh][i], qpart[hh]);
+          for (int hh = 0; hh < kGnHeads; ++hh) part[hh] = qpart[hh] = 0.f;
+          const int i0 = qq * (G.d / 4), i1 = i0 + G.d / 4;
+          for (int i = i0; i < i1; ++i) {
+            const float c = G.bm > 0 ? __ldg(G.cent + gn_field(kc, i, G.bm, kcb)) : 0.f;
+            const float sg = G.prod ? (gn_bit(kj, i) ? 1.f : -1.f) : 0.f;
+#pragma unroll
+            for (int hh = 0; hh < kGnHeads; ++hh) {
+              if (hh < nh) {
+                part[hh] = fmaf(c, s_q[hh][G.off + i], part[hh]);
+                if (G.prod) qpart[hh] = fmaf(sg, s_qs[hh][G.off + i], qpart[hh]);
+              }
             }
           }
+          const float n = __ldg(G.norms + kr);
+          const float kap = G.prod ? __ldg(G.rnorms + kr) * (kGnSqrtHalfPi / (float)G.d) : 0.f;
+#pragma unroll
+          for (int hh = 0; hh < kGnHeads; ++hh) tot[hh] = fmaf(n, fmaf(kap, qpart[hh], part[hh]), tot[hh]);
         }
       }
 #pragma unroll
       for (int hh = 0; hh < kGnHeads; ++hh) {
-        part[hh] += __shfl_xor_sync(dev::kFull, part[hh], 1);
-        part[hh] += __shfl_xor_sync(dev::kFull, part[hh], 2);
-        qpart[hh] += __shfl_xor_sync(dev::kFull, qpart[hh], 1);
-        qpart[hh] += __shfl_xor_sync(dev::kFull, qpart[hh], 2);
+        tot[hh] += __shfl_xor_sync(dev::kFull, tot[hh], 1);
+        tot[hh] += __shfl_xor_sync(dev::kFull, tot[hh], 2);
       }
-      if (qq == 0 && tt < kGnTile) {
-        const float n = ok ? __ldg(p.k.norms + kr) : 0.f;
-        const float kap = (ok && p.k.prod) ? __ldg(p.k.rnorms + kr) * kkap : 0.f;
+      if (qq == 0) {
 #pragma unroll
         for (int hh = 0; hh < kGnHeads; ++hh) {
           if (hh < nh) {
-            const float s = n * (part[hh] + kap * qpart[hh]);
-            s_w[hh][tt] = ok ? s * p.scale_log2 : -INFINITY;
-            if (ok && p.scores) p.scores[((int64_t)b * p.Hq + h0 + hh) * p.seq_len + j] = s;
+            s_w[hh][tt] = ok ? tot[hh] * p.scale_log2 : -INFINITY;
+            if (ok && p.scores) p.scores[((int64_t)b * p.Hq + h0 + hh) * p.seq_len + j] = tot[hh];
           }
         }
-        const int64_t vr = vbase + j * p.v.sn;
-        s_vn[tt] = ok ? __ldg(p.v.norms + vr) : 0.f;
-        s_vr[tt] = (ok && p.v.prod) ? __ldg(p.v.rnorms + vr) * kkap : 0.f;
+      }
+      if (qq < p.nv) {  // thread qq of the token loads value group qq's norms
+        const GnGroup &G = p.v[qq];
+        const int64_t vr = (int64_t)b * G.sb + (int64_t)kvh * G.sh + j * G.sn;
+        s_vn[qq][tt] = ok ? __ldg(G.norms + vr) : 0.f;
+        s_vr[qq][tt] = (ok && G.prod) ? __ldg(G.rnorms + vr) * (kGnSqrtHalfPi / (float)G.d) : 0.f;
       }
     }
     __syncthreads();
@@ -243,27 +282,52 @@ __global__ void __launch_bounds__(kGnThreads) general_partial_kernel(GnParams p)
       }
     }
     __syncthreads();
-    // ---- values: thread (head, coordinate) pairs over the tile
+    // ---- values, kGnSub tokens at a time: every (token, coordinate) is
+    // decoded once into shared memory (n_V c[idx], and for prod groups
+    // n_V ||r|| sqrt(pi/2)/d sign), then each (head, coordinate) thread
+    // accumulates its weights times them
 #pragma unroll
     for (int c = 0; c < kGnCoords; ++c) {
-      const int e = tid + kGnThreads * c;
-      if (e < nh * d) {
-        const int hh = e / d, i = e % d;
-        float a = acc[c] * s_alpha[hh], sa = sacc[c] * s_alpha[hh];
-        for (int tt = 0; tt < nt; ++tt) {
-          const float w = s_w[hh][tt] * s_vn[tt];
-          const int64_t vr = vbase + (base + tt) * p.v.sn;
-          if (p.v.bm > 0) a = fmaf(w, __ldg(p.v.cent + gn_field(p.v.codes + vr * vcb, i, p.v.bm, vcb)), a);
-          if (p.v.prod) {
-            const float wr = w * s_vr[tt];
-            sa += gn_bit(p.v.qjl + vr * (d / 8), i) ? wr : -wr;
-          }
-        }
-        acc[c] = a;
-        sacc[c] = sa;
+      if (c_h[c] >= 0) {
+        acc[c] *= s_alpha[c_h[c]];
+        sacc[c] *= s_alpha[c_h[c]];
       }
     }
-    __syncthreads();
+    for (int t8 = 0; t8 < nt; t8 += kGnSub) {
+      const int ns = min(kGnSub, nt - t8);
+      if (dec_i >= 0) {
+        const int gv = (p.nv == 2 && dec_i >= p.v[1].off) ? 1 : 0;
+        const GnGroup &G = p.v[gv];
+        const int li = dec_i - G.off;
+        const int vcb = G.d * G.bm / 8;
+        const int64_t vbase = (int64_t)b * G.sb + (int64_t)kvh * G.sh;
+        for (int tt = dec_t; tt < ns; tt += dec_step) {
+          const int64_t vr = vbase + (base + t8 + tt) * G.sn;
+          const float n = s_vn[gv][t8 + tt];
+          s_vx[0][tt][dec_i] = G.bm > 0 ? n * __ldg(G.cent + gn_field(G.codes + vr * vcb, li, G.bm, vcb)) : 0.f;
+          if (G.prod) {
+            const float r = n * s_vr[gv][t8 + tt];
+            s_vx[1][tt][dec_i] = gn_bit(G.qjl + vr * (G.d / 8), li) ? r : -r;
+          }
+        }
+      }
+      __syncthreads();
+#pragma unroll
+      for (int c = 0; c < kGnCoords; ++c) {
+        if (c_h[c] >= 0) {
+          const int hh = c_h[c], i = c_i[c];
+          float a = acc[c], sa = sacc[c];
+          for (int tt = 0; tt < ns; ++tt) {
+            const float w = s_w[hh][t8 + tt];
+            a = fmaf(w, s_vx[0][tt][i], a);
+            if (c_prod[c]) sa = fmaf(w, s_vx[1][tt][i], sa);
+          }
+          acc[c] = a;
+          sacc[c] = sa;
+        }
+      }
+      __syncthreads();
+    }
   }
 
   // ---- the slice's partial state
@@ -323,47 +387,76 @@ __global__ void __launch_bounds__(kGnThreads) general_merge_kernel(GnParams p) {
     s_s[i] = so;
   }
   __syncthreads();
-  if (p.v.prod) {  // o' += S_V^T (weighted signs); sqrt(pi/2)/d is in the weights
-    float add[kGnMaxD / kGnThreads];
-    for (int i = tid, c = 0; i < d; i += kGnThreads, ++c) {
-      float a = 0.f;
-      for (int k = 0; k < d; ++k) a = fmaf(__ldg(p.v.S + (int64_t)k * d + i), s_s[k], a);
-      add[c] = a;
+  // prod value groups: o'_g += S_g^T (weighted signs); sqrt(pi/2)/d_g is in the weights
+  float add[kGnMaxD / kGnThreads];
+  for (int i = tid, c = 0; i < d; i += kGnThreads, ++c) {
+    const int gv = (p.nv == 2 && i >= p.v[1].off) ? 1 : 0;
+    const GnGroup &G = p.v[gv];
+    float a = 0.f;
+    if (G.prod) {
+      const int li = i - G.off;
+      for (int k = 0; k < G.d; ++k) a = fmaf(__ldg(G.S + (int64_t)k * G.d + li), s_s[G.off + k], a);
     }
-    __syncthreads();
-    for (int i = tid, c = 0; i < d; i += kGnThreads, ++c) s_o[i] += add[c];
-    __syncthreads();
+    add[c] = a;
   }
+  __syncthreads();
+  for (int i = tid, c = 0; i < d; i += kGnThreads, ++c) s_o[i] += add[c];
+  __syncthreads();
   const float inv_l = l > 0.f ? 1.0f / l : 0.f;
-  if (p.v.rot) {  // o = Pi^T o'
-    for (int c = tid; c < d; c += kGnThreads) {
+  if (p.v[0].rot) {  // o[channels_g] = Pi_g^T o'_g
+    for (int i = tid; i < d; i += kGnThreads) {
+      const int gv = (p.nv == 2 && i >= p.v[1].off) ? 1 : 0;
+      const GnGroup &G = p.v[gv];
+      const int c = i - G.off;
       float a = 0.f;
-      for (int r = 0; r < d; ++r) a = fmaf(__ldg(p.v.rot + (int64_t)r * d + c), s_o[r], a);
-      out[c] = a * inv_l;
+      for (int r = 0; r < G.d; ++r) a = fmaf(__ldg(G.rot + (int64_t)r * G.d + c), s_o[G.off + r], a);
+      const int ch = G.chan ? min(max(__ldg(G.chan + c), 0), d - 1) : c;
+      out[ch] = a * inv_l;
     }
-  } else {  // o = sigma * H o' / sqrt(d)
+  } else {  // a single Hadamard group: o = sigma * H o' / sqrt(d)
     gn_fwht(s_o, 1, d, kGnMaxD);
     const float f = rsqrtf((float)d) * inv_l;
-    for (int i = tid; i < d; i += kGnThreads) out[i] = (p.v.signs[i] < 0 ? -s_o[i] : s_o[i]) * f;
+    for (int i = tid; i < d; i += kGnThreads) out[i] = (p.v[0].signs[i] < 0 ? -s_o[i] : s_o[i]) * f;
   }
 }
 
-GnSide side_of(const QuantParams &q, const CacheView &v) {
-  GnSide s{};
-  s.bm = q.bm;
-  s.prod = q.prod;
-  s.cent = q.centroids;
-  s.rot = q.rot;
-  s.S = q.S;
-  s.signs = q.signs;
-  s.codes = v.codes;
-  s.qjl = v.qjl;
-  s.norms = v.norms;
-  s.rnorms = v.rnorms;
-  s.sb = v.sb;
-  s.sh = v.sh;
-  s.sn = v.sn;
-  return s;
+GnGroup group_of(const QuantParams &q, const CacheView &v, int off) {
+  GnGroup g{};
+  g.d = q.d;
+  g.off = off;
+  g.bm = q.bm;
+  g.prod = q.prod;
+  g.cent = q.centroids;
+  g.rot = q.rot;
+  g.S = q.S;
+  g.signs = q.signs;
+  g.chan = q.channels;
+  g.codes = v.codes;
+  g.qjl = v.qjl;
+  g.norms = v.norms;
+  g.rnorms = v.rnorms;
+  g.sb = v.sb;
+  g.sh = v.sh;
+  g.sn = v.sn;
+  return g;
+}
+
+cudaError_t launch_general(GnParams &p, cudaStream_t s) {
+  p.g = p.Hq / p.Hkv;
+  p.hg = (p.g + kGnHeads - 1) / kGnHeads;
+  if (p.d > kGnMaxD || p.d % 8) return cudaErrorInvalidValue;
+  p.splits = general_decode_splits(p.B, p.Hq, p.Hkv, p.seq_len);
+  p.per_split = (p.seq_len + p.splits - 1) / p.splits;
+  if (p.seq_len > 0) {
+    const dim3 grid((unsigned)p.splits, (unsigned)(p.B * p.Hkv * p.hg));
+    general_partial_kernel<<<grid, kGnThreads, 0, s>>>(p);
+    const cudaError_t e = cudaGetLastError();
+    if (e != cudaSuccess) return e;
+  } else {
+    p.splits = 0;
+  }
+  general_merge_kernel<<<(unsigned)(p.B * p.Hq), kGnThreads, 0, s>>>(p);
+  return cudaGetLastError();
 }
 
 }  // namespace
@@ -383,15 +476,14 @@ size_t general_decode_workspace_floats(int B, int Hq, int Hkv, int64_t seq_len, 
 
 cudaError_t launch_decode_general(const DecodeArgs &a, cudaStream_t s) {
   GnParams p{};
-  p.k = side_of(a.kq, a.k);
-  p.v = side_of(a.vq, a.v);
+  p.k[0] = group_of(a.kq, a.k, 0);
+  p.v[0] = group_of(a.vq, a.v, 0);
+  p.nk = p.nv = 1;
   p.q = a.q;
   p.q_dtype = a.q_dtype;
   p.B = a.B;
   p.Hq = a.Hq;
   p.Hkv = a.Hkv;
-  p.g = a.Hq / a.Hkv;
-  p.hg = (p.g + kGnHeads - 1) / kGnHeads;
   p.d = a.kq.d;
   p.seq_len = a.seq_len;
   p.seq_lens = a.seq_lens;
@@ -399,19 +491,29 @@ cudaError_t launch_decode_general(const DecodeArgs &a, cudaStream_t s) {
   p.out = a.out;
   p.scores = a.scores;
   p.ws = a.ws;
-  if (p.d > kGnMaxD || p.d % 8) return cudaErrorInvalidValue;
-  p.splits = general_decode_splits(a.B, a.Hq, a.Hkv, a.seq_len);
-  p.per_split = (a.seq_len + p.splits - 1) / p.splits;
-  if (a.seq_len > 0) {
-    const dim3 grid((unsigned)p.splits, (unsigned)(a.B * a.Hkv * p.hg));
-    general_partial_kernel<<<grid, kGnThreads, 0, s>>>(p);
-    const cudaError_t e = cudaGetLastError();
-    if (e != cudaSuccess) return e;
-  } else {
-    p.splits = 0;
+  return launch_general(p, s);
+}
+
+cudaError_t launch_decode_split(const SplitDecodeArgs &a, cudaStream_t s) {
+  GnParams p{};
+  for (int g = 0; g < 2; ++g) {
+    p.k[g] = group_of(a.kq[g], a.k[g], g == 0 ? 0 : a.kq[0].d);
+    p.v[g] = group_of(a.vq[g], a.v[g], g == 0 ? 0 : a.vq[0].d);
   }
-  general_merge_kernel<<<(unsigned)(a.B * a.Hq), kGnThreads, 0, s>>>(p);
-  return cudaGetLastError();
+  p.nk = p.nv = 2;
+  p.q = a.q;
+  p.q_dtype = a.q_dtype;
+  p.B = a.B;
+  p.Hq = a.Hq;
+  p.Hkv = a.Hkv;
+  p.d = a.d;
+  p.seq_len = a.seq_len;
+  p.seq_lens = a.seq_lens;
+  p.scale_log2 = a.scale * kGnLog2e;
+  p.out = a.out;
+  p.scores = nullptr;
+  p.ws = a.ws;
+  return launch_general(p, s);
 }
 
 }  // namespace tq

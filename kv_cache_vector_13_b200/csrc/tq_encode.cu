@@ -353,8 +353,8 @@ __device__ __forceinline__ void group_sync(int grp) {
 // butterfly and the fold-halves sum pair the same coordinates whatever the
 // layout), so r[] equals the residual the front half formed.
 template <int BM, int DT>
-__device__ __forceinline__ void residual_exact(const EncParams &p, int64_t v, const uint32_t *s_sign, const float *s_cent,
-                                               float (&r)[4]) {
+__device__ __forceinline__ void front_warp(const EncParams &p, int64_t v, const uint32_t *s_sign, const float *s_cent,
+                                           float (&r)[4], int (&idx)[4], float &nrm_out) {
   constexpr int K = 1 << BM;
   const int lane = threadIdx.x & 31;
   int64_t b, h, n;
@@ -384,6 +384,7 @@ __device__ __forceinline__ void residual_exact(const EncParams &p, int64_t v, co
   sq[0] = __fadd_rn(sq[0], sq[2]);
   sq[1] = __fadd_rn(sq[1], sq[3]);
   const float nrm = __fsqrt_rn(__shfl_sync(dev::kFull, __fadd_rn(sq[0], sq[1]), 0));
+  nrm_out = nrm;
   // sign flips, then the FWHT stages h = 64 .. 1
   const uint32_t sw = s_sign[lane >> 3] >> (4 * (lane & 7));
 #pragma unroll
@@ -415,11 +416,104 @@ __device__ __forceinline__ void residual_exact(const EncParams &p, int64_t v, co
     const float u = __fmul_rn(x[j], inv);
     if constexpr (BM == 0) {
       r[j] = u;
+      idx[j] = 0;
     } else {
-      const int idx = BM == 1 ? (u > 0.0f ? 1 : 0) : dev::quantize_sym<BM>(u, PP);
-      r[j] = __fsub_rn(u, s_cent[idx]);
+      idx[j] = BM == 1 ? (u > 0.0f ? 1 : 0) : dev::quantize_sym<BM>(u, PP);
+      r[j] = __fsub_rn(u, s_cent[idx[j]]);
     }
   }
+}
+
+template <int BM, int DT>
+__device__ __forceinline__ void residual_exact(const EncParams &p, int64_t v, const uint32_t *s_sign, const float *s_cent,
+                                               float (&r)[4]) {
+  int idx[4];
+  float nrm;
+  front_warp<BM, DT>(p, v, s_sign, s_cent, r, idx, nrm);
+}
+
+// Small d = 128 prod batches (the one-token append of a decode step, whose
+// latency sits on the step's critical path): one 128-thread CTA per vector.
+// Warp 0 runs the canonical front half, four coordinates a lane (the same
+// operations as every other encode path, so codes and norms are identical);
+// the residual's norm is the same fold-halves sum; then thread k forms
+// z_k = sum_i S_ki r_i in fp32 from the residual in shared memory, and each
+// warp's ballot is one 32-bit word of the sketch.
+template <int BM, int DT>
+__global__ void __launch_bounds__(128) encode_prod_small_kernel(EncParams p) {
+  constexpr int D = 128;
+  constexpr int K = 1 << BM;
+  __shared__ uint32_t s_sign[D / 32];
+  __shared__ float s_cent[16];
+  __shared__ __align__(16) float s_r[D];
+  __shared__ int s_idx[D];
+  const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
+  pdl_open();
+  load_sign_masks<D>(p.signs, s_sign, tid);
+  if constexpr (BM > 0) {
+    if (tid < K) s_cent[tid] = p.cent[tid];
+  }
+  __syncthreads();
+  const int64_t v = blockIdx.x;
+  int64_t b, h, n;
+  split_index(p, v, b, h, n);
+  const int64_t rec = b * p.osb + h * p.osh + n * p.osn;
+  if (warp == 0) {
+    float r[4];
+    int idx[4];
+    float nrm;
+    front_warp<BM, DT>(p, v, s_sign, s_cent, r, idx, nrm);
+    float sq[4];
+#pragma unroll
+    for (int j = 0; j < 4; ++j) sq[j] = __fmul_rn(r[j], r[j]);
+#pragma unroll
+    for (int sh = 16; sh >= 1; sh >>= 1) {
+#pragma unroll
+      for (int j = 0; j < 4; ++j) sq[j] = __fadd_rn(sq[j], __shfl_down_sync(dev::kFull, sq[j], sh));
+    }
+    sq[0] = __fadd_rn(sq[0], sq[2]);
+    sq[1] = __fadd_rn(sq[1], sq[3]);
+    const float gam = __fsqrt_rn(__fadd_rn(sq[0], sq[1]));  // lane 0's is the canonical sum
+    *reinterpret_cast<float4 *>(s_r + 4 * lane) = make_float4(r[0], r[1], r[2], r[3]);
+#pragma unroll
+    for (int j = 0; j < 4; ++j) s_idx[4 * lane + j] = idx[j];
+    if (lane == 0) {
+      p.norms[rec] = nrm;
+      p.rnorms[rec] = gam;
+    }
+  }
+  __syncthreads();
+  // codes: thread w < 4 BM builds word w of the record's 128 BM-bit stream
+  if constexpr (BM > 0) {
+    if (tid < 4 * BM) {
+      const int lo = 32 * tid;
+      uint32_t word = 0u;
+      for (int i = lo / BM; i * BM < lo + 32; ++i) {
+        const int pos = i * BM - lo;
+        const uint32_t f = (uint32_t)s_idx[i];
+        word |= pos >= 0 ? f << pos : f >> -pos;
+      }
+      reinterpret_cast<uint32_t *>(p.codes + rec * (D * BM / 8))[tid] = word;
+    }
+  }
+  // the sketch: z_k = sum_i S_ki r_i, bit k = (z_k >= 0)
+  {
+    const float4 *Sk = reinterpret_cast<const float4 *>(p.S + (size_t)tid * D);
+    const float4 *r4 = reinterpret_cast<const float4 *>(s_r);
+    float z0 = 0.f, z1 = 0.f, z2 = 0.f, z3 = 0.f;
+#pragma unroll 8
+    for (int i = 0; i < D / 4; ++i) {
+      const float4 a = __ldg(Sk + i), c = r4[i];
+      z0 = fmaf(a.x, c.x, z0);
+      z1 = fmaf(a.y, c.y, z1);
+      z2 = fmaf(a.z, c.z, z2);
+      z3 = fmaf(a.w, c.w, z3);
+    }
+    const float z = (z0 + z1) + (z2 + z3);
+    const unsigned bits = __ballot_sync(dev::kFull, z >= 0.0f);
+    if (lane == 0) reinterpret_cast<uint32_t *>(p.qjl + rec * (D / 8))[warp] = bits;
+  }
+  pdl_close(p.pdl);
 }
 
 // The warp's exact recheck of one 32-column chunk: lanes in `need` hold a
@@ -660,9 +754,7 @@ cudaError_t run_prod_tc(const EncParams &p, cudaStream_t s) {
   return cudaGetLastError();
 }
 
-template <int D, int BM, bool PROD, int DT, int EE>
-cudaError_t run_e(const EncodeArgs &a, cudaStream_t s) {
-  using Sh = Shape<D, EE>;
+EncParams make_params(const EncodeArgs &a) {
   EncParams p;
   p.x = a.x;
   p.xsb = a.xsb;
@@ -691,6 +783,22 @@ cudaError_t run_e(const EncodeArgs &a, cudaStream_t s) {
     magic31(a.N, p.mN, p.sN);
     magic31(a.H, p.mH, p.sH);
   }
+  return p;
+}
+
+template <int BM, int DT>
+cudaError_t run_prod_small(const EncodeArgs &a, cudaStream_t s) {
+  const EncParams p = make_params(a);
+  const cudaError_t e = launch_maybe_pdl(encode_prod_small_kernel<BM, DT>, dim3((unsigned)p.nvec), dim3(128), 0, s,
+                                         p.pdl, p);
+  if (e != cudaSuccess) return e;
+  return cudaGetLastError();
+}
+
+template <int D, int BM, bool PROD, int DT, int EE>
+cudaError_t run_e(const EncodeArgs &a, cudaStream_t s) {
+  using Sh = Shape<D, EE>;
+  const EncParams p = make_params(a);
   if constexpr (PROD && D == 128 && EE == 64) return run_prod_tc<BM, DT>(p, s);
   const size_t smem = enc_smem_bytes<D, PROD, EE>();
   auto kern = encode_kernel<D, BM, PROD, DT, EE>;
@@ -705,11 +813,18 @@ cudaError_t run_e(const EncodeArgs &a, cudaStream_t s) {
 }
 
 // Small batches (up to one vector per lane of a full wave at E = 64) take
-// the E = 16 layout: four times more lanes per vector, shorter chains.
+// the E = 16 layout: four times more lanes per vector, shorter chains; d =
+// 128 prod batches take one CTA per vector.
 template <int D, int BM, bool PROD, int DT>
 cudaError_t run(const EncodeArgs &a, cudaStream_t s) {
   const int64_t nvec = a.B * a.H * a.N;
-  if (nvec <= 148 * (kEncThreads / Shape<D, 64>::T)) return run_e<D, BM, PROD, DT, 16>(a, s);
+  if (nvec <= 148 * (kEncThreads / Shape<D, 64>::T)) {
+    if constexpr (PROD && D == 128) {
+      return run_prod_small<BM, DT>(a, s);
+    } else {
+      return run_e<D, BM, PROD, DT, 16>(a, s);
+    }
+  }
   return run_e<D, BM, PROD, DT, 64>(a, s);
 }
 

@@ -612,9 +612,9 @@ tq_status tq_decode_attention_noalloc(const tq_quantizer *kq, const tq_quantizer
                              scores_out, ws, need, stream);
 }
 
-size_t tq_decode_split_workspace_bytes(int32_t B, int32_t Hq, int64_t seq_len) {
-  if (B <= 0 || Hq <= 0 || seq_len <= 0) return 0;
-  return (size_t)B * Hq * (size_t)seq_len * sizeof(float);
+size_t tq_decode_split_workspace_bytes(int32_t B, int32_t Hq, int32_t Hkv, int64_t seq_len, int32_t d) {
+  if (B <= 0 || Hq <= 0 || Hkv <= 0 || seq_len <= 0 || Hq % Hkv || d < 16 || d > 256 || d % 8) return 0;
+  return tq::general_decode_workspace_floats(B, Hq, Hkv, seq_len, d) * sizeof(float);
 }
 
 tq_status tq_decode_attention_split(const tq_quantizer kq[2], const tq_quantizer vq[2], const void *q,
@@ -641,7 +641,6 @@ tq_status tq_decode_attention_split(const tq_quantizer kq[2], const tq_quantizer
   if (q_dtype != TQ_F32 && q_dtype != TQ_BF16 && q_dtype != TQ_F16)
     return fail(TQ_EINVAL, "%s: q_dtype=%d", name, (int)q_dtype);
   if (B < 0 || Hq < 0 || Hkv <= 0 || seq_len < 0 || Hq % Hkv) return fail(TQ_EINVAL, "%s: bad sizes", name);
-  if (Hq / Hkv > 8) return fail(TQ_EUNSUPPORTED, "%s: %d query heads per kv head (at most 8)", name, Hq / Hkv);
   if (!std::isfinite(softmax_scale)) return fail(TQ_EINVAL, "%s: softmax_scale not finite", name);
   if (B == 0 || Hq == 0) return TQ_OK;
   if (!q || !out) return fail(TQ_EINVAL, "%s: q or out is NULL", name);
@@ -655,7 +654,7 @@ tq_status tq_decode_attention_split(const tq_quantizer kq[2], const tq_quantizer
     const cudaError_t e = cudaMemsetAsync(out, 0, (size_t)B * Hq * d * sizeof(float), (cudaStream_t)stream);
     return e == cudaSuccess ? TQ_OK : cuda_fail(e, name);
   }
-  const size_t need = tq_decode_split_workspace_bytes(B, Hq, seq_len);
+  const size_t need = tq_decode_split_workspace_bytes(B, Hq, Hkv, seq_len, d);
   if (workspace_bytes < need || !workspace || !aligned(workspace, 16))
     return fail(TQ_EWORKSPACE, "%s: workspace %zu bytes, need %zu", name, workspace_bytes, need);
   a.q = q;

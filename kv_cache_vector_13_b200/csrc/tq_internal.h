@@ -89,7 +89,7 @@ struct SplitDecodeArgs {
   CacheView k[2], v[2];
   float scale;
   float *out;
-  float *ws;  // logits [B * Hq][seq_len], then per-head (max, sum)
+  float *ws;  // partial slots of the split over the sequence
 };
 cudaError_t launch_decode_split(const SplitDecodeArgs &a, cudaStream_t s);
 

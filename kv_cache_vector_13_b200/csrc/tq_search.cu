@@ -13,11 +13,14 @@
 //     pair-table lookups and mma.m16n8k16 of the decode kernel, and keeps,
 //     per query, its best 32 (estimate, index) pairs sorted in registers, one
 //     per lane.  A chunk whose candidates all rank below the current k-th
-//     best is dropped after one vote; otherwise the 32 candidates are sorted
-//     by a warp bitonic sort and merged (the better of pair l and the
-//     reversed pair 31 - l is a bitonic sequence holding the best 32, which
-//     five exchange stages sort).  The CTA's warps merge their lists the same
-//     way and write one list per (query, slice);
+//     best is dropped after one vote of the lanes that hold the query's
+//     estimates; a few that beat it are inserted one at a time at their
+//     rank (a vote counts the entries ahead, the rest shift down one lane);
+//     many (a list's first chunks) are sorted by a warp bitonic sort and
+//     merged (the better of pair l and the reversed pair 31 - l is a
+//     bitonic sequence holding the best 32, which five exchange stages
+//     sort).  The CTA's warps merge their lists the same way and write one
+//     list per (query, slice);
 //   * search_merge_kernel: one warp per query merges the slices' lists and
 //     writes the first k.
 // Order: estimate descending, ties by record index ascending (a total
@@ -158,12 +161,12 @@ __global__ void __launch_bounds__(kSrWarps * 32) search_score_kernel(SearchParam
     }
   }
 
-  float lv[8];
-  int li[8];
+  float lv[8], kth_v[8];  // the lists (one entry a lane) and their k-th entries
+  int li[8], kth_i[8];
 #pragma unroll
   for (int h = 0; h < 8; ++h) {
-    lv[h] = -INFINITY;
-    li[h] = INT_MAX;
+    lv[h] = kth_v[h] = -INFINITY;
+    li[h] = kth_i[h] = INT_MAX;
   }
   // this CTA's slice of the database, this warp's chunks of it
   const int64_t s0 = p.N * split / p.splits, s1 = p.N * (split + 1) / p.splits;
@@ -220,12 +223,28 @@ __global__ void __launch_bounds__(kSrWarps * 32) search_score_kernel(SearchParam
         est[ms][i] = kn >= 0.f ? s * (kn * inv_sK) : -INFINITY;
       }
     }
-    // per query: the chunk's 32 candidates, one per lane (lane L holds
-    // record r0 + L), offered to the query's list
+    // per query: does any of the chunk's 32 candidates beat the list's
+    // k-th entry?  The lanes holding query h's estimates (column h of the
+    // score tile: rows g8 + 8 r + 16 ms) answer with one vote.
 #pragma unroll
     for (int h = 0; h < 8; ++h) {
       if (h < gh) {
-        const int src = (lane & 7) * 4 + (h >> 1), c = h & 1;
+        const int c = h & 1;
+        const bool mine = tig == (h >> 1);
+        bool hit = false;
+#pragma unroll
+        for (int ms = 0; ms < 2; ++ms) {
+#pragma unroll
+          for (int r = 0; r < 2; ++r) {
+            const int idx = (int)(r0 + 16 * ms + 8 * r + g8);
+            hit |= mine && better(est[ms][2 * r + c], idx, kth_v[h], kth_i[h]);
+          }
+        }
+        const unsigned any = __ballot_sync(dev::kFull, hit);
+        if (any == 0u) continue;
+        // the chunk's candidates for query h, one per lane (lane L holds
+        // record r0 + L)
+        const int src = (lane & 7) * 4 + (h >> 1);
         float cv = -INFINITY;
 #pragma unroll
         for (int ms = 0; ms < 2; ++ms) {
@@ -236,13 +255,30 @@ __global__ void __launch_bounds__(kSrWarps * 32) search_score_kernel(SearchParam
           }
         }
         const int cidx = (int)(r0 + lane);
-        const float kv = __shfl_sync(dev::kFull, lv[h], p.k - 1);
-        const int kidx = __shfl_sync(dev::kFull, li[h], p.k - 1);
-        if (__any_sync(dev::kFull, better(cv, cidx, kv, kidx))) {
+        const unsigned up = __ballot_sync(dev::kFull, better(cv, cidx, kth_v[h], kth_i[h]));
+        if (__popc(up) > 4) {  // many (the lists' first chunks): sort and merge
           int ci2 = cidx;
           warp_sort(cv, ci2, lane);
           warp_merge(lv[h], li[h], cv, ci2, lane);
+        } else {  // a few: insert each at its rank, the entries below move down one
+          for (unsigned m = up; m; m &= m - 1) {
+            const int l = __ffs(m) - 1;
+            const float nv = __shfl_sync(dev::kFull, cv, l);
+            const int ni = __shfl_sync(dev::kFull, cidx, l);
+            const int pos = __popc(__ballot_sync(dev::kFull, better(lv[h], li[h], nv, ni)));
+            const float dv = __shfl_up_sync(dev::kFull, lv[h], 1);
+            const int di = __shfl_up_sync(dev::kFull, li[h], 1);
+            if (lane == pos) {
+              lv[h] = nv;
+              li[h] = ni;
+            } else if (lane > pos) {
+              lv[h] = dv;
+              li[h] = di;
+            }
+          }
         }
+        kth_v[h] = __shfl_sync(dev::kFull, lv[h], p.k - 1);
+        kth_i[h] = __shfl_sync(dev::kFull, li[h], p.k - 1);
       }
     }
   }

@@ -69,3 +69,24 @@ def test_split_record_sizes_and_empty_cache():
     assert kq.groups[0].code_bytes == 12 and kq.groups[1].code_bytes == 24
     caches = api.encode_split(kq, torch.zeros((0, d), device=DEV))
     assert caches[0].norms.numel() == 0
+
+
+def test_split_decode_twelve_query_heads_per_kv_head():
+    # a GQA group of 12 (two head groups of a block) and prod value groups
+    B, Hq, Hkv, N, d = 1, 24, 2, 700, 128
+    K, V = workload(B, Hkv, N, d, seed=9)
+    ch = SP.select_outlier_channels(host(K[0, 0, :64]), 32)
+    kq = api.SplitQuantizer(d, ch, 3, 2, "mse", seed_rot=21, device=DEV)
+    vq = api.SplitQuantizer(d, ch, 3, 2, "prod", seed_rot=23, seed_qjl=24, device=DEV)
+    kc, vc = api.encode_split(kq, K.to(DEV)), api.encode_split(vq, V.to(DEV))
+    q = torch.randn((B, Hq, d), generator=torch.Generator().manual_seed(6)).to(torch.bfloat16)
+    out = host(api.DecodeAttentionSplit(kq, vq, B, Hq, Hkv, N, device=DEV)(q.to(DEV), kc, vc))
+    okq = SP.SplitQuantizer(d, ch, 3, 2, "mse", seed_rot=21)
+    ovq = SP.SplitQuantizer(d, ch, 3, 2, "prod", seed_rot=23, seed_qjl=24)
+    qh = host(q)
+    for h in range(Hkv):
+        ke = SP.encode(okq, host(K[0, h]), aux=False)
+        ve = SP.encode(ovq, host(V[0, h]), aux=False)
+        for hq in range(h * 12, (h + 1) * 12):
+            ref = SP.decode_attention(okq, ovq, qh[0, hq], ke, ve, dtype=np.float32)
+            assert rel_err(out[0, hq], ref) <= 2e-3, hq
