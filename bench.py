@@ -82,7 +82,10 @@ FALLBACK_PEAKS = {"hbm_gbs": 6650.0, "bf16_tflops": 1590.0}
 # workload, from an ncu capture (dram__bytes_read.sum + dram__bytes_write.sum),
 # reported only for that workload and while the decode sources are the ones
 # it was taken on.
-TRAFFIC = {"workload": None, "bytes": None, "source_sha256": None}
+# Captured at B = 2 (reads 230,277,120 B, writes 5,879,552 B): reads scaled by
+# the 8x units of B = 16 (B = 4 read 2.02x the B = 2 bytes), writes kept.
+TRAFFIC = {"workload": ("batched", 16), "bytes": 8 * 230277120 + 5879552,
+           "source_sha256": "0179cded1ecf5e36e05931ef7266c44f456d8b764648a8bed29757fb8d27af79"}
 DECODE_SOURCES = ("tq_decode.cu", "tq_decode_split.cuh", "tq_decode_regs.cu")
 
 
@@ -223,6 +226,7 @@ class Setup:
                                      for t in (c.codes, c.norms, c.qjl, c.rnorms)))
 
         self.tails = [(tail(kc), tail(vc)) for kc, vc in zip(self.kcs, self.vcs)]
+        torch.cuda.synchronize()  # everything above runs on the default stream; the steps on another
 
     @property
     def copies(self):
@@ -249,6 +253,7 @@ class Setup:
 def time_decode_calls(torch, s, stream, reps):
     """Live CUDA-event time of one tq_decode_attention call (ms), averaged
     over `reps` back-to-back calls that cycle through the cache copies."""
+    torch.cuda.synchronize()  # inputs made on the default stream are complete
     with torch.cuda.stream(stream):
         for c in range(max(3, s.copies)):
             s.decode(c % s.copies, stream)
@@ -386,6 +391,9 @@ def run_ours(args):
                 torch.cuda.empty_cache()
             line["decode_other_workloads"] = extras
             line["encode"] = [bench_encode(api, inputs, torch, dev, stream, v) for v in ENCODE_VARIANTS]
+            with ClockSampler(local) as nclk:
+                line["next_rows"] = bench_next_rows(api, inputs, torch, dev, stream)
+            line["next_rows"]["clocks"] = nclk.summary()
         if not args.no_cpu_baseline and ws == 1:
             line["cpu_baseline"] = cpu_baseline_decode(args.workload, args.batch, budget_s=args.cpu_seconds)
         print(json.dumps(line), flush=True)
@@ -395,6 +403,77 @@ def run_ours(args):
 
 
 ENCODE_VARIANTS = ("mse4", "prod3", "mse3_bf16", "prod3_bf16")
+
+
+def _time_calls(torch, stream, fn, reps, warm=3):
+    """Live CUDA-event time (ms) of one fn(i) call, averaged over `reps`
+    back-to-back calls on `stream` after `warm` untimed ones."""
+    torch.cuda.synchronize()  # inputs made on the default stream are complete
+    with torch.cuda.stream(stream):
+        for i in range(warm):
+            fn(i)
+        torch.cuda.synchronize()
+        e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+        e0.record(stream)
+        for i in range(reps):
+            fn(i)
+        e1.record(stream)
+    torch.cuda.synchronize()
+    return e0.elapsed_time(e1) / reps
+
+
+def bench_next_rows(api, inputs, torch, dev, stream):
+    """The three kernels past the decode step, each on a synthetic workload
+    larger than L2: the dense (Haar) rotation encode on tensor cores, top-k
+    vector search over a packed database, and decode over an outlier-channel
+    split cache (the pages' 32 channels at 3 bits + 96 at 2)."""
+    pk, _ = peaks()
+    out = {}
+    n, d = 1 << 20, 128
+    # dense rotation encode: 2^20 unit vectors fp32, TurboQuant_mse b=4
+    qz = api.Quantizer(d, 4, "mse", seed_rot=7, device=dev, rotation="dense")
+    xs = [inputs.unit_vectors(n, d, seed=10 + i, device=dev) for i in range(2)]
+    cs = [api.empty_cache(qz, 1, 1, n, dev) for _ in xs]
+    ms = _time_calls(torch, stream, lambda i: api.encode(qz, xs[i % 2], out=cs[i % 2], stream=stream), 30)
+    by = n * (4 * d + qz.record_bytes)
+    out["dense_encode"] = {"workload": "2^20 unit vectors d=128 fp32, TurboQuant_mse b=4, dense Haar rotation",
+                           "vectors_per_s": n / (ms * 1e-3), "ms_per_launch": ms, "bytes_per_launch": by,
+                           "achieved_gbs": by / (ms * 1e-3) / 1e9, "frac": by / (ms * 1e-3) / 1e9 / pk["hbm_gbs"]}
+    del xs, cs
+    # search: 2^21 records (mse-4, 68 B each: 143 MB), 32 queries, top-10
+    n_db, n_q, k = 1 << 21, 32, 10
+    qz = api.Quantizer(d, 4, "mse", seed_rot=8, device=dev)
+    db = api.encode(qz, inputs.vectors(n_db, d, seed=20, device=dev))
+    qs = inputs.vectors(n_q, d, seed=21, device=dev)
+    srch = api.Search(qz, n_q, n_db, device=dev)
+    ms = _time_calls(torch, stream, lambda i: srch(qs, db, k, stream=stream), 20)
+    by = n_db * qz.record_bytes
+    out["search"] = {"workload": f"top-{k} of {n_q} fp32 queries over 2^21 packed records d=128 "
+                                 "TurboQuant_mse b=4", "scores_per_s": n_db * n_q / (ms * 1e-3),
+                     "ms_per_call": ms, "bytes_per_call": by, "achieved_gbs": by / (ms * 1e-3) / 1e9,
+                     "frac": by / (ms * 1e-3) / 1e9 / pk["hbm_gbs"]}
+    del db
+    # split decode: B=1, 32/8 heads, N=32768, 32 outlier channels at 3 bits +
+    # 96 at 2 bits for K and V (2.25 bits per channel), 8 rotating copies
+    B, Hq, Hkv, N = 1, 32, 8, 32768
+    K, V = inputs.outlier_kv(N=N, B=B, seed=4, device=dev)
+    ms_ch = K[0, 0, :256].float().pow(2).mean(0)
+    ch = torch.sort(torch.topk(ms_ch, 32).indices).values.cpu()
+    kq = api.SplitQuantizer(d, ch, 3, 2, "mse", seed_rot=40, device=dev)
+    vq = api.SplitQuantizer(d, ch, 3, 2, "mse", seed_rot=42, device=dev)
+    kcs = [api.encode_split(kq, K) for _ in range(8)]
+    vcs = [api.encode_split(vq, V) for _ in range(8)]
+    del K, V
+    q = inputs.queries(B, Hq, device=dev)
+    op = api.DecodeAttentionSplit(kq, vq, B, Hq, Hkv, N, device=dev)
+    ms = _time_calls(torch, stream, lambda i: op(q, kcs[i % 8], vcs[i % 8], stream=stream), 20)
+    rec = sum(g.record_bytes for g in kq.groups) + sum(g.record_bytes for g in vq.groups)
+    by = B * Hkv * N * rec
+    out["split_decode"] = {"workload": "outlier-channel split decode: B=1 Hq=32 Hkv=8 d=128 N=32768, K and V "
+                                       "32 channels at 3 bits + 96 at 2 bits (2.25 bits), dense rotations",
+                           "kv_tokens_per_s": B * N / (ms * 1e-3), "ms_per_call": ms, "bytes_per_call": by,
+                           "achieved_gbs": by / (ms * 1e-3) / 1e9, "frac": by / (ms * 1e-3) / 1e9 / pk["hbm_gbs"]}
+    return out
 
 
 def run_encode_only(variant):
@@ -425,7 +504,9 @@ def bench_encode(api, inputs, torch, dev, stream, variant="mse4"):
     else:
         xs = [inputs.unit_vectors(n, d, seed=i, device=dev) for i in range(2)]
     outs = [api.empty_cache(qz, 1, 1, n, dev) for _ in range(len(xs))]
-    with torch.cuda.stream(stream):
+    torch.cuda.synchronize()  # the inputs and the quantizer are made on the default stream
+    clocks = ClockSampler(dev.index or 0)
+    with clocks, torch.cuda.stream(stream):
         for i in range(3):
             api.encode(qz, xs[i % len(xs)], out=outs[i % len(xs)], stream=stream)
         torch.cuda.synchronize()
@@ -435,7 +516,7 @@ def bench_encode(api, inputs, torch, dev, stream, variant="mse4"):
         for i in range(reps):
             api.encode(qz, xs[i % len(xs)], out=outs[i % len(xs)], stream=stream)
         e1.record(stream)
-    torch.cuda.synchronize()
+        torch.cuda.synchronize()
     ms = e0.elapsed_time(e1) / reps
     byts = n * (d * xs[0].element_size() + qz.record_bytes)
     pk, _ = peaks()
@@ -445,7 +526,7 @@ def bench_encode(api, inputs, torch, dev, stream, variant="mse4"):
              "mse3_bf16": "2^20 N(0,1) vectors d=128 bf16, TurboQuant_mse b=3",
              "prod3_bf16": "2^20 N(0,1) vectors d=128 bf16, TurboQuant_prod b=3"}
     return {"workload": names[variant], "vectors_per_s": n / (ms * 1e-3), "ms_per_launch": ms,
-            "bytes_per_launch": byts, "achieved_gbs": gbs, "frac": gbs / pk["hbm_gbs"]}
+            "bytes_per_launch": byts, "achieved_gbs": gbs, "frac": gbs / pk["hbm_gbs"], "clocks": clocks.summary()}
 
 
 # ------------------------------------------------------------- CPU oracle

@@ -220,21 +220,27 @@ __global__ void __launch_bounds__(kDnWarps * 32) dequant_dense_kernel(DenseParam
 // hi = fp16(x), lo = fp16(x - hi), likewise Pi; the product is
 // Xh Ph + Xh Pl + Xl Ph (the dropped Xl Pl is below 2^-22 of the terms),
 // accumulated in fp32 in tensor memory.  u = y_scaled * fl(1 / fl(16 s n)).
-// Per CTA (persistent, one per SM, 256 threads):
+// Per CTA (persistent, one per SM, 512 threads in two groups of 8 warps
+// that walk alternate tiles, so one group's loads overlap the other's MMAs
+// and epilogue):
 //   * once: Pi's halves into shared memory in the K-major, no-swizzle
-//     canonical layout (8 x 16-byte core matrices), and d TMEM columns;
-//   * per tile: the warps load 16 rows each (all loads in flight first),
-//     take each row's canonical norm (fold-halves: in-register stages, then
-//     shuffles), scale, split and store the halves -- the A tile's core
-//     matrices are 144 bytes apart along K so that a warp's 2-byte stores of
-//     one row hit 32 different banks;
-//   * one thread issues the 3 d/16 tcgen05.mma and a tcgen05.commit to an
-//     mbarrier; every thread waits on it (bounded);
-//   * the epilogue: warp w reads TMEM lanes 32 (w % 4) + [0, 32) (its rows)
-//     and columns (w / 4) d/2 + [0, d/2) with tcgen05.ld, scales, quantizes
-//     and packs half a record per thread.
+//     canonical layout (8 x 16-byte core matrices), and d TMEM columns per
+//     group;
+//   * per tile: the group's warps load 16 rows each (8 at a time, all loads
+//     in flight first), take each row's canonical norm (fold-halves:
+//     in-register stages, then shuffles), scale, split and store the halves
+//     into the group's A operand -- its core matrices are 144 bytes apart
+//     along K so that a warp's 2-byte stores of one row hit 32 different
+//     banks;
+//   * one thread issues the 3 d/16 tcgen05.mma and a tcgen05.commit to the
+//     group's mbarrier; the group waits on it (bounded);
+//   * the epilogue: warp w of the group reads TMEM lanes 32 (w % 4) + [0, 32)
+//     (its rows) and half the d columns (w / 4), 32 at a time, scales,
+//     quantizes and packs half a record per thread.
 
-constexpr int kTcThreads = 256;
+constexpr int kTcGroups = 2;        // tiles in flight per CTA
+constexpr int kTcGroupWarps = 8;
+constexpr int kTcThreads = kTcGroups * kTcGroupWarps * 32;
 constexpr int kTcM = 128;          // vectors per tile
 constexpr int kTcLboA = 144;       // bytes between K-adjacent core matrices of A
 constexpr int kTcLboB = 128;
@@ -245,9 +251,11 @@ struct TcLayout {
   static constexpr int SBO_B = (D / 8) * kTcLboB;
   static constexpr int A_BYTES = (kTcM / 8) * SBO_A;
   static constexpr int B_BYTES = (D / 8) * SBO_B;
-  static constexpr int oBh = 0, oBl = B_BYTES, oAh = 2 * B_BYTES, oAl = 2 * B_BYTES + A_BYTES;
-  static constexpr int oInv = 2 * B_BYTES + 2 * A_BYTES;  // kTcM floats
-  static constexpr int kBytes = oInv + kTcM * 4;
+  static constexpr int oBh = 0, oBl = B_BYTES;
+  // group g: A halves at oA(g), oA(g) + A_BYTES
+  static constexpr int oA0 = 2 * B_BYTES;
+  static constexpr int oInv = oA0 + kTcGroups * 2 * A_BYTES;  // [kTcGroups][kTcM] floats
+  static constexpr int kBytes = oInv + kTcGroups * kTcM * 4;
 };
 
 template <int D, int BM, int DT>
@@ -255,19 +263,24 @@ __global__ void __launch_bounds__(kTcThreads, 1) encode_dense_tc_kernel(DensePar
                                                                         int64_t ntiles) {
   using L = TcLayout<D>;
   constexpr int J = D / 32;          // elements per lane per row in the loads
-  constexpr int HALF = D / 2;        // columns per epilogue thread
   constexpr int K = 1 << BM;
+  constexpr int kRows = kTcM / kTcGroupWarps;  // rows a warp loads per tile
   extern __shared__ __align__(1024) unsigned char smem[];
-  __shared__ __align__(8) uint64_t s_bar;
+  __shared__ __align__(8) uint64_t s_bar[kTcGroups];
   __shared__ uint32_t s_tmem;
   const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
+  const int grp = warp / kTcGroupWarps, gw = warp % kTcGroupWarps;
   const uint32_t sbase = (uint32_t)__cvta_generic_to_shared(smem);
-  const uint32_t bar = (uint32_t)__cvta_generic_to_shared(&s_bar);
-  float *s_inv = reinterpret_cast<float *>(smem + L::oInv);
+  const uint32_t bar = (uint32_t)__cvta_generic_to_shared(&s_bar[grp]);
+  const uint32_t oAh = (uint32_t)(L::oA0 + grp * 2 * L::A_BYTES), oAl = oAh + L::A_BYTES;
+  float *s_inv = reinterpret_cast<float *>(smem + L::oInv) + grp * kTcM;
 
-  // ---- once: TMEM columns, the mbarrier, Pi's halves (scaled by 16)
-  if (warp == 0) umma::alloc(&s_tmem, (uint32_t)D);
-  if (tid == 0) umma::mbar_init(bar, 1);
+  // ---- once: TMEM columns, the mbarriers, Pi's halves (scaled by 16)
+  if (warp == 0) umma::alloc(&s_tmem, (uint32_t)(kTcGroups * D));
+  if (tid == 0) {
+#pragma unroll
+    for (int g = 0; g < kTcGroups; ++g) umma::mbar_init((uint32_t)__cvta_generic_to_shared(&s_bar[g]), 1);
+  }
   for (int i = tid; i < D * D; i += kTcThreads) {
     const int n = i / D, k = i % D;
     const float v = 16.0f * __ldg(p.rot + i);
@@ -284,19 +297,21 @@ __global__ void __launch_bounds__(kTcThreads, 1) encode_dense_tc_kernel(DensePar
   umma::fence_before();
   __syncthreads();
   umma::fence_after();
-  const uint32_t tmem = s_tmem;
+  const uint32_t tmem = s_tmem + (uint32_t)(grp * D);
   constexpr uint32_t idesc = umma::idesc_f16(kTcM, D);
   bool dead = false;
 
-  for (int64_t tile = blockIdx.x, it = 0; tile < ntiles; tile += gridDim.x, ++it) {
-    // ---- phase 1: rows warp * 16 + [0, 16), in two batches of 8 whose
+  int64_t it = 0;
+  for (int64_t tile = (int64_t)blockIdx.x * kTcGroups + grp; tile < ntiles;
+       tile += (int64_t)gridDim.x * kTcGroups, ++it) {
+    // ---- phase 1: rows gw * kRows + [0, kRows), in batches of 8 whose
     // loads are all in flight before the first row is used
 #pragma unroll 1
-    for (int rb = 0; rb < 16; rb += 8) {
+    for (int rb = 0; rb < kRows; rb += 8) {
       float xr[8][J];
 #pragma unroll
       for (int r = 0; r < 8; ++r) {
-        const int64_t v = tile * kTcM + warp * 16 + rb + r;
+        const int64_t v = tile * kTcM + gw * kRows + rb + r;
         int64_t b, h, n;
         bhn(p, v < p.nvec ? v : 0, b, h, n);
         const int64_t xoff = b * p.xsb + h * p.xsh + n * p.xsn;
@@ -305,7 +320,7 @@ __global__ void __launch_bounds__(kTcThreads, 1) encode_dense_tc_kernel(DensePar
       }
 #pragma unroll
       for (int r = 0; r < 8; ++r) {
-        const int m = warp * 16 + rb + r;
+        const int m = gw * kRows + rb + r;
         const int64_t v = tile * kTcM + m;
         float sq[J];
 #pragma unroll
@@ -330,8 +345,8 @@ __global__ void __launch_bounds__(kTcThreads, 1) encode_dense_tc_kernel(DensePar
           const __half hi = __float2half_rn(xs);
           const __half lo = __float2half_rn(xs - __half2float(hi));
           const uint32_t o = umma::off(m, k, L::SBO_A, kTcLboA);
-          *reinterpret_cast<__half *>(smem + L::oAh + o) = hi;
-          *reinterpret_cast<__half *>(smem + L::oAl + o) = lo;
+          *reinterpret_cast<__half *>(smem + oAh + o) = hi;
+          *reinterpret_cast<__half *>(smem + oAl + o) = lo;
         }
         if (lane == 0) {
           s_inv[m] = normal ? __frcp_rn(__fmul_rn(16.0f * sc, nrm)) : 0.0f;
@@ -344,15 +359,16 @@ __global__ void __launch_bounds__(kTcThreads, 1) encode_dense_tc_kernel(DensePar
       }
     }
     umma::fence_async_smem();
-    __syncthreads();
+    umma::fence_before();
+    asm volatile("bar.sync %0, %1;\n" ::"r"(1 + grp), "r"(kTcGroupWarps * 32) : "memory");
 
-    // ---- phase 2: Y = Xh Ph + Xh Pl + Xl Ph into TMEM
-    if (tid == 0) {
+    // ---- phase 2: Y = Xh Ph + Xh Pl + Xl Ph into the group's TMEM columns
+    if (gw == 0 && lane == 0) {
       umma::fence_after();
 #pragma unroll 1
       for (int ks = 0; ks < D / 16; ++ks) {
-        const uint64_t ah = umma::desc(sbase + L::oAh + ks * 2 * kTcLboA, kTcLboA, L::SBO_A);
-        const uint64_t al = umma::desc(sbase + L::oAl + ks * 2 * kTcLboA, kTcLboA, L::SBO_A);
+        const uint64_t ah = umma::desc(sbase + oAh + ks * 2 * kTcLboA, kTcLboA, L::SBO_A);
+        const uint64_t al = umma::desc(sbase + oAl + ks * 2 * kTcLboA, kTcLboA, L::SBO_A);
         const uint64_t bh = umma::desc(sbase + L::oBh + ks * 2 * kTcLboB, kTcLboB, L::SBO_B);
         const uint64_t bl = umma::desc(sbase + L::oBl + ks * 2 * kTcLboB, kTcLboB, L::SBO_B);
         umma::mma_f16(tmem, ah, bh, idesc, ks > 0 ? 1u : 0u);
@@ -361,14 +377,15 @@ __global__ void __launch_bounds__(kTcThreads, 1) encode_dense_tc_kernel(DensePar
       }
       umma::commit(bar);
     }
-    // bounded wait for the MMAs (phase parity = tile count & 1)
+    // bounded wait for the MMAs (phase parity = the group's tile count & 1)
     if (!dead) dead = !umma::mbar_wait_bounded(bar, (uint32_t)(it & 1), faults, kFaultTimeout);
     umma::fence_after();
 
-    // ---- phase 3: half a record per thread, 32 columns (BM words of
-    // codes) at a time
+    // ---- phase 3: warp gw reads TMEM lanes 32 (gw % 4) + [0, 32) (its
+    // rows) and its share of the columns, 32 (BM words of codes) at a time
     {
-      const int q4 = warp & 3, hf = warp >> 2;
+      constexpr int kParts = kTcGroupWarps / 4, kCols = D / kParts;
+      const int q4 = gw & 3, part = gw >> 2;
       const int m = 32 * q4 + lane;
       const int64_t v = tile * kTcM + m;
       const float inv = s_inv[m];
@@ -376,12 +393,12 @@ __global__ void __launch_bounds__(kTcThreads, 1) encode_dense_tc_kernel(DensePar
       if (v < p.nvec) {
         int64_t b, h, n;
         bhn(p, v, b, h, n);
-        dst = p.codes + (b * p.osb + h * p.osh + n * p.osn) * (D * BM / 8) + hf * (HALF * BM / 8);
+        dst = p.codes + (b * p.osb + h * p.osh + n * p.osn) * (D * BM / 8) + part * (kCols * BM / 8);
       }
 #pragma unroll 1
-      for (int c = 0; c < HALF / 32; ++c) {
+      for (int c = 0; c < kCols / 32; ++c) {
         uint32_t y[32];
-        umma::ld32(tmem + ((uint32_t)(32 * q4) << 16) + (uint32_t)(hf * HALF + 32 * c), y);
+        umma::ld32(tmem + ((uint32_t)(32 * q4) << 16) + (uint32_t)(part * kCols + 32 * c), y);
         umma::wait_ld();
         uint32_t W[BM];
 #pragma unroll
@@ -401,11 +418,14 @@ __global__ void __launch_bounds__(kTcThreads, 1) encode_dense_tc_kernel(DensePar
       }
     }
     umma::fence_before();
-    __syncthreads();
+    // the group's next tile rewrites s_inv and A only after every thread of
+    // the group has read them
+    asm volatile("bar.sync %0, %1;\n" ::"r"(1 + grp), "r"(kTcGroupWarps * 32) : "memory");
   }
+  __syncthreads();
   if (warp == 0) {
     umma::fence_after();
-    umma::dealloc(tmem, (uint32_t)D);
+    umma::dealloc(s_tmem, (uint32_t)(kTcGroups * D));
   }
 }
 
@@ -416,7 +436,8 @@ cudaError_t run_dense_tc(const DenseParams &p, unsigned *faults, cudaStream_t s)
   cudaError_t e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, smem);
   if (e != cudaSuccess) return e;
   const int64_t ntiles = (p.nvec + kTcM - 1) / kTcM;
-  const int64_t grid = ntiles < decode_ctas() ? ntiles : decode_ctas();
+  const int64_t pairs = (ntiles + kTcGroups - 1) / kTcGroups;
+  const int64_t grid = pairs < decode_ctas() ? pairs : decode_ctas();
   kern<<<(unsigned)grid, kTcThreads, smem, s>>>(p, faults, ntiles);
   return cudaGetLastError();
 }

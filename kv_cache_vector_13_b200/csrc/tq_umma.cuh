@@ -86,12 +86,15 @@ __device__ __forceinline__ void mbar_init(uint32_t bar, uint32_t count) {
   asm volatile("fence.mbarrier_init.release.cluster;\n" ::: "memory");
 }
 
-__device__ __forceinline__ bool mbar_try(uint32_t bar, uint32_t parity) {
+// One try: the thread may be suspended until the phase completes or about
+// `hint_ns` pass, so a waiting warp takes no issue slots from the warps that
+// still work.
+__device__ __forceinline__ bool mbar_try(uint32_t bar, uint32_t parity, uint32_t hint_ns = 20000u) {
   uint32_t ok;
   asm volatile(
-      "{\n .reg .pred p;\n mbarrier.try_wait.parity.shared::cta.b64 p, [%1], %2;\n selp.u32 %0, 1, 0, p;\n}\n"
+      "{\n .reg .pred p;\n mbarrier.try_wait.parity.shared::cta.b64 p, [%1], %2, %3;\n selp.u32 %0, 1, 0, p;\n}\n"
       : "=r"(ok)
-      : "r"(bar), "r"(parity)
+      : "r"(bar), "r"(parity), "r"(hint_ns)
       : "memory");
   return ok != 0;
 }
@@ -102,7 +105,7 @@ __device__ __forceinline__ bool mbar_try(uint32_t bar, uint32_t parity) {
 __device__ __forceinline__ bool mbar_wait_bounded(uint32_t bar, uint32_t parity, unsigned *faults, unsigned flag) {
   uint64_t t0 = 0;
   for (uint32_t spin = 0; !mbar_try(bar, parity); ++spin) {
-    if ((spin & 255u) == 255u) {
+    if ((spin & 15u) == 15u) {
       uint64_t now;
       asm volatile("mov.u64 %0, %%globaltimer;\n" : "=l"(now));
       if (t0 == 0) {
