@@ -162,18 +162,43 @@ __global__ void __launch_bounds__(256) decode_prep_kernel(PrepParams p) {
     s_q[half][t] = acc;
     __syncthreads();
   }
-  if (valid && p.kS) {
-    const float4 *Sk = reinterpret_cast<const float4 *>(p.kS + (size_t)t * kD);
+  // S q' as two int8 digits per coordinate: x = round(Sq' / c) = 256 hi + lo
+  // with |x| <= 32000 (c = max |Sq'| / 32000), hi in [-125, 125], lo in
+  // [-128, 127]; and T = sum_k Sq'[k]
+  __shared__ int s_dig[2][2][kD];  // [half][hi / lo][k]
+  __shared__ float s_red[2][4][2];
+  float sq_c = 0.f, sq_t = 0.f;
+  if (p.kS) {
     float acc = 0.f;
+    if (valid) {
+      const float4 *Sk = reinterpret_cast<const float4 *>(p.kS + (size_t)t * kD);
 #pragma unroll 8
-    for (int i = 0; i < kD / 4; ++i) {
-      const float4 sv = __ldg(Sk + i);
-      acc = fmaf(sv.x, s_q[half][4 * i], acc);
-      acc = fmaf(sv.y, s_q[half][4 * i + 1], acc);
-      acc = fmaf(sv.z, s_q[half][4 * i + 2], acc);
-      acc = fmaf(sv.w, s_q[half][4 * i + 3], acc);
+      for (int i = 0; i < kD / 4; ++i) {
+        const float4 sv = __ldg(Sk + i);
+        acc = fmaf(sv.x, s_q[half][4 * i], acc);
+        acc = fmaf(sv.y, s_q[half][4 * i + 1], acc);
+        acc = fmaf(sv.z, s_q[half][4 * i + 2], acc);
+        acc = fmaf(sv.w, s_q[half][4 * i + 3], acc);
+      }
     }
-    s_qs[half][t] = acc;
+    float mx = fabsf(acc), sm = acc;
+#pragma unroll
+    for (int o = 16; o >= 1; o >>= 1) {
+      mx = fmaxf(mx, __shfl_xor_sync(dev::kFull, mx, o));
+      sm += __shfl_xor_sync(dev::kFull, sm, o);
+    }
+    if (lane == 0) {
+      s_red[half][t >> 5][0] = mx;
+      s_red[half][t >> 5][1] = sm;
+    }
+    __syncthreads();
+    mx = fmaxf(fmaxf(s_red[half][0][0], s_red[half][1][0]), fmaxf(s_red[half][2][0], s_red[half][3][0]));
+    sq_t = (s_red[half][0][1] + s_red[half][1][1]) + (s_red[half][2][1] + s_red[half][3][1]);
+    sq_c = mx > 0.f ? mx * (1.0f / 32000.0f) : 1.0f;
+    const int x = __float2int_rn(acc / sq_c);
+    const int hi = (x + 128) >> 8;
+    s_dig[half][0][t] = hi;
+    s_dig[half][1][t] = x - 256 * hi;
   }
   __syncthreads();
   if (!valid) return;
@@ -183,27 +208,34 @@ __global__ void __launch_bounds__(256) decode_prep_kernel(PrepParams p) {
   const int64_t u = ((int64_t)b * p.Hkv + kvh) * p.groups + grp;
   uint32_t *fu = p.frag + u * kFragWords;
   auto put = [&](int ln, int w, uint32_t v) { fu[((w >> 2) * 32 + ln) * 4 + (w & 3)] = v; };
-  const float *qv = s_q[half], *sv = s_qs[half];
+  const float *qv = s_q[half];
+  // the digit word of lane tig, step S, register j: bytes i = 0..3 hold the
+  // digit of Sq'[32 tig + 8 i + 7 - 2 S - j]
+  auto dig_word = [&](int which, int tig, int S, int j) {
+    uint32_t wv = 0u;
+#pragma unroll
+    for (int i = 0; i < 4; ++i)
+      wv |= ((uint32_t)s_dig[half][which][32 * tig + 8 * i + 7 - 2 * S - j] & 0xFFu) << (8 * i);
+    return wv;
+  };
   if (p.g <= 4) {
     const int ls = t >> 4, w = t & 15, sidx = w >> 1, j = w & 1;
     const int g8 = hh + 4 * (ls >> 2), tig = ls & 3, ln = g8 * 4 + tig;
     const bool lo = g8 >= 4;
     const int d0 = 32 * tig + 4 * sidx + 2 * j;
     put(ln, w, lo ? pack_lo(qv[d0], qv[d0 + 1]) : pack_hi(qv[d0], qv[d0 + 1]));
-    if (p.kS) {
-      const int e = 32 * tig + 15 - 2 * sidx - j;
-      put(ln, 16 + w, lo ? pack_lo(sv[e], sv[e + 16]) : pack_hi(sv[e], sv[e + 16]));
-    }
+    if (p.kS && w < 8) put(ln, 16 + w, dig_word(lo ? 1 : 0, tig, w >> 1, w & 1));
   } else {
     const int tig = t >> 5, w = t & 31, sidx = (w & 15) >> 1, j = w & 1;
     const int ln = hh * 4 + tig;
     const bool lo = w >= 16;
     const int d0 = 32 * tig + 4 * sidx + 2 * j;
     put(ln, w, lo ? pack_lo(qv[d0], qv[d0 + 1]) : pack_hi(qv[d0], qv[d0 + 1]));
-    if (p.kS) {
-      const int e = 32 * tig + 15 - 2 * sidx - j;
-      put(ln, 32 + w, lo ? pack_lo(sv[e], sv[e + 16]) : pack_hi(sv[e], sv[e + 16]));
-    }
+    if (p.kS && w < 16) put(ln, 32 + w, dig_word(w >> 3, tig, (w & 7) >> 1, w & 1));
+  }
+  if (p.kS && t == 0) {  // the head's digit scale and coordinate sum
+    put(hh, 60, __float_as_uint(sq_c));
+    put(hh, 61, __float_as_uint(sq_t));
   }
   // When this grid was launched early after the new tokens' encode (the
   // fused append + decode chain), one thread waits for that grid, so this

@@ -97,9 +97,14 @@ constexpr int kHdr = 1024;
 // Word w of lane (g8, tig), with q' the unit's rotated queries and
 // sel = lo half for PACK lanes g8 >= 4:
 //   PACK (<= 4 heads): w = 2s + j      : sel(q'[g8 & 3][32 tig + 4s + 2j, +1])
-//                      w = 16 + 2s + j : sel(Sq'[g8 & 3][32 tig + 15 - 2s - j, +16])
+//                      w = 16 + 2S + j : dig(Sq'[g8 & 3][32 tig + 8i + 7 - 2S - j]), i = 0..3
+//                                        (byte i; dig = hi digit, lo digit for g8 >= 4)
 //   8 heads          : w = 2s + j / 16 + 2s + j  : hi / lo of q'[g8][32 tig + 4s + 2j, +1]
-//                      w = 32 + ... / 48 + ...   : hi / lo of Sq'[g8][32 tig + 15 - 2s - j, +16]
+//                      w = 32 + 2S + j / 40 + 2S + j : hi / lo digit of Sq'[g8][...] as above
+//   (s < 8, S < 4, j < 2).  Sq' travels as int8 digits, round(Sq' / c_h) =
+//   256 hi + lo with |round(Sq' / c_h)| <= 32000; word 60 of lane h holds
+//   c_h and word 61 of lane h holds T_h = sum_k Sq'_h[k] (h < 8, the
+//   unit's heads).
 constexpr int kFragWords = 32 * 64;
 constexpr float kLog2e = 1.4426950408889634f;
 constexpr float kKappa = 1.2533141373155003f / (float)kD;  // sqrt(pi/2)/d
@@ -192,6 +197,23 @@ __device__ __forceinline__ void mma16816(float (&c)[4], const uint32_t (&a)[4], 
       : "r"(a[0]), "r"(a[1]), "r"(a[2]), "r"(a[3]), "r"(b0), "r"(b1));
 }
 
+// D += A B on int8 operands (mma.m16n8k32, s8 x s8 -> s32).
+__device__ __forceinline__ void mma16832_s8(int (&c)[4], const uint32_t (&a)[4], uint32_t b0, uint32_t b1) {
+  asm volatile(
+      "mma.sync.aligned.m16n8k32.row.col.s32.s8.s8.s32 {%0,%1,%2,%3}, {%4,%5,%6,%7}, {%8,%9}, "
+      "{%0,%1,%2,%3};\n"
+      : "+r"(c[0]), "+r"(c[1]), "+r"(c[2]), "+r"(c[3])
+      : "r"(a[0]), "r"(a[1]), "r"(a[2]), "r"(a[3]), "r"(b0), "r"(b1));
+}
+
+// Four int8 lanes, each 0 or -1 as bit 7 of byte 0..3 of w is clear or set
+// (a byte permute in sign-replicating mode).
+__device__ __forceinline__ uint32_t sign_bytes(uint32_t w) {
+  uint32_t r;
+  asm("prmt.b32 %0, %1, 0, 0xBA98;\n" : "=r"(r) : "r"(w));
+  return r;
+}
+
 __device__ __forceinline__ uint32_t movmatrix_trans(uint32_t x) {
   uint32_t y;
   asm volatile("movmatrix.sync.aligned.m8n8.trans.b16 %0, %1;\n" : "=r"(y) : "r"(x));
@@ -263,12 +285,6 @@ __device__ __forceinline__ uint32_t pair_addr(const uint32_t (&W)[NW], uint32_t 
   constexpr int w = off >> 5;
   constexpr int w1 = (w + 1 < NW) ? w + 1 : w;
   return lut_addr<off>(W[w], W[w1], laneoff);
-}
-
-// +-1 half2 from QJL bits (15 - sh, 31 - sh) of w: bit 1 -> +1, bit 0 -> -1
-template <int SH>
-__device__ __forceinline__ uint32_t qjl_half2(uint32_t w) {
-  return ((w << SH) & 0x80008000u) ^ 0xBC00BC00u;
 }
 
 template <int BM>
@@ -1065,15 +1081,19 @@ __global__ void __launch_bounds__(split_warps<PACK, KPROD, STAGED>() * 32, 1) de
     // g8.  Lanes whose head is absent (fewer than 4 or 8 heads) hold zeros.
     constexpr bool QS_SMEM = qs_in_smem<KPROD, STAGED>();
     uint32_t qf[8][2], qf2[PACK ? 1 : 8][2];
-    uint32_t qsf[(KPROD && !QS_SMEM) ? 8 : 1][2], qsf2[(KPROD && !PACK && !QS_SMEM) ? 8 : 1][2];
-    // QS_SMEM: the unit's S q' fragments at the start of the dynamic region,
-    // [S][hi 0 / lo 1][lane] words pairs (one 8-byte load per lane and step)
+    uint32_t qsf[(KPROD && !QS_SMEM) ? 4 : 1][2], qsf2[(KPROD && !PACK && !QS_SMEM) ? 4 : 1][2];
+    // QS_SMEM: the unit's S q' digit fragments at the start of the dynamic
+    // region, [S][hi 0 / lo 1][lane] word pairs (one 8-byte load per lane and
+    // step)
     const uint2 *s_qs = reinterpret_cast<const uint2 *>(smem + (((dyn_base + 15u) & ~15u) - dyn_base));
+    // the QJL term of this lane's two head columns c: sum_i digit-weighted
+    // MMA results, qd[c][0] * hi (+ qd[c][1] * lo) + qd[c][2] = <S q', sign>
+    float qd[2][3];
     {
       const bool has = (PACK ? (g8 & 3) : g8) < gh;
       const uint4 *fr = p.frag + (int64_t)u * (kFragWords / 4) + lane;
       auto ld4 = [&](int w4) { return has ? __ldg(fr + w4 * 32) : make_uint4(0u, 0u, 0u, 0u); };
-      auto put = [](uint32_t (&f)[8][2], int k, uint4 v) {
+      auto put = [](auto &f, int k, uint4 v) {
         f[2 * k][0] = v.x;
         f[2 * k][1] = v.y;
         f[2 * k + 1][0] = v.z;
@@ -1083,18 +1103,40 @@ __global__ void __launch_bounds__(split_warps<PACK, KPROD, STAGED>() * 32, 1) de
       for (int k = 0; k < 4; ++k) {
         put(qf, k, ld4(k));
         if constexpr (!PACK) put(qf2, k, ld4(4 + k));
+      }
+#pragma unroll
+      for (int k = 0; k < 2; ++k) {
         if constexpr (KPROD && !QS_SMEM) put(qsf, k, ld4((PACK ? 4 : 8) + k));
-        if constexpr (KPROD && !PACK && !QS_SMEM) put(qsf2, k, ld4(12 + k));
+        if constexpr (KPROD && !PACK && !QS_SMEM) put(qsf2, k, ld4(10 + k));
+      }
+      if constexpr (KPROD) {
+        const uint32_t *fw = reinterpret_cast<const uint32_t *>(p.frag + (int64_t)u * (kFragWords / 4));
+#pragma unroll
+        for (int c = 0; c < 2; ++c) {
+          const int h = PACK ? 2 * (tig & 1) + c : 2 * tig + c;  // this lane's head columns
+          const float ch = h < gh ? __uint_as_float(__ldg(fw + (15 * 32 + h) * 4 + 0)) : 0.f;
+          const float th = h < gh ? __uint_as_float(__ldg(fw + (15 * 32 + h) * 4 + 1)) : 0.f;
+          // the MMAs sum -bit * digit: <S q', 2 bit - 1> = -2 c_h (256 hi + lo) - T_h
+          if constexpr (PACK) {  // lanes tig < 2 hold the hi digits' columns, the others the lo digits'
+            qd[c][0] = -2.f * ch * (tig < 2 ? 256.f : 1.f);
+            qd[c][1] = 0.f;
+            qd[c][2] = tig < 2 ? -th : 0.f;
+          } else {
+            qd[c][0] = -512.f * ch;
+            qd[c][1] = -2.f * ch;
+            qd[c][2] = -th;
+          }
+        }
       }
       if constexpr (QS_SMEM) {
         // every thread copies its share; the barrier below (before the
         // chunk loop) publishes them
         uint2 *dst = const_cast<uint2 *>(s_qs);
-        for (int i = tid; i < 2 * 8 * 32; i += kThreads) {
-          const int ln = i & 31, S = (i >> 5) & 7, j2 = i >> 8;
+        for (int i = tid; i < 2 * 4 * 32; i += kThreads) {
+          const int ln = i & 31, S = (i >> 5) & 3, j2 = i >> 7;
           if (PACK && j2 == 1) continue;
           const bool h = (PACK ? ((ln >> 2) & 3) : (ln >> 2)) < gh;
-          const int w4 = (PACK ? 4 : (j2 ? 12 : 8)) + (S >> 1);
+          const int w4 = (PACK ? 4 : (j2 ? 10 : 8)) + (S >> 1);
           uint4 v = h ? __ldg(p.frag + (int64_t)u * (kFragWords / 4) + ln + w4 * 32) : make_uint4(0u, 0u, 0u, 0u);
           dst[(S * 2 + j2) * 32 + ln] = (S & 1) ? make_uint2(v.z, v.w) : make_uint2(v.x, v.y);
         }
@@ -1198,28 +1240,35 @@ __global__ void __launch_bounds__(split_warps<PACK, KPROD, STAGED>() * 32, 1) de
         }
         float cq[4] = {0.f, 0.f, 0.f, 0.f};
         if constexpr (KPROD) {
+          // the signs as int8 0 / -1 (four a register, bits 7, 15, 23, 31 of
+          // the lane's word shifted left by 2S + j) against the S q' digits
+          int ch[4] = {0, 0, 0, 0}, cl[4] = {0, 0, 0, 0};
 #define TQ_QSTEP(S)                                                               \
   {                                                                               \
     uint32_t a[4];                                                                \
-    a[0] = qjl_half2<2 * (S)>(qj[0]);                                             \
-    a[1] = qjl_half2<2 * (S)>(qj[1]);                                             \
-    a[2] = qjl_half2<2 * (S) + 1>(qj[0]);                                         \
-    a[3] = qjl_half2<2 * (S) + 1>(qj[1]);                                         \
+    a[0] = sign_bytes(qj[0] << (2 * (S)));                                        \
+    a[1] = sign_bytes(qj[1] << (2 * (S)));                                        \
+    a[2] = sign_bytes(qj[0] << (2 * (S) + 1));                                    \
+    a[3] = sign_bytes(qj[1] << (2 * (S) + 1));                                    \
     if constexpr (QS_SMEM) {                                                      \
       const uint2 f = s_qs[((S) * 2) * 32 + lane];                                \
-      mma16816(cq, a, f.x, f.y);                                                  \
+      mma16832_s8(ch, a, f.x, f.y);                                               \
       if constexpr (!PACK) {                                                      \
         const uint2 f2 = s_qs[((S) * 2 + 1) * 32 + lane];                         \
-        mma16816(cq, a, f2.x, f2.y);                                              \
+        mma16832_s8(cl, a, f2.x, f2.y);                                           \
       }                                                                           \
     } else {                                                                      \
-      mma16816(cq, a, qsf[S][0], qsf[S][1]);                                      \
-      if constexpr (!PACK) mma16816(cq, a, qsf2[S][0], qsf2[S][1]);               \
+      mma16832_s8(ch, a, qsf[S][0], qsf[S][1]);                                   \
+      if constexpr (!PACK) mma16832_s8(cl, a, qsf2[S][0], qsf2[S][1]);            \
     }                                                                             \
   }
           TQ_QSTEP(0) TQ_QSTEP(1) TQ_QSTEP(2) TQ_QSTEP(3)
-          TQ_QSTEP(4) TQ_QSTEP(5) TQ_QSTEP(6) TQ_QSTEP(7)
 #undef TQ_QSTEP
+#pragma unroll
+          for (int i = 0; i < 4; ++i) {
+            const int c = i & 1;
+            cq[i] = fmaf((float)ch[i], qd[c][0], PACK ? qd[c][2] : fmaf((float)cl[i], qd[c][1], qd[c][2]));
+          }
         }
         // raw score = main + kappa gamma s_K qjl (the table holds s_K c)
 #pragma unroll

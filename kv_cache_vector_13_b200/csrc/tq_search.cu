@@ -141,12 +141,13 @@ __global__ void __launch_bounds__(kSrWarps * 32) search_score_kernel(SearchParam
 
   // the unit's query fragments (layout of the decode prep kernel)
   uint32_t qf[8][2], qf2[PACK ? 1 : 8][2];
-  uint32_t qsf[KPROD ? 8 : 1][2], qsf2[(KPROD && !PACK) ? 8 : 1][2];
+  uint32_t qsf[KPROD ? 4 : 1][2], qsf2[(KPROD && !PACK) ? 4 : 1][2];
+  float qd[2][3];  // digit weights and constant of this lane's two query columns
   {
     const bool has = (PACK ? (g8 & 3) : g8) < gh;
     const uint4 *fr = p.frag + (int64_t)u * (kFragWords / 4) + lane;
     auto ld4 = [&](int w4) { return has ? __ldg(fr + w4 * 32) : make_uint4(0u, 0u, 0u, 0u); };
-    auto put = [](uint32_t (&f)[8][2], int k, uint4 v) {
+    auto put = [](auto &f, int k, uint4 v) {
       f[2 * k][0] = v.x;
       f[2 * k][1] = v.y;
       f[2 * k + 1][0] = v.z;
@@ -156,8 +157,21 @@ __global__ void __launch_bounds__(kSrWarps * 32) search_score_kernel(SearchParam
     for (int k = 0; k < 4; ++k) {
       put(qf, k, ld4(k));
       if constexpr (!PACK) put(qf2, k, ld4(4 + k));
+    }
+#pragma unroll
+    for (int k = 0; k < 2; ++k) {
       if constexpr (KPROD) put(qsf, k, ld4((PACK ? 4 : 8) + k));
-      if constexpr (KPROD && !PACK) put(qsf2, k, ld4(12 + k));
+      if constexpr (KPROD && !PACK) put(qsf2, k, ld4(10 + k));
+    }
+    const uint32_t *fw = reinterpret_cast<const uint32_t *>(p.frag + (int64_t)u * (kFragWords / 4));
+#pragma unroll
+    for (int c = 0; c < 2; ++c) {
+      const int h = PACK ? 2 * (tig & 1) + c : 2 * tig + c;
+      const float ch = (KPROD && h < gh) ? __uint_as_float(__ldg(fw + (15 * 32 + h) * 4 + 0)) : 0.f;
+      const float th = (KPROD && h < gh) ? __uint_as_float(__ldg(fw + (15 * 32 + h) * 4 + 1)) : 0.f;
+      qd[c][0] = PACK ? -2.f * ch * (tig < 2 ? 256.f : 1.f) : -512.f * ch;
+      qd[c][1] = PACK ? 0.f : -2.f * ch;
+      qd[c][2] = (PACK && tig >= 2) ? 0.f : -th;
     }
   }
 
@@ -200,19 +214,24 @@ __global__ void __launch_bounds__(kSrWarps * 32) search_score_kernel(SearchParam
       }
       float cq[4] = {0.f, 0.f, 0.f, 0.f};
       if constexpr (KPROD) {
-#define TQ_SQSTEP(S)                                            \
-  {                                                             \
-    uint32_t a[4];                                              \
-    a[0] = qjl_half2<2 * (S)>(qj[0]);                           \
-    a[1] = qjl_half2<2 * (S)>(qj[1]);                           \
-    a[2] = qjl_half2<2 * (S) + 1>(qj[0]);                       \
-    a[3] = qjl_half2<2 * (S) + 1>(qj[1]);                       \
-    mma16816(cq, a, qsf[S][0], qsf[S][1]);                      \
-    if constexpr (!PACK) mma16816(cq, a, qsf2[S][0], qsf2[S][1]); \
+        int ch[4] = {0, 0, 0, 0}, cl[4] = {0, 0, 0, 0};
+#define TQ_SQSTEP(S)                                                  \
+  {                                                                   \
+    uint32_t a[4];                                                    \
+    a[0] = sign_bytes(qj[0] << (2 * (S)));                            \
+    a[1] = sign_bytes(qj[1] << (2 * (S)));                            \
+    a[2] = sign_bytes(qj[0] << (2 * (S) + 1));                        \
+    a[3] = sign_bytes(qj[1] << (2 * (S) + 1));                        \
+    mma16832_s8(ch, a, qsf[S][0], qsf[S][1]);                         \
+    if constexpr (!PACK) mma16832_s8(cl, a, qsf2[S][0], qsf2[S][1]);  \
   }
         TQ_SQSTEP(0) TQ_SQSTEP(1) TQ_SQSTEP(2) TQ_SQSTEP(3)
-        TQ_SQSTEP(4) TQ_SQSTEP(5) TQ_SQSTEP(6) TQ_SQSTEP(7)
 #undef TQ_SQSTEP
+#pragma unroll
+        for (int i = 0; i < 4; ++i) {
+          const int c = i & 1;
+          cq[i] = fmaf((float)ch[i], qd[c][0], PACK ? qd[c][2] : fmaf((float)cl[i], qd[c][1], qd[c][2]));
+        }
       }
 #pragma unroll
       for (int i = 0; i < 4; ++i) {
