@@ -25,11 +25,13 @@ TOL = 2e-3
 
 
 def run_case(B, Hq, Hkv, N, kspec, vspec, seed=0, seq_lens=None, kv_scale=1.0, heads=None, scores=False, d=128,
-             rotation=("hadamard", "hadamard")):
+             rotation=("hadamard", "hadamard"), zero_q_heads=()):
     g = torch.Generator(device=DEV).manual_seed(seed)
     K = torch.randn((B, Hkv, N, d), generator=g, device=DEV) * kv_scale
     V = torch.randn((B, Hkv, N, d), generator=g, device=DEV)
     q = torch.randn((B, Hq, d), generator=g, device=DEV).to(torch.bfloat16)
+    for h in zero_q_heads:
+        q[:, h] = 0
     kq = api.Quantizer(d, kspec[0], kspec[1], seed_rot=seed + 1, seed_qjl=seed + 2, device=DEV, rotation=rotation[0])
     vq = api.Quantizer(d, vspec[0], vspec[1], seed_rot=seed + 3, seed_qjl=seed + 4, device=DEV,
                        rotation=rotation[1])
@@ -74,9 +76,16 @@ def test_decode_ragged_lengths(N):
     run_case(1, 4, 1, N, (4, "mse"), (4, "mse"), seed=N)
 
 
-@pytest.mark.parametrize("g", [1, 2, 4, 8, 16])
+@pytest.mark.parametrize("g", [1, 2, 3, 4, 6, 8, 16])
 def test_decode_gqa_group_sizes(g):
     run_case(1, 2 * g, 2, 700, (3, "prod"), (3, "mse"), seed=g)
+
+
+@pytest.mark.parametrize("Hq,kspec", [(8, (3, "prod")), (16, (4, "prod")), (8, (1, "prod"))])
+def test_decode_zero_query_heads(Hq, kspec):
+    # a zero query: S q' = 0 (its int8 digit scale falls back to 1), every
+    # score is 0 and the softmax is uniform
+    run_case(1, Hq, 2, 513, kspec, (3, "mse"), seed=40 + Hq, zero_q_heads=(0, 5), scores=True)
 
 
 def test_decode_per_batch_lengths_including_empty():
