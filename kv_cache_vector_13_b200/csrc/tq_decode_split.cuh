@@ -1317,13 +1317,18 @@ __global__ void __launch_bounds__(split_warps<PACK, KPROD, STAGED>() * 32, 1) de
       bool moved = false;
 #pragma unroll
       for (int c = 0; c < 2; ++c) {
-        float mx = fmaxf(fmaxf(sc[0][c], sc[0][2 + c]), fmaxf(sc[1][c], sc[1][2 + c]));
+        // m: this lane's own running maximum (the lanes' sums are rescaled
+        // to a common one after the loop); M: the column's, moved only when
+        // some lane's candidate passes it by more than kLazy (one vote, and
+        // the column maximum only then)
+        const float mx = fmaxf(fmaxf(sc[0][c], sc[0][2 + c]), fmaxf(sc[1][c], sc[1][2 + c]));
         float Mx = fmaxf(fmaxf(sc[0][c] + nvl[0][0], sc[0][2 + c] + nvl[0][1]),
                          fmaxf(sc[1][c] + nvl[1][0], sc[1][2 + c] + nvl[1][1]));
+        if (__any_sync(dev::kFull, Mx > M_run[c] + kLazy)) {
 #pragma unroll
-        for (int o = 4; o <= 16; o <<= 1) {
-          mx = fmaxf(mx, __shfl_xor_sync(dev::kFull, mx, o));
-          Mx = fmaxf(Mx, __shfl_xor_sync(dev::kFull, Mx, o));
+          for (int o = 4; o <= 16; o <<= 1) Mx = fmaxf(Mx, __shfl_xor_sync(dev::kFull, Mx, o));
+        } else {
+          Mx = M_run[c];
         }
         const float mn = fmaxf(m_run[c], mx);
         const float Mn = Mx > M_run[c] + kLazy ? Mx : M_run[c];
@@ -1414,9 +1419,15 @@ __global__ void __launch_bounds__(split_warps<PACK, KPROD, STAGED>() * 32, 1) de
       }
     }
 
-    // ---- warp totals: l over the 8 row groups; PACK: hi + lo columns of acc
+    // ---- warp totals: l over the 8 row groups, each lane's sum rescaled to
+    // the column's maximum; PACK: hi + lo columns of acc
 #pragma unroll
     for (int c = 0; c < 2; ++c) {
+      float mc = m_run[c];
+#pragma unroll
+      for (int o = 4; o <= 16; o <<= 1) mc = fmaxf(mc, __shfl_xor_sync(dev::kFull, mc, o));
+      l_run[c] *= ex2(m_run[c] - (mc == -INFINITY ? 0.f : mc));
+      m_run[c] = mc;
 #pragma unroll
       for (int o = 4; o <= 16; o <<= 1) l_run[c] += __shfl_xor_sync(dev::kFull, l_run[c], o);
     }
