@@ -49,6 +49,7 @@ struct DenseParams {
   int d, bm, kcb;
   bool prod;
   float *out;  // dequant
+  dev::IndexSplit ix;
 };
 
 __device__ __forceinline__ float load_elem(const void *base, int dtype, int64_t i) {
@@ -73,10 +74,7 @@ __device__ __forceinline__ float row_dot(const float *M, int row, int d, const f
 }
 
 __device__ __forceinline__ void bhn(const DenseParams &p, int64_t v, int64_t &b, int64_t &h, int64_t &n) {
-  n = v % p.N;
-  const int64_t bh = v / p.N;
-  h = bh % p.H;
-  b = bh / p.H;
+  dev::split_bhn(p.ix, v, b, h, n);
 }
 
 __global__ void __launch_bounds__(kDnWarps * 32) encode_dense_kernel(DenseParams p) {
@@ -492,6 +490,7 @@ cudaError_t launch_encode_dense(const EncodeArgs &a, cudaStream_t s) {
   p.bm = a.q.bm;
   p.kcb = a.q.d * a.q.bm / 8;
   p.prod = a.q.prod;
+  p.ix = dev::make_index_split(p.H, p.N, p.nvec);
   // large TurboQuant_mse batches at d = 64 / 128: the rotation on tcgen05
   if (!p.prod && !p.chan && (p.d == 64 || p.d == 128) && p.nvec >= 8 * kTcM) {
     unsigned *faults = nullptr;
@@ -525,6 +524,7 @@ cudaError_t launch_dequant_dense(const DequantArgs &a, cudaStream_t s) {
   p.kcb = a.q.d * a.q.bm / 8;
   p.prod = a.q.prod;
   p.out = a.out;
+  p.ix = dev::make_index_split(p.H, p.N, p.nvec);
   const int64_t blocks = (p.nvec + kDnWarps - 1) / kDnWarps;
   dequant_dense_kernel<<<(unsigned)blocks, kDnWarps * 32, 0, s>>>(p);
   return cudaGetLastError();

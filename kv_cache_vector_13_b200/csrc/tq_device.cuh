@@ -144,6 +144,55 @@ __device__ __forceinline__ float fold_halves_sumsq(const float (&a)[E]) {
   return fold_sumsq_node<T, E, 0, 1>(a);
 }
 
+// ------------------------------------------------------- index splitting
+
+// Vector index v -> (b, h, n) of a [B][H][N] batch.  When every index fits
+// in 31 bits the divisions are multiply-shifts, q = (x * m) >> (31 + l) with
+// l = ceil(log2 divisor), m = floor(2^(31+l) / divisor) + 1, exact for
+// x < 2^31 (Granlund and Montgomery, "Division by invariant integers using
+// multiplication"); else 64-bit division.
+struct IndexSplit {
+  int64_t H, N;
+  bool div32;
+  uint32_t mN, mH;
+  int sN, sH;
+};
+
+inline void magic31_div(int64_t d, uint32_t &m, int &s) {
+  int l = 0;
+  while (((int64_t)1 << l) < d) ++l;
+  m = (uint32_t)((((uint64_t)1 << (31 + l)) / (uint64_t)d) + 1);
+  s = 31 + l;
+}
+
+inline IndexSplit make_index_split(int64_t H, int64_t N, int64_t nvec) {
+  IndexSplit x{};
+  x.H = H;
+  x.N = N;
+  x.div32 = nvec < ((int64_t)1 << 31) && N > 0 && H > 0;
+  if (x.div32) {
+    magic31_div(N, x.mN, x.sN);
+    magic31_div(H, x.mH, x.sH);
+  }
+  return x;
+}
+
+__device__ __forceinline__ void split_bhn(const IndexSplit &x, int64_t v, int64_t &b, int64_t &h, int64_t &n) {
+  if (x.div32) {
+    const uint32_t u = (uint32_t)v;
+    const uint32_t bh = (uint32_t)(((uint64_t)u * x.mN) >> x.sN);
+    const uint32_t hb = (uint32_t)(((uint64_t)bh * x.mH) >> x.sH);
+    n = u - bh * (uint32_t)x.N;
+    h = bh - hb * (uint32_t)x.H;
+    b = hb;
+  } else {
+    n = v % x.N;
+    const int64_t bh = v / x.N;
+    h = bh % x.H;
+    b = bh / x.H;
+  }
+}
+
 // -------------------------------------------------------------- quantize
 
 // idx = #{j : u > t_j} for an antisymmetric codebook with K = 2^BM levels,
