@@ -36,7 +36,6 @@ constexpr int kGnMaxD = 256;
 constexpr int kGnHeads = 8;   // query heads a block
 constexpr int kGnTile = 64;   // tokens a tile
 constexpr int kGnSub = 8;     // tokens a value-decode step
-constexpr int kGnCoords = kGnHeads * kGnMaxD / kGnThreads;  // (head, coordinate) pairs a thread
 constexpr float kGnLog2e = 1.4426950408889634f;
 constexpr float kGnSqrtHalfPi = 1.2533141373155003f;
 
@@ -113,6 +112,9 @@ __device__ void gn_fwht(float *x, int nv, int d, int stride) {
   __syncthreads();
 }
 
+// NH: the most query heads a block handles (1, 2, 4 or 8): the per-token
+// head loops are unrolled to it.
+template <int NH>
 __global__ void __launch_bounds__(kGnThreads) general_partial_kernel(GnParams p) {
   __shared__ float s_q[kGnHeads][kGnMaxD];   // q'_g at the group's offset
   __shared__ float s_qs[kGnHeads][kGnMaxD];  // S_g q'_g (prod groups); staging of q[channels] first
@@ -127,7 +129,7 @@ __global__ void __launch_bounds__(kGnThreads) general_partial_kernel(GnParams p)
   const int hgi = u % p.hg, bk = u / p.hg;
   const int b = bk / p.Hkv, kvh = bk % p.Hkv;
   const int h0 = kvh * p.g + kGnHeads * hgi;
-  const int nh = min(kGnHeads, p.g - kGnHeads * hgi);
+  const int nh = min(NH, p.g - kGnHeads * hgi);
   const int64_t L = gn_len(p, b);
   const int64_t t0 = (int64_t)split * p.per_split;
   const int64_t t1 = min(L, t0 + p.per_split);
@@ -182,11 +184,12 @@ __global__ void __launch_bounds__(kGnThreads) general_partial_kernel(GnParams p)
   __syncthreads();
 
   // this thread's (head, coordinate) pairs: e = tid + kGnThreads * c
-  float acc[kGnCoords], sacc[kGnCoords];
-  int c_h[kGnCoords], c_i[kGnCoords];
-  bool c_prod[kGnCoords];
+  constexpr int kCoords = NH * kGnMaxD / kGnThreads > 0 ? NH * kGnMaxD / kGnThreads : 1;
+  float acc[kCoords], sacc[kCoords];
+  int c_h[kCoords], c_i[kCoords];
+  bool c_prod[kCoords];
 #pragma unroll
-  for (int c = 0; c < kGnCoords; ++c) {
+  for (int c = 0; c < kCoords; ++c) {
     acc[c] = sacc[c] = 0.f;
     const int e = tid + kGnThreads * c;
     c_h[c] = e < nh * d ? e / d : -1;
@@ -206,9 +209,9 @@ __global__ void __launch_bounds__(kGnThreads) general_partial_kernel(GnParams p)
       const int tt = tid >> 2, qq = tid & 3;
       const bool ok = tt < nt;
       const int64_t j = base + (ok ? tt : 0);
-      float tot[kGnHeads];
+      float tot[NH];
 #pragma unroll
-      for (int hh = 0; hh < kGnHeads; ++hh) tot[hh] = 0.f;
+      for (int hh = 0; hh < NH; ++hh) tot[hh] = 0.f;
       if (ok) {
         for (int gr = 0; gr < p.nk; ++gr) {
           const GnGroup &G = p.k[gr];
@@ -216,35 +219,38 @@ __global__ void __launch_bounds__(kGnThreads) general_partial_kernel(GnParams p)
           const int kcb = G.d * G.bm / 8;
           const uint8_t *kc = G.bm > 0 ? G.codes + kr * kcb : nullptr;
           const uint8_t *kj = G.prod ? G.qjl + kr * (G.d / 8) : nullptr;
-          float part[kGnHeads], qpart[kGnHeads];
+          float part[NH], qpart[NH];
 #pragma unroll
-          for (int hh = 0; hh < kGnHeads; ++hh) part[hh] = qpart[hh] = 0.f;
+          for (int hh = 0; hh < NH; ++hh) part[hh] = qpart[hh] = 0.f;
           const int i0 = qq * (G.d / 4), i1 = i0 + G.d / 4;
           for (int i = i0; i < i1; ++i) {
             const float c = G.bm > 0 ? __ldg(G.cent + gn_field(kc, i, G.bm, kcb)) : 0.f;
             const float sg = G.prod ? (gn_bit(kj, i) ? 1.f : -1.f) : 0.f;
+            if (G.prod) {
 #pragma unroll
-            for (int hh = 0; hh < kGnHeads; ++hh) {
-              if (hh < nh) {
+              for (int hh = 0; hh < NH; ++hh) {
                 part[hh] = fmaf(c, s_q[hh][G.off + i], part[hh]);
-                if (G.prod) qpart[hh] = fmaf(sg, s_qs[hh][G.off + i], qpart[hh]);
+                qpart[hh] = fmaf(sg, s_qs[hh][G.off + i], qpart[hh]);
               }
+            } else {
+#pragma unroll
+              for (int hh = 0; hh < NH; ++hh) part[hh] = fmaf(c, s_q[hh][G.off + i], part[hh]);
             }
           }
           const float n = __ldg(G.norms + kr);
           const float kap = G.prod ? __ldg(G.rnorms + kr) * (kGnSqrtHalfPi / (float)G.d) : 0.f;
 #pragma unroll
-          for (int hh = 0; hh < kGnHeads; ++hh) tot[hh] = fmaf(n, fmaf(kap, qpart[hh], part[hh]), tot[hh]);
+          for (int hh = 0; hh < NH; ++hh) tot[hh] = fmaf(n, fmaf(kap, qpart[hh], part[hh]), tot[hh]);
         }
       }
 #pragma unroll
-      for (int hh = 0; hh < kGnHeads; ++hh) {
+      for (int hh = 0; hh < NH; ++hh) {
         tot[hh] += __shfl_xor_sync(dev::kFull, tot[hh], 1);
         tot[hh] += __shfl_xor_sync(dev::kFull, tot[hh], 2);
       }
       if (qq == 0) {
 #pragma unroll
-        for (int hh = 0; hh < kGnHeads; ++hh) {
+        for (int hh = 0; hh < NH; ++hh) {
           if (hh < nh) {
             s_w[hh][tt] = ok ? tot[hh] * p.scale_log2 : -INFINITY;
             if (ok && p.scores) p.scores[((int64_t)b * p.Hq + h0 + hh) * p.seq_len + j] = tot[hh];
@@ -287,7 +293,7 @@ __global__ void __launch_bounds__(kGnThreads) general_partial_kernel(GnParams p)
     // n_V ||r|| sqrt(pi/2)/d sign), then each (head, coordinate) thread
     // accumulates its weights times them
 #pragma unroll
-    for (int c = 0; c < kGnCoords; ++c) {
+    for (int c = 0; c < kCoords; ++c) {
       if (c_h[c] >= 0) {
         acc[c] *= s_alpha[c_h[c]];
         sacc[c] *= s_alpha[c_h[c]];
@@ -313,7 +319,7 @@ __global__ void __launch_bounds__(kGnThreads) general_partial_kernel(GnParams p)
       }
       __syncthreads();
 #pragma unroll
-      for (int c = 0; c < kGnCoords; ++c) {
+      for (int c = 0; c < kCoords; ++c) {
         if (c_h[c] >= 0) {
           const int hh = c_h[c], i = c_i[c];
           float a = acc[c], sa = sacc[c];
@@ -333,7 +339,7 @@ __global__ void __launch_bounds__(kGnThreads) general_partial_kernel(GnParams p)
   // ---- the slice's partial state
   const int stride = 4 + 2 * d;
 #pragma unroll
-  for (int c = 0; c < kGnCoords; ++c) {
+  for (int c = 0; c < kCoords; ++c) {
     const int e = tid + kGnThreads * c;
     if (e < nh * d) {
       const int hh = e / d, i = e % d;
@@ -449,7 +455,15 @@ cudaError_t launch_general(GnParams &p, cudaStream_t s) {
   p.per_split = (p.seq_len + p.splits - 1) / p.splits;
   if (p.seq_len > 0) {
     const dim3 grid((unsigned)p.splits, (unsigned)(p.B * p.Hkv * p.hg));
-    general_partial_kernel<<<grid, kGnThreads, 0, s>>>(p);
+    if (p.g <= 1) {
+      general_partial_kernel<1><<<grid, kGnThreads, 0, s>>>(p);
+    } else if (p.g <= 2) {
+      general_partial_kernel<2><<<grid, kGnThreads, 0, s>>>(p);
+    } else if (p.g <= 4) {
+      general_partial_kernel<4><<<grid, kGnThreads, 0, s>>>(p);
+    } else {
+      general_partial_kernel<8><<<grid, kGnThreads, 0, s>>>(p);
+    }
     const cudaError_t e = cudaGetLastError();
     if (e != cudaSuccess) return e;
   } else {
