@@ -82,10 +82,10 @@ FALLBACK_PEAKS = {"hbm_gbs": 6650.0, "bf16_tflops": 1590.0}
 # workload, from an ncu capture (dram__bytes_read.sum + dram__bytes_write.sum),
 # reported only for that workload and while the decode sources are the ones
 # it was taken on.
-# Captured at B = 2 (reads 230,614,784 B, writes 5,357,568 B): reads scaled by
+# Captured at B = 2 (reads 230,584,576 B, writes 4,909,568 B): reads scaled by
 # the 8x units of B = 16 (B = 4 read 2.02x the B = 2 bytes), writes kept.
-TRAFFIC = {"workload": ("batched", 16), "bytes": 8 * 230614784 + 5357568,
-           "source_sha256": "e843492af00ef221305e93b467bd2d6a2c98a804c49963e91f7f9e7eda5e9638"}
+TRAFFIC = {"workload": ("batched", 16), "bytes": 8 * 230584576 + 4909568,
+           "source_sha256": "343a0ed3f5953b6e11dcebf16029f430d30dc8ff5c04d583407db6010b4803be"}
 DECODE_SOURCES = ("tq_decode.cu", "tq_decode_split.cuh", "tq_decode_regs.cu")
 
 
