@@ -76,6 +76,16 @@ constexpr int kLutBytes = 256 * 256;     // K and V pair tables, per-lane copies
 // 64 KiB boundary, one byte permute of (code byte, lane offset) yields the
 // complete shared address of a lookup.
 constexpr uint32_t kLutAddr = 0x10000;
+// Register-fed kernel with 2-bit key codes: one code byte (four codes) is
+// one lookup of a 64-bit entry (four fp16 centroids), so the key table takes
+// the whole 64 KiB window (entry e, lane l at kLutAddr + 256 e + 8 l) and the
+// value table moves to the next window (kVTab4Addr + 256 e + 4 l).  The query
+// digit fragments and the warps' partials then sit below kLutAddr.
+constexpr uint32_t kVTab4Addr = 0x20000;
+template <int KBM, bool STAGED>
+__host__ __device__ constexpr bool key_quads() {
+  return KBM == 2 && !STAGED;
+}
 constexpr int kPfWin = 4;                // chunks per L2 prefetch window (register-fed variant)
 constexpr int kMaxRing = 4;              // ring slots per warp (staged variant)
 // A bounded wait gives up after this long without progress (ns).
@@ -106,6 +116,8 @@ constexpr int kHdr = 1024;
 //   c_h and word 61 of lane h holds T_h = sum_k Sq'_h[k] (h < 8, the
 //   unit's heads).
 constexpr int kFragWords = 32 * 64;
+// Bytes of a unit's QJL digit fragments in shared memory ([4][2][32] uint2).
+constexpr uint32_t kQsBytes = 2 * 4 * 32 * 8;
 constexpr float kLog2e = 1.4426950408889634f;
 constexpr float kKappa = 1.2533141373155003f / (float)kD;  // sqrt(pi/2)/d
 
@@ -225,6 +237,13 @@ __device__ __forceinline__ uint32_t movmatrix_trans(uint32_t x) {
 __device__ __forceinline__ uint32_t lut(uint32_t addr) {
   uint32_t v;
   asm("ld.shared.b32 %0, [%1];\n" : "=r"(v) : "r"(addr));
+  return v;
+}
+
+// 64-bit table entry (two half2) at shared-window address `addr`
+__device__ __forceinline__ uint2 lut64(uint32_t addr) {
+  uint2 v;
+  asm("ld.shared.v2.b32 {%0, %1}, [%2];\n" : "=r"(v.x), "=r"(v.y) : "r"(addr));
   return v;
 }
 
@@ -925,8 +944,15 @@ __global__ void __launch_bounds__(split_warps<PACK, KPROD, STAGED>() * 32, 1) de
     if (threadIdx.x == 0) atomicOr(p.faults, kFaultSmemLayout);
     return;
   }
+  constexpr bool K4 = key_quads<KBM, STAGED>();
   char *s_lut = smem + (kLutAddr - dyn_base);
-  float *s_part = reinterpret_cast<float *>(s_lut + kLutBytes);  // [kWarps][8][kPW]
+  // [kWarps][8][kPW]; with key quads below the tables, past the digit fragments
+  float *s_part = K4 ? reinterpret_cast<float *>(smem + (((dyn_base + 15u) & ~15u) - dyn_base) + kQsBytes)
+                     : reinterpret_cast<float *>(s_lut + kLutBytes);
+  if (K4 && ((dyn_base + 15u) & ~15u) + kQsBytes + (uint32_t)(kWarps * 8 * kPW * 4) > kLutAddr) {
+    if (threadIdx.x == 0) atomicOr(p.faults, kFaultSmemLayout);  // excluded on the host
+    return;
+  }
   __shared__ int s_last;
   __shared__ int64_t s_cut[kMaxCtas + 1];
   __shared__ __align__(8) uint64_t s_bar[STAGED ? kWarps * kMaxRing : 1];
@@ -1041,16 +1067,30 @@ __global__ void __launch_bounds__(split_warps<PACK, KPROD, STAGED>() * 32, 1) de
     inv_sK = __ldg(p.ws + 0);
     inv_sV = __ldg(p.ws + 1);
     uint4 *tab = reinterpret_cast<uint4 *>(s_lut);
-    for (int i = tid; i < 256 * 16; i += kThreads) {  // 16 uint4 per 256-byte row
-      const int e = i >> 4, part = i & 15;
-      const uint32_t v = part < 8 ? (KBM > 0 ? __ldg(ktab + e) : 0u) : __ldg(vtab + e);
-      tab[i] = make_uint4(v, v, v, v);
+    if constexpr (K4) {
+      // key entry e: the pair entries of its low and high nibbles
+      for (int i = tid; i < 256 * 16; i += kThreads) {
+        const int e = i >> 4;
+        const uint32_t lo = __ldg(ktab + (e & 15)), hi = __ldg(ktab + (e >> 4));
+        tab[i] = make_uint4(lo, hi, lo, hi);
+      }
+      uint4 *vt = reinterpret_cast<uint4 *>(s_lut + (kVTab4Addr - kLutAddr));
+      for (int i = tid; i < 256 * 8; i += kThreads) {  // the first 128 bytes of each row
+        const uint32_t v = __ldg(vtab + (i >> 3));
+        vt[(i >> 3) * 16 + (i & 7)] = make_uint4(v, v, v, v);
+      }
+    } else {
+      for (int i = tid; i < 256 * 16; i += kThreads) {  // 16 uint4 per 256-byte row
+        const int e = i >> 4, part = i & 15;
+        const uint32_t v = part < 8 ? (KBM > 0 ? __ldg(ktab + e) : 0u) : __ldg(vtab + e);
+        tab[i] = make_uint4(v, v, v, v);
+      }
     }
   }
   const float sK = 1.0f / inv_sK;
   const float kscale = inv_sK * p.scale_log2;  // logit = raw score * n_K * kscale
-  const uint32_t koff = kLutAddr + lane * 4;
-  const uint32_t voff = kLutAddr + 128 + lane * 4;
+  const uint32_t koff = kLutAddr + lane * (K4 ? 8 : 4);
+  const uint32_t voff = (K4 ? kVTab4Addr : kLutAddr + 128) + lane * 4;
   const bool want_scores = p.scores != nullptr;
 
   bool first_piece = true;
@@ -1223,7 +1263,21 @@ __global__ void __launch_bounds__(split_warps<PACK, KPROD, STAGED>() * 32, 1) de
           nvl[ms][r] = ok[r] ? __log2f(kb.vn[ms][r]) : -INFINITY;
         }
         float cm[4] = {0.f, 0.f, 0.f, 0.f};
-        if constexpr (KBM > 0) {
+        if constexpr (K4) {
+          // byte S of a row's 64-bit stream: pairs 2S and 2S + 1 in one read
+#define TQ_KSTEP4(S)                                                              \
+  {                                                                               \
+    constexpr uint32_t sel = 0x7604u | (((S) & 3) << 4);                          \
+    const uint2 e0 = lut64(__byte_perm(kw[0][(S) >> 2], koff, sel));              \
+    const uint2 e1 = lut64(__byte_perm(kw[1][(S) >> 2], koff, sel));              \
+    const uint32_t a[4] = {e0.x, e1.x, e0.y, e1.y};                               \
+    mma16816(cm, a, qf[S][0], qf[S][1]);                                          \
+    if constexpr (!PACK) mma16816(cm, a, qf2[S][0], qf2[S][1]);                   \
+  }
+          TQ_KSTEP4(0) TQ_KSTEP4(1) TQ_KSTEP4(2) TQ_KSTEP4(3)
+          TQ_KSTEP4(4) TQ_KSTEP4(5) TQ_KSTEP4(6) TQ_KSTEP4(7)
+#undef TQ_KSTEP4
+        } else if constexpr (KBM > 0) {
 #define TQ_KSTEP(S)                                                               \
   {                                                                               \
     uint32_t a[4];                                                                \
@@ -1538,10 +1592,14 @@ __global__ void zero_out_kernel(float *out, int64_t n) {
   if (i < n) out[i] = 0.f;
 }
 
-// Register-fed variant's dynamic shared memory: enough to reach kLutAddr +
-// kLutBytes + the warps' partials from any dynamic base at or above 0.
-constexpr size_t split_smem_bytes(int warps) {
-  return (size_t)kLutAddr + kLutBytes + (size_t)warps * 8 * kPW * sizeof(float);
+// Register-fed variant's dynamic shared memory: enough to reach the end of
+// the tables (key quads: the value table's window; else the warps'
+// partials past the shared window) from any dynamic base at or above 0.
+// Every table keeps 256 rows: a lookup's byte may carry bits of the next
+// field above a pair index.
+constexpr size_t split_smem_bytes(int warps, bool k4) {
+  return k4 ? (size_t)kVTab4Addr + kLutBytes
+            : (size_t)kLutAddr + kLutBytes + (size_t)warps * 8 * kPW * sizeof(float);
 }
 
 // Static shared memory plus the per-block reserve must end at or below
@@ -1593,7 +1651,11 @@ cudaError_t run_split(SplitParams sp, cudaStream_t s) {
   static const cudaError_t layout = smem_layout(kern, &dyn_max, &base);
   static const size_t dyn_keep = dyn_max, base_keep = base;
   if (layout != cudaSuccess) return layout;
-  size_t smem = split_smem_bytes(warps);
+  constexpr bool k4 = key_quads<KBM, STAGED>();
+  size_t smem = split_smem_bytes(warps, k4);
+  // key quads: digit fragments and partials below the tables
+  if (k4 && ((base_keep + 15) & ~(size_t)15) + kQsBytes + (size_t)warps * 8 * kPW * 4 > kLutAddr)
+    return cudaErrorInvalidConfiguration;
   if constexpr (STAGED) {
     smem = dyn_keep;
     constexpr size_t sb = (ring_slot_bytes(KBM, KPROD, VBM) + 127) & ~(size_t)127;
