@@ -46,9 +46,11 @@
 //     weights) share one MMA as columns 0-3 and 4-7; with 5-8 heads they take
 //     two MMAs;
 //   * QJL bits become +-1 halves with one shift and one LOP3 per pair;
-//   * online softmax in base 2 with two running maxima, m over the logits
-//     (for the normaliser l) and M over logit + log2 n_V (for the PV weights
-//     2^(u - M), which keeps p_j n_j in fp16 range).
+//   * online softmax in base 2 against one reference M per head column,
+//     taken over u = logit + max(log2 n_V, kNvlFloor) and moved only when
+//     some u passes it by more than kLazy: the PV weights 2^(logit + log2 n_V
+//     - M) stay below 2^kLazy (fp16 range), the normaliser's terms
+//     2^(logit - M) below 2^(kLazy - kNvlFloor) (fp32 range).
 // The warps' partials (m, l, M, o') of a piece are merged in shared memory
 // and written to workspace slot (unit + CTA index).  Each CTA then bumps its
 // unit's counter; the CTA that completes the count merges the unit's slots,
@@ -60,6 +62,7 @@
 #include "tq_device.cuh"
 #include "tq_internal.h"
 
+#include <float.h>
 #include <math.h>
 
 #include <atomic>
@@ -94,6 +97,9 @@ constexpr uint64_t kWaitLimitNs = 1000000000ull;
 // logit + log2 n_V passes it by more than kLazy (log2 units); the weights
 // then stay below 2^kLazy and most rescales of the accumulators are skipped.
 constexpr float kLazy = 8.0f;
+// Floor of log2 n_V in the reference: the normaliser's terms 2^(logit - M)
+// then stay below 2^(kLazy - kNvlFloor), tiny or zero value norms included.
+constexpr float kNvlFloor = -64.0f;
 constexpr int kPW = kD + 4;              // floats per head in a partial: m, l, M, pad, o'[d]
 constexpr int kSlot = 8 * kPW;           // floats per partial slot (8 heads)
 constexpr int kScaleCands = 4096;
@@ -1187,7 +1193,9 @@ __global__ void __launch_bounds__(split_warps<PACK, KPROD, STAGED>() * 32, 1) de
     float acc[8][4];
 #pragma unroll
     for (int i = 0; i < 8; ++i) acc[i][0] = acc[i][1] = acc[i][2] = acc[i][3] = 0.f;
-    float m_run[2] = {-INFINITY, -INFINITY}, M_run[2] = {-INFINITY, -INFINITY};
+    // M_run: the column's reference (finite; -FLT_MAX until a valid token);
+    // M_thr = M_run + kLazy
+    float M_run[2] = {-FLT_MAX, -FLT_MAX}, M_thr[2] = {-FLT_MAX, -FLT_MAX};
     float l_run[2] = {0.f, 0.f};
 
     const int64_t kbase = (int64_t)b * p.ksb + (int64_t)kvh * p.ksh;
@@ -1248,7 +1256,7 @@ __global__ void __launch_bounds__(split_warps<PACK, KPROD, STAGED>() * 32, 1) de
       }
       // -------- scores: rows (ms, r) -> token cstart + 16 ms + 8 r + g8
       float sc[2][4];
-      float nvl[2][2];  // log2 n_V of the lane's rows
+      float nvl[2][2];  // log2 n_V of the lane's rows (masked rows: any value, their logit is -inf)
 #pragma unroll
       for (int ms = 0; ms < 2; ++ms) {
         const auto &kw = kb.w[ms];
@@ -1260,7 +1268,8 @@ __global__ void __launch_bounds__(split_warps<PACK, KPROD, STAGED>() * 32, 1) de
           ok[r] = kb.kn[ms][r] >= 0.f;
           fs[r] = kb.kn[ms][r] * kscale;
           kr[r] = KPROD ? kb.kr[ms][r] * (kKappa * sK) : 0.f;  // the table holds s_K c
-          nvl[ms][r] = ok[r] ? __log2f(kb.vn[ms][r]) : -INFINITY;
+          // (staged masked rows hold whatever the slot holds: kept finite)
+          nvl[ms][r] = (STAGED && !ok[r]) ? 0.f : __log2f(kb.vn[ms][r]);
         }
         float cm[4] = {0.f, 0.f, 0.f, 0.f};
         if constexpr (K4) {
@@ -1365,47 +1374,36 @@ __global__ void __launch_bounds__(split_warps<PACK, KPROD, STAGED>() * 32, 1) de
         }
       }
 
-      // -------- online softmax, per head column c
+      // -------- online softmax, per head column c, against the column's
+      // reference M_run, which moves only when some lane's u = logit +
+      // max(log2 n_V, kNvlFloor) passes it by more than kLazy: one vote for
+      // both columns, and the column maxima, the rescale of l and of the
+      // accumulators only then (warp-uniform branch)
       float wgt[2][4];
-      float aM[2];
-      bool moved = false;
+      float Mx[2];
 #pragma unroll
       for (int c = 0; c < 2; ++c) {
-        // m: this lane's own running maximum (the lanes' sums are rescaled
-        // to a common one after the loop); M: the column's, moved only when
-        // some lane's candidate passes it by more than kLazy (one vote, and
-        // the column maximum only then)
-        const float mx = fmaxf(fmaxf(sc[0][c], sc[0][2 + c]), fmaxf(sc[1][c], sc[1][2 + c]));
-        float Mx = fmaxf(fmaxf(sc[0][c] + nvl[0][0], sc[0][2 + c] + nvl[0][1]),
-                         fmaxf(sc[1][c] + nvl[1][0], sc[1][2 + c] + nvl[1][1]));
-        if (__any_sync(dev::kFull, Mx > M_run[c] + kLazy)) {
-#pragma unroll
-          for (int o = 4; o <= 16; o <<= 1) Mx = fmaxf(Mx, __shfl_xor_sync(dev::kFull, Mx, o));
-        } else {
-          Mx = M_run[c];
-        }
-        const float mn = fmaxf(m_run[c], mx);
-        const float Mn = Mx > M_run[c] + kLazy ? Mx : M_run[c];
-        const float ms_ = mn == -INFINITY ? 0.f : mn;
-        const float Ms_ = Mn == -INFINITY ? 0.f : Mn;
-        const float al = ex2(m_run[c] - ms_);
-        aM[c] = ex2(M_run[c] - Ms_);
-        moved |= Mn != M_run[c];
-        m_run[c] = mn;
-        M_run[c] = Mn;
-        float ls = 0.f;
+        float u[4];
 #pragma unroll
         for (int ms = 0; ms < 2; ++ms) {
 #pragma unroll
-          for (int r = 0; r < 2; ++r) {
-            const float t = sc[ms][2 * r + c];
-            ls += ex2(t - ms_);
-            wgt[ms][2 * r + c] = ex2(t + nvl[ms][r] - Ms_);
-          }
+          for (int r = 0; r < 2; ++r) u[2 * ms + r] = sc[ms][2 * r + c] + fmaxf(nvl[ms][r], kNvlFloor);
         }
-        l_run[c] = fmaf(l_run[c], al, ls);
+        Mx[c] = fmaxf(fmaxf(u[0], u[1]), fmaxf(u[2], u[3]));
       }
-      if (__any_sync(dev::kFull, moved)) {
+      if (__any_sync(dev::kFull, Mx[0] > M_thr[0] || Mx[1] > M_thr[1])) {
+        float aM[2];
+#pragma unroll
+        for (int c = 0; c < 2; ++c) {
+          float m = Mx[c];
+#pragma unroll
+          for (int o = 4; o <= 16; o <<= 1) m = fmaxf(m, __shfl_xor_sync(dev::kFull, m, o));
+          const float Mn = m > M_thr[c] ? m : M_run[c];
+          aM[c] = ex2(M_run[c] - Mn);
+          l_run[c] *= aM[c];
+          M_run[c] = Mn;
+          M_thr[c] = Mn + kLazy;
+        }
 #pragma unroll
         for (int mt = 0; mt < 8; ++mt) {
           acc[mt][0] *= aM[0];
@@ -1413,6 +1411,20 @@ __global__ void __launch_bounds__(split_warps<PACK, KPROD, STAGED>() * 32, 1) de
           acc[mt][2] *= aM[0];
           acc[mt][3] *= aM[1];
         }
+      }
+#pragma unroll
+      for (int c = 0; c < 2; ++c) {
+        float ls = 0.f;
+#pragma unroll
+        for (int ms = 0; ms < 2; ++ms) {
+#pragma unroll
+          for (int r = 0; r < 2; ++r) {
+            const float e = sc[ms][2 * r + c] - M_run[c];
+            ls += ex2(e);
+            wgt[ms][2 * r + c] = ex2(e + nvl[ms][r]);
+          }
+        }
+        l_run[c] += ls;
       }
 
       // -------- PV: for each 16-token half, B = W^T via movmatrix
@@ -1473,17 +1485,16 @@ __global__ void __launch_bounds__(split_warps<PACK, KPROD, STAGED>() * 32, 1) de
       }
     }
 
-    // ---- warp totals: l over the 8 row groups, each lane's sum rescaled to
-    // the column's maximum; PACK: hi + lo columns of acc
+    // ---- warp totals: l over the 8 row groups (one reference per column);
+    // a column that saw no valid token reports -inf; PACK: hi + lo columns
+    // of acc
+    float m_run[2];
 #pragma unroll
     for (int c = 0; c < 2; ++c) {
-      float mc = m_run[c];
-#pragma unroll
-      for (int o = 4; o <= 16; o <<= 1) mc = fmaxf(mc, __shfl_xor_sync(dev::kFull, mc, o));
-      l_run[c] *= ex2(m_run[c] - (mc == -INFINITY ? 0.f : mc));
-      m_run[c] = mc;
 #pragma unroll
       for (int o = 4; o <= 16; o <<= 1) l_run[c] += __shfl_xor_sync(dev::kFull, l_run[c], o);
+      if (M_run[c] == -FLT_MAX) M_run[c] = -INFINITY;
+      m_run[c] = M_run[c];
     }
     if constexpr (PACK) {
 #pragma unroll
