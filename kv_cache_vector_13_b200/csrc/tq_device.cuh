@@ -64,6 +64,45 @@ __device__ __forceinline__ void load_block(const void *p, float (&v)[E]) {
   }
 }
 
+// ------------------------------------------------- paired fp32 arithmetic
+
+// Two independent fp32 operations in one packed f32x2 instruction (sm_100).
+// Each half rounds to nearest exactly as the scalar add.rn / sub.rn / mul.rn
+// does (no flush to zero), so a paired step gives the same bits as the two
+// scalar ones -- with one exception the compiler makes: a packed product
+// whose result feeds a packed sum can be fused into a packed multiply-add,
+// which skips the product's rounding (measured on sm_100a).  So a product
+// that an addition or subtraction consumes is formed with scalar mul.rn;
+// packed products feed only comparisons, conversions and stores, or are
+// exact (scaling by a power of two).
+__device__ __forceinline__ void add_x2(float &d0, float &d1, float a0, float a1, float b0, float b1) {
+  asm("{\n .reg .b64 ra, rb, rd;\n mov.b64 ra, {%2, %3};\n mov.b64 rb, {%4, %5};\n"
+      " add.rn.f32x2 rd, ra, rb;\n mov.b64 {%0, %1}, rd;\n}\n"
+      : "=f"(d0), "=f"(d1)
+      : "f"(a0), "f"(a1), "f"(b0), "f"(b1));
+}
+__device__ __forceinline__ void sub_x2(float &d0, float &d1, float a0, float a1, float b0, float b1) {
+  asm("{\n .reg .b64 ra, rb, rd;\n mov.b64 ra, {%2, %3};\n mov.b64 rb, {%4, %5};\n"
+      " sub.rn.f32x2 rd, ra, rb;\n mov.b64 {%0, %1}, rd;\n}\n"
+      : "=f"(d0), "=f"(d1)
+      : "f"(a0), "f"(a1), "f"(b0), "f"(b1));
+}
+__device__ __forceinline__ void mul_x2(float &d0, float &d1, float a0, float a1, float b0, float b1) {
+  asm("{\n .reg .b64 ra, rb, rd;\n mov.b64 ra, {%2, %3};\n mov.b64 rb, {%4, %5};\n"
+      " mul.rn.f32x2 rd, ra, rb;\n mov.b64 {%0, %1}, rd;\n}\n"
+      : "=f"(d0), "=f"(d1)
+      : "f"(a0), "f"(a1), "f"(b0), "f"(b1));
+}
+
+// a_i <- fl(a_i * s) over an even-length array, in pairs (for products that
+// no addition consumes).
+template <int E>
+__device__ __forceinline__ void scale_x2(float (&a)[E], float s) {
+  static_assert(E % 2 == 0, "pairs");
+#pragma unroll
+  for (int i = 0; i < E; i += 2) mul_x2(a[i], a[i + 1], a[i], a[i + 1], s, s);
+}
+
 // ------------------------------------------------------------ butterflies
 
 // One cross-lane FWHT stage: the lane whose group index has bit P clear holds
@@ -72,25 +111,44 @@ __device__ __forceinline__ void load_block(const void *p, float (&v)[E]) {
 template <int E>
 __device__ __forceinline__ void fwht_cross(float (&a)[E], int P, bool low) {
   const uint32_t neg = low ? 0u : 0x80000000u;
+  if constexpr (E % 2 == 0) {
 #pragma unroll
-  for (int i = 0; i < E; ++i) {
-    const float o = __shfl_xor_sync(kFull, a[i], P);
-    a[i] = __fadd_rn(o, __uint_as_float(__float_as_uint(a[i]) ^ neg));
+    for (int i = 0; i < E; i += 2) {
+      const float o0 = __shfl_xor_sync(kFull, a[i], P), o1 = __shfl_xor_sync(kFull, a[i + 1], P);
+      add_x2(a[i], a[i + 1], o0, o1, __uint_as_float(__float_as_uint(a[i]) ^ neg),
+             __uint_as_float(__float_as_uint(a[i + 1]) ^ neg));
+    }
+  } else {
+#pragma unroll
+    for (int i = 0; i < E; ++i) {
+      const float o = __shfl_xor_sync(kFull, a[i], P);
+      a[i] = __fadd_rn(o, __uint_as_float(__float_as_uint(a[i]) ^ neg));
+    }
   }
 }
 
-// In-register FWHT stages h = E/2, ..., 1.
+// In-register FWHT stages h = E/2, ..., 1.  Stages h >= 2 take the
+// butterflies of elements i and i + 1 together (paired instructions); the
+// last stage pairs the two halves of a pair and stays scalar.
 template <int E>
 __device__ __forceinline__ void fwht_local(float (&a)[E]) {
 #pragma unroll
-  for (int h = E / 2; h >= 1; h >>= 1) {
+  for (int h = E / 2; h >= 2; h >>= 1) {
 #pragma unroll
-    for (int i = 0; i < E; ++i) {
+    for (int i = 0; i < E; i += 2) {
       if ((i & h) == 0) {
-        const float x = a[i], y = a[i + h];
-        a[i] = __fadd_rn(x, y);
-        a[i + h] = __fsub_rn(x, y);
+        const float x0 = a[i], x1 = a[i + 1], y0 = a[i + h], y1 = a[i + h + 1];
+        add_x2(a[i], a[i + 1], x0, x1, y0, y1);
+        sub_x2(a[i + h], a[i + h + 1], x0, x1, y0, y1);
       }
+    }
+  }
+  if constexpr (E >= 2) {
+#pragma unroll
+    for (int i = 0; i < E; i += 2) {
+      const float x = a[i], y = a[i + 1];
+      a[i] = __fadd_rn(x, y);
+      a[i + 1] = __fsub_rn(x, y);
     }
   }
 }
@@ -108,17 +166,34 @@ __device__ __forceinline__ void fwht(float (&a)[E], int t) {
 // returns the same value (fl(x+y) = fl(y+x)).
 template <int T, int E>
 __device__ __forceinline__ float fold_halves_sum(float (&a)[E]) {
+  if constexpr (E % 2 == 0) {
 #pragma unroll
-  for (int P = T / 2; P >= 1; P >>= 1) {
+    for (int P = T / 2; P >= 1; P >>= 1) {
 #pragma unroll
-    for (int i = 0; i < E; ++i) a[i] = __fadd_rn(a[i], __shfl_xor_sync(kFull, a[i], P));
+      for (int i = 0; i < E; i += 2) {
+        const float o0 = __shfl_xor_sync(kFull, a[i], P), o1 = __shfl_xor_sync(kFull, a[i + 1], P);
+        add_x2(a[i], a[i + 1], a[i], a[i + 1], o0, o1);
+      }
+    }
+#pragma unroll
+    for (int h = E / 2; h >= 2; h >>= 1) {
+#pragma unroll
+      for (int i = 0; i < h; i += 2) add_x2(a[i], a[i + 1], a[i], a[i + 1], a[i + h], a[i + h + 1]);
+    }
+    return __fadd_rn(a[0], a[1]);
+  } else {
+#pragma unroll
+    for (int P = T / 2; P >= 1; P >>= 1) {
+#pragma unroll
+      for (int i = 0; i < E; ++i) a[i] = __fadd_rn(a[i], __shfl_xor_sync(kFull, a[i], P));
+    }
+#pragma unroll
+    for (int h = E / 2; h >= 1; h >>= 1) {
+#pragma unroll
+      for (int i = 0; i < h; ++i) a[i] = __fadd_rn(a[i], a[i + h]);
+    }
+    return a[0];
   }
-#pragma unroll
-  for (int h = E / 2; h >= 1; h >>= 1) {
-#pragma unroll
-    for (int i = 0; i < h; ++i) a[i] = __fadd_rn(a[i], a[i + h]);
-  }
-  return a[0];
 }
 
 // The same fold-halves sum of the squares fl(a_i * a_i), without a second
@@ -139,9 +214,37 @@ __device__ __forceinline__ float fold_sumsq_node(const float (&a)[E]) {
   }
 }
 
+// The same recursion on the pairs (W(I, H), W(I + 1, H)) for even I and
+// H >= 2, one paired instruction per step.
+template <int T, int E, int I, int H>
+__device__ __forceinline__ void fold_sumsq_node2(const float (&a)[E], float &w0, float &w1) {
+  if constexpr (H == E) {
+    // scalar squares: a packed product whose one use is a packed sum may be
+    // fused into it, which would skip the product's rounding
+    w0 = __fmul_rn(a[I], a[I]);
+    w1 = __fmul_rn(a[I + 1], a[I + 1]);
+#pragma unroll
+    for (int P = T / 2; P >= 1; P >>= 1) {
+      const float o0 = __shfl_xor_sync(kFull, w0, P), o1 = __shfl_xor_sync(kFull, w1, P);
+      add_x2(w0, w1, w0, w1, o0, o1);
+    }
+  } else {
+    float l0, l1, h0, h1;
+    fold_sumsq_node2<T, E, I, 2 * H>(a, l0, l1);
+    fold_sumsq_node2<T, E, I + H, 2 * H>(a, h0, h1);
+    add_x2(w0, w1, l0, l1, h0, h1);
+  }
+}
+
 template <int T, int E>
 __device__ __forceinline__ float fold_halves_sumsq(const float (&a)[E]) {
-  return fold_sumsq_node<T, E, 0, 1>(a);
+  if constexpr (E % 2 == 0) {
+    float w0, w1;
+    fold_sumsq_node2<T, E, 0, 2>(a, w0, w1);
+    return __fadd_rn(w0, w1);
+  } else {
+    return fold_sumsq_node<T, E, 0, 1>(a);
+  }
 }
 
 // ------------------------------------------------------- index splitting

@@ -149,10 +149,7 @@ __device__ __forceinline__ float encode_front(const EncParams &p, int64_t xoff, 
   dev::load_block<DT, E>(static_cast<const char *>(p.x) + xoff * ES, a);
 
   // norm: fold-halves sum of squares, then sqrt_rn
-  float sq[E];
-#pragma unroll
-  for (int i = 0; i < E; ++i) sq[i] = __fmul_rn(a[i], a[i]);
-  const float nrm = __fsqrt_rn(dev::fold_halves_sum<T, E>(sq));
+  const float nrm = __fsqrt_rn(dev::fold_halves_sumsq<T, E>(a));
 
   // rotate: sign flips, then the unnormalised FWHT
   uint32_t sw[(E + 31) / 32];
@@ -166,23 +163,32 @@ __device__ __forceinline__ float encode_front(const EncParams &p, int64_t xoff, 
   // scale to the unit sphere: u = y * fl(1 / fl(n * fl(sqrt d)))
   const float wsc = __fmul_rn(nrm, p.sqrt_d);
   const float inv = wsc > 0.0f ? __frcp_rn(wsc) : 0.0f;
+  if constexpr (PROD) {
+    // the residual subtracts from these products: scalar, so that no
+    // product is fused into the subtraction
 #pragma unroll
-  for (int i = 0; i < E; ++i) a[i] = __fmul_rn(a[i], inv);
+    for (int i = 0; i < E; ++i) a[i] = __fmul_rn(a[i], inv);
+  } else {
+    dev::scale_x2<E>(a, inv);
+  }
 
   // quantize and pack; prod keeps the residual in a[]
 #pragma unroll
   for (int w = 0; w < NWC; ++w) W[w] = 0u;
   if constexpr (BM > 0) {
 #pragma unroll
-    for (int i = 0; i < E; ++i) {
-      int idx;
-      if constexpr (BM == 1) {
-        idx = a[i] > 0.0f ? 1 : 0;
-      } else {
-        idx = dev::quantize_sym<BM>(a[i], P);
+    for (int i = 0; i < E; i += 2) {
+      int idx[2];
+#pragma unroll
+      for (int j = 0; j < 2; ++j) {
+        if constexpr (BM == 1) {
+          idx[j] = a[i + j] > 0.0f ? 1 : 0;
+        } else {
+          idx[j] = dev::quantize_sym<BM>(a[i + j], P);
+        }
+        dev::put_field<BM>(W, i + j, (uint32_t)idx[j]);
       }
-      dev::put_field<BM>(W, i, (uint32_t)idx);
-      if constexpr (PROD) a[i] = __fsub_rn(a[i], s_cent[idx]);
+      if constexpr (PROD) dev::sub_x2(a[i], a[i + 1], a[i], a[i + 1], s_cent[idx[0]], s_cent[idx[1]]);
     }
   }
   return nrm;
@@ -239,10 +245,7 @@ __global__ void __launch_bounds__(kEncThreads, EE == 64 ? 3 : 1) encode_kernel(E
   if (active && t == 0) p.norms[rec] = nrm;
 
   if constexpr (PROD) {
-    float rr[E];
-#pragma unroll
-    for (int i = 0; i < E; ++i) rr[i] = __fmul_rn(a[i], a[i]);
-    const float gam = __fsqrt_rn(dev::fold_halves_sum<T, E>(rr));
+    const float gam = __fsqrt_rn(dev::fold_halves_sumsq<T, E>(a));
     // z_k = sum_i S[k][i] r_i for this lane's k-block, fp32
     float *rv = s_r + (size_t)vl * RS;
 #pragma unroll
@@ -337,7 +340,9 @@ __device__ __forceinline__ void split8(const float (&x)[8], uint4 &H, uint4 &L) 
   for (int i = 0; i < 4; ++i) {
     h[i] = pack_h2(x[2 * i], x[2 * i + 1]);
     const float2 f = __half22float2(*reinterpret_cast<const __half2 *>(&h[i]));
-    l[i] = pack_h2(x[2 * i] - f.x, x[2 * i + 1] - f.y);
+    float d0, d1;
+    dev::sub_x2(d0, d1, x[2 * i], x[2 * i + 1], f.x, f.y);
+    l[i] = pack_h2(d0, d1);
   }
   H = make_uint4(h[0], h[1], h[2], h[3]);
   L = make_uint4(l[0], l[1], l[2], l[3]);
@@ -654,7 +659,8 @@ __global__ void __launch_bounds__(kPtThreads, 1) encode_prod_tc_kernel(EncParams
       for (int c = 0; c < E / 8; ++c) {
         float x[8];
 #pragma unroll
-        for (int i = 0; i < 8; ++i) x[i] = a[8 * c + i] * sc;
+        for (int i = 0; i < 8; i += 2)  // sc is a power of two: exact products
+          dev::mul_x2(x[i], x[i + 1], a[8 * c + i], a[8 * c + i + 1], sc, sc);
         uint4 H, L;
         split8(x, H, L);
         const uint32_t o = umma::off(vl, t * E + 8 * c, kPtSbo, kPtLbo);
