@@ -262,7 +262,9 @@ __device__ __forceinline__ uint32_t pack_half2(float lo, float hi) {
 __device__ __forceinline__ void split_pair(float a, float b, uint32_t &hi, uint32_t &lo) {
   hi = pack_half2(a, b);
   const float2 f = __half22float2(*reinterpret_cast<const __half2 *>(&hi));
-  lo = pack_half2(a - f.x, b - f.y);
+  float d0, d1;
+  dev::sub_x2(d0, d1, a, b, f.x, f.y);
+  lo = pack_half2(d0, d1);
 }
 
 // hi = fp16(x), lo = fp16(x - hi): x to ~22 significant bits
@@ -1162,15 +1164,17 @@ __global__ void __launch_bounds__(split_warps<PACK, KPROD, STAGED>() * 32, 1) de
           const int h = PACK ? 2 * (tig & 1) + c : 2 * tig + c;  // this lane's head columns
           const float ch = h < gh ? __uint_as_float(__ldg(fw + (15 * 32 + h) * 4 + 0)) : 0.f;
           const float th = h < gh ? __uint_as_float(__ldg(fw + (15 * 32 + h) * 4 + 1)) : 0.f;
-          // the MMAs sum -bit * digit: <S q', 2 bit - 1> = -2 c_h (256 hi + lo) - T_h
+          // the MMAs sum -bit * digit: <S q', 2 bit - 1> = -2 c_h (256 hi + lo) - T_h,
+          // scaled by kappa s_K (the estimator's sqrt(pi/2)/d; the table holds s_K c)
+          const float ks = kKappa * sK;
           if constexpr (PACK) {  // lanes tig < 2 hold the hi digits' columns, the others the lo digits'
-            qd[c][0] = -2.f * ch * (tig < 2 ? 256.f : 1.f);
+            qd[c][0] = -2.f * ch * (tig < 2 ? 256.f : 1.f) * ks;
             qd[c][1] = 0.f;
-            qd[c][2] = tig < 2 ? -th : 0.f;
+            qd[c][2] = tig < 2 ? -th * ks : 0.f;
           } else {
-            qd[c][0] = -512.f * ch;
-            qd[c][1] = -2.f * ch;
-            qd[c][2] = -th;
+            qd[c][0] = -512.f * ch * ks;
+            qd[c][1] = -2.f * ch * ks;
+            qd[c][2] = -th * ks;
           }
         }
       }
@@ -1267,7 +1271,7 @@ __global__ void __launch_bounds__(split_warps<PACK, KPROD, STAGED>() * 32, 1) de
         for (int r = 0; r < 2; ++r) {
           ok[r] = kb.kn[ms][r] >= 0.f;
           fs[r] = kb.kn[ms][r] * kscale;
-          kr[r] = KPROD ? kb.kr[ms][r] * (kKappa * sK) : 0.f;  // the table holds s_K c
+          kr[r] = KPROD ? kb.kr[ms][r] : 0.f;
           // (staged masked rows hold whatever the slot holds: kept finite)
           nvl[ms][r] = (STAGED && !ok[r]) ? 0.f : __log2f(kb.vn[ms][r]);
         }
@@ -1327,24 +1331,33 @@ __global__ void __launch_bounds__(split_warps<PACK, KPROD, STAGED>() * 32, 1) de
   }
           TQ_QSTEP(0) TQ_QSTEP(1) TQ_QSTEP(2) TQ_QSTEP(3)
 #undef TQ_QSTEP
+          // the two head columns of a row as one pair
 #pragma unroll
-          for (int i = 0; i < 4; ++i) {
-            const int c = i & 1;
-            cq[i] = fmaf((float)ch[i], qd[c][0], PACK ? qd[c][2] : fmaf((float)cl[i], qd[c][1], qd[c][2]));
+          for (int r = 0; r < 2; ++r) {
+            float b0 = qd[0][2], b1 = qd[1][2];
+            if constexpr (!PACK)
+              dev::fma_x2(b0, b1, (float)cl[2 * r], (float)cl[2 * r + 1], qd[0][1], qd[1][1], b0, b1);
+            dev::fma_x2(cq[2 * r], cq[2 * r + 1], (float)ch[2 * r], (float)ch[2 * r + 1], qd[0][0], qd[1][0], b0, b1);
           }
         }
-        // raw score = main + kappa gamma s_K qjl (the table holds s_K c)
+        // raw score = main + kappa gamma s_K qjl (the table holds s_K c; kappa
+        // s_K is folded into qd)
 #pragma unroll
-        for (int i = 0; i < 4; ++i) {
-          float s = cm[i];
-          if constexpr (KPROD) s = fmaf(kr[i >> 1], cq[i], s);
-          if constexpr (PACK) s += __shfl_xor_sync(dev::kFull, s, 2);  // hi + lo columns
-          cm[i] = s;
+        for (int r = 0; r < 2; ++r) {
+          if constexpr (KPROD)
+            dev::fma_x2(cm[2 * r], cm[2 * r + 1], kr[r], kr[r], cq[2 * r], cq[2 * r + 1], cm[2 * r], cm[2 * r + 1]);
+          if constexpr (PACK) {  // hi + lo columns
+            const float o0 = __shfl_xor_sync(dev::kFull, cm[2 * r], 2);
+            const float o1 = __shfl_xor_sync(dev::kFull, cm[2 * r + 1], 2);
+            dev::add_x2(cm[2 * r], cm[2 * r + 1], cm[2 * r], cm[2 * r + 1], o0, o1);
+          }
         }
 #pragma unroll
         for (int r = 0; r < 2; ++r) {
-#pragma unroll
-          for (int c = 0; c < 2; ++c) sc[ms][2 * r + c] = ok[r] ? cm[2 * r + c] * fs[r] : -INFINITY;
+          float t0, t1;
+          dev::mul_x2(t0, t1, cm[2 * r], cm[2 * r + 1], fs[r], fs[r]);
+          sc[ms][2 * r] = ok[r] ? t0 : -INFINITY;
+          sc[ms][2 * r + 1] = ok[r] ? t1 : -INFINITY;
         }
         if (want_scores) {
 #pragma unroll
@@ -1381,15 +1394,19 @@ __global__ void __launch_bounds__(split_warps<PACK, KPROD, STAGED>() * 32, 1) de
       // accumulators only then (warp-uniform branch)
       float wgt[2][4];
       float Mx[2];
-#pragma unroll
-      for (int c = 0; c < 2; ++c) {
-        float u[4];
+      {
+        // u[row][c], the two columns of a row as one pair
+        float u[4][2];
 #pragma unroll
         for (int ms = 0; ms < 2; ++ms) {
 #pragma unroll
-          for (int r = 0; r < 2; ++r) u[2 * ms + r] = sc[ms][2 * r + c] + fmaxf(nvl[ms][r], kNvlFloor);
+          for (int r = 0; r < 2; ++r) {
+            const float nf = fmaxf(nvl[ms][r], kNvlFloor);
+            dev::add_x2(u[2 * ms + r][0], u[2 * ms + r][1], sc[ms][2 * r], sc[ms][2 * r + 1], nf, nf);
+          }
         }
-        Mx[c] = fmaxf(fmaxf(u[0], u[1]), fmaxf(u[2], u[3]));
+#pragma unroll
+        for (int c = 0; c < 2; ++c) Mx[c] = fmaxf(fmaxf(u[0][c], u[1][c]), fmaxf(u[2][c], u[3][c]));
       }
       if (__any_sync(dev::kFull, Mx[0] > M_thr[0] || Mx[1] > M_thr[1])) {
         float aM[2];
@@ -1412,19 +1429,21 @@ __global__ void __launch_bounds__(split_warps<PACK, KPROD, STAGED>() * 32, 1) de
           acc[mt][3] *= aM[1];
         }
       }
-#pragma unroll
-      for (int c = 0; c < 2; ++c) {
-        float ls = 0.f;
+      {
+        float ls0 = 0.f, ls1 = 0.f;
 #pragma unroll
         for (int ms = 0; ms < 2; ++ms) {
 #pragma unroll
           for (int r = 0; r < 2; ++r) {
-            const float e = sc[ms][2 * r + c] - M_run[c];
-            ls += ex2(e);
-            wgt[ms][2 * r + c] = ex2(e + nvl[ms][r]);
+            float e0, e1, w0, w1;
+            dev::sub_x2(e0, e1, sc[ms][2 * r], sc[ms][2 * r + 1], M_run[0], M_run[1]);
+            dev::add_x2(ls0, ls1, ls0, ls1, ex2(e0), ex2(e1));
+            dev::add_x2(w0, w1, e0, e1, nvl[ms][r], nvl[ms][r]);
+            wgt[ms][2 * r] = ex2(w0);
+            wgt[ms][2 * r + 1] = ex2(w1);
           }
         }
-        l_run[c] += ls;
+        dev::add_x2(l_run[0], l_run[1], l_run[0], l_run[1], ls0, ls1);
       }
 
       // -------- PV: for each 16-token half, B = W^T via movmatrix

@@ -94,6 +94,15 @@ __device__ __forceinline__ void mul_x2(float &d0, float &d1, float a0, float a1,
       : "f"(a0), "f"(a1), "f"(b0), "f"(b1));
 }
 
+// d = a * b + c, each half one fused multiply-add (rounded once).
+__device__ __forceinline__ void fma_x2(float &d0, float &d1, float a0, float a1, float b0, float b1, float c0,
+                                       float c1) {
+  asm("{\n .reg .b64 ra, rb, rc, rd;\n mov.b64 ra, {%2, %3};\n mov.b64 rb, {%4, %5};\n"
+      " mov.b64 rc, {%6, %7};\n fma.rn.f32x2 rd, ra, rb, rc;\n mov.b64 {%0, %1}, rd;\n}\n"
+      : "=f"(d0), "=f"(d1)
+      : "f"(a0), "f"(a1), "f"(b0), "f"(b1), "f"(c0), "f"(c1));
+}
+
 // a_i <- fl(a_i * s) over an even-length array, in pairs (for products that
 // no addition consumes).
 template <int E>
