@@ -15,11 +15,13 @@
 // Flash-decoding split over the sequence:
 //   general_partial_kernel, grid (splits, B * Hkv * head groups): up to 8
 //     query heads of one kv head over one token slice, in tiles of 64
-//     tokens: scores (4 threads a token), an online softmax per head, then
-//     the values 8 tokens at a time: each (token, coordinate) decoded once
-//     into shared memory, and a thread per (head, coordinate) accumulating
-//     the weighted centroids (and, for prod values, the weighted signs); the
-//     slice's (m, l, o', signs) go to a workspace slot;
+//     tokens: the tile's records and norms staged in shared memory with
+//     coalesced copies, scores (4 threads a token, q' and S q' read
+//     coordinate-major, all heads of a coordinate in one vector load), an
+//     online softmax per head, then the values: a thread per coordinate (and
+//     token class when d <= 128) accumulating every head's weighted
+//     centroids (and, for prod values, weighted signs); the slice's (m, l,
+//     o', signs) go to a workspace slot;
 //   general_merge_kernel, a block per (batch, query head): merges the slots,
 //   adds S_g^T of the sign sums, applies each group's inverse rotation and
 //   1/l, and scatters the groups into their channels.
@@ -35,7 +37,7 @@ constexpr int kGnThreads = 256;
 constexpr int kGnMaxD = 256;
 constexpr int kGnHeads = 8;   // query heads a block
 constexpr int kGnTile = 64;   // tokens a tile
-constexpr int kGnSub = 8;     // tokens a value-decode step
+constexpr int kGnMaxSplits = 64;  // sequence splits at most
 constexpr float kGnLog2e = 1.4426950408889634f;
 constexpr float kGnSqrtHalfPi = 1.2533141373155003f;
 
@@ -78,17 +80,6 @@ __device__ __forceinline__ float gn_q(const GnParams &p, int64_t i) {
   return p.q_dtype == TQ_BF16 ? __uint_as_float((uint32_t)h << 16) : __half2float(__ushort_as_half(h));
 }
 
-// Index i of a record's LSB-first bm-bit stream (bm <= 4: at most two bytes).
-__device__ __forceinline__ int gn_field(const uint8_t *rec, int i, int bm, int nbytes) {
-  const int q = i * bm;
-  const int by = q >> 3, sh = q & 7;
-  uint32_t w = __ldg(rec + by);
-  if (sh + bm > 8 && by + 1 < nbytes) w |= (uint32_t)__ldg(rec + by + 1) << 8;
-  return (int)((w >> sh) & ((1u << bm) - 1u));
-}
-
-__device__ __forceinline__ bool gn_bit(const uint8_t *rec, int i) { return (__ldg(rec + (i >> 3)) >> (i & 7)) & 1; }
-
 __device__ __forceinline__ float gn_ex2(float x) {
   float y;
   asm("ex2.approx.ftz.f32 %0, %1;\n" : "=f"(y) : "f"(x));
@@ -112,16 +103,102 @@ __device__ void gn_fwht(float *x, int nv, int d, int stride) {
   __syncthreads();
 }
 
+// Field i of an LSB-first bm-bit stream of nbytes bytes in shared memory.
+__device__ __forceinline__ int gn_field_s(const uint8_t *rec, int i, int bm, int nbytes) {
+  const int q = i * bm;
+  const int by = q >> 3, sh = q & 7;
+  uint32_t w = rec[by];
+  if (sh + bm > 8 && by + 1 < nbytes) w |= (uint32_t)rec[by + 1] << 8;
+  return (int)((w >> sh) & ((1u << bm) - 1u));
+}
+
+// Copies nbytes-byte records rec0, rec0 + sn, ... (nt of them) of src into
+// dst, token-major; 32-bit words when the records are contiguous and word
+// sized (the cache arrays are 16-byte aligned), else bytes.  The whole block
+// takes part.
+__device__ __forceinline__ void gn_stage(const uint8_t *src, int64_t rec0, int64_t sn, int nbytes, int nt,
+                                         uint8_t *dst) {
+  if (sn == 1 && (nbytes & 3) == 0) {
+    const uint32_t *s4 = reinterpret_cast<const uint32_t *>(src + rec0 * nbytes);
+    uint32_t *d4 = reinterpret_cast<uint32_t *>(dst);
+    const int nw = nt * (nbytes >> 2);
+    for (int e = threadIdx.x; e < nw; e += kGnThreads) d4[e] = __ldg(s4 + e);
+  } else {
+    const int nb = nt * nbytes;
+    for (int e = threadIdx.x; e < nb; e += kGnThreads) {
+      const int tt = e / nbytes, by = e - tt * nbytes;
+      dst[e] = __ldg(src + (rec0 + tt * sn) * nbytes + by);
+    }
+  }
+}
+
+// Staging capacity of one side's tile: codes (at most 4 bits a coordinate)
+// and QJL signs of kGnTile tokens.
+constexpr int kGnCodeBytes = kGnTile * kGnMaxD / 2;
+constexpr int kGnSignBytes = kGnTile * kGnMaxD / 8;
+constexpr int kGnStageBytes = 2 * (kGnCodeBytes + kGnSignBytes);
+
+// Loads of the query fragments by head count: NH consecutive floats.
+template <int NH>
+__device__ __forceinline__ void gn_ld_heads(const float *src, float (&v)[NH]) {
+  if constexpr (NH % 4 == 0) {
+#pragma unroll
+    for (int k = 0; k < NH / 4; ++k) {
+      const float4 t = reinterpret_cast<const float4 *>(src)[k];
+      v[4 * k] = t.x, v[4 * k + 1] = t.y, v[4 * k + 2] = t.z, v[4 * k + 3] = t.w;
+    }
+  } else if constexpr (NH == 2) {
+    const float2 t = *reinterpret_cast<const float2 *>(src);
+    v[0] = t.x, v[1] = t.y;
+  } else {
+    v[0] = src[0];
+  }
+}
+
+// y_h = A x_h for the block's heads h < nh: A is n x n row-major in global
+// memory, x_h and y_h rows of shared memory kGnMaxD floats apart.  A warp
+// takes a row, its lanes read consecutive columns (coalesced) and sum across
+// the warp; the whole block takes part.
+template <int NH>
+__device__ __forceinline__ void gn_rows_times(const float *A, int n, const float *x, float *y, int nh) {
+  const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5;
+  for (int r = warp; r < n; r += kGnThreads / 32) {
+    const float *row = A + (int64_t)r * n;
+    float acc[NH];
+#pragma unroll
+    for (int hh = 0; hh < NH; ++hh) acc[hh] = 0.f;
+    for (int c = lane; c < n; c += 32) {
+      const float a = __ldg(row + c);
+#pragma unroll
+      for (int hh = 0; hh < NH; ++hh)
+        if (hh < nh) acc[hh] = fmaf(a, x[hh * kGnMaxD + c], acc[hh]);
+    }
+#pragma unroll
+    for (int hh = 0; hh < NH; ++hh) {
+#pragma unroll
+      for (int o = 16; o >= 1; o >>= 1) acc[hh] += __shfl_xor_sync(dev::kFull, acc[hh], o);
+      if (lane == 0 && hh < nh) y[hh * kGnMaxD + r] = acc[hh];
+    }
+  }
+}
+
 // NH: the most query heads a block handles (1, 2, 4 or 8): the per-token
 // head loops are unrolled to it.
 template <int NH>
 __global__ void __launch_bounds__(kGnThreads) general_partial_kernel(GnParams p) {
-  __shared__ float s_q[kGnHeads][kGnMaxD];   // q'_g at the group's offset
-  __shared__ float s_qs[kGnHeads][kGnMaxD];  // S_g q'_g (prod groups); staging of q[channels] first
-  __shared__ float s_w[kGnHeads][kGnTile];   // logits, then weights
-  __shared__ float s_vn[2][kGnTile], s_vr[2][kGnTile];
+  // setup: q'_g and S_g q'_g by head ([8][kGnMaxD] each); tiles: the staged
+  // records, K codes | K signs | V codes | V signs; end: the halves' sums
+  __shared__ __align__(16) unsigned char s_raw[kGnStageBytes];
+  __shared__ __align__(16) float s_qT[kGnMaxD][NH];   // q'_g, coordinate-major
+  __shared__ __align__(16) float s_qsT[kGnMaxD][NH];  // S_g q'_g (prod key groups)
+  __shared__ float s_w[kGnHeads][kGnTile];            // logits
+  __shared__ __align__(16) float s_wT[kGnTile][NH];   // weights, token-major
+  __shared__ float s_kn[2][kGnTile], s_kr[2][kGnTile], s_vn[2][kGnTile], s_vr[2][kGnTile];
+  __shared__ float s_cent[2][2][16];  // [K / V][group]
   __shared__ float s_alpha[kGnHeads], s_m[kGnHeads], s_l[kGnHeads];
-  __shared__ float s_vx[2][kGnSub][kGnMaxD];  // decoded values (and prod sign terms)
+  float(*s_q)[kGnMaxD] = reinterpret_cast<float(*)[kGnMaxD]>(s_raw);
+  float(*s_qs)[kGnMaxD] = reinterpret_cast<float(*)[kGnMaxD]>(s_raw + kGnHeads * kGnMaxD * 4);
+  static_assert(2 * kGnHeads * kGnMaxD * 4 <= kGnStageBytes, "setup scratch");
   const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
   const int d = p.d;
   const int split = blockIdx.x;
@@ -134,6 +211,12 @@ __global__ void __launch_bounds__(kGnThreads) general_partial_kernel(GnParams p)
   const int64_t t0 = (int64_t)split * p.per_split;
   const int64_t t1 = min(L, t0 + p.per_split);
 
+  if (tid < 64) {  // the codebooks
+    const int side = tid >> 5, gr = (tid >> 4) & 1, c = tid & 15;
+    const GnGroup &G = side ? p.v[gr] : p.k[gr];
+    const int ng = side ? p.nv : p.nk;
+    s_cent[side][gr][c] = (gr < ng && G.bm > 0 && c < (1 << G.bm)) ? __ldg(G.cent + c) : 0.f;
+  }
   // ---- q'_g = Pi_g q[channels_g] for the block's heads (and S_g q'_g)
   for (int gr = 0; gr < p.nk; ++gr) {
     const GnGroup &G = p.k[gr];
@@ -152,13 +235,7 @@ __global__ void __launch_bounds__(kGnThreads) general_partial_kernel(GnParams p)
   for (int gr = 0; gr < p.nk; ++gr) {
     const GnGroup &G = p.k[gr];
     if (G.rot) {
-      for (int e = tid; e < nh * G.d; e += kGnThreads) {
-        const int hh = e / G.d, r = e % G.d;
-        const float *row = G.rot + (int64_t)r * G.d;
-        float acc = 0.f;
-        for (int c = 0; c < G.d; ++c) acc = fmaf(__ldg(row + c), s_qs[hh][G.off + c], acc);
-        s_q[hh][G.off + r] = acc;
-      }
+      gn_rows_times<NH>(G.rot, G.d, &s_qs[0][G.off], &s_q[0][G.off], nh);
     } else {  // Hadamard: a single group at offset 0
       gn_fwht(&s_q[0][0], nh, G.d, kGnMaxD);
       const float inv = rsqrtf((float)G.d);
@@ -168,14 +245,7 @@ __global__ void __launch_bounds__(kGnThreads) general_partial_kernel(GnParams p)
   __syncthreads();
   for (int gr = 0; gr < p.nk; ++gr) {
     const GnGroup &G = p.k[gr];
-    if (!G.prod) continue;
-    for (int e = tid; e < nh * G.d; e += kGnThreads) {
-      const int hh = e / G.d, r = e % G.d;
-      const float *row = G.S + (int64_t)r * G.d;
-      float acc = 0.f;
-      for (int c = 0; c < G.d; ++c) acc = fmaf(__ldg(row + c), s_q[hh][G.off + c], acc);
-      s_qs[hh][G.off + r] = acc;
-    }
+    if (G.prod) gn_rows_times<NH>(G.S, G.d, &s_q[0][G.off], &s_qs[0][G.off], nh);
   }
   if (tid < kGnHeads) {
     s_m[tid] = -INFINITY;
@@ -183,27 +253,81 @@ __global__ void __launch_bounds__(kGnThreads) general_partial_kernel(GnParams p)
   }
   __syncthreads();
 
-  // this thread's (head, coordinate) pairs: e = tid + kGnThreads * c
-  constexpr int kCoords = NH * kGnMaxD / kGnThreads > 0 ? NH * kGnMaxD / kGnThreads : 1;
-  float acc[kCoords], sacc[kCoords];
-  int c_h[kCoords], c_i[kCoords];
-  bool c_prod[kCoords];
-#pragma unroll
-  for (int c = 0; c < kCoords; ++c) {
-    acc[c] = sacc[c] = 0.f;
-    const int e = tid + kGnThreads * c;
-    c_h[c] = e < nh * d ? e / d : -1;
-    c_i[c] = e % d;
-    c_prod[c] = p.v[(p.nv == 2 && c_i[c] >= p.v[1].off) ? 1 : 0].prod;
+  if (tid < kGnHeads) s_alpha[tid] = 1.f;
+  // coordinate-major copies of q' and S q' (zero for absent heads)
+  for (int e = tid; e < kGnMaxD * NH; e += kGnThreads) {
+    const int i = e / NH, hh = e - i * NH;
+    const bool live = hh < nh && i < d;
+    s_qT[i][hh] = live ? s_q[hh][i] : 0.f;
+    s_qsT[i][hh] = live ? s_qs[hh][i] : 0.f;
   }
-  // the value decode's (token, coordinate) share: coordinate dec_i of
-  // tokens dec_t, dec_t + dec_step, ...
-  const int dec_step = kGnThreads / d;
-  const int dec_i = tid < dec_step * d ? tid % d : -1;
-  const int dec_t = tid / d;
+  __syncthreads();
+
+  // staged-record offsets in s_raw: K codes | K signs | V codes | V signs,
+  // each side's groups one after the other (a tile of a group is a
+  // multiple of 64 bytes, so every part stays 16-byte aligned)
+  int kc_off[2] = {0, 0}, kj_off[2] = {0, 0}, vc_off[2] = {0, 0}, vj_off[2] = {0, 0};
+  {
+    int oc = 0, oj = kGnCodeBytes;
+    for (int gr = 0; gr < p.nk; ++gr) {
+      kc_off[gr] = oc;
+      kj_off[gr] = oj;
+      oc += kGnTile * (p.k[gr].d * p.k[gr].bm / 8);
+      oj += kGnTile * (p.k[gr].d / 8);
+    }
+    oc = kGnCodeBytes + kGnSignBytes;
+    oj = 2 * kGnCodeBytes + kGnSignBytes;
+    for (int gr = 0; gr < p.nv; ++gr) {
+      vc_off[gr] = oc;
+      vj_off[gr] = oj;
+      oc += kGnTile * (p.v[gr].d * p.v[gr].bm / 8);
+      oj += kGnTile * (p.v[gr].d / 8);
+    }
+  }
+
+  // value threads: coordinate vi of the tokens tt = half (mod nhalf)
+  const int nhalf = d >= kGnThreads ? 1 : kGnThreads / d;
+  const int half = tid / d, vi = tid - half * d;
+  const bool vact = half < nhalf;
+  const int gv = (p.nv == 2 && vi >= p.v[1].off) ? 1 : 0;
+  const int li = vi - p.v[gv].off;
+  float acc[NH], sacc[NH];
+#pragma unroll
+  for (int hh = 0; hh < NH; ++hh) acc[hh] = sacc[hh] = 0.f;
 
   for (int64_t base = t0; base < t1; base += kGnTile) {
     const int nt = (int)min((int64_t)kGnTile, t1 - base);
+    // ---- stage the tile's records and norms
+    for (int gr = 0; gr < p.nk; ++gr) {
+      const GnGroup &G = p.k[gr];
+      const int64_t rec0 = (int64_t)b * G.sb + (int64_t)kvh * G.sh + base * G.sn;
+      if (G.bm > 0) gn_stage(G.codes, rec0, G.sn, G.d * G.bm / 8, nt, s_raw + kc_off[gr]);
+      if (G.prod) gn_stage(G.qjl, rec0, G.sn, G.d / 8, nt, s_raw + kj_off[gr]);
+    }
+    for (int gr = 0; gr < p.nv; ++gr) {
+      const GnGroup &G = p.v[gr];
+      const int64_t rec0 = (int64_t)b * G.sb + (int64_t)kvh * G.sh + base * G.sn;
+      if (G.bm > 0) gn_stage(G.codes, rec0, G.sn, G.d * G.bm / 8, nt, s_raw + vc_off[gr]);
+      if (G.prod) gn_stage(G.qjl, rec0, G.sn, G.d / 8, nt, s_raw + vj_off[gr]);
+    }
+    for (int e = tid; e < 4 * kGnTile; e += kGnThreads) {  // (side, group, token)
+      const int side = e / (2 * kGnTile), gr = (e / kGnTile) & 1, tt = e % kGnTile;
+      const GnGroup &G = side ? p.v[gr] : p.k[gr];
+      if (gr < (side ? p.nv : p.nk) && tt < nt) {
+        const int64_t r = (int64_t)b * G.sb + (int64_t)kvh * G.sh + (base + tt) * G.sn;
+        const float n = __ldg(G.norms + r);
+        const float kr = G.prod ? __ldg(G.rnorms + r) * (kGnSqrtHalfPi / (float)G.d) : 0.f;
+        if (side) {
+          s_vn[gr][tt] = n;
+          s_vr[gr][tt] = kr;
+        } else {
+          s_kn[gr][tt] = n;
+          s_kr[gr][tt] = kr;
+        }
+      }
+    }
+    __syncthreads();
+
     // ---- scores: 4 threads a token, a quarter of every group's coordinates each
     {
       const int tt = tid >> 2, qq = tid & 3;
@@ -215,30 +339,28 @@ __global__ void __launch_bounds__(kGnThreads) general_partial_kernel(GnParams p)
       if (ok) {
         for (int gr = 0; gr < p.nk; ++gr) {
           const GnGroup &G = p.k[gr];
-          const int64_t kr = (int64_t)b * G.sb + (int64_t)kvh * G.sh + j * G.sn;
           const int kcb = G.d * G.bm / 8;
-          const uint8_t *kc = G.bm > 0 ? G.codes + kr * kcb : nullptr;
-          const uint8_t *kj = G.prod ? G.qjl + kr * (G.d / 8) : nullptr;
+          const uint8_t *kc = s_raw + kc_off[gr] + tt * kcb;
+          const uint8_t *kj = s_raw + kj_off[gr] + tt * (G.d / 8);
           float part[NH], qpart[NH];
 #pragma unroll
           for (int hh = 0; hh < NH; ++hh) part[hh] = qpart[hh] = 0.f;
           const int i0 = qq * (G.d / 4), i1 = i0 + G.d / 4;
           for (int i = i0; i < i1; ++i) {
-            const float c = G.bm > 0 ? __ldg(G.cent + gn_field(kc, i, G.bm, kcb)) : 0.f;
-            const float sg = G.prod ? (gn_bit(kj, i) ? 1.f : -1.f) : 0.f;
+            float qv[NH];
+            gn_ld_heads<NH>(&s_qT[G.off + i][0], qv);
+            const float c = G.bm > 0 ? s_cent[0][gr][gn_field_s(kc, i, G.bm, kcb)] : 0.f;
+#pragma unroll
+            for (int hh = 0; hh < NH; ++hh) part[hh] = fmaf(c, qv[hh], part[hh]);
             if (G.prod) {
+              float sv[NH];
+              gn_ld_heads<NH>(&s_qsT[G.off + i][0], sv);
+              const float sg = ((kj[i >> 3] >> (i & 7)) & 1) ? 1.f : -1.f;
 #pragma unroll
-              for (int hh = 0; hh < NH; ++hh) {
-                part[hh] = fmaf(c, s_q[hh][G.off + i], part[hh]);
-                qpart[hh] = fmaf(sg, s_qs[hh][G.off + i], qpart[hh]);
-              }
-            } else {
-#pragma unroll
-              for (int hh = 0; hh < NH; ++hh) part[hh] = fmaf(c, s_q[hh][G.off + i], part[hh]);
+              for (int hh = 0; hh < NH; ++hh) qpart[hh] = fmaf(sg, sv[hh], qpart[hh]);
             }
           }
-          const float n = __ldg(G.norms + kr);
-          const float kap = G.prod ? __ldg(G.rnorms + kr) * (kGnSqrtHalfPi / (float)G.d) : 0.f;
+          const float n = s_kn[gr][tt], kap = s_kr[gr][tt];
 #pragma unroll
           for (int hh = 0; hh < NH; ++hh) tot[hh] = fmaf(n, fmaf(kap, qpart[hh], part[hh]), tot[hh]);
         }
@@ -257,15 +379,10 @@ __global__ void __launch_bounds__(kGnThreads) general_partial_kernel(GnParams p)
           }
         }
       }
-      if (qq < p.nv) {  // thread qq of the token loads value group qq's norms
-        const GnGroup &G = p.v[qq];
-        const int64_t vr = (int64_t)b * G.sb + (int64_t)kvh * G.sh + j * G.sn;
-        s_vn[qq][tt] = ok ? __ldg(G.norms + vr) : 0.f;
-        s_vr[qq][tt] = (ok && G.prod) ? __ldg(G.rnorms + vr) * (kGnSqrtHalfPi / (float)G.d) : 0.f;
-      }
     }
     __syncthreads();
-    // ---- online softmax: warp hh updates head hh
+    // ---- online softmax: warp hh updates head hh and writes its weights
+    // token-major
     if (warp < nh) {
       const float a0 = s_w[warp][lane], a1 = s_w[warp][lane + 32];
       float mx = fmaxf(a0, a1);
@@ -275,8 +392,8 @@ __global__ void __launch_bounds__(kGnThreads) general_partial_kernel(GnParams p)
       const float mn = fmaxf(mo, mx);
       const float ms = mn == -INFINITY ? 0.f : mn;
       const float w0 = gn_ex2(a0 - ms), w1 = gn_ex2(a1 - ms);
-      s_w[warp][lane] = w0;
-      s_w[warp][lane + 32] = w1;
+      s_wT[lane][warp] = w0;
+      s_wT[lane + 32][warp] = w1;
       float sum = w0 + w1;
 #pragma unroll
       for (int o = 16; o >= 1; o >>= 1) sum += __shfl_xor_sync(dev::kFull, sum, o);
@@ -286,70 +403,68 @@ __global__ void __launch_bounds__(kGnThreads) general_partial_kernel(GnParams p)
         s_l[warp] = fmaf(s_l[warp], al, sum);
         s_m[warp] = mn;
       }
+    } else if (warp < NH) {  // absent heads: zero weights
+      s_wT[lane][warp] = 0.f;
+      s_wT[lane + 32][warp] = 0.f;
     }
     __syncthreads();
-    // ---- values, kGnSub tokens at a time: every (token, coordinate) is
-    // decoded once into shared memory (n_V c[idx], and for prod groups
-    // n_V ||r|| sqrt(pi/2)/d sign), then each (head, coordinate) thread
-    // accumulates its weights times them
+    // ---- values: this thread's coordinate of every head, its token class
+    if (vact) {
+      const GnGroup &G = p.v[gv];
 #pragma unroll
-    for (int c = 0; c < kCoords; ++c) {
-      if (c_h[c] >= 0) {
-        acc[c] *= s_alpha[c_h[c]];
-        sacc[c] *= s_alpha[c_h[c]];
+      for (int hh = 0; hh < NH; ++hh) {
+        const float al = s_alpha[hh];
+        acc[hh] *= al;
+        sacc[hh] *= al;
       }
-    }
-    for (int t8 = 0; t8 < nt; t8 += kGnSub) {
-      const int ns = min(kGnSub, nt - t8);
-      if (dec_i >= 0) {
-        const int gv = (p.nv == 2 && dec_i >= p.v[1].off) ? 1 : 0;
-        const GnGroup &G = p.v[gv];
-        const int li = dec_i - G.off;
-        const int vcb = G.d * G.bm / 8;
-        const int64_t vbase = (int64_t)b * G.sb + (int64_t)kvh * G.sh;
-        for (int tt = dec_t; tt < ns; tt += dec_step) {
-          const int64_t vr = vbase + (base + t8 + tt) * G.sn;
-          const float n = s_vn[gv][t8 + tt];
-          s_vx[0][tt][dec_i] = G.bm > 0 ? n * __ldg(G.cent + gn_field(G.codes + vr * vcb, li, G.bm, vcb)) : 0.f;
-          if (G.prod) {
-            const float r = n * s_vr[gv][t8 + tt];
-            s_vx[1][tt][dec_i] = gn_bit(G.qjl + vr * (G.d / 8), li) ? r : -r;
-          }
+      const int vcb = G.d * G.bm / 8;
+      const uint8_t *vc = s_raw + vc_off[gv];
+      const uint8_t *vj = s_raw + vj_off[gv];
+      for (int tt = half; tt < nt; tt += nhalf) {
+        float w[NH];
+        gn_ld_heads<NH>(&s_wT[tt][0], w);
+        const float n = s_vn[gv][tt];
+        const float c = G.bm > 0 ? s_cent[1][gv][gn_field_s(vc + tt * vcb, li, G.bm, vcb)] * n : 0.f;
+#pragma unroll
+        for (int hh = 0; hh < NH; ++hh) acc[hh] = fmaf(w[hh], c, acc[hh]);
+        if (G.prod) {
+          const float r = n * s_vr[gv][tt];
+          const float sr = ((vj[tt * (G.d / 8) + (li >> 3)] >> (li & 7)) & 1) ? r : -r;
+#pragma unroll
+          for (int hh = 0; hh < NH; ++hh) sacc[hh] = fmaf(w[hh], sr, sacc[hh]);
         }
       }
-      __syncthreads();
-#pragma unroll
-      for (int c = 0; c < kCoords; ++c) {
-        if (c_h[c] >= 0) {
-          const int hh = c_h[c], i = c_i[c];
-          float a = acc[c], sa = sacc[c];
-          for (int tt = 0; tt < ns; ++tt) {
-            const float w = s_w[hh][t8 + tt];
-            a = fmaf(w, s_vx[0][tt][i], a);
-            if (c_prod[c]) sa = fmaf(w, s_vx[1][tt][i], sa);
-          }
-          acc[c] = a;
-          sacc[c] = sa;
-        }
-      }
-      __syncthreads();
     }
+    __syncthreads();  // the staged records are read before the next tile's copy
   }
 
-  // ---- the slice's partial state
-  const int stride = 4 + 2 * d;
+  // ---- the slice's partial state: the token classes' sums added per
+  // (head, coordinate)
+  float *s_red = reinterpret_cast<float *>(s_raw);  // [threads][2 NH]
+  static_assert(kGnThreads * 2 * kGnHeads * 4 <= kGnStageBytes, "reduction scratch");
+  if (vact) {
 #pragma unroll
-  for (int c = 0; c < kCoords; ++c) {
-    const int e = tid + kGnThreads * c;
-    if (e < nh * d) {
-      const int hh = e / d, i = e % d;
-      float *slot = p.ws + ((int64_t)split * p.B * p.Hq + (int64_t)b * p.Hq + h0 + hh) * stride;
-      slot[4 + i] = acc[c];
-      slot[4 + d + i] = sacc[c];
-      if (i == 0) {
-        slot[0] = s_m[hh];
-        slot[1] = s_l[hh];
-      }
+    for (int hh = 0; hh < NH; ++hh) {
+      s_red[tid * 2 * NH + hh] = acc[hh];
+      s_red[tid * 2 * NH + NH + hh] = sacc[hh];
+    }
+  }
+  __syncthreads();
+  const int stride = 4 + 2 * d;
+  for (int e = tid; e < nh * d; e += kGnThreads) {
+    const int hh = e / d, i = e - hh * d;
+    float a = 0.f, sa = 0.f;
+    for (int hf = 0; hf < nhalf; ++hf) {
+      const float *r = s_red + (hf * d + i) * 2 * NH;
+      a += r[hh];
+      sa += r[NH + hh];
+    }
+    float *slot = p.ws + ((int64_t)split * p.B * p.Hq + (int64_t)b * p.Hq + h0 + hh) * stride;
+    slot[4 + i] = a;
+    slot[4 + d + i] = sa;
+    if (i == 0) {
+      slot[0] = s_m[hh];
+      slot[1] = s_l[hh];
     }
   }
 }
@@ -357,6 +472,7 @@ __global__ void __launch_bounds__(kGnThreads) general_partial_kernel(GnParams p)
 __global__ void __launch_bounds__(kGnThreads) general_merge_kernel(GnParams p) {
   __shared__ float s_o[kGnMaxD], s_s[kGnMaxD];
   __shared__ float s_hdr[2];
+  __shared__ float s_f[kGnMaxSplits];  // each slot's factor 2^(m_s - M), 0 for an empty slot
   const int head = blockIdx.x;  // b * Hq + hq
   const int b = head / p.Hq;
   const int tid = threadIdx.x;
@@ -367,27 +483,45 @@ __global__ void __launch_bounds__(kGnThreads) general_merge_kernel(GnParams p) {
     for (int i = tid; i < d; i += kGnThreads) out[i] = 0.f;
     return;
   }
-  if (tid == 0) {
+  if (tid < 32) {  // the first warp: the slots' maximum, factors and l, lanes over slots
+    const int lane = tid;
+    float m[kGnMaxSplits / 32], lv[kGnMaxSplits / 32];
     float M = -INFINITY;
-    for (int s = 0; s < p.splits; ++s) M = fmaxf(M, p.ws[((int64_t)s * p.B * p.Hq + head) * stride]);
-    float l = 0.f;
-    for (int s = 0; s < p.splits; ++s) {
-      const float *slot = p.ws + ((int64_t)s * p.B * p.Hq + head) * stride;
-      if (slot[0] != -INFINITY) l += slot[1] * gn_ex2(slot[0] - M);
+#pragma unroll
+    for (int k = 0; k < kGnMaxSplits / 32; ++k) {
+      const int sl = lane + 32 * k;
+      const float *slot = p.ws + ((int64_t)sl * p.B * p.Hq + head) * stride;
+      m[k] = sl < p.splits ? slot[0] : -INFINITY;
+      lv[k] = sl < p.splits ? slot[1] : 0.f;
+      M = fmaxf(M, m[k]);
     }
-    s_hdr[0] = M;
-    s_hdr[1] = l;
+#pragma unroll
+    for (int o = 16; o >= 1; o >>= 1) M = fmaxf(M, __shfl_xor_sync(dev::kFull, M, o));
+    float l = 0.f;
+#pragma unroll
+    for (int k = 0; k < kGnMaxSplits / 32; ++k) {
+      const float f = m[k] == -INFINITY ? 0.f : gn_ex2(m[k] - M);
+      s_f[lane + 32 * k] = f;
+      l = fmaf(lv[k], f, l);
+    }
+#pragma unroll
+    for (int o = 16; o >= 1; o >>= 1) l += __shfl_xor_sync(dev::kFull, l, o);
+    if (lane == 0) {
+      s_hdr[0] = M;
+      s_hdr[1] = l;
+    }
   }
   __syncthreads();
-  const float M = s_hdr[0], l = s_hdr[1];
+  const float l = s_hdr[1];
   for (int i = tid; i < d; i += kGnThreads) {
     float o = 0.f, so = 0.f;
-    for (int s = 0; s < p.splits; ++s) {
-      const float *slot = p.ws + ((int64_t)s * p.B * p.Hq + head) * stride;
-      if (slot[0] == -INFINITY) continue;
-      const float f = gn_ex2(slot[0] - M);
-      o = fmaf(slot[4 + i], f, o);
-      so = fmaf(slot[4 + d + i], f, so);
+    const float *slot = p.ws + (int64_t)head * stride + 4 + i;
+    const int64_t sstride = (int64_t)p.B * p.Hq * stride;
+#pragma unroll 8
+    for (int sl = 0; sl < p.splits; ++sl) {  // empty slots have f = 0 and finite sums
+      const float f = s_f[sl];
+      o = fmaf(slot[sl * sstride], f, o);
+      so = fmaf(slot[sl * sstride + d], f, so);
     }
     s_o[i] = o;
     s_s[i] = so;
@@ -477,10 +611,10 @@ cudaError_t launch_general(GnParams &p, cudaStream_t s) {
 
 int general_decode_splits(int B, int Hq, int Hkv, int64_t seq_len) {
   const int64_t blocks = (int64_t)B * Hkv * ((Hq / Hkv + kGnHeads - 1) / kGnHeads);
-  int64_t s = (2 * (int64_t)decode_ctas() + blocks - 1) / blocks;
+  int64_t s = (4 * (int64_t)decode_ctas() + blocks - 1) / blocks;  // about 4 blocks an SM
   const int64_t by_len = (seq_len + 4 * kGnTile - 1) / (4 * kGnTile);  // at least 4 tiles a split
   if (s > by_len) s = by_len;
-  if (s > 64) s = 64;
+  if (s > kGnMaxSplits) s = kGnMaxSplits;
   return (int)(s < 1 ? 1 : s);
 }
 
