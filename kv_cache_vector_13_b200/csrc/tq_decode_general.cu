@@ -30,6 +30,8 @@
 #include "tq_device.cuh"
 #include "tq_internal.h"
 
+#include <atomic>
+
 namespace tq {
 namespace {
 
@@ -103,19 +105,27 @@ __device__ void gn_fwht(float *x, int nv, int d, int stride) {
   __syncthreads();
 }
 
-// Field i of an LSB-first bm-bit stream of nbytes bytes in shared memory.
-__device__ __forceinline__ int gn_field_s(const uint8_t *rec, int i, int bm, int nbytes) {
+// Staged records sit in shared memory token-major with a pitch of whole
+// 32-bit words, so that a field is read as a word (two at a word boundary).
+__device__ __forceinline__ int gn_pitch(int nbytes) { return (nbytes + 3) & ~3; }
+
+// Index pair (fields i, i + 1; i even) of an LSB-first bm-bit stream held in
+// the words rec[]: a 2 bm-bit pair-table index, field i in the low bits.
+__device__ __forceinline__ uint32_t gn_pair_s(const uint32_t *rec, int i, int bm) {
   const int q = i * bm;
-  const int by = q >> 3, sh = q & 7;
-  uint32_t w = rec[by];
-  if (sh + bm > 8 && by + 1 < nbytes) w |= (uint32_t)rec[by + 1] << 8;
-  return (int)((w >> sh) & ((1u << bm) - 1u));
+  const int wi = q >> 5, sh = q & 31;
+  uint32_t v = rec[wi] >> sh;
+  if (sh + 2 * bm > 32) v |= rec[wi + 1] << (32 - sh);
+  return v & ((1u << (2 * bm)) - 1u);
 }
 
+// Bits i, i + 1 (i even) of a sign stream held in words: bit 0 / bit 1.
+__device__ __forceinline__ uint32_t gn_bits2_s(const uint32_t *rec, int i) { return (rec[i >> 5] >> (i & 31)) & 3u; }
+
 // Copies nbytes-byte records rec0, rec0 + sn, ... (nt of them) of src into
-// dst, token-major; 32-bit words when the records are contiguous and word
-// sized (the cache arrays are 16-byte aligned), else bytes.  The whole block
-// takes part.
+// dst, token-major at gn_pitch(nbytes) bytes a token: 32-bit words when the
+// records are contiguous whole words (the cache arrays are 16-byte
+// aligned), else bytes.  The whole block takes part.
 __device__ __forceinline__ void gn_stage(const uint8_t *src, int64_t rec0, int64_t sn, int nbytes, int nt,
                                          uint8_t *dst) {
   if (sn == 1 && (nbytes & 3) == 0) {
@@ -124,19 +134,22 @@ __device__ __forceinline__ void gn_stage(const uint8_t *src, int64_t rec0, int64
     const int nw = nt * (nbytes >> 2);
     for (int e = threadIdx.x; e < nw; e += kGnThreads) d4[e] = __ldg(s4 + e);
   } else {
+    const int pitch = gn_pitch(nbytes);
     const int nb = nt * nbytes;
     for (int e = threadIdx.x; e < nb; e += kGnThreads) {
       const int tt = e / nbytes, by = e - tt * nbytes;
-      dst[e] = __ldg(src + (rec0 + tt * sn) * nbytes + by);
+      dst[tt * pitch + by] = __ldg(src + (rec0 + tt * sn) * nbytes + by);
     }
   }
 }
 
-// Staging capacity of one side's tile: codes (at most 4 bits a coordinate)
-// and QJL signs of kGnTile tokens.
-constexpr int kGnCodeBytes = kGnTile * kGnMaxD / 2;
-constexpr int kGnSignBytes = kGnTile * kGnMaxD / 8;
+// Staging capacity of one side's tile (two groups at most, each padded to
+// whole words): codes at most 4 bits a coordinate, and the QJL signs.
+constexpr int kGnCodeBytes = kGnTile * (kGnMaxD / 2 + 8);
+constexpr int kGnSignBytes = kGnTile * (kGnMaxD / 8 + 8);
 constexpr int kGnStageBytes = 2 * (kGnCodeBytes + kGnSignBytes);
+// Pair tables in dynamic shared memory: [K / V][group][256] centroid pairs.
+constexpr int kGnPairBytes = 2 * 2 * 256 * 8;
 
 // Loads of the query fragments by head count: NH consecutive floats.
 template <int NH>
@@ -194,7 +207,7 @@ __global__ void __launch_bounds__(kGnThreads) general_partial_kernel(GnParams p)
   __shared__ float s_w[kGnHeads][kGnTile];            // logits
   __shared__ __align__(16) float s_wT[kGnTile][NH];   // weights, token-major
   __shared__ float s_kn[2][kGnTile], s_kr[2][kGnTile], s_vn[2][kGnTile], s_vr[2][kGnTile];
-  __shared__ float s_cent[2][2][16];  // [K / V][group]
+  extern __shared__ float2 s_pt[];   // pair tables [K / V][group][256]
   __shared__ float s_alpha[kGnHeads], s_m[kGnHeads], s_l[kGnHeads];
   float(*s_q)[kGnMaxD] = reinterpret_cast<float(*)[kGnMaxD]>(s_raw);
   float(*s_qs)[kGnMaxD] = reinterpret_cast<float(*)[kGnMaxD]>(s_raw + kGnHeads * kGnMaxD * 4);
@@ -211,11 +224,13 @@ __global__ void __launch_bounds__(kGnThreads) general_partial_kernel(GnParams p)
   const int64_t t0 = (int64_t)split * p.per_split;
   const int64_t t1 = min(L, t0 + p.per_split);
 
-  if (tid < 64) {  // the codebooks
-    const int side = tid >> 5, gr = (tid >> 4) & 1, c = tid & 15;
+  for (int e = tid; e < 4 * 256; e += kGnThreads) {  // pair tables: entry e = (c[e & m], c[e >> bm])
+    const int side = e >> 9, gr = (e >> 8) & 1, pe = e & 255;
     const GnGroup &G = side ? p.v[gr] : p.k[gr];
-    const int ng = side ? p.nv : p.nk;
-    s_cent[side][gr][c] = (gr < ng && G.bm > 0 && c < (1 << G.bm)) ? __ldg(G.cent + c) : 0.f;
+    float2 v = make_float2(0.f, 0.f);
+    if (gr < (side ? p.nv : p.nk) && G.bm > 0 && pe < (1 << (2 * G.bm)))
+      v = make_float2(__ldg(G.cent + (pe & ((1 << G.bm) - 1))), __ldg(G.cent + (pe >> G.bm)));
+    s_pt[e] = v;
   }
   // ---- q'_g = Pi_g q[channels_g] for the block's heads (and S_g q'_g)
   for (int gr = 0; gr < p.nk; ++gr) {
@@ -272,28 +287,31 @@ __global__ void __launch_bounds__(kGnThreads) general_partial_kernel(GnParams p)
     for (int gr = 0; gr < p.nk; ++gr) {
       kc_off[gr] = oc;
       kj_off[gr] = oj;
-      oc += kGnTile * (p.k[gr].d * p.k[gr].bm / 8);
-      oj += kGnTile * (p.k[gr].d / 8);
+      oc += kGnTile * gn_pitch(p.k[gr].d * p.k[gr].bm / 8);
+      oj += kGnTile * gn_pitch(p.k[gr].d / 8);
     }
     oc = kGnCodeBytes + kGnSignBytes;
     oj = 2 * kGnCodeBytes + kGnSignBytes;
     for (int gr = 0; gr < p.nv; ++gr) {
       vc_off[gr] = oc;
       vj_off[gr] = oj;
-      oc += kGnTile * (p.v[gr].d * p.v[gr].bm / 8);
-      oj += kGnTile * (p.v[gr].d / 8);
+      oc += kGnTile * gn_pitch(p.v[gr].d * p.v[gr].bm / 8);
+      oj += kGnTile * gn_pitch(p.v[gr].d / 8);
     }
   }
 
-  // value threads: coordinate vi of the tokens tt = half (mod nhalf)
-  const int nhalf = d >= kGnThreads ? 1 : kGnThreads / d;
-  const int half = tid / d, vi = tid - half * d;
+  // value threads: coordinates (2 vp, 2 vp + 1) of the tokens tt = half
+  // (mod nhalf); a group's coordinates start at a multiple of 8, so a pair
+  // never straddles two groups
+  const int np = d / 2;
+  const int nhalf = kGnThreads / np;
+  const int half = tid / np, vp = tid - half * np;
   const bool vact = half < nhalf;
-  const int gv = (p.nv == 2 && vi >= p.v[1].off) ? 1 : 0;
-  const int li = vi - p.v[gv].off;
-  float acc[NH], sacc[NH];
+  const int gv = (p.nv == 2 && 2 * vp >= p.v[1].off) ? 1 : 0;
+  const int li = 2 * vp - p.v[gv].off;
+  float acc[NH][2], sacc[NH][2];
 #pragma unroll
-  for (int hh = 0; hh < NH; ++hh) acc[hh] = sacc[hh] = 0.f;
+  for (int hh = 0; hh < NH; ++hh) acc[hh][0] = acc[hh][1] = sacc[hh][0] = sacc[hh][1] = 0.f;
 
   for (int64_t base = t0; base < t1; base += kGnTile) {
     const int nt = (int)min((int64_t)kGnTile, t1 - base);
@@ -339,25 +357,30 @@ __global__ void __launch_bounds__(kGnThreads) general_partial_kernel(GnParams p)
       if (ok) {
         for (int gr = 0; gr < p.nk; ++gr) {
           const GnGroup &G = p.k[gr];
-          const int kcb = G.d * G.bm / 8;
-          const uint8_t *kc = s_raw + kc_off[gr] + tt * kcb;
-          const uint8_t *kj = s_raw + kj_off[gr] + tt * (G.d / 8);
+          const uint32_t *kc = reinterpret_cast<const uint32_t *>(
+              s_raw + kc_off[gr] + tt * gn_pitch(G.d * G.bm / 8));
+          const uint32_t *kj = reinterpret_cast<const uint32_t *>(s_raw + kj_off[gr] + tt * gn_pitch(G.d / 8));
+          const float2 *pt = s_pt + gr * 256;
           float part[NH], qpart[NH];
 #pragma unroll
           for (int hh = 0; hh < NH; ++hh) part[hh] = qpart[hh] = 0.f;
+          // a quarter of the group's coordinates, two at a time (G.d / 4 is even)
           const int i0 = qq * (G.d / 4), i1 = i0 + G.d / 4;
-          for (int i = i0; i < i1; ++i) {
-            float qv[NH];
-            gn_ld_heads<NH>(&s_qT[G.off + i][0], qv);
-            const float c = G.bm > 0 ? s_cent[0][gr][gn_field_s(kc, i, G.bm, kcb)] : 0.f;
+          for (int i = i0; i < i1; i += 2) {
+            float q0[NH], q1[NH];
+            gn_ld_heads<NH>(&s_qT[G.off + i][0], q0);
+            gn_ld_heads<NH>(&s_qT[G.off + i + 1][0], q1);
+            const float2 c = G.bm > 0 ? pt[gn_pair_s(kc, i, G.bm)] : make_float2(0.f, 0.f);
 #pragma unroll
-            for (int hh = 0; hh < NH; ++hh) part[hh] = fmaf(c, qv[hh], part[hh]);
+            for (int hh = 0; hh < NH; ++hh) part[hh] = fmaf(c.y, q1[hh], fmaf(c.x, q0[hh], part[hh]));
             if (G.prod) {
-              float sv[NH];
-              gn_ld_heads<NH>(&s_qsT[G.off + i][0], sv);
-              const float sg = ((kj[i >> 3] >> (i & 7)) & 1) ? 1.f : -1.f;
+              float s0[NH], s1[NH];
+              gn_ld_heads<NH>(&s_qsT[G.off + i][0], s0);
+              gn_ld_heads<NH>(&s_qsT[G.off + i + 1][0], s1);
+              const uint32_t bb = gn_bits2_s(kj, i);
+              const float g0 = (bb & 1u) ? 1.f : -1.f, g1 = (bb & 2u) ? 1.f : -1.f;
 #pragma unroll
-              for (int hh = 0; hh < NH; ++hh) qpart[hh] = fmaf(sg, sv[hh], qpart[hh]);
+              for (int hh = 0; hh < NH; ++hh) qpart[hh] = fmaf(g1, s1[hh], fmaf(g0, s0[hh], qpart[hh]));
             }
           }
           const float n = s_kn[gr][tt], kap = s_kr[gr][tt];
@@ -408,30 +431,42 @@ __global__ void __launch_bounds__(kGnThreads) general_partial_kernel(GnParams p)
       s_wT[lane + 32][warp] = 0.f;
     }
     __syncthreads();
-    // ---- values: this thread's coordinate of every head, its token class
+    // ---- values: this thread's coordinate pair of every head, its token class
     if (vact) {
       const GnGroup &G = p.v[gv];
 #pragma unroll
       for (int hh = 0; hh < NH; ++hh) {
         const float al = s_alpha[hh];
-        acc[hh] *= al;
-        sacc[hh] *= al;
+        acc[hh][0] *= al;
+        acc[hh][1] *= al;
+        sacc[hh][0] *= al;
+        sacc[hh][1] *= al;
       }
-      const int vcb = G.d * G.bm / 8;
-      const uint8_t *vc = s_raw + vc_off[gv];
-      const uint8_t *vj = s_raw + vj_off[gv];
+      const int cw = gn_pitch(G.d * G.bm / 8) >> 2, jw = gn_pitch(G.d / 8) >> 2;  // words a token
+      const uint32_t *vc = reinterpret_cast<const uint32_t *>(s_raw + vc_off[gv]);
+      const uint32_t *vj = reinterpret_cast<const uint32_t *>(s_raw + vj_off[gv]);
+      const float2 *pt = s_pt + (2 + gv) * 256;
       for (int tt = half; tt < nt; tt += nhalf) {
         float w[NH];
         gn_ld_heads<NH>(&s_wT[tt][0], w);
         const float n = s_vn[gv][tt];
-        const float c = G.bm > 0 ? s_cent[1][gv][gn_field_s(vc + tt * vcb, li, G.bm, vcb)] * n : 0.f;
+        float2 c = G.bm > 0 ? pt[gn_pair_s(vc + tt * cw, li, G.bm)] : make_float2(0.f, 0.f);
+        c.x *= n;
+        c.y *= n;
 #pragma unroll
-        for (int hh = 0; hh < NH; ++hh) acc[hh] = fmaf(w[hh], c, acc[hh]);
+        for (int hh = 0; hh < NH; ++hh) {
+          acc[hh][0] = fmaf(w[hh], c.x, acc[hh][0]);
+          acc[hh][1] = fmaf(w[hh], c.y, acc[hh][1]);
+        }
         if (G.prod) {
           const float r = n * s_vr[gv][tt];
-          const float sr = ((vj[tt * (G.d / 8) + (li >> 3)] >> (li & 7)) & 1) ? r : -r;
+          const uint32_t bb = gn_bits2_s(vj + tt * jw, li);
+          const float r0 = (bb & 1u) ? r : -r, r1 = (bb & 2u) ? r : -r;
 #pragma unroll
-          for (int hh = 0; hh < NH; ++hh) sacc[hh] = fmaf(w[hh], sr, sacc[hh]);
+          for (int hh = 0; hh < NH; ++hh) {
+            sacc[hh][0] = fmaf(w[hh], r0, sacc[hh][0]);
+            sacc[hh][1] = fmaf(w[hh], r1, sacc[hh][1]);
+          }
         }
       }
     }
@@ -439,33 +474,34 @@ __global__ void __launch_bounds__(kGnThreads) general_partial_kernel(GnParams p)
   }
 
   // ---- the slice's partial state: the token classes' sums added per
-  // (head, coordinate)
-  float *s_red = reinterpret_cast<float *>(s_raw);  // [threads][2 NH]
-  static_assert(kGnThreads * 2 * kGnHeads * 4 <= kGnStageBytes, "reduction scratch");
-  if (vact) {
-#pragma unroll
-    for (int hh = 0; hh < NH; ++hh) {
-      s_red[tid * 2 * NH + hh] = acc[hh];
-      s_red[tid * 2 * NH + NH + hh] = sacc[hh];
-    }
-  }
-  __syncthreads();
+  // (head, coordinate), the value sums first, then (prod value groups) the
+  // sign sums, through the staging memory
+  float *s_red = reinterpret_cast<float *>(s_raw);  // [threads][NH][2]
+  static_assert(kGnThreads * kGnHeads * 2 * 4 <= kGnStageBytes, "reduction scratch");
   const int stride = 4 + 2 * d;
-  for (int e = tid; e < nh * d; e += kGnThreads) {
-    const int hh = e / d, i = e - hh * d;
-    float a = 0.f, sa = 0.f;
-    for (int hf = 0; hf < nhalf; ++hf) {
-      const float *r = s_red + (hf * d + i) * 2 * NH;
-      a += r[hh];
-      sa += r[NH + hh];
+  const bool any_prod = p.v[0].prod || (p.nv == 2 && p.v[1].prod);
+  for (int round = 0; round < (any_prod ? 2 : 1); ++round) {
+    if (vact) {
+#pragma unroll
+      for (int hh = 0; hh < NH; ++hh) {
+        s_red[(tid * NH + hh) * 2] = round ? sacc[hh][0] : acc[hh][0];
+        s_red[(tid * NH + hh) * 2 + 1] = round ? sacc[hh][1] : acc[hh][1];
+      }
     }
-    float *slot = p.ws + ((int64_t)split * p.B * p.Hq + (int64_t)b * p.Hq + h0 + hh) * stride;
-    slot[4 + i] = a;
-    slot[4 + d + i] = sa;
-    if (i == 0) {
-      slot[0] = s_m[hh];
-      slot[1] = s_l[hh];
+    __syncthreads();
+    for (int e = tid; e < nh * d; e += kGnThreads) {
+      const int hh = e / d, i = e - hh * d;
+      float a = 0.f;
+      for (int hf = 0; hf < nhalf; ++hf) a += s_red[((hf * np + (i >> 1)) * NH + hh) * 2 + (i & 1)];
+      float *slot = p.ws + ((int64_t)split * p.B * p.Hq + (int64_t)b * p.Hq + h0 + hh) * stride;
+      slot[4 + round * d + i] = a;
+      if (round == 0 && i == 0) {
+        slot[0] = s_m[hh];
+        slot[1] = s_l[hh];
+      }
+      if (!any_prod) slot[4 + d + i] = 0.f;
     }
+    __syncthreads();
   }
 }
 
@@ -517,11 +553,22 @@ __global__ void __launch_bounds__(kGnThreads) general_merge_kernel(GnParams p) {
     float o = 0.f, so = 0.f;
     const float *slot = p.ws + (int64_t)head * stride + 4 + i;
     const int64_t sstride = (int64_t)p.B * p.Hq * stride;
-#pragma unroll 8
-    for (int sl = 0; sl < p.splits; ++sl) {  // empty slots have f = 0 and finite sums
-      const float f = s_f[sl];
-      o = fmaf(slot[sl * sstride], f, o);
-      so = fmaf(slot[sl * sstride + d], f, so);
+    // batches of 8 slots, every load of a batch issued before its sums
+    // (empty slots have f = 0 and finite sums)
+    for (int s0 = 0; s0 < p.splits; s0 += 8) {
+      float x[8], y[8];
+#pragma unroll
+      for (int k = 0; k < 8; ++k) {
+        const int sl = min(s0 + k, p.splits - 1);
+        x[k] = __ldcg(slot + sl * sstride);
+        y[k] = __ldcg(slot + sl * sstride + d);
+      }
+#pragma unroll
+      for (int k = 0; k < 8; ++k) {
+        const float f = s0 + k < p.splits ? s_f[s0 + k] : 0.f;
+        o = fmaf(x[k], f, o);
+        so = fmaf(y[k], f, so);
+      }
     }
     s_o[i] = o;
     s_s[i] = so;
@@ -535,7 +582,13 @@ __global__ void __launch_bounds__(kGnThreads) general_merge_kernel(GnParams p) {
     float a = 0.f;
     if (G.prod) {
       const int li = i - G.off;
-      for (int k = 0; k < G.d; ++k) a = fmaf(__ldg(G.S + (int64_t)k * G.d + li), s_s[G.off + k], a);
+      for (int k0 = 0; k0 < G.d; k0 += 8) {  // batches of 8 loads
+        float x[8];
+#pragma unroll
+        for (int k = 0; k < 8; ++k) x[k] = __ldg(G.S + (int64_t)(k0 + k) * G.d + li);
+#pragma unroll
+        for (int k = 0; k < 8; ++k) a = fmaf(x[k], s_s[G.off + k0 + k], a);
+      }
     }
     add[c] = a;
   }
@@ -549,7 +602,13 @@ __global__ void __launch_bounds__(kGnThreads) general_merge_kernel(GnParams p) {
       const GnGroup &G = p.v[gv];
       const int c = i - G.off;
       float a = 0.f;
-      for (int r = 0; r < G.d; ++r) a = fmaf(__ldg(G.rot + (int64_t)r * G.d + c), s_o[G.off + r], a);
+      for (int r0 = 0; r0 < G.d; r0 += 8) {  // G.d is a multiple of 8: batches of 8 loads
+        float x[8];
+#pragma unroll
+        for (int k = 0; k < 8; ++k) x[k] = __ldg(G.rot + (int64_t)(r0 + k) * G.d + c);
+#pragma unroll
+        for (int k = 0; k < 8; ++k) a = fmaf(x[k], s_o[G.off + r0 + k], a);
+      }
       const int ch = G.chan ? min(max(__ldg(G.chan + c), 0), d - 1) : c;
       out[ch] = a * inv_l;
     }
@@ -581,6 +640,25 @@ GnGroup group_of(const QuantParams &q, const CacheView &v, int off) {
   return g;
 }
 
+// One partial-kernel launch with the pair tables' dynamic shared memory;
+// the kernel's limit is raised once per device (the setting belongs to the
+// kernel, so later launches skip the driver call).
+template <int NH>
+cudaError_t launch_partial(const GnParams &p, dim3 grid, cudaStream_t s) {
+  static std::atomic<uint64_t> done{0};
+  int dev = 0;
+  cudaError_t e = cudaGetDevice(&dev);
+  if (e != cudaSuccess) return e;
+  const uint64_t bit = dev >= 0 && dev < 64 ? (uint64_t)1 << dev : 0;
+  if (!bit || !(done.load(std::memory_order_acquire) & bit)) {
+    e = cudaFuncSetAttribute(general_partial_kernel<NH>, cudaFuncAttributeMaxDynamicSharedMemorySize, kGnPairBytes);
+    if (e != cudaSuccess) return e;
+    if (bit) done.fetch_or(bit, std::memory_order_release);
+  }
+  general_partial_kernel<NH><<<grid, kGnThreads, kGnPairBytes, s>>>(p);
+  return cudaGetLastError();
+}
+
 cudaError_t launch_general(GnParams &p, cudaStream_t s) {
   p.g = p.Hq / p.Hkv;
   p.hg = (p.g + kGnHeads - 1) / kGnHeads;
@@ -589,16 +667,10 @@ cudaError_t launch_general(GnParams &p, cudaStream_t s) {
   p.per_split = (p.seq_len + p.splits - 1) / p.splits;
   if (p.seq_len > 0) {
     const dim3 grid((unsigned)p.splits, (unsigned)(p.B * p.Hkv * p.hg));
-    if (p.g <= 1) {
-      general_partial_kernel<1><<<grid, kGnThreads, 0, s>>>(p);
-    } else if (p.g <= 2) {
-      general_partial_kernel<2><<<grid, kGnThreads, 0, s>>>(p);
-    } else if (p.g <= 4) {
-      general_partial_kernel<4><<<grid, kGnThreads, 0, s>>>(p);
-    } else {
-      general_partial_kernel<8><<<grid, kGnThreads, 0, s>>>(p);
-    }
-    const cudaError_t e = cudaGetLastError();
+    const cudaError_t e = p.g <= 1   ? launch_partial<1>(p, grid, s)
+                          : p.g <= 2 ? launch_partial<2>(p, grid, s)
+                          : p.g <= 4 ? launch_partial<4>(p, grid, s)
+                                     : launch_partial<8>(p, grid, s);
     if (e != cudaSuccess) return e;
   } else {
     p.splits = 0;
