@@ -82,10 +82,10 @@ FALLBACK_PEAKS = {"hbm_gbs": 6650.0, "bf16_tflops": 1590.0}
 # workload, from an ncu capture (dram__bytes_read.sum + dram__bytes_write.sum),
 # reported only for that workload and while the decode sources are the ones
 # it was taken on.
-# Captured at B = 2 (reads 230,584,576 B, writes 4,909,568 B): reads scaled by
+# Captured at B = 2 (reads 230,603,776 B, writes 6,578,432 B): reads scaled by
 # the 8x units of B = 16 (B = 4 read 2.02x the B = 2 bytes), writes kept.
-TRAFFIC = {"workload": ("batched", 16), "bytes": 8 * 230584576 + 4909568,
-           "source_sha256": "343a0ed3f5953b6e11dcebf16029f430d30dc8ff5c04d583407db6010b4803be"}
+TRAFFIC = {"workload": ("batched", 16), "bytes": 8 * 230603776 + 6578432,
+           "source_sha256": "a9341d60c8f0be0698b70685d21f39be65745671de9322120b370182fa5353e9"}
 DECODE_SOURCES = ("tq_decode.cu", "tq_decode_split.cuh", "tq_decode_regs.cu")
 
 
