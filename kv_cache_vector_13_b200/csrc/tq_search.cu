@@ -128,7 +128,9 @@ __global__ void __launch_bounds__(kSrWarps * 32) search_score_kernel(SearchParam
   static_assert(sizeof(s_tab) >= (size_t)kSrWarps * 8 * kTop * 8, "merge lists fit in the table");
   const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
   const int g8 = lane >> 2, tig = lane & 3;
-  const int u = blockIdx.y, split = blockIdx.x;
+  // the units of one slice are adjacent in launch order, so that they read
+  // the slice at about the same time and share it through L2
+  const int u = blockIdx.x, split = blockIdx.y;
   const int gh = min(8, p.nq - u * 8);
   for (int i = tid; i < 256 * 32; i += blockDim.x)
     s_tab[i] = KBM > 0 ? __ldg(reinterpret_cast<const uint32_t *>(p.ws + 64) + (i >> 5)) : 0u;
@@ -341,7 +343,7 @@ __global__ void __launch_bounds__(256) search_merge_kernel(SearchParams p) {
 
 template <int KBM, bool KPROD, bool PACK>
 cudaError_t run_search(const SearchParams &sp, cudaStream_t s) {
-  search_score_kernel<KBM, KPROD, PACK><<<dim3((unsigned)sp.splits, (unsigned)sp.units), kSrWarps * 32, 0, s>>>(sp);
+  search_score_kernel<KBM, KPROD, PACK><<<dim3((unsigned)sp.units, (unsigned)sp.splits), kSrWarps * 32, 0, s>>>(sp);
   cudaError_t e = cudaGetLastError();
   if (e != cudaSuccess) return e;
   search_merge_kernel<<<(unsigned)((sp.nq + 7) / 8), 256, 0, s>>>(sp);
