@@ -281,23 +281,46 @@ cudaError_t take_device_faults(unsigned *faults) {
 
 namespace {
 
-// Device address of a __device__ symbol on the current device, looked up
-// once per device (with that device current) and cached.
+// The driver's current-context query, reached through the runtime (no
+// link against the driver library); NULL when the runtime cannot provide it.
+using CtxCurrentFn = int (*)(void **);
+CtxCurrentFn ctx_current_fn() {
+  static const CtxCurrentFn fn = [] {
+    void *f = nullptr;
+    cudaDriverEntryPointQueryResult q = cudaDriverEntryPointSymbolNotFound;
+    if (cudaGetDriverEntryPoint("cuCtxGetCurrent", &f, cudaEnableDefault, &q) != cudaSuccess ||
+        q != cudaDriverEntryPointSuccess)
+      f = nullptr;
+    return reinterpret_cast<CtxCurrentFn>(f);
+  }();
+  return fn;
+}
+
+// Device address of a __device__ symbol in the current context.  Cached per
+// device together with the context it was looked up in, and looked up again
+// when the device's context has changed (a reset destroys the primary
+// context, and the symbol's address with it); without the context query it
+// is looked up on every call.
 template <typename Sym>
 cudaError_t symbol_address(const Sym &sym, void **ptr) {
   constexpr int kMaxDevices = 64;
   static std::mutex mu;
   static void *addr[kMaxDevices] = {};
+  static void *ctx_of[kMaxDevices] = {};
   int dev = 0;
   cudaError_t e = cudaGetDevice(&dev);
   if (e != cudaSuccess) return e;
   if (dev < 0 || dev >= kMaxDevices) return cudaErrorInvalidDevice;
+  void *ctx = nullptr;  // no context yet: looked up (which creates it) and not cached
+  const CtxCurrentFn fn = ctx_current_fn();
+  const bool keyed = fn && fn(&ctx) == 0 && ctx;
   std::lock_guard<std::mutex> lock(mu);
-  if (!addr[dev]) {
+  if (!keyed || !addr[dev] || ctx_of[dev] != ctx) {
     void *a = nullptr;
     e = cudaGetSymbolAddress(&a, sym);
     if (e != cudaSuccess) return e;
     addr[dev] = a;
+    ctx_of[dev] = keyed ? ctx : nullptr;
   }
   *ptr = addr[dev];
   return cudaSuccess;
@@ -313,7 +336,7 @@ cudaError_t fault_word(unsigned **ptr) {
 }
 
 cudaError_t static_scratch(void **ptr) {
-  // looked up once per device, with that device current, and cached
+  // cached per device and context
   return symbol_address(g_tq_noalloc_scratch, ptr);
 }
 
