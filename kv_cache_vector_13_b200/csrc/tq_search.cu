@@ -184,6 +184,11 @@ __global__ void __launch_bounds__(kSrWarps * 32) search_score_kernel(SearchParam
     lv[h] = kth_v[h] = -INFINITY;
     li[h] = kth_i[h] = INT_MAX;
   }
+  // the k-th entries of this lane's own two query columns h = 2 tig + c
+  // (PACK: lanes tig >= 2 repeat the columns of tig - 2 and own none)
+  const bool own = PACK ? tig < 2 : true;
+  float kthm_v[2] = {-INFINITY, -INFINITY};
+  int kthm_i[2] = {INT_MAX, INT_MAX};
   // this CTA's slice of the database, this warp's chunks of it
   const int64_t s0 = p.N * split / p.splits, s1 = p.N * (split + 1) / p.splits;
   const int64_t nch = (s1 - s0 + kChunk - 1) / kChunk;
@@ -245,24 +250,30 @@ __global__ void __launch_bounds__(kSrWarps * 32) search_score_kernel(SearchParam
       }
     }
     // per query: does any of the chunk's 32 candidates beat the list's
-    // k-th entry?  The lanes holding query h's estimates (column h of the
-    // score tile: rows g8 + 8 r + 16 ms) answer with one vote.
+    // k-th entry?  Each lane tests its own two columns (rows g8 + 8 r +
+    // 16 ms of the score tile) against their k-th entries; two votes answer
+    // for every query, and most chunks end here.
+    bool hc[2] = {false, false};
+#pragma unroll
+    for (int c = 0; c < 2; ++c) {
+#pragma unroll
+      for (int ms = 0; ms < 2; ++ms) {
+#pragma unroll
+        for (int r = 0; r < 2; ++r) {
+          const int idx = (int)(r0 + 16 * ms + 8 * r + g8);
+          hc[c] |= better(est[ms][2 * r + c], idx, kthm_v[c], kthm_i[c]);
+        }
+      }
+      hc[c] = hc[c] && own && 2 * tig + c < gh;
+    }
+    const unsigned hit0 = __ballot_sync(dev::kFull, hc[0]), hit1 = __ballot_sync(dev::kFull, hc[1]);
+    if ((hit0 | hit1) == 0u) continue;
 #pragma unroll
     for (int h = 0; h < 8; ++h) {
       if (h < gh) {
         const int c = h & 1;
-        const bool mine = tig == (h >> 1);
-        bool hit = false;
-#pragma unroll
-        for (int ms = 0; ms < 2; ++ms) {
-#pragma unroll
-          for (int r = 0; r < 2; ++r) {
-            const int idx = (int)(r0 + 16 * ms + 8 * r + g8);
-            hit |= mine && better(est[ms][2 * r + c], idx, kth_v[h], kth_i[h]);
-          }
-        }
-        const unsigned any = __ballot_sync(dev::kFull, hit);
-        if (any == 0u) continue;
+        // lanes l with l % 4 == h / 2 hold column h
+        if ((((c ? hit1 : hit0) >> (h >> 1)) & 0x11111111u) == 0u) continue;
         // the chunk's candidates for query h, one per lane (lane L holds
         // record r0 + L)
         const int src = (lane & 7) * 4 + (h >> 1);
@@ -300,6 +311,10 @@ __global__ void __launch_bounds__(kSrWarps * 32) search_score_kernel(SearchParam
         }
         kth_v[h] = __shfl_sync(dev::kFull, lv[h], p.k - 1);
         kth_i[h] = __shfl_sync(dev::kFull, li[h], p.k - 1);
+        if (tig == (h >> 1)) {
+          kthm_v[c] = kth_v[h];
+          kthm_i[c] = kth_i[h];
+        }
       }
     }
   }
@@ -326,18 +341,38 @@ __global__ void __launch_bounds__(kSrWarps * 32) search_score_kernel(SearchParam
   }
 }
 
+// One block per query: warp w merges the slices' lists w, w + 8, ... (the
+// next list's loads issued before the current merge), then warp 0 merges
+// the eight results and writes the first k.
 __global__ void __launch_bounds__(256) search_merge_kernel(SearchParams p) {
-  const int lane = threadIdx.x & 31;
-  const int qg = blockIdx.x * 8 + (threadIdx.x >> 5);
-  if (qg >= p.nq) return;
+  __shared__ float s_v[8][kTop];
+  __shared__ int s_i[8][kTop];
+  const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5;
+  const int qg = blockIdx.x;
   const int64_t base = (int64_t)qg * p.splits * kTop + lane;
-  float v = p.cand_v[base];
-  int i = p.cand_i[base];
-  for (int s = 1; s < p.splits; ++s) warp_merge(v, i, p.cand_v[base + (int64_t)s * kTop], p.cand_i[base + (int64_t)s * kTop], lane);
-  if (lane < p.k) {
-    const bool real = v > -INFINITY;
-    p.top_v[(int64_t)qg * p.k + lane] = v;
-    p.top_i[(int64_t)qg * p.k + lane] = real ? (int64_t)i : -1;
+  float v = -INFINITY;
+  int i = INT_MAX;
+  float nv = warp < p.splits ? p.cand_v[base + (int64_t)warp * kTop] : -INFINITY;
+  int ni = warp < p.splits ? p.cand_i[base + (int64_t)warp * kTop] : INT_MAX;
+  for (int sl = warp; sl < p.splits; sl += 8) {
+    const float cv = nv;
+    const int ci = ni;
+    if (sl + 8 < p.splits) {
+      nv = p.cand_v[base + (int64_t)(sl + 8) * kTop];
+      ni = p.cand_i[base + (int64_t)(sl + 8) * kTop];
+    }
+    warp_merge(v, i, cv, ci, lane);
+  }
+  s_v[warp][lane] = v;
+  s_i[warp][lane] = i;
+  __syncthreads();
+  if (warp == 0) {
+    for (int w = 1; w < 8; ++w) warp_merge(v, i, s_v[w][lane], s_i[w][lane], lane);
+    if (lane < p.k) {
+      const bool real = v > -INFINITY;
+      p.top_v[(int64_t)qg * p.k + lane] = v;
+      p.top_i[(int64_t)qg * p.k + lane] = real ? (int64_t)i : -1;
+    }
   }
 }
 
@@ -346,7 +381,7 @@ cudaError_t run_search(const SearchParams &sp, cudaStream_t s) {
   search_score_kernel<KBM, KPROD, PACK><<<dim3((unsigned)sp.units, (unsigned)sp.splits), kSrWarps * 32, 0, s>>>(sp);
   cudaError_t e = cudaGetLastError();
   if (e != cudaSuccess) return e;
-  search_merge_kernel<<<(unsigned)((sp.nq + 7) / 8), 256, 0, s>>>(sp);
+  search_merge_kernel<<<(unsigned)sp.nq, 256, 0, s>>>(sp);
   return cudaGetLastError();
 }
 
