@@ -50,6 +50,14 @@ struct SearchParams {
   int64_t *top_i;
 };
 
+// Order-preserving int key of a float (signed int order = float order), so
+// that atomicMax keeps a running float maximum.
+__device__ __forceinline__ int fkey(float f) {
+  const int b = __float_as_int(f);
+  return b ^ ((b >> 31) & 0x7fffffff);
+}
+__device__ __forceinline__ float funkey(int k) { return __int_as_float(k ^ ((k >> 31) & 0x7fffffff)); }
+
 __device__ __forceinline__ bool better(float va, int ia, float vb, int ib) {
   return va > vb || (va == vb && ia < ib);
 }
@@ -134,6 +142,11 @@ __global__ void __launch_bounds__(kSrWarps * 32) search_score_kernel(SearchParam
   const int gh = min(8, p.nq - u * 8);
   for (int i = tid; i < 256 * 32; i += blockDim.x)
     s_tab[i] = KBM > 0 ? __ldg(reinterpret_cast<const uint32_t *>(p.ws + 64) + (i >> 5)) : 0u;
+  // the CTA's k-th best estimate per query so far (the best over the warps'
+  // k-th entries, only ever raised): a candidate below it is beaten by k
+  // others in this CTA and cannot reach the result
+  __shared__ int s_kkey[8];
+  if (tid < 8) s_kkey[tid] = fkey(-INFINITY);
   const float inv_sK = __ldg(p.ws + 0);
   const float sK = 1.0f / inv_sK;
   __syncthreads();
@@ -256,12 +269,14 @@ __global__ void __launch_bounds__(kSrWarps * 32) search_score_kernel(SearchParam
     bool hc[2] = {false, false};
 #pragma unroll
     for (int c = 0; c < 2; ++c) {
+      const float cta = funkey(*reinterpret_cast<volatile int *>(&s_kkey[2 * tig + c]));
 #pragma unroll
       for (int ms = 0; ms < 2; ++ms) {
 #pragma unroll
         for (int r = 0; r < 2; ++r) {
           const int idx = (int)(r0 + 16 * ms + 8 * r + g8);
-          hc[c] |= better(est[ms][2 * r + c], idx, kthm_v[c], kthm_i[c]);
+          const float e = est[ms][2 * r + c];
+          hc[c] |= e >= cta && better(e, idx, kthm_v[c], kthm_i[c]);
         }
       }
       hc[c] = hc[c] && own && 2 * tig + c < gh;
@@ -287,7 +302,8 @@ __global__ void __launch_bounds__(kSrWarps * 32) search_score_kernel(SearchParam
           }
         }
         const int cidx = (int)(r0 + lane);
-        const unsigned up = __ballot_sync(dev::kFull, better(cv, cidx, kth_v[h], kth_i[h]));
+        const float cta = funkey(*reinterpret_cast<volatile int *>(&s_kkey[h]));
+        const unsigned up = __ballot_sync(dev::kFull, cv >= cta && better(cv, cidx, kth_v[h], kth_i[h]));
         if (__popc(up) > 4) {  // many (the lists' first chunks): sort and merge
           int ci2 = cidx;
           warp_sort(cv, ci2, lane);
@@ -315,6 +331,7 @@ __global__ void __launch_bounds__(kSrWarps * 32) search_score_kernel(SearchParam
           kthm_v[c] = kth_v[h];
           kthm_i[c] = kth_i[h];
         }
+        if (lane == 0 && kth_v[h] > -INFINITY) atomicMax(&s_kkey[h], fkey(kth_v[h]));
       }
     }
   }
