@@ -311,6 +311,16 @@ def run_ours(args):
 
     # the dominant kernels (prep + split of tq_decode_attention), live
     dec_ms = time_decode_calls(torch, s, stream, max(10, min(K_steps, 200)))
+    # the same call through the bulk-copy staging feed (an extra record; the
+    # register feed above is the default)
+    staged_ms = None
+    if not args.no_extras and ws == 1:
+        prev = api.set_decode_feed(True)
+        try:
+            staged_ms = time_decode_calls(torch, s, stream, max(10, min(K_steps, 100)))
+            api.check(stream)
+        finally:
+            api.set_decode_feed(prev)
 
     # end to end through the public API with host buffers, every step: H2D of
     # the step's inputs (q, k_new, v_new, bf16, one pinned buffer), the step,
@@ -394,6 +404,13 @@ def run_ours(args):
             with ClockSampler(local) as nclk:
                 line["next_rows"] = bench_next_rows(api, inputs, torch, dev, stream)
             line["next_rows"]["clocks"] = nclk.summary()
+            if staged_ms is not None:
+                line["next_rows"]["decode_bulk_staged"] = {
+                    "workload": line["config"]["workload"] + "; records fed through shared-memory rings filled by "
+                                "bulk asynchronous copies (cp.async.bulk, mbarrier waits)",
+                    "ms_per_call": staged_ms, "bytes_per_call": line["roofline"]["bytes_per_launch"],
+                    "achieved_gbs": line["roofline"]["bytes_per_launch"] / (staged_ms * 1e-3) / 1e9,
+                    "frac": line["roofline"]["bytes_per_launch"] / (staged_ms * 1e-3) / 1e9 / pk["hbm_gbs"]}
         if not args.no_cpu_baseline and ws == 1:
             line["cpu_baseline"] = cpu_baseline_decode(args.workload, args.batch, budget_s=args.cpu_seconds)
         print(json.dumps(line), flush=True)

@@ -302,6 +302,24 @@ tq_status tq_search_topk(const tq_quantizer *q, const tq_cache_view *db, int64_t
                          float *top_scores, int64_t *top_index, void *workspace,
                          size_t workspace_bytes, tq_stream_t stream);
 
+/* How the decode's tensor-core split kernel feeds the packed records of a
+ * unit-stride cache to its warps, for the whole process (host threads
+ * included; calls already enqueued keep the feed they were launched with):
+ *   TQ_FEED_REGISTERS (0, the default and the faster one measured on B200):
+ *     each warp loads the next chunk's records from global memory straight
+ *     into registers while it works on the current one;
+ *   TQ_FEED_BULK_STAGED (1): each warp keeps a ring of 2 to 4 shared-memory
+ *     slots filled by bulk asynchronous copies (cp.async.bulk, this GPU's
+ *     own memory) that complete on one mbarrier per slot, waited on with a
+ *     bounded loop (a timeout sets the fault word tq_check reports); the
+ *     cache's norm rows must be 16-byte aligned, and a cache or launch that
+ *     does not fit it falls back to the register feed.
+ * Both compute the same attention ("I Spent 31 Hours On The Math Behind
+ * Turboquant", section "KV Cache: The problem"); results agree to rounding.
+ * Returns the previous setting, or -1 (setting unchanged) for another value. */
+typedef enum { TQ_FEED_REGISTERS = 0, TQ_FEED_BULK_STAGED = 1 } tq_decode_feed;
+int32_t tq_set_decode_feed(int32_t feed);
+
 /* Synchronize `stream` and report any asynchronous CUDA error, then read and
  * clear the current GPU's fault word, which the kernels set themselves
  * instead of trapping: TQ_ETIMEOUT when a kernel gave up a bounded wait on

@@ -11,6 +11,7 @@ _HERE = os.path.dirname(os.path.abspath(__file__))
 LIB_PATH = os.path.join(_HERE, "libtq_b200.so")
 
 TQ_OK, TQ_EINVAL, TQ_EUNSUPPORTED, TQ_ECUDA, TQ_EWORKSPACE, TQ_ETIMEOUT = range(6)
+TQ_FEED_REGISTERS, TQ_FEED_BULK_STAGED = 0, 1  # tq_decode_feed
 TQ_MSE, TQ_PROD = 0, 1
 TQ_ROT_HADAMARD, TQ_ROT_DENSE = 0, 1
 TQ_CB_GAUSS, TQ_CB_BETA = 0, 1
@@ -24,7 +25,7 @@ EXPORTS = (
     "tq_append_decode_attention", "tq_decode_attention_noalloc",
     "tq_search_workspace_bytes", "tq_search_topk",
     "tq_decode_split_workspace_bytes", "tq_decode_attention_split",
-    "tq_check", "tq_status_string", "tq_last_error", "tq_version",
+    "tq_set_decode_feed", "tq_check", "tq_status_string", "tq_last_error", "tq_version",
 )
 
 
@@ -108,6 +109,8 @@ def lib() -> ctypes.CDLL:
         POINTER(TqQuantizer), POINTER(TqQuantizer), c_void_p, c_int32, c_int32, c_int32, c_int32, c_int64,
         c_void_p, POINTER(TqCacheView), POINTER(TqCacheView), c_float, c_void_p, c_void_p, c_size_t, c_void_p]
     L.tq_decode_attention_split.restype = c_int32
+    L.tq_set_decode_feed.argtypes = [c_int32]
+    L.tq_set_decode_feed.restype = c_int32
     L.tq_check.argtypes = [c_void_p]
     L.tq_check.restype = c_int32
     L.tq_status_string.argtypes = [c_int32]

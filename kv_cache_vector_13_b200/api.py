@@ -350,5 +350,13 @@ def search_topk(qz: Quantizer, queries: torch.Tensor, db: PackedCache, k: int):
     return Search(qz, queries.shape[0], n_db, device=queries.device)(queries, db, k)
 
 
+def set_decode_feed(staged: bool) -> bool:
+    """Feed of the tensor-core decode for this process: bulk-copy staging
+    through shared memory (True) or straight into registers (False, the
+    default). Returns whether staging was on before."""
+    prev = L.lib().tq_set_decode_feed(L.TQ_FEED_BULK_STAGED if staged else L.TQ_FEED_REGISTERS)
+    return prev == L.TQ_FEED_BULK_STAGED
+
+
 def check(stream=None) -> None:
     L.check(L.lib().tq_check(_stream(stream)))

@@ -19,13 +19,13 @@
 
 #include "tq_decode_split.cuh"
 
+#include <atomic>
 #include <mutex>
 
 // Which split-kernel variant feeds unit-stride caches: the register-fed one
-// (0, the faster one measured on B200) or the bulk-copy ring (1).
-#ifndef TQ_DECODE_STAGED
-#define TQ_DECODE_STAGED 0
-#endif
+// (TQ_FEED_REGISTERS, the faster one measured on B200) or the bulk-copy ring
+// (TQ_FEED_BULK_STAGED); set by tq_set_decode_feed.
+static std::atomic<int> g_decode_feed{TQ_FEED_REGISTERS};
 
 // Scratch for tq_decode_attention_noalloc: a fixed array in device memory,
 // one copy per GPU that loads the library, held until the process exits.
@@ -437,8 +437,9 @@ cudaError_t launch_decode(const DecodeArgs &a, cudaStream_t s) {
   auto rows16 = [&](const void *ptr, int64_t sb, int64_t sh) {
     return ptr == nullptr || (((uintptr_t)ptr % 16) == 0 && (a.B == 1 || sb % 4 == 0) && (a.Hkv == 1 || sh % 4 == 0));
   };
-  const bool staged = TQ_DECODE_STAGED && a.k.sn == 1 && a.v.sn == 1 && rows16(a.k.norms, a.k.sb, a.k.sh) &&
-                      rows16(a.k.rnorms, a.k.sb, a.k.sh) && rows16(a.v.norms, a.v.sb, a.v.sh);
+  const bool staged = g_decode_feed.load(std::memory_order_relaxed) == TQ_FEED_BULK_STAGED && a.k.sn == 1 &&
+                      a.v.sn == 1 && rows16(a.k.norms, a.k.sb, a.k.sh) && rows16(a.k.rnorms, a.k.sb, a.k.sh) &&
+                      rows16(a.v.norms, a.v.sb, a.v.sh);
   cudaError_t e = cudaErrorInvalidValue;
   if (staged) e = dec::launch_split_staged(a.kq.bm, a.kq.prod, a.vq.bm, pack, sp, s);
   if (!staged || e == cudaErrorInvalidConfiguration) {
@@ -450,3 +451,8 @@ cudaError_t launch_decode(const DecodeArgs &a, cudaStream_t s) {
 }
 
 }  // namespace tq
+
+extern "C" int32_t tq_set_decode_feed(int32_t feed) {
+  if (feed != TQ_FEED_REGISTERS && feed != TQ_FEED_BULK_STAGED) return -1;
+  return g_decode_feed.exchange(feed);
+}

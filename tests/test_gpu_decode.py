@@ -408,3 +408,42 @@ def test_decode_cuda_core_path_long_cache():
     out = run_case(1, 4, 1, 40000, (4, "prod"), (4, "prod"), seed=77, d=256, kv_scale=3.0)
     assert np.all(np.isfinite(out))
 
+
+
+@pytest.fixture
+def bulk_staged_feed():
+    prev = api.set_decode_feed(True)
+    yield
+    api.set_decode_feed(prev)
+
+
+@pytest.mark.parametrize("kspec,vspec,Hq", [((3, "prod"), (3, "mse"), 32), ((4, "mse"), (4, "mse"), 32),
+                                            ((4, "prod"), (4, "mse"), 64), ((2, "mse"), (2, "mse"), 16)])
+def test_decode_bulk_staged_feed_matches_oracle(bulk_staged_feed, kspec, vspec, Hq):
+    # the bulk-copy ring feed (shared-memory slots filled by cp.async.bulk,
+    # mbarrier waits) on unit-stride caches with 16-byte aligned norm rows:
+    # <= 4 and 8 query heads per kv head, prod and mse keys, a ragged batch
+    B, Hkv, N = 2, 8, 1000
+    heads = [(0, 0), (0, Hq - 1), (1, 1), (1, Hq // 2)]
+    out = run_case(B, Hq, Hkv, N, kspec, vspec, seed=21, seq_lens=[N, 613], heads=heads)
+    api.check()  # no bounded wait gave up, no layout fault
+    assert torch.isfinite(torch.as_tensor(out)).all()
+
+
+def test_decode_bulk_staged_feed_agrees_with_register_feed(bulk_staged_feed):
+    # the same call through both feeds: equal up to the summation order of
+    # the warps' partials
+    g = torch.Generator(device=DEV).manual_seed(5)
+    B, Hq, Hkv, N, d = 3, 32, 8, 2048, 128
+    K = torch.randn((B, Hkv, N, d), generator=g, device=DEV)
+    V = torch.randn((B, Hkv, N, d), generator=g, device=DEV)
+    q = torch.randn((B, Hq, d), generator=g, device=DEV).to(torch.bfloat16)
+    kq = api.Quantizer(d, 3, "prod", seed_rot=1, seed_qjl=2, device=DEV)
+    vq = api.Quantizer(d, 3, "mse", seed_rot=3, device=DEV)
+    kc, vc = api.encode(kq, K), api.encode(vq, V)
+    staged = api.decode_attention(kq, vq, q, kc, vc)
+    api.check()
+    api.set_decode_feed(False)
+    regs = api.decode_attention(kq, vq, q, kc, vc)
+    e = ((staged - regs).abs().amax(dim=-1) / regs.abs().amax(dim=-1)).max().item()
+    assert e <= 1e-4, e

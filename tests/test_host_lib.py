@@ -166,3 +166,16 @@ def test_noalloc_scratch_size_matches_header():
 def test_status_strings():
     assert L.status_name(L.TQ_EWORKSPACE) == "TQ_EWORKSPACE"
     assert L.status_name(99) == "TQ_UNKNOWN"
+
+
+def test_decode_feed_setter_round_trip():
+    # the feed switch returns the previous setting and refuses unknown values
+    lib = L.lib()
+    prev = lib.tq_set_decode_feed(L.TQ_FEED_BULK_STAGED)
+    try:
+        assert prev in (L.TQ_FEED_REGISTERS, L.TQ_FEED_BULK_STAGED)
+        assert lib.tq_set_decode_feed(7) == -1
+        assert lib.tq_set_decode_feed(L.TQ_FEED_REGISTERS) == L.TQ_FEED_BULK_STAGED
+        assert lib.tq_set_decode_feed(L.TQ_FEED_REGISTERS) == L.TQ_FEED_REGISTERS
+    finally:
+        lib.tq_set_decode_feed(prev if prev >= 0 else L.TQ_FEED_REGISTERS)
