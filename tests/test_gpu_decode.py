@@ -396,6 +396,10 @@ def test_append_decode_with_batch_lengths_and_scores():
     (128, (2, "mse"), (2, "prod"), ("dense", "dense"), 4),
     (200, (3, "mse"), (4, "mse"), ("dense", "dense"), 2),
     (64, (1, "prod"), (1, "prod"), ("hadamard", "dense"), 1),
+    # the smallest dense d (one-word records, 64 token classes) and a d whose
+    # code and sign records are not whole words (byte-wise staging)
+    (8, (2, "mse"), (3, "mse"), ("dense", "dense"), 4),
+    (40, (4, "prod"), (2, "prod"), ("dense", "dense"), 8),
 ])
 def test_decode_cuda_core_path(d, kspec, vspec, rotation, g):
     Hkv = 2
