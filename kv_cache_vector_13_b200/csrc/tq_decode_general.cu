@@ -509,6 +509,7 @@ __global__ void __launch_bounds__(kGnThreads) general_merge_kernel(GnParams p) {
   __shared__ float s_o[kGnMaxD], s_s[kGnMaxD];
   __shared__ float s_hdr[2];
   __shared__ float s_f[kGnMaxSplits];  // each slot's factor 2^(m_s - M), 0 for an empty slot
+  __shared__ float s_part[2 * kGnThreads];  // the parts' partial sums, [thread]
   const int head = blockIdx.x;  // b * Hq + hq
   const int b = head / p.Hq;
   const int tid = threadIdx.x;
@@ -549,13 +550,23 @@ __global__ void __launch_bounds__(kGnThreads) general_merge_kernel(GnParams p) {
   }
   __syncthreads();
   const float l = s_hdr[1];
-  for (int i = tid; i < d; i += kGnThreads) {
+  // the coordinates' loops split over P parts (P threads a coordinate when d
+  // leaves threads idle), each part a stride of the batches of 8 loads, the
+  // parts' sums added through shared memory (thread part * d + i)
+  const int P = d >= kGnThreads ? 1 : min(8, kGnThreads / d);
+  const int part = tid / d, pi = tid - part * d;
+  const bool pact = part < P;
+  const int pgv = (p.nv == 2 && pi >= p.v[1].off) ? 1 : 0;
+  const GnGroup &PG = p.v[pgv];
+  const int pc = pi - PG.off;  // the coordinate inside its group
+  float *s_pa = s_part, *s_pb = s_part + kGnThreads;
+  if (pact) {
     float o = 0.f, so = 0.f;
-    const float *slot = p.ws + (int64_t)head * stride + 4 + i;
+    const float *slot = p.ws + (int64_t)head * stride + 4 + pi;
     const int64_t sstride = (int64_t)p.B * p.Hq * stride;
     // batches of 8 slots, every load of a batch issued before its sums
     // (empty slots have f = 0 and finite sums)
-    for (int s0 = 0; s0 < p.splits; s0 += 8) {
+    for (int s0 = 8 * part; s0 < p.splits; s0 += 8 * P) {
       float x[8], y[8];
 #pragma unroll
       for (int k = 0; k < 8; ++k) {
@@ -570,45 +581,63 @@ __global__ void __launch_bounds__(kGnThreads) general_merge_kernel(GnParams p) {
         so = fmaf(y[k], f, so);
       }
     }
+    s_pa[tid] = o;
+    s_pb[tid] = so;
+  }
+  __syncthreads();
+  for (int i = tid; i < d; i += kGnThreads) {
+    float o = 0.f, so = 0.f;
+    for (int q = 0; q < P; ++q) {
+      o += s_pa[q * d + i];
+      so += s_pb[q * d + i];
+    }
     s_o[i] = o;
     s_s[i] = so;
   }
   __syncthreads();
   // prod value groups: o'_g += S_g^T (weighted signs); sqrt(pi/2)/d_g is in the weights
-  float add[kGnMaxD / kGnThreads];
-  for (int i = tid, c = 0; i < d; i += kGnThreads, ++c) {
-    const int gv = (p.nv == 2 && i >= p.v[1].off) ? 1 : 0;
-    const GnGroup &G = p.v[gv];
-    float a = 0.f;
-    if (G.prod) {
-      const int li = i - G.off;
-      for (int k0 = 0; k0 < G.d; k0 += 8) {  // batches of 8 loads
-        float x[8];
+  if (p.v[0].prod || (p.nv == 2 && p.v[1].prod)) {
+    if (pact) {
+      float a = 0.f;
+      if (PG.prod) {
+        for (int k0 = 8 * part; k0 < PG.d; k0 += 8 * P) {  // PG.d is a multiple of 8: batches of 8 loads
+          float x[8];
 #pragma unroll
-        for (int k = 0; k < 8; ++k) x[k] = __ldg(G.S + (int64_t)(k0 + k) * G.d + li);
+          for (int k = 0; k < 8; ++k) x[k] = __ldg(PG.S + (int64_t)(k0 + k) * PG.d + pc);
 #pragma unroll
-        for (int k = 0; k < 8; ++k) a = fmaf(x[k], s_s[G.off + k0 + k], a);
+          for (int k = 0; k < 8; ++k) a = fmaf(x[k], s_s[PG.off + k0 + k], a);
+        }
       }
+      s_pa[tid] = a;
     }
-    add[c] = a;
+    __syncthreads();
+    for (int i = tid; i < d; i += kGnThreads) {
+      float a = 0.f;
+      for (int q = 0; q < P; ++q) a += s_pa[q * d + i];
+      s_o[i] += a;
+    }
+    __syncthreads();
   }
-  __syncthreads();
-  for (int i = tid, c = 0; i < d; i += kGnThreads, ++c) s_o[i] += add[c];
-  __syncthreads();
   const float inv_l = l > 0.f ? 1.0f / l : 0.f;
   if (p.v[0].rot) {  // o[channels_g] = Pi_g^T o'_g
+    if (pact) {
+      float a = 0.f;
+      for (int r0 = 8 * part; r0 < PG.d; r0 += 8 * P) {  // batches of 8 loads
+        float x[8];
+#pragma unroll
+        for (int k = 0; k < 8; ++k) x[k] = __ldg(PG.rot + (int64_t)(r0 + k) * PG.d + pc);
+#pragma unroll
+        for (int k = 0; k < 8; ++k) a = fmaf(x[k], s_o[PG.off + r0 + k], a);
+      }
+      s_pa[tid] = a;
+    }
+    __syncthreads();
     for (int i = tid; i < d; i += kGnThreads) {
       const int gv = (p.nv == 2 && i >= p.v[1].off) ? 1 : 0;
       const GnGroup &G = p.v[gv];
       const int c = i - G.off;
       float a = 0.f;
-      for (int r0 = 0; r0 < G.d; r0 += 8) {  // G.d is a multiple of 8: batches of 8 loads
-        float x[8];
-#pragma unroll
-        for (int k = 0; k < 8; ++k) x[k] = __ldg(G.rot + (int64_t)(r0 + k) * G.d + c);
-#pragma unroll
-        for (int k = 0; k < 8; ++k) a = fmaf(x[k], s_o[G.off + r0 + k], a);
-      }
+      for (int q = 0; q < P; ++q) a += s_pa[q * d + i];
       const int ch = G.chan ? min(max(__ldg(G.chan + c), 0), d - 1) : c;
       out[ch] = a * inv_l;
     }
