@@ -39,7 +39,7 @@ constexpr int kGnThreads = 256;
 constexpr int kGnMaxD = 256;
 constexpr int kGnHeads = 8;   // query heads a block
 constexpr int kGnTile = 64;   // tokens a tile
-constexpr int kGnMaxSplits = 64;  // sequence splits at most
+constexpr int kGnMaxSplits = 128;  // sequence splits at most
 constexpr float kGnLog2e = 1.4426950408889634f;
 constexpr float kGnSqrtHalfPi = 1.2533141373155003f;
 
