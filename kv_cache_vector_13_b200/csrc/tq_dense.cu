@@ -52,6 +52,15 @@ struct DenseParams {
   dev::IndexSplit ix;
 };
 
+// Elements i, i + 1 (i even, the pair 8- or 4-byte aligned), widened to fp32.
+__device__ __forceinline__ float2 load_pair(const void *base, int dtype, int64_t i) {
+  if (dtype == TQ_F32) return __ldg(reinterpret_cast<const float2 *>(static_cast<const float *>(base) + i));
+  const uint32_t w = __ldg(reinterpret_cast<const unsigned int *>(static_cast<const unsigned short *>(base) + i));
+  if (dtype == TQ_BF16) return make_float2(__uint_as_float(w << 16), __uint_as_float(w & 0xffff0000u));
+  return make_float2(__half2float(__ushort_as_half((unsigned short)(w & 0xffffu))),
+                     __half2float(__ushort_as_half((unsigned short)(w >> 16))));
+}
+
 __device__ __forceinline__ float load_elem(const void *base, int dtype, int64_t i) {
   if (dtype == TQ_F32) return __ldg(static_cast<const float *>(base) + i);
   const unsigned short h = __ldg(static_cast<const unsigned short *>(base) + i);
@@ -306,45 +315,51 @@ __global__ void __launch_bounds__(kTcThreads, 1) encode_dense_tc_kernel(DensePar
     // loads are all in flight before the first row is used
 #pragma unroll 1
     for (int rb = 0; rb < kRows; rb += 8) {
-      float xr[8][J];
+      // lane holds the element pairs (2 lane + 64 jj, + 1), jj < J / 2
+      float2 xr[8][J / 2];
 #pragma unroll
       for (int r = 0; r < 8; ++r) {
         const int64_t v = tile * kTcM + gw * kRows + rb + r;
         int64_t b, h, n;
         bhn(p, v < p.nvec ? v : 0, b, h, n);
-        const int64_t xoff = b * p.xsb + h * p.xsh + n * p.xsn;
+        const int64_t xoff = b * p.xsb + h * p.xsh + n * p.xsn;  // even: the rows are 16-byte aligned
 #pragma unroll
-        for (int j = 0; j < J; ++j) xr[r][j] = v < p.nvec ? load_elem(p.x, DT, xoff + lane + 32 * j) : 0.0f;
+        for (int jj = 0; jj < J / 2; ++jj)
+          xr[r][jj] = v < p.nvec ? load_pair(p.x, DT, xoff + 2 * lane + 64 * jj) : make_float2(0.0f, 0.0f);
       }
 #pragma unroll
       for (int r = 0; r < 8; ++r) {
         const int m = gw * kRows + rb + r;
         const int64_t v = tile * kTcM + m;
-        float sq[J];
-#pragma unroll
-        for (int j = 0; j < J; ++j) sq[j] = __fmul_rn(xr[r][j], xr[r][j]);
-#pragma unroll
-        for (int st = J / 2; st >= 1; st >>= 1) {
-#pragma unroll
-          for (int j = 0; j < st; ++j) sq[j] = __fadd_rn(sq[j], sq[j + st]);
+        // norm: fold-halves in the canonical stage order, h = 64 in the
+        // lane, h = 32 .. 2 across lanes 16 .. 1 apart, h = 1 in the lane
+        float2 sq = make_float2(__fmul_rn(xr[r][0].x, xr[r][0].x), __fmul_rn(xr[r][0].y, xr[r][0].y));
+        if constexpr (J / 2 == 2) {
+          const float2 t = make_float2(__fmul_rn(xr[r][1].x, xr[r][1].x), __fmul_rn(xr[r][1].y, xr[r][1].y));
+          dev::add_x2(sq.x, sq.y, sq.x, sq.y, t.x, t.y);
         }
-        float s = sq[0];
 #pragma unroll
-        for (int hh = 16; hh >= 1; hh >>= 1) s = __fadd_rn(s, __shfl_down_sync(dev::kFull, s, hh));
-        const float nrm = __fsqrt_rn(__shfl_sync(dev::kFull, s, 0));
+        for (int hh = 16; hh >= 1; hh >>= 1) {
+          const float o0 = __shfl_down_sync(dev::kFull, sq.x, hh), o1 = __shfl_down_sync(dev::kFull, sq.y, hh);
+          dev::add_x2(sq.x, sq.y, sq.x, sq.y, o0, o1);
+        }
+        const float nrm = __fsqrt_rn(__shfl_sync(dev::kFull, __fadd_rn(sq.x, sq.y), 0));
         // 2^(13 - floor(log2 n)) for a normal n > 0, else 1
         const int ex = ((__float_as_int(nrm) >> 23) & 0xff) - 127;
         const bool normal = nrm > 0.0f && ex > -127;
         const float sc = normal ? __int_as_float((127 + 13 - ex) << 23) : 1.0f;
 #pragma unroll
-        for (int j = 0; j < J; ++j) {
-          const int k = lane + 32 * j;
-          const float xs = xr[r][j] * sc;
-          const __half hi = __float2half_rn(xs);
-          const __half lo = __float2half_rn(xs - __half2float(hi));
-          const uint32_t o = umma::off(m, k, L::SBO_A, kTcLboA);
-          *reinterpret_cast<__half *>(smem + oAh + o) = hi;
-          *reinterpret_cast<__half *>(smem + oAl + o) = lo;
+        for (int jj = 0; jj < J / 2; ++jj) {
+          const int k = 2 * lane + 64 * jj;
+          float xs0, xs1, lo0, lo1;
+          dev::mul_x2(xs0, xs1, xr[r][jj].x, xr[r][jj].y, sc, sc);  // sc is a power of two: exact
+          const __half2 hi = __floats2half2_rn(xs0, xs1);
+          const float2 hf = __half22float2(hi);
+          dev::sub_x2(lo0, lo1, xs0, xs1, hf.x, hf.y);
+          const __half2 lo = __floats2half2_rn(lo0, lo1);
+          const uint32_t o = umma::off(m, k, L::SBO_A, kTcLboA);  // k even: a 4-byte aligned pair
+          *reinterpret_cast<__half2 *>(smem + oAh + o) = hi;
+          *reinterpret_cast<__half2 *>(smem + oAl + o) = lo;
         }
         if (lane == 0) {
           s_inv[m] = normal ? __frcp_rn(__fmul_rn(16.0f * sc, nrm)) : 0.0f;
