@@ -1275,7 +1275,9 @@ __global__ void __launch_bounds__(split_warps<PACK, KPROD, STAGED>() * 32, 1) de
           // (staged masked rows hold whatever the slot holds: kept finite)
           nvl[ms][r] = (STAGED && !ok[r]) ? 0.f : __log2f(kb.vn[ms][r]);
         }
-        float cm[4] = {0.f, 0.f, 0.f, 0.f};
+        // the lo halves (more than 4 heads) accumulate apart: two chains of
+        // dependent MMAs instead of one twice as long
+        float cm[4] = {0.f, 0.f, 0.f, 0.f}, cm2[4] = {0.f, 0.f, 0.f, 0.f};
         if constexpr (K4) {
           // byte S of a row's 64-bit stream: pairs 2S and 2S + 1 in one read
 #define TQ_KSTEP4(S)                                                              \
@@ -1285,7 +1287,7 @@ __global__ void __launch_bounds__(split_warps<PACK, KPROD, STAGED>() * 32, 1) de
     const uint2 e1 = lut64(__byte_perm(kw[1][(S) >> 2], koff, sel));              \
     const uint32_t a[4] = {e0.x, e1.x, e0.y, e1.y};                               \
     mma16816(cm, a, qf[S][0], qf[S][1]);                                          \
-    if constexpr (!PACK) mma16816(cm, a, qf2[S][0], qf2[S][1]);                   \
+    if constexpr (!PACK) mma16816(cm2, a, qf2[S][0], qf2[S][1]);                  \
   }
           TQ_KSTEP4(0) TQ_KSTEP4(1) TQ_KSTEP4(2) TQ_KSTEP4(3)
           TQ_KSTEP4(4) TQ_KSTEP4(5) TQ_KSTEP4(6) TQ_KSTEP4(7)
@@ -1299,11 +1301,15 @@ __global__ void __launch_bounds__(split_warps<PACK, KPROD, STAGED>() * 32, 1) de
     a[2] = lut(pair_addr<KBM, 2 * (S) + 1, KW>(kw[0], koff));                     \
     a[3] = lut(pair_addr<KBM, 2 * (S) + 1, KW>(kw[1], koff));                     \
     mma16816(cm, a, qf[S][0], qf[S][1]);                                          \
-    if constexpr (!PACK) mma16816(cm, a, qf2[S][0], qf2[S][1]);                   \
+    if constexpr (!PACK) mma16816(cm2, a, qf2[S][0], qf2[S][1]);                  \
   }
           TQ_KSTEP(0) TQ_KSTEP(1) TQ_KSTEP(2) TQ_KSTEP(3)
           TQ_KSTEP(4) TQ_KSTEP(5) TQ_KSTEP(6) TQ_KSTEP(7)
 #undef TQ_KSTEP
+        }
+        if constexpr (!PACK) {
+#pragma unroll
+          for (int i = 0; i < 4; ++i) cm[i] += cm2[i];
         }
         float cq[4] = {0.f, 0.f, 0.f, 0.f};
         if constexpr (KPROD) {
