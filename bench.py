@@ -85,7 +85,7 @@ FALLBACK_PEAKS = {"hbm_gbs": 6650.0, "bf16_tflops": 1590.0}
 # Captured at B = 2 (reads 230,603,776 B, writes 6,578,432 B): reads scaled by
 # the 8x units of B = 16 (B = 4 read 2.02x the B = 2 bytes), writes kept.
 TRAFFIC = {"workload": ("batched", 16), "bytes": 8 * 230603776 + 6578432,
-           "source_sha256": "1b64f155a123bc58686ff16ffe4ca8e901340d6cb95a56af1c44441a97ae49e1"}
+           "source_sha256": "2965f51ec95d5ecc9c99c0b44894bab9ab749320b2f4c15193ec00b9640644a0"}
 DECODE_SOURCES = ("tq_decode.cu", "tq_decode_split.cuh", "tq_decode_regs.cu")
 
 

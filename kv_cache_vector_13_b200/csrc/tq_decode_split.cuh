@@ -45,7 +45,9 @@
 //     query heads per kv head the hi and lo halves of q' (and of the PV
 //     weights) share one MMA as columns 0-3 and 4-7; with 5-8 heads they take
 //     two MMAs;
-//   * QJL bits become +-1 halves with one shift and one LOP3 per pair;
+//   * the QJL term runs on int8 MMAs (mma.m16n8k32.s8): a sign-replicating
+//     byte permute turns four sign bits into four 0 / -1 bytes, against S q'
+//     held as two int8 digits (<S q', 2 bit - 1> = -2 (digit sum) - sum S q');
 //   * online softmax in base 2 against one reference M per head column,
 //     taken over u = logit + max(log2 n_V, kNvlFloor) and moved only when
 //     some u passes it by more than kLazy: the PV weights 2^(logit + log2 n_V
