@@ -12,17 +12,20 @@
 //     database; each warp streams 32-record chunks, scores them with the
 //     pair-table lookups and mma.m16n8k16 of the decode kernel, and keeps,
 //     per query, its best 32 (estimate, index) pairs sorted in registers, one
-//     per lane.  A chunk whose candidates all rank below the current k-th
-//     best is dropped after one vote of the lanes that hold the query's
-//     estimates; a few that beat it are inserted one at a time at their
-//     rank (a vote counts the entries ahead, the rest shift down one lane);
-//     many (a list's first chunks) are sorted by a warp bitonic sort and
-//     merged (the better of pair l and the reversed pair 31 - l is a
+//     per lane.  Each lane tests its own two query columns against their
+//     lists' k-th entries and against the CTA's k-th estimate per query (the
+//     best of its warps' k-th entries, kept with an atomic maximum in shared
+//     memory: a candidate below it is beaten by k others); two votes say
+//     which queries have a candidate that passes, and most chunks stop
+//     there.  For those, a few candidates are inserted one at a time at
+//     their rank (a vote counts the entries ahead, the rest shift down one
+//     lane); many (a list's first chunks) are sorted by a warp bitonic sort
+//     and merged (the better of pair l and the reversed pair 31 - l is a
 //     bitonic sequence holding the best 32, which five exchange stages
 //     sort).  The CTA's warps merge their lists the same way and write one
 //     list per (query, slice);
-//   * search_merge_kernel: one warp per query merges the slices' lists and
-//     writes the first k.
+//   * search_merge_kernel: a block per query, eight warps merging every
+//     eighth slice list, then one merge of the eight; writes the first k.
 // Order: estimate descending, ties by record index ascending (a total
 // order, so the result is unique).
 
