@@ -1077,22 +1077,34 @@ __global__ void __launch_bounds__(split_warps<PACK, KPROD, STAGED>() * 32, 1) de
     inv_sK = __ldg(p.ws + 0);
     inv_sV = __ldg(p.ws + 1);
     uint4 *tab = reinterpret_cast<uint4 *>(s_lut);
+    // register-fed: the 256 + 256 distinct entries first (one load a thread,
+    // all in flight) into the partials' memory, idle until the first piece
+    // ends, then the per-lane copies from there; staged: the partials'
+    // memory may hold ring slots already in flight, so from L2 directly
+    const uint32_t *ks = ktab, *vs = vtab;
+    if constexpr (!STAGED) {
+      uint32_t *raw = reinterpret_cast<uint32_t *>(s_part);
+      for (int i = tid; i < 512; i += kThreads) raw[i] = i < 256 ? (KBM > 0 ? __ldg(ktab + i) : 0u) : __ldg(vtab + i - 256);
+      __syncthreads();
+      ks = raw;
+      vs = raw + 256;
+    }
     if constexpr (K4) {
       // key entry e: the pair entries of its low and high nibbles
       for (int i = tid; i < 256 * 16; i += kThreads) {
         const int e = i >> 4;
-        const uint32_t lo = __ldg(ktab + (e & 15)), hi = __ldg(ktab + (e >> 4));
+        const uint32_t lo = ks[e & 15], hi = ks[e >> 4];
         tab[i] = make_uint4(lo, hi, lo, hi);
       }
       uint4 *vt = reinterpret_cast<uint4 *>(s_lut + (kVTab4Addr - kLutAddr));
       for (int i = tid; i < 256 * 8; i += kThreads) {  // the first 128 bytes of each row
-        const uint32_t v = __ldg(vtab + (i >> 3));
+        const uint32_t v = vs[i >> 3];
         vt[(i >> 3) * 16 + (i & 7)] = make_uint4(v, v, v, v);
       }
     } else {
       for (int i = tid; i < 256 * 16; i += kThreads) {  // 16 uint4 per 256-byte row
         const int e = i >> 4, part = i & 15;
-        const uint32_t v = part < 8 ? (KBM > 0 ? __ldg(ktab + e) : 0u) : __ldg(vtab + e);
+        const uint32_t v = part < 8 ? (KBM > 0 ? ks[e] : 0u) : vs[e];
         tab[i] = make_uint4(v, v, v, v);
       }
     }
