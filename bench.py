@@ -82,10 +82,10 @@ FALLBACK_PEAKS = {"hbm_gbs": 6650.0, "bf16_tflops": 1590.0}
 # workload, from an ncu capture (dram__bytes_read.sum + dram__bytes_write.sum),
 # reported only for that workload and while the decode sources are the ones
 # it was taken on.
-# Captured at B = 2 (reads 230,603,776 B, writes 6,578,432 B): reads scaled by
+# Captured at B = 2 (reads 230,536,192 B, writes 4,043,520 B): reads scaled by
 # the 8x units of B = 16 (B = 4 read 2.02x the B = 2 bytes), writes kept.
-TRAFFIC = {"workload": ("batched", 16), "bytes": 8 * 230603776 + 6578432,
-           "source_sha256": "2965f51ec95d5ecc9c99c0b44894bab9ab749320b2f4c15193ec00b9640644a0"}
+TRAFFIC = {"workload": ("batched", 16), "bytes": 8 * 230536192 + 4043520,
+           "source_sha256": "be1a913840ea164638a20dcb50b885af95c308fb41ae4683bc8ee9649f68d1a5"}
 DECODE_SOURCES = ("tq_decode.cu", "tq_decode_split.cuh", "tq_decode_regs.cu")
 
 
